@@ -1,0 +1,233 @@
+"""Python binding of libdbf.so, the sm_100a double-binary layer forward.
+
+Argument marshalling only: every step of the forward runs in the library's
+CUDA kernels (see include/dbf.h for the operation, layouts and errors).
+PyTorch supplies device memory and the current CUDA stream. There is no CPU
+fallback: if the shared library is missing, importing this package raises.
+Build it with ``python -m double_binary_rank_b200.build``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+from typing import List, Optional, Sequence
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libdbf.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"{LIB_PATH} is missing: the CUDA library must be built "
+                      "(python -m double_binary_rank_b200.build); there is no CPU fallback")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+# ---- enums (dbf.h)
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_ALIGNMENT, ERR_WORKSPACE, ERR_CUDA, ERR_TIMEOUT = range(7)
+F32, BF16, F16, I8 = range(4)
+PATH_AUTO, PATH_GEMV, PATH_GEMM = range(3)
+ACCUMULATE, WEIGHTS_STATIC = 1, 2
+_PATHS = {"auto": PATH_AUTO, "gemv": PATH_GEMV, "gemm": PATH_GEMM}
+_DT = {torch.float32: F32, torch.bfloat16: BF16, torch.float16: F16, torch.int8: I8}
+
+
+class DbfLayerC(ctypes.Structure):
+    """dbf_layer of dbf.h."""
+    _fields_ = [("M", ctypes.c_int32), ("N", ctypes.c_int32), ("R", ctypes.c_int32),
+                ("ell", ctypes.c_int32), ("b1_packed", ctypes.c_void_p),
+                ("b2_packed", ctypes.c_void_p), ("alpha", ctypes.c_void_p),
+                ("beta", ctypes.c_void_p), ("gamma", ctypes.c_void_p)]
+
+
+_vp, _i64, _i32, _sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_size_t
+_LP = ctypes.POINTER(DbfLayerC)
+_SIGS = {
+    "dbf_packed_bytes": (_sz, [_i64, _i64]),
+    "dbf_pack_signs": (ctypes.c_int, [_vp, ctypes.c_int, _i64, _i64, _vp, _sz, _vp, _vp]),
+    "dbf_unpack_signs": (ctypes.c_int, [_vp, _i64, _i64, _vp, _vp]),
+    "dbf_gemm_min_tokens": (_i64, []),
+    "dbf_workspace_bytes": (_sz, [_LP, _i64, ctypes.c_int]),
+    "dbf_forward": (ctypes.c_int, [_LP, _vp, ctypes.c_int, _vp, ctypes.c_int, _i64, ctypes.c_int,
+                                   ctypes.c_int, _vp, _sz, _vp]),
+    "dbf_segmented_workspace_bytes": (_sz, [_i32, _i32, _i64]),
+    "dbf_forward_segmented": (ctypes.c_int, [_vp, _i32, _vp, _vp, _i32, _i32, _i32, _i32, _i32,
+                                             _vp, ctypes.c_int, _vp, ctypes.c_int, _i64,
+                                             ctypes.c_int, _vp, _sz, _vp, _vp]),
+    "dbf_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "dbf_version": (ctypes.c_char_p, []),
+}
+for _name, (_res, _args) in _SIGS.items():
+    _f = getattr(_lib, _name)
+    _f.restype = _res
+    _f.argtypes = _args
+
+EXPORTED = tuple(_SIGS)
+
+
+class DbfError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {_lib.dbf_status_string(status).decode()} (status {status})")
+
+
+def _check(status: int, where: str) -> None:
+    if status != OK:
+        raise DbfError(status, where)
+
+
+def _stream(stream: Optional[torch.cuda.Stream]) -> int:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def version() -> str:
+    return _lib.dbf_version().decode()
+
+
+def status_string(status: int) -> str:
+    return _lib.dbf_status_string(status).decode()
+
+
+def packed_bytes(rows: int, k: int) -> int:
+    return int(_lib.dbf_packed_bytes(rows, k))
+
+
+def gemm_min_tokens() -> int:
+    return int(_lib.dbf_gemm_min_tokens())
+
+
+def pack_signs(src: torch.Tensor, out: Optional[torch.Tensor] = None,
+               status: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Pack a rows x k int8 (+-1) or float latent tensor (dbf_pack_signs).
+
+    Returns int32 words [rows, ceil(k/32)] (the uint32 bit patterns)."""
+    rows, k = src.shape
+    src = src.contiguous()
+    if out is None:
+        out = torch.empty((rows, (k + 31) // 32), dtype=torch.int32, device=src.device)
+    _check(_lib.dbf_pack_signs(_ptr(src), _DT[src.dtype], rows, k, _ptr(out),
+                               out.numel() * 4, _ptr(status), _stream(stream)), "dbf_pack_signs")
+    return out
+
+
+def unpack_signs(words: torch.Tensor, rows: int, k: int, out: Optional[torch.Tensor] = None,
+                 stream=None) -> torch.Tensor:
+    if out is None:
+        out = torch.empty((rows, k), dtype=torch.int8, device=words.device)
+    _check(_lib.dbf_unpack_signs(_ptr(words), rows, k, _ptr(out), _stream(stream)),
+           "dbf_unpack_signs")
+    return out
+
+
+@dataclass
+class Layer:
+    """Device-resident layer: packed signs (int32 words) and fp16 scales.
+
+    b1: [N, ceil(R/32)] packed words; b2: [R, ceil(M/32)] packed words;
+    alpha [ell, N], beta [ell, R], gamma [ell, M] as torch.float16 tensors.
+    """
+    M: int
+    N: int
+    R: int
+    ell: int
+    b1: torch.Tensor
+    b2: torch.Tensor
+    alpha: torch.Tensor
+    beta: torch.Tensor
+    gamma: torch.Tensor
+
+    def descriptor(self) -> DbfLayerC:
+        return DbfLayerC(self.M, self.N, self.R, self.ell, _ptr(self.b1), _ptr(self.b2),
+                         _ptr(self.alpha), _ptr(self.beta), _ptr(self.gamma))
+
+    @staticmethod
+    def from_signs(b1_signs: torch.Tensor, b2_signs: torch.Tensor, alpha: torch.Tensor,
+                   beta: torch.Tensor, gamma: torch.Tensor, stream=None) -> "Layer":
+        """Pack +-1 sign matrices (N x R and R x M, on the device) into a Layer."""
+        N, R = b1_signs.shape
+        R2, M = b2_signs.shape
+        assert R == R2
+        ell = alpha.shape[0]
+        return Layer(M, N, R, ell, pack_signs(b1_signs, stream=stream),
+                     pack_signs(b2_signs, stream=stream), alpha.contiguous(), beta.contiguous(),
+                     gamma.contiguous())
+
+
+def workspace_bytes(layer: Layer, T: int, path: str = "auto") -> int:
+    d = layer.descriptor()
+    return int(_lib.dbf_workspace_bytes(ctypes.byref(d), T, _PATHS[path]))
+
+
+def alloc_workspace(nbytes: int, device) -> torch.Tensor:
+    return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+
+
+def _flags(accumulate: bool, static_weights: bool) -> int:
+    return (ACCUMULATE if accumulate else 0) | (WEIGHTS_STATIC if static_weights else 0)
+
+
+def forward(layer: Layer, x: torch.Tensor, y: Optional[torch.Tensor] = None,
+            accumulate: bool = False, path: str = "auto", ws: Optional[torch.Tensor] = None,
+            y_dtype: Optional[torch.dtype] = None, static_weights: bool = False,
+            stream=None) -> torch.Tensor:
+    """y = [acc] y + dW x (dbf_forward). x: [T, M] float32/bfloat16 on the device.
+
+    static_weights: the packed signs were not written by the preceding work
+    on the stream (lets the kernels prefetch them across the kernel boundary)."""
+    T = x.shape[0]
+    if y is None:
+        y = torch.empty((T, layer.N), dtype=y_dtype or x.dtype, device=x.device)
+    d = layer.descriptor()
+    need = int(_lib.dbf_workspace_bytes(ctypes.byref(d), T, _PATHS[path]))
+    if ws is None:
+        ws = alloc_workspace(need, x.device)
+    _check(_lib.dbf_forward(ctypes.byref(d), _ptr(x), _DT[x.dtype], _ptr(y), _DT[y.dtype], T,
+                            _flags(accumulate, static_weights), _PATHS[path], _ptr(ws), ws.numel(),
+                            _stream(stream)), "dbf_forward")
+    return y
+
+
+class AdapterTable:
+    """Device array of dbf_layer descriptors for segmented serving."""
+
+    def __init__(self, layers: Sequence[Layer], device):
+        self.layers = list(layers)
+        n = len(self.layers)
+        arr = (DbfLayerC * max(n, 1))(*[l.descriptor() for l in self.layers])
+        raw = bytes(ctypes.string_at(ctypes.addressof(arr), ctypes.sizeof(arr)))
+        self.dev = torch.frombuffer(bytearray(raw), dtype=torch.uint8).to(device)
+        self.num = n
+        self.max_R = max(l.R for l in self.layers)
+        self.max_ell = max(l.ell for l in self.layers)
+        self.M = self.layers[0].M
+        self.N = self.layers[0].N
+
+
+def segmented_workspace_bytes(max_R: int, max_ell: int, T: int) -> int:
+    return int(_lib.dbf_segmented_workspace_bytes(max_R, max_ell, T))
+
+
+def forward_segmented(table: AdapterTable, seg_offsets: torch.Tensor, seg_adapter: torch.Tensor,
+                      x: torch.Tensor, y: Optional[torch.Tensor] = None, accumulate: bool = False,
+                      ws: Optional[torch.Tensor] = None, status: Optional[torch.Tensor] = None,
+                      y_dtype: Optional[torch.dtype] = None, stream=None) -> torch.Tensor:
+    """Segmented multi-adapter forward (dbf_forward_segmented)."""
+    T = x.shape[0]
+    S = seg_adapter.numel()
+    if y is None:
+        y = torch.empty((T, table.N), dtype=y_dtype or x.dtype, device=x.device)
+    need = segmented_workspace_bytes(table.max_R, table.max_ell, T)
+    if ws is None:
+        ws = alloc_workspace(need, x.device)
+    _check(_lib.dbf_forward_segmented(_ptr(table.dev), table.num, _ptr(seg_offsets),
+                                      _ptr(seg_adapter), S, table.max_R, table.max_ell, table.M,
+                                      table.N, _ptr(x), _DT[x.dtype], _ptr(y), _DT[y.dtype], T,
+                                      _flags(accumulate, False), _ptr(ws), ws.numel(), _ptr(status),
+                                      _stream(stream)), "dbf_forward_segmented")
+    return y

@@ -1,0 +1,153 @@
+// Host entry points of the C ABI declared in include/dbf.h: argument checks
+// (no launch on a failed check), path choice and the workspace contract.
+#include "dbf_internal.cuh"
+
+namespace {
+
+using namespace dbf;
+
+constexpr int64_t kGemmMinTokens = 128;
+
+bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+dbf_status from_cuda(cudaError_t e) { return e == cudaSuccess ? DBF_OK : DBF_ERR_CUDA; }
+
+bool act_dtype_ok(dbf_dtype d) { return d == DBF_F32 || d == DBF_BF16; }
+
+dbf_status check_layer(const dbf_layer *L)
+{
+    if (!L) return DBF_ERR_INVALID_ARG;
+    if (L->M <= 0 || L->N <= 0 || L->R <= 0 || L->ell < 1 || L->ell > kMaxEll)
+        return DBF_ERR_INVALID_ARG;
+    if (!L->b1_packed || !L->b2_packed || !L->alpha || !L->beta || !L->gamma)
+        return DBF_ERR_INVALID_ARG;
+    if (!aligned(L->b1_packed, 16) || !aligned(L->b2_packed, 16) || !aligned(L->alpha, 2) ||
+        !aligned(L->beta, 2) || !aligned(L->gamma, 2))
+        return DBF_ERR_ALIGNMENT;
+    return DBF_OK;
+}
+
+// The path dbf_forward takes; DBF_PATH_GEMM only when the shape allows it.
+dbf_path resolve(const dbf_layer &L, int64_t T, dbf_path p)
+{
+    if (p == DBF_PATH_AUTO) return (gemm_shape_ok(L) && T >= kGemmMinTokens) ? DBF_PATH_GEMM : DBF_PATH_GEMV;
+    return p;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t dbf_packed_bytes(int64_t rows, int64_t k)
+{
+    if (rows <= 0 || k <= 0) return 0;
+    return static_cast<size_t>(rows) * static_cast<size_t>(pitch_words(k)) * 4u;
+}
+
+dbf_status dbf_pack_signs(const void *src, dbf_dtype src_dtype, int64_t rows, int64_t k,
+                          uint32_t *dst, size_t dst_bytes, int32_t *status_dev, void *stream)
+{
+    if (!src || !dst || rows <= 0 || k <= 0) return DBF_ERR_INVALID_ARG;
+    if (src_dtype != DBF_I8 && src_dtype != DBF_F32 && src_dtype != DBF_BF16 && src_dtype != DBF_F16)
+        return DBF_ERR_INVALID_ARG;
+    if (dst_bytes < dbf_packed_bytes(rows, k)) return DBF_ERR_INVALID_ARG;
+    const uintptr_t esz = src_dtype == DBF_I8 ? 1 : (src_dtype == DBF_F32 ? 4 : 2);
+    if (!aligned(src, esz) || !aligned(dst, 4) || (status_dev && !aligned(status_dev, 4)))
+        return DBF_ERR_ALIGNMENT;
+    return from_cuda(launch_pack(src, src_dtype, rows, k, dst, status_dev,
+                                 static_cast<cudaStream_t>(stream)));
+}
+
+dbf_status dbf_unpack_signs(const uint32_t *src, int64_t rows, int64_t k, int8_t *dst, void *stream)
+{
+    if (!src || !dst || rows <= 0 || k <= 0) return DBF_ERR_INVALID_ARG;
+    if (!aligned(src, 4)) return DBF_ERR_ALIGNMENT;
+    return from_cuda(launch_unpack(src, rows, k, dst, static_cast<cudaStream_t>(stream)));
+}
+
+int64_t dbf_gemm_min_tokens(void) { return kGemmMinTokens; }
+
+size_t dbf_workspace_bytes(const dbf_layer *L, int64_t T, dbf_path path)
+{
+    if (!L || L->M <= 0 || L->N <= 0 || L->R <= 0 || L->ell < 1 || L->ell > kMaxEll || T < 0)
+        return 0;
+    if (path != DBF_PATH_AUTO && path != DBF_PATH_GEMV && path != DBF_PATH_GEMM) return 0;
+    const dbf_path p = resolve(*L, T, path);
+    if (p == DBF_PATH_GEMM) return gemm_shape_ok(*L) ? gemm_workspace_bytes(*L, T) : 0;
+    return gemv_workspace_bytes(L->R, L->ell, T);
+}
+
+dbf_status dbf_forward(const dbf_layer *L, const void *x, dbf_dtype x_dtype, void *y,
+                       dbf_dtype y_dtype, int64_t T, int flags, dbf_path path, void *ws,
+                       size_t ws_bytes, void *stream)
+{
+    dbf_status st = check_layer(L);
+    if (st != DBF_OK) return st;
+    if (T < 0 || !act_dtype_ok(x_dtype) || !act_dtype_ok(y_dtype)) return DBF_ERR_INVALID_ARG;
+    if (flags & ~(DBF_ACCUMULATE | DBF_WEIGHTS_STATIC)) return DBF_ERR_INVALID_ARG;
+    if (path != DBF_PATH_AUTO && path != DBF_PATH_GEMV && path != DBF_PATH_GEMM)
+        return DBF_ERR_INVALID_ARG;
+    if (T == 0) return DBF_OK;
+    if (!x || !y) return DBF_ERR_INVALID_ARG;
+    if (!aligned(x, 16) || !aligned(y, 16)) return DBF_ERR_ALIGNMENT;
+    const dbf_path p = resolve(*L, T, path);
+    if (p == DBF_PATH_GEMM && !gemm_shape_ok(*L)) return DBF_ERR_UNSUPPORTED;
+    const size_t need = dbf_workspace_bytes(L, T, p);
+    if (need > 0 && (!ws || ws_bytes < need)) return DBF_ERR_WORKSPACE;
+    if (ws && !aligned(ws, 256)) return DBF_ERR_ALIGNMENT;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (p == DBF_PATH_GEMM) return from_cuda(gemm_forward(*L, x, x_dtype, y, y_dtype, T, flags, ws, s));
+    return from_cuda(gemv_forward(*L, x, x_dtype, y, y_dtype, T, flags, ws, s));
+}
+
+size_t dbf_segmented_workspace_bytes(int32_t max_R, int32_t max_ell, int64_t T)
+{
+    if (max_R <= 0 || max_ell < 1 || max_ell > kMaxEll || T < 0) return 0;
+    return gemv_workspace_bytes(max_R, max_ell, T);
+}
+
+dbf_status dbf_forward_segmented(const dbf_layer *adapters_dev, int32_t num_adapters,
+                                 const int32_t *seg_offsets_dev, const int32_t *seg_adapter_dev,
+                                 int32_t S, int32_t max_R, int32_t max_ell, int32_t M, int32_t N,
+                                 const void *x, dbf_dtype x_dtype, void *y, dbf_dtype y_dtype,
+                                 int64_t T, int flags, void *ws, size_t ws_bytes,
+                                 int32_t *status_dev, void *stream)
+{
+    if (num_adapters < 0 || S < 0 || max_R <= 0 || max_ell < 1 || max_ell > kMaxEll || M <= 0 ||
+        N <= 0 || T < 0 || !act_dtype_ok(x_dtype) || !act_dtype_ok(y_dtype) ||
+        (flags & ~(DBF_ACCUMULATE | DBF_WEIGHTS_STATIC)))
+        return DBF_ERR_INVALID_ARG;
+    if (S > 65535) return DBF_ERR_UNSUPPORTED;
+    if (T == 0 || S == 0) return DBF_OK;
+    if (!seg_offsets_dev || !seg_adapter_dev || !x || !y || (num_adapters > 0 && !adapters_dev))
+        return DBF_ERR_INVALID_ARG;
+    if (!aligned(x, 16) || !aligned(y, 16) || !aligned(seg_offsets_dev, 4) ||
+        !aligned(seg_adapter_dev, 4) || (adapters_dev && !aligned(adapters_dev, 8)) ||
+        (status_dev && !aligned(status_dev, 4)))
+        return DBF_ERR_ALIGNMENT;
+    const size_t need = dbf_segmented_workspace_bytes(max_R, max_ell, T);
+    if (!ws || ws_bytes < need) return DBF_ERR_WORKSPACE;
+    if (!aligned(ws, 256)) return DBF_ERR_ALIGNMENT;
+    return from_cuda(gemv_forward_segmented(adapters_dev, num_adapters, seg_offsets_dev,
+                                            seg_adapter_dev, S, max_R, max_ell, M, N, x, x_dtype,
+                                            y, y_dtype, T, flags, ws, status_dev,
+                                            static_cast<cudaStream_t>(stream)));
+}
+
+const char *dbf_status_string(dbf_status s)
+{
+    switch (s) {
+    case DBF_OK: return "ok";
+    case DBF_ERR_INVALID_ARG: return "invalid argument";
+    case DBF_ERR_UNSUPPORTED: return "unsupported shape or path";
+    case DBF_ERR_ALIGNMENT: return "misaligned pointer";
+    case DBF_ERR_WORKSPACE: return "workspace missing or too small";
+    case DBF_ERR_CUDA: return "CUDA error";
+    case DBF_ERR_TIMEOUT: return "device wait timed out";
+    }
+    return "unknown status";
+}
+
+const char *dbf_version(void) { return "dbf-b200 0.1 (sm_100a)"; }
+
+}  // extern "C"

@@ -1,0 +1,66 @@
+// Internal declarations shared by the library's translation units.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_fp16.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "dbf.h"
+
+namespace dbf {
+
+constexpr int kMaxEll = 8;
+
+// ---- packed layout helpers (see "Packed sign layout" in dbf.h) -----------
+__host__ __device__ inline int64_t pitch_words(int64_t k) { return (k + 31) / 32; }
+
+// ---- launchers (each returns the first CUDA error it meets) --------------
+cudaError_t launch_pack(const void *src, dbf_dtype dt, int64_t rows, int64_t k, uint32_t *dst,
+                        int32_t *status, cudaStream_t s);
+cudaError_t launch_unpack(const uint32_t *src, int64_t rows, int64_t k, int8_t *dst,
+                          cudaStream_t s);
+
+// decode path
+size_t gemv_workspace_bytes(int64_t R, int64_t ell, int64_t T);
+cudaError_t gemv_forward(const dbf_layer &L, const void *x, dbf_dtype xd, void *y, dbf_dtype yd,
+                         int64_t T, int flags, void *ws, cudaStream_t s);
+cudaError_t gemv_forward_segmented(const dbf_layer *adapters, int32_t num_adapters,
+                                   const int32_t *seg_off, const int32_t *seg_adp, int32_t S,
+                                   int32_t max_R, int32_t max_ell, int32_t M, int32_t N,
+                                   const void *x, dbf_dtype xd, void *y, dbf_dtype yd, int64_t T,
+                                   int flags, void *ws, int32_t *status, cudaStream_t s);
+
+// prefill path (tcgen05)
+bool gemm_shape_ok(const dbf_layer &L);
+size_t gemm_workspace_bytes(const dbf_layer &L, int64_t T);
+cudaError_t gemm_forward(const dbf_layer &L, const void *x, dbf_dtype xd, void *y, dbf_dtype yd,
+                         int64_t T, int flags, void *ws, cudaStream_t s);
+
+inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+}  // namespace dbf
+
+// ---- small device helpers -------------------------------------------------
+namespace dbf {
+
+__device__ __forceinline__ float load_act(const void *p, dbf_dtype dt, int64_t i)
+{
+    if (dt == DBF_F32) return static_cast<const float *>(p)[i];
+    return __bfloat162float(static_cast<const __nv_bfloat16 *>(p)[i]);
+}
+
+__device__ __forceinline__ void store_act(void *p, dbf_dtype dt, int64_t i, float v)
+{
+    if (dt == DBF_F32)
+        static_cast<float *>(p)[i] = v;
+    else
+        static_cast<__nv_bfloat16 *>(p)[i] = __float2bfloat16_rn(v);
+}
+
+__device__ __forceinline__ float h2f(uint16_t h)
+{
+    return __half2float(__ushort_as_half(h));
+}
+
+}  // namespace dbf

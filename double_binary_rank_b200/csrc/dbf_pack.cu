@@ -1,0 +1,133 @@
+// Sign packing into the one-bit-per-weight layout of dbf.h.
+//
+// LoRDBA page, section 2 ("Arquitetura Central": sign carriers at 1 bit per
+// weight; training pipeline step 2: B = sign(H)); DBF page, section 2 (the
+// factors are {-1, +1} sign matrices).
+//
+// One warp builds one 32-bit word per step with a single ballot: lane L reads
+// the column that bit L of the word holds (bit p < 16 -> column 2p, bit
+// 16 + p -> column 2p + 1), so the ballot result is the packed word itself.
+// The 32 lanes read one 32-column span of the row, which is contiguous.
+#include "dbf_internal.cuh"
+
+namespace dbf {
+namespace {
+
+template <typename T>
+__device__ __forceinline__ bool is_negative(T v, bool &nan);
+
+template <>
+__device__ __forceinline__ bool is_negative<int8_t>(int8_t v, bool &nan)
+{
+    nan = false;
+    return v < 0;
+}
+template <>
+__device__ __forceinline__ bool is_negative<float>(float v, bool &nan)
+{
+    nan = isnan(v);
+    return v < 0.0f;   // -0.0 and NaN compare false -> +1
+}
+template <>
+__device__ __forceinline__ bool is_negative<__half>(__half v, bool &nan)
+{
+    float f = __half2float(v);
+    nan = isnan(f);
+    return f < 0.0f;
+}
+template <>
+__device__ __forceinline__ bool is_negative<__nv_bfloat16>(__nv_bfloat16 v, bool &nan)
+{
+    float f = __bfloat162float(v);
+    nan = isnan(f);
+    return f < 0.0f;
+}
+
+template <typename T>
+__global__ void __launch_bounds__(256) pack_kernel(const T *__restrict__ src, int64_t rows,
+                                                   int64_t k, uint32_t *__restrict__ dst,
+                                                   int32_t *status)
+{
+    const int lane = threadIdx.x & 31;
+    const int64_t pitch = pitch_words(k);
+    const int64_t total = rows * pitch;
+    const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+    const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+    // column of this lane inside a 32-column word
+    const int col = lane < 16 ? 2 * lane : 2 * (lane - 16) + 1;
+    bool saw_nan = false;
+    for (int64_t w = warp; w < total; w += nwarps) {
+        const int64_t row = w / pitch;
+        const int64_t c = (w - row * pitch) * 32 + col;
+        bool neg = false, nan = false;
+        if (c < k) neg = is_negative<T>(src[row * k + c], nan);
+        saw_nan |= nan;
+        const uint32_t word = __ballot_sync(0xffffffffu, neg);
+        if (lane == 0) dst[w] = word;
+    }
+    if (saw_nan && status) atomicExch(status, static_cast<int32_t>(DBF_ERR_INVALID_ARG));
+}
+
+__global__ void __launch_bounds__(256) unpack_kernel(const uint32_t *__restrict__ src, int64_t rows,
+                                                     int64_t k, int8_t *__restrict__ dst)
+{
+    const int64_t pitch = pitch_words(k);
+    const int64_t n = rows * k;
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+         i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const int64_t row = i / k;
+        const int64_t c = i - row * k;
+        const int j = static_cast<int>(c & 31);
+        const int bit = (j & 1) ? 16 + (j >> 1) : (j >> 1);
+        const uint32_t word = src[row * pitch + (c >> 5)];
+        dst[i] = ((word >> bit) & 1u) ? int8_t(-1) : int8_t(1);
+    }
+}
+
+int grid_for(int64_t work, int per_block)
+{
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess)
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    int64_t g = (work + per_block - 1) / per_block;
+    const int64_t cap = static_cast<int64_t>(sms) * 16;
+    if (g > cap) g = cap;
+    if (g < 1) g = 1;
+    return static_cast<int>(g);
+}
+
+}  // namespace
+
+cudaError_t launch_pack(const void *src, dbf_dtype dt, int64_t rows, int64_t k, uint32_t *dst,
+                        int32_t *status, cudaStream_t s)
+{
+    const int64_t words = rows * pitch_words(k);
+    const int grid = grid_for(words, 8);   // 8 warps per block, one word each per step
+    switch (dt) {
+    case DBF_I8:
+        pack_kernel<int8_t><<<grid, 256, 0, s>>>(static_cast<const int8_t *>(src), rows, k, dst, status);
+        break;
+    case DBF_F32:
+        pack_kernel<float><<<grid, 256, 0, s>>>(static_cast<const float *>(src), rows, k, dst, status);
+        break;
+    case DBF_F16:
+        pack_kernel<__half><<<grid, 256, 0, s>>>(static_cast<const __half *>(src), rows, k, dst, status);
+        break;
+    case DBF_BF16:
+        pack_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(static_cast<const __nv_bfloat16 *>(src), rows, k,
+                                                        dst, status);
+        break;
+    default:
+        return cudaErrorInvalidValue;
+    }
+    return cudaGetLastError();
+}
+
+cudaError_t launch_unpack(const uint32_t *src, int64_t rows, int64_t k, int8_t *dst, cudaStream_t s)
+{
+    const int grid = grid_for(rows * k, 256);
+    unpack_kernel<<<grid, 256, 0, s>>>(src, rows, k, dst);
+    return cudaGetLastError();
+}
+
+}  // namespace dbf

@@ -1,0 +1,178 @@
+/*
+ * dbf.h -- C ABI of the B200 (sm_100a) double-binary factorised layer forward.
+ *
+ * The operation (LoRDBA page, section 2 "Arquitetura Central", Delta-W
+ * equation; DBF page, section 2, W ~ (a . A . m^T)(B . b^T) with ell = 1):
+ *
+ *   y[t,:] = [accumulate] y[t,:]
+ *            + sum_{i=1..ell} diag(alpha_i) B1 diag(beta_i) B2 diag(gamma_i) x[t,:]
+ *
+ * with sign matrices B1 in {+-1}^{N x R} and B2 in {+-1}^{R x M} shared by
+ * every envelope i, and fp16 per-channel scales alpha_i (N), beta_i (R),
+ * gamma_i (M). Following the LoRDBA page's inference-kernel paragraph, it is
+ * evaluated as two sign-accumulation products with per-channel scaling
+ * between them: h = B2 (gamma . x), v = beta . h, z = B1 v, y += alpha . z.
+ * The DBF_ACCUMULATE flag adds the branch into an existing output, the
+ * unmerged adapter mode of the LoRDBA page (sections 1, 3 and 5); a
+ * full-weight replacement layer (DBF page, section 2 "Inferencia") calls
+ * without it.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - Every data pointer is a DEVICE pointer owned by the caller. The library
+ *   allocates nothing, keeps no state between calls, never synchronises the
+ *   device and enqueues all work on 'stream' (a cudaStream_t; NULL = the
+ *   legacy default stream).
+ * - Arguments are checked on the host before any launch; a failed check
+ *   returns an error status and launches nothing. Data-dependent faults
+ *   found by a kernel (NaN latents, bad segment tables) are reported through
+ *   an optional device status word: the kernel stores the dbf_status code
+ *   there; it is never cleared by the library.
+ * - Matrices are row-major. x is T x M (token-major), y is T x N.
+ * - Packed sign layout (one bit per weight; LoRDBA page section 2 storage
+ *   efficiency, DBF page section 2): a rows x k sign matrix is stored as rows
+ *   of ceil(k/32) little-endian 32-bit words with no other padding. In word w
+ *   of a row, bit p (0 <= p < 16) holds column k = 32w + 2p and bit 16 + p
+ *   holds column k = 32w + 2p + 1. A set bit is the sign -1, a clear bit +1.
+ *   Bits past the last column are zero. B1 is packed along R (N rows of
+ *   ceil(R/32) words), B2 along M (R rows of ceil(M/32) words), so both are
+ *   packed along their contraction dimension.
+ * - Scales are fp16 bit patterns, laid out [ell][len].
+ */
+#ifndef DBF_H_
+#define DBF_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    DBF_OK = 0,
+    DBF_ERR_INVALID_ARG = 1,   /* null pointer, bad size, bad enum, bad table */
+    DBF_ERR_UNSUPPORTED = 2,   /* valid arguments the requested path cannot serve */
+    DBF_ERR_ALIGNMENT = 3,     /* a pointer misses its required alignment */
+    DBF_ERR_WORKSPACE = 4,     /* workspace null or smaller than *_workspace_bytes */
+    DBF_ERR_CUDA = 5,          /* a CUDA runtime call or launch failed */
+    DBF_ERR_TIMEOUT = 6        /* a bounded device-side wait expired */
+} dbf_status;
+
+typedef enum { DBF_F32 = 0, DBF_BF16 = 1, DBF_F16 = 2, DBF_I8 = 3 } dbf_dtype;
+
+/* Flags of dbf_forward / dbf_forward_segmented (bitwise or).
+ * DBF_ACCUMULATE: y += branch instead of y = branch.
+ * DBF_WEIGHTS_STATIC: the caller promises that the packed sign matrices are
+ *   not written by the work enqueued just before this call on the stream.
+ *   The kernels are launched as programmatic dependents of the preceding
+ *   kernel; with this flag they start streaming the sign matrices before
+ *   that kernel has finished (activations, scales, segment tables and every
+ *   write still wait for it). Without it nothing is read early. */
+enum { DBF_ACCUMULATE = 1, DBF_WEIGHTS_STATIC = 2 };
+
+/* GEMV: the decode kernel (few tokens, bandwidth bound, any shape).
+ * GEMM: the prefill kernel (tcgen05 tensor cores; needs M % 128 == 0,
+ *       R % 128 == 0 and N % 16 == 0).
+ * AUTO: GEMM when the shape allows it and T is at least dbf_gemm_min_tokens(),
+ *       else GEMV. */
+typedef enum { DBF_PATH_AUTO = 0, DBF_PATH_GEMV = 1, DBF_PATH_GEMM = 2 } dbf_path;
+
+/* One layer or adapter. All pointers are device pointers, caller owned.
+ * b1_packed: N rows x ceil(R/32) words; b2_packed: R rows x ceil(M/32) words;
+ * both 16-byte aligned. alpha: fp16 [ell][N]; beta: fp16 [ell][R];
+ * gamma: fp16 [ell][M]; each 2-byte aligned. 1 <= ell <= 8. */
+typedef struct {
+    int32_t M, N, R, ell;
+    const uint32_t *b1_packed;
+    const uint32_t *b2_packed;
+    const uint16_t *alpha;
+    const uint16_t *beta;
+    const uint16_t *gamma;
+} dbf_layer;
+
+/* Bytes of a packed rows x k sign matrix: rows * ceil(k/32) * 4. */
+size_t dbf_packed_bytes(int64_t rows, int64_t k);
+
+/* Pack a rows x k sign source into the packed layout (LoRDBA page, section 2
+ * training pipeline step 2: B = sign(H)).
+ * src: device, rows x k, row-major, dtype DBF_I8 (any value < 0 is -1, others
+ *      +1), or DBF_F32 / DBF_BF16 / DBF_F16 latents H where H < 0 gives -1 and
+ *      H >= 0 (including -0.0) gives +1.
+ * dst: device, dbf_packed_bytes(rows, k) bytes, 4-byte aligned.
+ * status_dev: optional device int32; a NaN latent stores DBF_ERR_INVALID_ARG
+ *      there (its bit is packed as +1).
+ * Errors: DBF_ERR_INVALID_ARG (null, rows or k <= 0, bad dtype, dst_bytes too
+ *      small), DBF_ERR_ALIGNMENT, DBF_ERR_CUDA. */
+dbf_status dbf_pack_signs(const void *src, dbf_dtype src_dtype, int64_t rows, int64_t k,
+                          uint32_t *dst, size_t dst_bytes, int32_t *status_dev, void *stream);
+
+/* Unpack to int8 +-1 (rows x k, row-major). Inverse of dbf_pack_signs on
+ * sign matrices. Errors as dbf_pack_signs. */
+dbf_status dbf_unpack_signs(const uint32_t *src, int64_t rows, int64_t k, int8_t *dst,
+                            void *stream);
+
+/* Smallest T for which DBF_PATH_AUTO takes the GEMM path on a shape it allows. */
+int64_t dbf_gemm_min_tokens(void);
+
+/* Workspace bytes dbf_forward needs for this layer, T and path (AUTO is
+ * resolved as dbf_forward resolves it). Returns 0 for invalid input. */
+size_t dbf_workspace_bytes(const dbf_layer *L, int64_t T, dbf_path path);
+
+/* The forward of one layer (host-side descriptor L).
+ * x: device T x M, DBF_F32 or DBF_BF16, 16-byte aligned.
+ * y: device T x N, DBF_F32 or DBF_BF16, 16-byte aligned; read first when
+ *    flags has DBF_ACCUMULATE. Results are rounded to nearest-even into y's
+ *    dtype.
+ * flags: DBF_ACCUMULATE | DBF_WEIGHTS_STATIC (see above); other bits must be 0.
+ * ws: device workspace of at least dbf_workspace_bytes(L, T, path) bytes,
+ *    256-byte aligned, contents scratch.
+ * T == 0 is a no-op. Numerics: the GEMV path turns each activation column
+ * (gamma.x, then beta.h) into 22-bit fixed point with one power-of-two scale
+ * per column and accumulates sign sums exactly in integers (relative error
+ * about 2^-22 of the column's largest value per element); the GEMM path
+ * rounds gamma.x and beta.h to fp16 operands (|values| below 65504) and
+ * accumulates in fp32.
+ * Errors: DBF_ERR_INVALID_ARG, DBF_ERR_ALIGNMENT, DBF_ERR_WORKSPACE,
+ *    DBF_ERR_UNSUPPORTED (path GEMM on a shape it does not serve), DBF_ERR_CUDA. */
+dbf_status dbf_forward(const dbf_layer *L, const void *x, dbf_dtype x_dtype, void *y,
+                       dbf_dtype y_dtype, int64_t T, int flags, dbf_path path, void *ws,
+                       size_t ws_bytes, void *stream);
+
+/* Workspace bytes dbf_forward_segmented needs. */
+size_t dbf_segmented_workspace_bytes(int32_t max_R, int32_t max_ell, int64_t T);
+
+/* Many adapters served in one call (LoRDBA page, section 1: multi-adapter
+ * serving as in S-LoRA / Punica). Tokens are pre-sorted into S segments:
+ * tokens seg_offsets_dev[s] .. seg_offsets_dev[s+1]-1 use adapter
+ * seg_adapter_dev[s]. An adapter id of -1 means no adapter: those rows get a
+ * zero branch (y is left as is when accumulating, else set to 0).
+ * adapters_dev: device array of num_adapters dbf_layer descriptors, each with
+ *    the given M and N, R <= max_R and ell <= max_ell (ell <= 8).
+ * seg_offsets_dev: device int32 [S+1], nondecreasing, from 0 to T.
+ * seg_adapter_dev: device int32 [S].
+ * x, y, flags as in dbf_forward (decode-path numerics; DBF_WEIGHTS_STATIC
+ *    has no effect here because the segment tables are read first).
+ * status_dev: optional device int32. A segment whose adapter id is outside
+ *    [-1, num_adapters) or whose descriptor does not match M, N, max_R,
+ *    max_ell, or an offsets table that is not nondecreasing within [0, T],
+ *    stores DBF_ERR_INVALID_ARG there and that segment is skipped.
+ * Errors: as dbf_forward. */
+dbf_status dbf_forward_segmented(const dbf_layer *adapters_dev, int32_t num_adapters,
+                                 const int32_t *seg_offsets_dev, const int32_t *seg_adapter_dev,
+                                 int32_t S, int32_t max_R, int32_t max_ell, int32_t M, int32_t N,
+                                 const void *x, dbf_dtype x_dtype, void *y, dbf_dtype y_dtype,
+                                 int64_t T, int flags, void *ws, size_t ws_bytes,
+                                 int32_t *status_dev, void *stream);
+
+/* Static description of a status code. */
+const char *dbf_status_string(dbf_status s);
+
+/* Library version string. */
+const char *dbf_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DBF_H_ */

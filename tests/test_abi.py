@@ -1,0 +1,114 @@
+"""The C ABI library loads and exports every symbol include/dbf.h declares;
+host-side argument checks (which return before any CUDA call) behave."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "dbf.h")
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(dbf_[a-z_0-9]+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    import double_binary_rank_b200 as dbf
+    return dbf._lib
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for n in ("dbf_pack_signs", "dbf_forward", "dbf_forward_segmented", "dbf_unpack_signs",
+              "dbf_workspace_bytes", "dbf_packed_bytes", "dbf_status_string"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_binding_covers_header():
+    import double_binary_rank_b200 as dbf
+    assert sorted(dbf.EXPORTED) == declared_functions()
+
+
+def test_packed_bytes(lib):
+    import double_binary_rank_b200 as dbf
+    assert dbf.packed_bytes(3, 33) == 3 * 2 * 4
+    assert dbf.packed_bytes(11008, 5888) == 8101888
+    assert dbf.packed_bytes(5888, 4096) == 3014656
+    assert dbf.packed_bytes(0, 5) == 0
+
+
+def test_status_strings(lib):
+    import double_binary_rank_b200 as dbf
+    assert dbf.status_string(dbf.OK) == "ok"
+    assert "workspace" in dbf.status_string(dbf.ERR_WORKSPACE)
+    assert dbf.version().startswith("dbf-b200")
+
+
+def _layer(M=64, N=48, R=32, ell=1, p=0x1000):
+    import double_binary_rank_b200 as dbf
+    return dbf.DbfLayerC(M, N, R, ell, p, p, p, p, p)
+
+
+def test_forward_rejects_bad_arguments_without_launch(lib):
+    import double_binary_rank_b200 as dbf
+    L = _layer()
+    f = lib.dbf_forward
+    by = ctypes.byref
+    assert f(None, 0x1000, dbf.F32, 0x1000, dbf.F32, 4, 0, 0, 0x1000, 1 << 20, None) == dbf.ERR_INVALID_ARG
+    assert f(by(_layer(ell=0)), 0x1000, dbf.F32, 0x1000, dbf.F32, 4, 0, 0, 0x1000, 1 << 20, None) == dbf.ERR_INVALID_ARG
+    assert f(by(_layer(ell=9)), 0x1000, dbf.F32, 0x1000, dbf.F32, 4, 0, 0, 0x1000, 1 << 20, None) == dbf.ERR_INVALID_ARG
+    assert f(by(_layer(R=-1)), 0x1000, dbf.F32, 0x1000, dbf.F32, 4, 0, 0, 0x1000, 1 << 20, None) == dbf.ERR_INVALID_ARG
+    assert f(by(L), 0x1000, dbf.F16, 0x1000, dbf.F32, 4, 0, 0, 0x1000, 1 << 20, None) == dbf.ERR_INVALID_ARG
+    assert f(by(L), 0x1000, dbf.F32, 0x1000, dbf.I8, 4, 0, 0, 0x1000, 1 << 20, None) == dbf.ERR_INVALID_ARG
+    assert f(by(L), 0x1000, dbf.F32, 0x1000, dbf.F32, 4, 0, 7, 0x1000, 1 << 20, None) == dbf.ERR_INVALID_ARG
+    assert f(by(L), 0x1000, dbf.F32, 0x1000, dbf.F32, 4, 4, 0, 0x1000, 1 << 20, None) == dbf.ERR_INVALID_ARG
+    assert f(by(L), 0x1008, dbf.F32, 0x1000, dbf.F32, 4, 0, 0, 0x1000, 1 << 20, None) == dbf.ERR_ALIGNMENT
+    assert f(by(L), 0x1000, dbf.F32, 0x1004, dbf.F32, 4, 0, 0, 0x1000, 1 << 20, None) == dbf.ERR_ALIGNMENT
+    assert f(by(_layer(p=0x1004)), 0x1000, dbf.F32, 0x1000, dbf.F32, 4, 0, 0, 0x1000, 1 << 20, None) == dbf.ERR_ALIGNMENT
+    assert f(by(L), 0x1000, dbf.F32, 0x1000, dbf.F32, 4, 0, 0, None, 0, None) == dbf.ERR_WORKSPACE
+    assert f(by(L), 0x1000, dbf.F32, 0x1000, dbf.F32, 4, 0, 0, 0x1000, 16, None) == dbf.ERR_WORKSPACE
+    # GEMM path needs M % 128 == 0 and R % 128 == 0
+    assert f(by(L), 0x1000, dbf.F32, 0x1000, dbf.F32, 4, 0, dbf.PATH_GEMM, 0x1000, 1 << 30, None) == dbf.ERR_UNSUPPORTED
+    # T == 0 is a no-op
+    assert f(by(L), None, dbf.F32, None, dbf.F32, 0, 0, 0, None, 0, None) == dbf.OK
+
+
+def test_workspace_query(lib):
+    import double_binary_rank_b200 as dbf
+    L = _layer(M=64, N=48, R=32, ell=2)
+    ws = lib.dbf_workspace_bytes(ctypes.byref(L), 5, dbf.PATH_GEMV)
+    assert ws >= 5 * 2 * 32 * 4 and ws % 256 == 0
+    assert lib.dbf_workspace_bytes(None, 5, dbf.PATH_GEMV) == 0
+    assert lib.dbf_segmented_workspace_bytes(32, 2, 256) >= 256 * 2 * 32 * 4
+
+
+def test_pack_rejects_bad_arguments(lib):
+    import double_binary_rank_b200 as dbf
+    f = lib.dbf_pack_signs
+    assert f(None, dbf.I8, 4, 4, 0x1000, 16, None, None) == dbf.ERR_INVALID_ARG
+    assert f(0x1000, dbf.I8, 0, 4, 0x1000, 16, None, None) == dbf.ERR_INVALID_ARG
+    assert f(0x1000, dbf.I8, 4, 40, 0x1000, 16, None, None) == dbf.ERR_INVALID_ARG   # dst too small
+    assert f(0x1000, 9, 4, 4, 0x1000, 16, None, None) == dbf.ERR_INVALID_ARG
+    assert f(0x1002, dbf.F32, 4, 4, 0x1000, 16, None, None) == dbf.ERR_ALIGNMENT
+    assert f(0x1000, dbf.I8, 4, 4, 0x1002, 16, None, None) == dbf.ERR_ALIGNMENT
+
+
+def test_segmented_rejects_bad_arguments(lib):
+    import double_binary_rank_b200 as dbf
+    f = lib.dbf_forward_segmented
+    a = 0x1000
+    assert f(a, 4, a, a, 3, 0, 1, 64, 64, a, dbf.F32, a, dbf.F32, 8, 0, a, 1 << 20, None, None) == dbf.ERR_INVALID_ARG
+    assert f(a, 4, a, a, 3, 32, 9, 64, 64, a, dbf.F32, a, dbf.F32, 8, 0, a, 1 << 20, None, None) == dbf.ERR_INVALID_ARG
+    assert f(a, 4, a, a, 3, 32, 1, 64, 64, a, dbf.F32, a, dbf.F32, 8, 0, None, 0, None, None) == dbf.ERR_WORKSPACE
+    assert f(a, 4, a + 2, a, 3, 32, 1, 64, 64, a, dbf.F32, a, dbf.F32, 8, 0, a, 1 << 20, None, None) == dbf.ERR_ALIGNMENT
+    assert f(a, 4, a, a, 0, 32, 1, 64, 64, a, dbf.F32, a, dbf.F32, 8, 0, None, 0, None, None) == dbf.OK
