@@ -44,7 +44,6 @@ constexpr int kMaxNcl = kMaxBcols / kPlanes;   // logical columns per pass (8)
 constexpr int kGroupWords = 8;     // words per work unit (256 columns of K)
 constexpr int kWarps = 8;
 constexpr int kThreads = kWarps * 32;
-constexpr int kQuadRound = 8;      // quads (4 columns of K) per thread per load round
 constexpr int kMaxCtas = 160;      // per segment; sizes the per-CTA partial sums
 constexpr int kSmemCap = 220 * 1024;
 constexpr int kPrefetchCap = 128 * 1024;
@@ -197,21 +196,6 @@ __device__ __forceinline__ float scale_pow2(float v, int e)
 
 // |q| <= 2^22 for every value below 'bound': sh = 22 - e with bound < 2^e
 __device__ __forceinline__ int scale_exponent(float bound) { return bound > 0.f ? 22 - (ilogbf(bound) + 1) : 0; }
-
-// balanced base-256 digits of q (|q| <= 2^22)
-__device__ __forceinline__ void digits3(int q, int &d0, int &d1, int &d2)
-{
-    d0 = ((q + 128) & 255) - 128;
-    const int q1 = (q - d0) >> 8;
-    d1 = ((q1 + 128) & 255) - 128;
-    d2 = (q1 - d1) >> 8;
-}
-
-__device__ __forceinline__ uint32_t pack4(int a, int b, int c, int d)
-{
-    return (static_cast<uint32_t>(a) & 255u) | ((static_cast<uint32_t>(b) & 255u) << 8) |
-           ((static_cast<uint32_t>(c) & 255u) << 16) | (static_cast<uint32_t>(d) << 24);
-}
 
 __device__ __forceinline__ long long warp_sum64(long long v)
 {

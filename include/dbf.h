@@ -72,8 +72,8 @@ typedef enum { DBF_F32 = 0, DBF_BF16 = 1, DBF_F16 = 2, DBF_I8 = 3 } dbf_dtype;
 enum { DBF_ACCUMULATE = 1, DBF_WEIGHTS_STATIC = 2 };
 
 /* GEMV: the decode kernel (few tokens, bandwidth bound, any shape).
- * GEMM: the prefill kernel (tcgen05 tensor cores; needs M % 128 == 0,
- *       R % 128 == 0 and N % 16 == 0).
+ * GEMM: the prefill kernel (tcgen05 tensor cores; needs M % 128 == 0 and
+ *       R % 128 == 0; any N).
  * AUTO: GEMM when the shape allows it and T is at least dbf_gemm_min_tokens(),
  *       else GEMV. */
 typedef enum { DBF_PATH_AUTO = 0, DBF_PATH_GEMV = 1, DBF_PATH_GEMM = 2 } dbf_path;

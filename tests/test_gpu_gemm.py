@@ -1,0 +1,103 @@
+"""The tcgen05 prefill path (DBF_PATH_GEMM) against the fp64 oracle.
+
+The GEMM rounds gamma.x and beta.h to fp16 operands and accumulates in fp32,
+so its error is a few 1e-4 of max|y|, inside the 2e-3 contract. Integer
+inputs chosen so that every fp16 operand and fp32 sum is exact must give
+bit-identical results: that pins the shared-memory layouts, descriptors,
+tile indexing and the alpha fold independently of rounding.
+"""
+import numpy as np
+import pytest
+import torch
+
+import dbf_synth as S
+import oracle
+from gpu_util import TOL, bf16_ok, dev_layer, dev_x, host_y, random_layer, rel_err
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def dbf():
+    import double_binary_rank_b200 as m
+    return m
+
+
+def run(dbf, L, x, y_dtype=torch.float32, acc=False, y_in=None, path="gemm"):
+    dl = dev_layer(L)
+    y = torch.from_numpy(y_in).cuda().to(y_dtype) if acc else None
+    out = dbf.forward(dl, dev_x(x), y=y, accumulate=acc, path=path, y_dtype=y_dtype)
+    torch.cuda.synchronize()
+    return host_y(out)
+
+
+def exact_layer(rng, M, N, R, ell):
+    b1 = rng.choice(np.array([-1, 1], dtype=np.int8), size=(N, R))
+    b2 = rng.choice(np.array([-1, 1], dtype=np.int8), size=(R, M))
+    f = lambda vals, n: S.to_f16_bits(rng.choice(vals, n))
+    return S.Layer(M, N, R, ell, b1, b2,
+                   np.stack([f([0.5, 1.0, 2.0, -0.5, -1.0, -2.0], N) for _ in range(ell)]),
+                   np.stack([f([1.0, 2.0, -1.0, -2.0], R) for _ in range(ell)]),
+                   np.stack([f([1.0, -1.0], M) for _ in range(ell)]))
+
+
+@pytest.mark.parametrize("shape", [(128, 16, 128, 1, 1), (256, 200, 128, 1, 7), (128, 136, 256, 2, 300),
+                                   (384, 64, 128, 3, 33)], ids=lambda s: "M{}N{}R{}l{}T{}".format(*s))
+def test_gemm_exact_bit_identical(dbf, shape):
+    M, N, R, ell, T = shape
+    rng = np.random.default_rng(sum(shape))
+    L = exact_layer(rng, M, N, R, ell)
+    x = rng.integers(-1, 2, size=(T, M)).astype(np.float32)
+    ref = oracle.forward(L, x)
+    got = run(dbf, L, x)
+    assert np.array_equal(got, ref), float(np.max(np.abs(got - ref)))
+
+
+@pytest.mark.parametrize("shape", [(128, 48, 128, 1, 5), (512, 300, 384, 2, 260), (256, 1024, 256, 1, 513)],
+                         ids=lambda s: "M{}N{}R{}l{}T{}".format(*s))
+@pytest.mark.parametrize("acc", [False, True])
+def test_gemm_random(dbf, shape, acc):
+    M, N, R, ell, T = shape
+    rng = np.random.default_rng(sum(shape) + 7)
+    L = random_layer(rng, M, N, R, ell)
+    x = S.to_bf16_bits(rng.standard_normal((T, M)))
+    y_in = rng.standard_normal((T, N)).astype(np.float32)
+    ref = oracle.forward(L, x, y_in=y_in, accumulate=acc)
+    got = run(dbf, L, x, acc=acc, y_in=y_in)
+    assert rel_err(got, ref) < TOL
+
+
+def test_gemm_matches_gemv(dbf):
+    rng = np.random.default_rng(70)
+    L = random_layer(rng, 256, 160, 128, 2)
+    x = S.to_bf16_bits(rng.standard_normal((40, 256)))
+    a = run(dbf, L, x, path="gemm")
+    b = run(dbf, L, x, path="gemv")
+    assert rel_err(a, b) < TOL
+
+
+def test_dbf_mlp_prefill_sampled_rows(dbf):
+    # the DBF MLP layer at 2048 tokens, checked on a fixed sample of token rows
+    w = S.WORKLOADS["dbf_mlp"]
+    L = S.workload_layers(w)[0]
+    T = 2048
+    x = S.make_x(w.seed, T, w.M, "bf16")
+    rows = S.sample_rows(w.seed, T, 64)
+    ref = oracle.forward(L, x, rows=rows)
+    got = run(dbf, L, x, y_dtype=torch.float32)[rows]
+    assert rel_err(got, ref) < TOL
+    got_b = run(dbf, L, x, y_dtype=torch.bfloat16)[rows]
+    ok, worst = bf16_ok(got_b, ref)
+    assert ok, worst
+
+
+def test_large_prefill_sampled_rows(dbf):
+    # M = N = R = 8192 at 8192 tokens, checked on a fixed sample of token rows
+    w = S.WORKLOADS["large_prefill"]
+    L = S.workload_layers(w)[0]
+    T = 8192
+    x = S.make_x(w.seed, T, w.M, "bf16")
+    rows = S.sample_rows(w.seed, T, 32)
+    ref = oracle.forward(L, x, rows=rows)
+    got = run(dbf, L, x, y_dtype=torch.float32)[rows]
+    assert rel_err(got, ref) < TOL
