@@ -1,0 +1,352 @@
+"""Benchmark of the double-binary layer forward on B200.
+
+Workload: the DBF full-weight MLP layer (DBF page, section 2 form with
+ell = 1): M = 4096 inputs, N = 11008 outputs, R = 5888 (~1.97 bits/weight),
+bf16 activations ~ N(0, 1), iid +-1 factors, fp16 lognormal(0, 0.5) scales.
+One step runs the whole forward (gamma scaling, sign accumulation over B2,
+beta scaling, sign accumulation over B1, alpha scaling, write) twice: once
+in the decode regime (1 token) and once in the prefill regime (2048 tokens).
+Reported: tokens/s for the whole job, the decode kernel pair against the HBM
+roofline and the prefill pair against the tensor-core roofline.
+
+L2: every step reads a different one of 24 device copies of the layer
+(24 x 11.2 MB, more than twice the 126 MB L2), so the sign matrices come
+from HBM. Multi-GPU (torchrun): each rank runs the same per-GPU work
+(weak scaling); the timing is the max over ranks.
+
+python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import dbf_synth as S  # noqa: E402
+
+METRIC = "DBF layer tokens/s; HBM GB/s (decode) & tensor TFLOP/s (prefill) vs roofline"
+WORKLOAD = "dbf_mlp"
+T_DECODE = 1
+T_PREFILL = 2048
+COPIES = 24
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_traffic(key: str, src: str):
+    """DRAM bytes per launch from profiles/traffic.txt, or None when the
+    kernel source changed since the counters were taken."""
+    path = os.path.join(ROOT, "profiles", "traffic.txt")
+    if not os.path.exists(path):
+        return None
+    with open(os.path.join(ROOT, src), "rb") as f:
+        digest = hashlib.sha256(f.read()).hexdigest()[:16]
+    with open(path) as f:
+        for line in f:
+            parts = line.split()
+            if len(parts) >= 3 and parts[0] == key and not line.startswith("#"):
+                return float(parts[2]) if parts[1] == digest else None
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+
+    def __init__(self, index: int):
+        self.index = index
+        self.samples = []
+        self.proc = None
+        self.thread = None
+
+    def __enter__(self):
+        cmd = ["nvidia-smi", "-i", str(self.index), "--query-gpu=clocks.sm,clocks.max.sm,power.draw,"
+               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap",
+               "--format=csv,noheader,nounits", "-lms", "100"]
+        try:
+            self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return self
+
+        def reader():
+            for line in self.proc.stdout:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 7:
+                    self.samples.append(parts)
+
+        self.thread = threading.Thread(target=reader, daemon=True)
+        self.thread.start()
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+        if self.thread is not None:
+            self.thread.join(timeout=2)
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = []
+        smax = None
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        seen = set()
+        for p in self.samples:
+            try:
+                sm.append(float(p[0]))
+                smax = float(p[1])
+            except ValueError:
+                continue
+            for name, val in zip(names, p[3:7]):
+                if val.lower() == "active":
+                    seen.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax, "reasons": sorted(seen),
+                "samples": len(sm)}
+
+
+def algorithmic(w, T):
+    """Algorithmic bytes and flops of one forward call (decode-path numbers
+    count the packed signs, scales, x in and y out)."""
+    sign_bytes = w.R * (w.M + w.N) / 8
+    scale_bytes = 2 * w.ell * (w.M + w.N + w.R)
+    act_bytes = T * w.M * 2 + T * w.N * 2
+    flops = 2 * T * w.ell * w.R * (w.M + w.N)
+    return sign_bytes + scale_bytes + act_bytes, flops
+
+
+def oracle_sample_rate(w, L, x_dec, x_pre, rows, nthreads):
+    """The fp64 oracle on a bounded sample: tokens / second on host cores."""
+    import oracle
+    t0 = time.perf_counter()
+    oracle.forward(L, x_dec, nthreads=nthreads)
+    oracle.forward(L, x_pre, rows=rows, nthreads=nthreads)
+    dt = time.perf_counter() - t0
+    return (1 + len(rows)) / dt, dt
+
+
+def run_reference(args, rank, world):
+    """Reference arm: the fp64 CPU oracle, timed on the host cores."""
+    import oracle
+    w = S.WORKLOADS[WORKLOAD]
+    if world > 1 and rank != 0:
+        return
+    L = S.workload_layers(w)[0]
+    x_dec = S.make_x(w.seed, T_DECODE, w.M, "bf16")
+    x_pre = S.make_x(w.seed + 100, T_PREFILL, w.M, "bf16")
+    rows = S.sample_rows(w.seed, T_PREFILL, 7)
+    nthreads = oracle.default_threads()
+    for _ in range(args.warmup):
+        oracle_sample_rate(w, L, x_dec, x_pre, rows[:1], nthreads)
+    tokens = 0
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        rate, dt = oracle_sample_rate(w, L, x_dec, x_pre, rows, nthreads)
+        tokens += 1 + len(rows)
+    dt = time.perf_counter() - t0
+    value = tokens / dt
+    sample = f"per step: 1 decode token + {len(rows)} of the {T_PREFILL} prefill tokens (fixed seeded rows)"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * dt / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.description, "decode_tokens": T_DECODE, "prefill_tokens": T_PREFILL},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": nthreads, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1500)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+
+    import torch
+    import torch.distributed as dist
+    import double_binary_rank_b200 as dbf
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    w = S.WORKLOADS[WORKLOAD]
+    L = S.workload_layers(w)[0]
+    base = dbf.Layer.from_signs(torch.from_numpy(L.b1).to(dev), torch.from_numpy(L.b2).to(dev),
+                                torch.from_numpy(L.alpha.view(np.float16)).to(dev),
+                                torch.from_numpy(L.beta.view(np.float16)).to(dev),
+                                torch.from_numpy(L.gamma.view(np.float16)).to(dev))
+    layers = [base] + [dbf.Layer(base.M, base.N, base.R, base.ell, base.b1.clone(), base.b2.clone(),
+                                 base.alpha.clone(), base.beta.clone(), base.gamma.clone())
+                       for _ in range(COPIES - 1)]
+    x_dec_h = S.make_x(w.seed, T_DECODE, w.M, "bf16")
+    x_pre_h = S.make_x(w.seed + 100, T_PREFILL, w.M, "bf16")
+    to_dev = lambda a: torch.from_numpy(a.view(np.int16)).to(dev).view(torch.bfloat16)
+    x_dec, x_pre = to_dev(x_dec_h), to_dev(x_pre_h)
+    y_dec = torch.empty((T_DECODE, w.N), dtype=torch.bfloat16, device=dev)
+    y_pre = torch.empty((T_PREFILL, w.N), dtype=torch.bfloat16, device=dev)
+    ws_dec = dbf.alloc_workspace(dbf.workspace_bytes(base, T_DECODE), dev)
+    ws_pre = dbf.alloc_workspace(dbf.workspace_bytes(base, T_PREFILL), dev)
+    stream = torch.cuda.Stream(device=dev)
+
+    def step(i, ev=None):
+        Lk = layers[i % COPIES]
+        if ev is not None:
+            ev[0].record(stream)
+        dbf.forward(Lk, x_dec, y=y_dec, ws=ws_dec, static_weights=True, stream=stream)
+        if ev is not None:
+            ev[1].record(stream)
+        dbf.forward(Lk, x_pre, y=y_pre, ws=ws_pre, static_weights=True, stream=stream)
+        if ev is not None:
+            ev[2].record(stream)
+
+    with torch.cuda.stream(stream):
+        for i in range(args.warmup):
+            step(i)
+    torch.cuda.synchronize(dev)
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local) as clk:
+        with torch.cuda.stream(stream):
+            t_start.record(stream)
+            for i in range(args.steps):
+                step(i, evs[i])
+            t_end.record(stream)
+        torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    elapsed_ms = t_start.elapsed_time(t_end)
+    if world > 1:
+        tt = torch.tensor([elapsed_ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        elapsed_ms = float(tt.item())
+    dec_us = statistics.mean(1e3 * e[0].elapsed_time(e[1]) for e in evs)
+    pre_us = statistics.mean(1e3 * e[1].elapsed_time(e[2]) for e in evs)
+    tokens_per_step = T_DECODE + T_PREFILL
+    value = world * tokens_per_step * args.steps / (elapsed_ms * 1e-3)
+
+    # ---- end to end through the public API: host buffers, copies timed
+    x_dec_pin = torch.from_numpy(x_dec_h.view(np.int16)).view(torch.bfloat16).pin_memory()
+    x_pre_pin = torch.from_numpy(x_pre_h.view(np.int16)).view(torch.bfloat16).pin_memory()
+    y_dec_pin = torch.empty((T_DECODE, w.N), dtype=torch.bfloat16).pin_memory()
+    y_pre_pin = torch.empty((T_PREFILL, w.N), dtype=torch.bfloat16).pin_memory()
+    e2e_steps = max(3, args.steps // 5)
+
+    def e2e_step(i):
+        x_dec.copy_(x_dec_pin, non_blocking=True)
+        x_pre.copy_(x_pre_pin, non_blocking=True)
+        step(i)
+        y_dec_pin.copy_(y_dec, non_blocking=True)
+        y_pre_pin.copy_(y_pre, non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        e2e_step(0)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for i in range(e2e_steps):
+            e2e_step(i)
+        e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = e0.elapsed_time(e1)
+    if world > 1:
+        tt = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        e2e_ms = float(tt.item())
+    e2e_value = world * tokens_per_step * e2e_steps / (e2e_ms * 1e-3)
+    h2d = x_dec_pin.numel() * 2 + x_pre_pin.numel() * 2
+    d2h = y_dec_pin.numel() * 2 + y_pre_pin.numel() * 2
+
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+
+    pk, pk_kind = peaks()
+    b_dec, f_dec = algorithmic(w, T_DECODE)
+    b_pre, f_pre = algorithmic(w, T_PREFILL)
+    gbs = b_dec / (dec_us * 1e-6) / 1e9
+    tfs = f_pre / (pre_us * 1e-6) / 1e12
+    roof_pre = {"bound": "tensor", "achieved": tfs, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": tfs / pk["bf16_tflops"], "traffic": kernel_traffic("gemm_prefill", "double_binary_rank_b200/csrc/dbf_gemm.cu"),
+                "kernel": "prefill forward (fp16 operand pre-pass + two tcgen05 GEMM launches), one call",
+                "peak_source": f"{pk_kind} bf16 dense (fp16 runs at the same rate)"}
+    roof_dec = {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                "frac": gbs / pk["hbm_gbs"], "traffic": kernel_traffic("gemv_decode", "double_binary_rank_b200/csrc/dbf_gemv.cu"),
+                "kernel": "decode forward (two GEMV launches), one call", "peak_source": f"{pk_kind} copy bandwidth",
+                "us_per_call": dec_us}
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f16", "data": "synthetic",
+        "config": {"workload": w.description, "decode_tokens": T_DECODE, "prefill_tokens": T_PREFILL,
+                   "l2": f"inputs larger than L2: {COPIES} rotating copies of the layer weights",
+                   "arithmetic": "prefill: fp16 x fp16 tensor cores, fp32 accumulate; decode: u8 x s8 tensor cores, exact int32 accumulate"},
+        "roofline": roof_pre,
+        "roofline_decode": roof_dec,
+        "prefill_us_per_call": pre_us,
+        "clocks": clk.summary(),
+        "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": args.steps * 5,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        import oracle
+        nthreads = oracle.default_threads()
+        rows = S.sample_rows(w.seed, T_PREFILL, 1023)
+        rate, dt = oracle_sample_rate(w, L, x_dec_h, x_pre_h, rows, nthreads)
+        line["cpu_baseline"] = {"value": rate, "unit": "tokens/s", "cores": nthreads, "kind": "oracle",
+                                "sample": f"1 decode token + {len(rows)} fixed seeded rows of the {T_PREFILL}-token prefill ({dt:.1f} s)"}
+    print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -4,7 +4,7 @@ Argument marshalling only: every step of the forward runs in the library's
 CUDA kernels (see include/dbf.h for the operation, layouts and errors).
 PyTorch supplies device memory and the current CUDA stream. There is no CPU
 fallback: if the shared library is missing, importing this package raises.
-Build it with ``python -m double_binary_rank_b200.build``.
+Build it with ``python double_binary_rank_b200/build.py``.
 """
 from __future__ import annotations
 
@@ -20,7 +20,7 @@ LIB_PATH = os.path.join(_PKG, "libdbf.so")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(f"{LIB_PATH} is missing: the CUDA library must be built "
-                      "(python -m double_binary_rank_b200.build); there is no CPU fallback")
+                      "(python double_binary_rank_b200/build.py); there is no CPU fallback")
 
 _lib = ctypes.CDLL(LIB_PATH)
 

@@ -3,7 +3,7 @@
 Every CUDA source under csrc/ is compiled for sm_100a only
 (-gencode arch=compute_100a,code=sm_100a) and linked into one shared library
 with the CUDA runtime linked statically, so the library needs nothing from
-torch at load time. Run ``python -m double_binary_rank_b200.build``.
+torch at load time. Run ``python double_binary_rank_b200/build.py``.
 """
 from __future__ import annotations
 
