@@ -55,6 +55,8 @@ _SIGS = {
     "dbf_forward_segmented": (ctypes.c_int, [_vp, _i32, _vp, _vp, _i32, _i32, _i32, _i32, _i32,
                                              _vp, ctypes.c_int, _vp, ctypes.c_int, _i64,
                                              ctypes.c_int, _vp, _sz, _vp, _vp]),
+    "dbf_forward_decode_noalloc": (ctypes.c_int, [_LP, _vp, ctypes.c_int, _vp, ctypes.c_int, _i64,
+                                                  ctypes.c_int, _vp]),
     "dbf_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "dbf_version": (ctypes.c_char_p, []),
 }
@@ -190,6 +192,23 @@ def forward(layer: Layer, x: torch.Tensor, y: Optional[torch.Tensor] = None,
     _check(_lib.dbf_forward(ctypes.byref(d), _ptr(x), _DT[x.dtype], _ptr(y), _DT[y.dtype], T,
                             _flags(accumulate, static_weights), _PATHS[path], _ptr(ws), ws.numel(),
                             _stream(stream)), "dbf_forward")
+    return y
+
+
+def forward_decode_noalloc(layer: Layer, x: torch.Tensor, y: Optional[torch.Tensor] = None,
+                           accumulate: bool = False, y_dtype: Optional[torch.dtype] = None,
+                           stream=None) -> torch.Tensor:
+    """Decode forward with the library's fixed scratch array instead of a
+    workspace (dbf_forward_decode_noalloc), for callers that cannot allocate
+    device memory. At most 1 MiB of decode workspace per call; calls that
+    overlap on the GPU share the array and must be ordered by the caller."""
+    T = x.shape[0]
+    if y is None:
+        y = torch.empty((T, layer.N), dtype=y_dtype or x.dtype, device=x.device)
+    d = layer.descriptor()
+    _check(_lib.dbf_forward_decode_noalloc(ctypes.byref(d), _ptr(x), _DT[x.dtype], _ptr(y), _DT[y.dtype], T,
+                                           _flags(accumulate, False), _stream(stream)),
+           "dbf_forward_decode_noalloc")
     return y
 
 

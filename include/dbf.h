@@ -165,6 +165,29 @@ dbf_status dbf_forward_segmented(const dbf_layer *adapters_dev, int32_t num_adap
                                  int64_t T, int flags, void *ws, size_t ws_bytes,
                                  int32_t *status_dev, void *stream);
 
+/* Decode forward without a caller workspace. The papers have no counterpart
+ * to this entry point; it exists for callers that cannot allocate device
+ * memory (a framework or serving runtime that owns every allocation, or a
+ * thread that must not call cudaMalloc because it may synchronise the device
+ * or fail under a memory cap). It runs the same decode (GEMV) kernels as
+ * dbf_forward with DBF_PATH_GEMV, taking its scratch memory from a fixed
+ * 1 MiB device array inside the library (one copy on every GPU that loads
+ * the library, held until the process exits). It allocates nothing and
+ * calls no allocating routine.
+ * Arguments as dbf_forward, without path and workspace.
+ * Limit: the decode workspace of the call (dbf_workspace_bytes(L, T,
+ * DBF_PATH_GEMV)) must be at most 1 MiB (1048576 bytes), else
+ * DBF_ERR_WORKSPACE; that is ell*T <= 55 at R = 5888, M = 4096.
+ * The first call on each device looks the array's device address up once
+ * (cudaGetSymbolAddress, with that device current); make that first call
+ * before any stream capture. Every call on a device shares the array and it
+ * keeps the last call's contents; nothing in it needs to start at zero, but
+ * calls whose work overlaps on the GPU race on it and must be ordered by the
+ * caller. Errors: as dbf_forward, and DBF_ERR_CUDA if the address lookup
+ * fails. */
+dbf_status dbf_forward_decode_noalloc(const dbf_layer *L, const void *x, dbf_dtype x_dtype, void *y,
+                                      dbf_dtype y_dtype, int64_t T, int flags, void *stream);
+
 /* Static description of a status code. */
 const char *dbf_status_string(dbf_status s);
 
