@@ -129,6 +129,23 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
+def max_over_ranks(value: float, device=None) -> float:
+    """Max of a per-rank timing over all ranks (the job's time is the slowest
+    rank's); the identity without a process group."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def weak_scaling_value(world: int, tokens_per_step: int, steps: int, elapsed_ms: float) -> float:
+    """Whole-job tokens/s: every rank processes tokens_per_step per step."""
+    return world * tokens_per_step * steps / (elapsed_ms * 1e-3)
+
+
 def algorithmic(w, T):
     """Algorithmic bytes and flops of one forward call (decode-path numbers
     count the packed signs, scales, x in and y out)."""
@@ -259,15 +276,11 @@ def main():
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize(dev)
-    elapsed_ms = t_start.elapsed_time(t_end)
-    if world > 1:
-        tt = torch.tensor([elapsed_ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        elapsed_ms = float(tt.item())
+    elapsed_ms = max_over_ranks(t_start.elapsed_time(t_end), dev)
     dec_us = statistics.mean(1e3 * e[0].elapsed_time(e[1]) for e in evs)
     pre_us = statistics.mean(1e3 * e[1].elapsed_time(e[2]) for e in evs)
     tokens_per_step = T_DECODE + T_PREFILL
-    value = world * tokens_per_step * args.steps / (elapsed_ms * 1e-3)
+    value = weak_scaling_value(world, tokens_per_step, args.steps, elapsed_ms)
 
     # ---- end to end through the public API: host buffers, copies timed
     x_dec_pin = torch.from_numpy(x_dec_h.view(np.int16)).view(torch.bfloat16).pin_memory()
@@ -295,12 +308,8 @@ def main():
             e2e_step(i)
         e1.record(stream)
     torch.cuda.synchronize(dev)
-    e2e_ms = e0.elapsed_time(e1)
-    if world > 1:
-        tt = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        e2e_ms = float(tt.item())
-    e2e_value = world * tokens_per_step * e2e_steps / (e2e_ms * 1e-3)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), dev)
+    e2e_value = weak_scaling_value(world, tokens_per_step, e2e_steps, e2e_ms)
     h2d = x_dec_pin.numel() * 2 + x_pre_pin.numel() * 2
     d2h = y_dec_pin.numel() * 2 + y_pre_pin.numel() * 2
 

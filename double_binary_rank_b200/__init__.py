@@ -167,7 +167,8 @@ def workspace_bytes(layer: Layer, T: int, path: str = "auto") -> int:
 
 
 def alloc_workspace(nbytes: int, device) -> torch.Tensor:
-    return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+    # zeroed: the first 256 bytes are a header that must start at zero
+    return torch.zeros(max(int(nbytes), 256), dtype=torch.uint8, device=device)
 
 
 def _flags(accumulate: bool, static_weights: bool) -> int:

@@ -9,19 +9,25 @@
 // In stage 2 the envelope sum is one longer contraction (K = ell R) whose A
 // operand is the exact fp16 product alpha_i[n] * (+-1).
 //
-// One CTA computes a 128 x 256 tile of D = A B^T (A: 128 sign rows, B: 256
-// token rows) with the accumulator in tensor memory:
+// Persistent kernel, one CTA per SM; each CTA walks 128 x 256 tiles of
+// D = A B^T (A: 128 sign rows, B: 256 token rows) with two 256-column
+// accumulators in tensor memory, so the epilogue of one tile overlaps the
+// K loop of the next:
 //   warp 0      TMA producer: fp16 activation tiles (64 K x 256 rows, 128-byte
-//               swizzle) into a 4-stage ring;
-//   warp 1      allocates 256 TMEM columns; one thread issues tcgen05.mma
-//               (M = 128, N = 256, K = 16) and commits each stage back;
-//   warps 2..5  one sign row per thread: the packed words are streamed with
-//               cp.async into a private ring 7 pairs of K steps ahead and
-//               expanded to exact fp16 +-1 (or +-alpha) pairs -- a shift and
-//               one LOP3 per two signs, the packed layout keeping columns 2p and
-//               2p+1 in bits p and 16+p -- written in the same 128-byte swizzled
-//               K-major layout; after the K loop the same warps read the
-//               accumulator back (tcgen05.ld) and run the epilogue.
+//               swizzle) into a 5-stage ring;
+//   warp 1      allocates 512 TMEM columns; one thread issues tcgen05.mma
+//               (M = 128, N = 256, K = 16) into the free accumulator and
+//               commits each stage back;
+//   warps 2..5  sign expansion, one tile row per thread: the row's packed
+//               words are read 16 bytes (two K steps) at a time into a
+//               register queue four loads deep, by a cursor that walks the
+//               CTA's tiles without divisions, and expanded to exact fp16 +-1
+//               (or +-alpha) pairs -- a shift and one LOP3 per two signs, the
+//               packed layout keeping columns 2p and 2p+1 in bits p and 16+p --
+//               written in the same 128-byte swizzled K-major layout;
+//   warps 6..9  epilogue, one per lane quarter: tcgen05.ld of a finished
+//               accumulator, scaling, stores, then the accumulator is handed
+//               back to the MMA warp.
 // Every wait is bounded; on expiry the CTA records DBF_ERR_TIMEOUT, stops
 // issuing work, and still frees its tensor memory.
 #include "dbf_internal.cuh"
@@ -35,12 +41,15 @@ namespace {
 constexpr int BM = 128;             // sign rows per tile (MMA M)
 constexpr int BN = 256;             // token rows per tile (MMA N)
 constexpr int BK = 64;              // K per stage: one 128-byte swizzle row of fp16
-constexpr int STAGES = 4;
-constexpr int kThreads = 192;
+constexpr int SA = 6;                // stages of expanded sign tiles (produced on chip)
+constexpr int SB = 4;                // stages of TMA activation tiles
+constexpr int kExpandGroups = 2;      // groups of four expansion warps, alternating pairs of K steps
+constexpr int kExpandWarps = 4 * kExpandGroups;
+constexpr int kEpiWarps = 4;          // one per TMEM lane quarter
+constexpr int kThreads = 32 * (2 + kExpandWarps + kEpiWarps);
 constexpr int A_BYTES = BM * BK * 2;   // 16 KB
 constexpr int B_BYTES = BN * BK * 2;   // 32 KB
-constexpr int RING = 8;                // cp.async ring slots per expansion thread (16 B each)
-constexpr int TMEM_COLS = 256;
+constexpr int TMEM_COLS = 512;          // two 256-column accumulators
 constexpr unsigned long long kWaitNs = 1000000000ull;   // bounded waits: 1 s
 
 struct GemmArgs {
@@ -132,13 +141,6 @@ __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, i
         : "memory");
 }
 
-__device__ __forceinline__ void cp_async16(void *dst, const void *src)
-{
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
 __device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
@@ -196,35 +198,51 @@ __device__ __forceinline__ uint32_t sign_pair(uint32_t w, int p, uint32_t mag2)
 }
 
 struct GemmSmem {
-    uint64_t full_a[STAGES], full_b[STAGES], empty[STAGES], acc_full;
+    uint64_t full_a[SA], empty_a[SA], full_b[SB], empty_b[SB], acc_full[2], acc_empty[2];
     uint32_t tmem_base;
     int abort;
 };
 
+__device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volatile int *abort)
+{
+    bool ok = true;
+    if ((threadIdx.x & 31) == 0) ok = bar_wait(bar, parity, abort);
+    return __shfl_sync(0xffffffffu, ok, 0);
+}
+
+// Persistent: CTA b takes tiles b, b + gridDim.x, ... (token-tile major, so
+// the CTAs running together share activation tiles in L2).
 __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant__ CUtensorMap tmB, const GemmArgs g)
 {
     extern __shared__ uint8_t smem_raw[];
     // 1024-byte alignment for the swizzled tiles
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *smA = smem;
-    uint8_t *smB = smA + STAGES * A_BYTES;
-    uint4 *ring = reinterpret_cast<uint4 *>(smB + STAGES * B_BYTES);   // [RING][128]
-    GemmSmem *sh = reinterpret_cast<GemmSmem *>(ring + RING * BM);
+    uint8_t *smB = smA + SA * A_BYTES;
+    GemmSmem *sh = reinterpret_cast<GemmSmem *>(smB + SB * B_BYTES);
     volatile int *abort = &sh->abort;
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int p0 = blockIdx.x * BM;    // first sign row
-    const int c0 = blockIdx.y * BN;    // first token row
+    const int n_p = (g.P + BM - 1) / BM;
+    const int n_c = (g.C + BN - 1) / BN;
+    const int ntiles = n_p * n_c;
+    const int my_tiles = blockIdx.x < ntiles ? (ntiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
     const int nk = g.Ktot / BK;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < STAGES; ++s) {
-            bar_init(&sh->full_a[s], 128);
-            bar_init(&sh->full_b[s], 1);
-            bar_init(&sh->empty[s], 1);
+        for (int i = 0; i < SA; ++i) {
+            bar_init(&sh->full_a[i], 4);   // the four warps of one expansion group
+            bar_init(&sh->empty_a[i], 1);
         }
-        bar_init(&sh->acc_full, 1);
+        for (int i = 0; i < SB; ++i) {
+            bar_init(&sh->full_b[i], 1);
+            bar_init(&sh->empty_b[i], 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            bar_init(&sh->acc_full[i], 1);
+            bar_init(&sh->acc_empty[i], kEpiWarps);
+        }
         sh->abort = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         asm volatile("prefetch.tensormap [%0];" ::"l"(&tmB) : "memory");
@@ -242,129 +260,200 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
     if (warp == 0) {
         // ---------------- TMA producer ----------------
         if (lane == 0) {
-            for (int s = 0; s < nk; ++s) {
-                const int st = s % STAGES;
-                if (!bar_wait(&sh->empty[st], ((s / STAGES) & 1) ^ 1, abort)) break;
-                bar_expect_tx(&sh->full_b[st], B_BYTES);
-                tma_load_2d(smB + st * B_BYTES, &tmB, s * BK, c0, &sh->full_b[st]);
+            int s = 0;
+            for (int j = 0; j < my_tiles && !*abort; ++j) {
+                const int tile = blockIdx.x + j * gridDim.x;
+                const int c0 = (tile / n_p) * BN;
+                for (int k = 0; k < nk; ++k, ++s) {
+                    const int st = s % SB;
+                    if (!bar_wait(&sh->empty_b[st], ((s / SB) & 1) ^ 1, abort)) break;
+                    bar_expect_tx(&sh->full_b[st], B_BYTES);
+                    tma_load_2d(smB + st * B_BYTES, &tmB, k * BK, c0, &sh->full_b[st]);
+                }
             }
         }
     } else if (warp == 1) {
         // ---------------- MMA issuer ----------------
         if (lane == 0) {
+            int s = 0;
             bool ok = true;
-            for (int s = 0; s < nk && ok; ++s) {
-                const int st = s % STAGES;
-                const uint32_t ph = (s / STAGES) & 1;
-                ok = bar_wait(&sh->full_a[st], ph, abort) && bar_wait(&sh->full_b[st], ph, abort);
+            for (int j = 0; j < my_tiles && ok; ++j) {
+                const int ab = j & 1;
+                ok = bar_wait(&sh->acc_empty[ab], ((j >> 1) & 1) ^ 1, abort);
                 if (!ok) break;
                 tc_fence_after();
-                const uint64_t da = sw128_desc(smem_u32(smA + st * A_BYTES));
-                const uint64_t db = sw128_desc(smem_u32(smB + st * B_BYTES));
+                const uint32_t dt = tmem + static_cast<uint32_t>(ab * BN);
+                for (int k = 0; k < nk; ++k, ++s) {
+                    const int sa = s % SA, sb = s % SB;
+                    ok = bar_wait(&sh->full_a[sa], (s / SA) & 1, abort) && bar_wait(&sh->full_b[sb], (s / SB) & 1, abort);
+                    if (!ok) break;
+                    tc_fence_after();
+                    const uint64_t da = sw128_desc(smem_u32(smA + sa * A_BYTES));
+                    const uint64_t db = sw128_desc(smem_u32(smB + sb * B_BYTES));
 #pragma unroll
-                for (int kk = 0; kk < BK / 16; ++kk)   // 32 bytes of K per MMA: +2 in 16-byte units
-                    mma_f16(tmem, da + 2 * kk, db + 2 * kk, (s | kk) != 0);
-                mma_commit(&sh->empty[st]);
+                    for (int kk = 0; kk < BK / 16; ++kk)   // 32 bytes of K per MMA: +2 in 16-byte units
+                        mma_f16(dt, da + 2 * kk, db + 2 * kk, (k | kk) != 0);
+                    mma_commit(&sh->empty_a[sa]);   // each commit arrives once these MMAs are done
+                    mma_commit(&sh->empty_b[sb]);
+                }
+                mma_commit(&sh->acc_full[ab]);
             }
-            mma_commit(&sh->acc_full);   // also after an abort: completes once issued MMAs are done
         }
-    } else {
-        // ---------------- sign expansion, then epilogue ----------------
-        const int q = warp & 3;                 // TMEM lane quarter of this warp
-        const int prow = q * 32 + lane;         // tile row of this thread
-        const int grow = p0 + prow;             // sign row
-        const bool valid = grow < g.P;
-        const uint32_t *srow = g.signs + static_cast<int64_t>(valid ? grow : 0) * g.pitch;
-        // cp.async ring: slot j holds the 4 words (2 K steps) of pair j mod RING
-        const int npairs = (nk + 1) / 2;
-        auto issue = [&](int pr) {
-            if (pr < npairs) {
-                const int k = pr * 2 * BK;      // first column of the pair
-                const int env = k / g.Kp, kk = k - env * g.Kp;
-                cp_async16(&ring[(pr % RING) * BM + prow], srow + kk / 32);
+    } else if (warp < 2 + kExpandWarps) {
+        // ---------------- sign expansion: one tile row per thread ----------------
+        // kExpandGroups groups of four warps take turns by pairs of K steps;
+        // each thread of a group owns one tile row.
+        const int grp = (warp - 2) >> 2;
+        const int prow = ((warp - 2) & 3) * 32 + lane;
+        const int npairs = nk / 2;                 // pairs of K steps (K is a multiple of 128)
+        const int total_pairs = my_tiles * npairs;
+        const int env_words = g.Kp / 32;           // packed words of one envelope block of K
+        const uint32_t swz = static_cast<uint32_t>(prow & 7) << 4;
+        // cursor over this CTA's (tile, pair) sequence, advanced without divisions
+        int cj = 0, cpair = 0, cword = 0, cenv = 0, cgrow = 0;
+        const uint32_t *crow = nullptr;
+        bool cvalid = false;
+        uint32_t cmag = 0u;
+        auto seat_mag = [&]() {
+            if (g.arow_scale) {
+                const uint32_t a = cvalid ? __ldg(g.arow_scale + static_cast<int64_t>(cenv) * g.N + cgrow) : 0u;
+                cmag = a | (a << 16);
+            } else {
+                cmag = cvalid ? 0x3C003C00u : 0u;   // +-1
             }
-            cp_async_commit();
         };
-#pragma unroll
-        for (int pr = 0; pr < RING - 1; ++pr) issue(pr);
-        uint32_t mag_env = 0x3C003C00u;   // +-1
-        int cur_env = -1;
-        for (int s = 0; s < nk; ++s) {
-            const int st = s % STAGES;
-            if ((s & 1) == 0) cp_async_wait<RING - 2>();   // pair s/2 has landed
-            const uint4 w4 = ring[((s >> 1) % RING) * BM + prow];
-            if (s & 1) issue((s >> 1) + RING - 1);        // refill the slot consumed last
-            const int env = (s * BK) / g.Kp;
-            if (env != cur_env) {
-                cur_env = env;
-                if (g.arow_scale) {
-                    const uint32_t a = valid ? __ldg(g.arow_scale + static_cast<int64_t>(env) * g.N + grow) : 0u;
-                    mag_env = a | (a << 16);
+        auto seat_tile = [&]() {
+            const int tile = blockIdx.x + cj * gridDim.x;
+            cgrow = (tile % n_p) * BM + prow;
+            cvalid = cgrow < g.P;
+            crow = g.signs + static_cast<int64_t>(cvalid ? cgrow : 0) * g.pitch;
+            seat_mag();
+        };
+        auto advance = [&]() {
+            if (++cpair == npairs) {
+                cpair = 0;
+                cword = 0;
+                cenv = 0;
+                if (++cj < my_tiles) seat_tile();
+            } else {
+                cword += 4;
+                if (cword == env_words) {
+                    cword = 0;
+                    ++cenv;
+                    seat_mag();
                 }
             }
-            const uint32_t w0 = valid ? ((s & 1) ? w4.z : w4.x) : 0u;
-            const uint32_t w1 = valid ? ((s & 1) ? w4.w : w4.y) : 0u;
-            const uint32_t mag = valid ? mag_env : 0u;
-            if (!bar_wait(&sh->empty[st], ((s / STAGES) & 1) ^ 1, abort)) break;
+        };
+        // this row's four words of the cursor's pair (two K steps) and the
+        // magnitude pattern of its envelope block; then move on to the group's
+        // next pair
+        auto fetch = [&](uint4 &w, uint32_t &mag) {
+            w = cvalid ? __ldg(reinterpret_cast<const uint4 *>(crow + cword)) : make_uint4(0u, 0u, 0u, 0u);
+            mag = cmag;
+#pragma unroll
+            for (int e = 0; e < kExpandGroups; ++e) advance();
+        };
+        if (my_tiles > 0) seat_tile();
+#pragma unroll
+        for (int e = 0; e < kExpandGroups; ++e)
+            if (e < grp) advance();
+        constexpr int D = 4;   // pairs in flight per thread
+        uint4 qw[D];
+        uint32_t qm[D];
+#pragma unroll
+        for (int d = 0; d < D; ++d) {
+            qw[d] = make_uint4(0u, 0u, 0u, 0u);
+            qm[d] = 0u;
+            if (grp + d * kExpandGroups < total_pairs) fetch(qw[d], qm[d]);
+        }
+        bool ok = true;
+        auto write_stage = [&](int st, uint32_t w0, uint32_t w1, uint32_t mag) {
             uint8_t *arow = smA + st * A_BYTES + prow * 128;
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {   // 16-byte chunk j: columns 8j..8j+7
+            for (int j = 0; j < 8; ++j) {   // 16-byte chunk j: columns 8j .. 8j + 7
                 const uint32_t w = j < 4 ? w0 : w1;
                 const int pb = 4 * (j & 3);
                 uint4 v;
-                v.x = valid ? sign_pair(w, pb + 0, mag) : 0u;
-                v.y = valid ? sign_pair(w, pb + 1, mag) : 0u;
-                v.z = valid ? sign_pair(w, pb + 2, mag) : 0u;
-                v.w = valid ? sign_pair(w, pb + 3, mag) : 0u;
-                *reinterpret_cast<uint4 *>(arow + ((j ^ (prow & 7)) << 4)) = v;
+                v.x = sign_pair(w, pb + 0, mag);
+                v.y = sign_pair(w, pb + 1, mag);
+                v.z = sign_pair(w, pb + 2, mag);
+                v.w = sign_pair(w, pb + 3, mag);
+                *reinterpret_cast<uint4 *>(arow + ((static_cast<uint32_t>(j) << 4) ^ swz)) = v;
             }
+        };
+        // both K steps of pair p, one proxy fence for the two stages
+        auto expand_pair = [&](int p, const uint4 &w, uint32_t mag) {
+            const int s0 = 2 * p, s1 = 2 * p + 1;
+            const int st0 = s0 % SA, st1 = s1 % SA;
+            ok = bar_wait(&sh->empty_a[st0], ((s0 / SA) & 1) ^ 1, abort) &&
+                 bar_wait(&sh->empty_a[st1], ((s1 / SA) & 1) ^ 1, abort);
+            ok = __all_sync(0xffffffffu, ok);
+            if (!ok) return;
+            write_stage(st0, w.x, w.y, mag);
+            write_stage(st1, w.z, w.w, mag);
             fence_proxy_async();   // generic-proxy writes -> visible to the tensor core
-            bar_arrive(&sh->full_a[st]);
+            __syncwarp();
+            if (lane == 0) {
+                bar_arrive(&sh->full_a[st0]);
+                bar_arrive(&sh->full_a[st1]);
+            }
+        };
+        for (int base = grp; base < total_pairs && ok; base += D * kExpandGroups) {
+#pragma unroll
+            for (int d = 0; d < D; ++d) {
+                const int p = base + d * kExpandGroups;
+                if (p < total_pairs && ok) {
+                    const uint4 w = qw[d];
+                    const uint32_t mag = qm[d];
+                    if (p + D * kExpandGroups < total_pairs) fetch(qw[d], qm[d]);
+                    expand_pair(p, w, mag);
+                }
+            }
         }
-        cp_async_wait<0>();
-
-        // ---------------- epilogue ----------------
-        if (bar_wait(&sh->acc_full, 0, abort)) {
+    } else {
+        // ---------------- epilogue: one warp per TMEM lane quarter ----------------
+        const int q = warp & 3;
+        for (int j = 0; j < my_tiles; ++j) {
+            const int ab = j & 1;
+            if (!warp_wait(&sh->acc_full[ab], (j >> 1) & 1, abort)) break;
             tc_fence_after();
-            const uint32_t taddr = tmem + (static_cast<uint32_t>(q * 32) << 16);
-            if (g.stage == 1) {
-                // column c = i T + t; v[t, i R + r] = fp16(beta_i[r] h)
-                const int r = grow;
-                for (int cc = 0; cc < BN; cc += 16) {
-                    uint32_t v[16];
-                    tmem_ld16(taddr + cc, v);
-                    if (r < g.R) {
+            const int tile = blockIdx.x + j * gridDim.x;
+            const int p0 = (tile % n_p) * BM, c0 = (tile / n_p) * BN;
+            const int grow = p0 + q * 32 + lane;
+            const uint32_t taddr = tmem + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(ab * BN);
+            for (int cc = 0; cc < BN; cc += 16) {
+                uint32_t v[16];
+                tmem_ld16(taddr + cc, v);
+                if (g.stage == 1) {
+                    // column c = i T + t; v[t, i R + r] = fp16(beta_i[r] h)
+                    if (grow < g.R) {
 #pragma unroll
                         for (int e = 0; e < 16; ++e) {
                             const int c = c0 + cc + e;
                             if (c < g.C) {
                                 const int i = c / g.T, t = c - i * g.T;
-                                const float b = h2f(g.beta[static_cast<int64_t>(i) * g.R + r]);
-                                g.V[static_cast<int64_t>(t) * g.ell * g.R + static_cast<int64_t>(i) * g.R + r] =
+                                const float b = h2f(g.beta[static_cast<int64_t>(i) * g.R + grow]);
+                                g.V[static_cast<int64_t>(t) * g.ell * g.R + static_cast<int64_t>(i) * g.R + grow] =
                                     __float2half_rn(b * __uint_as_float(v[e]));
                             }
                         }
                     }
-                }
-            } else {
-                const int n = grow;
-                for (int cc = 0; cc < BN; cc += 16) {
-                    uint32_t v[16];
-                    tmem_ld16(taddr + cc, v);
-                    if (n < g.N) {
+                } else if (grow < g.N) {
 #pragma unroll
-                        for (int e = 0; e < 16; ++e) {
-                            const int t = c0 + cc + e;
-                            if (t < g.C) {
-                                const int64_t idx = static_cast<int64_t>(t) * g.N + n;
-                                float yv = __uint_as_float(v[e]);
-                                if (g.accumulate) yv += load_act(g.y, g.yd, idx);
-                                store_act(g.y, g.yd, idx, yv);
-                            }
+                    for (int e = 0; e < 16; ++e) {
+                        const int t = c0 + cc + e;
+                        if (t < g.C) {
+                            const int64_t idx = static_cast<int64_t>(t) * g.N + grow;
+                            float yv = __uint_as_float(v[e]);
+                            if (g.accumulate) yv += load_act(g.y, g.yd, idx);
+                            store_act(g.y, g.yd, idx, yv);
                         }
                     }
                 }
             }
+            tc_fence_before();   // the accumulator reads are done before it is handed back
+            __syncwarp();
+            if (lane == 0) bar_arrive(&sh->acc_empty[ab]);
         }
     }
 
@@ -377,11 +466,43 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
     }
 }
 
-// u[(i T + t), m] = fp16(gamma_i[m] x[t, m])
+// u[(i T + t), m] = fp16(gamma_i[m] x[t, m]); eight columns per thread with
+// 16-byte loads and stores when M % 8 == 0 and gamma is 16-byte aligned.
 __global__ void __launch_bounds__(256) scale_cast_kernel(const void *x, dbf_dtype xd, const uint16_t *gamma, int M,
-                                                         int T, int ell, __half *U)
+                                                         int T, int ell, __half *U, int vec8)
 {
     const int64_t total = static_cast<int64_t>(ell) * T * M;
+    if (vec8) {
+        const int64_t total8 = total / 8;
+        const int M8 = M / 8;
+        for (int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; idx < total8;
+             idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+            const int64_t row = idx / M8;
+            const int m8 = static_cast<int>(idx - row * M8);
+            const int i = static_cast<int>(row / T);
+            const int64_t t = row - static_cast<int64_t>(i) * T;
+            const uint4 gw = __ldg(reinterpret_cast<const uint4 *>(gamma + static_cast<int64_t>(i) * M) + m8);
+            float xv[8];
+            if (xd == DBF_BF16) {
+                const uint4 xw = __ldg(reinterpret_cast<const uint4 *>(static_cast<const __nv_bfloat16 *>(x) + t * M) + m8);
+                const __nv_bfloat16 *xb = reinterpret_cast<const __nv_bfloat16 *>(&xw);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) xv[e] = __bfloat162float(xb[e]);
+            } else {
+                const float4 *xf = reinterpret_cast<const float4 *>(static_cast<const float *>(x) + t * M) + 2 * m8;
+                const float4 a = __ldg(xf), b = __ldg(xf + 1);
+                xv[0] = a.x; xv[1] = a.y; xv[2] = a.z; xv[3] = a.w;
+                xv[4] = b.x; xv[5] = b.y; xv[6] = b.z; xv[7] = b.w;
+            }
+            const __half *gh = reinterpret_cast<const __half *>(&gw);
+            uint4 out;
+            __half *oh = reinterpret_cast<__half *>(&out);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) oh[e] = __float2half_rn(__half2float(gh[e]) * xv[e]);
+            reinterpret_cast<uint4 *>(U)[idx] = out;
+        }
+        return;
+    }
     for (int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; idx < total;
          idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
         const int64_t row = idx / M;
@@ -420,7 +541,7 @@ bool make_map(CUtensorMap *map, const void *base, int64_t K, int64_t rows)
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-constexpr size_t kGemmSmem = 1024 + STAGES * (A_BYTES + B_BYTES) + RING * BM * 16 + sizeof(GemmSmem) + 64;
+constexpr size_t kGemmSmem = 1024 + SA * A_BYTES + SB * B_BYTES + sizeof(GemmSmem) + 64;
 
 cudaError_t launch_gemm(const CUtensorMap &map, const GemmArgs &a, cudaStream_t s)
 {
@@ -431,8 +552,14 @@ cudaError_t launch_gemm(const CUtensorMap &map, const GemmArgs &a, cudaStream_t 
         if (e != cudaSuccess) return e;
         configured = true;
     }
-    dim3 grid((a.P + BM - 1) / BM, (a.C + BN - 1) / BN);
-    gemm_kernel<<<grid, kThreads, kGemmSmem, s>>>(map, a);
+    static int sms = 0;
+    if (!sms) {
+        int dev = 0, v = 0;
+        cudaGetDevice(&dev);
+        sms = (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && v > 0) ? v : 148;
+    }
+    const int tiles = ((a.P + BM - 1) / BM) * ((a.C + BN - 1) / BN);
+    gemm_kernel<<<tiles < sms ? tiles : sms, kThreads, kGemmSmem, s>>>(map, a);
     return cudaGetLastError();
 }
 
@@ -446,20 +573,22 @@ bool gemm_shape_ok(const dbf_layer &L)
     return L.M % 128 == 0 && L.R % 128 == 0 && L.M > 0 && L.R > 0 && L.N > 0;
 }
 
-size_t gemm_workspace_bytes(const dbf_layer &L, int64_t T) { return u_bytes(L, T) + v_bytes(L, T); }
+size_t gemm_workspace_bytes(const dbf_layer &L, int64_t T) { return kWsHeaderBytes + u_bytes(L, T) + v_bytes(L, T); }
 
 cudaError_t gemm_forward(const dbf_layer &L, const void *x, dbf_dtype xd, void *y, dbf_dtype yd, int64_t T,
                          int flags, void *ws, cudaStream_t s)
 {
     if (T > (1 << 30) / L.ell) return cudaErrorInvalidValue;
-    __half *U = static_cast<__half *>(ws);
-    __half *V = reinterpret_cast<__half *>(static_cast<char *>(ws) + u_bytes(L, T));
+    char *body = static_cast<char *>(ws) + kWsHeaderBytes;   // the header belongs to the decode path
+    __half *U = reinterpret_cast<__half *>(body);
+    __half *V = reinterpret_cast<__half *>(body + u_bytes(L, T));
     const int Ti = static_cast<int>(T);
     {
         const int64_t total = static_cast<int64_t>(L.ell) * T * L.M;
         int64_t blocks = (total + 255) / 256;
         if (blocks > 148 * 32) blocks = 148 * 32;
-        scale_cast_kernel<<<static_cast<int>(blocks), 256, 0, s>>>(x, xd, L.gamma, L.M, Ti, L.ell, U);
+        const int vec8 = (L.M % 8 == 0) && ((reinterpret_cast<uintptr_t>(L.gamma) & 15u) == 0);
+        scale_cast_kernel<<<static_cast<int>(blocks), 256, 0, s>>>(x, xd, L.gamma, L.M, Ti, L.ell, U, vec8);
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }

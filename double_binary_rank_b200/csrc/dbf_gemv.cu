@@ -77,6 +77,9 @@ struct GemvParams {
     int32_t off_digits, off_colinfo, off_tiles, off_bar, off_ubuf, off_rscale;
     int32_t nb_max;               // row blocks per CTA batch (tiles)
     int32_t pdl_wait;             // launched as a programmatic dependent of the previous kernel
+    // single-launch decode: second slice, its row scales, and the barrier counter
+    int32_t off_s2, off_rscale2, slice_rows2;
+    unsigned *hdr;
 };
 
 // Bytes per digit column: 32 per packed word (one byte per column of K),
@@ -227,7 +230,7 @@ struct Smem {
     int *tiles;          // [nb_max][16][kMaxBcols] int32
     uint32_t *signs;     // [prefetch_rows][pitch]
     float4 *ubuf;        // staging of gamma.x quads when K needs several load rounds
-    uint64_t *bar;       // [0] sign slice, [1] digit image
+    uint64_t *bar;       // [0] sign slice, [1] digit image, [2] second sign slice (single launch)
     int *flag;
 };
 
@@ -749,6 +752,491 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_kernel(const GemvParams P)
     }
 }
 
+// ---- single-launch decode ------------------------------------------------------
+// When every column of the call fits one pass (T ell <= 8) the two stages run
+// in one kernel: each CTA owns a range of stage-1 rows and a range of
+// stage-2 rows, copies both sign slices to shared memory at once, and the
+// exchange of the v image goes through a grid-wide barrier on a counter in
+// the workspace header instead of a kernel boundary.
+//
+// Barrier counter: header word 0 counts arrivals, word 1 is the count at which
+// the current call's barrier started. Every CTA reads word 1 (after the
+// previous kernel in the stream has completed), adds one arrival, waits until
+// G arrivals past that start, and writes start + G back to word 1. Each CTA
+// arrives exactly once, even after a timed-out wait, so the two words are
+// equal again when the kernel ends. They must be equal (zero) when the
+// workspace is first used.
+
+// Digits of one stage-1 column u = gamma_i . x_t (layout and scales as in
+// stage1_column). Two threads per packed word: unit (w, hf) holds columns
+// 32w + 8hf + [0, 8) and 32w + 16 + 8hf + [0, 8), which make up the quads
+// k0 = 32w + 8hf + 2p, p = 0..3. VEC: 16-byte loads (K % 8 == 0 and gamma
+// 16-byte aligned).
+constexpr int kFusedUnits = 2;   // units per thread held in registers
+
+// max |beta| over every envelope and rank into *S.bmax (zeroed and published
+// by the caller): the same value in every CTA. fp16 magnitudes order like
+// their bit patterns, so the maximum is taken on the bits, two at a time.
+__device__ __forceinline__ void beta_absmax(const dbf_layer &L, unsigned *bmax)
+{
+    const int nb = L.R * L.ell;
+    unsigned m2 = 0u;   // two 16-bit magnitudes
+    int done = 0;
+    if ((reinterpret_cast<uintptr_t>(L.beta) & 15u) == 0) {
+        const int nv = nb / 8;
+        const uint4 *bp = reinterpret_cast<const uint4 *>(L.beta);
+        for (int v0 = threadIdx.x; v0 < nv; v0 += 4 * kThreads) {
+            uint4 w[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int idx = v0 + e * kThreads;
+                w[e] = idx < nv ? __ldg(bp + idx) : make_uint4(0u, 0u, 0u, 0u);
+            }
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                m2 = __vmaxu2(m2, w[e].x & 0x7FFF7FFFu);
+                m2 = __vmaxu2(m2, w[e].y & 0x7FFF7FFFu);
+                m2 = __vmaxu2(m2, w[e].z & 0x7FFF7FFFu);
+                m2 = __vmaxu2(m2, w[e].w & 0x7FFF7FFFu);
+            }
+        }
+        done = nv * 8;
+    }
+    for (int base = done + threadIdx.x; base < nb; base += 8 * kThreads) {
+        unsigned h[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            const int idx = base + e * kThreads;
+            h[e] = idx < nb ? (__ldg(L.beta + idx) & 0x7FFFu) : 0u;
+        }
+#pragma unroll
+        for (int e = 0; e < 8; ++e) m2 = __vmaxu2(m2, h[e]);
+    }
+    const unsigned bits = max(m2 & 0xFFFFu, m2 >> 16);
+    const unsigned mf = warp_max(__float_as_uint(__half2float(__ushort_as_half(static_cast<unsigned short>(bits)))));
+    if ((threadIdx.x & 31) == 0) atomicMax(bmax, mf);
+}
+
+// Row scales of a CTA in two steps, so that their load latency overlaps other
+// work: fetch into registers, later store to shared memory.
+__device__ __forceinline__ void fetch_row_scales(const uint16_t *scale, int ld, int ell, int row_lo, int nrows,
+                                                 float (&v)[kScalesPerThread])
+{
+    const int n = nrows * ell;
+#pragma unroll
+    for (int e = 0; e < kScalesPerThread; ++e) {
+        const int idx = threadIdx.x + e * kThreads;
+        const bool ok = idx < n;   // n == 0 when the CTA has no rows
+        const int i = ok ? idx / nrows : 0, r = ok ? idx - (idx / nrows) * nrows : 0;
+        v[e] = ldg_h(scale + (ok ? static_cast<int64_t>(i) * ld + row_lo + r : 0));
+    }
+}
+
+__device__ __forceinline__ void store_row_scales(const float (&v)[kScalesPerThread], int ell, int nrows, float *dst)
+{
+    const int n = nrows * ell;
+#pragma unroll
+    for (int e = 0; e < kScalesPerThread; ++e) {
+        const int idx = threadIdx.x + e * kThreads;
+        if (idx < n) dst[idx] = v[e];
+    }
+}
+
+
+template <bool XBF16, bool VEC>
+__device__ void fused_column(const GemvParams &P, const dbf_layer &L, int64_t t, int i, int lc, char *digits, int cb,
+                             const Smem &S)
+{
+    const int K = L.M;
+    const int pitch = static_cast<int>(pitch_words(K));
+    const int units = 2 * ((pitch + kGroupWords - 1) / kGroupWords * kGroupWords);
+    const int lane = threadIdx.x & 31;
+    const uint16_t *gp = L.gamma + static_cast<int64_t>(i) * K;
+    const int64_t xb = t * K;
+    if (threadIdx.x == 0) {
+        S.col[lc].amax = 0u;
+        S.col[lc].qsum = 0;
+        S.col[lc].qabs = 0;
+    }
+    // ---- loads: every one issued before any use
+    float g[kFusedUnits][16], xv[kFusedUnits][16];
+#pragma unroll
+    for (int e = 0; e < kFusedUnits; ++e) {
+        const int u = threadIdx.x + e * kThreads;
+        const int w = u >> 1, hf = u & 1;
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+            const int k0 = 32 * w + 16 * half + 8 * hf;
+            if (VEC) {
+                const bool in = u < units && k0 < K;   // K % 8 == 0: a chunk is wholly in or out
+                const int kc = in ? k0 : 0;
+                const uint4 gw = __ldg(reinterpret_cast<const uint4 *>(gp + kc));
+                const __half *gh = reinterpret_cast<const __half *>(&gw);
+#pragma unroll
+                for (int c = 0; c < 8; ++c) g[e][8 * half + c] = in ? __half2float(gh[c]) : 0.f;
+                if (XBF16) {
+                    const uint4 xw = __ldg(reinterpret_cast<const uint4 *>(static_cast<const __nv_bfloat16 *>(P.x) + xb + kc));
+                    const __nv_bfloat16 *xh = reinterpret_cast<const __nv_bfloat16 *>(&xw);
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) xv[e][8 * half + c] = __bfloat162float(xh[c]);
+                } else {
+                    const float4 *xf = reinterpret_cast<const float4 *>(static_cast<const float *>(P.x) + xb + kc);
+                    const float4 a = __ldg(xf), b = __ldg(xf + 1);
+                    xv[e][8 * half + 0] = a.x; xv[e][8 * half + 1] = a.y; xv[e][8 * half + 2] = a.z; xv[e][8 * half + 3] = a.w;
+                    xv[e][8 * half + 4] = b.x; xv[e][8 * half + 5] = b.y; xv[e][8 * half + 6] = b.z; xv[e][8 * half + 7] = b.w;
+                }
+            } else {
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    const bool in = u < units && k0 + c < K;
+                    const int kk = in ? k0 + c : 0;
+                    g[e][8 * half + c] = in ? ldg_h(gp + kk) : 0.f;
+                    xv[e][8 * half + c] = ldg_x<XBF16>(P.x, xb + kk);
+                }
+            }
+        }
+    }
+    float m = 0.f;
+#pragma unroll
+    for (int e = 0; e < kFusedUnits; ++e)
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+            xv[e][c] *= g[e][c];   // gamma . x, exact in fp32
+            m = fmaxf(m, fabsf(xv[e][c]));
+        }
+    __syncthreads();   // column info initialised
+    const unsigned mw = warp_max(__float_as_uint(m));
+    if (lane == 0) atomicMax(&S.col[lc].amax, mw);
+    __syncthreads();
+    const int sh = scale_exponent(__uint_as_float(S.col[lc].amax));
+    const bool plain = sh >= -126 && sh <= 126;
+    const float scale = plain ? exp2i(sh) : 0.f;
+    char *plane0 = digits + static_cast<size_t>(kPlanes * lc) * cb;
+    int sq = 0, sa = 0;
+#pragma unroll
+    for (int e = 0; e < kFusedUnits; ++e) {
+        const int u = threadIdx.x + e * kThreads;
+        if (u < units) {
+            const int w = u >> 1, hf = u & 1;
+#pragma unroll
+            for (int p = 0; p < 4; ++p) {
+                // quad k0, k0 + 16, k0 + 1, k0 + 17 with k0 = 32 w + 8 hf + 2 p
+                const int q0 = quantize(xv[e][2 * p], scale, sh, plain);
+                const int q1 = quantize(xv[e][8 + 2 * p], scale, sh, plain);
+                const int q2 = quantize(xv[e][2 * p + 1], scale, sh, plain);
+                const int q3 = quantize(xv[e][8 + 2 * p + 1], scale, sh, plain);
+                sq += q0 + q1 + q2 + q3;
+                sa += abs(q0) + abs(q1) + abs(q2) + abs(q3);
+                store_quad(plane0, cb, digit_offset(32 * w + 8 * hf + 2 * p), q0, q1, q2, q3);
+            }
+        }
+    }
+    const long long sq64 = warp_sum64(sq), sa64 = warp_sum64(sa);
+    if (lane == 0) {
+        atomicAdd(reinterpret_cast<unsigned long long *>(&S.col[lc].qsum), static_cast<unsigned long long>(sq64));
+        atomicAdd(reinterpret_cast<unsigned long long *>(&S.col[lc].qabs), static_cast<unsigned long long>(sa64));
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        S.col[lc].sh = sh;
+        const float bound = __uint_as_float(*S.bmax) * scale_pow2(static_cast<float>(S.col[lc].qabs), -sh) *
+                            (1.0f + 1.0f / 1024.0f);
+        S.col[lc].sh_next = scale_exponent(bound);
+    }
+}
+
+__device__ __forceinline__ unsigned ld_acquire(const unsigned *p)
+{
+    unsigned v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// Grid-wide barrier on the header counter (see above); false on timeout.
+__device__ bool grid_barrier(unsigned *hdr, unsigned start, int32_t *status, int *flag)
+{
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        __threadfence();
+        atomicAdd(hdr, 1u);
+        bool ok = true;
+        const unsigned long long t0 = global_ns();
+        while (ld_acquire(hdr) - start < gridDim.x) {
+            if (global_ns() - t0 > kWaitNs) {
+                ok = false;
+                set_status(status, DBF_ERR_TIMEOUT);
+                break;
+            }
+        }
+        __threadfence();
+        hdr[1] = start + gridDim.x;
+        *flag = ok ? 1 : 0;
+    }
+    __syncthreads();
+    return *flag != 0;
+}
+
+// Rows [rb_begin, rb_end) of one stage: MMA units over the CTA's row blocks in
+// chunks of nb_max, then the stage's epilogue (stage 1: v into the digit
+// image and the CTA's sums of q; stage 2: y).
+template <int STAGE>
+__device__ __forceinline__ void fused_rows(const GemvParams &P, const dbf_layer &L, int rb_begin, int rb_end,
+                                           const uint32_t *Sg, const uint32_t *slice, int K, int rows,
+                                           const char *digits, const char *zero_col, int cb, int ncl,
+                                           const float *rscale, int nb_max, const Smem &S,
+                                           long long (&qpart_local)[kMaxNcl])
+{
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int ell = L.ell;
+    const int pitch = static_cast<int>(pitch_words(K));
+    const bool even = (pitch % 2 == 0) && ((reinterpret_cast<uintptr_t>(Sg) & 7u) == 0);
+    const int ngrp = (pitch + kGroupWords - 1) / kGroupWords;
+    const int bcols = kPlanes * ncl;
+    const int ngroups = (bcols + 7) / 8;
+    const int ntok = ncl / ell;
+    const int row_lo = rb_begin * kRows;
+    const int nrows = min(rb_end * kRows, rows) - row_lo;
+    int *tiles = S.tiles;
+    for (int rbb = rb_begin; rbb < rb_end; rbb += nb_max) {
+        const int nb = min(nb_max, rb_end - rbb);
+        for (int idx = threadIdx.x; idx < nb * kRows * kMaxBcols; idx += blockDim.x) tiles[idx] = 0;
+        __syncthreads();
+        const int units = nb * ngrp;
+        int u = units * warp / kWarps;
+        const int uend = units * (warp + 1) / kWarps;
+        while (u < uend) {
+            const int b = u / ngrp;
+            const int g0 = u - b * ngrp;
+            const int g1 = min(ngrp, g0 + (uend - u));
+            const int row0 = (rbb + b) * kRows;
+            const int g = lane >> 2;
+            const bool va = row0 + g < rows, vb = row0 + g + 8 < rows;
+            if (slice) {
+                const uint32_t *base = slice + static_cast<int64_t>(row0 + g - row_lo) * pitch;
+                warp_run<true>(base, base + 8 * pitch, va, vb, pitch, even, g0, g1, digits, zero_col, ngroups, bcols,
+                               cb, tiles + b * kRows * kMaxBcols);
+            } else {
+                const uint32_t *base = Sg + static_cast<int64_t>(row0 + g) * pitch;
+                warp_run<false>(base, base + 8 * pitch, va, vb, pitch, even, g0, g1, digits, zero_col, ngroups, bcols,
+                                cb, tiles + b * kRows * kMaxBcols);
+            }
+            u += g1 - g0;
+        }
+        __syncthreads();
+        if (STAGE == 1) {
+            // v = beta . h, digitised with the scale every CTA derived alike
+            for (int idx = threadIdx.x; idx < nb * kRows * ncl; idx += blockDim.x) {
+                const int row = idx % (nb * kRows);
+                const int lc = idx / (nb * kRows);
+                const int r = rbb * kRows + row;
+                if (r >= rows) continue;
+                const ColInfo &ci = S.col[lc];
+                const float h =
+                    scale_pow2(__ll2float_rn(ci.qsum - 2 * plane_sum(tiles + row * kMaxBcols, lc)), -ci.sh);
+                const int tok = lc / ell, i = lc - tok * ell;
+                const float v = rscale[i * nrows + (r - row_lo)] * h;
+                const int sh2 = ci.sh_next;
+                const bool plain = sh2 >= -126 && sh2 <= 126;
+                const int q = quantize(v, plain ? exp2i(sh2) : 0.f, sh2, plain);
+                const uint32_t db = digit_bytes(q);
+                char *img = P.img + static_cast<size_t>(tok * P.ell_cap + i) * kPlanes * P.cb2 + digit_offset(r);
+                img[0] = static_cast<char>(db & 255u);
+                img[P.cb2] = static_cast<char>((db >> 8) & 255u);
+                img[2 * P.cb2] = static_cast<char>(db >> 16);
+#pragma unroll
+                for (int c = 0; c < kMaxNcl; ++c)
+                    if (c == lc) qpart_local[c] += q;
+            }
+        } else {
+            for (int idx = threadIdx.x; idx < nb * kRows * ntok; idx += blockDim.x) {
+                const int row = idx % (nb * kRows);
+                const int tok = idx / (nb * kRows);
+                const int n = rbb * kRows + row;
+                if (n >= rows) continue;
+                const int64_t t = tok;
+                float yv = (P.flags & DBF_ACCUMULATE) ? load_act(P.y, P.yd, t * P.N + n) : 0.f;
+                for (int i = 0; i < ell; ++i) {
+                    const int lc = tok * ell + i;
+                    const ColInfo &ci = S.col[lc];
+                    const float z =
+                        scale_pow2(__ll2float_rn(ci.qsum - 2 * plane_sum(tiles + row * kMaxBcols, lc)), -ci.sh);
+                    yv += rscale[i * nrows + (n - row_lo)] * z;
+                }
+                store_act(P.y, P.yd, t * P.N + n, yv);
+            }
+        }
+        __syncthreads();
+    }
+}
+
+template <bool XBF16, bool VEC>
+__global__ void __launch_bounds__(kThreads, 2) gemv_fused_kernel(const GemvParams P)
+{
+    extern __shared__ __align__(128) char smem[];
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    pdl_trigger();
+    const bool early = (P.flags & DBF_WEIGHTS_STATIC) != 0;
+    if (!early) pdl_wait();
+
+    const dbf_layer &L = P.layer;
+    const int ell = L.ell;
+    const int ncl = static_cast<int>(P.T) * ell;
+    const int G = gridDim.x, b = blockIdx.x;
+    const int nrb1 = (L.R + kRows - 1) / kRows, nrb2 = (L.N + kRows - 1) / kRows;
+    const int rb1b = static_cast<int>(static_cast<int64_t>(nrb1) * b / G);
+    const int rb1e = static_cast<int>(static_cast<int64_t>(nrb1) * (b + 1) / G);
+    const int rb2b = static_cast<int>(static_cast<int64_t>(nrb2) * b / G);
+    const int rb2e = static_cast<int>(static_cast<int64_t>(nrb2) * (b + 1) / G);
+    const int pitch1 = static_cast<int>(pitch_words(L.M)), pitch2 = static_cast<int>(pitch_words(L.R));
+    const int cb1 = col_bytes(pitch1), cb2 = P.cb2;
+    const int lo1 = rb1b * kRows, lo2 = rb2b * kRows;
+    const int nrows1 = rb1e > rb1b ? min(rb1e * kRows, L.R) - lo1 : 0;
+    const int nrows2 = rb2e > rb2b ? min(rb2e * kRows, L.N) - lo2 : 0;
+
+    Smem S;
+    S.signs = reinterpret_cast<uint32_t *>(smem);   // stage-1 slice at offset 0
+    uint32_t *slice2 = reinterpret_cast<uint32_t *>(smem + P.off_s2);
+    S.digits = smem + P.off_digits;
+    S.col = reinterpret_cast<ColInfo *>(smem + P.off_colinfo);
+    S.bmax = reinterpret_cast<unsigned *>(S.col + kMaxNcl);
+    S.tiles = reinterpret_cast<int *>(smem + P.off_tiles);
+    S.bar = reinterpret_cast<uint64_t *>(smem + P.off_bar);
+    S.flag = reinterpret_cast<int *>(smem + P.off_bar + 32);
+    float *rs1 = reinterpret_cast<float *>(smem + P.off_rscale);
+    float *rs2 = reinterpret_cast<float *>(smem + P.off_rscale2);
+    const bool use1 = P.prefetch_rows > 0 && nrows1 > 0;
+    const bool use2 = P.slice_rows2 > 0 && nrows2 > 0;
+
+    // ---- both sign slices -> shared memory, in flight from the start
+    if (threadIdx.x == 0) {
+        bar_init(&S.bar[0], 1);
+        bar_init(&S.bar[1], 1);
+        bar_init(&S.bar[2], 1);
+        *S.bmax = 0u;
+        if (use1) {
+            const uint32_t bytes = static_cast<uint32_t>(nrows1) * pitch1 * 4u;
+            bar_expect_tx(&S.bar[0], bytes);
+            bulk_copy(S.signs, L.b2_packed + static_cast<int64_t>(lo1) * pitch1, bytes, &S.bar[0]);
+        }
+        if (use2) {
+            const uint32_t bytes = static_cast<uint32_t>(nrows2) * pitch2 * 4u;
+            bar_expect_tx(&S.bar[2], bytes);
+            bulk_copy(slice2, L.b1_packed + static_cast<int64_t>(lo2) * pitch2, bytes, &S.bar[2]);
+        }
+    }
+    // weights (signs and scales) may be read before the previous kernel ends
+    // only with static weights
+    if (!early) pdl_wait();
+    float sv1[kScalesPerThread], sv2[kScalesPerThread];
+    fetch_row_scales(L.beta, L.R, ell, lo1, nrows1, sv1);
+    fetch_row_scales(L.alpha, L.N, ell, lo2, nrows2, sv2);
+    __syncthreads();   // *S.bmax zeroed
+    beta_absmax(L, S.bmax);
+    if (early) pdl_wait();
+    // the barrier's starting count: stable once the previous kernel has completed
+    const unsigned start = threadIdx.x == 0 ? *reinterpret_cast<volatile unsigned *>(P.hdr + 1) : 0u;
+    store_row_scales(sv1, ell, nrows1, rs1);
+    store_row_scales(sv2, ell, nrows2, rs2);
+    char *zero1 = S.digits + static_cast<size_t>(kPlanes) * ncl * cb1;
+    for (int i = threadIdx.x; i < cb1 / 16; i += blockDim.x) reinterpret_cast<uint4 *>(zero1)[i] = make_uint4(0u, 0u, 0u, 0u);
+
+    // ---- stage 1: digits of gamma . x, then the CTA's rows of v
+    for (int lc = 0; lc < ncl; ++lc) {
+        const int tok = lc / ell, i = lc - tok * ell;
+        fused_column<XBF16, VEC>(P, L, tok, i, lc, S.digits, cb1, S);
+    }
+    __syncthreads();
+    bool ok = true;
+    long long qpart_local[kMaxNcl];
+#pragma unroll
+    for (int c = 0; c < kMaxNcl; ++c) qpart_local[c] = 0;
+    if (nrows1 > 0) {
+        if (use1) ok = wait_flag(S, 0, 0, P.status);
+        if (ok)
+            fused_rows<1>(P, L, rb1b, rb1e, L.b2_packed, use1 ? S.signs : nullptr, L.M, L.R, S.digits, zero1, cb1,
+                          ncl, rs1, P.nb_max, S, qpart_local);
+    }
+    if (rb1e == nrb1 && rb1e > rb1b) {
+        // the owner of the last row block zeroes the image past the rank
+        const int kp2 = cb2 - 32;
+        for (int idx = threadIdx.x; idx < ncl * (kp2 - L.R); idx += blockDim.x) {
+            const int lc = idx / (kp2 - L.R);
+            const int r = L.R + idx % (kp2 - L.R);
+            const int tok = lc / ell, i = lc - tok * ell;
+            char *img = P.img + static_cast<size_t>(tok * P.ell_cap + i) * kPlanes * cb2 + digit_offset(r);
+            img[0] = 0;
+            img[cb2] = 0;
+            img[2 * cb2] = 0;
+        }
+    }
+    {
+        long long *red = reinterpret_cast<long long *>(S.tiles);
+        for (int lc = threadIdx.x; lc < ncl; lc += blockDim.x) red[lc] = 0;
+        __syncthreads();
+        for (int lc = 0; lc < ncl; ++lc) {
+            long long v = 0;
+#pragma unroll
+            for (int c = 0; c < kMaxNcl; ++c)
+                if (c == lc) v = qpart_local[c];
+            v = warp_sum64(v);
+            if (lane == 0) atomicAdd(reinterpret_cast<unsigned long long *>(&red[lc]), static_cast<unsigned long long>(v));
+        }
+        __syncthreads();
+        for (int lc = threadIdx.x; lc < ncl; lc += blockDim.x) {
+            const int tok = lc / ell, i = lc - tok * ell;
+            P.qpart[static_cast<int64_t>(b) * P.T * P.ell_cap + tok * P.ell_cap + i] = red[lc];
+        }
+    }
+
+    // ---- every CTA's image rows and sums are written; stage 2 reads the image
+    // through the async proxy
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+    const bool passed = grid_barrier(P.hdr, start, P.status, S.flag);
+    if (!passed || !ok || nrows2 <= 0) {
+        if (use2) wait_flag(S, 2, 0, P.status);   // no copy left in flight
+        return;
+    }
+
+    // ---- stage 2: the v image, the sums of q, then the CTA's rows of y
+    if (threadIdx.x == 0) {
+        asm volatile("fence.proxy.async.global;" ::: "memory");
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        bar_expect_tx(&S.bar[1], static_cast<uint32_t>(ncl * kPlanes * cb2));
+        for (int lc = 0; lc < ncl; ++lc) {
+            const int tok = lc / ell, i = lc - tok * ell;
+            bulk_copy(S.digits + static_cast<size_t>(kPlanes) * lc * cb2,
+                      P.img + static_cast<size_t>(tok * P.ell_cap + i) * kPlanes * cb2,
+                      static_cast<uint32_t>(kPlanes) * cb2, &S.bar[1]);
+        }
+    }
+    char *zero2 = S.digits + static_cast<size_t>(kPlanes) * ncl * cb2;
+    for (int i = threadIdx.x; i < cb2 / 16; i += blockDim.x) reinterpret_cast<uint4 *>(zero2)[i] = make_uint4(0u, 0u, 0u, 0u);
+    for (int lc = warp; lc < ncl; lc += kWarps) {
+        const int tok = lc / ell, i = lc - tok * ell;
+        const int64_t c = tok * P.ell_cap + i;
+        long long part[kMaxCtas / 32];
+#pragma unroll
+        for (int e = 0; e < kMaxCtas / 32; ++e) {
+            const int k = lane + 32 * e;
+            part[e] = k < G ? __ldcg(P.qpart + static_cast<int64_t>(k) * P.T * P.ell_cap + c) : 0;
+        }
+        long long sq = 0;
+#pragma unroll
+        for (int e = 0; e < kMaxCtas / 32; ++e) sq += part[e];
+        sq = warp_sum64(sq);
+        if (lane == 0) {
+            S.col[lc].qsum = sq;
+            S.col[lc].sh = S.col[lc].sh_next;
+        }
+    }
+    if (!wait_flag(S, 1, 0, P.status)) return;
+    if (use2 && !wait_flag(S, 2, 0, P.status)) return;
+    fused_rows<2>(P, L, rb2b, rb2e, L.b1_packed, use2 ? slice2 : nullptr, L.R, L.N, S.digits, zero2, cb2, ncl, rs2,
+                  P.nb_max, S, qpart_local);
+}
+
 int num_sms()
 {
     static int sms = 0;
@@ -853,6 +1341,97 @@ cudaError_t launch(GemvParams P, int K, int rows_max, int nseg, int ctas, int ma
     return cudaGetLastError();
 }
 
+// Single-launch plan: shared-memory offsets for both slices; false when the
+// call does not fit one pass, one register load round or shared memory.
+bool plan_fused(GemvParams &P, const dbf_layer &L, int G, size_t &smem)
+{
+    const int ncl = static_cast<int>(P.T) * L.ell;
+    if (P.T < 1 || ncl > kMaxNcl) return false;
+    const int pitch1 = static_cast<int>(pitch_words(L.M)), pitch2 = static_cast<int>(pitch_words(L.R));
+    if (2 * ((pitch1 + kGroupWords - 1) / kGroupWords * kGroupWords) > kFusedUnits * kThreads) return false;
+    const int nrb1 = (L.R + kRows - 1) / kRows, nrb2 = (L.N + kRows - 1) / kRows;
+    const int per1 = (nrb1 + G - 1) / G, per2 = (nrb2 + G - 1) / G;
+    if (per1 * kRows * L.ell > kScalesPerThread * kThreads || per2 * kRows * L.ell > kScalesPerThread * kThreads)
+        return false;
+    const int cb1 = col_bytes(pitch1), cb2 = col_bytes(pitch2);
+    const int nb = 2;
+    auto carve = [&](int rows1, int rows2, bool commit) -> size_t {
+        size_t off = align_up(static_cast<size_t>(rows1) * pitch1 * 4, 128);
+        const size_t o_s2 = off;
+        off = align_up(off + static_cast<size_t>(rows2) * pitch2 * 4, 128);
+        const size_t o_dig = off;
+        off += static_cast<size_t>(kPlanes * ncl + 1) * (cb1 > cb2 ? cb1 : cb2);
+        off = align_up(off, 16);
+        const size_t o_col = off;
+        off += static_cast<size_t>(kMaxNcl) * sizeof(ColInfo) + 16;
+        off = align_up(off, 16);
+        const size_t o_tiles = off;
+        off += static_cast<size_t>(nb) * kRows * kMaxBcols * 4;
+        off = align_up(off, 16);
+        const size_t o_bar = off;
+        off += 64;   // three mbarriers + wait flag
+        const size_t o_rs1 = off;
+        off += static_cast<size_t>(per1) * kRows * L.ell * 4;
+        off = align_up(off, 16);
+        const size_t o_rs2 = off;
+        off += static_cast<size_t>(per2) * kRows * L.ell * 4;
+        off = align_up(off, 16);
+        if (commit) {
+            P.off_s2 = static_cast<int>(o_s2);
+            P.off_digits = static_cast<int>(o_dig);
+            P.off_colinfo = static_cast<int>(o_col);
+            P.off_tiles = static_cast<int>(o_tiles);
+            P.off_bar = static_cast<int>(o_bar);
+            P.off_rscale = static_cast<int>(o_rs1);
+            P.off_rscale2 = static_cast<int>(o_rs2);
+            P.prefetch_rows = rows1;
+            P.slice_rows2 = rows2;
+            P.nb_max = nb;
+            P.ncl_pass = ncl;
+            P.pitch_max = pitch1;
+        }
+        return off;
+    };
+    // slices need whole 16-byte rows for the bulk copy
+    int rows1 = pitch1 % 4 == 0 ? per1 * kRows : 0;
+    int rows2 = pitch2 % 4 == 0 ? per2 * kRows : 0;
+    while (carve(rows1, rows2, false) > kSmemCap) {
+        if (rows2 > 0) rows2 = 0;
+        else if (rows1 > 0) rows1 = 0;
+        else return false;
+    }
+    smem = carve(rows1, rows2, true);
+    return true;
+}
+
+template <bool XBF16, bool VEC>
+cudaError_t launch_fused(const GemvParams &P, int G, size_t smem, cudaStream_t s)
+{
+    static size_t configured = 0;
+    if (smem > configured) {
+        cudaError_t e = cudaFuncSetAttribute(gemv_fused_kernel<XBF16, VEC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             static_cast<int>(smem));
+        if (e != cudaSuccess) return e;
+        e = cudaFuncSetAttribute(gemv_fused_kernel<XBF16, VEC>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                 cudaSharedmemCarveoutMaxShared);
+        if (e != cudaSuccess) return e;
+        configured = smem;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(G);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, gemv_fused_kernel<XBF16, VEC>, P);
+    if (e != cudaSuccess) return e;
+    return cudaGetLastError();
+}
+
 struct WsLayout {
     size_t img, qpart, sh2, total;
 };
@@ -869,14 +1448,21 @@ WsLayout ws_layout(int64_t R, int64_t ell, int64_t T)
     return w;
 }
 
+void bind_workspace(GemvParams &P, int max_R, int max_ell, void *ws)
+{
+    const WsLayout w = ws_layout(max_R, max_ell, P.T);
+    char *body = static_cast<char *>(ws) + kWsHeaderBytes;
+    P.hdr = static_cast<unsigned *>(ws);
+    P.img = body + w.img;
+    P.qpart = reinterpret_cast<long long *>(body + w.qpart);
+    P.sh2 = reinterpret_cast<int *>(body + w.sh2);
+    P.cb2 = col_bytes(static_cast<int>(pitch_words(max_R)));
+}
+
 template <bool SEG>
 cudaError_t run_both(GemvParams P, int M, int max_R, int N, int nseg, int budget, int max_ell, void *ws, cudaStream_t s)
 {
-    const WsLayout w = ws_layout(max_R, max_ell, P.T);
-    P.img = static_cast<char *>(ws) + w.img;
-    P.qpart = reinterpret_cast<long long *>(static_cast<char *>(ws) + w.qpart);
-    P.sh2 = reinterpret_cast<int *>(static_cast<char *>(ws) + w.sh2);
-    P.cb2 = col_bytes(static_cast<int>(pitch_words(max_R)));
+    bind_workspace(P, max_R, max_ell, ws);
     // CTAs per segment: the budget, at least enough that a CTA's row scales
     // fit the loader, never more than there are row blocks
     auto ctas_for = [&](int rows) {
@@ -898,7 +1484,7 @@ cudaError_t run_both(GemvParams P, int M, int max_R, int N, int nseg, int budget
 
 }  // namespace
 
-size_t gemv_workspace_bytes(int64_t R, int64_t ell, int64_t T) { return ws_layout(R, ell, T).total; }
+size_t gemv_workspace_bytes(int64_t R, int64_t ell, int64_t T) { return kWsHeaderBytes + ws_layout(R, ell, T).total; }
 
 cudaError_t gemv_forward(const dbf_layer &L, const void *x, dbf_dtype xd, void *y, dbf_dtype yd, int64_t T,
                          int flags, void *ws, cudaStream_t s)
@@ -917,6 +1503,23 @@ cudaError_t gemv_forward(const dbf_layer &L, const void *x, dbf_dtype xd, void *
     P.ell_cap = L.ell;
     P.R_cap = L.R;
     P.T = T;
+    // one launch when the call fits one pass
+    {
+        const int nrb = ((L.R > L.N ? L.R : L.N) + kRows - 1) / kRows;
+        int G = num_sms();
+        if (G > kMaxCtas) G = kMaxCtas;
+        if (G > nrb) G = nrb;
+        GemvParams F = P;
+        size_t smem = 0;
+        if (plan_fused(F, L, G, smem)) {
+            bind_workspace(F, L.R, L.ell, ws);
+            F.stage1_ctas = G;
+            const bool vec = L.M % 8 == 0 && (reinterpret_cast<uintptr_t>(L.gamma) & 15u) == 0;
+            if (xd == DBF_BF16)
+                return vec ? launch_fused<true, true>(F, G, smem, s) : launch_fused<true, false>(F, G, smem, s);
+            return vec ? launch_fused<false, true>(F, G, smem, s) : launch_fused<false, false>(F, G, smem, s);
+        }
+    }
     return run_both<false>(P, L.M, L.R, L.N, 1, num_sms(), L.ell, ws, s);
 }
 

@@ -12,6 +12,11 @@ namespace dbf {
 
 constexpr int kMaxEll = 8;
 
+// Every workspace starts with this many bytes of header that only the
+// single-launch decode kernel uses (its grid barrier counter); they must be
+// zero before the workspace's first use and every call leaves them valid.
+constexpr size_t kWsHeaderBytes = 256;
+
 // ---- packed layout helpers (see "Packed sign layout" in dbf.h) -----------
 __host__ __device__ inline int64_t pitch_words(int64_t k) { return (k + 31) / 32; }
 

@@ -16,10 +16,12 @@
 // should therefore come before any stream capture.
 //
 // All calls on a device share the one array and it keeps whatever the last
-// call left in it. Nothing in it needs to start at zero: every location the
-// decode kernels read is written earlier by the same call. Calls whose work
-// overlaps on the GPU (different streams, or work that runs concurrently)
-// race on the array; callers must order them.
+// call left in it. Only its first bytes, the workspace header that holds the
+// single-launch decode kernel's barrier counter, must start at zero; static
+// device storage is zero-initialised and every call leaves the header valid.
+// Every other location the decode kernels read is written earlier by the same
+// call. Calls whose work overlaps on the GPU (different streams, or work that
+// runs concurrently) race on the array; callers must order them.
 #include "dbf_internal.cuh"
 
 #include <mutex>

@@ -63,12 +63,13 @@ typedef enum { DBF_F32 = 0, DBF_BF16 = 1, DBF_F16 = 2, DBF_I8 = 3 } dbf_dtype;
 
 /* Flags of dbf_forward / dbf_forward_segmented (bitwise or).
  * DBF_ACCUMULATE: y += branch instead of y = branch.
- * DBF_WEIGHTS_STATIC: the caller promises that the packed sign matrices are
- *   not written by the work enqueued just before this call on the stream.
- *   The kernels are launched as programmatic dependents of the preceding
- *   kernel; with this flag they start streaming the sign matrices before
- *   that kernel has finished (activations, scales, segment tables and every
- *   write still wait for it). Without it nothing is read early. */
+ * DBF_WEIGHTS_STATIC: the caller promises that the layer's weights (the
+ *   packed sign matrices and the alpha, beta, gamma scales) are not written
+ *   by the work enqueued just before this call on the stream. The kernels
+ *   are launched as programmatic dependents of the preceding kernel; with
+ *   this flag they start reading weights before that kernel has finished
+ *   (activations, the workspace, segment tables and every write still wait
+ *   for it). Without it nothing is read early. */
 enum { DBF_ACCUMULATE = 1, DBF_WEIGHTS_STATIC = 2 };
 
 /* GEMV: the decode kernel (few tokens, bandwidth bound, any shape).
@@ -126,7 +127,12 @@ size_t dbf_workspace_bytes(const dbf_layer *L, int64_t T, dbf_path path);
  *    dtype.
  * flags: DBF_ACCUMULATE | DBF_WEIGHTS_STATIC (see above); other bits must be 0.
  * ws: device workspace of at least dbf_workspace_bytes(L, T, path) bytes,
- *    256-byte aligned, contents scratch.
+ *    256-byte aligned. Its first 256 bytes are a header (the grid-barrier
+ *    counter of the single-launch decode kernel, which runs when T * ell <= 8):
+ *    they must be zero before the workspace is first used (cudaMemsetAsync
+ *    once after allocating it) and every call leaves them valid for the next;
+ *    the rest is scratch. Calls that share a workspace must be ordered on the
+ *    GPU (one stream, or events).
  * T == 0 is a no-op. Numerics: the GEMV path turns each activation column
  * (gamma.x, then beta.h) into 22-bit fixed point with one power-of-two scale
  * per column and accumulates sign sums exactly in integers (relative error
@@ -181,10 +187,11 @@ dbf_status dbf_forward_segmented(const dbf_layer *adapters_dev, int32_t num_adap
  * The first call on each device looks the array's device address up once
  * (cudaGetSymbolAddress, with that device current); make that first call
  * before any stream capture. Every call on a device shares the array and it
- * keeps the last call's contents; nothing in it needs to start at zero, but
- * calls whose work overlaps on the GPU race on it and must be ordered by the
- * caller. Errors: as dbf_forward, and DBF_ERR_CUDA if the address lookup
- * fails. */
+ * keeps the last call's contents; its workspace header (see dbf_forward)
+ * starts at zero because the array is zero-initialised static storage, and
+ * every call leaves it valid. Calls whose work overlaps on the GPU race on
+ * the array and must be ordered by the caller. Errors: as dbf_forward, and
+ * DBF_ERR_CUDA if the address lookup fails. */
 dbf_status dbf_forward_decode_noalloc(const dbf_layer *L, const void *x, dbf_dtype x_dtype, void *y,
                                       dbf_dtype y_dtype, int64_t T, int flags, void *stream);
 

@@ -1,0 +1,120 @@
+"""The single-launch decode path (T * ell <= 8) against the fp64 oracle.
+
+That path exchanges the rank-R intermediate through a grid-wide barrier
+whose counter lives in the workspace header, so besides plain parity these
+tests check that many calls sharing one workspace (with different grid
+sizes) stay correct, that the header is left consistent (arrival count ==
+starting count) after every call, and the size limits where the library
+switches to the two-launch path.
+"""
+import numpy as np
+import pytest
+import torch
+
+import dbf_synth as S
+import oracle
+from gpu_util import dev_layer, dev_x, host_y, random_layer, rel_err
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def dbf():
+    import double_binary_rank_b200 as m
+    return m
+
+
+def header_words(ws):
+    return ws[:8].view(torch.int32).cpu().tolist()
+
+
+@pytest.mark.parametrize("T,ell", [(8, 1), (4, 2), (1, 8), (2, 3), (9, 1), (3, 3)])
+def test_column_limit(dbf, T, ell):
+    # T * ell <= 8 runs in one launch, above it in two; both must match
+    rng = np.random.default_rng(700 + 10 * T + ell)
+    L = random_layer(rng, 512, 384, 160, ell)
+    x = S.to_bf16_bits(rng.standard_normal((T, 512)))
+    ref = oracle.forward(L, x)
+    got = host_y(dbf.forward(dev_layer(L), dev_x(x), y_dtype=torch.float32))
+    assert rel_err(got, ref) < 1e-4
+
+
+@pytest.mark.parametrize("M", [8192, 8224])
+def test_input_width_limit(dbf, M):
+    # one register round holds up to 8192 inputs; wider inputs take two launches
+    rng = np.random.default_rng(710 + M)
+    L = random_layer(rng, M, 256, 96, 1)
+    x = S.to_bf16_bits(rng.standard_normal((1, M)))
+    ref = oracle.forward(L, x)
+    got = host_y(dbf.forward(dev_layer(L), dev_x(x), y_dtype=torch.float32))
+    assert rel_err(got, ref) < 1e-4
+
+
+def test_fp32_input_unaligned_gamma(dbf):
+    # fp32 activations, and gamma at an odd 2-byte offset (scalar loads)
+    rng = np.random.default_rng(720)
+    L = random_layer(rng, 264, 200, 70, 2)
+    dl = dev_layer(L)
+    g = torch.empty(dl.gamma.numel() + 1, dtype=torch.float16, device="cuda")
+    g[1:] = dl.gamma.reshape(-1)
+    dl2 = dbf.Layer(dl.M, dl.N, dl.R, dl.ell, dl.b1, dl.b2, dl.alpha, dl.beta, g[1:].view(dl.gamma.shape))
+    x = rng.standard_normal((3, 264)).astype(np.float32)
+    ref = oracle.forward(L, x)
+    got = host_y(dbf.forward(dl2, torch.from_numpy(x).cuda(), y_dtype=torch.float32))
+    assert rel_err(got, ref) < 1e-4
+
+
+def test_shared_workspace_many_layers(dbf):
+    # layers of different sizes (so different grid sizes) take turns on one
+    # workspace; each call queued behind the previous one on one stream
+    rng = np.random.default_rng(730)
+    shapes = [(256, 256, 16), (1024, 2048, 512), (4096, 700, 48), (96, 5000, 300)]
+    layers = [random_layer(rng, M, N, R, 1) for M, N, R in shapes]
+    dls = [dev_layer(L) for L in layers]
+    xs = [S.to_bf16_bits(rng.standard_normal((1, M))) for M, _, _ in shapes]
+    refs = [oracle.forward(L, x) for L, x in zip(layers, xs)]
+    need = max(dbf.workspace_bytes(d, 1) for d in dls)
+    ws = dbf.alloc_workspace(need, "cuda")
+    xd = [dev_x(x) for x in xs]
+    outs = []
+    for k in range(40):
+        i = k % len(layers)
+        outs.append((i, dbf.forward(dls[i], xd[i], ws=ws, y_dtype=torch.float32, static_weights=bool(k & 1))))
+    torch.cuda.synchronize()
+    for i, y in outs:
+        assert rel_err(host_y(y), refs[i]) < 1e-4
+    a, b = header_words(ws)
+    assert a == b and a != 0
+
+
+def test_consistent_nonzero_header(dbf):
+    # only equality of the two header words matters, not their value
+    rng = np.random.default_rng(740)
+    L = random_layer(rng, 640, 320, 96, 1)
+    dl = dev_layer(L)
+    x = S.to_bf16_bits(rng.standard_normal((2, 640)))
+    ref = oracle.forward(L, x)
+    ws = dbf.alloc_workspace(dbf.workspace_bytes(dl, 2), "cuda")
+    ws[:8].view(torch.int32).fill_(0x7FFFFFF0)   # wraps past 2^32 during the calls
+    for _ in range(3):
+        got = host_y(dbf.forward(dl, dev_x(x), ws=ws, y_dtype=torch.float32))
+        assert rel_err(got, ref) < 1e-4
+    a, b = header_words(ws)
+    assert a == b
+
+
+def test_dbf_mlp_decode_repeat_bit_identical(dbf):
+    # integer accumulation: the result does not depend on timing or on which
+    # call came before
+    w = S.WORKLOADS["dbf_mlp"]
+    L = S.workload_layers(w)[0]
+    dl = dev_layer(L)
+    x = dev_x(S.make_x(w.seed, 1, w.M, "bf16"))
+    ws = dbf.alloc_workspace(dbf.workspace_bytes(dl, 1), "cuda")
+    ys = [dbf.forward(dl, x, ws=ws, y_dtype=torch.float32, static_weights=True) for _ in range(6)]
+    torch.cuda.synchronize()
+    first = host_y(ys[0])
+    for y in ys[1:]:
+        assert np.array_equal(host_y(y), first)
+    ref = oracle.forward(L, S.make_x(w.seed, 1, w.M, "bf16"))
+    assert rel_err(first, ref) < 1e-4
