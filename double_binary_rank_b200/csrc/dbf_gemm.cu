@@ -179,13 +179,15 @@ __device__ __forceinline__ void mma_commit(uint64_t *bar)
                  : "memory");
 }
 
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&v)[16])
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32])
 {
     asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
-        "%15}, [%16];"
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+        "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
         : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
-          "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
+          "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15]),
+          "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]),
+          "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
         : "r"(taddr));
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
@@ -421,32 +423,52 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
             const int p0 = (tile % n_p) * BM, c0 = (tile / n_p) * BN;
             const int grow = p0 + q * 32 + lane;
             const uint32_t taddr = tmem + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(ab * BN);
-            for (int cc = 0; cc < BN; cc += 16) {
-                uint32_t v[16];
-                tmem_ld16(taddr + cc, v);
+            const bool row_ok = grow < (g.stage == 1 ? g.R : g.N);
+            for (int cc = 0; cc < BN; cc += 32) {
+                uint32_t v[32];
+                tmem_ld32(taddr + cc, v);   // every lane takes part (.sync.aligned)
+                if (!row_ok) continue;
+                const int cb = c0 + cc;
                 if (g.stage == 1) {
-                    // column c = i T + t; v[t, i R + r] = fp16(beta_i[r] h)
-                    if (grow < g.R) {
+                    // column c = i T + t; v[t, i R + r] = fp16(beta_i[r] h); (i, t)
+                    // advance with c, beta reloaded only when i changes
+                    int i = cb / g.T, t = cb - i * g.T;
+                    const int64_t tstride = static_cast<int64_t>(g.ell) * g.R;
+                    float b = i < g.ell ? h2f(g.beta[static_cast<int64_t>(i) * g.R + grow]) : 0.f;
+                    __half *vp = g.V + static_cast<int64_t>(t) * tstride + static_cast<int64_t>(i) * g.R + grow;
 #pragma unroll
-                        for (int e = 0; e < 16; ++e) {
-                            const int c = c0 + cc + e;
-                            if (c < g.C) {
-                                const int i = c / g.T, t = c - i * g.T;
-                                const float b = h2f(g.beta[static_cast<int64_t>(i) * g.R + grow]);
-                                g.V[static_cast<int64_t>(t) * g.ell * g.R + static_cast<int64_t>(i) * g.R + grow] =
-                                    __float2half_rn(b * __uint_as_float(v[e]));
-                            }
+                    for (int e = 0; e < 32; ++e) {
+                        if (cb + e < g.C) *vp = __float2half_rn(b * __uint_as_float(v[e]));
+                        vp += tstride;
+                        if (++t == g.T) {
+                            t = 0;
+                            ++i;
+                            b = i < g.ell ? h2f(g.beta[static_cast<int64_t>(i) * g.R + grow]) : 0.f;
+                            vp = g.V + static_cast<int64_t>(i) * g.R + grow;
                         }
                     }
-                } else if (grow < g.N) {
+                } else {
+                    const int64_t base = static_cast<int64_t>(cb) * g.N + grow;
+                    const int n_ok = g.C - cb;   // tokens of this chunk inside the batch
+                    if (g.yd == DBF_BF16) {
+                        __nv_bfloat16 *yp = static_cast<__nv_bfloat16 *>(g.y) + base;
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) {
-                        const int t = c0 + cc + e;
-                        if (t < g.C) {
-                            const int64_t idx = static_cast<int64_t>(t) * g.N + grow;
-                            float yv = __uint_as_float(v[e]);
-                            if (g.accumulate) yv += load_act(g.y, g.yd, idx);
-                            store_act(g.y, g.yd, idx, yv);
+                        for (int e = 0; e < 32; ++e) {
+                            if (e < n_ok) {
+                                float yv = __uint_as_float(v[e]);
+                                if (g.accumulate) yv += __bfloat162float(yp[static_cast<int64_t>(e) * g.N]);
+                                yp[static_cast<int64_t>(e) * g.N] = __float2bfloat16_rn(yv);
+                            }
+                        }
+                    } else {
+                        float *yp = static_cast<float *>(g.y) + base;
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) {
+                            if (e < n_ok) {
+                                float yv = __uint_as_float(v[e]);
+                                if (g.accumulate) yv += yp[static_cast<int64_t>(e) * g.N];
+                                yp[static_cast<int64_t>(e) * g.N] = yv;
+                            }
                         }
                     }
                 }

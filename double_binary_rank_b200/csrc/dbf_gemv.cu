@@ -46,6 +46,7 @@ constexpr int kWarps = 8;
 constexpr int kThreads = kWarps * 32;
 constexpr int kMaxCtas = 160;      // per segment; sizes the per-CTA partial sums
 constexpr int kSmemCap = 220 * 1024;
+constexpr int kCoResidentSmem = 113 * 1024;   // two CTAs per SM (228 KB, 1 KB reserved per CTA)
 constexpr int kPrefetchCap = 128 * 1024;
 constexpr unsigned long long kWaitNs = 2000000000ull;   // bounded wait: 2 s
 
@@ -774,35 +775,59 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_kernel(const GemvParams P)
 // 16-byte aligned).
 constexpr int kFusedUnits = 2;   // units per thread held in registers
 
-// max |beta| over every envelope and rank into *S.bmax (zeroed and published
-// by the caller): the same value in every CTA. fp16 magnitudes order like
-// their bit patterns, so the maximum is taken on the bits, two at a time.
-__device__ __forceinline__ void beta_absmax(const dbf_layer &L, unsigned *bmax)
+// max |beta| over every envelope and rank (the same value in every CTA). The
+// first 8192 values are loaded by beta_prefetch, 16 bytes per thread and
+// load, so that their latency overlaps other loads; beta_absmax folds them
+// and reads any rest. fp16 magnitudes order like their bit patterns, so the
+// maximum is taken on the bits, two at a time.
+constexpr int kBetaVecs = 4;   // 16-byte beta loads per thread in the first round
+
+__device__ __forceinline__ bool beta_vec_ok(const dbf_layer &L)
+{
+    return (reinterpret_cast<uintptr_t>(L.beta) & 15u) == 0;
+}
+
+__device__ __forceinline__ void beta_prefetch(const dbf_layer &L, uint4 (&bq)[kBetaVecs])
+{
+    const int nv = beta_vec_ok(L) ? L.R * L.ell / 8 : 0;
+    const uint4 *bp = reinterpret_cast<const uint4 *>(L.beta);
+#pragma unroll
+    for (int e = 0; e < kBetaVecs; ++e) {
+        const int idx = threadIdx.x + e * kThreads;
+        bq[e] = idx < nv ? __ldg(bp + idx) : make_uint4(0u, 0u, 0u, 0u);
+    }
+}
+
+// max |beta| of this thread's share, as a float bit pattern
+__device__ __forceinline__ unsigned beta_absmax(const dbf_layer &L, const uint4 (&bq)[kBetaVecs])
 {
     const int nb = L.R * L.ell;
+    const int nv = beta_vec_ok(L) ? nb / 8 : 0;
     unsigned m2 = 0u;   // two 16-bit magnitudes
-    int done = 0;
-    if ((reinterpret_cast<uintptr_t>(L.beta) & 15u) == 0) {
-        const int nv = nb / 8;
-        const uint4 *bp = reinterpret_cast<const uint4 *>(L.beta);
-        for (int v0 = threadIdx.x; v0 < nv; v0 += 4 * kThreads) {
-            uint4 w[4];
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int idx = v0 + e * kThreads;
-                w[e] = idx < nv ? __ldg(bp + idx) : make_uint4(0u, 0u, 0u, 0u);
-            }
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                m2 = __vmaxu2(m2, w[e].x & 0x7FFF7FFFu);
-                m2 = __vmaxu2(m2, w[e].y & 0x7FFF7FFFu);
-                m2 = __vmaxu2(m2, w[e].z & 0x7FFF7FFFu);
-                m2 = __vmaxu2(m2, w[e].w & 0x7FFF7FFFu);
-            }
-        }
-        done = nv * 8;
+    for (int e = 0; e < kBetaVecs; ++e) {
+        m2 = __vmaxu2(m2, bq[e].x & 0x7FFF7FFFu);
+        m2 = __vmaxu2(m2, bq[e].y & 0x7FFF7FFFu);
+        m2 = __vmaxu2(m2, bq[e].z & 0x7FFF7FFFu);
+        m2 = __vmaxu2(m2, bq[e].w & 0x7FFF7FFFu);
     }
-    for (int base = done + threadIdx.x; base < nb; base += 8 * kThreads) {
+    const uint4 *bp = reinterpret_cast<const uint4 *>(L.beta);
+    for (int v0 = threadIdx.x + kBetaVecs * kThreads; v0 < nv; v0 += kBetaVecs * kThreads) {
+        uint4 w[kBetaVecs];
+#pragma unroll
+        for (int e = 0; e < kBetaVecs; ++e) {
+            const int idx = v0 + e * kThreads;
+            w[e] = idx < nv ? __ldg(bp + idx) : make_uint4(0u, 0u, 0u, 0u);
+        }
+#pragma unroll
+        for (int e = 0; e < kBetaVecs; ++e) {
+            m2 = __vmaxu2(m2, w[e].x & 0x7FFF7FFFu);
+            m2 = __vmaxu2(m2, w[e].y & 0x7FFF7FFFu);
+            m2 = __vmaxu2(m2, w[e].z & 0x7FFF7FFFu);
+            m2 = __vmaxu2(m2, w[e].w & 0x7FFF7FFFu);
+        }
+    }
+    for (int base = nv * 8 + threadIdx.x; base < nb; base += 8 * kThreads) {
         unsigned h[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
@@ -813,8 +838,7 @@ __device__ __forceinline__ void beta_absmax(const dbf_layer &L, unsigned *bmax)
         for (int e = 0; e < 8; ++e) m2 = __vmaxu2(m2, h[e]);
     }
     const unsigned bits = max(m2 & 0xFFFFu, m2 >> 16);
-    const unsigned mf = warp_max(__float_as_uint(__half2float(__ushort_as_half(static_cast<unsigned short>(bits)))));
-    if ((threadIdx.x & 31) == 0) atomicMax(bmax, mf);
+    return __float_as_uint(__half2float(__ushort_as_half(static_cast<unsigned short>(bits))));
 }
 
 // Row scales of a CTA in two steps, so that their load latency overlaps other
@@ -845,7 +869,7 @@ __device__ __forceinline__ void store_row_scales(const float (&v)[kScalesPerThre
 
 template <bool XBF16, bool VEC>
 __device__ void fused_column(const GemvParams &P, const dbf_layer &L, int64_t t, int i, int lc, char *digits, int cb,
-                             const Smem &S)
+                             const Smem &S, bool with_beta, const uint4 (&bq)[kBetaVecs])
 {
     const int K = L.M;
     const int pitch = static_cast<int>(pitch_words(K));
@@ -853,12 +877,8 @@ __device__ void fused_column(const GemvParams &P, const dbf_layer &L, int64_t t,
     const int lane = threadIdx.x & 31;
     const uint16_t *gp = L.gamma + static_cast<int64_t>(i) * K;
     const int64_t xb = t * K;
-    if (threadIdx.x == 0) {
-        S.col[lc].amax = 0u;
-        S.col[lc].qsum = 0;
-        S.col[lc].qabs = 0;
-    }
-    // ---- loads: every one issued before any use
+    // ---- loads: every one issued before any use (column info was zeroed and
+    // published by the caller)
     float g[kFusedUnits][16], xv[kFusedUnits][16];
 #pragma unroll
     for (int e = 0; e < kFusedUnits; ++e) {
@@ -904,9 +924,12 @@ __device__ void fused_column(const GemvParams &P, const dbf_layer &L, int64_t t,
             xv[e][c] *= g[e][c];   // gamma . x, exact in fp32
             m = fmaxf(m, fabsf(xv[e][c]));
         }
-    __syncthreads();   // column info initialised
     const unsigned mw = warp_max(__float_as_uint(m));
     if (lane == 0) atomicMax(&S.col[lc].amax, mw);
+    if (with_beta) {
+        const unsigned bw = warp_max(beta_absmax(L, bq));
+        if (lane == 0) atomicMax(S.bmax, bw);
+    }
     __syncthreads();
     const int sh = scale_exponent(__uint_as_float(S.col[lc].amax));
     const bool plain = sh >= -126 && sh <= 126;
@@ -1115,6 +1138,11 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_fused_kernel(const GemvParam
         bar_init(&S.bar[1], 1);
         bar_init(&S.bar[2], 1);
         *S.bmax = 0u;
+        for (int lc = 0; lc < ncl; ++lc) {
+            S.col[lc].amax = 0u;
+            S.col[lc].qsum = 0;
+            S.col[lc].qabs = 0;
+        }
         if (use1) {
             const uint32_t bytes = static_cast<uint32_t>(nrows1) * pitch1 * 4u;
             bar_expect_tx(&S.bar[0], bytes);
@@ -1132,21 +1160,23 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_fused_kernel(const GemvParam
     float sv1[kScalesPerThread], sv2[kScalesPerThread];
     fetch_row_scales(L.beta, L.R, ell, lo1, nrows1, sv1);
     fetch_row_scales(L.alpha, L.N, ell, lo2, nrows2, sv2);
-    __syncthreads();   // *S.bmax zeroed
-    beta_absmax(L, S.bmax);
+    uint4 bq[kBetaVecs];
+    beta_prefetch(L, bq);
     if (early) pdl_wait();
     // the barrier's starting count: stable once the previous kernel has completed
     const unsigned start = threadIdx.x == 0 ? *reinterpret_cast<volatile unsigned *>(P.hdr + 1) : 0u;
-    store_row_scales(sv1, ell, nrows1, rs1);
-    store_row_scales(sv2, ell, nrows2, rs2);
     char *zero1 = S.digits + static_cast<size_t>(kPlanes) * ncl * cb1;
     for (int i = threadIdx.x; i < cb1 / 16; i += blockDim.x) reinterpret_cast<uint4 *>(zero1)[i] = make_uint4(0u, 0u, 0u, 0u);
+    __syncthreads();   // column info and *S.bmax zeroed
 
     // ---- stage 1: digits of gamma . x, then the CTA's rows of v
     for (int lc = 0; lc < ncl; ++lc) {
         const int tok = lc / ell, i = lc - tok * ell;
-        fused_column<XBF16, VEC>(P, L, tok, i, lc, S.digits, cb1, S);
+        fused_column<XBF16, VEC>(P, L, tok, i, lc, S.digits, cb1, S, lc == 0, bq);
     }
+    // the row scales arrived during the digit build
+    store_row_scales(sv1, ell, nrows1, rs1);
+    store_row_scales(sv2, ell, nrows2, rs2);
     __syncthreads();
     bool ok = true;
     long long qpart_local[kMaxNcl];
@@ -1354,7 +1384,9 @@ bool plan_fused(GemvParams &P, const dbf_layer &L, int G, size_t &smem)
     if (per1 * kRows * L.ell > kScalesPerThread * kThreads || per2 * kRows * L.ell > kScalesPerThread * kThreads)
         return false;
     const int cb1 = col_bytes(pitch1), cb2 = col_bytes(pitch2);
-    const int nb = 2;
+    int nb = per1 > per2 ? per1 : per2;   // every row block of a stage in one MMA pass
+    if (nb > 8) nb = 8;
+    const int nb_full = nb;
     auto carve = [&](int rows1, int rows2, bool commit) -> size_t {
         size_t off = align_up(static_cast<size_t>(rows1) * pitch1 * 4, 128);
         const size_t o_s2 = off;
@@ -1400,6 +1432,11 @@ bool plan_fused(GemvParams &P, const dbf_layer &L, int G, size_t &smem)
         else if (rows1 > 0) rows1 = 0;
         else return false;
     }
+    // fewer row blocks per MMA pass when that lets two CTAs share an SM, so
+    // that the next call's CTAs can start their weight copies while this
+    // call finishes
+    while (nb > 2 && carve(rows1, rows2, false) > kCoResidentSmem) --nb;
+    if (carve(rows1, rows2, false) > kCoResidentSmem) nb = nb_full;
     smem = carve(rows1, rows2, true);
     return true;
 }
