@@ -999,12 +999,35 @@ __device__ bool grid_barrier(unsigned *hdr, unsigned start, int32_t *status, int
     return *flag != 0;
 }
 
+// Row stride in shared memory of a sign slice. The MMA units read 8 bytes per
+// lane from rows g = 0..7 at once; a stride of 0 or 16 words modulo 32 puts
+// those rows on the same banks, so such pitches get 4 words of padding (the
+// copy then goes row by row).
+__host__ __device__ inline int slice_stride(int pitch) { return (pitch % 16 == 0) ? pitch + 4 : pitch; }
+
+// Copy rows x pitch packed words into a slice with row stride
+// slice_stride(pitch); called by one whole warp after the barrier's
+// expect_tx. One bulk copy when unpadded, else one per row.
+__device__ __forceinline__ void copy_slice(uint32_t *dst, const uint32_t *src, int rows, int pitch, uint64_t *bar)
+{
+    if (rows <= 0) return;
+    const int lane = threadIdx.x & 31;
+    const int ss = slice_stride(pitch);
+    if (ss == pitch) {
+        if (lane == 0) bulk_copy(dst, src, static_cast<uint32_t>(rows) * pitch * 4u, bar);
+        return;
+    }
+    for (int r = lane; r < rows; r += 32)
+        bulk_g2s(dst + static_cast<int64_t>(r) * ss, src + static_cast<int64_t>(r) * pitch, static_cast<uint32_t>(pitch) * 4u,
+                 bar);
+}
+
 // Rows [rb_begin, rb_end) of one stage: MMA units over the CTA's row blocks in
 // chunks of nb_max, then the stage's epilogue (stage 1: v into the digit
 // image and the CTA's sums of q; stage 2: y).
 template <int STAGE>
 __device__ __forceinline__ void fused_rows(const GemvParams &P, const dbf_layer &L, int rb_begin, int rb_end,
-                                           const uint32_t *Sg, const uint32_t *slice, int K, int rows,
+                                           const uint32_t *Sg, const uint32_t *slice, int sstride, int K, int rows,
                                            const char *digits, const char *zero_col, int cb, int ncl,
                                            const float *rscale, int nb_max, const Smem &S,
                                            long long (&qpart_local)[kMaxNcl])
@@ -1036,8 +1059,8 @@ __device__ __forceinline__ void fused_rows(const GemvParams &P, const dbf_layer 
             const int g = lane >> 2;
             const bool va = row0 + g < rows, vb = row0 + g + 8 < rows;
             if (slice) {
-                const uint32_t *base = slice + static_cast<int64_t>(row0 + g - row_lo) * pitch;
-                warp_run<true>(base, base + 8 * pitch, va, vb, pitch, even, g0, g1, digits, zero_col, ngroups, bcols,
+                const uint32_t *base = slice + static_cast<int64_t>(row0 + g - row_lo) * sstride;
+                warp_run<true>(base, base + 8 * sstride, va, vb, pitch, even, g0, g1, digits, zero_col, ngroups, bcols,
                                cb, tiles + b * kRows * kMaxBcols);
             } else {
                 const uint32_t *base = Sg + static_cast<int64_t>(row0 + g) * pitch;
@@ -1143,16 +1166,13 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_fused_kernel(const GemvParam
             S.col[lc].qsum = 0;
             S.col[lc].qabs = 0;
         }
-        if (use1) {
-            const uint32_t bytes = static_cast<uint32_t>(nrows1) * pitch1 * 4u;
-            bar_expect_tx(&S.bar[0], bytes);
-            bulk_copy(S.signs, L.b2_packed + static_cast<int64_t>(lo1) * pitch1, bytes, &S.bar[0]);
-        }
-        if (use2) {
-            const uint32_t bytes = static_cast<uint32_t>(nrows2) * pitch2 * 4u;
-            bar_expect_tx(&S.bar[2], bytes);
-            bulk_copy(slice2, L.b1_packed + static_cast<int64_t>(lo2) * pitch2, bytes, &S.bar[2]);
-        }
+        if (use1) bar_expect_tx(&S.bar[0], static_cast<uint32_t>(nrows1) * pitch1 * 4u);
+        if (use2) bar_expect_tx(&S.bar[2], static_cast<uint32_t>(nrows2) * pitch2 * 4u);
+    }
+    if (warp == 0) {
+        __syncwarp();
+        copy_slice(S.signs, L.b2_packed + static_cast<int64_t>(lo1) * pitch1, use1 ? nrows1 : 0, pitch1, &S.bar[0]);
+        copy_slice(slice2, L.b1_packed + static_cast<int64_t>(lo2) * pitch2, use2 ? nrows2 : 0, pitch2, &S.bar[2]);
     }
     // weights (signs and scales) may be read before the previous kernel ends
     // only with static weights
@@ -1185,7 +1205,8 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_fused_kernel(const GemvParam
     if (nrows1 > 0) {
         if (use1) ok = wait_flag(S, 0, 0, P.status);
         if (ok)
-            fused_rows<1>(P, L, rb1b, rb1e, L.b2_packed, use1 ? S.signs : nullptr, L.M, L.R, S.digits, zero1, cb1,
+            fused_rows<1>(P, L, rb1b, rb1e, L.b2_packed, use1 ? S.signs : nullptr, slice_stride(pitch1), L.M, L.R,
+                          S.digits, zero1, cb1,
                           ncl, rs1, P.nb_max, S, qpart_local);
     }
     if (rb1e == nrb1 && rb1e > rb1b) {
@@ -1220,25 +1241,33 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_fused_kernel(const GemvParam
         }
     }
 
-    // ---- every CTA's image rows and sums are written; stage 2 reads the image
-    // through the async proxy
-    asm volatile("fence.proxy.async.global;" ::: "memory");
+    // ---- every CTA's image rows and sums are written
     const bool passed = grid_barrier(P.hdr, start, P.status, S.flag);
     if (!passed || !ok || nrows2 <= 0) {
         if (use2) wait_flag(S, 2, 0, P.status);   // no copy left in flight
         return;
     }
 
-    // ---- stage 2: the v image, the sums of q, then the CTA's rows of y
-    if (threadIdx.x == 0) {
-        asm volatile("fence.proxy.async.global;" ::: "memory");
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-        bar_expect_tx(&S.bar[1], static_cast<uint32_t>(ncl * kPlanes * cb2));
-        for (int lc = 0; lc < ncl; ++lc) {
-            const int tok = lc / ell, i = lc - tok * ell;
-            bulk_copy(S.digits + static_cast<size_t>(kPlanes) * lc * cb2,
-                      P.img + static_cast<size_t>(tok * P.ell_cap + i) * kPlanes * cb2,
-                      static_cast<uint32_t>(kPlanes) * cb2, &S.bar[1]);
+    // ---- stage 2: the v image (coherent 16-byte loads: other CTAs wrote it in
+    // this kernel), the sums of q, then the CTA's rows of y
+    {
+        const int n16 = ncl * kPlanes * cb2 / 16;   // the image of column lc is contiguous, columns back to back
+        uint4 *dst = reinterpret_cast<uint4 *>(S.digits);
+        constexpr int kImgLoads = 8;
+        for (int i0 = threadIdx.x; i0 < n16; i0 += kImgLoads * kThreads) {
+            uint4 v[kImgLoads];
+#pragma unroll
+            for (int e = 0; e < kImgLoads; ++e) {
+                const int i = i0 + e * kThreads;
+                const int lc = i / (kPlanes * cb2 / 16), w = i - lc * (kPlanes * cb2 / 16);
+                const int tok = lc / ell, ii = lc - tok * ell;
+                v[e] = i < n16 ? __ldcg(reinterpret_cast<const uint4 *>(P.img + static_cast<size_t>(tok * P.ell_cap + ii) *
+                                                                                      kPlanes * cb2) + w)
+                               : make_uint4(0u, 0u, 0u, 0u);
+            }
+#pragma unroll
+            for (int e = 0; e < kImgLoads; ++e)
+                if (i0 + e * kThreads < n16) dst[i0 + e * kThreads] = v[e];
         }
     }
     char *zero2 = S.digits + static_cast<size_t>(kPlanes) * ncl * cb2;
@@ -1261,9 +1290,10 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_fused_kernel(const GemvParam
             S.col[lc].sh = S.col[lc].sh_next;
         }
     }
-    if (!wait_flag(S, 1, 0, P.status)) return;
-    if (use2 && !wait_flag(S, 2, 0, P.status)) return;
-    fused_rows<2>(P, L, rb2b, rb2e, L.b1_packed, use2 ? slice2 : nullptr, L.R, L.N, S.digits, zero2, cb2, ncl, rs2,
+    if (use2 && !wait_flag(S, 2, 0, P.status)) return;   // also publishes the image and the sums
+    __syncthreads();
+    fused_rows<2>(P, L, rb2b, rb2e, L.b1_packed, use2 ? slice2 : nullptr, slice_stride(pitch2), L.R, L.N, S.digits,
+                  zero2, cb2, ncl, rs2,
                   P.nb_max, S, qpart_local);
 }
 
@@ -1388,9 +1418,9 @@ bool plan_fused(GemvParams &P, const dbf_layer &L, int G, size_t &smem)
     if (nb > 8) nb = 8;
     const int nb_full = nb;
     auto carve = [&](int rows1, int rows2, bool commit) -> size_t {
-        size_t off = align_up(static_cast<size_t>(rows1) * pitch1 * 4, 128);
+        size_t off = align_up(static_cast<size_t>(rows1) * slice_stride(pitch1) * 4, 128);
         const size_t o_s2 = off;
-        off = align_up(off + static_cast<size_t>(rows2) * pitch2 * 4, 128);
+        off = align_up(off + static_cast<size_t>(rows2) * slice_stride(pitch2) * 4, 128);
         const size_t o_dig = off;
         off += static_cast<size_t>(kPlanes * ncl + 1) * (cb1 > cb2 ? cb1 : cb2);
         off = align_up(off, 16);
