@@ -433,7 +433,7 @@ __device__ __forceinline__ uint2 load_pair(const uint32_t *row, int w, int pitch
 // mask accumulators are live. Exact int32 results are added into the shared
 // tile.
 template <bool SMEM>
-__device__ __forceinline__ void warp_run(const uint32_t *pa, const uint32_t *pb, bool va, bool vb, int pitch,
+__device__ __noinline__ void warp_run(const uint32_t *pa, const uint32_t *pb, bool va, bool vb, int pitch,
                                          bool even, int u0, int u1, const char *dig, const char *zero_col,
                                          int ngroups, int bcols, int cb, int *tile)
 {
@@ -846,13 +846,21 @@ __device__ __forceinline__ unsigned beta_absmax(const dbf_layer &L, const uint4 
 __device__ __forceinline__ void fetch_row_scales(const uint16_t *scale, int ld, int ell, int row_lo, int nrows,
                                                  float (&v)[kScalesPerThread])
 {
-    const int n = nrows * ell;
+    const int n = nrows * ell;   // 0 when the CTA has no rows
+    if (ell == 1) {
+#pragma unroll
+        for (int e = 0; e < kScalesPerThread; ++e) {
+            const int idx = threadIdx.x + e * kThreads;
+            v[e] = idx < n ? ldg_h(scale + row_lo + idx) : 0.f;
+        }
+        return;
+    }
 #pragma unroll
     for (int e = 0; e < kScalesPerThread; ++e) {
         const int idx = threadIdx.x + e * kThreads;
-        const bool ok = idx < n;   // n == 0 when the CTA has no rows
+        const bool ok = idx < n;
         const int i = ok ? idx / nrows : 0, r = ok ? idx - (idx / nrows) * nrows : 0;
-        v[e] = ldg_h(scale + (ok ? static_cast<int64_t>(i) * ld + row_lo + r : 0));
+        v[e] = ok ? ldg_h(scale + static_cast<int64_t>(i) * ld + row_lo + r) : 0.f;
     }
 }
 
@@ -1251,7 +1259,9 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_fused_kernel(const GemvParam
     // ---- stage 2: the v image (coherent 16-byte loads: other CTAs wrote it in
     // this kernel), the sums of q, then the CTA's rows of y
     {
-        const int n16 = ncl * kPlanes * cb2 / 16;   // the image of column lc is contiguous, columns back to back
+        // columns lc = tok ell + i are stored back to back (ell_cap == ell here)
+        const int n16 = ncl * kPlanes * cb2 / 16;
+        const uint4 *src = reinterpret_cast<const uint4 *>(P.img);
         uint4 *dst = reinterpret_cast<uint4 *>(S.digits);
         constexpr int kImgLoads = 8;
         for (int i0 = threadIdx.x; i0 < n16; i0 += kImgLoads * kThreads) {
@@ -1259,11 +1269,7 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_fused_kernel(const GemvParam
 #pragma unroll
             for (int e = 0; e < kImgLoads; ++e) {
                 const int i = i0 + e * kThreads;
-                const int lc = i / (kPlanes * cb2 / 16), w = i - lc * (kPlanes * cb2 / 16);
-                const int tok = lc / ell, ii = lc - tok * ell;
-                v[e] = i < n16 ? __ldcg(reinterpret_cast<const uint4 *>(P.img + static_cast<size_t>(tok * P.ell_cap + ii) *
-                                                                                      kPlanes * cb2) + w)
-                               : make_uint4(0u, 0u, 0u, 0u);
+                v[e] = i < n16 ? __ldcg(src + i) : make_uint4(0u, 0u, 0u, 0u);
             }
 #pragma unroll
             for (int e = 0; e < kImgLoads; ++e)
