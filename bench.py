@@ -313,6 +313,28 @@ def main():
     h2d = x_dec_pin.numel() * 2 + x_pre_pin.numel() * 2
     d2h = y_dec_pin.numel() * 2 + y_pre_pin.numel() * 2
 
+    # ---- decode calls back to back (one token through the rotating layer
+    # copies, as through the layers of a model): per-call time when nothing
+    # else runs in between
+    dec_launches = dbf.forward_launches(base, T_DECODE)
+    pre_launches = dbf.forward_launches(base, T_PREFILL)
+    # (captured in a CUDA graph, so that host launch cost is not timed)
+    n_stream = 4 * COPIES
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        for i in range(n_stream):
+            dbf.forward(layers[i % COPIES], x_dec, y=y_dec, ws=ws_dec, static_weights=True, stream=stream)
+    graph.replay()
+    torch.cuda.synchronize(dev)
+    s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        s0.record(stream)
+        graph.replay()
+        s1.record(stream)
+    torch.cuda.synchronize(dev)
+    stream_us = max_over_ranks(1e3 * s0.elapsed_time(s1) / n_stream, dev)
+    del graph
+
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
@@ -330,8 +352,9 @@ def main():
                 "peak_source": f"{pk_kind} bf16 dense (fp16 runs at the same rate)"}
     roof_dec = {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
                 "frac": gbs / pk["hbm_gbs"], "traffic": kernel_traffic("gemv_decode", "double_binary_rank_b200/csrc/dbf_gemv.cu"),
-                "kernel": "decode forward (two GEMV launches), one call", "peak_source": f"{pk_kind} copy bandwidth",
-                "us_per_call": dec_us}
+                "kernel": f"decode forward ({dec_launches} launch: stage 1, grid barrier, stage 2), one call inside the step",
+                "peak_source": f"{pk_kind} copy bandwidth", "us_per_call": dec_us,
+                "stream_us_per_call": stream_us, "stream_frac": b_dec / (stream_us * 1e-6) / 1e9 / pk["hbm_gbs"]}
 
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
@@ -345,7 +368,7 @@ def main():
         "prefill_us_per_call": pre_us,
         "clocks": clk.summary(),
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": args.steps * 5,
+        "gpu_launches": args.steps * (dec_launches + pre_launches),
     }
     if world == 1 and not args.no_cpu_baseline:
         import oracle

@@ -49,6 +49,7 @@ _SIGS = {
     "dbf_unpack_signs": (ctypes.c_int, [_vp, _i64, _i64, _vp, _vp]),
     "dbf_gemm_min_tokens": (_i64, []),
     "dbf_workspace_bytes": (_sz, [_LP, _i64, ctypes.c_int]),
+    "dbf_forward_launches": (_i32, [_LP, _i64, ctypes.c_int]),
     "dbf_forward": (ctypes.c_int, [_LP, _vp, ctypes.c_int, _vp, ctypes.c_int, _i64, ctypes.c_int,
                                    ctypes.c_int, _vp, _sz, _vp]),
     "dbf_segmented_workspace_bytes": (_sz, [_i32, _i32, _i64]),
@@ -164,6 +165,11 @@ class Layer:
 def workspace_bytes(layer: Layer, T: int, path: str = "auto") -> int:
     d = layer.descriptor()
     return int(_lib.dbf_workspace_bytes(ctypes.byref(d), T, _PATHS[path]))
+
+
+def forward_launches(layer: Layer, T: int, path: str = "auto") -> int:
+    d = layer.descriptor()
+    return int(_lib.dbf_forward_launches(ctypes.byref(d), T, _PATHS[path]))
 
 
 def alloc_workspace(nbytes: int, device) -> torch.Tensor:

@@ -77,6 +77,17 @@ size_t dbf_workspace_bytes(const dbf_layer *L, int64_t T, dbf_path path)
     return gemv_workspace_bytes(L->R, L->ell, T);
 }
 
+int32_t dbf_forward_launches(const dbf_layer *L, int64_t T, dbf_path path)
+{
+    if (!L || L->M <= 0 || L->N <= 0 || L->R <= 0 || L->ell < 1 || L->ell > kMaxEll || T < 0)
+        return 0;
+    if (path != DBF_PATH_AUTO && path != DBF_PATH_GEMV && path != DBF_PATH_GEMM) return 0;
+    if (T == 0) return 0;
+    const dbf_path p = resolve(*L, T, path);
+    if (p == DBF_PATH_GEMM) return gemm_shape_ok(*L) ? 3 : 0;
+    return gemv_launches(*L, T);
+}
+
 dbf_status dbf_forward(const dbf_layer *L, const void *x, dbf_dtype x_dtype, void *y,
                        dbf_dtype y_dtype, int64_t T, int flags, dbf_path path, void *ws,
                        size_t ws_bytes, void *stream)

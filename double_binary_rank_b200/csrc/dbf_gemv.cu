@@ -1505,6 +1505,16 @@ cudaError_t launch_fused(const GemvParams &P, int G, size_t smem, cudaStream_t s
     return cudaGetLastError();
 }
 
+// The single-launch plan for this layer and P.T, with its grid size.
+bool fused_plan_for(const dbf_layer &L, GemvParams &F, int &G, size_t &smem)
+{
+    const int nrb = ((L.R > L.N ? L.R : L.N) + kRows - 1) / kRows;
+    G = num_sms();
+    if (G > kMaxCtas) G = kMaxCtas;
+    if (G > nrb) G = nrb;
+    return plan_fused(F, L, G, smem);
+}
+
 struct WsLayout {
     size_t img, qpart, sh2, total;
 };
@@ -1559,6 +1569,15 @@ cudaError_t run_both(GemvParams P, int M, int max_R, int N, int nseg, int budget
 
 size_t gemv_workspace_bytes(int64_t R, int64_t ell, int64_t T) { return kWsHeaderBytes + ws_layout(R, ell, T).total; }
 
+int gemv_launches(const dbf_layer &L, int64_t T)
+{
+    GemvParams F{};
+    F.T = T;
+    int G = 0;
+    size_t smem = 0;
+    return fused_plan_for(L, F, G, smem) ? 1 : 2;
+}
+
 cudaError_t gemv_forward(const dbf_layer &L, const void *x, dbf_dtype xd, void *y, dbf_dtype yd, int64_t T,
                          int flags, void *ws, cudaStream_t s)
 {
@@ -1578,13 +1597,10 @@ cudaError_t gemv_forward(const dbf_layer &L, const void *x, dbf_dtype xd, void *
     P.T = T;
     // one launch when the call fits one pass
     {
-        const int nrb = ((L.R > L.N ? L.R : L.N) + kRows - 1) / kRows;
-        int G = num_sms();
-        if (G > kMaxCtas) G = kMaxCtas;
-        if (G > nrb) G = nrb;
         GemvParams F = P;
+        int G = 0;
         size_t smem = 0;
-        if (plan_fused(F, L, G, smem)) {
+        if (fused_plan_for(L, F, G, smem)) {
             bind_workspace(F, L.R, L.ell, ws);
             F.stage1_ctas = G;
             const bool vec = L.M % 8 == 0 && (reinterpret_cast<uintptr_t>(L.gamma) & 15u) == 0;

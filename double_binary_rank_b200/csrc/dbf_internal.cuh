@@ -28,6 +28,7 @@ cudaError_t launch_unpack(const uint32_t *src, int64_t rows, int64_t k, int8_t *
 
 // decode path
 size_t gemv_workspace_bytes(int64_t R, int64_t ell, int64_t T);
+int gemv_launches(const dbf_layer &L, int64_t T);   // 1 (single launch) or 2
 cudaError_t gemv_forward(const dbf_layer &L, const void *x, dbf_dtype xd, void *y, dbf_dtype yd,
                          int64_t T, int flags, void *ws, cudaStream_t s);
 cudaError_t gemv_forward_segmented(const dbf_layer *adapters, int32_t num_adapters,

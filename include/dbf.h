@@ -120,6 +120,13 @@ int64_t dbf_gemm_min_tokens(void);
  * resolved as dbf_forward resolves it). Returns 0 for invalid input. */
 size_t dbf_workspace_bytes(const dbf_layer *L, int64_t T, dbf_path path);
 
+/* How many kernels one dbf_forward call with this layer, T and path
+ * launches: 3 on the GEMM path (operand pre-pass, stage 1, stage 2); on the
+ * GEMV path 1 when T * ell <= 8 and the call fits one pass (single-launch
+ * kernel with a grid barrier), else 2. 0 for invalid input or T == 0. Host
+ * only; it reads the device's SM count. */
+int32_t dbf_forward_launches(const dbf_layer *L, int64_t T, dbf_path path);
+
 /* The forward of one layer (host-side descriptor L).
  * x: device T x M, DBF_F32 or DBF_BF16, 16-byte aligned.
  * y: device T x N, DBF_F32 or DBF_BF16, 16-byte aligned; read first when

@@ -112,3 +112,22 @@ def test_segmented_rejects_bad_arguments(lib):
     assert f(a, 4, a, a, 3, 32, 1, 64, 64, a, dbf.F32, a, dbf.F32, 8, 0, None, 0, None, None) == dbf.ERR_WORKSPACE
     assert f(a, 4, a + 2, a, 3, 32, 1, 64, 64, a, dbf.F32, a, dbf.F32, 8, 0, a, 1 << 20, None, None) == dbf.ERR_ALIGNMENT
     assert f(a, 4, a, a, 0, 32, 1, 64, 64, a, dbf.F32, a, dbf.F32, 8, 0, None, 0, None, None) == dbf.OK
+
+
+def test_forward_launch_count(lib):
+    # host-side query, no launch: GEMM path = pre-pass + two stages; GEMV path
+    # = one kernel while T * ell <= 8 (and one register round of inputs), else two
+    import double_binary_rank_b200 as dbf
+    by = ctypes.byref
+    L = _layer(M=4096, N=11008, R=5888, ell=1)
+    assert lib.dbf_forward_launches(by(L), 2048, dbf.PATH_AUTO) == 3
+    assert lib.dbf_forward_launches(by(L), 1, dbf.PATH_AUTO) == 1
+    assert lib.dbf_forward_launches(by(L), 8, dbf.PATH_GEMV) == 1
+    assert lib.dbf_forward_launches(by(L), 9, dbf.PATH_GEMV) == 2
+    L2 = _layer(M=256, N=256, R=16, ell=3)
+    assert lib.dbf_forward_launches(by(L2), 2, dbf.PATH_GEMV) == 1
+    assert lib.dbf_forward_launches(by(L2), 3, dbf.PATH_GEMV) == 2
+    L3 = _layer(M=8224, N=256, R=96, ell=1)   # wider than one register round
+    assert lib.dbf_forward_launches(by(L3), 1, dbf.PATH_GEMV) == 2
+    assert lib.dbf_forward_launches(by(L), 0, dbf.PATH_AUTO) == 0
+    assert lib.dbf_forward_launches(None, 1, dbf.PATH_AUTO) == 0
