@@ -1,4 +1,4 @@
-"""fp64 CPU oracle of the double-binary layer forward (test infrastructure).
+"""fp64 CPU oracle of the double-binary layer forward and backward (test infrastructure).
 
 Only the test suite, ``__graft_entry__.smoke()`` and the benchmark's
 CPU-baseline leg may import this package. The CUDA product path neither
@@ -57,6 +57,9 @@ def _load():
     lib.dbf_oracle_forward.argtypes = [i64, i64, i64, i64, vp, vp, vp, vp, vp, vp, i32, vp, i64,
                                        vp, i32, i32, vp, i32]
     lib.dbf_oracle_forward.restype = i32
+    lib.dbf_oracle_backward.argtypes = [i64, i64, i64, i64, vp, vp, vp, vp, vp, vp, i32, vp, i32, i64,
+                                        vp, vp, vp, vp, vp, vp, i32]
+    lib.dbf_oracle_backward.restype = i32
     lib.dbf_oracle_pack.argtypes = [vp, i64, i64, vp]
     lib.dbf_oracle_unpack.argtypes = [vp, i64, i64, vp]
     lib.dbf_oracle_f16_to_f64.argtypes = [ctypes.c_uint16]
@@ -126,6 +129,49 @@ def forward(layer, x: np.ndarray, rows: Optional[Sequence[int]] = None,
     if rc != 0:
         raise ValueError("oracle rejected its arguments")
     return out
+
+
+class Grads:
+    """Backward outputs (float64): dx [T, M], dalpha [ell, N], dbeta [ell, R],
+    dgamma [ell, M], db1 [N, R], db2 [R, M] (None when not requested)."""
+
+    def __init__(self, dx, dalpha, dbeta, dgamma, db1, db2):
+        self.dx, self.dalpha, self.dbeta, self.dgamma, self.db1, self.db2 = dx, dalpha, dbeta, dgamma, db1, db2
+
+
+def backward(layer, x: np.ndarray, dy: np.ndarray, want_signs: bool = False,
+             nthreads: Optional[int] = None) -> Grads:
+    """Gradients of a loss through the forward, given dy = dL/dy (T x N).
+
+    The chain rule through the forward's own steps (LoRDBA page, section 2:
+    the training pipeline differentiates this forward; the straight-through
+    estimator hands the sign-matrix gradients db1, db2 to the latents). x and
+    dy: float32 values or uint16 bf16 bits. Scale gradients and db1, db2 sum
+    over all tokens; dx is per token. db1, db2 only when want_signs.
+    """
+    lib = _load()
+    M, N, R, ell = int(layer.M), int(layer.N), int(layer.R), int(layer.ell)
+    b1 = np.ascontiguousarray(layer.b1, dtype=np.int8)
+    b2 = np.ascontiguousarray(layer.b2, dtype=np.int8)
+    al = np.ascontiguousarray(layer.alpha, dtype=np.uint16).reshape(ell, N)
+    be = np.ascontiguousarray(layer.beta, dtype=np.uint16).reshape(ell, R)
+    ga = np.ascontiguousarray(layer.gamma, dtype=np.uint16).reshape(ell, M)
+    assert b1.shape == (N, R) and b2.shape == (R, M)
+    xa, xk = _act(x)
+    da, dk = _act(dy)
+    T = xa.shape[0]
+    assert xa.shape == (T, M) and da.shape == (T, N)
+    dx = np.zeros((T, M))
+    dal, dbe, dga = np.zeros((ell, N)), np.zeros((ell, R)), np.zeros((ell, M))
+    db1 = np.zeros((N, R)) if want_signs else None
+    db2 = np.zeros((R, M)) if want_signs else None
+    rc = lib.dbf_oracle_backward(M, N, R, ell, _ptr(b1), _ptr(b2), _ptr(al), _ptr(be), _ptr(ga),
+                                 _ptr(xa), xk, _ptr(da), dk, T, _ptr(dx), _ptr(dal), _ptr(dbe), _ptr(dga),
+                                 _ptr(db1) if want_signs else None, _ptr(db2) if want_signs else None,
+                                 int(nthreads or default_threads()))
+    if rc != 0:
+        raise ValueError("oracle rejected its arguments")
+    return Grads(dx, dal, dbe, dga, db1, db2)
 
 
 def forward_segmented(layers, seg_offsets, seg_adapter, x: np.ndarray,

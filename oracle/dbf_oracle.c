@@ -213,3 +213,165 @@ void dbf_oracle_unpack(const uint32_t *w, int64_t rows, int64_t k, int8_t *s)
         for (int64_t c = 0; c < k; ++c)
             s[i * k + c] = ((w[i * pitch + c / 32] >> bit_of((int)(c % 32))) & 1u) ? -1 : 1;
 }
+
+/* ---- the backward ----------------------------------------------------- */
+/*
+ * Gradients of a loss L through the forward above, given dL/dy = dy
+ * (LoRDBA page, section 2, training pipeline: quantisation-aware training
+ * of the factors with a straight-through estimator; the pages give the
+ * forward only, so these are its derivatives, written out by the chain rule
+ * in the forward's own order). Per token t and envelope i, in fp64:
+ *
+ *   u_i = gamma_i . x_t          h_i = B2 u_i        v_i = beta_i . h_i
+ *   z_i = B1 v_i                 y_t = sum_i alpha_i . z_i
+ *   a_i = alpha_i . dy_t         g_i = B1^T a_i      w_i = beta_i . g_i
+ *   e_i = B2^T w_i
+ *
+ *   dalpha_i += dy_t . z_i       dbeta_i += g_i . h_i
+ *   dgamma_i += x_t . e_i        dx_t = sum_i gamma_i . e_i
+ *   dB1 += a_i v_i^T             dB2 += w_i u_i^T
+ *
+ * dB1 and dB2 are the gradients with respect to the sign matrices taken as
+ * real variables: what a straight-through estimator hands to the latents.
+ * Scale-gradient and dB outputs are sums over all tokens (rows); dx is per
+ * row. Any output pointer may be NULL.
+ */
+typedef struct {
+    int64_t M, N, R, ell;
+    const int8_t *b1, *b2;
+    const uint16_t *alpha, *beta, *gamma;
+    const void *x;
+    int x_kind;
+    const void *dy;
+    int dy_kind;
+    int64_t row_begin, row_end;
+    double *dx;                                  /* [T][M] */
+    double *dalpha, *dbeta, *dgamma, *db1, *db2; /* private partial sums of this worker */
+} bwd_job;
+
+static void backward_rows(const bwd_job *J)
+{
+    const int64_t M = J->M, N = J->N, R = J->R;
+    double *u = (double *)malloc(sizeof(double) * (size_t)M);
+    double *h = (double *)malloc(sizeof(double) * (size_t)R);
+    double *v = (double *)malloc(sizeof(double) * (size_t)R);
+    double *z = (double *)malloc(sizeof(double) * (size_t)N);
+    double *a = (double *)malloc(sizeof(double) * (size_t)N);
+    double *g = (double *)malloc(sizeof(double) * (size_t)R);
+    double *w = (double *)malloc(sizeof(double) * (size_t)R);
+    double *e = (double *)malloc(sizeof(double) * (size_t)M);
+    for (int64_t t = J->row_begin; t < J->row_end; ++t) {
+        if (J->dx)
+            for (int64_t m = 0; m < M; ++m) J->dx[t * M + m] = 0.0;
+        for (int64_t i = 0; i < J->ell; ++i) {
+            /* forward quantities of this token and envelope */
+            for (int64_t m = 0; m < M; ++m)
+                u[m] = dbf_oracle_f16_to_f64(J->gamma[i * M + m]) * load_act(J->x, J->x_kind, t * M + m);
+            for (int64_t r = 0; r < R; ++r) {
+                double s = 0.0;
+                for (int64_t m = 0; m < M; ++m) s += (double)J->b2[r * M + m] * u[m];
+                h[r] = s;
+                v[r] = dbf_oracle_f16_to_f64(J->beta[i * R + r]) * s;
+            }
+            for (int64_t n = 0; n < N; ++n) {
+                double s = 0.0;
+                for (int64_t r = 0; r < R; ++r) s += (double)J->b1[n * R + r] * v[r];
+                z[n] = s;
+            }
+            /* backward: alpha, then B1 transposed, beta, B2 transposed, gamma */
+            for (int64_t n = 0; n < N; ++n) {
+                const double d = load_act(J->dy, J->dy_kind, t * N + n);
+                a[n] = dbf_oracle_f16_to_f64(J->alpha[i * N + n]) * d;
+                if (J->dalpha) J->dalpha[i * N + n] += d * z[n];
+            }
+            for (int64_t r = 0; r < R; ++r) {
+                double s = 0.0;
+                for (int64_t n = 0; n < N; ++n) s += (double)J->b1[n * R + r] * a[n];
+                g[r] = s;
+                w[r] = dbf_oracle_f16_to_f64(J->beta[i * R + r]) * s;
+                if (J->dbeta) J->dbeta[i * R + r] += s * h[r];
+            }
+            for (int64_t m = 0; m < M; ++m) {
+                double s = 0.0;
+                for (int64_t r = 0; r < R; ++r) s += (double)J->b2[r * M + m] * w[r];
+                e[m] = s;
+                if (J->dgamma) J->dgamma[i * M + m] += load_act(J->x, J->x_kind, t * M + m) * s;
+                if (J->dx) J->dx[t * M + m] += dbf_oracle_f16_to_f64(J->gamma[i * M + m]) * s;
+            }
+            if (J->db1)
+                for (int64_t n = 0; n < N; ++n)
+                    for (int64_t r = 0; r < R; ++r) J->db1[n * R + r] += a[n] * v[r];
+            if (J->db2)
+                for (int64_t r = 0; r < R; ++r)
+                    for (int64_t m = 0; m < M; ++m) J->db2[r * M + m] += w[r] * u[m];
+        }
+    }
+    free(u); free(h); free(v); free(z); free(a); free(g); free(w); free(e);
+}
+
+static void *backward_worker(void *arg)
+{
+    backward_rows((const bwd_job *)arg);
+    return NULL;
+}
+
+static double *zeros_or_null(int want, int64_t n)
+{
+    return want ? (double *)calloc((size_t)n, sizeof(double)) : NULL;
+}
+
+/* Returns 0 on success, -1 on bad arguments. Rows 0 .. T-1. */
+int dbf_oracle_backward(int64_t M, int64_t N, int64_t R, int64_t ell,
+                        const int8_t *b1, const int8_t *b2,
+                        const uint16_t *alpha, const uint16_t *beta, const uint16_t *gamma,
+                        const void *x, int x_kind, const void *dy, int dy_kind, int64_t T,
+                        double *dx, double *dalpha, double *dbeta, double *dgamma,
+                        double *db1, double *db2, int nthreads)
+{
+    if (M <= 0 || N <= 0 || R <= 0 || ell <= 0 || T < 0 || !b1 || !b2 || !alpha || !beta || !gamma ||
+        !x || !dy)
+        return -1;
+    if (nthreads < 1)
+        nthreads = 1;
+    if (nthreads > T)
+        nthreads = T > 0 ? (int)T : 1;
+    bwd_job *jobs = (bwd_job *)calloc((size_t)nthreads, sizeof(bwd_job));
+    pthread_t *th = (pthread_t *)calloc((size_t)nthreads, sizeof(pthread_t));
+    for (int k = 0; k < nthreads; ++k) {
+        bwd_job *J = &jobs[k];
+        J->M = M; J->N = N; J->R = R; J->ell = ell;
+        J->b1 = b1; J->b2 = b2; J->alpha = alpha; J->beta = beta; J->gamma = gamma;
+        J->x = x; J->x_kind = x_kind; J->dy = dy; J->dy_kind = dy_kind;
+        J->row_begin = T * k / nthreads;
+        J->row_end = T * (k + 1) / nthreads;
+        J->dx = dx;
+        J->dalpha = zeros_or_null(dalpha != NULL, ell * N);
+        J->dbeta = zeros_or_null(dbeta != NULL, ell * R);
+        J->dgamma = zeros_or_null(dgamma != NULL, ell * M);
+        J->db1 = zeros_or_null(db1 != NULL, N * R);
+        J->db2 = zeros_or_null(db2 != NULL, R * M);
+    }
+    for (int k = 1; k < nthreads; ++k)
+        pthread_create(&th[k], NULL, backward_worker, &jobs[k]);
+    backward_rows(&jobs[0]);
+    for (int k = 1; k < nthreads; ++k)
+        pthread_join(th[k], NULL);
+    /* sum the workers' partial sums in worker order */
+    double *outs[5] = {dalpha, dbeta, dgamma, db1, db2};
+    const int64_t lens[5] = {ell * N, ell * R, ell * M, N * R, R * M};
+    for (int o = 0; o < 5; ++o) {
+        if (!outs[o]) continue;
+        for (int64_t q = 0; q < lens[o]; ++q) outs[o][q] = 0.0;
+        for (int k = 0; k < nthreads; ++k) {
+            double *part = o == 0 ? jobs[k].dalpha : o == 1 ? jobs[k].dbeta : o == 2 ? jobs[k].dgamma
+                         : o == 3 ? jobs[k].db1 : jobs[k].db2;
+            for (int64_t q = 0; q < lens[o]; ++q) outs[o][q] += part[q];
+        }
+    }
+    for (int k = 0; k < nthreads; ++k) {
+        free(jobs[k].dalpha); free(jobs[k].dbeta); free(jobs[k].dgamma); free(jobs[k].db1); free(jobs[k].db2);
+    }
+    free(jobs);
+    free(th);
+    return 0;
+}
