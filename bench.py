@@ -335,6 +335,27 @@ def main():
     stream_us = max_over_ranks(1e3 * s0.elapsed_time(s1) / n_stream, dev)
     del graph
 
+    # ---- backward of the prefill batch (gradients through the layer for
+    # training), timed separately: not part of the forward step above
+    dy_h = S.make_x(w.seed + 200, T_PREFILL, w.N, "bf16")
+    dy = to_dev(dy_h)
+    signs_t = dbf.transposed_signs(base, stream=stream)
+    ws_bwd = dbf.alloc_workspace(dbf.backward_workspace_bytes(base, T_PREFILL), dev)
+    with torch.cuda.stream(stream):
+        grads = dbf.backward(base, x_pre, dy, signs_t=signs_t, ws=ws_bwd, stream=stream)
+        for _ in range(2):
+            dbf.backward(base, x_pre, dy, signs_t=signs_t, grads=grads, ws=ws_bwd, stream=stream)
+    torch.cuda.synchronize(dev)
+    n_bwd = 5
+    b0, b1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        b0.record(stream)
+        for _ in range(n_bwd):
+            dbf.backward(base, x_pre, dy, signs_t=signs_t, grads=grads, ws=ws_bwd, stream=stream)
+        b1.record(stream)
+    torch.cuda.synchronize(dev)
+    bwd_us = max_over_ranks(1e3 * b0.elapsed_time(b1) / n_bwd, dev)
+
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
@@ -366,6 +387,9 @@ def main():
         "roofline": roof_pre,
         "roofline_decode": roof_dec,
         "prefill_us_per_call": pre_us,
+        "backward": {"kernel": "gradients dx, dalpha, dbeta, dgamma of the T=2048 prefill batch (two pre-passes + four tcgen05 sign GEMMs), one call",
+                     "us_per_call": bwd_us, "achieved": 2 * f_pre / (bwd_us * 1e-6) / 1e12, "unit": "TFLOP/s",
+                     "peak": pk["bf16_tflops"], "frac": 2 * f_pre / (bwd_us * 1e-6) / 1e12 / pk["bf16_tflops"]},
         "clocks": clk.summary(),
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": args.steps * (dec_launches + pre_launches),

@@ -47,11 +47,15 @@ _SIGS = {
     "dbf_packed_bytes": (_sz, [_i64, _i64]),
     "dbf_pack_signs": (ctypes.c_int, [_vp, ctypes.c_int, _i64, _i64, _vp, _sz, _vp, _vp]),
     "dbf_unpack_signs": (ctypes.c_int, [_vp, _i64, _i64, _vp, _vp]),
+    "dbf_transpose_signs": (ctypes.c_int, [_vp, _i64, _i64, _vp, _sz, _vp]),
     "dbf_gemm_min_tokens": (_i64, []),
     "dbf_workspace_bytes": (_sz, [_LP, _i64, ctypes.c_int]),
     "dbf_forward_launches": (_i32, [_LP, _i64, ctypes.c_int]),
     "dbf_forward": (ctypes.c_int, [_LP, _vp, ctypes.c_int, _vp, ctypes.c_int, _i64, ctypes.c_int,
                                    ctypes.c_int, _vp, _sz, _vp]),
+    "dbf_backward_workspace_bytes": (_sz, [_LP, _i64]),
+    "dbf_backward": (ctypes.c_int, [_LP, _vp, _vp, _vp, ctypes.c_int, _vp, ctypes.c_int, _i64, _vp, _vp, _vp,
+                                    _vp, ctypes.c_int, _vp, _sz, _vp]),
     "dbf_segmented_workspace_bytes": (_sz, [_i32, _i32, _i64]),
     "dbf_forward_segmented": (ctypes.c_int, [_vp, _i32, _vp, _vp, _i32, _i32, _i32, _i32, _i32,
                                              _vp, ctypes.c_int, _vp, ctypes.c_int, _i64,
@@ -128,6 +132,17 @@ def unpack_signs(words: torch.Tensor, rows: int, k: int, out: Optional[torch.Ten
     return out
 
 
+def transpose_signs(words: torch.Tensor, rows: int, k: int, out: Optional[torch.Tensor] = None,
+                    stream=None) -> torch.Tensor:
+    """Packed rows x k -> packed k x rows (dbf_transpose_signs); int32 words
+    [k, ceil(rows/32)]."""
+    if out is None:
+        out = torch.empty((k, (rows + 31) // 32), dtype=torch.int32, device=words.device)
+    _check(_lib.dbf_transpose_signs(_ptr(words), rows, k, _ptr(out), out.numel() * 4, _stream(stream)),
+           "dbf_transpose_signs")
+    return out
+
+
 @dataclass
 class Layer:
     """Device-resident layer: packed signs (int32 words) and fp16 scales.
@@ -200,6 +215,50 @@ def forward(layer: Layer, x: torch.Tensor, y: Optional[torch.Tensor] = None,
                             _flags(accumulate, static_weights), _PATHS[path], _ptr(ws), ws.numel(),
                             _stream(stream)), "dbf_forward")
     return y
+
+
+@dataclass
+class Grads:
+    dx: Optional[torch.Tensor]       # [T, M] fp32
+    dalpha: Optional[torch.Tensor]   # [ell, N] fp32
+    dbeta: Optional[torch.Tensor]    # [ell, R] fp32
+    dgamma: Optional[torch.Tensor]   # [ell, M] fp32
+
+
+def transposed_signs(layer: Layer, stream=None):
+    """(B1^T packed along N, B2^T packed along R) for dbf_backward."""
+    return (transpose_signs(layer.b1, layer.N, layer.R, stream=stream),
+            transpose_signs(layer.b2, layer.R, layer.M, stream=stream))
+
+
+def backward_workspace_bytes(layer: Layer, T: int) -> int:
+    d = layer.descriptor()
+    return int(_lib.dbf_backward_workspace_bytes(ctypes.byref(d), T))
+
+
+def backward(layer: Layer, x: torch.Tensor, dy: torch.Tensor, signs_t=None, grads: Optional[Grads] = None,
+             want=("dx", "dalpha", "dbeta", "dgamma"), accumulate: bool = False,
+             ws: Optional[torch.Tensor] = None, stream=None) -> Grads:
+    """Gradients through the forward given dy = dL/dy (dbf_backward).
+
+    signs_t: (B1^T, B2^T) packed, from transposed_signs(layer) (computed here
+    if None). grads: output tensors to write (or add to, with accumulate)."""
+    T = x.shape[0]
+    dev = x.device
+    if signs_t is None:
+        signs_t = transposed_signs(layer, stream=stream)
+    if grads is None:
+        mk = lambda name, shape: torch.empty(shape, dtype=torch.float32, device=dev) if name in want else None
+        grads = Grads(mk("dx", (T, layer.M)), mk("dalpha", (layer.ell, layer.N)), mk("dbeta", (layer.ell, layer.R)),
+                      mk("dgamma", (layer.ell, layer.M)))
+    d = layer.descriptor()
+    if ws is None:
+        ws = alloc_workspace(backward_workspace_bytes(layer, T), dev)
+    _check(_lib.dbf_backward(ctypes.byref(d), _ptr(signs_t[0]), _ptr(signs_t[1]), _ptr(x), _DT[x.dtype], _ptr(dy),
+                             _DT[dy.dtype], T, _ptr(grads.dx), _ptr(grads.dalpha), _ptr(grads.dbeta),
+                             _ptr(grads.dgamma), ACCUMULATE if accumulate else 0, _ptr(ws), ws.numel(),
+                             _stream(stream)), "dbf_backward")
+    return grads
 
 
 def forward_decode_noalloc(layer: Layer, x: torch.Tensor, y: Optional[torch.Tensor] = None,

@@ -65,6 +65,15 @@ dbf_status dbf_unpack_signs(const uint32_t *src, int64_t rows, int64_t k, int8_t
     return from_cuda(launch_unpack(src, rows, k, dst, static_cast<cudaStream_t>(stream)));
 }
 
+dbf_status dbf_transpose_signs(const uint32_t *src, int64_t rows, int64_t k, uint32_t *dst, size_t dst_bytes,
+                               void *stream)
+{
+    if (!src || !dst || rows <= 0 || k <= 0) return DBF_ERR_INVALID_ARG;
+    if (dst_bytes < dbf_packed_bytes(k, rows)) return DBF_ERR_INVALID_ARG;
+    if (!aligned(src, 4) || !aligned(dst, 4)) return DBF_ERR_ALIGNMENT;
+    return from_cuda(launch_transpose(src, rows, k, dst, static_cast<cudaStream_t>(stream)));
+}
+
 int64_t dbf_gemm_min_tokens(void) { return kGemmMinTokens; }
 
 size_t dbf_workspace_bytes(const dbf_layer *L, int64_t T, dbf_path path)
@@ -109,6 +118,37 @@ dbf_status dbf_forward(const dbf_layer *L, const void *x, dbf_dtype x_dtype, voi
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (p == DBF_PATH_GEMM) return from_cuda(gemm_forward(*L, x, x_dtype, y, y_dtype, T, flags, ws, s));
     return from_cuda(gemv_forward(*L, x, x_dtype, y, y_dtype, T, flags, ws, s));
+}
+
+size_t dbf_backward_workspace_bytes(const dbf_layer *L, int64_t T)
+{
+    if (!L || L->M <= 0 || L->N <= 0 || L->R <= 0 || L->ell < 1 || L->ell > kMaxEll || T < 0)
+        return 0;
+    if (!gemm_backward_shape_ok(*L)) return 0;
+    return gemm_backward_workspace_bytes(*L, T);
+}
+
+dbf_status dbf_backward(const dbf_layer *L, const uint32_t *b1t_packed, const uint32_t *b2t_packed,
+                        const void *x, dbf_dtype x_dtype, const void *dy, dbf_dtype dy_dtype, int64_t T,
+                        float *dx, float *dalpha, float *dbeta, float *dgamma, int flags, void *ws,
+                        size_t ws_bytes, void *stream)
+{
+    dbf_status st = check_layer(L);
+    if (st != DBF_OK) return st;
+    if (T < 0 || !act_dtype_ok(x_dtype) || !act_dtype_ok(dy_dtype)) return DBF_ERR_INVALID_ARG;
+    if (flags & ~DBF_ACCUMULATE) return DBF_ERR_INVALID_ARG;
+    if (!gemm_backward_shape_ok(*L)) return DBF_ERR_UNSUPPORTED;
+    if (T == 0) return DBF_OK;
+    if (!b1t_packed || !b2t_packed || !x || !dy) return DBF_ERR_INVALID_ARG;
+    if (!aligned(b1t_packed, 16) || !aligned(b2t_packed, 16) || !aligned(x, 16) || !aligned(dy, 16) ||
+        (dbeta && !aligned(dbeta, 4)) || (dx && !aligned(dx, 4)) || (dalpha && !aligned(dalpha, 4)) ||
+        (dgamma && !aligned(dgamma, 4)))
+        return DBF_ERR_ALIGNMENT;
+    const size_t need = gemm_backward_workspace_bytes(*L, T);
+    if (!ws || ws_bytes < need) return DBF_ERR_WORKSPACE;
+    if (!aligned(ws, 256)) return DBF_ERR_ALIGNMENT;
+    return from_cuda(gemm_backward(*L, b1t_packed, b2t_packed, x, x_dtype, dy, dy_dtype, T, dx, dalpha, dbeta,
+                                   dgamma, flags, ws, static_cast<cudaStream_t>(stream)));
 }
 
 size_t dbf_segmented_workspace_bytes(int32_t max_R, int32_t max_ell, int64_t T)

@@ -72,6 +72,15 @@ struct GemmArgs {
     int N;
     int accumulate;
     int32_t *status;
+    // backward epilogues (stages 3..6); columns c = i T + t (envelope-major)
+    float *H32;               // stage 3 writes h [C][P]; stage 4 reads it
+    __half *Vout;             // stages 3, 4: fp16(cscale_i[p] acc) [C][P]
+    const uint16_t *cscale;   // stages 3, 4: beta [ell][P]; stage 6: gamma [ell][P]
+    float *red;               // stages 4, 5, 6 (optional): [ell][P] += sum_t acc * W (stage 4: * H32)
+    const void *W;            // stage 5: dy [T][P]; stage 6: x [T][P]
+    dbf_dtype wd;
+    float *dx;                // stage 6 (optional): [T][P] receives sum_i gamma_i[p] acc
+    int dx_mode;              // 0 store, 1 add, 2 atomic add
 };
 
 // ---- small PTX helpers --------------------------------------------------------
@@ -210,6 +219,73 @@ __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volati
     bool ok = true;
     if ((threadIdx.x & 31) == 0) ok = bar_wait(bar, parity, abort);
     return __shfl_sync(0xffffffffu, ok, 0);
+}
+
+__device__ __forceinline__ float load_w(const void *w, dbf_dtype wd, int64_t i)
+{
+    return wd == DBF_BF16 ? __bfloat162float(static_cast<const __nv_bfloat16 *>(w)[i])
+                          : static_cast<const float *>(w)[i];
+}
+
+// Backward epilogue of 32 accumulator columns c = cb .. cb + 31 of tile row
+// p (see GemmArgs): c = i T + t, so (i, t) advance with c. Every operand the
+// chunk reads (H32 or W) is loaded first, all 32 loads in flight together;
+// then the per-(i, p) sums over tokens are formed and flushed with one
+// atomic add when i changes and at the end of the chunk.
+__device__ __forceinline__ void backward_chunk(const GemmArgs &g, const uint32_t (&v)[32], int cb, int p)
+{
+    const int i0 = cb / g.T, t0 = cb - i0 * g.T;
+    float w[32];
+    {
+        int t = t0;
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+            const bool ok = cb + e < g.C;
+            if (g.stage == 4) {
+                w[e] = g.H32[ok ? static_cast<int64_t>(cb + e) * g.P + p : 0];
+            } else if (g.stage >= 5 && g.red) {
+                w[e] = load_w(g.W, g.wd, ok ? static_cast<int64_t>(t) * g.P + p : 0);
+            } else {
+                w[e] = 0.f;
+            }
+            if (++t == g.T) t = 0;
+        }
+    }
+    int i = i0, t = t0;
+    float cs = (g.cscale && i < g.ell) ? h2f(g.cscale[static_cast<int64_t>(i) * g.P + p]) : 0.f;
+    float part = 0.f;
+#pragma unroll
+    for (int e = 0; e < 32; ++e) {
+        const int c = cb + e;
+        if (c < g.C) {
+            const float a = __uint_as_float(v[e]);
+            const int64_t ic = static_cast<int64_t>(c) * g.P + p;
+            if (g.stage == 3) {
+                g.H32[ic] = a;
+                g.Vout[ic] = __float2half_rn(cs * a);
+            } else if (g.stage == 4) {
+                part += a * w[e];
+                g.Vout[ic] = __float2half_rn(cs * a);
+            } else {
+                part += a * w[e];
+                if (g.stage == 6 && g.dx) {
+                    const int64_t it = static_cast<int64_t>(t) * g.P + p;
+                    const float d = cs * a;
+                    if (g.dx_mode == 0) g.dx[it] = d;
+                    else if (g.dx_mode == 1) g.dx[it] += d;
+                    else atomicAdd(g.dx + it, d);
+                }
+            }
+        }
+        if (++t == g.T) {
+            if (g.red && i < g.ell) atomicAdd(g.red + static_cast<int64_t>(i) * g.P + p, part);
+            part = 0.f;
+            t = 0;
+            ++i;
+            cs = (g.cscale && i < g.ell) ? h2f(g.cscale[static_cast<int64_t>(i) * g.P + p]) : 0.f;
+        }
+    }
+    if (g.red && i < g.ell && part != 0.f) atomicAdd(g.red + static_cast<int64_t>(i) * g.P + p, part);
 }
 
 // Persistent: CTA b takes tiles b, b + gridDim.x, ... (token-tile major, so
@@ -423,7 +499,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
             const int p0 = (tile % n_p) * BM, c0 = (tile / n_p) * BN;
             const int grow = p0 + q * 32 + lane;
             const uint32_t taddr = tmem + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(ab * BN);
-            const bool row_ok = grow < (g.stage == 1 ? g.R : g.N);
+            const bool row_ok = grow < g.P;
             for (int cc = 0; cc < BN; cc += 32) {
                 uint32_t v[32];
                 tmem_ld32(taddr + cc, v);   // every lane takes part (.sync.aligned)
@@ -447,29 +523,29 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
                             vp = g.V + static_cast<int64_t>(i) * g.R + grow;
                         }
                     }
+                } else if (g.stage >= 3) {
+                    backward_chunk(g, v, cb, grow);
                 } else {
                     const int64_t base = static_cast<int64_t>(cb) * g.N + grow;
                     const int n_ok = g.C - cb;   // tokens of this chunk inside the batch
+                    // with accumulation every y_in value of the chunk is loaded first
+                    float yin[32];
                     if (g.yd == DBF_BF16) {
                         __nv_bfloat16 *yp = static_cast<__nv_bfloat16 *>(g.y) + base;
 #pragma unroll
-                        for (int e = 0; e < 32; ++e) {
-                            if (e < n_ok) {
-                                float yv = __uint_as_float(v[e]);
-                                if (g.accumulate) yv += __bfloat162float(yp[static_cast<int64_t>(e) * g.N]);
-                                yp[static_cast<int64_t>(e) * g.N] = __float2bfloat16_rn(yv);
-                            }
-                        }
+                        for (int e = 0; e < 32; ++e)
+                            yin[e] = g.accumulate ? __bfloat162float(yp[static_cast<int64_t>(e < n_ok ? e : 0) * g.N]) : 0.f;
+#pragma unroll
+                        for (int e = 0; e < 32; ++e)
+                            if (e < n_ok) yp[static_cast<int64_t>(e) * g.N] = __float2bfloat16_rn(__uint_as_float(v[e]) + yin[e]);
                     } else {
                         float *yp = static_cast<float *>(g.y) + base;
 #pragma unroll
-                        for (int e = 0; e < 32; ++e) {
-                            if (e < n_ok) {
-                                float yv = __uint_as_float(v[e]);
-                                if (g.accumulate) yv += yp[static_cast<int64_t>(e) * g.N];
-                                yp[static_cast<int64_t>(e) * g.N] = yv;
-                            }
-                        }
+                        for (int e = 0; e < 32; ++e)
+                            yin[e] = g.accumulate ? yp[static_cast<int64_t>(e < n_ok ? e : 0) * g.N] : 0.f;
+#pragma unroll
+                        for (int e = 0; e < 32; ++e)
+                            if (e < n_ok) yp[static_cast<int64_t>(e) * g.N] = __uint_as_float(v[e]) + yin[e];
                     }
                 }
             }
@@ -651,6 +727,133 @@ cudaError_t gemm_forward(const dbf_layer &L, const void *x, dbf_dtype xd, void *
     a2.N = L.N;
     a2.accumulate = (flags & DBF_ACCUMULATE) ? 1 : 0;
     return launch_gemm(mv, a2, s);
+}
+
+}  // namespace dbf
+
+// ---- backward (tcgen05, four sign GEMMs) ---------------------------------------
+namespace dbf {
+namespace {
+
+cudaError_t scale_cast(const void *x, dbf_dtype xd, const uint16_t *scale, int K, int64_t T, int ell, __half *out,
+                       cudaStream_t s)
+{
+    const int64_t total = static_cast<int64_t>(ell) * T * K;
+    int64_t blocks = (total + 255) / 256;
+    if (blocks > 148 * 32) blocks = 148 * 32;
+    const int vec8 = (K % 8 == 0) && ((reinterpret_cast<uintptr_t>(scale) & 15u) == 0);
+    scale_cast_kernel<<<static_cast<int>(blocks), 256, 0, s>>>(x, xd, scale, K, static_cast<int>(T), ell, out, vec8);
+    return cudaGetLastError();
+}
+
+struct BwdLayout {
+    size_t u, a, h32, vh, vg, total;   // offsets after the header
+};
+
+BwdLayout bwd_layout(const dbf_layer &L, int64_t T)
+{
+    const int64_t C = static_cast<int64_t>(L.ell) * T;
+    BwdLayout b;
+    b.u = 0;
+    b.a = b.u + align_up(static_cast<size_t>(C) * L.M * 2, 256);
+    b.h32 = b.a + align_up(static_cast<size_t>(C) * L.N * 2, 256);
+    b.vh = b.h32 + align_up(static_cast<size_t>(C) * L.R * 4, 256);
+    b.vg = b.vh + align_up(static_cast<size_t>(C) * L.R * 2, 256);
+    b.total = b.vg + align_up(static_cast<size_t>(C) * L.R * 2, 256);
+    return b;
+}
+
+GemmArgs sign_gemm_args(const uint32_t *signs, int P, int K, int C, int T, int ell, int stage)
+{
+    GemmArgs a = {};
+    a.signs = signs;
+    a.pitch = static_cast<int>(pitch_words(K));
+    a.P = P;
+    a.Kp = K;
+    a.Ktot = K;
+    a.C = C;
+    a.T = T;
+    a.ell = ell;
+    a.stage = stage;
+    return a;
+}
+
+}  // namespace
+
+bool gemm_backward_shape_ok(const dbf_layer &L)
+{
+    return L.M % 128 == 0 && L.N % 128 == 0 && L.R % 128 == 0 && L.M > 0 && L.N > 0 && L.R > 0;
+}
+
+size_t gemm_backward_workspace_bytes(const dbf_layer &L, int64_t T) { return kWsHeaderBytes + bwd_layout(L, T).total; }
+
+// Gradients through the forward (see dbf.h, dbf_backward), as four sign
+// GEMMs whose epilogues do the per-channel scalings and the reductions over
+// tokens. Columns of every GEMM are c = i T + t (envelope-major).
+//   G3: h_i = B2 u_i,      u_i = fp16(gamma_i . x)    -> H32 = h, Vh = fp16(beta_i . h)
+//   G4: g_i = B1^T a_i,    a_i = fp16(alpha_i . dy)   -> dbeta_i += sum_t g h, Vg = fp16(beta_i . g)
+//   G5: z_i = B1 Vh_i                                 -> dalpha_i += sum_t z dy
+//   G6: e_i = B2^T Vg_i                               -> dgamma_i += sum_t e x, dx = sum_i gamma_i . e
+cudaError_t gemm_backward(const dbf_layer &L, const uint32_t *b1t, const uint32_t *b2t, const void *x, dbf_dtype xd,
+                          const void *dy, dbf_dtype dyd, int64_t T, float *dx, float *dalpha, float *dbeta,
+                          float *dgamma, int flags, void *ws, cudaStream_t s)
+{
+    if (T > (1 << 30) / L.ell) return cudaErrorInvalidValue;
+    const bool acc = (flags & DBF_ACCUMULATE) != 0;
+    const int ell = L.ell, Ti = static_cast<int>(T), C = ell * Ti;
+    const BwdLayout b = bwd_layout(L, T);
+    char *body = static_cast<char *>(ws) + kWsHeaderBytes;
+    __half *U = reinterpret_cast<__half *>(body + b.u);
+    __half *A = reinterpret_cast<__half *>(body + b.a);
+    float *H32 = reinterpret_cast<float *>(body + b.h32);
+    __half *Vh = reinterpret_cast<__half *>(body + b.vh);
+    __half *Vg = reinterpret_cast<__half *>(body + b.vg);
+    cudaError_t e;
+    if (!acc) {
+        if (dalpha && (e = cudaMemsetAsync(dalpha, 0, sizeof(float) * ell * L.N, s)) != cudaSuccess) return e;
+        if (dbeta && (e = cudaMemsetAsync(dbeta, 0, sizeof(float) * ell * L.R, s)) != cudaSuccess) return e;
+        if (dgamma && (e = cudaMemsetAsync(dgamma, 0, sizeof(float) * ell * L.M, s)) != cudaSuccess) return e;
+        if (dx && ell > 1 && (e = cudaMemsetAsync(dx, 0, sizeof(float) * T * L.M, s)) != cudaSuccess) return e;
+    }
+    if ((e = scale_cast(x, xd, L.gamma, L.M, T, ell, U, s)) != cudaSuccess) return e;
+    if ((e = scale_cast(dy, dyd, L.alpha, L.N, T, ell, A, s)) != cudaSuccess) return e;
+    CUtensorMap mu, ma, mvh, mvg;
+    if (!make_map(&mu, U, L.M, C) || !make_map(&ma, A, L.N, C) || !make_map(&mvh, Vh, L.R, C) ||
+        !make_map(&mvg, Vg, L.R, C))
+        return cudaErrorInvalidValue;
+    // G3
+    GemmArgs g3 = sign_gemm_args(L.b2_packed, L.R, L.M, C, Ti, ell, 3);
+    g3.H32 = H32;
+    g3.Vout = Vh;
+    g3.cscale = L.beta;
+    if ((e = launch_gemm(mu, g3, s)) != cudaSuccess) return e;
+    // G4
+    GemmArgs g4 = sign_gemm_args(b1t, L.R, L.N, C, Ti, ell, 4);
+    g4.H32 = H32;
+    g4.Vout = Vg;
+    g4.cscale = L.beta;
+    g4.red = dbeta;
+    if ((e = launch_gemm(ma, g4, s)) != cudaSuccess) return e;
+    // G5
+    if (dalpha) {
+        GemmArgs g5 = sign_gemm_args(L.b1_packed, L.N, L.R, C, Ti, ell, 5);
+        g5.red = dalpha;
+        g5.W = dy;
+        g5.wd = dyd;
+        if ((e = launch_gemm(mvh, g5, s)) != cudaSuccess) return e;
+    }
+    // G6
+    if (dx || dgamma) {
+        GemmArgs g6 = sign_gemm_args(b2t, L.M, L.R, C, Ti, ell, 6);
+        g6.red = dgamma;
+        g6.W = x;
+        g6.wd = xd;
+        g6.cscale = L.gamma;
+        g6.dx = dx;
+        g6.dx_mode = ell > 1 ? 2 : (acc ? 1 : 0);
+        if ((e = launch_gemm(mvg, g6, s)) != cudaSuccess) return e;
+    }
+    return cudaSuccess;
 }
 
 }  // namespace dbf

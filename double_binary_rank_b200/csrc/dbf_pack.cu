@@ -84,6 +84,38 @@ __global__ void __launch_bounds__(256) unpack_kernel(const uint32_t *__restrict_
     }
 }
 
+// Transpose of a packed sign matrix: src is rows x k (packed along k), dst is
+// k x rows (packed along rows). A warp takes one 32 x 32 block: lane L loads
+// the src word of row r0 + col(L), where col(L) is the in-word column that
+// bit L of a packed word holds; then for each of the block's 32 columns c one
+// ballot of "bit of column c is set" is already the dst word of row 32w + c
+// (its bit L is old row r0 + col(L)). Rows past 'rows' load as zero, which
+// keeps the dst padding bits zero.
+__global__ void __launch_bounds__(256) transpose_kernel(const uint32_t *__restrict__ src, int64_t rows,
+                                                        int64_t k, uint32_t *__restrict__ dst)
+{
+    const int lane = threadIdx.x & 31;
+    const int64_t sp = pitch_words(k), dp = pitch_words(rows);
+    const int64_t nblk = dp * sp;   // (row block, word column) pairs
+    const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+    const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+    const int col = lane < 16 ? 2 * lane : 2 * (lane - 16) + 1;
+    for (int64_t b = warp; b < nblk; b += nwarps) {
+        const int64_t rb = b / sp, w = b - rb * sp;
+        const int64_t row = rb * 32 + col;
+        const uint32_t word = row < rows ? src[row * sp + w] : 0u;
+        uint32_t mine = 0u;
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
+            const int bit = (c & 1) ? 16 + (c >> 1) : (c >> 1);
+            const uint32_t t = __ballot_sync(0xffffffffu, (word >> bit) & 1u);
+            if (lane == c) mine = t;
+        }
+        const int64_t nrow = w * 32 + lane;   // dst row = src column
+        if (nrow < k) dst[nrow * dp + rb] = mine;
+    }
+}
+
 int grid_for(int64_t work, int per_block)
 {
     int dev = 0, sms = 148;
@@ -120,6 +152,13 @@ cudaError_t launch_pack(const void *src, dbf_dtype dt, int64_t rows, int64_t k, 
     default:
         return cudaErrorInvalidValue;
     }
+    return cudaGetLastError();
+}
+
+cudaError_t launch_transpose(const uint32_t *src, int64_t rows, int64_t k, uint32_t *dst, cudaStream_t s)
+{
+    const int grid = grid_for(pitch_words(rows) * pitch_words(k), 8);
+    transpose_kernel<<<grid, 256, 0, s>>>(src, rows, k, dst);
     return cudaGetLastError();
 }
 

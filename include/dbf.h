@@ -113,6 +113,16 @@ dbf_status dbf_pack_signs(const void *src, dbf_dtype src_dtype, int64_t rows, in
 dbf_status dbf_unpack_signs(const uint32_t *src, int64_t rows, int64_t k, int8_t *dst,
                             void *stream);
 
+/* Transpose of a packed sign matrix: src is rows x k packed along k, dst
+ * becomes k x rows packed along rows, in the same layout (bit set = -1,
+ * pair-interleaved bits, zero padding). The backward (dbf_backward) needs
+ * B1^T and B2^T in this form: its transposed contractions then read packed
+ * rows like the forward does. Bit-exact; no arithmetic.
+ * src, dst: device, 4-byte aligned; dst_bytes >= dbf_packed_bytes(k, rows).
+ * Errors: DBF_ERR_INVALID_ARG, DBF_ERR_ALIGNMENT, DBF_ERR_CUDA. */
+dbf_status dbf_transpose_signs(const uint32_t *src, int64_t rows, int64_t k, uint32_t *dst,
+                               size_t dst_bytes, void *stream);
+
 /* Smallest T for which DBF_PATH_AUTO takes the GEMM path on a shape it allows. */
 int64_t dbf_gemm_min_tokens(void);
 
@@ -151,6 +161,38 @@ int32_t dbf_forward_launches(const dbf_layer *L, int64_t T, dbf_path path);
 dbf_status dbf_forward(const dbf_layer *L, const void *x, dbf_dtype x_dtype, void *y,
                        dbf_dtype y_dtype, int64_t T, int flags, dbf_path path, void *ws,
                        size_t ws_bytes, void *stream);
+
+/* Workspace bytes dbf_backward needs (0 for invalid input or a shape the
+ * backward does not serve). */
+size_t dbf_backward_workspace_bytes(const dbf_layer *L, int64_t T);
+
+/* Gradients of a loss through dbf_forward, given dy = dL/dy (LoRDBA page,
+ * section 2, training pipeline: quantisation-aware training differentiates
+ * this forward; the pages give no formula, these are the forward's
+ * derivatives by the chain rule). With u_i = gamma_i.x, h_i = B2 u_i,
+ * v_i = beta_i.h_i, z_i = B1 v_i, a_i = alpha_i.dy, g_i = B1^T a_i,
+ * e_i = B2^T (beta_i.g_i), per token:
+ *   dx      = sum_i gamma_i . e_i                     (T x M)
+ *   dalpha_i = sum_t dy . z_i,  dbeta_i = sum_t g_i . h_i,
+ *   dgamma_i = sum_t x . e_i                          ([ell][N], [ell][R], [ell][M])
+ * Runs on the tensor cores as four sign GEMMs (needs M, N, R multiples of
+ * 128; any T); u_i, alpha_i.dy, beta_i.h_i and beta_i.g_i are fp16 operands
+ * (|values| below 65504; apply loss scaling to tiny dy), fp32 accumulation.
+ * L: the layer (device pointers as in dbf_forward).
+ * b1t_packed: B1^T (R x N, packed along N), b2t_packed: B2^T (M x R, packed
+ *    along R), both from dbf_transpose_signs, 16-byte aligned.
+ * x: T x M and dy: T x N, DBF_F32 or DBF_BF16, 16-byte aligned.
+ * dx, dalpha, dbeta, dgamma: device fp32 outputs, each optional (NULL skips
+ *    it; dalpha's GEMM and the dx/dgamma GEMM are skipped when not wanted).
+ *    Overwritten, or added to with flags = DBF_ACCUMULATE.
+ * ws: dbf_backward_workspace_bytes(L, T) bytes, 256-byte aligned, header as
+ *    in dbf_forward.
+ * Errors: DBF_ERR_INVALID_ARG, DBF_ERR_ALIGNMENT, DBF_ERR_WORKSPACE,
+ *    DBF_ERR_UNSUPPORTED (shape), DBF_ERR_CUDA. */
+dbf_status dbf_backward(const dbf_layer *L, const uint32_t *b1t_packed, const uint32_t *b2t_packed,
+                        const void *x, dbf_dtype x_dtype, const void *dy, dbf_dtype dy_dtype, int64_t T,
+                        float *dx, float *dalpha, float *dbeta, float *dgamma, int flags, void *ws,
+                        size_t ws_bytes, void *stream);
 
 /* Workspace bytes dbf_forward_segmented needs. */
 size_t dbf_segmented_workspace_bytes(int32_t max_R, int32_t max_ell, int64_t T);

@@ -131,3 +131,34 @@ def test_forward_launch_count(lib):
     assert lib.dbf_forward_launches(by(L3), 1, dbf.PATH_GEMV) == 2
     assert lib.dbf_forward_launches(by(L), 0, dbf.PATH_AUTO) == 0
     assert lib.dbf_forward_launches(None, 1, dbf.PATH_AUTO) == 0
+
+
+def test_backward_rejects_bad_arguments_without_launch(lib):
+    import double_binary_rank_b200 as dbf
+    by = ctypes.byref
+    L = _layer(M=256, N=384, R=128, ell=2)
+    f = lib.dbf_backward
+    p = 0x1000
+    # flags other than ACCUMULATE, bad dtypes, null operands
+    assert f(by(L), p, p, p, dbf.F32, p, dbf.F32, 4, p, p, p, p, 2, p, 1 << 30, None) == dbf.ERR_INVALID_ARG
+    assert f(by(L), p, p, p, dbf.I8, p, dbf.F32, 4, p, p, p, p, 0, p, 1 << 30, None) == dbf.ERR_INVALID_ARG
+    assert f(by(L), None, p, p, dbf.F32, p, dbf.F32, 4, p, p, p, p, 0, p, 1 << 30, None) == dbf.ERR_INVALID_ARG
+    # shapes off the 128 grid are not served
+    L2 = _layer(M=200, N=384, R=128)
+    assert f(by(L2), p, p, p, dbf.F32, p, dbf.F32, 4, p, p, p, p, 0, p, 1 << 30, None) == dbf.ERR_UNSUPPORTED
+    assert lib.dbf_backward_workspace_bytes(by(L2), 4) == 0
+    # alignment and workspace
+    assert f(by(L), p, p, p + 4, dbf.F32, p, dbf.F32, 4, p, p, p, p, 0, p, 1 << 30, None) == dbf.ERR_ALIGNMENT
+    need = lib.dbf_backward_workspace_bytes(by(L), 4)
+    assert need >= 256 + 2 * 4 * (256 + 384) * 2 + 2 * 4 * 128 * 8
+    assert f(by(L), p, p, p, dbf.F32, p, dbf.F32, 4, p, p, p, p, 0, p, need - 1, None) == dbf.ERR_WORKSPACE
+    # T == 0 is a no-op
+    assert f(by(L), p, p, p, dbf.F32, p, dbf.F32, 0, p, p, p, p, 0, None, 0, None) == dbf.OK
+
+
+def test_transpose_rejects_bad_arguments(lib):
+    import double_binary_rank_b200 as dbf
+    t = lib.dbf_transpose_signs
+    assert t(None, 4, 4, 0x1000, 1 << 20, None) == dbf.ERR_INVALID_ARG
+    assert t(0x1000, 40, 64, 0x1000, lib.dbf_packed_bytes(64, 40) - 1, None) == dbf.ERR_INVALID_ARG
+    assert t(0x1002, 40, 64, 0x1000, 1 << 20, None) == dbf.ERR_ALIGNMENT

@@ -1,0 +1,130 @@
+"""dbf_transpose_signs and dbf_backward on the GPU against the fp64 oracle.
+
+Transposition is bit-exact. Gradients: max|g - g_ref| / max|g_ref| <= 2e-3
+per output (the forward's bound; operands are fp16, accumulation fp32). At
+the DBF MLP layer's full size (T = 2048, the bench's backward call) dx is
+compared on sampled token rows (rows are independent) and the scale
+gradients through Euler's identity, which holds at any size:
+sum(alpha . dalpha) = sum(beta . dbeta) = sum(gamma . dgamma) =
+sum(x . dx) = sum(dy . y).
+"""
+import numpy as np
+import pytest
+import torch
+
+import dbf_synth as S
+import oracle
+from gpu_util import dev_layer, dev_x, random_layer, rel_err
+
+pytestmark = pytest.mark.gpu
+
+TOL = 2e-3
+
+
+@pytest.fixture(scope="module")
+def dbf():
+    import double_binary_rank_b200 as m
+    return m
+
+
+@pytest.mark.parametrize("rows,k", [(1, 1), (33, 70), (256, 128), (130, 4100), (1000, 31)])
+def test_transpose_bit_exact(dbf, rows, k):
+    rng = np.random.default_rng(rows * 13 + k)
+    s = rng.choice(np.array([-1, 1], dtype=np.int8), size=(rows, k))
+    words = torch.from_numpy(oracle.pack(s).reshape(rows, -1).view(np.int32)).cuda()
+    t = dbf.transpose_signs(words, rows, k)
+    ref = oracle.pack(np.ascontiguousarray(s.T)).reshape(k, -1)
+    assert np.array_equal(t.cpu().numpy().view(np.uint32), ref)
+    back = dbf.transpose_signs(t, k, rows)
+    assert torch.equal(back, words)
+
+
+def gpu_grads(dbf, L, x, dy, **kw):
+    dl = dev_layer(L)
+    g = dbf.backward(dl, dev_x(x), dev_x(dy), **kw)
+    torch.cuda.synchronize()
+    return dl, g
+
+
+CASES = [  # M, N, R, ell, T: several 128-row tiles, ragged token counts, ell*T across 256-column tiles
+    (256, 384, 128, 1, 1), (256, 384, 128, 2, 37), (384, 256, 256, 1, 300), (128, 640, 384, 3, 100),
+    (512, 128, 128, 2, 257),
+]
+
+
+@pytest.mark.parametrize("case", CASES, ids=lambda c: "M{}N{}R{}l{}T{}".format(*c))
+@pytest.mark.parametrize("kind", ["bf16", "f32"])
+def test_backward_matches_oracle(dbf, case, kind):
+    M, N, R, ell, T = case
+    rng = np.random.default_rng(M + 3 * N + 7 * R + ell + T)
+    L = random_layer(rng, M, N, R, ell)
+    if kind == "bf16":
+        x = S.to_bf16_bits(rng.standard_normal((T, M)))
+        dy = S.to_bf16_bits(rng.standard_normal((T, N)))
+    else:
+        x = rng.standard_normal((T, M)).astype(np.float32)
+        dy = rng.standard_normal((T, N)).astype(np.float32)
+    ref = oracle.backward(L, x, dy)
+    _, g = gpu_grads(dbf, L, x, dy)
+    assert rel_err(g.dx.cpu().numpy(), ref.dx) < TOL
+    assert rel_err(g.dalpha.cpu().numpy(), ref.dalpha) < TOL
+    assert rel_err(g.dbeta.cpu().numpy(), ref.dbeta) < TOL
+    assert rel_err(g.dgamma.cpu().numpy(), ref.dgamma) < TOL
+
+
+def test_backward_accumulate_and_optional_outputs(dbf):
+    rng = np.random.default_rng(91)
+    L = random_layer(rng, 256, 256, 128, 2)
+    x = S.to_bf16_bits(rng.standard_normal((50, 256)))
+    dy = S.to_bf16_bits(rng.standard_normal((50, 256)))
+    ref = oracle.backward(L, x, dy)
+    dl = dev_layer(L)
+    xd, dyd = dev_x(x), dev_x(dy)
+    base = dbf.Grads(torch.full((50, 256), 0.5, device="cuda"), torch.full((2, 256), -1.0, device="cuda"),
+                     torch.full((2, 128), 2.0, device="cuda"), torch.full((2, 256), 0.25, device="cuda"))
+    g = dbf.backward(dl, xd, dyd, grads=base, accumulate=True)
+    torch.cuda.synchronize()
+    assert rel_err(g.dx.cpu().numpy() - 0.5, ref.dx) < TOL
+    assert rel_err(g.dalpha.cpu().numpy() + 1.0, ref.dalpha) < TOL
+    assert rel_err(g.dbeta.cpu().numpy() - 2.0, ref.dbeta) < TOL
+    assert rel_err(g.dgamma.cpu().numpy() - 0.25, ref.dgamma) < TOL
+    only = dbf.backward(dl, xd, dyd, want=("dbeta",))
+    torch.cuda.synchronize()
+    assert only.dx is None and only.dalpha is None and only.dgamma is None
+    assert rel_err(only.dbeta.cpu().numpy(), ref.dbeta) < TOL
+
+
+def test_backward_rejects_unsupported_shape(dbf):
+    rng = np.random.default_rng(92)
+    L = random_layer(rng, 200, 256, 128, 1)
+    dl = dev_layer(L)
+    x = dev_x(S.to_bf16_bits(rng.standard_normal((4, 200))))
+    dy = dev_x(S.to_bf16_bits(rng.standard_normal((4, 256))))
+    with pytest.raises(dbf.DbfError) as e:
+        dbf.backward(dl, x, dy, ws=torch.zeros(1 << 20, dtype=torch.uint8, device="cuda"))
+    assert e.value.status == dbf.ERR_UNSUPPORTED
+
+
+def test_dbf_mlp_full_size(dbf):
+    w = S.WORKLOADS["dbf_mlp"]
+    L = S.workload_layers(w)[0]
+    T = 2048
+    x = S.make_x(w.seed + 100, T, w.M, "bf16")
+    dy = S.make_x(w.seed + 200, T, w.N, "bf16")
+    dl, g = gpu_grads(dbf, L, x, dy)
+    rows = S.sample_rows(w.seed, T, 16)
+    ref = oracle.backward(L, x[rows], dy[rows])
+    assert rel_err(g.dx.cpu().numpy()[rows], ref.dx) < TOL
+    # Euler's identity over the whole batch
+    y = oracle.forward(L, x)
+    loss = float((y * S.bf16_bits_to_f32(dy).astype(np.float64)).sum())
+    dec = lambda b: np.asarray(b, dtype=np.uint16).view(np.float16).astype(np.float64)
+    sums = [
+        float((dec(L.alpha) * g.dalpha.double().cpu().numpy()).sum()),
+        float((dec(L.beta) * g.dbeta.double().cpu().numpy()).sum()),
+        float((dec(L.gamma) * g.dgamma.double().cpu().numpy()).sum()),
+        float((S.bf16_bits_to_f32(x).astype(np.float64) * g.dx.double().cpu().numpy()).sum()),
+    ]
+    scale = float(np.abs(y).max()) * np.sqrt(T * w.N)   # size of the terms of the sum
+    for v in sums:
+        assert abs(v - loss) <= TOL * scale, (v, loss)
