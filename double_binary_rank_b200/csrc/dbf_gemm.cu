@@ -41,12 +41,24 @@ namespace {
 constexpr int BM = 128;             // sign rows per tile (MMA M)
 constexpr int BN = 256;             // token rows per tile (MMA N)
 constexpr int BK = 64;              // K per stage: one 128-byte swizzle row of fp16
-constexpr int SA = 6;                // stages of expanded sign tiles (produced on chip)
-constexpr int SB = 4;                // stages of TMA activation tiles
-constexpr int kExpandGroups = 2;      // groups of four expansion warps, alternating pairs of K steps
-constexpr int kExpandWarps = 4 * kExpandGroups;
-constexpr int kEpiWarps = 4;          // one per TMEM lane quarter
-constexpr int kThreads = 32 * (2 + kExpandWarps + kEpiWarps);
+// Pipeline shapes, per kernel instance. The forward keeps two expansion
+// groups (alternating pairs of K steps) and four epilogue warps; the
+// backward, whose epilogues read and write an operand per element, takes
+// eight epilogue warps (two per TMEM lane quarter, each with half of the
+// columns) and one expansion group.
+template <int kGroups, int kSA, int kSB, int kEpi, bool kBackward>
+struct GemmCfg {
+    static constexpr bool kBwd = kBackward;      // epilogues of stages 3..6 compiled in
+    static constexpr int SA = kSA;               // stages of expanded sign tiles (produced on chip)
+    static constexpr int SB = kSB;               // stages of TMA activation tiles
+    static constexpr int kExpandGroups = kGroups;
+    static constexpr int kExpandWarps = 4 * kGroups;
+    static constexpr int kEpiWarps = kEpi;       // multiple of 4: kEpi / 4 warps per TMEM lane quarter
+    static constexpr int kThreads = 32 * (2 + kExpandWarps + kEpiWarps);
+};
+using FwdCfg = GemmCfg<2, 6, 4, 4, false>;
+using BwdCfg = GemmCfg<1, 4, 5, 8, true>;
+constexpr int kMaxStages = 8;
 constexpr int A_BYTES = BM * BK * 2;   // 16 KB
 constexpr int B_BYTES = BN * BK * 2;   // 32 KB
 constexpr int TMEM_COLS = 512;          // two 256-column accumulators
@@ -209,7 +221,7 @@ __device__ __forceinline__ uint32_t sign_pair(uint32_t w, int p, uint32_t mag2)
 }
 
 struct GemmSmem {
-    uint64_t full_a[SA], empty_a[SA], full_b[SB], empty_b[SB], acc_full[2], acc_empty[2];
+    uint64_t full_a[kMaxStages], empty_a[kMaxStages], full_b[kMaxStages], empty_b[kMaxStages], acc_full[2], acc_empty[2];
     uint32_t tmem_base;
     int abort;
 };
@@ -290,8 +302,13 @@ __device__ __forceinline__ void backward_chunk(const GemmArgs &g, const uint32_t
 
 // Persistent: CTA b takes tiles b, b + gridDim.x, ... (token-tile major, so
 // the CTAs running together share activation tiles in L2).
-__global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant__ CUtensorMap tmB, const GemmArgs g)
+template <class Cfg>
+__global__ void __launch_bounds__(Cfg::kThreads, 1) gemm_kernel(const __grid_constant__ CUtensorMap tmB, const GemmArgs g)
 {
+    constexpr int SA = Cfg::SA, SB = Cfg::SB, kExpandGroups = Cfg::kExpandGroups;
+    constexpr int kExpandWarps = Cfg::kExpandWarps, kEpiWarps = Cfg::kEpiWarps;
+    static_assert(SA <= kMaxStages && SB <= kMaxStages && kEpiWarps % 4 == 0 && BN % (32 * (kEpiWarps / 4)) == 0,
+                  "pipeline shape");
     extern __shared__ uint8_t smem_raw[];
     // 1024-byte alignment for the swizzled tiles
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -490,7 +507,9 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
         }
     } else {
         // ---------------- epilogue: one warp per TMEM lane quarter ----------------
-        const int q = warp & 3;
+        const int q = warp & 3;   // a warp reads the TMEM lane quarter warp % 4
+        const int ch = kEpiWarps == 4 ? 0 : (warp - 2 - kExpandWarps) >> 2;   // which share of the columns
+        constexpr int kColShare = BN / (kEpiWarps / 4);
         for (int j = 0; j < my_tiles; ++j) {
             const int ab = j & 1;
             if (!warp_wait(&sh->acc_full[ab], (j >> 1) & 1, abort)) break;
@@ -500,7 +519,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
             const int grow = p0 + q * 32 + lane;
             const uint32_t taddr = tmem + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(ab * BN);
             const bool row_ok = grow < g.P;
-            for (int cc = 0; cc < BN; cc += 32) {
+            for (int cc = ch * kColShare; cc < (ch + 1) * kColShare; cc += 32) {
                 uint32_t v[32];
                 tmem_ld32(taddr + cc, v);   // every lane takes part (.sync.aligned)
                 if (!row_ok) continue;
@@ -523,29 +542,38 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
                             vp = g.V + static_cast<int64_t>(i) * g.R + grow;
                         }
                     }
-                } else if (g.stage >= 3) {
+                } else if (Cfg::kBwd) {
                     backward_chunk(g, v, cb, grow);
                 } else {
                     const int64_t base = static_cast<int64_t>(cb) * g.N + grow;
                     const int n_ok = g.C - cb;   // tokens of this chunk inside the batch
-                    // with accumulation every y_in value of the chunk is loaded first
-                    float yin[32];
+                    // with accumulation the y_in values are loaded eight at a time,
+                    // all eight in flight together
                     if (g.yd == DBF_BF16) {
                         __nv_bfloat16 *yp = static_cast<__nv_bfloat16 *>(g.y) + base;
 #pragma unroll
-                        for (int e = 0; e < 32; ++e)
-                            yin[e] = g.accumulate ? __bfloat162float(yp[static_cast<int64_t>(e < n_ok ? e : 0) * g.N]) : 0.f;
+                        for (int e0 = 0; e0 < 32; e0 += 8) {
+                            float yin[8];
 #pragma unroll
-                        for (int e = 0; e < 32; ++e)
-                            if (e < n_ok) yp[static_cast<int64_t>(e) * g.N] = __float2bfloat16_rn(__uint_as_float(v[e]) + yin[e]);
+                            for (int e = 0; e < 8; ++e)
+                                yin[e] = g.accumulate ? __bfloat162float(yp[static_cast<int64_t>(e0 + e < n_ok ? e0 + e : 0) * g.N]) : 0.f;
+#pragma unroll
+                            for (int e = 0; e < 8; ++e)
+                                if (e0 + e < n_ok)
+                                    yp[static_cast<int64_t>(e0 + e) * g.N] = __float2bfloat16_rn(__uint_as_float(v[e0 + e]) + yin[e]);
+                        }
                     } else {
                         float *yp = static_cast<float *>(g.y) + base;
 #pragma unroll
-                        for (int e = 0; e < 32; ++e)
-                            yin[e] = g.accumulate ? yp[static_cast<int64_t>(e < n_ok ? e : 0) * g.N] : 0.f;
+                        for (int e0 = 0; e0 < 32; e0 += 8) {
+                            float yin[8];
 #pragma unroll
-                        for (int e = 0; e < 32; ++e)
-                            if (e < n_ok) yp[static_cast<int64_t>(e) * g.N] = __uint_as_float(v[e]) + yin[e];
+                            for (int e = 0; e < 8; ++e)
+                                yin[e] = g.accumulate ? yp[static_cast<int64_t>(e0 + e < n_ok ? e0 + e : 0) * g.N] : 0.f;
+#pragma unroll
+                            for (int e = 0; e < 8; ++e)
+                                if (e0 + e < n_ok) yp[static_cast<int64_t>(e0 + e) * g.N] = __uint_as_float(v[e0 + e]) + yin[e];
+                        }
                     }
                 }
             }
@@ -639,14 +667,16 @@ bool make_map(CUtensorMap *map, const void *base, int64_t K, int64_t rows)
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-constexpr size_t kGemmSmem = 1024 + SA * A_BYTES + SB * B_BYTES + sizeof(GemmSmem) + 64;
+template <class Cfg>
+constexpr size_t gemm_smem() { return 1024 + Cfg::SA * A_BYTES + Cfg::SB * B_BYTES + sizeof(GemmSmem) + 64; }
 
+template <class Cfg>
 cudaError_t launch_gemm(const CUtensorMap &map, const GemmArgs &a, cudaStream_t s)
 {
     static bool configured = false;
     if (!configured) {
-        cudaError_t e = cudaFuncSetAttribute(gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             static_cast<int>(kGemmSmem));
+        cudaError_t e = cudaFuncSetAttribute(gemm_kernel<Cfg>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             static_cast<int>(gemm_smem<Cfg>()));
         if (e != cudaSuccess) return e;
         configured = true;
     }
@@ -657,7 +687,7 @@ cudaError_t launch_gemm(const CUtensorMap &map, const GemmArgs &a, cudaStream_t 
         sms = (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && v > 0) ? v : 148;
     }
     const int tiles = ((a.P + BM - 1) / BM) * ((a.C + BN - 1) / BN);
-    gemm_kernel<<<tiles < sms ? tiles : sms, kThreads, kGemmSmem, s>>>(map, a);
+    gemm_kernel<Cfg><<<tiles < sms ? tiles : sms, Cfg::kThreads, gemm_smem<Cfg>(), s>>>(map, a);
     return cudaGetLastError();
 }
 
@@ -708,7 +738,7 @@ cudaError_t gemm_forward(const dbf_layer &L, const void *x, dbf_dtype xd, void *
     a1.ell = L.ell;
     a1.R = L.R;
     a1.N = L.N;
-    cudaError_t e = launch_gemm(mu, a1, s);
+    cudaError_t e = launch_gemm<FwdCfg>(mu, a1, s);
     if (e != cudaSuccess) return e;
     GemmArgs a2 = {};
     a2.signs = L.b1_packed;
@@ -726,7 +756,7 @@ cudaError_t gemm_forward(const dbf_layer &L, const void *x, dbf_dtype xd, void *
     a2.yd = yd;
     a2.N = L.N;
     a2.accumulate = (flags & DBF_ACCUMULATE) ? 1 : 0;
-    return launch_gemm(mv, a2, s);
+    return launch_gemm<FwdCfg>(mv, a2, s);
 }
 
 }  // namespace dbf
@@ -826,21 +856,21 @@ cudaError_t gemm_backward(const dbf_layer &L, const uint32_t *b1t, const uint32_
     g3.H32 = H32;
     g3.Vout = Vh;
     g3.cscale = L.beta;
-    if ((e = launch_gemm(mu, g3, s)) != cudaSuccess) return e;
+    if ((e = launch_gemm<BwdCfg>(mu, g3, s)) != cudaSuccess) return e;
     // G4
     GemmArgs g4 = sign_gemm_args(b1t, L.R, L.N, C, Ti, ell, 4);
     g4.H32 = H32;
     g4.Vout = Vg;
     g4.cscale = L.beta;
     g4.red = dbeta;
-    if ((e = launch_gemm(ma, g4, s)) != cudaSuccess) return e;
+    if ((e = launch_gemm<BwdCfg>(ma, g4, s)) != cudaSuccess) return e;
     // G5
     if (dalpha) {
         GemmArgs g5 = sign_gemm_args(L.b1_packed, L.N, L.R, C, Ti, ell, 5);
         g5.red = dalpha;
         g5.W = dy;
         g5.wd = dyd;
-        if ((e = launch_gemm(mvh, g5, s)) != cudaSuccess) return e;
+        if ((e = launch_gemm<BwdCfg>(mvh, g5, s)) != cudaSuccess) return e;
     }
     // G6
     if (dx || dgamma) {
@@ -851,7 +881,7 @@ cudaError_t gemm_backward(const dbf_layer &L, const uint32_t *b1t, const uint32_
         g6.cscale = L.gamma;
         g6.dx = dx;
         g6.dx_mode = ell > 1 ? 2 : (acc ? 1 : 0);
-        if ((e = launch_gemm(mvg, g6, s)) != cudaSuccess) return e;
+        if ((e = launch_gemm<BwdCfg>(mvg, g6, s)) != cudaSuccess) return e;
     }
     return cudaSuccess;
 }
