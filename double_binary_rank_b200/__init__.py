@@ -53,9 +53,10 @@ _SIGS = {
     "dbf_forward_launches": (_i32, [_LP, _i64, ctypes.c_int]),
     "dbf_forward": (ctypes.c_int, [_LP, _vp, ctypes.c_int, _vp, ctypes.c_int, _i64, ctypes.c_int,
                                    ctypes.c_int, _vp, _sz, _vp]),
-    "dbf_backward_workspace_bytes": (_sz, [_LP, _i64]),
+    "dbf_backward_workspace_bytes": (_sz, [_LP, _i64, ctypes.c_int]),
     "dbf_backward": (ctypes.c_int, [_LP, _vp, _vp, _vp, ctypes.c_int, _vp, ctypes.c_int, _i64, _vp, _vp, _vp,
-                                    _vp, ctypes.c_int, _vp, _sz, _vp]),
+                                    _vp, _vp, _vp, ctypes.c_int, _vp, _sz, _vp]),
+    "dbf_ste_backward": (ctypes.c_int, [_vp, _vp, ctypes.c_int, _i64, ctypes.c_float, _vp, ctypes.c_int, _vp]),
     "dbf_segmented_workspace_bytes": (_sz, [_i32, _i32, _i64]),
     "dbf_forward_segmented": (ctypes.c_int, [_vp, _i32, _vp, _vp, _i32, _i32, _i32, _i32, _i32,
                                              _vp, ctypes.c_int, _vp, ctypes.c_int, _i64,
@@ -223,6 +224,8 @@ class Grads:
     dalpha: Optional[torch.Tensor]   # [ell, N] fp32
     dbeta: Optional[torch.Tensor]    # [ell, R] fp32
     dgamma: Optional[torch.Tensor]   # [ell, M] fp32
+    db1: Optional[torch.Tensor] = None   # [N, R] fp32, sign-matrix gradient
+    db2: Optional[torch.Tensor] = None   # [R, M] fp32
 
 
 def transposed_signs(layer: Layer, stream=None):
@@ -231,9 +234,9 @@ def transposed_signs(layer: Layer, stream=None):
             transpose_signs(layer.b2, layer.R, layer.M, stream=stream))
 
 
-def backward_workspace_bytes(layer: Layer, T: int) -> int:
+def backward_workspace_bytes(layer: Layer, T: int, sign_grads: bool = False) -> int:
     d = layer.descriptor()
-    return int(_lib.dbf_backward_workspace_bytes(ctypes.byref(d), T))
+    return int(_lib.dbf_backward_workspace_bytes(ctypes.byref(d), T, int(sign_grads)))
 
 
 def backward(layer: Layer, x: torch.Tensor, dy: torch.Tensor, signs_t=None, grads: Optional[Grads] = None,
@@ -250,15 +253,28 @@ def backward(layer: Layer, x: torch.Tensor, dy: torch.Tensor, signs_t=None, grad
     if grads is None:
         mk = lambda name, shape: torch.empty(shape, dtype=torch.float32, device=dev) if name in want else None
         grads = Grads(mk("dx", (T, layer.M)), mk("dalpha", (layer.ell, layer.N)), mk("dbeta", (layer.ell, layer.R)),
-                      mk("dgamma", (layer.ell, layer.M)))
+                      mk("dgamma", (layer.ell, layer.M)), mk("db1", (layer.N, layer.R)), mk("db2", (layer.R, layer.M)))
     d = layer.descriptor()
     if ws is None:
-        ws = alloc_workspace(backward_workspace_bytes(layer, T), dev)
+        ws = alloc_workspace(backward_workspace_bytes(layer, T, grads.db1 is not None or grads.db2 is not None), dev)
     _check(_lib.dbf_backward(ctypes.byref(d), _ptr(signs_t[0]), _ptr(signs_t[1]), _ptr(x), _DT[x.dtype], _ptr(dy),
                              _DT[dy.dtype], T, _ptr(grads.dx), _ptr(grads.dalpha), _ptr(grads.dbeta),
-                             _ptr(grads.dgamma), ACCUMULATE if accumulate else 0, _ptr(ws), ws.numel(),
-                             _stream(stream)), "dbf_backward")
+                             _ptr(grads.dgamma), _ptr(grads.db1), _ptr(grads.db2), ACCUMULATE if accumulate else 0,
+                             _ptr(ws), ws.numel(), _stream(stream)), "dbf_backward")
     return grads
+
+
+def ste_backward(db: torch.Tensor, h: torch.Tensor, tau: float = 0.0, dh: Optional[torch.Tensor] = None,
+                 accumulate: bool = False, stream=None) -> torch.Tensor:
+    """dH = dB * s'(H) (dbf_ste_backward): s = tanh(H / tau) for tau > 0, else
+    the identity clipped to |H| <= 1."""
+    db = db.contiguous()
+    h = h.contiguous()
+    if dh is None:
+        dh = torch.empty(h.shape, dtype=torch.float32, device=h.device)
+    _check(_lib.dbf_ste_backward(_ptr(db), _ptr(h), _DT[h.dtype], h.numel(), float(tau), _ptr(dh),
+                                 ACCUMULATE if accumulate else 0, _stream(stream)), "dbf_ste_backward")
+    return dh
 
 
 def forward_decode_noalloc(layer: Layer, x: torch.Tensor, y: Optional[torch.Tensor] = None,

@@ -74,6 +74,19 @@ dbf_status dbf_transpose_signs(const uint32_t *src, int64_t rows, int64_t k, uin
     return from_cuda(launch_transpose(src, rows, k, dst, static_cast<cudaStream_t>(stream)));
 }
 
+dbf_status dbf_ste_backward(const float *db, const void *h, dbf_dtype h_dtype, int64_t count, float tau,
+                            float *dh, int flags, void *stream)
+{
+    if (count < 0 || (h_dtype != DBF_F32 && h_dtype != DBF_F16 && h_dtype != DBF_BF16) ||
+        (flags & ~DBF_ACCUMULATE) || !(tau == tau))
+        return DBF_ERR_INVALID_ARG;
+    if (count == 0) return DBF_OK;
+    if (!db || !h || !dh) return DBF_ERR_INVALID_ARG;
+    if (!aligned(db, 4) || !aligned(dh, 4) || !aligned(h, h_dtype == DBF_F32 ? 4 : 2)) return DBF_ERR_ALIGNMENT;
+    return from_cuda(launch_ste(db, h, h_dtype, count, tau, dh, (flags & DBF_ACCUMULATE) ? 1 : 0,
+                                static_cast<cudaStream_t>(stream)));
+}
+
 int64_t dbf_gemm_min_tokens(void) { return kGemmMinTokens; }
 
 size_t dbf_workspace_bytes(const dbf_layer *L, int64_t T, dbf_path path)
@@ -120,18 +133,18 @@ dbf_status dbf_forward(const dbf_layer *L, const void *x, dbf_dtype x_dtype, voi
     return from_cuda(gemv_forward(*L, x, x_dtype, y, y_dtype, T, flags, ws, s));
 }
 
-size_t dbf_backward_workspace_bytes(const dbf_layer *L, int64_t T)
+size_t dbf_backward_workspace_bytes(const dbf_layer *L, int64_t T, int with_sign_grads)
 {
     if (!L || L->M <= 0 || L->N <= 0 || L->R <= 0 || L->ell < 1 || L->ell > kMaxEll || T < 0)
         return 0;
     if (!gemm_backward_shape_ok(*L)) return 0;
-    return gemm_backward_workspace_bytes(*L, T);
+    return gemm_backward_workspace_bytes(*L, T, with_sign_grads != 0);
 }
 
 dbf_status dbf_backward(const dbf_layer *L, const uint32_t *b1t_packed, const uint32_t *b2t_packed,
                         const void *x, dbf_dtype x_dtype, const void *dy, dbf_dtype dy_dtype, int64_t T,
-                        float *dx, float *dalpha, float *dbeta, float *dgamma, int flags, void *ws,
-                        size_t ws_bytes, void *stream)
+                        float *dx, float *dalpha, float *dbeta, float *dgamma, float *db1, float *db2,
+                        int flags, void *ws, size_t ws_bytes, void *stream)
 {
     dbf_status st = check_layer(L);
     if (st != DBF_OK) return st;
@@ -142,13 +155,13 @@ dbf_status dbf_backward(const dbf_layer *L, const uint32_t *b1t_packed, const ui
     if (!b1t_packed || !b2t_packed || !x || !dy) return DBF_ERR_INVALID_ARG;
     if (!aligned(b1t_packed, 16) || !aligned(b2t_packed, 16) || !aligned(x, 16) || !aligned(dy, 16) ||
         (dbeta && !aligned(dbeta, 4)) || (dx && !aligned(dx, 4)) || (dalpha && !aligned(dalpha, 4)) ||
-        (dgamma && !aligned(dgamma, 4)))
+        (dgamma && !aligned(dgamma, 4)) || (db1 && !aligned(db1, 4)) || (db2 && !aligned(db2, 4)))
         return DBF_ERR_ALIGNMENT;
-    const size_t need = gemm_backward_workspace_bytes(*L, T);
+    const size_t need = gemm_backward_workspace_bytes(*L, T, db1 || db2);
     if (!ws || ws_bytes < need) return DBF_ERR_WORKSPACE;
     if (!aligned(ws, 256)) return DBF_ERR_ALIGNMENT;
     return from_cuda(gemm_backward(*L, b1t_packed, b2t_packed, x, x_dtype, dy, dy_dtype, T, dx, dalpha, dbeta,
-                                   dgamma, flags, ws, static_cast<cudaStream_t>(stream)));
+                                   dgamma, db1, db2, flags, ws, static_cast<cudaStream_t>(stream)));
 }
 
 size_t dbf_segmented_workspace_bytes(int32_t max_R, int32_t max_ell, int64_t T)

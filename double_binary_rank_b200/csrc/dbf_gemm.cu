@@ -93,6 +93,7 @@ struct GemmArgs {
     dbf_dtype wd;
     float *dx;                // stage 6 (optional): [T][P] receives sum_i gamma_i[p] acc
     int dx_mode;              // 0 store, 1 add, 2 atomic add
+    int dense_a;              // A is a dense fp16 [P][Ktot] matrix loaded by TMA (tmA), not packed signs
 };
 
 // ---- small PTX helpers --------------------------------------------------------
@@ -303,7 +304,8 @@ __device__ __forceinline__ void backward_chunk(const GemmArgs &g, const uint32_t
 // Persistent: CTA b takes tiles b, b + gridDim.x, ... (token-tile major, so
 // the CTAs running together share activation tiles in L2).
 template <class Cfg>
-__global__ void __launch_bounds__(Cfg::kThreads, 1) gemm_kernel(const __grid_constant__ CUtensorMap tmB, const GemmArgs g)
+__global__ void __launch_bounds__(Cfg::kThreads, 1) gemm_kernel(const __grid_constant__ CUtensorMap tmB,
+                                                                const __grid_constant__ CUtensorMap tmA, const GemmArgs g)
 {
     constexpr int SA = Cfg::SA, SB = Cfg::SB, kExpandGroups = Cfg::kExpandGroups;
     constexpr int kExpandWarps = Cfg::kExpandWarps, kEpiWarps = Cfg::kEpiWarps;
@@ -327,7 +329,7 @@ __global__ void __launch_bounds__(Cfg::kThreads, 1) gemm_kernel(const __grid_con
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < SA; ++i) {
-            bar_init(&sh->full_a[i], 4);   // the four warps of one expansion group
+            bar_init(&sh->full_a[i], g.dense_a ? 1 : 4);   // the TMA producer, or the four warps of one expansion group
             bar_init(&sh->empty_a[i], 1);
         }
         for (int i = 0; i < SB; ++i) {
@@ -341,6 +343,7 @@ __global__ void __launch_bounds__(Cfg::kThreads, 1) gemm_kernel(const __grid_con
         sh->abort = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         asm volatile("prefetch.tensormap [%0];" ::"l"(&tmB) : "memory");
+        if (g.dense_a) asm volatile("prefetch.tensormap [%0];" ::"l"(&tmA) : "memory");
     }
     if (warp == 1) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&sh->tmem_base)),
@@ -359,11 +362,20 @@ __global__ void __launch_bounds__(Cfg::kThreads, 1) gemm_kernel(const __grid_con
             for (int j = 0; j < my_tiles && !*abort; ++j) {
                 const int tile = blockIdx.x + j * gridDim.x;
                 const int c0 = (tile / n_p) * BN;
+                const int p0 = (tile % n_p) * BM;
                 for (int k = 0; k < nk; ++k, ++s) {
                     const int st = s % SB;
                     if (!bar_wait(&sh->empty_b[st], ((s / SB) & 1) ^ 1, abort)) break;
                     bar_expect_tx(&sh->full_b[st], B_BYTES);
                     tma_load_2d(smB + st * B_BYTES, &tmB, k * BK, c0, &sh->full_b[st]);
+                    if (g.dense_a) {
+                        // a dense fp16 A operand: its tile comes by TMA too, in the
+                        // same swizzled K-major layout the expansion writes
+                        const int sa = s % SA;
+                        if (!bar_wait(&sh->empty_a[sa], ((s / SA) & 1) ^ 1, abort)) break;
+                        bar_expect_tx(&sh->full_a[sa], A_BYTES);
+                        tma_load_2d(smA + sa * A_BYTES, &tmA, k * BK, p0, &sh->full_a[sa]);
+                    }
                 }
             }
         }
@@ -395,6 +407,7 @@ __global__ void __launch_bounds__(Cfg::kThreads, 1) gemm_kernel(const __grid_con
             }
         }
     } else if (warp < 2 + kExpandWarps) {
+        if (g.dense_a) goto teardown;   // A tiles come by TMA
         // ---------------- sign expansion: one tile row per thread ----------------
         // kExpandGroups groups of four warps take turns by pairs of K steps;
         // each thread of a group owns one tile row.
@@ -583,12 +596,32 @@ __global__ void __launch_bounds__(Cfg::kThreads, 1) gemm_kernel(const __grid_con
         }
     }
 
+teardown:
     tc_fence_before();
     __syncthreads();
     if (sh->abort && threadIdx.x == 0 && g.status) atomicExch(g.status, static_cast<int32_t>(DBF_ERR_TIMEOUT));
     if (warp == 1) {
         tc_fence_after();
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS));
+    }
+}
+
+// out[k][c] = in[c][k] for an fp16 matrix in[C][K]; columns C .. Cp-1 of out
+// are zero (the row pitch of out is Cp). 32 x 32 tiles through shared memory.
+__global__ void __launch_bounds__(256) transpose_f16_kernel(const uint16_t *__restrict__ in, int C, int K,
+                                                            uint16_t *__restrict__ out, int Cp)
+{
+    __shared__ uint16_t tile[32][34];
+    const int k0 = blockIdx.x * 32, c0 = blockIdx.y * 32;
+    const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;   // 32 x 8 threads
+    for (int r = ty; r < 32; r += 8) {
+        const int c = c0 + r, k = k0 + tx;
+        tile[r][tx] = (c < C && k < K) ? in[static_cast<int64_t>(c) * K + k] : uint16_t(0);
+    }
+    __syncthreads();
+    for (int r = ty; r < 32; r += 8) {
+        const int k = k0 + r, c = c0 + tx;
+        if (k < K && c < Cp) out[static_cast<int64_t>(k) * Cp + c] = tile[tx][r];
     }
 }
 
@@ -654,13 +687,15 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn()
 }
 
 // 2-D fp16 map of a [rows x K] row-major matrix, boxes of 64 K x 256 rows.
-bool make_map(CUtensorMap *map, const void *base, int64_t K, int64_t rows)
+// box_rows: BN for the B operand, BM for a dense A operand; ld: elements
+// per row (>= K, a multiple of 8).
+bool make_map(CUtensorMap *map, const void *base, int64_t K, int64_t rows, int box_rows = BN, int64_t ld = 0)
 {
     auto fn = encode_fn();
     if (!fn) return false;
     const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows)};
-    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K) * 2};
-    const cuuint32_t box[2] = {BK, BN};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld > 0 ? ld : K) * 2};
+    const cuuint32_t box[2] = {BK, static_cast<cuuint32_t>(box_rows)};
     const cuuint32_t estr[2] = {1, 1};
     return fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -671,7 +706,7 @@ template <class Cfg>
 constexpr size_t gemm_smem() { return 1024 + Cfg::SA * A_BYTES + Cfg::SB * B_BYTES + sizeof(GemmSmem) + 64; }
 
 template <class Cfg>
-cudaError_t launch_gemm(const CUtensorMap &map, const GemmArgs &a, cudaStream_t s)
+cudaError_t launch_gemm(const CUtensorMap &map, const GemmArgs &a, cudaStream_t s, const CUtensorMap *map_a = nullptr)
 {
     static bool configured = false;
     if (!configured) {
@@ -687,7 +722,7 @@ cudaError_t launch_gemm(const CUtensorMap &map, const GemmArgs &a, cudaStream_t 
         sms = (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && v > 0) ? v : 148;
     }
     const int tiles = ((a.P + BM - 1) / BM) * ((a.C + BN - 1) / BN);
-    gemm_kernel<Cfg><<<tiles < sms ? tiles : sms, Cfg::kThreads, gemm_smem<Cfg>(), s>>>(map, a);
+    gemm_kernel<Cfg><<<tiles < sms ? tiles : sms, Cfg::kThreads, gemm_smem<Cfg>(), s>>>(map, map_a ? *map_a : map, a);
     return cudaGetLastError();
 }
 
@@ -777,20 +812,65 @@ cudaError_t scale_cast(const void *x, dbf_dtype xd, const uint16_t *scale, int K
 }
 
 struct BwdLayout {
-    size_t u, a, h32, vh, vg, total;   // offsets after the header
+    size_t u, a, h32, vh, vg;       // offsets after the header
+    size_t ut, at, vht, vgt;        // transposed operands of the sign-matrix gradients
+    size_t total;
+    int64_t cp;                     // row pitch of the transposed operands (elements)
 };
 
-BwdLayout bwd_layout(const dbf_layer &L, int64_t T)
+BwdLayout bwd_layout(const dbf_layer &L, int64_t T, bool signs)
 {
     const int64_t C = static_cast<int64_t>(L.ell) * T;
     BwdLayout b;
+    b.cp = (C + 7) / 8 * 8;
     b.u = 0;
     b.a = b.u + align_up(static_cast<size_t>(C) * L.M * 2, 256);
     b.h32 = b.a + align_up(static_cast<size_t>(C) * L.N * 2, 256);
     b.vh = b.h32 + align_up(static_cast<size_t>(C) * L.R * 4, 256);
     b.vg = b.vh + align_up(static_cast<size_t>(C) * L.R * 2, 256);
     b.total = b.vg + align_up(static_cast<size_t>(C) * L.R * 2, 256);
+    b.ut = b.at = b.vht = b.vgt = 0;
+    if (signs) {
+        b.ut = b.total;
+        b.at = b.ut + align_up(static_cast<size_t>(b.cp) * L.M * 2, 256);
+        b.vht = b.at + align_up(static_cast<size_t>(b.cp) * L.N * 2, 256);
+        b.vgt = b.vht + align_up(static_cast<size_t>(b.cp) * L.R * 2, 256);
+        b.total = b.vgt + align_up(static_cast<size_t>(b.cp) * L.R * 2, 256);
+    }
     return b;
+}
+
+cudaError_t transpose_f16(const __half *in, int64_t C, int64_t K, __half *out, int64_t Cp, cudaStream_t s)
+{
+    const dim3 grid(static_cast<unsigned>((K + 31) / 32), static_cast<unsigned>((Cp + 31) / 32));
+    transpose_f16_kernel<<<grid, 256, 0, s>>>(reinterpret_cast<const uint16_t *>(in), static_cast<int>(C),
+                                              static_cast<int>(K), reinterpret_cast<uint16_t *>(out),
+                                              static_cast<int>(Cp));
+    return cudaGetLastError();
+}
+
+// out[q][p] (+)= sum_c A[p][c] Bm[q][c] over the Kpad contraction (fp16
+// operands [P][cp] and [Q][cp], zero past the real length), fp32 out with row
+// pitch P: the dense GEMM of the sign-matrix gradients.
+cudaError_t dense_outer(const __half *A, int64_t P, const __half *Bm, int64_t Q, int64_t cp, float *out, bool acc,
+                        cudaStream_t s)
+{
+    CUtensorMap ma, mb;
+    if (!make_map(&ma, A, cp, P, BM) || !make_map(&mb, Bm, cp, Q, BN)) return cudaErrorInvalidValue;
+    GemmArgs g = {};
+    g.dense_a = 1;
+    g.P = static_cast<int>(P);
+    g.Ktot = g.Kp = static_cast<int>((cp + 2 * BK - 1) / (2 * BK) * (2 * BK));
+    g.pitch = 1;
+    g.C = static_cast<int>(Q);
+    g.T = static_cast<int>(Q);
+    g.ell = 1;
+    g.stage = 2;
+    g.y = out;
+    g.yd = DBF_F32;
+    g.N = static_cast<int>(P);
+    g.accumulate = acc ? 1 : 0;
+    return launch_gemm<FwdCfg>(mb, g, s, &ma);
 }
 
 GemmArgs sign_gemm_args(const uint32_t *signs, int P, int K, int C, int T, int ell, int stage)
@@ -815,7 +895,10 @@ bool gemm_backward_shape_ok(const dbf_layer &L)
     return L.M % 128 == 0 && L.N % 128 == 0 && L.R % 128 == 0 && L.M > 0 && L.N > 0 && L.R > 0;
 }
 
-size_t gemm_backward_workspace_bytes(const dbf_layer &L, int64_t T) { return kWsHeaderBytes + bwd_layout(L, T).total; }
+size_t gemm_backward_workspace_bytes(const dbf_layer &L, int64_t T, bool signs)
+{
+    return kWsHeaderBytes + bwd_layout(L, T, signs).total;
+}
 
 // Gradients through the forward (see dbf.h, dbf_backward), as four sign
 // GEMMs whose epilogues do the per-channel scalings and the reductions over
@@ -826,12 +909,13 @@ size_t gemm_backward_workspace_bytes(const dbf_layer &L, int64_t T) { return kWs
 //   G6: e_i = B2^T Vg_i                               -> dgamma_i += sum_t e x, dx = sum_i gamma_i . e
 cudaError_t gemm_backward(const dbf_layer &L, const uint32_t *b1t, const uint32_t *b2t, const void *x, dbf_dtype xd,
                           const void *dy, dbf_dtype dyd, int64_t T, float *dx, float *dalpha, float *dbeta,
-                          float *dgamma, int flags, void *ws, cudaStream_t s)
+                          float *dgamma, float *db1, float *db2, int flags, void *ws, cudaStream_t s)
 {
     if (T > (1 << 30) / L.ell) return cudaErrorInvalidValue;
     const bool acc = (flags & DBF_ACCUMULATE) != 0;
     const int ell = L.ell, Ti = static_cast<int>(T), C = ell * Ti;
-    const BwdLayout b = bwd_layout(L, T);
+    const bool signs = db1 || db2;
+    const BwdLayout b = bwd_layout(L, T, signs);
     char *body = static_cast<char *>(ws) + kWsHeaderBytes;
     __half *U = reinterpret_cast<__half *>(body + b.u);
     __half *A = reinterpret_cast<__half *>(body + b.a);
@@ -882,6 +966,22 @@ cudaError_t gemm_backward(const dbf_layer &L, const uint32_t *b1t, const uint32_
         g6.dx = dx;
         g6.dx_mode = ell > 1 ? 2 : (acc ? 1 : 0);
         if ((e = launch_gemm<BwdCfg>(mvg, g6, s)) != cudaSuccess) return e;
+    }
+    // sign-matrix gradients: dB1 = sum_c a_c v_c^T (N x R), dB2 = sum_c w_c u_c^T
+    // (R x M), dense products contracting over the envelope-major token index
+    if (signs) {
+        __half *Ut = reinterpret_cast<__half *>(body + b.ut), *At = reinterpret_cast<__half *>(body + b.at);
+        __half *Vht = reinterpret_cast<__half *>(body + b.vht), *Vgt = reinterpret_cast<__half *>(body + b.vgt);
+        if (db1) {
+            if ((e = transpose_f16(Vh, C, L.R, Vht, b.cp, s)) != cudaSuccess) return e;
+            if ((e = transpose_f16(A, C, L.N, At, b.cp, s)) != cudaSuccess) return e;
+            if ((e = dense_outer(Vht, L.R, At, L.N, b.cp, db1, acc, s)) != cudaSuccess) return e;
+        }
+        if (db2) {
+            if ((e = transpose_f16(U, C, L.M, Ut, b.cp, s)) != cudaSuccess) return e;
+            if ((e = transpose_f16(Vg, C, L.R, Vgt, b.cp, s)) != cudaSuccess) return e;
+            if ((e = dense_outer(Ut, L.M, Vgt, L.R, b.cp, db2, acc, s)) != cudaSuccess) return e;
+        }
     }
     return cudaSuccess;
 }

@@ -27,6 +27,8 @@ cudaError_t launch_unpack(const uint32_t *src, int64_t rows, int64_t k, int8_t *
                           cudaStream_t s);
 cudaError_t launch_transpose(const uint32_t *src, int64_t rows, int64_t k, uint32_t *dst,
                              cudaStream_t s);
+cudaError_t launch_ste(const float *db, const void *h, dbf_dtype hd, int64_t n, float tau, float *dh,
+                       int accumulate, cudaStream_t s);
 
 // decode path
 size_t gemv_workspace_bytes(int64_t R, int64_t ell, int64_t T);
@@ -45,11 +47,11 @@ size_t gemm_workspace_bytes(const dbf_layer &L, int64_t T);
 cudaError_t gemm_forward(const dbf_layer &L, const void *x, dbf_dtype xd, void *y, dbf_dtype yd,
                          int64_t T, int flags, void *ws, cudaStream_t s);
 bool gemm_backward_shape_ok(const dbf_layer &L);
-size_t gemm_backward_workspace_bytes(const dbf_layer &L, int64_t T);
+size_t gemm_backward_workspace_bytes(const dbf_layer &L, int64_t T, bool signs);
 cudaError_t gemm_backward(const dbf_layer &L, const uint32_t *b1t, const uint32_t *b2t, const void *x,
                           dbf_dtype xd, const void *dy, dbf_dtype dyd, int64_t T, float *dx,
-                          float *dalpha, float *dbeta, float *dgamma, int flags, void *ws,
-                          cudaStream_t s);
+                          float *dalpha, float *dbeta, float *dgamma, float *db1, float *db2,
+                          int flags, void *ws, cudaStream_t s);
 
 inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 

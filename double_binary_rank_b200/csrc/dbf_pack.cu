@@ -116,6 +116,39 @@ __global__ void __launch_bounds__(256) transpose_kernel(const uint32_t *__restri
     }
 }
 
+// Straight-through estimator on the latents: dH = dB * s'(H) with the
+// surrogate s = tanh(H / tau) (tau > 0) or the identity clipped to |H| <= 1.
+template <typename T>
+__device__ __forceinline__ float latent_value(const T *h, int64_t i);
+template <>
+__device__ __forceinline__ float latent_value<float>(const float *h, int64_t i) { return h[i]; }
+template <>
+__device__ __forceinline__ float latent_value<__half>(const __half *h, int64_t i) { return __half2float(h[i]); }
+template <>
+__device__ __forceinline__ float latent_value<__nv_bfloat16>(const __nv_bfloat16 *h, int64_t i)
+{
+    return __bfloat162float(h[i]);
+}
+
+template <typename T>
+__global__ void __launch_bounds__(256) ste_kernel(const float *__restrict__ db, const T *__restrict__ h, int64_t n,
+                                                  float tau, float *__restrict__ dh, int accumulate)
+{
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+         i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const float v = latent_value<T>(h, i);
+        float d;
+        if (tau > 0.f) {
+            const float th = tanhf(v / tau);
+            d = (1.f - th * th) / tau;
+        } else {
+            d = fabsf(v) <= 1.f ? 1.f : 0.f;
+        }
+        const float g = db[i] * d;
+        dh[i] = accumulate ? dh[i] + g : g;
+    }
+}
+
 int grid_for(int64_t work, int per_block)
 {
     int dev = 0, sms = 148;
@@ -151,6 +184,21 @@ cudaError_t launch_pack(const void *src, dbf_dtype dt, int64_t rows, int64_t k, 
         break;
     default:
         return cudaErrorInvalidValue;
+    }
+    return cudaGetLastError();
+}
+
+cudaError_t launch_ste(const float *db, const void *h, dbf_dtype hd, int64_t n, float tau, float *dh,
+                       int accumulate, cudaStream_t s)
+{
+    const int grid = grid_for(n, 256);
+    switch (hd) {
+    case DBF_F32: ste_kernel<float><<<grid, 256, 0, s>>>(db, static_cast<const float *>(h), n, tau, dh, accumulate); break;
+    case DBF_F16: ste_kernel<__half><<<grid, 256, 0, s>>>(db, static_cast<const __half *>(h), n, tau, dh, accumulate); break;
+    case DBF_BF16:
+        ste_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(db, static_cast<const __nv_bfloat16 *>(h), n, tau, dh, accumulate);
+        break;
+    default: return cudaErrorInvalidValue;
     }
     return cudaGetLastError();
 }

@@ -123,6 +123,19 @@ dbf_status dbf_unpack_signs(const uint32_t *src, int64_t rows, int64_t k, int8_t
 dbf_status dbf_transpose_signs(const uint32_t *src, int64_t rows, int64_t k, uint32_t *dst,
                                size_t dst_bytes, void *stream);
 
+/* Straight-through estimator for latent weights H whose signs form a sign
+ * matrix B = sign(H) (LoRDBA page, section 2, training pipeline: the signs
+ * are trained through an STE; the pages do not give its surrogate, so the
+ * caller picks it): dH = dB * s'(H), elementwise over count values, with
+ *   tau > 0:  s(H) = tanh(H / tau), s'(H) = (1 - tanh^2(H / tau)) / tau;
+ *   tau <= 0: s = identity clipped to |H| <= 1 (s' = 1 there, else 0).
+ * dB: device fp32 (e.g. db1 or db2 of dbf_backward); H: device fp32, fp16 or
+ * bf16, same shape; dH: device fp32, overwritten or added to with
+ * flags = DBF_ACCUMULATE. Errors: DBF_ERR_INVALID_ARG (also tau NaN),
+ * DBF_ERR_ALIGNMENT, DBF_ERR_CUDA. */
+dbf_status dbf_ste_backward(const float *db, const void *h, dbf_dtype h_dtype, int64_t count, float tau,
+                            float *dh, int flags, void *stream);
+
 /* Smallest T for which DBF_PATH_AUTO takes the GEMM path on a shape it allows. */
 int64_t dbf_gemm_min_tokens(void);
 
@@ -163,8 +176,8 @@ dbf_status dbf_forward(const dbf_layer *L, const void *x, dbf_dtype x_dtype, voi
                        size_t ws_bytes, void *stream);
 
 /* Workspace bytes dbf_backward needs (0 for invalid input or a shape the
- * backward does not serve). */
-size_t dbf_backward_workspace_bytes(const dbf_layer *L, int64_t T);
+ * backward does not serve); with_sign_grads != 0 when db1 or db2 is wanted. */
+size_t dbf_backward_workspace_bytes(const dbf_layer *L, int64_t T, int with_sign_grads);
 
 /* Gradients of a loss through dbf_forward, given dy = dL/dy (LoRDBA page,
  * section 2, training pipeline: quantisation-aware training differentiates
@@ -184,15 +197,21 @@ size_t dbf_backward_workspace_bytes(const dbf_layer *L, int64_t T);
  * x: T x M and dy: T x N, DBF_F32 or DBF_BF16, 16-byte aligned.
  * dx, dalpha, dbeta, dgamma: device fp32 outputs, each optional (NULL skips
  *    it; dalpha's GEMM and the dx/dgamma GEMM are skipped when not wanted).
- *    Overwritten, or added to with flags = DBF_ACCUMULATE.
+ * db1 (N x R), db2 (R x M): optional fp32 gradients with respect to the sign
+ *    matrices taken as real variables, dB1 = sum_{t,i} a_i v_i^T and
+ *    dB2 = sum_{t,i} (beta_i.g_i) u_i^T: what a straight-through estimator
+ *    passes to the latent weights (the estimator's own shape is the caller's;
+ *    see dbf_ste_backward). Dense fp16 x fp16 tensor-core products over the
+ *    tokens; they need a larger workspace (with_sign_grads).
+ *    Every output is overwritten, or added to with flags = DBF_ACCUMULATE.
  * ws: dbf_backward_workspace_bytes(L, T) bytes, 256-byte aligned, header as
  *    in dbf_forward.
  * Errors: DBF_ERR_INVALID_ARG, DBF_ERR_ALIGNMENT, DBF_ERR_WORKSPACE,
  *    DBF_ERR_UNSUPPORTED (shape), DBF_ERR_CUDA. */
 dbf_status dbf_backward(const dbf_layer *L, const uint32_t *b1t_packed, const uint32_t *b2t_packed,
                         const void *x, dbf_dtype x_dtype, const void *dy, dbf_dtype dy_dtype, int64_t T,
-                        float *dx, float *dalpha, float *dbeta, float *dgamma, int flags, void *ws,
-                        size_t ws_bytes, void *stream);
+                        float *dx, float *dalpha, float *dbeta, float *dgamma, float *db1, float *db2,
+                        int flags, void *ws, size_t ws_bytes, void *stream);
 
 /* Workspace bytes dbf_forward_segmented needs. */
 size_t dbf_segmented_workspace_bytes(int32_t max_R, int32_t max_ell, int64_t T);

@@ -174,6 +174,19 @@ def backward(layer, x: np.ndarray, dy: np.ndarray, want_signs: bool = False,
     return Grads(dx, dal, dbe, dga, db1, db2)
 
 
+def ste_backward(db: np.ndarray, h: np.ndarray, tau: float) -> np.ndarray:
+    """Straight-through estimator for latents h with signs B = sign(h) (LoRDBA
+    page, section 2, training pipeline; the surrogate is not given there):
+    dH = dB * s'(h) with s(h) = tanh(h / tau) for tau > 0, else the identity
+    clipped to |h| <= 1. fp64."""
+    h = np.asarray(h, dtype=np.float64)
+    db = np.asarray(db, dtype=np.float64)
+    if tau > 0:
+        th = np.tanh(h / tau)
+        return db * (1.0 - th * th) / tau
+    return db * (np.abs(h) <= 1.0)
+
+
 def forward_segmented(layers, seg_offsets, seg_adapter, x: np.ndarray,
                       y_in: Optional[np.ndarray] = None, accumulate: bool = False,
                       nthreads: Optional[int] = None) -> np.ndarray:

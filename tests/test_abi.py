@@ -140,20 +140,21 @@ def test_backward_rejects_bad_arguments_without_launch(lib):
     f = lib.dbf_backward
     p = 0x1000
     # flags other than ACCUMULATE, bad dtypes, null operands
-    assert f(by(L), p, p, p, dbf.F32, p, dbf.F32, 4, p, p, p, p, 2, p, 1 << 30, None) == dbf.ERR_INVALID_ARG
-    assert f(by(L), p, p, p, dbf.I8, p, dbf.F32, 4, p, p, p, p, 0, p, 1 << 30, None) == dbf.ERR_INVALID_ARG
-    assert f(by(L), None, p, p, dbf.F32, p, dbf.F32, 4, p, p, p, p, 0, p, 1 << 30, None) == dbf.ERR_INVALID_ARG
+    assert f(by(L), p, p, p, dbf.F32, p, dbf.F32, 4, p, p, p, p, None, None, 2, p, 1 << 30, None) == dbf.ERR_INVALID_ARG
+    assert f(by(L), p, p, p, dbf.I8, p, dbf.F32, 4, p, p, p, p, None, None, 0, p, 1 << 30, None) == dbf.ERR_INVALID_ARG
+    assert f(by(L), None, p, p, dbf.F32, p, dbf.F32, 4, p, p, p, p, None, None, 0, p, 1 << 30, None) == dbf.ERR_INVALID_ARG
     # shapes off the 128 grid are not served
     L2 = _layer(M=200, N=384, R=128)
-    assert f(by(L2), p, p, p, dbf.F32, p, dbf.F32, 4, p, p, p, p, 0, p, 1 << 30, None) == dbf.ERR_UNSUPPORTED
-    assert lib.dbf_backward_workspace_bytes(by(L2), 4) == 0
+    assert f(by(L2), p, p, p, dbf.F32, p, dbf.F32, 4, p, p, p, p, None, None, 0, p, 1 << 30, None) == dbf.ERR_UNSUPPORTED
+    assert lib.dbf_backward_workspace_bytes(by(L2), 4, 0) == 0
     # alignment and workspace
-    assert f(by(L), p, p, p + 4, dbf.F32, p, dbf.F32, 4, p, p, p, p, 0, p, 1 << 30, None) == dbf.ERR_ALIGNMENT
-    need = lib.dbf_backward_workspace_bytes(by(L), 4)
+    assert f(by(L), p, p, p + 4, dbf.F32, p, dbf.F32, 4, p, p, p, p, None, None, 0, p, 1 << 30, None) == dbf.ERR_ALIGNMENT
+    need = lib.dbf_backward_workspace_bytes(by(L), 4, 0)
+    assert lib.dbf_backward_workspace_bytes(by(L), 4, 1) > need
     assert need >= 256 + 2 * 4 * (256 + 384) * 2 + 2 * 4 * 128 * 8
-    assert f(by(L), p, p, p, dbf.F32, p, dbf.F32, 4, p, p, p, p, 0, p, need - 1, None) == dbf.ERR_WORKSPACE
+    assert f(by(L), p, p, p, dbf.F32, p, dbf.F32, 4, p, p, p, p, None, None, 0, p, need - 1, None) == dbf.ERR_WORKSPACE
     # T == 0 is a no-op
-    assert f(by(L), p, p, p, dbf.F32, p, dbf.F32, 0, p, p, p, p, 0, None, 0, None) == dbf.OK
+    assert f(by(L), p, p, p, dbf.F32, p, dbf.F32, 0, p, p, p, p, None, None, 0, None, 0, None) == dbf.OK
 
 
 def test_transpose_rejects_bad_arguments(lib):
@@ -162,3 +163,13 @@ def test_transpose_rejects_bad_arguments(lib):
     assert t(None, 4, 4, 0x1000, 1 << 20, None) == dbf.ERR_INVALID_ARG
     assert t(0x1000, 40, 64, 0x1000, lib.dbf_packed_bytes(64, 40) - 1, None) == dbf.ERR_INVALID_ARG
     assert t(0x1002, 40, 64, 0x1000, 1 << 20, None) == dbf.ERR_ALIGNMENT
+
+
+def test_ste_rejects_bad_arguments(lib):
+    import double_binary_rank_b200 as dbf
+    st = lib.dbf_ste_backward
+    assert st(0x1000, 0x1000, dbf.I8, 16, 1.0, 0x1000, 0, None) == dbf.ERR_INVALID_ARG
+    assert st(0x1000, 0x1000, dbf.F32, 16, float("nan"), 0x1000, 0, None) == dbf.ERR_INVALID_ARG
+    assert st(0x1000, 0x1000, dbf.F32, 16, 1.0, 0x1000, 4, None) == dbf.ERR_INVALID_ARG
+    assert st(0x1002, 0x1000, dbf.F32, 16, 1.0, 0x1000, 0, None) == dbf.ERR_ALIGNMENT
+    assert st(None, None, dbf.F32, 0, 1.0, None, 0, None) == dbf.OK

@@ -128,3 +128,43 @@ def test_dbf_mlp_full_size(dbf):
     scale = float(np.abs(y).max()) * np.sqrt(T * w.N)   # size of the terms of the sum
     for v in sums:
         assert abs(v - loss) <= TOL * scale, (v, loss)
+
+
+@pytest.mark.parametrize("case", [(256, 384, 128, 1, 37), (128, 256, 256, 2, 300), (384, 128, 128, 3, 5)],
+                         ids=lambda c: "M{}N{}R{}l{}T{}".format(*c))
+def test_sign_matrix_gradients(dbf, case):
+    M, N, R, ell, T = case
+    rng = np.random.default_rng(500 + M + N + R + ell + T)
+    L = random_layer(rng, M, N, R, ell)
+    x = S.to_bf16_bits(rng.standard_normal((T, M)))
+    dy = S.to_bf16_bits(rng.standard_normal((T, N)))
+    ref = oracle.backward(L, x, dy, want_signs=True)
+    _, g = gpu_grads(dbf, L, x, dy, want=("dx", "dbeta", "db1", "db2"))
+    assert g.dalpha is None and g.dgamma is None
+    assert rel_err(g.db1.cpu().numpy(), ref.db1) < TOL
+    assert rel_err(g.db2.cpu().numpy(), ref.db2) < TOL
+    assert rel_err(g.dx.cpu().numpy(), ref.dx) < TOL
+    # accumulate adds onto what is there
+    dl = dev_layer(L)
+    g2 = dbf.backward(dl, dev_x(x), dev_x(dy), grads=g, accumulate=True)
+    torch.cuda.synchronize()
+    assert rel_err(g2.db1.cpu().numpy(), 2 * ref.db1) < TOL
+    assert rel_err(g2.db2.cpu().numpy(), 2 * ref.db2) < TOL
+
+
+@pytest.mark.parametrize("tau", [0.0, 0.5, 2.0])
+@pytest.mark.parametrize("hdt", [torch.float32, torch.bfloat16, torch.float16])
+def test_ste_backward(dbf, tau, hdt):
+    rng = np.random.default_rng(int(tau * 10) + 3)
+    h = torch.from_numpy(rng.standard_normal((37, 129)).astype(np.float32) * 1.5).to(hdt)
+    db = torch.from_numpy(rng.standard_normal((37, 129)).astype(np.float32))
+    ref = oracle.ste_backward(db.numpy(), h.float().numpy(), tau)
+    got = dbf.ste_backward(db.cuda(), h.cuda(), tau)
+    torch.cuda.synchronize()
+    if tau > 0:
+        np.testing.assert_allclose(got.cpu().numpy(), ref, rtol=2e-6, atol=2e-6)
+    else:
+        np.testing.assert_array_equal(got.cpu().numpy(), ref.astype(np.float32))
+    acc = dbf.ste_backward(db.cuda(), h.cuda(), tau, dh=got.clone(), accumulate=True)
+    torch.cuda.synchronize()
+    np.testing.assert_allclose(acc.cpu().numpy(), 2 * got.cpu().numpy(), rtol=1e-6, atol=1e-7)

@@ -122,3 +122,20 @@ def test_thread_split_does_not_change_results():
     g4 = oracle.backward(L, x, dy, want_signs=True, nthreads=4)
     np.testing.assert_allclose(g4.dalpha, g1.dalpha, rtol=1e-13)
     np.testing.assert_array_equal(g4.dx, g1.dx)
+
+
+@pytest.mark.parametrize("tau", [0.25, 1.0, 3.0])
+def test_ste_surrogate_derivative_matches_the_surrogate(tau):
+    # the derivative the oracle uses against a central difference of tanh(h/tau)
+    h = np.linspace(-4, 4, 97)
+    eps = 1e-6
+    fd = (np.tanh((h + eps) / tau) - np.tanh((h - eps) / tau)) / (2 * eps)
+    np.testing.assert_allclose(oracle.ste_backward(np.ones_like(h), h, tau), fd, rtol=1e-7, atol=1e-9)
+    # slope 1/tau at zero, odd-symmetric surrogate -> even derivative
+    assert oracle.ste_backward(np.array([2.0]), np.array([0.0]), tau)[0] == pytest.approx(2.0 / tau)
+
+
+def test_ste_clipped_identity():
+    h = np.array([-1.5, -1.0, -0.3, 0.0, 0.999, 1.0, 1.0001, 7.0])
+    db = np.arange(1, 9, dtype=np.float64)
+    np.testing.assert_array_equal(oracle.ste_backward(db, h, 0.0), db * np.array([0, 1, 1, 1, 1, 1, 0, 0]))
