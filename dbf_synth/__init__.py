@@ -170,6 +170,26 @@ def make_x(seed: int, T: int, M: int, dtype: str, tag: int = TAG_X) -> np.ndarra
 
 
 @dataclasses.dataclass
+class MbokLayer:
+    """A multi-boolean-kernel layer, host side: K sign kernels w [K, N, M]
+    (int8 +-1) with fp16 bit patterns s_in [K, M] and s_out [K, N]."""
+    M: int
+    N: int
+    K: int
+    w: np.ndarray
+    s_in: np.ndarray
+    s_out: np.ndarray
+
+
+def make_mbok_layer(seed: int, M: int, N: int, K: int, sigma: float = 0.5) -> MbokLayer:
+    """Seeded MBOK layer: iid +-1 kernels, lognormal(0, sigma) fp16 scales."""
+    w = np.stack([signs(stream_key(seed, 0x31, k, 0), N, M) for k in range(K)])
+    s_in = np.stack([lognormal_f16_bits(stream_key(seed, 0x32, k, 0), M, sigma) for k in range(K)])
+    s_out = np.stack([lognormal_f16_bits(stream_key(seed, 0x33, k, 0), N, sigma) for k in range(K)])
+    return MbokLayer(M, N, K, w, s_in, s_out)
+
+
+@dataclasses.dataclass
 class Segments:
     """Tokens sorted by adapter id into contiguous segments."""
     offsets: np.ndarray   # int32 [S+1], offsets[0] = 0, offsets[S] = T

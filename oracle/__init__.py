@@ -60,6 +60,8 @@ def _load():
     lib.dbf_oracle_backward.argtypes = [i64, i64, i64, i64, vp, vp, vp, vp, vp, vp, i32, vp, i32, i64,
                                         vp, vp, vp, vp, vp, vp, i32]
     lib.dbf_oracle_backward.restype = i32
+    lib.dbf_oracle_mbok_forward.argtypes = [i64, i64, i64, vp, vp, vp, vp, i32, i64, vp]
+    lib.dbf_oracle_mbok_forward.restype = i32
     lib.dbf_oracle_pack.argtypes = [vp, i64, i64, vp]
     lib.dbf_oracle_unpack.argtypes = [vp, i64, i64, vp]
     lib.dbf_oracle_f16_to_f64.argtypes = [ctypes.c_uint16]
@@ -172,6 +174,27 @@ def backward(layer, x: np.ndarray, dy: np.ndarray, want_signs: bool = False,
     if rc != 0:
         raise ValueError("oracle rejected its arguments")
     return Grads(dx, dal, dbe, dga, db1, db2)
+
+
+def mbok_forward(layer, x: np.ndarray) -> np.ndarray:
+    """Multi-boolean-kernel layer forward (Multi-Boolean Architectures page,
+    section 2): y = sum_k s_out_k . (W_k (s_in_k . x)), fp64.
+
+    layer: object with M, N, K, w (int8 +-1 [K, N, M]), s_in (fp16 bits
+    [K, M]), s_out (fp16 bits [K, N]). x: T x M float32 or bf16 bits."""
+    lib = _load()
+    M, N, K = int(layer.M), int(layer.N), int(layer.K)
+    w = np.ascontiguousarray(layer.w, dtype=np.int8)
+    si = np.ascontiguousarray(layer.s_in, dtype=np.uint16).reshape(K, M)
+    so = np.ascontiguousarray(layer.s_out, dtype=np.uint16).reshape(K, N)
+    assert w.shape == (K, N, M)
+    xa, xk = _act(x)
+    T = xa.shape[0]
+    assert xa.shape == (T, M)
+    out = np.zeros((T, N))
+    if lib.dbf_oracle_mbok_forward(M, N, K, _ptr(w), _ptr(si), _ptr(so), _ptr(xa), xk, T, _ptr(out)) != 0:
+        raise ValueError("oracle rejected its arguments")
+    return out
 
 
 def ste_backward(db: np.ndarray, h: np.ndarray, tau: float) -> np.ndarray:

@@ -375,3 +375,38 @@ int dbf_oracle_backward(int64_t M, int64_t N, int64_t R, int64_t ell,
     free(th);
     return 0;
 }
+
+/* ---- multi-boolean-kernel layer (MBOK) --------------------------------- */
+/*
+ * Multi-Boolean Architectures page, section 2 ("Metodologia Proposta"):
+ * a weight matrix is approximated by a sum of K boolean kernels, each with
+ * an output and an input scale vector,
+ *     W ~ sum_{k=1..K} W_bool^[k] . (s_out^[k] s_in^[k]^T),
+ * so the layer's forward is
+ *     y[t,n] = sum_k s_out^[k][n] * sum_m W^[k][n,m] * s_in^[k][m] * x[t,m].
+ * w: int8 +-1 [K][N][M]; s_in: fp16 bits [K][M]; s_out: fp16 bits [K][N].
+ * Rows 0 .. T-1. Returns 0, or -1 on bad arguments.
+ */
+int dbf_oracle_mbok_forward(int64_t M, int64_t N, int64_t K, const int8_t *w, const uint16_t *s_in,
+                            const uint16_t *s_out, const void *x, int x_kind, int64_t T, double *y_out)
+{
+    if (M <= 0 || N <= 0 || K <= 0 || T < 0 || !w || !s_in || !s_out || !x || !y_out)
+        return -1;
+    double *u = (double *)malloc(sizeof(double) * (size_t)M);
+    for (int64_t t = 0; t < T; ++t) {
+        double *y = y_out + t * N;
+        for (int64_t n = 0; n < N; ++n) y[n] = 0.0;
+        for (int64_t k = 0; k < K; ++k) {
+            for (int64_t m = 0; m < M; ++m)
+                u[m] = dbf_oracle_f16_to_f64(s_in[k * M + m]) * load_act(x, x_kind, t * M + m);
+            for (int64_t n = 0; n < N; ++n) {
+                const int8_t *row = w + (k * N + n) * M;
+                double s = 0.0;
+                for (int64_t m = 0; m < M; ++m) s += (double)row[m] * u[m];
+                y[n] += dbf_oracle_f16_to_f64(s_out[k * N + n]) * s;
+            }
+        }
+    }
+    free(u);
+    return 0;
+}
