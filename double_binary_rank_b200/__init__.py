@@ -41,6 +41,11 @@ class DbfLayerC(ctypes.Structure):
                 ("beta", ctypes.c_void_p), ("gamma", ctypes.c_void_p)]
 
 
+class DbfMbokLayerC(ctypes.Structure):
+    _fields_ = [("M", ctypes.c_int32), ("N", ctypes.c_int32), ("K", ctypes.c_int32),
+                ("w_packed", ctypes.c_void_p), ("s_in", ctypes.c_void_p), ("s_out", ctypes.c_void_p)]
+
+
 _vp, _i64, _i32, _sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_size_t
 _LP = ctypes.POINTER(DbfLayerC)
 _SIGS = {
@@ -57,6 +62,9 @@ _SIGS = {
     "dbf_backward": (ctypes.c_int, [_LP, _vp, _vp, _vp, ctypes.c_int, _vp, ctypes.c_int, _i64, _vp, _vp, _vp,
                                     _vp, _vp, _vp, ctypes.c_int, _vp, _sz, _vp]),
     "dbf_ste_backward": (ctypes.c_int, [_vp, _vp, ctypes.c_int, _i64, ctypes.c_float, _vp, ctypes.c_int, _vp]),
+    "dbf_mbok_workspace_bytes": (_sz, [ctypes.POINTER(DbfMbokLayerC), _i64]),
+    "dbf_mbok_forward": (ctypes.c_int, [ctypes.POINTER(DbfMbokLayerC), _vp, ctypes.c_int, _vp, ctypes.c_int, _i64,
+                                        ctypes.c_int, _vp, _sz, _vp]),
     "dbf_segmented_workspace_bytes": (_sz, [_i32, _i32, _i64]),
     "dbf_forward_segmented": (ctypes.c_int, [_vp, _i32, _vp, _vp, _i32, _i32, _i32, _i32, _i32,
                                              _vp, ctypes.c_int, _vp, ctypes.c_int, _i64,
@@ -275,6 +283,50 @@ def ste_backward(db: torch.Tensor, h: torch.Tensor, tau: float = 0.0, dh: Option
     _check(_lib.dbf_ste_backward(_ptr(db), _ptr(h), _DT[h.dtype], h.numel(), float(tau), _ptr(dh),
                                  ACCUMULATE if accumulate else 0, _stream(stream)), "dbf_ste_backward")
     return dh
+
+
+@dataclass
+class MbokLayer:
+    """Device-resident multi-boolean-kernel layer: w [N, ceil(K M / 32)] packed
+    words (row n = the K kernels' rows side by side), fp16 s_in [K, M] and
+    s_out [K, N]."""
+    M: int
+    N: int
+    K: int
+    w: torch.Tensor
+    s_in: torch.Tensor
+    s_out: torch.Tensor
+
+    @staticmethod
+    def from_signs(w_signs: torch.Tensor, s_in: torch.Tensor, s_out: torch.Tensor, stream=None) -> "MbokLayer":
+        """w_signs: int8 +-1 [K, N, M] on the device; scales fp16."""
+        K, N, M = w_signs.shape
+        cat = w_signs.permute(1, 0, 2).reshape(N, K * M).contiguous()
+        return MbokLayer(M, N, K, pack_signs(cat, stream=stream), s_in.contiguous(), s_out.contiguous())
+
+    def descriptor(self) -> DbfMbokLayerC:
+        return DbfMbokLayerC(self.M, self.N, self.K, _ptr(self.w), _ptr(self.s_in), _ptr(self.s_out))
+
+
+def mbok_workspace_bytes(layer: MbokLayer, T: int) -> int:
+    d = layer.descriptor()
+    return int(_lib.dbf_mbok_workspace_bytes(ctypes.byref(d), T))
+
+
+def mbok_forward(layer: MbokLayer, x: torch.Tensor, y: Optional[torch.Tensor] = None, accumulate: bool = False,
+                 ws: Optional[torch.Tensor] = None, y_dtype: Optional[torch.dtype] = None,
+                 stream=None) -> torch.Tensor:
+    """y = [acc] y + sum_k s_out_k . (W_k (s_in_k . x)) (dbf_mbok_forward)."""
+    T = x.shape[0]
+    if y is None:
+        y = torch.empty((T, layer.N), dtype=y_dtype or x.dtype, device=x.device)
+    d = layer.descriptor()
+    if ws is None:
+        ws = alloc_workspace(mbok_workspace_bytes(layer, T), x.device)
+    _check(_lib.dbf_mbok_forward(ctypes.byref(d), _ptr(x), _DT[x.dtype], _ptr(y), _DT[y.dtype], T,
+                                 ACCUMULATE if accumulate else 0, _ptr(ws), ws.numel(), _stream(stream)),
+           "dbf_mbok_forward")
+    return y
 
 
 def forward_decode_noalloc(layer: Layer, x: torch.Tensor, y: Optional[torch.Tensor] = None,

@@ -164,6 +164,30 @@ dbf_status dbf_backward(const dbf_layer *L, const uint32_t *b1t_packed, const ui
                                    dgamma, db1, db2, flags, ws, static_cast<cudaStream_t>(stream)));
 }
 
+size_t dbf_mbok_workspace_bytes(const dbf_mbok_layer *L, int64_t T)
+{
+    if (!L || T < 0 || !mbok_shape_ok(L->M, L->N, L->K)) return 0;
+    return mbok_workspace_bytes(L->M, L->K, T);
+}
+
+dbf_status dbf_mbok_forward(const dbf_mbok_layer *L, const void *x, dbf_dtype x_dtype, void *y, dbf_dtype y_dtype,
+                            int64_t T, int flags, void *ws, size_t ws_bytes, void *stream)
+{
+    if (!L || L->M <= 0 || L->N <= 0 || L->K < 1 || T < 0 || !act_dtype_ok(x_dtype) || !act_dtype_ok(y_dtype))
+        return DBF_ERR_INVALID_ARG;
+    if (flags & ~DBF_ACCUMULATE) return DBF_ERR_INVALID_ARG;
+    if (!mbok_shape_ok(L->M, L->N, L->K)) return DBF_ERR_UNSUPPORTED;
+    if (T == 0) return DBF_OK;
+    if (!L->w_packed || !L->s_in || !L->s_out || !x || !y) return DBF_ERR_INVALID_ARG;
+    if (!aligned(L->w_packed, 16) || !aligned(L->s_in, 2) || !aligned(L->s_out, 2) || !aligned(x, 16) ||
+        !aligned(y, 16))
+        return DBF_ERR_ALIGNMENT;
+    if (!ws || ws_bytes < mbok_workspace_bytes(L->M, L->K, T)) return DBF_ERR_WORKSPACE;
+    if (!aligned(ws, 256)) return DBF_ERR_ALIGNMENT;
+    return from_cuda(mbok_forward(L->M, L->N, L->K, L->w_packed, L->s_in, L->s_out, x, x_dtype, y, y_dtype, T,
+                                  flags, ws, static_cast<cudaStream_t>(stream)));
+}
+
 size_t dbf_segmented_workspace_bytes(int32_t max_R, int32_t max_ell, int64_t T)
 {
     if (max_R <= 0 || max_ell < 1 || max_ell > kMaxEll || T < 0) return 0;

@@ -94,6 +94,8 @@ struct GemmArgs {
     float *dx;                // stage 6 (optional): [T][P] receives sum_i gamma_i[p] acc
     int dx_mode;              // 0 store, 1 add, 2 atomic add
     int dense_a;              // A is a dense fp16 [P][Ktot] matrix loaded by TMA (tmA), not packed signs
+    int env_advance;          // K blocks of Kp columns read successive blocks of the sign row (one sign
+                              // matrix per block, multi-kernel layers) instead of the same row again
 };
 
 // ---- small PTX helpers --------------------------------------------------------
@@ -418,7 +420,7 @@ __global__ void __launch_bounds__(Cfg::kThreads, 1) gemm_kernel(const __grid_con
         const int env_words = g.Kp / 32;           // packed words of one envelope block of K
         const uint32_t swz = static_cast<uint32_t>(prow & 7) << 4;
         // cursor over this CTA's (tile, pair) sequence, advanced without divisions
-        int cj = 0, cpair = 0, cword = 0, cenv = 0, cgrow = 0;
+        int cj = 0, cpair = 0, cword = 0, cenv = 0, cgrow = 0, cbase = 0;   // cbase: first word of the envelope block
         const uint32_t *crow = nullptr;
         bool cvalid = false;
         uint32_t cmag = 0u;
@@ -442,12 +444,14 @@ __global__ void __launch_bounds__(Cfg::kThreads, 1) gemm_kernel(const __grid_con
                 cpair = 0;
                 cword = 0;
                 cenv = 0;
+                cbase = 0;
                 if (++cj < my_tiles) seat_tile();
             } else {
                 cword += 4;
                 if (cword == env_words) {
                     cword = 0;
                     ++cenv;
+                    cbase += g.env_advance ? env_words : 0;   // a new block of the row, or the same row again
                     seat_mag();
                 }
             }
@@ -456,7 +460,7 @@ __global__ void __launch_bounds__(Cfg::kThreads, 1) gemm_kernel(const __grid_con
         // magnitude pattern of its envelope block; then move on to the group's
         // next pair
         auto fetch = [&](uint4 &w, uint32_t &mag) {
-            w = cvalid ? __ldg(reinterpret_cast<const uint4 *>(crow + cword)) : make_uint4(0u, 0u, 0u, 0u);
+            w = cvalid ? __ldg(reinterpret_cast<const uint4 *>(crow + cbase + cword)) : make_uint4(0u, 0u, 0u, 0u);
             mag = cmag;
 #pragma unroll
             for (int e = 0; e < kExpandGroups; ++e) advance();
@@ -627,8 +631,10 @@ __global__ void __launch_bounds__(256) transpose_f16_kernel(const uint16_t *__re
 
 // u[(i T + t), m] = fp16(gamma_i[m] x[t, m]); eight columns per thread with
 // 16-byte loads and stores when M % 8 == 0 and gamma is 16-byte aligned.
+// tok_major: output row t ell + i (U is [T][ell M], blocks of one token side
+// by side) instead of i T + t.
 __global__ void __launch_bounds__(256) scale_cast_kernel(const void *x, dbf_dtype xd, const uint16_t *gamma, int M,
-                                                         int T, int ell, __half *U, int vec8)
+                                                         int T, int ell, __half *U, int vec8, int tok_major)
 {
     const int64_t total = static_cast<int64_t>(ell) * T * M;
     if (vec8) {
@@ -638,8 +644,8 @@ __global__ void __launch_bounds__(256) scale_cast_kernel(const void *x, dbf_dtyp
              idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
             const int64_t row = idx / M8;
             const int m8 = static_cast<int>(idx - row * M8);
-            const int i = static_cast<int>(row / T);
-            const int64_t t = row - static_cast<int64_t>(i) * T;
+            const int i = tok_major ? static_cast<int>(row % ell) : static_cast<int>(row / T);
+            const int64_t t = tok_major ? row / ell : row - static_cast<int64_t>(i) * T;
             const uint4 gw = __ldg(reinterpret_cast<const uint4 *>(gamma + static_cast<int64_t>(i) * M) + m8);
             float xv[8];
             if (xd == DBF_BF16) {
@@ -666,8 +672,8 @@ __global__ void __launch_bounds__(256) scale_cast_kernel(const void *x, dbf_dtyp
          idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
         const int64_t row = idx / M;
         const int m = static_cast<int>(idx - row * M);
-        const int i = static_cast<int>(row / T);
-        const int64_t t = row - static_cast<int64_t>(i) * T;
+        const int i = tok_major ? static_cast<int>(row % ell) : static_cast<int>(row / T);
+        const int64_t t = tok_major ? row / ell : row - static_cast<int64_t>(i) * T;
         U[idx] = __float2half_rn(h2f(gamma[static_cast<int64_t>(i) * M + m]) * load_act(x, xd, t * M + m));
     }
 }
@@ -751,7 +757,7 @@ cudaError_t gemm_forward(const dbf_layer &L, const void *x, dbf_dtype xd, void *
         int64_t blocks = (total + 255) / 256;
         if (blocks > 148 * 32) blocks = 148 * 32;
         const int vec8 = (L.M % 8 == 0) && ((reinterpret_cast<uintptr_t>(L.gamma) & 15u) == 0);
-        scale_cast_kernel<<<static_cast<int>(blocks), 256, 0, s>>>(x, xd, L.gamma, L.M, Ti, L.ell, U, vec8);
+        scale_cast_kernel<<<static_cast<int>(blocks), 256, 0, s>>>(x, xd, L.gamma, L.M, Ti, L.ell, U, vec8, 0);
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
@@ -801,13 +807,14 @@ namespace dbf {
 namespace {
 
 cudaError_t scale_cast(const void *x, dbf_dtype xd, const uint16_t *scale, int K, int64_t T, int ell, __half *out,
-                       cudaStream_t s)
+                       cudaStream_t s, int tok_major = 0)
 {
     const int64_t total = static_cast<int64_t>(ell) * T * K;
     int64_t blocks = (total + 255) / 256;
     if (blocks > 148 * 32) blocks = 148 * 32;
     const int vec8 = (K % 8 == 0) && ((reinterpret_cast<uintptr_t>(scale) & 15u) == 0);
-    scale_cast_kernel<<<static_cast<int>(blocks), 256, 0, s>>>(x, xd, scale, K, static_cast<int>(T), ell, out, vec8);
+    scale_cast_kernel<<<static_cast<int>(blocks), 256, 0, s>>>(x, xd, scale, K, static_cast<int>(T), ell, out, vec8,
+                                                               tok_major);
     return cudaGetLastError();
 }
 
@@ -984,6 +991,52 @@ cudaError_t gemm_backward(const dbf_layer &L, const uint32_t *b1t, const uint32_
         }
     }
     return cudaSuccess;
+}
+
+}  // namespace dbf
+
+// ---- multi-boolean-kernel layer (MBOK) on the same GEMM -------------------------
+// Multi-Boolean Architectures page, section 2: y = sum_k s_out_k . (W_k (s_in_k . x)).
+// One GEMM with K blocks of M contraction columns: the A operand of block k
+// is s_out_k[n] * W_k[n, :] (the packed row of W holds the K kernels' rows
+// side by side, so the cursor moves on to the next block instead of reading
+// the same row again), the B operand is u[t][k M + m] = fp16(s_in_k[m] x[t, m]).
+namespace dbf {
+
+bool mbok_shape_ok(int64_t M, int64_t N, int64_t K) { return M > 0 && N > 0 && K >= 1 && K <= 64 && M % 128 == 0; }
+
+size_t mbok_workspace_bytes(int64_t M, int64_t K, int64_t T)
+{
+    return kWsHeaderBytes + align_up(static_cast<size_t>(T) * K * M * 2, 256);
+}
+
+cudaError_t mbok_forward(int M, int N, int K, const uint32_t *w_packed, const uint16_t *s_in, const uint16_t *s_out,
+                         const void *x, dbf_dtype xd, void *y, dbf_dtype yd, int64_t T, int flags, void *ws,
+                         cudaStream_t s)
+{
+    if (T > (1 << 30) / K) return cudaErrorInvalidValue;
+    __half *U = reinterpret_cast<__half *>(static_cast<char *>(ws) + kWsHeaderBytes);
+    cudaError_t e = scale_cast(x, xd, s_in, M, T, K, U, s, 1);
+    if (e != cudaSuccess) return e;
+    CUtensorMap mu;
+    if (!make_map(&mu, U, static_cast<int64_t>(K) * M, T)) return cudaErrorInvalidValue;
+    GemmArgs a = {};
+    a.signs = w_packed;
+    a.pitch = static_cast<int>(pitch_words(static_cast<int64_t>(K) * M));
+    a.P = N;
+    a.Kp = M;
+    a.Ktot = K * M;
+    a.arow_scale = s_out;
+    a.env_advance = 1;
+    a.C = static_cast<int>(T);
+    a.T = static_cast<int>(T);
+    a.ell = K;
+    a.stage = 2;
+    a.y = y;
+    a.yd = yd;
+    a.N = N;
+    a.accumulate = (flags & DBF_ACCUMULATE) ? 1 : 0;
+    return launch_gemm<FwdCfg>(mu, a, s);
 }
 
 }  // namespace dbf

@@ -41,6 +41,13 @@ cudaError_t gemv_forward_segmented(const dbf_layer *adapters, int32_t num_adapte
                                    const void *x, dbf_dtype xd, void *y, dbf_dtype yd, int64_t T,
                                    int flags, void *ws, int32_t *status, cudaStream_t s);
 
+// multi-boolean-kernel layer (tcgen05 GEMM for any T)
+bool mbok_shape_ok(int64_t M, int64_t N, int64_t K);
+size_t mbok_workspace_bytes(int64_t M, int64_t K, int64_t T);
+cudaError_t mbok_forward(int M, int N, int K, const uint32_t *w_packed, const uint16_t *s_in,
+                         const uint16_t *s_out, const void *x, dbf_dtype xd, void *y, dbf_dtype yd,
+                         int64_t T, int flags, void *ws, cudaStream_t s);
+
 // prefill path (tcgen05)
 bool gemm_shape_ok(const dbf_layer &L);
 size_t gemm_workspace_bytes(const dbf_layer &L, int64_t T);

@@ -213,6 +213,35 @@ dbf_status dbf_backward(const dbf_layer *L, const uint32_t *b1t_packed, const ui
                         float *dx, float *dalpha, float *dbeta, float *dgamma, float *db1, float *db2,
                         int flags, void *ws, size_t ws_bytes, void *stream);
 
+/* Multi-boolean-kernel layer (Multi-Boolean Architectures page, section 2):
+ * W ~ sum_{k=1..K} W_bool^[k] . (s_out^[k] s_in^[k]^T), K boolean kernels
+ * with per-kernel input and output scales; a single-stage sign contraction
+ * (no rank-R intermediate), served by the same tensor-core GEMM. */
+typedef struct {
+    int32_t M, N, K;             /* in, out, number of boolean kernels (1 .. 64) */
+    const uint32_t *w_packed;    /* N x (K M) signs packed along the K M columns: row n holds
+                                    W^[1][n, :], ..., W^[K][n, :] side by side (bit set = -1) */
+    const uint16_t *s_in;        /* fp16 [K][M] */
+    const uint16_t *s_out;       /* fp16 [K][N] */
+} dbf_mbok_layer;
+
+/* Workspace bytes dbf_mbok_forward needs (0 for invalid input or a shape it
+ * does not serve). */
+size_t dbf_mbok_workspace_bytes(const dbf_mbok_layer *L, int64_t T);
+
+/* y = [acc] y + sum_k s_out^[k] . (W^[k] (s_in^[k] . x)) for T tokens.
+ * L: host descriptor of device arrays (w_packed 16-byte aligned; pack the
+ *    N x (K M) int8 sign matrix with dbf_pack_signs). Needs M % 128 == 0.
+ * x: T x M, y: T x N, DBF_F32 or DBF_BF16, 16-byte aligned; flags:
+ *    DBF_ACCUMULATE or 0. Numerics: s_in . x rounded to fp16 operands,
+ *    exact +-s_out fp16 sign operands, fp32 accumulation.
+ * ws: dbf_mbok_workspace_bytes bytes, 256-byte aligned, header as in
+ *    dbf_forward. Errors: DBF_ERR_INVALID_ARG, DBF_ERR_UNSUPPORTED,
+ *    DBF_ERR_ALIGNMENT, DBF_ERR_WORKSPACE, DBF_ERR_CUDA. */
+dbf_status dbf_mbok_forward(const dbf_mbok_layer *L, const void *x, dbf_dtype x_dtype, void *y,
+                            dbf_dtype y_dtype, int64_t T, int flags, void *ws, size_t ws_bytes,
+                            void *stream);
+
 /* Workspace bytes dbf_forward_segmented needs. */
 size_t dbf_segmented_workspace_bytes(int32_t max_R, int32_t max_ell, int64_t T);
 

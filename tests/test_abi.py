@@ -173,3 +173,20 @@ def test_ste_rejects_bad_arguments(lib):
     assert st(0x1000, 0x1000, dbf.F32, 16, 1.0, 0x1000, 4, None) == dbf.ERR_INVALID_ARG
     assert st(0x1002, 0x1000, dbf.F32, 16, 1.0, 0x1000, 0, None) == dbf.ERR_ALIGNMENT
     assert st(None, None, dbf.F32, 0, 1.0, None, 0, None) == dbf.OK
+
+
+def test_mbok_rejects_bad_arguments(lib):
+    import double_binary_rank_b200 as dbf
+    by = ctypes.byref
+    p = 0x1000
+    L = dbf.DbfMbokLayerC(256, 100, 3, p, p, p)
+    f = lib.dbf_mbok_forward
+    need = lib.dbf_mbok_workspace_bytes(by(L), 8)
+    assert need >= 256 + 8 * 3 * 256 * 2
+    assert f(by(L), p, dbf.F32, p, dbf.F32, 8, 2, p, need, None) == dbf.ERR_INVALID_ARG
+    assert f(by(L), p, dbf.I8, p, dbf.F32, 8, 0, p, need, None) == dbf.ERR_INVALID_ARG
+    assert f(by(dbf.DbfMbokLayerC(200, 100, 3, p, p, p)), p, dbf.F32, p, dbf.F32, 8, 0, p, need, None) == dbf.ERR_UNSUPPORTED
+    assert lib.dbf_mbok_workspace_bytes(by(dbf.DbfMbokLayerC(200, 100, 3, p, p, p)), 8) == 0
+    assert f(by(L), p + 8, dbf.F32, p, dbf.F32, 8, 0, p, need, None) == dbf.ERR_ALIGNMENT
+    assert f(by(L), p, dbf.F32, p, dbf.F32, 8, 0, p, need - 1, None) == dbf.ERR_WORKSPACE
+    assert f(by(L), None, dbf.F32, None, dbf.F32, 0, 0, None, 0, None) == dbf.OK
