@@ -356,6 +356,28 @@ def main():
     torch.cuda.synchronize(dev)
     bwd_us = max_over_ranks(1e3 * b0.elapsed_time(b1) / n_bwd, dev)
 
+    # ---- multi-boolean-kernel layer (4096 -> 4096, K = 3 kernels) on the
+    # prefill batch, timed separately
+    mb = S.make_mbok_layer(0xDBF00006, w.M, w.M, 3)
+    f16t = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.float16)).to(dev)
+    mlayer = dbf.MbokLayer.from_signs(torch.from_numpy(mb.w).to(dev), f16t(mb.s_in), f16t(mb.s_out))
+    y_mb = torch.empty((T_PREFILL, mb.N), dtype=torch.bfloat16, device=dev)
+    ws_mb = dbf.alloc_workspace(dbf.mbok_workspace_bytes(mlayer, T_PREFILL), dev)
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            dbf.mbok_forward(mlayer, x_pre, y=y_mb, ws=ws_mb, stream=stream)
+    torch.cuda.synchronize(dev)
+    m0, m1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    n_mb = 10
+    with torch.cuda.stream(stream):
+        m0.record(stream)
+        for _ in range(n_mb):
+            dbf.mbok_forward(mlayer, x_pre, y=y_mb, ws=ws_mb, stream=stream)
+        m1.record(stream)
+    torch.cuda.synchronize(dev)
+    mb_us = max_over_ranks(1e3 * m0.elapsed_time(m1) / n_mb, dev)
+    mb_flops = 2 * T_PREFILL * mb.K * mb.M * mb.N
+
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
@@ -390,6 +412,9 @@ def main():
         "backward": {"kernel": "gradients dx, dalpha, dbeta, dgamma of the T=2048 prefill batch (two pre-passes + four tcgen05 sign GEMMs), one call",
                      "us_per_call": bwd_us, "achieved": 2 * f_pre / (bwd_us * 1e-6) / 1e12, "unit": "TFLOP/s",
                      "peak": pk["bf16_tflops"], "frac": 2 * f_pre / (bwd_us * 1e-6) / 1e12 / pk["bf16_tflops"]},
+        "mbok": {"kernel": "multi-boolean-kernel layer 4096 -> 4096, K=3, T=2048 (fp16 pre-pass + one tcgen05 sign GEMM), one call",
+                 "us_per_call": mb_us, "achieved": mb_flops / (mb_us * 1e-6) / 1e12, "unit": "TFLOP/s",
+                 "peak": pk["bf16_tflops"], "frac": mb_flops / (mb_us * 1e-6) / 1e12 / pk["bf16_tflops"]},
         "clocks": clk.summary(),
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": args.steps * (dec_launches + pre_launches),
