@@ -378,6 +378,33 @@ def main():
     mb_us = max_over_ranks(1e3 * m0.elapsed_time(m1) / n_mb, dev)
     mb_flops = 2 * T_PREFILL * mb.K * mb.M * mb.N
 
+    # ---- segmented prefill planned on the host: 32 adapters (4096 -> 4096,
+    # R = 128, two envelopes), 256 tokens each, one forward per segment
+    n_ad, per = 32, 256
+    seg_layers = []
+    for a in range(n_ad):
+        La = S.make_layer(0xDBF00007, w.M, w.M, 128, 2, 0.5, adapter=a)
+        seg_layers.append(dbf.Layer.from_signs(torch.from_numpy(La.b1).to(dev), torch.from_numpy(La.b2).to(dev),
+                                               f16t(La.alpha), f16t(La.beta), f16t(La.gamma)))
+    seg_offs = np.arange(0, (n_ad + 1) * per, per, dtype=np.int32)
+    seg_ids = np.arange(n_ad, dtype=np.int32)
+    x_seg = torch.randn((n_ad * per, w.M), device=dev).to(torch.bfloat16)
+    y_seg = torch.empty((n_ad * per, w.M), dtype=torch.bfloat16, device=dev)
+    with torch.cuda.stream(stream):
+        dbf.forward_segmented_planned(seg_layers, seg_offs, seg_ids, x_seg, y=y_seg, stream=stream)
+        ws_seg = dbf.alloc_workspace(dbf.workspace_bytes(seg_layers[0], per), dev)
+        dbf.forward_segmented_planned(seg_layers, seg_offs, seg_ids, x_seg, y=y_seg, ws=ws_seg, stream=stream)
+    torch.cuda.synchronize(dev)
+    g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        g0.record(stream)
+        for _ in range(5):
+            dbf.forward_segmented_planned(seg_layers, seg_offs, seg_ids, x_seg, y=y_seg, ws=ws_seg, stream=stream)
+        g1.record(stream)
+    torch.cuda.synchronize(dev)
+    seg_us = max_over_ranks(1e3 * g0.elapsed_time(g1) / 5, dev)
+    seg_flops = 2 * n_ad * per * 2 * 128 * (w.M + w.M)
+
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
@@ -415,6 +442,10 @@ def main():
         "mbok": {"kernel": "multi-boolean-kernel layer 4096 -> 4096, K=3, T=2048 (fp16 pre-pass + one tcgen05 sign GEMM), one call",
                  "us_per_call": mb_us, "achieved": mb_flops / (mb_us * 1e-6) / 1e12, "unit": "TFLOP/s",
                  "peak": pk["bf16_tflops"], "frac": mb_flops / (mb_us * 1e-6) / 1e12 / pk["bf16_tflops"]},
+        "segmented_prefill": {"kernel": "32 adapters 4096 -> 4096 (R=128, 2 envelopes) x 256 tokens, host-planned, one forward per segment",
+                              "us_per_call": seg_us, "tokens_per_s": n_ad * per / (seg_us * 1e-6),
+                              "achieved": seg_flops / (seg_us * 1e-6) / 1e12, "unit": "TFLOP/s", "peak": pk["bf16_tflops"],
+                              "frac": seg_flops / (seg_us * 1e-6) / 1e12 / pk["bf16_tflops"]},
         "clocks": clk.summary(),
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": args.steps * (dec_launches + pre_launches),

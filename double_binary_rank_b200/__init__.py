@@ -13,6 +13,7 @@ import os
 from dataclasses import dataclass
 from typing import List, Optional, Sequence
 
+import numpy as np
 import torch
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -62,6 +63,9 @@ _SIGS = {
     "dbf_backward": (ctypes.c_int, [_LP, _vp, _vp, _vp, ctypes.c_int, _vp, ctypes.c_int, _i64, _vp, _vp, _vp,
                                     _vp, _vp, _vp, ctypes.c_int, _vp, _sz, _vp]),
     "dbf_ste_backward": (ctypes.c_int, [_vp, _vp, ctypes.c_int, _i64, ctypes.c_float, _vp, ctypes.c_int, _vp]),
+    "dbf_forward_segmented_planned_workspace_bytes": (_sz, [_LP, _i32, _vp, _vp, _i32, _i32, _i32, _i64]),
+    "dbf_forward_segmented_planned": (ctypes.c_int, [_LP, _i32, _vp, _vp, _i32, _i32, _i32, _vp, ctypes.c_int, _vp,
+                                                     ctypes.c_int, _i64, ctypes.c_int, _vp, _sz, _vp]),
     "dbf_mbok_workspace_bytes": (_sz, [ctypes.POINTER(DbfMbokLayerC), _i64]),
     "dbf_mbok_forward": (ctypes.c_int, [ctypes.POINTER(DbfMbokLayerC), _vp, ctypes.c_int, _vp, ctypes.c_int, _i64,
                                         ctypes.c_int, _vp, _sz, _vp]),
@@ -283,6 +287,35 @@ def ste_backward(db: torch.Tensor, h: torch.Tensor, tau: float = 0.0, dh: Option
     _check(_lib.dbf_ste_backward(_ptr(db), _ptr(h), _DT[h.dtype], h.numel(), float(tau), _ptr(dh),
                                  ACCUMULATE if accumulate else 0, _stream(stream)), "dbf_ste_backward")
     return dh
+
+
+def forward_segmented_planned(layers, seg_offsets, seg_adapter, x: torch.Tensor, y: Optional[torch.Tensor] = None,
+                              accumulate: bool = False, ws: Optional[torch.Tensor] = None,
+                              y_dtype: Optional[torch.dtype] = None, static_weights: bool = False,
+                              stream=None) -> torch.Tensor:
+    """Segmented forward with the segment tables on the host
+    (dbf_forward_segmented_planned): one dbf_forward per segment, each on the
+    path its token count calls for.
+
+    layers: list of Layer; seg_offsets: S+1 ints; seg_adapter: S ints (-1 = none)."""
+    T = x.shape[0]
+    N = layers[0].N if layers else (y.shape[1] if y is not None else 0)
+    M = x.shape[1]
+    if y is None:
+        y = torch.empty((T, N), dtype=y_dtype or x.dtype, device=x.device)
+    arr = (DbfLayerC * max(1, len(layers)))(*[l.descriptor() for l in layers])
+    offs = np.ascontiguousarray(seg_offsets, dtype=np.int32)
+    ids = np.ascontiguousarray(seg_adapter, dtype=np.int32)
+    S = int(ids.size)
+    if ws is None:
+        need = int(_lib.dbf_forward_segmented_planned_workspace_bytes(arr, len(layers), offs.ctypes.data,
+                                                                      ids.ctypes.data, S, M, N, T))
+        ws = alloc_workspace(need, x.device)
+    _check(_lib.dbf_forward_segmented_planned(arr, len(layers), offs.ctypes.data, ids.ctypes.data, S, M, N, _ptr(x),
+                                              _DT[x.dtype], _ptr(y), _DT[y.dtype], T,
+                                              _flags(accumulate, static_weights), _ptr(ws), ws.numel(),
+                                              _stream(stream)), "dbf_forward_segmented_planned")
+    return y
 
 
 @dataclass

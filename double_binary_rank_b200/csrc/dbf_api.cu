@@ -164,6 +164,79 @@ dbf_status dbf_backward(const dbf_layer *L, const uint32_t *b1t_packed, const ui
                                    dgamma, db1, db2, flags, ws, static_cast<cudaStream_t>(stream)));
 }
 
+// Host-planned segmented forward: validation shared by the size query and the call.
+static dbf_status check_plan(const dbf_layer *adapters, int32_t num_adapters, const int32_t *offs,
+                             const int32_t *ids, int32_t S, int32_t M, int32_t N, int64_t T)
+{
+    if (num_adapters < 0 || S < 0 || M <= 0 || N <= 0 || T < 0) return DBF_ERR_INVALID_ARG;
+    if (S == 0) return DBF_OK;
+    if (!offs || !ids || (num_adapters > 0 && !adapters)) return DBF_ERR_INVALID_ARG;
+    if (offs[0] < 0 || offs[S] > T) return DBF_ERR_INVALID_ARG;
+    for (int32_t q = 0; q < S; ++q) {
+        if (offs[q + 1] < offs[q] || ids[q] < -1 || ids[q] >= num_adapters) return DBF_ERR_INVALID_ARG;
+        if (ids[q] >= 0) {
+            const dbf_status st = check_layer(&adapters[ids[q]]);
+            if (st != DBF_OK) return st;
+            if (adapters[ids[q]].M != M || adapters[ids[q]].N != N) return DBF_ERR_INVALID_ARG;
+        }
+    }
+    return DBF_OK;
+}
+
+size_t dbf_forward_segmented_planned_workspace_bytes(const dbf_layer *adapters_host, int32_t num_adapters,
+                                                     const int32_t *seg_offsets_host,
+                                                     const int32_t *seg_adapter_host, int32_t S, int32_t M,
+                                                     int32_t N, int64_t T)
+{
+    if (check_plan(adapters_host, num_adapters, seg_offsets_host, seg_adapter_host, S, M, N, T) != DBF_OK) return 0;
+    size_t need = kWsHeaderBytes;
+    for (int32_t q = 0; q < S; ++q) {
+        const int64_t n = static_cast<int64_t>(seg_offsets_host[q + 1]) - seg_offsets_host[q];
+        if (seg_adapter_host[q] < 0 || n <= 0) continue;
+        const size_t b = dbf_workspace_bytes(&adapters_host[seg_adapter_host[q]], n, DBF_PATH_AUTO);
+        if (b > need) need = b;
+    }
+    return need;
+}
+
+dbf_status dbf_forward_segmented_planned(const dbf_layer *adapters_host, int32_t num_adapters,
+                                         const int32_t *seg_offsets_host, const int32_t *seg_adapter_host,
+                                         int32_t S, int32_t M, int32_t N, const void *x, dbf_dtype x_dtype,
+                                         void *y, dbf_dtype y_dtype, int64_t T, int flags, void *ws,
+                                         size_t ws_bytes, void *stream)
+{
+    dbf_status st = check_plan(adapters_host, num_adapters, seg_offsets_host, seg_adapter_host, S, M, N, T);
+    if (st != DBF_OK) return st;
+    if (!act_dtype_ok(x_dtype) || !act_dtype_ok(y_dtype) || (flags & ~(DBF_ACCUMULATE | DBF_WEIGHTS_STATIC)))
+        return DBF_ERR_INVALID_ARG;
+    if (T == 0 || S == 0) return DBF_OK;
+    if (!x || !y) return DBF_ERR_INVALID_ARG;
+    const size_t xe = x_dtype == DBF_F32 ? 4 : 2, ye = y_dtype == DBF_F32 ? 4 : 2;
+    // every segment's rows must start on a 16-byte boundary
+    if (!aligned(x, 16) || !aligned(y, 16) || (static_cast<size_t>(M) * xe) % 16 || (static_cast<size_t>(N) * ye) % 16)
+        return DBF_ERR_ALIGNMENT;
+    const size_t need = dbf_forward_segmented_planned_workspace_bytes(adapters_host, num_adapters, seg_offsets_host,
+                                                                      seg_adapter_host, S, M, N, T);
+    if (!ws || ws_bytes < need) return DBF_ERR_WORKSPACE;
+    if (!aligned(ws, 256)) return DBF_ERR_ALIGNMENT;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    for (int32_t q = 0; q < S; ++q) {
+        const int64_t off = seg_offsets_host[q], n = static_cast<int64_t>(seg_offsets_host[q + 1]) - off;
+        if (n <= 0) continue;
+        char *yq = static_cast<char *>(y) + off * N * ye;
+        if (seg_adapter_host[q] < 0) {
+            // no adapter: a zero branch
+            if (!(flags & DBF_ACCUMULATE) && cudaMemsetAsync(yq, 0, static_cast<size_t>(n) * N * ye, s) != cudaSuccess)
+                return DBF_ERR_CUDA;
+            continue;
+        }
+        st = dbf_forward(&adapters_host[seg_adapter_host[q]], static_cast<const char *>(x) + off * M * xe, x_dtype, yq,
+                         y_dtype, n, flags, DBF_PATH_AUTO, ws, ws_bytes, stream);
+        if (st != DBF_OK) return st;
+    }
+    return DBF_OK;
+}
+
 size_t dbf_mbok_workspace_bytes(const dbf_mbok_layer *L, int64_t T)
 {
     if (!L || T < 0 || !mbok_shape_ok(L->M, L->N, L->K)) return 0;

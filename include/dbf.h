@@ -213,6 +213,36 @@ dbf_status dbf_backward(const dbf_layer *L, const uint32_t *b1t_packed, const ui
                         float *dx, float *dalpha, float *dbeta, float *dgamma, float *db1, float *db2,
                         int flags, void *ws, size_t ws_bytes, void *stream);
 
+/* Segmented serving planned on the host (LoRDBA page, section 1: many
+ * adapters served at once): the same routing as dbf_forward_segmented, but
+ * the segment tables and adapter descriptors are HOST arrays, as a serving
+ * scheduler that built the batch has them. Each segment then runs as its
+ * own dbf_forward on its token rows with the path AUTO picks for its length
+ * (the tensor-core GEMM for segments of dbf_gemm_min_tokens() tokens or more
+ * on shapes it serves, the decode kernels otherwise), all on one stream and
+ * one workspace; segments with adapter id -1 get a zero branch. Suited to
+ * prefill batches with many tokens per adapter.
+ * adapters_host: host array of num_adapters descriptors (device pointers
+ *    inside), each with the given M and N. seg_offsets_host: host int32
+ *    [S+1], nondecreasing within [0, T]; seg_adapter_host: host int32 [S],
+ *    each in [-1, num_adapters). x, y, flags as in dbf_forward; every
+ *    segment's rows must be 16-byte aligned (M and N times the element size
+ *    multiples of 16 bytes, else DBF_ERR_ALIGNMENT).
+ * ws: dbf_forward_segmented_planned_workspace_bytes bytes (the largest
+ *    segment's), 256-byte aligned, header as in dbf_forward.
+ * Errors: DBF_ERR_INVALID_ARG (bad tables or descriptors, checked on the
+ *    host before any launch), DBF_ERR_ALIGNMENT, DBF_ERR_WORKSPACE,
+ *    DBF_ERR_CUDA. */
+size_t dbf_forward_segmented_planned_workspace_bytes(const dbf_layer *adapters_host, int32_t num_adapters,
+                                                     const int32_t *seg_offsets_host,
+                                                     const int32_t *seg_adapter_host, int32_t S, int32_t M,
+                                                     int32_t N, int64_t T);
+dbf_status dbf_forward_segmented_planned(const dbf_layer *adapters_host, int32_t num_adapters,
+                                         const int32_t *seg_offsets_host, const int32_t *seg_adapter_host,
+                                         int32_t S, int32_t M, int32_t N, const void *x, dbf_dtype x_dtype,
+                                         void *y, dbf_dtype y_dtype, int64_t T, int flags, void *ws,
+                                         size_t ws_bytes, void *stream);
+
 /* Multi-boolean-kernel layer (Multi-Boolean Architectures page, section 2):
  * W ~ sum_{k=1..K} W_bool^[k] . (s_out^[k] s_in^[k]^T), K boolean kernels
  * with per-kernel input and output scales; a single-stage sign contraction

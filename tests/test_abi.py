@@ -190,3 +190,29 @@ def test_mbok_rejects_bad_arguments(lib):
     assert f(by(L), p + 8, dbf.F32, p, dbf.F32, 8, 0, p, need, None) == dbf.ERR_ALIGNMENT
     assert f(by(L), p, dbf.F32, p, dbf.F32, 8, 0, p, need - 1, None) == dbf.ERR_WORKSPACE
     assert f(by(L), None, dbf.F32, None, dbf.F32, 0, 0, None, 0, None) == dbf.OK
+
+
+def test_segmented_planned_rejects_bad_tables(lib):
+    import numpy as np
+    import double_binary_rank_b200 as dbf
+    arr = (dbf.DbfLayerC * 2)(_layer(M=64, N=48, R=32), _layer(M=64, N=48, R=128))
+    f = lib.dbf_forward_segmented_planned
+    q = lib.dbf_forward_segmented_planned_workspace_bytes
+    offs = np.array([0, 5, 9], dtype=np.int32)
+    ok_ids = np.array([0, 1], dtype=np.int32)
+    need = q(arr, 2, offs.ctypes.data, ok_ids.ctypes.data, 2, 64, 48, 9)
+    assert need >= 256
+    for bad_offs, bad_ids in (([0, 5, 10], [0, 1]), ([0, 6, 5], [0, 1]), ([0, 5, 9], [0, 2]), ([0, 5, 9], [-2, 0])):
+        o = np.array(bad_offs, dtype=np.int32)
+        i = np.array(bad_ids, dtype=np.int32)
+        assert q(arr, 2, o.ctypes.data, i.ctypes.data, 2, 64, 48, 9) == 0
+        assert f(arr, 2, o.ctypes.data, i.ctypes.data, 2, 64, 48, 0x1000, dbf.F32, 0x1000, dbf.F32, 9, 0,
+                 0x1000, 1 << 30, None) == dbf.ERR_INVALID_ARG
+    # a descriptor whose N differs from the call's
+    assert f(arr, 2, offs.ctypes.data, ok_ids.ctypes.data, 2, 64, 40, 0x1000, dbf.F32, 0x1000, dbf.F32, 9, 0,
+             0x1000, 1 << 30, None) == dbf.ERR_INVALID_ARG
+    # rows of a segment must stay 16-byte aligned: M = 60 bf16 rows are 120 bytes
+    arr2 = (dbf.DbfLayerC * 1)(_layer(M=60, N=48, R=32))
+    z = np.array([0], dtype=np.int32)
+    assert f(arr2, 1, np.array([0, 4], dtype=np.int32).ctypes.data, z.ctypes.data, 1, 60, 48, 0x1000, dbf.BF16,
+             0x1000, dbf.F32, 4, 0, 0x1000, 1 << 30, None) == dbf.ERR_ALIGNMENT
