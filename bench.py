@@ -392,7 +392,8 @@ def main():
     y_seg = torch.empty((n_ad * per, w.M), dtype=torch.bfloat16, device=dev)
     with torch.cuda.stream(stream):
         dbf.forward_segmented_planned(seg_layers, seg_offs, seg_ids, x_seg, y=y_seg, stream=stream)
-        ws_seg = dbf.alloc_workspace(dbf.workspace_bytes(seg_layers[0], per), dev)
+        ws_seg = dbf.alloc_workspace(dbf.segmented_planned_workspace_bytes(seg_layers, seg_offs, seg_ids, w.M, w.M,
+                                                                           n_ad * per), dev)
         dbf.forward_segmented_planned(seg_layers, seg_offs, seg_ids, x_seg, y=y_seg, ws=ws_seg, stream=stream)
     torch.cuda.synchronize(dev)
     g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -442,7 +443,7 @@ def main():
         "mbok": {"kernel": "multi-boolean-kernel layer 4096 -> 4096, K=3, T=2048 (fp16 pre-pass + one tcgen05 sign GEMM), one call",
                  "us_per_call": mb_us, "achieved": mb_flops / (mb_us * 1e-6) / 1e12, "unit": "TFLOP/s",
                  "peak": pk["bf16_tflops"], "frac": mb_flops / (mb_us * 1e-6) / 1e12 / pk["bf16_tflops"]},
-        "segmented_prefill": {"kernel": "32 adapters 4096 -> 4096 (R=128, 2 envelopes) x 256 tokens, host-planned, one forward per segment",
+        "segmented_prefill": {"kernel": "32 adapters 4096 -> 4096 (R=128, 2 envelopes) x 256 tokens, host-planned: one grouped pre-pass + two grouped tcgen05 GEMM launches",
                               "us_per_call": seg_us, "tokens_per_s": n_ad * per / (seg_us * 1e-6),
                               "achieved": seg_flops / (seg_us * 1e-6) / 1e12, "unit": "TFLOP/s", "peak": pk["bf16_tflops"],
                               "frac": seg_flops / (seg_us * 1e-6) / 1e12 / pk["bf16_tflops"]},

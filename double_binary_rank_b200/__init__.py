@@ -289,6 +289,14 @@ def ste_backward(db: torch.Tensor, h: torch.Tensor, tau: float = 0.0, dh: Option
     return dh
 
 
+def segmented_planned_workspace_bytes(layers, seg_offsets, seg_adapter, M: int, N: int, T: int) -> int:
+    arr = (DbfLayerC * max(1, len(layers)))(*[l.descriptor() for l in layers])
+    offs = np.ascontiguousarray(seg_offsets, dtype=np.int32)
+    ids = np.ascontiguousarray(seg_adapter, dtype=np.int32)
+    return int(_lib.dbf_forward_segmented_planned_workspace_bytes(arr, len(layers), offs.ctypes.data, ids.ctypes.data,
+                                                                  int(ids.size), M, N, T))
+
+
 def forward_segmented_planned(layers, seg_offsets, seg_adapter, x: torch.Tensor, y: Optional[torch.Tensor] = None,
                               accumulate: bool = False, ws: Optional[torch.Tensor] = None,
                               y_dtype: Optional[torch.dtype] = None, static_weights: bool = False,

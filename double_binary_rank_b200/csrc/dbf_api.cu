@@ -2,6 +2,8 @@
 // (no launch on a failed check), path choice and the workspace contract.
 #include "dbf_internal.cuh"
 
+#include <vector>
+
 namespace {
 
 using namespace dbf;
@@ -183,6 +185,10 @@ static dbf_status check_plan(const dbf_layer *adapters, int32_t num_adapters, co
     return DBF_OK;
 }
 
+// Segments served by a grouped GEMM launch: an adapter on a shape the GEMM
+// serves; they are grouped by (R, ell).
+static bool grouped_ok(const dbf_layer &L) { return gemm_shape_ok(L); }
+
 size_t dbf_forward_segmented_planned_workspace_bytes(const dbf_layer *adapters_host, int32_t num_adapters,
                                                      const int32_t *seg_offsets_host,
                                                      const int32_t *seg_adapter_host, int32_t S, int32_t M,
@@ -193,7 +199,9 @@ size_t dbf_forward_segmented_planned_workspace_bytes(const dbf_layer *adapters_h
     for (int32_t q = 0; q < S; ++q) {
         const int64_t n = static_cast<int64_t>(seg_offsets_host[q + 1]) - seg_offsets_host[q];
         if (seg_adapter_host[q] < 0 || n <= 0) continue;
-        const size_t b = dbf_workspace_bytes(&adapters_host[seg_adapter_host[q]], n, DBF_PATH_AUTO);
+        const dbf_layer &L = adapters_host[seg_adapter_host[q]];
+        // grouped: the pre-pass and v buffers span all T token rows
+        const size_t b = grouped_ok(L) ? gemm_workspace_bytes(L, T) : dbf_workspace_bytes(&L, n, DBF_PATH_AUTO);
         if (b > need) need = b;
     }
     return need;
@@ -220,9 +228,41 @@ dbf_status dbf_forward_segmented_planned(const dbf_layer *adapters_host, int32_t
     if (!ws || ws_bytes < need) return DBF_ERR_WORKSPACE;
     if (!aligned(ws, 256)) return DBF_ERR_ALIGNMENT;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
+    // adapters the GEMM serves: one grouped launch per (R, ell) class, up to
+    // kMaxGroupsPerLaunch segments each
+    std::vector<char> done(static_cast<size_t>(S), 0);
+    for (int32_t q0 = 0; q0 < S; ++q0) {
+        const int32_t a0 = seg_adapter_host[q0];
+        if (done[q0] || a0 < 0 || seg_offsets_host[q0 + 1] <= seg_offsets_host[q0] || !grouped_ok(adapters_host[a0]))
+            continue;
+        const int R0 = adapters_host[a0].R, ell0 = adapters_host[a0].ell;
+        std::vector<const dbf_layer *> ls;
+        std::vector<int> offs, ns;
+        for (int32_t q = q0; q < S; ++q) {
+            const int32_t a = seg_adapter_host[q];
+            if (done[q] || a < 0 || seg_offsets_host[q + 1] <= seg_offsets_host[q]) continue;
+            const dbf_layer &L = adapters_host[a];
+            if (!grouped_ok(L) || L.R != R0 || L.ell != ell0) continue;
+            done[q] = 1;
+            ls.push_back(&L);
+            offs.push_back(seg_offsets_host[q]);
+            ns.push_back(seg_offsets_host[q + 1] - seg_offsets_host[q]);
+            if (static_cast<int>(ls.size()) == kMaxGroupsPerLaunch) {
+                if (gemm_forward_grouped(ls.data(), offs.data(), ns.data(), static_cast<int>(ls.size()), x, x_dtype,
+                                         y, y_dtype, T, flags, ws, s) != cudaSuccess)
+                    return DBF_ERR_CUDA;
+                ls.clear();
+                offs.clear();
+                ns.clear();
+            }
+        }
+        if (!ls.empty() && gemm_forward_grouped(ls.data(), offs.data(), ns.data(), static_cast<int>(ls.size()), x,
+                                                x_dtype, y, y_dtype, T, flags, ws, s) != cudaSuccess)
+            return DBF_ERR_CUDA;
+    }
     for (int32_t q = 0; q < S; ++q) {
         const int64_t off = seg_offsets_host[q], n = static_cast<int64_t>(seg_offsets_host[q + 1]) - off;
-        if (n <= 0) continue;
+        if (n <= 0 || done[q]) continue;
         char *yq = static_cast<char *>(y) + off * N * ye;
         if (seg_adapter_host[q] < 0) {
             // no adapter: a zero branch

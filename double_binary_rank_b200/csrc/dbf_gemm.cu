@@ -64,6 +64,18 @@ constexpr int B_BYTES = BN * BK * 2;   // 32 KB
 constexpr int TMEM_COLS = 512;          // two 256-column accumulators
 constexpr unsigned long long kWaitNs = 1000000000ull;   // bounded waits: 1 s
 
+// One adapter's share of a grouped launch (segmented serving): its sign rows,
+// scales and token rows; tiles tile0 .. of the launch belong to it.
+constexpr int kMaxGroups = 48;
+struct GroupRef {
+    const uint32_t *signs;      // stage 1: B2, stage 2: B1 of this adapter
+    const uint16_t *arow;       // stage 2: alpha [ell][N]
+    const uint16_t *beta;       // stage 1: beta [ell][R]
+    int off, n;                 // token rows off .. off + n - 1
+    int tile0;                  // first tile of the group
+    int ncpe;                   // token tiles per envelope: ceil(n / BN)
+};
+
 struct GemmArgs {
     // A operand: packed sign rows
     const uint32_t *signs;
@@ -96,7 +108,44 @@ struct GemmArgs {
     int dense_a;              // A is a dense fp16 [P][Ktot] matrix loaded by TMA (tmA), not packed signs
     int env_advance;          // K blocks of Kp columns read successive blocks of the sign row (one sign
                               // matrix per block, multi-kernel layers) instead of the same row again
+    // grouped launch (stages 1 and 2): ngroups adapters of one shape, tiles_total tiles
+    int ngroups, tiles_total;
+    GroupRef grp[kMaxGroups];
 };
+
+// Where tile 'tile' of the launch reads and writes: its sign-row block p0,
+// its first B row, its token range [t0, t1) and envelope (grouped stage 1
+// tiles stay inside one envelope), and its group (null when not grouped).
+struct TileRef {
+    int p0, brow, t0, t1, env;
+    const GroupRef *gr;
+};
+
+__device__ __forceinline__ TileRef tile_ref(const GemmArgs &g, int tile, int n_p)
+{
+    TileRef r;
+    if (g.ngroups == 0) {
+        r.p0 = (tile % n_p) * BM;
+        r.brow = (tile / n_p) * BN;
+        r.t0 = r.brow;
+        r.t1 = g.C;
+        r.env = 0;
+        r.gr = nullptr;
+        return r;
+    }
+    int gi = 0;
+    while (gi + 1 < g.ngroups && tile >= g.grp[gi + 1].tile0) ++gi;
+    const GroupRef &G = g.grp[gi];
+    const int local = tile - G.tile0;
+    const int c = local / n_p;
+    r.p0 = (local - c * n_p) * BM;
+    r.env = g.stage == 1 ? c / G.ncpe : 0;
+    r.t0 = G.off + (c - r.env * G.ncpe) * BN;
+    r.t1 = G.off + G.n;
+    r.brow = g.stage == 1 ? r.env * g.T + r.t0 : r.t0;
+    r.gr = &G;
+    return r;
+}
 
 // ---- small PTX helpers --------------------------------------------------------
 __device__ __forceinline__ uint32_t smem_u32(const void *p)
@@ -236,6 +285,47 @@ __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volati
     return __shfl_sync(0xffffffffu, ok, 0);
 }
 
+// Epilogue of a grouped tile, 32 columns = tokens t0 .. t0 + 31 (those below
+// the group's end): stage 1 writes v = fp16(beta h) of envelope tr.env,
+// stage 2 writes y.
+__device__ __forceinline__ void grouped_chunk(const GemmArgs &g, const TileRef &tr, const uint32_t (&v)[32], int t0,
+                                              int p)
+{
+    const int n_ok = tr.t1 - t0;
+    if (g.stage == 1) {
+        const float b = h2f(tr.gr->beta[static_cast<int64_t>(tr.env) * g.R + p]);
+        const int64_t ts = static_cast<int64_t>(g.ell) * g.R;
+        __half *vp = g.V + static_cast<int64_t>(t0) * ts + static_cast<int64_t>(tr.env) * g.R + p;
+#pragma unroll
+        for (int e = 0; e < 32; ++e)
+            if (e < n_ok) vp[e * ts] = __float2half_rn(b * __uint_as_float(v[e]));
+    } else if (g.yd == DBF_BF16) {
+        __nv_bfloat16 *yp = static_cast<__nv_bfloat16 *>(g.y) + static_cast<int64_t>(t0) * g.N + p;
+#pragma unroll
+        for (int e0 = 0; e0 < 32; e0 += 8) {
+            float yin[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+                yin[e] = g.accumulate ? __bfloat162float(yp[static_cast<int64_t>(e0 + e < n_ok ? e0 + e : 0) * g.N]) : 0.f;
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+                if (e0 + e < n_ok) yp[static_cast<int64_t>(e0 + e) * g.N] = __float2bfloat16_rn(__uint_as_float(v[e0 + e]) + yin[e]);
+        }
+    } else {
+        float *yp = static_cast<float *>(g.y) + static_cast<int64_t>(t0) * g.N + p;
+#pragma unroll
+        for (int e0 = 0; e0 < 32; e0 += 8) {
+            float yin[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+                yin[e] = g.accumulate ? yp[static_cast<int64_t>(e0 + e < n_ok ? e0 + e : 0) * g.N] : 0.f;
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+                if (e0 + e < n_ok) yp[static_cast<int64_t>(e0 + e) * g.N] = __uint_as_float(v[e0 + e]) + yin[e];
+        }
+    }
+}
+
 __device__ __forceinline__ float load_w(const void *w, dbf_dtype wd, int64_t i)
 {
     return wd == DBF_BF16 ? __bfloat162float(static_cast<const __nv_bfloat16 *>(w)[i])
@@ -307,7 +397,7 @@ __device__ __forceinline__ void backward_chunk(const GemmArgs &g, const uint32_t
 // the CTAs running together share activation tiles in L2).
 template <class Cfg>
 __global__ void __launch_bounds__(Cfg::kThreads, 1) gemm_kernel(const __grid_constant__ CUtensorMap tmB,
-                                                                const __grid_constant__ CUtensorMap tmA, const GemmArgs g)
+                                                                const __grid_constant__ CUtensorMap tmA, const __grid_constant__ GemmArgs g)
 {
     constexpr int SA = Cfg::SA, SB = Cfg::SB, kExpandGroups = Cfg::kExpandGroups;
     constexpr int kExpandWarps = Cfg::kExpandWarps, kEpiWarps = Cfg::kEpiWarps;
@@ -325,7 +415,7 @@ __global__ void __launch_bounds__(Cfg::kThreads, 1) gemm_kernel(const __grid_con
     const int lane = threadIdx.x & 31;
     const int n_p = (g.P + BM - 1) / BM;
     const int n_c = (g.C + BN - 1) / BN;
-    const int ntiles = n_p * n_c;
+    const int ntiles = g.ngroups ? g.tiles_total : n_p * n_c;
     const int my_tiles = blockIdx.x < ntiles ? (ntiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
     const int nk = g.Ktot / BK;
 
@@ -362,9 +452,9 @@ __global__ void __launch_bounds__(Cfg::kThreads, 1) gemm_kernel(const __grid_con
         if (lane == 0) {
             int s = 0;
             for (int j = 0; j < my_tiles && !*abort; ++j) {
-                const int tile = blockIdx.x + j * gridDim.x;
-                const int c0 = (tile / n_p) * BN;
-                const int p0 = (tile % n_p) * BM;
+                const TileRef tr = tile_ref(g, blockIdx.x + j * gridDim.x, n_p);
+                const int c0 = tr.brow;
+                const int p0 = tr.p0;
                 for (int k = 0; k < nk; ++k, ++s) {
                     const int st = s % SB;
                     if (!bar_wait(&sh->empty_b[st], ((s / SB) & 1) ^ 1, abort)) break;
@@ -424,19 +514,21 @@ __global__ void __launch_bounds__(Cfg::kThreads, 1) gemm_kernel(const __grid_con
         const uint32_t *crow = nullptr;
         bool cvalid = false;
         uint32_t cmag = 0u;
+        const uint16_t *carow = g.arow_scale;
         auto seat_mag = [&]() {
-            if (g.arow_scale) {
-                const uint32_t a = cvalid ? __ldg(g.arow_scale + static_cast<int64_t>(cenv) * g.N + cgrow) : 0u;
+            if (carow) {
+                const uint32_t a = cvalid ? __ldg(carow + static_cast<int64_t>(cenv) * g.N + cgrow) : 0u;
                 cmag = a | (a << 16);
             } else {
                 cmag = cvalid ? 0x3C003C00u : 0u;   // +-1
             }
         };
         auto seat_tile = [&]() {
-            const int tile = blockIdx.x + cj * gridDim.x;
-            cgrow = (tile % n_p) * BM + prow;
+            const TileRef tr = tile_ref(g, blockIdx.x + cj * gridDim.x, n_p);
+            cgrow = tr.p0 + prow;
             cvalid = cgrow < g.P;
-            crow = g.signs + static_cast<int64_t>(cvalid ? cgrow : 0) * g.pitch;
+            carow = tr.gr ? tr.gr->arow : g.arow_scale;
+            crow = (tr.gr ? tr.gr->signs : g.signs) + static_cast<int64_t>(cvalid ? cgrow : 0) * g.pitch;
             seat_mag();
         };
         auto advance = [&]() {
@@ -531,8 +623,8 @@ __global__ void __launch_bounds__(Cfg::kThreads, 1) gemm_kernel(const __grid_con
             const int ab = j & 1;
             if (!warp_wait(&sh->acc_full[ab], (j >> 1) & 1, abort)) break;
             tc_fence_after();
-            const int tile = blockIdx.x + j * gridDim.x;
-            const int p0 = (tile % n_p) * BM, c0 = (tile / n_p) * BN;
+            const TileRef tr = tile_ref(g, blockIdx.x + j * gridDim.x, n_p);
+            const int p0 = tr.p0, c0 = tr.brow;
             const int grow = p0 + q * 32 + lane;
             const uint32_t taddr = tmem + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(ab * BN);
             const bool row_ok = grow < g.P;
@@ -540,6 +632,10 @@ __global__ void __launch_bounds__(Cfg::kThreads, 1) gemm_kernel(const __grid_con
                 uint32_t v[32];
                 tmem_ld32(taddr + cc, v);   // every lane takes part (.sync.aligned)
                 if (!row_ok) continue;
+                if (tr.gr) {
+                    grouped_chunk(g, tr, v, tr.t0 + cc, grow);
+                    continue;
+                }
                 const int cb = c0 + cc;
                 if (g.stage == 1) {
                     // column c = i T + t; v[t, i R + r] = fp16(beta_i[r] h); (i, t)
@@ -678,6 +774,59 @@ __global__ void __launch_bounds__(256) scale_cast_kernel(const void *x, dbf_dtyp
     }
 }
 
+// Grouped pre-pass: u[(i T + t), m] = fp16(gamma_{a(t), i}[m] x[t, m]) where
+// a(t) is the group holding token t; rows of tokens outside every group are
+// not written (no tile reads them into a stored column).
+struct GammaGroups {
+    int ngroups;
+    int off[kMaxGroups], n[kMaxGroups];
+    const uint16_t *gamma[kMaxGroups];
+};
+
+__global__ void __launch_bounds__(256) scale_cast_grouped_kernel(const void *x, dbf_dtype xd,
+                                                                 const __grid_constant__ GammaGroups gg, int M, int T,
+                                                                 int ell, __half *U, int vec8)
+{
+    // one row (i T + t) per block step: the group is found once per row
+    for (int64_t row = blockIdx.x; row < static_cast<int64_t>(ell) * T; row += gridDim.x) {
+        const int i = static_cast<int>(row / T);
+        const int t = static_cast<int>(row - static_cast<int64_t>(i) * T);
+        int gi = -1;
+        for (int q = 0; q < gg.ngroups; ++q)
+            if (t >= gg.off[q] && t < gg.off[q] + gg.n[q]) gi = q;
+        if (gi < 0) continue;
+        const uint16_t *gp = gg.gamma[gi] + static_cast<int64_t>(i) * M;
+        __half *up = U + row * M;
+        if (vec8 && (reinterpret_cast<uintptr_t>(gp) & 15u) == 0) {
+            for (int m8 = threadIdx.x; m8 < M / 8; m8 += blockDim.x) {
+                const uint4 gw = __ldg(reinterpret_cast<const uint4 *>(gp) + m8);
+                float xv[8];
+                if (xd == DBF_BF16) {
+                    const uint4 xw = __ldg(reinterpret_cast<const uint4 *>(static_cast<const __nv_bfloat16 *>(x) +
+                                                                           static_cast<int64_t>(t) * M) + m8);
+                    const __nv_bfloat16 *xb = reinterpret_cast<const __nv_bfloat16 *>(&xw);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) xv[e] = __bfloat162float(xb[e]);
+                } else {
+                    const float4 *xf = reinterpret_cast<const float4 *>(static_cast<const float *>(x) + static_cast<int64_t>(t) * M) + 2 * m8;
+                    const float4 c0 = __ldg(xf), c1 = __ldg(xf + 1);
+                    xv[0] = c0.x; xv[1] = c0.y; xv[2] = c0.z; xv[3] = c0.w;
+                    xv[4] = c1.x; xv[5] = c1.y; xv[6] = c1.z; xv[7] = c1.w;
+                }
+                const __half *gh = reinterpret_cast<const __half *>(&gw);
+                uint4 out;
+                __half *oh = reinterpret_cast<__half *>(&out);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) oh[e] = __float2half_rn(__half2float(gh[e]) * xv[e]);
+                reinterpret_cast<uint4 *>(up)[m8] = out;
+            }
+        } else {
+            for (int m = threadIdx.x; m < M; m += blockDim.x)
+                up[m] = __float2half_rn(h2f(gp[m]) * load_act(x, xd, static_cast<int64_t>(t) * M + m));
+        }
+    }
+}
+
 // ---- host side ----------------------------------------------------------------
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn()
 {
@@ -727,7 +876,7 @@ cudaError_t launch_gemm(const CUtensorMap &map, const GemmArgs &a, cudaStream_t 
         cudaGetDevice(&dev);
         sms = (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && v > 0) ? v : 148;
     }
-    const int tiles = ((a.P + BM - 1) / BM) * ((a.C + BN - 1) / BN);
+    const int tiles = a.ngroups ? a.tiles_total : ((a.P + BM - 1) / BM) * ((a.C + BN - 1) / BN);
     gemm_kernel<Cfg><<<tiles < sms ? tiles : sms, Cfg::kThreads, gemm_smem<Cfg>(), s>>>(map, map_a ? *map_a : map, a);
     return cudaGetLastError();
 }
@@ -1037,6 +1186,86 @@ cudaError_t mbok_forward(int M, int N, int K, const uint32_t *w_packed, const ui
     a.N = N;
     a.accumulate = (flags & DBF_ACCUMULATE) ? 1 : 0;
     return launch_gemm<FwdCfg>(mu, a, s);
+}
+
+}  // namespace dbf
+
+// ---- grouped forward (segmented serving of adapters of one shape) ----------------
+namespace dbf {
+
+// Adapters 'layers[k]' (same M, N, R, ell; GEMM-eligible) on token rows
+// [off[k], off[k] + n[k]) of x / y, count <= kMaxGroups: one pre-pass and two
+// grouped GEMM launches, tiles of all groups side by side in each launch.
+cudaError_t gemm_forward_grouped(const dbf_layer *const *layers, const int *off, const int *n, int count,
+                                 const void *x, dbf_dtype xd, void *y, dbf_dtype yd, int64_t T, int flags, void *ws,
+                                 cudaStream_t s)
+{
+    if (count < 1 || count > kMaxGroups) return cudaErrorInvalidValue;
+    const dbf_layer &L = *layers[0];
+    if (T > (1 << 30) / L.ell) return cudaErrorInvalidValue;
+    char *body = static_cast<char *>(ws) + kWsHeaderBytes;
+    __half *U = reinterpret_cast<__half *>(body);
+    __half *V = reinterpret_cast<__half *>(body + u_bytes(L, T));
+    const int Ti = static_cast<int>(T);
+    GammaGroups gg = {};
+    gg.ngroups = count;
+    for (int k = 0; k < count; ++k) {
+        gg.off[k] = off[k];
+        gg.n[k] = n[k];
+        gg.gamma[k] = layers[k]->gamma;
+    }
+    {
+        int64_t blocks = static_cast<int64_t>(L.ell) * T;
+        if (blocks > 148 * 16) blocks = 148 * 16;
+        scale_cast_grouped_kernel<<<static_cast<int>(blocks), 256, 0, s>>>(x, xd, gg, L.M, Ti, L.ell, U, L.M % 8 == 0);
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    CUtensorMap mu, mv;
+    if (!make_map(&mu, U, L.M, static_cast<int64_t>(L.ell) * T)) return cudaErrorInvalidValue;
+    if (!make_map(&mv, V, static_cast<int64_t>(L.ell) * L.R, T)) return cudaErrorInvalidValue;
+    // stage 1: per group ell x ceil(n / BN) token tiles, each inside one envelope
+    GemmArgs a1 = {};
+    a1.pitch = static_cast<int>(pitch_words(L.M));
+    a1.P = L.R;
+    a1.Kp = L.M;
+    a1.Ktot = L.M;
+    a1.C = L.ell * Ti;
+    a1.stage = 1;
+    a1.V = V;
+    a1.T = Ti;
+    a1.ell = L.ell;
+    a1.R = L.R;
+    a1.N = L.N;
+    GemmArgs a2 = {};
+    a2.pitch = static_cast<int>(pitch_words(L.R));
+    a2.P = L.N;
+    a2.Kp = L.R;
+    a2.Ktot = L.ell * L.R;
+    a2.C = Ti;
+    a2.stage = 2;
+    a2.T = Ti;
+    a2.ell = L.ell;
+    a2.R = L.R;
+    a2.y = y;
+    a2.yd = yd;
+    a2.N = L.N;
+    a2.accumulate = (flags & DBF_ACCUMULATE) ? 1 : 0;
+    const int np1 = (L.R + BM - 1) / BM, np2 = (L.N + BM - 1) / BM;
+    int t1 = 0, t2 = 0;
+    for (int k = 0; k < count; ++k) {
+        const int ncpe = (n[k] + BN - 1) / BN;
+        a1.grp[k] = GroupRef{layers[k]->b2_packed, nullptr, layers[k]->beta, off[k], n[k], t1, ncpe};
+        a2.grp[k] = GroupRef{layers[k]->b1_packed, layers[k]->alpha, nullptr, off[k], n[k], t2, ncpe};
+        t1 += np1 * L.ell * ncpe;
+        t2 += np2 * ncpe;
+    }
+    a1.ngroups = a2.ngroups = count;
+    a1.tiles_total = t1;
+    a2.tiles_total = t2;
+    cudaError_t e = launch_gemm<FwdCfg>(mu, a1, s);
+    if (e != cudaSuccess) return e;
+    return launch_gemm<FwdCfg>(mv, a2, s);
 }
 
 }  // namespace dbf

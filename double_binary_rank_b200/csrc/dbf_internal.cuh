@@ -41,6 +41,12 @@ cudaError_t gemv_forward_segmented(const dbf_layer *adapters, int32_t num_adapte
                                    const void *x, dbf_dtype xd, void *y, dbf_dtype yd, int64_t T,
                                    int flags, void *ws, int32_t *status, cudaStream_t s);
 
+// grouped prefill of adapters of one shape (segmented serving)
+constexpr int kMaxGroupsPerLaunch = 48;
+cudaError_t gemm_forward_grouped(const dbf_layer *const *layers, const int *off, const int *n, int count,
+                                 const void *x, dbf_dtype xd, void *y, dbf_dtype yd, int64_t T, int flags,
+                                 void *ws, cudaStream_t s);
+
 // multi-boolean-kernel layer (tcgen05 GEMM for any T)
 bool mbok_shape_ok(int64_t M, int64_t N, int64_t K);
 size_t mbok_workspace_bytes(int64_t M, int64_t K, int64_t T);

@@ -216,20 +216,20 @@ dbf_status dbf_backward(const dbf_layer *L, const uint32_t *b1t_packed, const ui
 /* Segmented serving planned on the host (LoRDBA page, section 1: many
  * adapters served at once): the same routing as dbf_forward_segmented, but
  * the segment tables and adapter descriptors are HOST arrays, as a serving
- * scheduler that built the batch has them. Each segment then runs as its
- * own dbf_forward on its token rows with the path AUTO picks for its length
- * (the tensor-core GEMM for segments of dbf_gemm_min_tokens() tokens or more
- * on shapes it serves, the decode kernels otherwise), all on one stream and
- * one workspace; segments with adapter id -1 get a zero branch. Suited to
- * prefill batches with many tokens per adapter.
+ * scheduler that built the batch has them. Segments whose adapter is on a
+ * shape the tensor-core GEMM serves (M, R multiples of 128) run as grouped
+ * GEMM launches: adapters of equal (R, ell), up to 48 per launch, share one
+ * pre-pass and two GEMM launches whose tiles cover all their segments. Other
+ * segments run as their own dbf_forward (decode kernels). All on one stream
+ * and one workspace; segments with adapter id -1 get a zero branch.
  * adapters_host: host array of num_adapters descriptors (device pointers
  *    inside), each with the given M and N. seg_offsets_host: host int32
  *    [S+1], nondecreasing within [0, T]; seg_adapter_host: host int32 [S],
  *    each in [-1, num_adapters). x, y, flags as in dbf_forward; every
  *    segment's rows must be 16-byte aligned (M and N times the element size
  *    multiples of 16 bytes, else DBF_ERR_ALIGNMENT).
- * ws: dbf_forward_segmented_planned_workspace_bytes bytes (the largest
- *    segment's), 256-byte aligned, header as in dbf_forward.
+ * ws: dbf_forward_segmented_planned_workspace_bytes bytes, 256-byte
+ *    aligned, header as in dbf_forward.
  * Errors: DBF_ERR_INVALID_ARG (bad tables or descriptors, checked on the
  *    host before any launch), DBF_ERR_ALIGNMENT, DBF_ERR_WORKSPACE,
  *    DBF_ERR_CUDA. */

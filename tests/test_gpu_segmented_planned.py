@@ -39,3 +39,22 @@ def test_planned_matches_oracle(dbf, acc):
     got = host_y(dbf.forward_segmented_planned(dls, offs, ids, dev_x(x), y=y, accumulate=acc,
                                                y_dtype=torch.float32))
     assert rel_err(got, ref) < TOL
+
+
+def test_planned_grouped_many_segments(dbf):
+    # 60 segments of one GEMM-eligible shape (more than one grouped launch),
+    # lengths from 1 to 300 tokens, two shape classes plus an ineligible one
+    rng = np.random.default_rng(881)
+    M, N = 256, 384
+    layers = [random_layer(rng, M, N, 128, 1) for _ in range(5)] + [random_layer(rng, M, N, 256, 2),
+                                                                     random_layer(rng, M, N, 64, 1)]
+    lens = list(rng.integers(1, 40, size=57)) + [255, 256, 300]
+    ids = [int(v) for v in rng.integers(0, 5, size=57)] + [5, 6, 5]
+    ids[10] = -1
+    offs = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    T = int(offs[-1])
+    x = S.to_bf16_bits(rng.standard_normal((T, M)))
+    ref = oracle.forward_segmented(layers, offs, ids, x)
+    dls = [dev_layer(L) for L in layers]
+    got = host_y(dbf.forward_segmented_planned(dls, offs, ids, dev_x(x), y_dtype=torch.float32))
+    assert rel_err(got, ref) < TOL
