@@ -197,6 +197,47 @@ def mbok_forward(layer, x: np.ndarray) -> np.ndarray:
     return out
 
 
+def svid(X: np.ndarray):
+    """Sign-value-independent decomposition (DBF page, section 2: the SVID
+    projection from OneBit used inside ADMM; Multi-Boolean Architectures
+    page, section 2: W ~ W_bool . (s_out s_in^T) with W_bool = sign(W)):
+    X ~ sign(X) . (s_out s_in^T) with s_out s_in^T the best rank-1
+    approximation of |X| in the Frobenius norm. sign(0) = +1. The rank-1
+    factor sigma u v^T (u, v >= 0, unit norm) is split evenly:
+    s_out = sqrt(sigma) u, s_in = sqrt(sigma) v. fp64.
+    Returns (signs int8 [n, m], s_out [n], s_in [m])."""
+    X = np.asarray(X, dtype=np.float64)
+    S = np.where(X < 0, -1, 1).astype(np.int8)
+    U, sig, Vt = np.linalg.svd(np.abs(X), full_matrices=False)
+    u, v = U[:, 0], Vt[0]
+    if u.sum() < 0:   # the Perron vectors of a nonnegative matrix are nonnegative
+        u, v = -u, -v
+    r = np.sqrt(sig[0])
+    return S, r * u, r * v
+
+
+def mbok_extract(W: np.ndarray, K: int):
+    """Successive SVID extraction of K boolean kernels (Multi-Boolean
+    Architectures page, section 2: the first kernel takes the main
+    information, the next ones the residuals): R_0 = W, kernel k = SVID of
+    R_{k-1}, R_k = R_{k-1} - kernel k. Scales are rounded to fp16 before
+    the residual is formed (the layer stores them in fp16). fp64.
+    Returns (w int8 [K, n, m], s_out fp16 bits [K, n], s_in fp16 bits [K, m],
+    residual norms [K + 1])."""
+    R = np.asarray(W, dtype=np.float64).copy()
+    ws, so, si, norms = [], [], [], [float(np.linalg.norm(R))]
+    for _ in range(K):
+        S, a, b = svid(R)
+        a16 = a.astype(np.float16)
+        b16 = b.astype(np.float16)
+        R -= S * np.outer(a16.astype(np.float64), b16.astype(np.float64))
+        ws.append(S)
+        so.append(a16.view(np.uint16))
+        si.append(b16.view(np.uint16))
+        norms.append(float(np.linalg.norm(R)))
+    return np.stack(ws), np.stack(so), np.stack(si), np.array(norms)
+
+
 def ste_backward(db: np.ndarray, h: np.ndarray, tau: float) -> np.ndarray:
     """Straight-through estimator for latents h with signs B = sign(h) (LoRDBA
     page, section 2, training pipeline; the surrogate is not given there):
