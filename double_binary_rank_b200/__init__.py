@@ -54,6 +54,8 @@ _SIGS = {
     "dbf_pack_signs": (ctypes.c_int, [_vp, ctypes.c_int, _i64, _i64, _vp, _sz, _vp, _vp]),
     "dbf_unpack_signs": (ctypes.c_int, [_vp, _i64, _i64, _vp, _vp]),
     "dbf_transpose_signs": (ctypes.c_int, [_vp, _i64, _i64, _vp, _sz, _vp]),
+    "dbf_svid_scratch_bytes": (_sz, [_i64, _i64, _i32]),
+    "dbf_svid": (ctypes.c_int, [_vp, _i64, _i64, _i32, ctypes.c_int, _vp, _i64, _vp, _vp, _vp, _sz, _vp]),
     "dbf_gemm_min_tokens": (_i64, []),
     "dbf_workspace_bytes": (_sz, [_LP, _i64, ctypes.c_int]),
     "dbf_forward_launches": (_i32, [_LP, _i64, ctypes.c_int]),
@@ -326,6 +328,25 @@ def forward_segmented_planned(layers, seg_offsets, seg_adapter, x: torch.Tensor,
     return y
 
 
+def svid(X: torch.Tensor, iters: int = 24, subtract: bool = False, signs: Optional[torch.Tensor] = None,
+         s_out: Optional[torch.Tensor] = None, s_in: Optional[torch.Tensor] = None, stream=None):
+    """X ~ sign(X) . (s_out s_in^T) (dbf_svid). X: fp32 [n, m] on the device,
+    replaced by the residual when subtract. Returns (packed signs, s_out, s_in)."""
+    assert X.dtype == torch.float32 and X.is_contiguous()
+    n, m = X.shape
+    dev = X.device
+    if signs is None:
+        signs = torch.empty((n, (m + 31) // 32), dtype=torch.int32, device=dev)
+    if s_out is None:
+        s_out = torch.empty(n, dtype=torch.float16, device=dev)
+    if s_in is None:
+        s_in = torch.empty(m, dtype=torch.float16, device=dev)
+    scratch = alloc_workspace(int(_lib.dbf_svid_scratch_bytes(n, m, iters)), dev)
+    _check(_lib.dbf_svid(_ptr(X), n, m, iters, int(subtract), _ptr(signs), signs.stride(0), _ptr(s_out), _ptr(s_in),
+                         _ptr(scratch), scratch.numel(), _stream(stream)), "dbf_svid")
+    return signs, s_out, s_in
+
+
 @dataclass
 class MbokLayer:
     """Device-resident multi-boolean-kernel layer: w [N, ceil(K M / 32)] packed
@@ -347,6 +368,21 @@ class MbokLayer:
 
     def descriptor(self) -> DbfMbokLayerC:
         return DbfMbokLayerC(self.M, self.N, self.K, _ptr(self.w), _ptr(self.s_in), _ptr(self.s_out))
+
+    @staticmethod
+    def extract(W: torch.Tensor, K: int, iters: int = 24, stream=None) -> "MbokLayer":
+        """K boolean kernels extracted successively from a dense fp32 weight
+        W [N, M] (SVID of W, then of each residual); W is not modified."""
+        N, M = W.shape
+        R = W.float().clone().contiguous()
+        words = (K * M + 31) // 32
+        assert M % 32 == 0, "kernels side by side in a packed row need M % 32 == 0"
+        w = torch.empty((N, words), dtype=torch.int32, device=W.device)
+        s_out = torch.empty((K, N), dtype=torch.float16, device=W.device)
+        s_in = torch.empty((K, M), dtype=torch.float16, device=W.device)
+        for k in range(K):
+            svid(R, iters, subtract=True, signs=w[:, k * (M // 32):], s_out=s_out[k], s_in=s_in[k], stream=stream)
+        return MbokLayer(M, N, K, w, s_in, s_out)
 
 
 def mbok_workspace_bytes(layer: MbokLayer, T: int) -> int:

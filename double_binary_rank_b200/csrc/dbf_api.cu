@@ -89,6 +89,26 @@ dbf_status dbf_ste_backward(const float *db, const void *h, dbf_dtype h_dtype, i
                                 static_cast<cudaStream_t>(stream)));
 }
 
+size_t dbf_svid_scratch_bytes(int64_t n, int64_t m, int32_t iters)
+{
+    if (n <= 0 || m <= 0 || iters < 1 || iters > 1000) return 0;
+    return svid_scratch_bytes(n, m, iters);
+}
+
+dbf_status dbf_svid(float *X, int64_t n, int64_t m, int32_t iters, int subtract, uint32_t *signs,
+                    int64_t signs_ld_words, uint16_t *s_out, uint16_t *s_in, void *scratch, size_t scratch_bytes,
+                    void *stream)
+{
+    if (!X || !signs || !s_out || !s_in || n <= 0 || m <= 0 || iters < 1 || iters > 1000 ||
+        signs_ld_words < pitch_words(m))
+        return DBF_ERR_INVALID_ARG;
+    if (!aligned(X, 4) || !aligned(signs, 4) || !aligned(s_out, 2) || !aligned(s_in, 2)) return DBF_ERR_ALIGNMENT;
+    if (!scratch || scratch_bytes < svid_scratch_bytes(n, m, iters)) return DBF_ERR_WORKSPACE;
+    if (!aligned(scratch, 256)) return DBF_ERR_ALIGNMENT;
+    return from_cuda(svid_run(X, n, m, iters, subtract ? 1 : 0, signs, signs_ld_words, s_out, s_in, scratch,
+                              static_cast<cudaStream_t>(stream)));
+}
+
 int64_t dbf_gemm_min_tokens(void) { return kGemmMinTokens; }
 
 size_t dbf_workspace_bytes(const dbf_layer *L, int64_t T, dbf_path path)

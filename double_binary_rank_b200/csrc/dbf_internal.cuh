@@ -54,6 +54,11 @@ cudaError_t mbok_forward(int M, int N, int K, const uint32_t *w_packed, const ui
                          const uint16_t *s_out, const void *x, dbf_dtype xd, void *y, dbf_dtype yd,
                          int64_t T, int flags, void *ws, cudaStream_t s);
 
+// SVID (sign times the best rank-1 fit of the magnitudes), by power iteration
+size_t svid_scratch_bytes(int64_t n, int64_t m, int iters);
+cudaError_t svid_run(float *X, int64_t n, int64_t m, int iters, int subtract, uint32_t *signs,
+                     int64_t signs_ld, uint16_t *s_out, uint16_t *s_in, void *scratch, cudaStream_t s);
+
 // prefill path (tcgen05)
 bool gemm_shape_ok(const dbf_layer &L);
 size_t gemm_workspace_bytes(const dbf_layer &L, int64_t T);

@@ -136,6 +136,28 @@ dbf_status dbf_transpose_signs(const uint32_t *src, int64_t rows, int64_t k, uin
 dbf_status dbf_ste_backward(const float *db, const void *h, dbf_dtype h_dtype, int64_t count, float tau,
                             float *dh, int flags, void *stream);
 
+/* Sign-value-independent decomposition of a dense fp32 matrix X (n x m,
+ * row-major): X ~ sign(X) . (s_out s_in^T), s_out s_in^T the best rank-1
+ * approximation of |X|, split evenly between the two vectors (DBF page,
+ * section 2: the SVID projection inside the factorisation; Multi-Boolean
+ * Architectures page, section 2: a boolean kernel with its scales, and
+ * successive extraction of further kernels from the residual). The rank-1
+ * factor comes from `iters` power iterations from the all-positive start.
+ * signs: device, packed sign(X) (bit set = -1, sign(0) = +1), n rows with
+ *    signs_ld_words words each (>= ceil(m/32); a larger pitch places the
+ *    kernel inside a wider packed matrix, e.g. one block of an MBOK layer).
+ * s_out [n], s_in [m]: device fp16 outputs.
+ * subtract != 0: X is replaced by the residual X - sign(X) . (s_out s_in^T)
+ *    computed with the stored fp16 scales (the next kernel of a successive
+ *    extraction); else X is only read.
+ * scratch: dbf_svid_scratch_bytes(n, m, iters) bytes, 256-byte aligned.
+ * Errors: DBF_ERR_INVALID_ARG, DBF_ERR_ALIGNMENT, DBF_ERR_WORKSPACE,
+ *    DBF_ERR_CUDA. */
+size_t dbf_svid_scratch_bytes(int64_t n, int64_t m, int32_t iters);
+dbf_status dbf_svid(float *X, int64_t n, int64_t m, int32_t iters, int subtract, uint32_t *signs,
+                    int64_t signs_ld_words, uint16_t *s_out, uint16_t *s_in, void *scratch,
+                    size_t scratch_bytes, void *stream);
+
 /* Smallest T for which DBF_PATH_AUTO takes the GEMM path on a shape it allows. */
 int64_t dbf_gemm_min_tokens(void);
 
