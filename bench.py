@@ -406,6 +406,21 @@ def main():
     seg_us = max_over_ranks(1e3 * g0.elapsed_time(g1) / 5, dev)
     seg_flops = 2 * n_ad * per * 2 * 128 * (w.M + w.M)
 
+    # ---- SVID of a dense 11008 x 4096 fp32 weight (24 power iterations), the
+    # projection of the factorisation and the first MBOK kernel
+    Wd = torch.randn((w.N, w.M), device=dev)
+    dbf.svid(Wd, iters=24, stream=stream)
+    torch.cuda.synchronize(dev)
+    v0, v1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        v0.record(stream)
+        dbf.svid(Wd, iters=24, stream=stream)
+        v1.record(stream)
+    torch.cuda.synchronize(dev)
+    svid_us = max_over_ranks(1e3 * v0.elapsed_time(v1), dev)
+    svid_bytes = (2 * 24 + 1) * Wd.numel() * 4
+    del Wd
+
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
@@ -447,6 +462,9 @@ def main():
                               "us_per_call": seg_us, "tokens_per_s": n_ad * per / (seg_us * 1e-6),
                               "achieved": seg_flops / (seg_us * 1e-6) / 1e12, "unit": "TFLOP/s", "peak": pk["bf16_tflops"],
                               "frac": seg_flops / (seg_us * 1e-6) / 1e12 / pk["bf16_tflops"]},
+        "svid": {"kernel": "SVID of an 11008 x 4096 fp32 matrix, 24 power iterations (signs packed, fp16 scales)",
+                 "us_per_call": svid_us, "achieved": svid_bytes / (svid_us * 1e-6) / 1e9, "unit": "GB/s",
+                 "peak": pk["hbm_gbs"], "frac": svid_bytes / (svid_us * 1e-6) / 1e9 / pk["hbm_gbs"]},
         "clocks": clk.summary(),
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": args.steps * (dec_launches + pre_launches),
