@@ -418,8 +418,37 @@ def main():
         v1.record(stream)
     torch.cuda.synchronize(dev)
     svid_us = max_over_ranks(1e3 * v0.elapsed_time(v1), dev)
-    svid_bytes = (2 * 24 + 1) * Wd.numel() * 4
+    # algorithmic bytes: one read of X per power iteration (u and v come from
+    # the same pass), one read for the signs, the packed signs written
+    svid_bytes = (24 + 1) * Wd.numel() * 4 + Wd.numel() // 8
     del Wd
+
+    # ---- DBF factorisation of an 11008 x 4096 fp32 weight at k = 5888 (the
+    # DBF MLP layer's shape): one outer iteration, 4 ADMM steps per factor,
+    # 24-iteration SVID projections, seeded random start
+    fn, fm, fk, f_admm = w.N, w.M, w.R, 4
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(w.seed)
+    Wf = (torch.randn((fn, fm), device=dev, generator=gen) * torch.exp(0.25 * torch.randn((fn, 1), device=dev, generator=gen))
+          * torch.exp(0.25 * torch.randn((1, fm), device=dev, generator=gen)))
+    s0 = float(Wf.square().mean().sqrt()) ** 0.5 * fk ** -0.25
+    U0f = s0 * torch.randn((fn, fk), device=dev, generator=gen)
+    V0f = s0 * torch.randn((fk, fm), device=dev, generator=gen)
+    f_ws = dbf.alloc_workspace(dbf.factorize_workspace_bytes(fn, fm, fk, 1, 24), dev)
+    dbf.factorize(Wf, U0f, V0f, outer=1, admm_iters=f_admm, objective=False, ws=f_ws, stream=stream)
+    torch.cuda.synchronize(dev)
+    q0, q1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        q0.record(stream)
+        dbf.factorize(Wf, U0f, V0f, outer=1, admm_iters=f_admm, objective=False, ws=f_ws, stream=stream)
+        q1.record(stream)
+    torch.cuda.synchronize(dev)
+    fact_us = max_over_ranks(1e3 * q0.elapsed_time(q1), dev)
+    # fp32 contraction flops of one outer iteration: W V^T, V V^T, the sweep
+    # inverse, the U solves; U^T W, U^T U, the sweep inverse, the V solves
+    fact_flops = (2 * fn * fm * fk + 2 * fk * fk * fm + 2 * fk ** 3 + f_admm * 2 * fn * fk * fk
+                  + 2 * fn * fm * fk + 2 * fk * fk * fn + 2 * fk ** 3 + f_admm * 2 * fk * fk * fm)
+    del Wf, U0f, V0f, f_ws
 
     if world > 1:
         dist.barrier()
@@ -428,6 +457,7 @@ def main():
         return
 
     pk, pk_kind = peaks()
+    fp32_peak = 148 * 128 * 2 * 1.965e9 / 1e12
     b_dec, f_dec = algorithmic(w, T_DECODE)
     b_pre, f_pre = algorithmic(w, T_PREFILL)
     gbs = b_dec / (dec_us * 1e-6) / 1e9
@@ -465,6 +495,12 @@ def main():
         "svid": {"kernel": "SVID of an 11008 x 4096 fp32 matrix, 24 power iterations (signs packed, fp16 scales)",
                  "us_per_call": svid_us, "achieved": svid_bytes / (svid_us * 1e-6) / 1e9, "unit": "GB/s",
                  "peak": pk["hbm_gbs"], "frac": svid_bytes / (svid_us * 1e-6) / 1e9 / pk["hbm_gbs"]},
+        "factorize": {"kernel": "DBF factorisation of an 11008 x 4096 fp32 weight at k=5888: one outer iteration "
+                                "(4 ADMM steps per factor, fp32 SIMT GEMMs, blocked sweep inverse, single-read SVID)",
+                      "ms_per_outer_iteration": fact_us / 1e3, "achieved": fact_flops / (fact_us * 1e-6) / 1e12,
+                      "unit": "TFLOP/s", "bound": "alu", "peak": fp32_peak,
+                      "frac": fact_flops / (fact_us * 1e-6) / 1e12 / fp32_peak,
+                      "peak_source": "derived: 148 SMs x 128 fp32 lanes x 2 flops x 1965 MHz max SM clock"},
         "clocks": clk.summary(),
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": args.steps * (dec_launches + pre_launches),

@@ -45,6 +45,11 @@ TAG_BETA = 5
 TAG_GAMMA = 6
 TAG_IDS = 7
 TAG_YIN = 8
+TAG_WEIGHT = 9
+TAG_WROW = 10
+TAG_WCOL = 11
+TAG_U0 = 12
+TAG_V0 = 13
 
 BASE_SEED = 0xDBF00000
 
@@ -179,6 +184,26 @@ class MbokLayer:
     w: np.ndarray
     s_in: np.ndarray
     s_out: np.ndarray
+
+
+def make_weight(seed: int, n: int, m: int, sigma: float = 0.25) -> np.ndarray:
+    """A dense fp32 weight n x m with the row and column scale structure of
+    trained layers: W[i, j] = g[i, j] r[i] c[j], g ~ N(0, 1), r and c
+    lognormal with parameter sigma."""
+    g = normal(stream_key(seed, TAG_WEIGHT), n * m).reshape(n, m)
+    r = np.exp(sigma * normal(stream_key(seed, TAG_WROW), n))
+    c = np.exp(sigma * normal(stream_key(seed, TAG_WCOL), m))
+    return (g * r[:, None] * c[None, :]).astype(np.float32)
+
+
+def make_factor_start(seed: int, n: int, m: int, k: int, scale: float = 1.0):
+    """A seeded random start (U0 n x k, V0 k x m, fp32) for the
+    factorisation: N(0, s^2) entries with s = sqrt(scale) k^-1/4, so that
+    U0 V0 has entries of about 'scale'."""
+    s = np.sqrt(scale) * k ** -0.25
+    U0 = (s * normal(stream_key(seed, TAG_U0), n * k)).astype(np.float32).reshape(n, k)
+    V0 = (s * normal(stream_key(seed, TAG_V0), k * m)).astype(np.float32).reshape(k, m)
+    return U0, V0
 
 
 def make_mbok_layer(seed: int, M: int, N: int, K: int, sigma: float = 0.5) -> MbokLayer:

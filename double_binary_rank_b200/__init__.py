@@ -56,6 +56,9 @@ _SIGS = {
     "dbf_transpose_signs": (ctypes.c_int, [_vp, _i64, _i64, _vp, _sz, _vp]),
     "dbf_svid_scratch_bytes": (_sz, [_i64, _i64, _i32]),
     "dbf_svid": (ctypes.c_int, [_vp, _i64, _i64, _i32, ctypes.c_int, _vp, _i64, _vp, _vp, _vp, _sz, _vp]),
+    "dbf_factorize_workspace_bytes": (_sz, [_i64, _i64, _i64, _i32, _i32]),
+    "dbf_factorize": (ctypes.c_int, [_vp, _i64, _i64, _i64, _vp, _vp, _i32, _i32, _i32, ctypes.c_float, _vp, _vp,
+                                     _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "dbf_gemm_min_tokens": (_i64, []),
     "dbf_workspace_bytes": (_sz, [_LP, _i64, ctypes.c_int]),
     "dbf_forward_launches": (_i32, [_LP, _i64, ctypes.c_int]),
@@ -345,6 +348,37 @@ def svid(X: torch.Tensor, iters: int = 24, subtract: bool = False, signs: Option
     _check(_lib.dbf_svid(_ptr(X), n, m, iters, int(subtract), _ptr(signs), signs.stride(0), _ptr(s_out), _ptr(s_in),
                          _ptr(scratch), scratch.numel(), _stream(stream)), "dbf_svid")
     return signs, s_out, s_in
+
+
+def factorize_workspace_bytes(n: int, m: int, k: int, outer: int, svid_iters: int = 24) -> int:
+    return int(_lib.dbf_factorize_workspace_bytes(n, m, k, outer, svid_iters))
+
+
+def factorize(W: torch.Tensor, U0: torch.Tensor, V0: torch.Tensor, outer: int, admm_iters: int = 4,
+              svid_iters: int = 24, rho_rel: float = 1.0, objective: bool = True, ws: Optional[torch.Tensor] = None,
+              stream=None):
+    """Double binary factorisation W ~ (a . A . mid^T)(B . b^T) (dbf_factorize).
+    W: fp32 [n, m]; U0: fp32 [n, k]; V0: fp32 [k, m], on the device. Returns
+    (Layer with M = m, N = n, R = k, ell = 1, objective fp32 [outer + 1] or None)."""
+    for t in (W, U0, V0):
+        assert t.dtype == torch.float32 and t.is_contiguous()
+    n, m = W.shape
+    k = U0.shape[1]
+    assert U0.shape == (n, k) and V0.shape == (k, m)
+    dev = W.device
+    b1 = torch.empty((n, (k + 31) // 32), dtype=torch.int32, device=dev)
+    b2 = torch.empty((k, (m + 31) // 32), dtype=torch.int32, device=dev)
+    alpha = torch.empty((1, n), dtype=torch.float16, device=dev)
+    beta = torch.empty((1, k), dtype=torch.float16, device=dev)
+    gamma = torch.empty((1, m), dtype=torch.float16, device=dev)
+    obj = torch.empty(outer + 1, dtype=torch.float32, device=dev) if objective else None
+    if ws is None:
+        ws = alloc_workspace(factorize_workspace_bytes(n, m, k, outer, svid_iters), dev)
+    _check(_lib.dbf_factorize(_ptr(W), n, m, k, _ptr(U0), _ptr(V0), outer, admm_iters, svid_iters, rho_rel,
+                              _ptr(b1), _ptr(b2), _ptr(alpha), _ptr(beta), _ptr(gamma),
+                              _ptr(obj) if obj is not None else None, _ptr(ws), ws.numel(), _stream(stream)),
+           "dbf_factorize")
+    return Layer(m, n, k, 1, b1, b2, alpha, beta, gamma), obj
 
 
 @dataclass

@@ -2,6 +2,7 @@
 // (no launch on a failed check), path choice and the workspace contract.
 #include "dbf_internal.cuh"
 
+#include <cmath>
 #include <vector>
 
 namespace {
@@ -107,6 +108,41 @@ dbf_status dbf_svid(float *X, int64_t n, int64_t m, int32_t iters, int subtract,
     if (!aligned(scratch, 256)) return DBF_ERR_ALIGNMENT;
     return from_cuda(svid_run(X, n, m, iters, subtract ? 1 : 0, signs, signs_ld_words, s_out, s_in, scratch,
                               static_cast<cudaStream_t>(stream)));
+}
+
+namespace {
+constexpr int64_t kFactorMaxDim = int64_t(65535) * 128;   // GEMM grid rows of 128 stay <= 65535
+
+bool factor_args_ok(int64_t n, int64_t m, int64_t k, int32_t outer, int32_t svid_iters)
+{
+    return n > 0 && m > 0 && k > 0 && outer >= 0 && outer <= 100000 && svid_iters >= 1 && svid_iters <= 1000;
+}
+}  // namespace
+
+size_t dbf_factorize_workspace_bytes(int64_t n, int64_t m, int64_t k, int32_t outer, int32_t svid_iters)
+{
+    if (!factor_args_ok(n, m, k, outer, svid_iters) || n > kFactorMaxDim || m > kFactorMaxDim || k > kFactorMaxDim)
+        return 0;
+    return factorize_workspace_bytes(n, m, k, outer, svid_iters);
+}
+
+dbf_status dbf_factorize(const float *W, int64_t n, int64_t m, int64_t k, const float *U0, const float *V0,
+                         int32_t outer, int32_t admm_iters, int32_t svid_iters, float rho_rel, uint32_t *a_signs,
+                         uint32_t *b_signs, uint16_t *alpha, uint16_t *beta, uint16_t *gamma, float *objective,
+                         void *ws, size_t ws_bytes, void *stream)
+{
+    if (!W || !U0 || !V0 || !a_signs || !b_signs || !alpha || !beta || !gamma ||
+        !factor_args_ok(n, m, k, outer, svid_iters) || admm_iters < 1 || admm_iters > 1000 ||
+        !(rho_rel > 0.f) || !std::isfinite(rho_rel))
+        return DBF_ERR_INVALID_ARG;
+    if (n > kFactorMaxDim || m > kFactorMaxDim || k > kFactorMaxDim) return DBF_ERR_UNSUPPORTED;
+    if (!aligned(W, 4) || !aligned(U0, 4) || !aligned(V0, 4) || !aligned(a_signs, 4) || !aligned(b_signs, 4) ||
+        !aligned(alpha, 2) || !aligned(beta, 2) || !aligned(gamma, 2) || (objective && !aligned(objective, 4)))
+        return DBF_ERR_ALIGNMENT;
+    if (!ws || ws_bytes < factorize_workspace_bytes(n, m, k, outer, svid_iters)) return DBF_ERR_WORKSPACE;
+    if (!aligned(ws, 256)) return DBF_ERR_ALIGNMENT;
+    return from_cuda(factorize_run(W, n, m, k, U0, V0, outer, admm_iters, svid_iters, rho_rel, a_signs, b_signs,
+                                   alpha, beta, gamma, objective, ws, static_cast<cudaStream_t>(stream)));
 }
 
 int64_t dbf_gemm_min_tokens(void) { return kGemmMinTokens; }

@@ -1,0 +1,502 @@
+// DBF factorisation of a dense fp32 weight on the GPU.
+//
+// DBF page, section 2 ("Metodologia", "Algoritmo de Computação"): W (n x m)
+// ~ (a . A . m^T)(B . b^T) with sign matrices A (n x k), B (k x m) and scale
+// vectors a, m, b, found by alternating minimisation with ADMM and the SVID
+// projection. The page gives only that outline; the steps implemented here
+// (the plainest reading, no importance weights):
+//   U = diag(a) A diag(m1) and V = diag(m2) B diag(b) (m = m1 . m2);
+//   U-subproblem (V fixed), ADMM in scaled form from Z = U, Lam = 0:
+//     U <- (W V^T + rho (Z - Lam)) (V V^T + rho I)^-1
+//     Z <- SVID(U + Lam),  Lam <- Lam + U - Z        (admm_iters times)
+//   then the V-subproblem (U fixed) with the operands transposed;
+//   rho = rho_rel * trace(Gram) / k.
+//
+// Work per outer iteration (k x k Gram and inverse, n x k and k x m
+// right-hand sides) is dense fp32 contraction: a register-tiled SIMT GEMM
+// (128 x 128 tiles, 8 x 8 outputs per thread, double-buffered shared
+// memory) does all of it, including the rank-64 updates of the blocked
+// inverse. The inverse of the SPD matrix V V^T + rho I is an in-place
+// blocked sweep (Gauss-Jordan without pivoting, stable for SPD): per 64-wide
+// pivot block, the block's inverse D (one CTA), E = P D with P the block
+// column, A -= E P^T, then the block row / column / diagonal are set to E^T,
+// E and -D; after all blocks A holds -(V V^T + rho I)^-1. The SVID
+// projection is the library's power iteration (fp32 scales).
+#include "dbf_internal.cuh"
+
+namespace dbf {
+namespace {
+
+// ---- fp32 GEMM: Cout = alpha op(A) op(B) + beta Cin ---------------------------
+// Row-major. op(A) is M x K: A stored M x K (TA = false) or K x M (TA = true);
+// op(B) is K x N: B stored K x N (TB = false) or N x K (TB = true). Cin may
+// alias Cout. With sumsq non-null nothing is stored: the squares of the
+// results are added to *sumsq (the objective's residual norm).
+constexpr int kGT = 256;
+constexpr int kGM = 128, kGN = 128, kGK = 16;
+constexpr int kGPad = 4;
+constexpr int kVecA = 1, kVecB = 2, kVecC = 4;   // float4 access allowed (aligned base, ld % 4 == 0)
+
+__device__ __forceinline__ float4 ld4_guard(const float *p, int64_t ld, int64_t r, int64_t c, int64_t R, int64_t C,
+                                            bool vec)
+{
+    // four consecutive elements (r, c .. c + 3) of an R x C row-major matrix
+    if (r >= R) return make_float4(0.f, 0.f, 0.f, 0.f);
+    const float *q = p + r * ld + c;
+    if (vec && c + 3 < C) return *reinterpret_cast<const float4 *>(q);
+    float4 v;
+    v.x = c < C ? q[0] : 0.f;
+    v.y = c + 1 < C ? q[1] : 0.f;
+    v.z = c + 2 < C ? q[2] : 0.f;
+    v.w = c + 3 < C ? q[3] : 0.f;
+    return v;
+}
+
+// Load this thread's share of a 128 x 16 (rows x k) operand tile. K-major
+// storage (TRANS == false for A: rows of A hold k contiguously) is read as
+// 4 consecutive k of one row; the other storage as 4 consecutive rows of
+// one k.
+template <bool KCONTIG>
+__device__ __forceinline__ void load_tile(const float *p, int64_t ld, int64_t rows, int64_t kdim, int64_t r0,
+                                          int64_t k0, bool vec, float4 (&t)[2])
+{
+    const int tid = threadIdx.x;
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        if (KCONTIG) {
+            const int r = tid / 4 + 64 * i, kq = (tid % 4) * 4;
+            t[i] = ld4_guard(p, ld, r0 + r, k0 + kq, rows, kdim, vec);
+        } else {
+            const int kr = tid / 32 + 8 * i, rq = (tid % 32) * 4;
+            t[i] = ld4_guard(p, ld, k0 + kr, r0 + rq, kdim, rows, vec);
+        }
+    }
+}
+
+template <bool KCONTIG>
+__device__ __forceinline__ void store_tile(float (*s)[kGM + kGPad], const float4 (&t)[2])
+{
+    const int tid = threadIdx.x;
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        if (KCONTIG) {
+            const int r = tid / 4 + 64 * i, kq = (tid % 4) * 4;
+            s[kq + 0][r] = t[i].x;
+            s[kq + 1][r] = t[i].y;
+            s[kq + 2][r] = t[i].z;
+            s[kq + 3][r] = t[i].w;
+        } else {
+            const int kr = tid / 32 + 8 * i, rq = (tid % 32) * 4;
+            *reinterpret_cast<float4 *>(&s[kr][rq]) = t[i];
+        }
+    }
+}
+
+template <bool TA, bool TB>
+__global__ void __launch_bounds__(kGT, 2)
+    sgemm_kernel(int64_t M, int64_t N, int64_t K, float alpha, const float *__restrict__ A, int64_t lda,
+                 const float *__restrict__ B, int64_t ldb, float beta, const float *Cin, int64_t ldci, float *Cout,
+                 int64_t ldco, int vec, double *sumsq)
+{
+    __shared__ __align__(16) float As[2][kGK][kGM + kGPad];
+    __shared__ __align__(16) float Bs[2][kGK][kGN + kGPad];
+    const int tid = threadIdx.x, tx = tid % 16, ty = tid / 16;
+    const int64_t m0 = static_cast<int64_t>(blockIdx.y) * kGM, n0 = static_cast<int64_t>(blockIdx.x) * kGN;
+    const int64_t nk = (K + kGK - 1) / kGK;
+    // A: rows M, k contiguous unless TA; B as rows N: k contiguous when TB
+    float4 ra[2], rb[2];
+    load_tile<!TA>(A, lda, M, K, m0, 0, vec & kVecA, ra);
+    load_tile<TB>(B, ldb, N, K, n0, 0, vec & kVecB, rb);
+    store_tile<!TA>(As[0], ra);
+    store_tile<TB>(Bs[0], rb);
+    __syncthreads();
+
+    float acc[8][8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
+
+    for (int64_t kt = 0; kt < nk; ++kt) {
+        const int cur = static_cast<int>(kt & 1);
+        const bool more = kt + 1 < nk;
+        if (more) {
+            load_tile<!TA>(A, lda, M, K, m0, (kt + 1) * kGK, vec & kVecA, ra);
+            load_tile<TB>(B, ldb, N, K, n0, (kt + 1) * kGK, vec & kVecB, rb);
+        }
+#pragma unroll
+        for (int kk = 0; kk < kGK; ++kk) {
+            const float4 a0 = *reinterpret_cast<const float4 *>(&As[cur][kk][ty * 4]);
+            const float4 a1 = *reinterpret_cast<const float4 *>(&As[cur][kk][64 + ty * 4]);
+            const float4 b0 = *reinterpret_cast<const float4 *>(&Bs[cur][kk][tx * 4]);
+            const float4 b1 = *reinterpret_cast<const float4 *>(&Bs[cur][kk][64 + tx * 4]);
+            const float a[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+            const float b[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+#pragma unroll
+                for (int j = 0; j < 8; ++j) acc[i][j] += a[i] * b[j];
+        }
+        if (more) {
+            store_tile<!TA>(As[cur ^ 1], ra);
+            store_tile<TB>(Bs[cur ^ 1], rb);
+        }
+        __syncthreads();
+    }
+
+    float sq = 0.f;
+    const bool vc = (vec & kVecC) != 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const int64_t row = m0 + (i < 4 ? ty * 4 + i : 64 + ty * 4 + i - 4);
+        if (row >= M) continue;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const int64_t col = n0 + h * 64 + tx * 4;
+            if (col >= N) continue;
+            float v[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) v[e] = alpha * acc[i][h * 4 + e];
+            if (beta != 0.f) {
+                const float4 c = ld4_guard(Cin, ldci, row, col, M, N, vc);
+                v[0] += beta * c.x;
+                v[1] += beta * c.y;
+                v[2] += beta * c.z;
+                v[3] += beta * c.w;
+            }
+            if (sumsq) {
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    if (col + e < N) sq += v[e] * v[e];
+            } else if (vc && col + 3 < N) {
+                *reinterpret_cast<float4 *>(Cout + row * ldco + col) = make_float4(v[0], v[1], v[2], v[3]);
+            } else {
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    if (col + e < N) Cout[row * ldco + col + e] = v[e];
+            }
+        }
+    }
+    if (sumsq) {
+        for (int o = 16; o; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
+        if ((tid & 31) == 0) atomicAdd(sumsq, static_cast<double>(sq));
+    }
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+// Cout[M x N] = alpha op(A) op(B) + beta Cin (see sgemm_kernel)
+cudaError_t sgemm(bool ta, bool tb, int64_t M, int64_t N, int64_t K, float alpha, const float *A, int64_t lda,
+                  const float *B, int64_t ldb, float beta, const float *Cin, int64_t ldci, float *Cout, int64_t ldco,
+                  cudaStream_t s, double *sumsq = nullptr)
+{
+    if (M <= 0 || N <= 0) return cudaSuccess;
+    int vec = 0;
+    if (aligned16(A) && lda % 4 == 0) vec |= kVecA;
+    if (aligned16(B) && ldb % 4 == 0) vec |= kVecB;
+    if ((sumsq || (aligned16(Cout) && ldco % 4 == 0)) && (beta == 0.f || (aligned16(Cin) && ldci % 4 == 0)))
+        vec |= kVecC;
+    const dim3 grid(static_cast<unsigned>((N + kGN - 1) / kGN), static_cast<unsigned>((M + kGM - 1) / kGM));
+    if (!ta && !tb)
+        sgemm_kernel<false, false><<<grid, kGT, 0, s>>>(M, N, K, alpha, A, lda, B, ldb, beta, Cin, ldci, Cout, ldco,
+                                                        vec, sumsq);
+    else if (!ta && tb)
+        sgemm_kernel<false, true><<<grid, kGT, 0, s>>>(M, N, K, alpha, A, lda, B, ldb, beta, Cin, ldci, Cout, ldco,
+                                                       vec, sumsq);
+    else if (ta && !tb)
+        sgemm_kernel<true, false><<<grid, kGT, 0, s>>>(M, N, K, alpha, A, lda, B, ldb, beta, Cin, ldci, Cout, ldco,
+                                                       vec, sumsq);
+    else
+        sgemm_kernel<true, true><<<grid, kGT, 0, s>>>(M, N, K, alpha, A, lda, B, ldb, beta, Cin, ldci, Cout, ldco,
+                                                      vec, sumsq);
+    return cudaGetLastError();
+}
+
+// ---- blocked sweep inverse of an SPD matrix ---------------------------------
+constexpr int kSweepBlock = 64;
+
+// P = A[:, p0 : p0 + bs] (k x bs, ld bs)
+__global__ void sweep_panel_kernel(const float *__restrict__ A, int64_t k, int64_t p0, int bs, float *__restrict__ P)
+{
+    for (int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; idx < k * bs;
+         idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const int64_t i = idx / bs;
+        const int l = static_cast<int>(idx - i * bs);
+        P[idx] = A[i * k + p0 + l];
+    }
+}
+
+// D = T^-1 for the bs x bs SPD block T = P[p0 : p0 + bs, :], by the scalar
+// sweep in shared memory (pivot p: T_ij -= T_ip T_pj / T_pp for i, j != p,
+// then T_ip *= 1 / T_pp, T_pj *= 1 / T_pp, T_pp = -1 / T_pp; after every
+// pivot T = -(original T)^-1). One CTA.
+__global__ void __launch_bounds__(256) sweep_block_inverse_kernel(const float *__restrict__ P, int64_t p0, int bs,
+                                                                  float *__restrict__ D)
+{
+    __shared__ float T[kSweepBlock][kSweepBlock + 1];
+    __shared__ float colp[kSweepBlock], rowp[kSweepBlock];
+    const int tid = threadIdx.x;
+    for (int idx = tid; idx < bs * bs; idx += blockDim.x) T[idx / bs][idx % bs] = P[(p0 + idx / bs) * bs + idx % bs];
+    __syncthreads();
+    for (int p = 0; p < bs; ++p) {
+        if (tid < bs) {
+            colp[tid] = T[tid][p];
+            rowp[tid] = T[p][tid];
+        }
+        __syncthreads();
+        const float d = 1.0f / colp[p];
+        for (int idx = tid; idx < bs * bs; idx += blockDim.x) {
+            const int i = idx / bs, j = idx % bs;
+            float v;
+            if (i != p && j != p) v = T[i][j] - colp[i] * d * rowp[j];
+            else if (i == p && j == p) v = -d;
+            else if (j == p) v = colp[i] * d;
+            else v = d * rowp[j];
+            T[i][j] = v;
+        }
+        __syncthreads();
+    }
+    for (int idx = tid; idx < bs * bs; idx += blockDim.x) D[idx] = -T[idx / bs][idx % bs];
+}
+
+// After A -= E P^T: the pivot block column and row become E and E^T, the
+// pivot block -D. Column writes run along l (contiguous in a row of A), row
+// writes along i (contiguous in a row of A).
+__global__ void sweep_fixup_kernel(float *__restrict__ A, int64_t k, int64_t p0, int bs, const float *__restrict__ E,
+                                   const float *__restrict__ D)
+{
+    const int64_t total = k * bs;
+    for (int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; idx < total;
+         idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        {   // column block: (i, p0 + l), l fastest
+            const int64_t i = idx / bs;
+            const int l = static_cast<int>(idx - i * bs);
+            A[i * k + p0 + l] = (i >= p0 && i < p0 + bs) ? -D[(i - p0) * bs + l] : E[i * bs + l];
+        }
+        {   // row block: (p0 + l, i), i fastest
+            const int l = static_cast<int>(idx / k);
+            const int64_t i = idx - static_cast<int64_t>(l) * k;
+            if (i < p0 || i >= p0 + bs) A[(p0 + l) * k + i] = E[i * bs + l];
+        }
+    }
+}
+
+// ---- ADMM element-wise steps ------------------------------------------------
+
+// rho = rho_rel * trace(G) / k, then G += rho I. One CTA.
+__global__ void __launch_bounds__(256) rho_kernel(float *__restrict__ G, int64_t k, float rho_rel, float *rho_out)
+{
+    __shared__ float part[8];
+    __shared__ float rho_s;
+    float t = 0.f;
+    for (int64_t i = threadIdx.x; i < k; i += blockDim.x) t += G[i * k + i];
+    for (int o = 16; o; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+    if ((threadIdx.x & 31) == 0) part[threadIdx.x >> 5] = t;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        float s = 0.f;
+        for (int w = 0; w < 8; ++w) s += part[w];
+        rho_s = rho_rel * s / static_cast<float>(k);
+        *rho_out = rho_s;
+    }
+    __syncthreads();
+    const float r = rho_s;
+    for (int64_t i = threadIdx.x; i < k; i += blockDim.x) G[i * k + i] += r;
+}
+
+// Rhs = C + rho (Z - Lam)
+__global__ void rhs_kernel(const float *__restrict__ C, const float *__restrict__ Z, const float *__restrict__ Lam,
+                           const float *rho, int64_t count, float *__restrict__ Rhs)
+{
+    const float r = *rho;
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < count;
+         i += static_cast<int64_t>(gridDim.x) * blockDim.x)
+        Rhs[i] = C[i] + r * (Z[i] - Lam[i]);
+}
+
+// Z = sign(X) . p q^T (sign(0) = +1) and Lam = X - Z, X rows x cols
+__global__ void project_kernel(const float *__restrict__ X, int64_t rows, int64_t cols, const float *__restrict__ p,
+                               const float *__restrict__ q, float *__restrict__ Z, float *__restrict__ Lam)
+{
+    const int64_t count = rows * cols;
+    for (int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; idx < count;
+         idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const int64_t i = idx / cols, j = idx - i * cols;
+        const float x = X[idx];
+        const float mag = p[i] * q[j];
+        const float z = x < 0.f ? -mag : mag;
+        Z[idx] = z;
+        Lam[idx] = x - z;
+    }
+}
+
+__global__ void objective_kernel(const double *sumsq, float *objective)
+{
+    *objective = static_cast<float>(sqrt(*sumsq));
+}
+
+// alpha = fp16(a), beta = fp16(m1 . m2), gamma = fp16(b)
+__global__ void factor_scales_kernel(const float *__restrict__ a, int64_t n, const float *__restrict__ m1,
+                                     const float *__restrict__ m2, int64_t k, const float *__restrict__ b, int64_t m,
+                                     uint16_t *alpha, uint16_t *beta, uint16_t *gamma)
+{
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n + k + m;
+         i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        if (i < n) alpha[i] = __half_as_ushort(__float2half_rn(a[i]));
+        else if (i < n + k) beta[i - n] = __half_as_ushort(__float2half_rn(m1[i - n] * m2[i - n]));
+        else gamma[i - n - k] = __half_as_ushort(__float2half_rn(b[i - n - k]));
+    }
+}
+
+int sm_count()
+{
+    int dev = 0, v = 0;
+    cudaGetDevice(&dev);
+    return (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && v > 0) ? v : 148;
+}
+
+int ew_grid(int64_t count, int sms)
+{
+    const int64_t g = (count + 255) / 256;
+    return static_cast<int>(g < sms * 8 ? (g > 0 ? g : 1) : sms * 8);
+}
+
+// A (k x k, SPD) <- -A^-1 in place. Scratch: P, E (k x kSweepBlock), D.
+cudaError_t sweep_inverse(float *A, int64_t k, float *P, float *E, float *D, int sms, cudaStream_t s)
+{
+    cudaError_t e;
+    for (int64_t p0 = 0; p0 < k; p0 += kSweepBlock) {
+        const int bs = static_cast<int>(k - p0 < kSweepBlock ? k - p0 : kSweepBlock);
+        sweep_panel_kernel<<<ew_grid(k * bs, sms), 256, 0, s>>>(A, k, p0, bs, P);
+        sweep_block_inverse_kernel<<<1, 256, 0, s>>>(P, p0, bs, D);
+        if ((e = sgemm(false, false, k, bs, bs, 1.f, P, bs, D, bs, 0.f, nullptr, 0, E, bs, s)) != cudaSuccess) return e;
+        if ((e = sgemm(false, true, k, k, bs, -1.f, E, bs, P, bs, 1.f, A, k, A, k, s)) != cudaSuccess) return e;
+        sweep_fixup_kernel<<<ew_grid(k * bs, sms), 256, 0, s>>>(A, k, p0, bs, E, D);
+    }
+    return cudaGetLastError();
+}
+
+// ---- workspace --------------------------------------------------------------
+struct FactorWs {
+    float *Zu, *Zv, *C, *Lam, *X, *Rhs, *G, *P, *E, *D;
+    float *a, *m1, *m2, *b, *rho;
+    double *sumsq;   // [outer + 1]
+    void *svid;
+    size_t bytes;
+};
+
+FactorWs carve(void *base, int64_t n, int64_t m, int64_t k, int outer, int svid_iters)
+{
+    FactorWs w{};
+    char *p = static_cast<char *>(base);
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        char *q = p ? p + off : nullptr;
+        off += align_up(bytes, 256);
+        return q;
+    };
+    const size_t nk = static_cast<size_t>(n) * k, km = static_cast<size_t>(k) * m;
+    const size_t mx = nk > km ? nk : km;
+    w.Zu = reinterpret_cast<float *>(take(nk * 4));
+    w.Zv = reinterpret_cast<float *>(take(km * 4));
+    w.C = reinterpret_cast<float *>(take(mx * 4));
+    w.Lam = reinterpret_cast<float *>(take(mx * 4));
+    w.X = reinterpret_cast<float *>(take(mx * 4));
+    w.Rhs = reinterpret_cast<float *>(take(mx * 4));
+    w.G = reinterpret_cast<float *>(take(static_cast<size_t>(k) * k * 4));
+    w.P = reinterpret_cast<float *>(take(static_cast<size_t>(k) * kSweepBlock * 4));
+    w.E = reinterpret_cast<float *>(take(static_cast<size_t>(k) * kSweepBlock * 4));
+    w.D = reinterpret_cast<float *>(take(kSweepBlock * kSweepBlock * 4));
+    w.a = reinterpret_cast<float *>(take(static_cast<size_t>(n) * 4));
+    w.m1 = reinterpret_cast<float *>(take(static_cast<size_t>(k) * 4));
+    w.m2 = reinterpret_cast<float *>(take(static_cast<size_t>(k) * 4));
+    w.b = reinterpret_cast<float *>(take(static_cast<size_t>(m) * 4));
+    w.rho = reinterpret_cast<float *>(take(4));
+    w.sumsq = reinterpret_cast<double *>(take(static_cast<size_t>(outer + 1) * 8));
+    w.svid = take(svid_scratch_bytes(n > k ? n : k, k > m ? k : m, svid_iters));
+    w.bytes = off;
+    return w;
+}
+
+}  // namespace
+
+size_t factorize_workspace_bytes(int64_t n, int64_t m, int64_t k, int outer, int svid_iters)
+{
+    return carve(nullptr, n, m, k, outer, svid_iters).bytes;
+}
+
+cudaError_t factorize_run(const float *W, int64_t n, int64_t m, int64_t k, const float *U0, const float *V0,
+                          int outer, int admm_iters, int svid_iters, float rho_rel, uint32_t *A_packed,
+                          uint32_t *B_packed, uint16_t *alpha, uint16_t *beta, uint16_t *gamma, float *objective,
+                          void *ws, cudaStream_t s)
+{
+    const FactorWs w = carve(ws, n, m, k, outer, svid_iters);
+    const int sms = sm_count();
+    const int64_t nk = n * k, km = k * m;
+    cudaError_t e;
+    // project the start onto the constraint set: Zu = SVID(U0), Zv = SVID(V0)
+    auto project = [&](int64_t rows, int64_t cols, float *p, float *q, float *Z) -> cudaError_t {
+        cudaError_t r = svid_power(w.X, rows, cols, svid_iters, nullptr, nullptr, p, q, w.svid, s);
+        if (r != cudaSuccess) return r;
+        project_kernel<<<ew_grid(rows * cols, sms), 256, 0, s>>>(w.X, rows, cols, p, q, Z, w.Lam);
+        return cudaGetLastError();
+    };
+    auto objective_at = [&](int slot) -> cudaError_t {
+        if (!objective) return cudaSuccess;
+        cudaError_t r = sgemm(false, false, n, m, k, -1.f, w.Zu, k, w.Zv, m, 1.f, W, m, nullptr, 0, s, w.sumsq + slot);
+        if (r != cudaSuccess) return r;
+        objective_kernel<<<1, 1, 0, s>>>(w.sumsq + slot, objective + slot);
+        return cudaGetLastError();
+    };
+    if ((e = cudaMemsetAsync(w.sumsq, 0, static_cast<size_t>(outer + 1) * 8, s)) != cudaSuccess) return e;
+    if ((e = cudaMemcpyAsync(w.X, U0, nk * 4, cudaMemcpyDeviceToDevice, s)) != cudaSuccess) return e;
+    if ((e = project(n, k, w.a, w.m1, w.Zu)) != cudaSuccess) return e;
+    if (outer == 0 && (e = launch_pack_ld(w.X, DBF_F32, n, k, A_packed, pitch_words(k), nullptr, s)) != cudaSuccess)
+        return e;
+    if ((e = cudaMemcpyAsync(w.X, V0, km * 4, cudaMemcpyDeviceToDevice, s)) != cudaSuccess) return e;
+    if ((e = project(k, m, w.m2, w.b, w.Zv)) != cudaSuccess) return e;
+    if (outer == 0 && (e = launch_pack_ld(w.X, DBF_F32, k, m, B_packed, pitch_words(m), nullptr, s)) != cudaSuccess)
+        return e;
+    if ((e = objective_at(0)) != cudaSuccess) return e;
+
+    for (int t = 0; t < outer; ++t) {
+        const bool last = t + 1 == outer;
+        // U-subproblem: C = W Zv^T, G = Zv Zv^T + rho I, G <- -G^-1
+        if ((e = sgemm(false, true, n, k, m, 1.f, W, m, w.Zv, m, 0.f, nullptr, 0, w.C, k, s)) != cudaSuccess) return e;
+        if ((e = sgemm(false, true, k, k, m, 1.f, w.Zv, m, w.Zv, m, 0.f, nullptr, 0, w.G, k, s)) != cudaSuccess)
+            return e;
+        rho_kernel<<<1, 256, 0, s>>>(w.G, k, rho_rel, w.rho);
+        if ((e = sweep_inverse(w.G, k, w.P, w.E, w.D, sms, s)) != cudaSuccess) return e;
+        if ((e = cudaMemsetAsync(w.Lam, 0, nk * 4, s)) != cudaSuccess) return e;
+        for (int j = 0; j < admm_iters; ++j) {
+            rhs_kernel<<<ew_grid(nk, sms), 256, 0, s>>>(w.C, w.Zu, w.Lam, w.rho, nk, w.Rhs);
+            // X = U + Lam = -(Rhs G) + Lam
+            if ((e = sgemm(false, false, n, k, k, -1.f, w.Rhs, k, w.G, k, 1.f, w.Lam, k, w.X, k, s)) != cudaSuccess)
+                return e;
+            if ((e = project(n, k, w.a, w.m1, w.Zu)) != cudaSuccess) return e;
+        }
+        if (last && (e = launch_pack_ld(w.X, DBF_F32, n, k, A_packed, pitch_words(k), nullptr, s)) != cudaSuccess)
+            return e;
+        // V-subproblem: C = Zu^T W, G = Zu^T Zu + rho I, G <- -G^-1
+        if ((e = sgemm(true, false, k, m, n, 1.f, w.Zu, k, W, m, 0.f, nullptr, 0, w.C, m, s)) != cudaSuccess) return e;
+        if ((e = sgemm(true, false, k, k, n, 1.f, w.Zu, k, w.Zu, k, 0.f, nullptr, 0, w.G, k, s)) != cudaSuccess)
+            return e;
+        rho_kernel<<<1, 256, 0, s>>>(w.G, k, rho_rel, w.rho);
+        if ((e = sweep_inverse(w.G, k, w.P, w.E, w.D, sms, s)) != cudaSuccess) return e;
+        if ((e = cudaMemsetAsync(w.Lam, 0, km * 4, s)) != cudaSuccess) return e;
+        for (int j = 0; j < admm_iters; ++j) {
+            rhs_kernel<<<ew_grid(km, sms), 256, 0, s>>>(w.C, w.Zv, w.Lam, w.rho, km, w.Rhs);
+            // X = V + Lam = -(G Rhs) + Lam
+            if ((e = sgemm(false, false, k, m, k, -1.f, w.G, k, w.Rhs, m, 1.f, w.Lam, m, w.X, m, s)) != cudaSuccess)
+                return e;
+            if ((e = project(k, m, w.m2, w.b, w.Zv)) != cudaSuccess) return e;
+        }
+        if (last && (e = launch_pack_ld(w.X, DBF_F32, k, m, B_packed, pitch_words(m), nullptr, s)) != cudaSuccess)
+            return e;
+        if ((e = objective_at(t + 1)) != cudaSuccess) return e;
+    }
+    factor_scales_kernel<<<ew_grid(n + k + m, sms), 256, 0, s>>>(w.a, n, w.m1, w.m2, k, w.b, m, alpha, beta, gamma);
+    return cudaGetLastError();
+}
+
+}  // namespace dbf

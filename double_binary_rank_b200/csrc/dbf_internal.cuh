@@ -23,6 +23,9 @@ __host__ __device__ inline int64_t pitch_words(int64_t k) { return (k + 31) / 32
 // ---- launchers (each returns the first CUDA error it meets) --------------
 cudaError_t launch_pack(const void *src, dbf_dtype dt, int64_t rows, int64_t k, uint32_t *dst,
                         int32_t *status, cudaStream_t s);
+// the same with a destination row stride of dst_ld >= pitch_words(k) words
+cudaError_t launch_pack_ld(const void *src, dbf_dtype dt, int64_t rows, int64_t k, uint32_t *dst,
+                           int64_t dst_ld, int32_t *status, cudaStream_t s);
 cudaError_t launch_unpack(const uint32_t *src, int64_t rows, int64_t k, int8_t *dst,
                           cudaStream_t s);
 cudaError_t launch_transpose(const uint32_t *src, int64_t rows, int64_t k, uint32_t *dst,
@@ -56,8 +59,18 @@ cudaError_t mbok_forward(int M, int N, int K, const uint32_t *w_packed, const ui
 
 // SVID (sign times the best rank-1 fit of the magnitudes), by power iteration
 size_t svid_scratch_bytes(int64_t n, int64_t m, int iters);
+// the power iteration alone: fp16 and/or fp32 scale outputs (null ones skipped)
+cudaError_t svid_power(const float *X, int64_t n, int64_t m, int iters, uint16_t *s_out, uint16_t *s_in,
+                       float *s_out32, float *s_in32, void *scratch, cudaStream_t s);
 cudaError_t svid_run(float *X, int64_t n, int64_t m, int iters, int subtract, uint32_t *signs,
                      int64_t signs_ld, uint16_t *s_out, uint16_t *s_in, void *scratch, cudaStream_t s);
+
+// DBF factorisation (alternating ADMM with the SVID projection, fp32)
+size_t factorize_workspace_bytes(int64_t n, int64_t m, int64_t k, int outer, int svid_iters);
+cudaError_t factorize_run(const float *W, int64_t n, int64_t m, int64_t k, const float *U0, const float *V0,
+                          int outer, int admm_iters, int svid_iters, float rho_rel, uint32_t *A_packed,
+                          uint32_t *B_packed, uint16_t *alpha, uint16_t *beta, uint16_t *gamma, float *objective,
+                          void *ws, cudaStream_t s);
 
 // prefill path (tcgen05)
 bool gemm_shape_ok(const dbf_layer &L);

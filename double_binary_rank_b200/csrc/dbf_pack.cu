@@ -43,27 +43,52 @@ __device__ __forceinline__ bool is_negative<__nv_bfloat16>(__nv_bfloat16 v, bool
     return f < 0.0f;
 }
 
+// A work item is a run of up to kPackSeg words of one row (one division per
+// item, not per word); the warp issues the loads of U words before their
+// ballots so U row segments are in flight at once. Lane u < U stores word u.
+constexpr int kPackSeg = 64;
+
 template <typename T>
 __global__ void __launch_bounds__(256) pack_kernel(const T *__restrict__ src, int64_t rows,
                                                    int64_t k, uint32_t *__restrict__ dst,
-                                                   int32_t *status)
+                                                   int64_t dst_ld, int32_t *status)
 {
+    constexpr int U = sizeof(T) == 1 ? 8 : 4;
     const int lane = threadIdx.x & 31;
     const int64_t pitch = pitch_words(k);
-    const int64_t total = rows * pitch;
+    const int64_t segs = (pitch + kPackSeg - 1) / kPackSeg;
+    const int64_t total = rows * segs;
     const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
     const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
     // column of this lane inside a 32-column word
     const int col = lane < 16 ? 2 * lane : 2 * (lane - 16) + 1;
     bool saw_nan = false;
-    for (int64_t w = warp; w < total; w += nwarps) {
-        const int64_t row = w / pitch;
-        const int64_t c = (w - row * pitch) * 32 + col;
-        bool neg = false, nan = false;
-        if (c < k) neg = is_negative<T>(src[row * k + c], nan);
-        saw_nan |= nan;
-        const uint32_t word = __ballot_sync(0xffffffffu, neg);
-        if (lane == 0) dst[w] = word;
+    for (int64_t item = warp; item < total; item += nwarps) {
+        const int64_t row = item / segs;
+        const int64_t w0 = (item - row * segs) * kPackSeg;
+        const int64_t w1 = w0 + kPackSeg < pitch ? w0 + kPackSeg : pitch;
+        const T *rp = src + row * k;
+        uint32_t *dp = dst + row * dst_ld;
+        for (int64_t w = w0; w < w1; w += U) {
+            T v[U];
+            bool ok[U];
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int64_t c = (w + u) * 32 + col;
+                ok[u] = w + u < w1 && c < k;
+                v[u] = ok[u] ? rp[c] : T();
+            }
+            uint32_t mine = 0u;
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                bool nan = false, neg = false;
+                if (ok[u]) neg = is_negative<T>(v[u], nan);
+                saw_nan |= nan;
+                const uint32_t word = __ballot_sync(0xffffffffu, neg);
+                if (lane == u) mine = word;
+            }
+            if (lane < U && w + lane < w1) dp[w + lane] = mine;
+        }
     }
     if (saw_nan && status) atomicExch(status, static_cast<int32_t>(DBF_ERR_INVALID_ARG));
 }
@@ -166,21 +191,27 @@ int grid_for(int64_t work, int per_block)
 cudaError_t launch_pack(const void *src, dbf_dtype dt, int64_t rows, int64_t k, uint32_t *dst,
                         int32_t *status, cudaStream_t s)
 {
-    const int64_t words = rows * pitch_words(k);
-    const int grid = grid_for(words, 8);   // 8 warps per block, one word each per step
+    return launch_pack_ld(src, dt, rows, k, dst, pitch_words(k), status, s);
+}
+
+cudaError_t launch_pack_ld(const void *src, dbf_dtype dt, int64_t rows, int64_t k, uint32_t *dst,
+                           int64_t dst_ld, int32_t *status, cudaStream_t s)
+{
+    const int64_t items = rows * ((pitch_words(k) + kPackSeg - 1) / kPackSeg);
+    const int grid = grid_for(items, 8);   // 8 warps per block, one item each per step
     switch (dt) {
     case DBF_I8:
-        pack_kernel<int8_t><<<grid, 256, 0, s>>>(static_cast<const int8_t *>(src), rows, k, dst, status);
+        pack_kernel<int8_t><<<grid, 256, 0, s>>>(static_cast<const int8_t *>(src), rows, k, dst, dst_ld, status);
         break;
     case DBF_F32:
-        pack_kernel<float><<<grid, 256, 0, s>>>(static_cast<const float *>(src), rows, k, dst, status);
+        pack_kernel<float><<<grid, 256, 0, s>>>(static_cast<const float *>(src), rows, k, dst, dst_ld, status);
         break;
     case DBF_F16:
-        pack_kernel<__half><<<grid, 256, 0, s>>>(static_cast<const __half *>(src), rows, k, dst, status);
+        pack_kernel<__half><<<grid, 256, 0, s>>>(static_cast<const __half *>(src), rows, k, dst, dst_ld, status);
         break;
     case DBF_BF16:
         pack_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(static_cast<const __nv_bfloat16 *>(src), rows, k,
-                                                        dst, status);
+                                                        dst, dst_ld, status);
         break;
     default:
         return cudaErrorInvalidValue;

@@ -158,6 +158,43 @@ dbf_status dbf_svid(float *X, int64_t n, int64_t m, int32_t iters, int subtract,
                     int64_t signs_ld_words, uint16_t *s_out, uint16_t *s_in, void *scratch,
                     size_t scratch_bytes, void *stream);
 
+/* Double binary factorisation of a dense fp32 weight W (n x m, row-major):
+ * W ~ (a . A . mid^T)(B . b^T) with sign matrices A (n x k), B (k x m) and
+ * scale vectors a [n], mid [k], b [m] (DBF page, section 2: the
+ * factorisation by alternating minimisation with ADMM and the SVID
+ * projection; the page gives no update formulas, and this is the plainest
+ * reading, unweighted). With U = diag(a) A diag(m1), V = diag(m2) B diag(b),
+ * mid = m1 . m2, each outer iteration runs admm_iters scaled-form ADMM steps
+ * on U with V fixed,
+ *     U <- (W V^T + rho (Z - L)) (V V^T + rho I)^-1,
+ *     Z <- SVID(U + L),  L <- L + U - Z     (Z from the current U, L = 0),
+ * the factor becoming Z, then the same on V with U fixed (operands
+ * transposed); rho = rho_rel * trace(Gram) / k; SVID as in dbf_svid with
+ * svid_iters power iterations.
+ * W [n x m], U0 [n x k], V0 [k x m]: device fp32, row-major, read only; the
+ *    start is the SVID projection of (U0, V0) (e.g. a truncated SVD split
+ *    evenly, or any seeded matrices).
+ * outer >= 0 (0 returns the projected start), admm_iters >= 1,
+ *    1 <= svid_iters <= 1000, rho_rel > 0.
+ * Outputs (device, caller-owned): a_signs = A packed (n rows of ceil(k/32)
+ *    words), b_signs = B packed (k rows of ceil(m/32) words), fp16 alpha = a
+ *    [n], beta = mid [k], gamma = b [m]: exactly a one-envelope dbf_layer
+ *    with M = m, N = n, R = k (b1 = a_signs, b2 = b_signs).
+ * objective: optional device fp32 [outer + 1]: |W - U V|_F of the projected
+ *    start and after each outer iteration (fp32 scales; costs one n x m x k
+ *    product per entry). NULL skips it.
+ * ws: dbf_factorize_workspace_bytes(n, m, k, outer, svid_iters) bytes,
+ *    256-byte aligned, scratch. Arithmetic is fp32 (products accumulated in
+ *    fp32; the k x k inverse by an in-place blocked Gauss-Jordan sweep).
+ * U0 and V0 must not be zero (a zero Gram matrix gives rho = 0 and NaN).
+ * Errors: DBF_ERR_INVALID_ARG, DBF_ERR_ALIGNMENT, DBF_ERR_WORKSPACE,
+ *    DBF_ERR_UNSUPPORTED (a dimension above 65535 * 128), DBF_ERR_CUDA. */
+size_t dbf_factorize_workspace_bytes(int64_t n, int64_t m, int64_t k, int32_t outer, int32_t svid_iters);
+dbf_status dbf_factorize(const float *W, int64_t n, int64_t m, int64_t k, const float *U0, const float *V0,
+                         int32_t outer, int32_t admm_iters, int32_t svid_iters, float rho_rel,
+                         uint32_t *a_signs, uint32_t *b_signs, uint16_t *alpha, uint16_t *beta,
+                         uint16_t *gamma, float *objective, void *ws, size_t ws_bytes, void *stream);
+
 /* Smallest T for which DBF_PATH_AUTO takes the GEMM path on a shape it allows. */
 int64_t dbf_gemm_min_tokens(void);
 

@@ -330,3 +330,6 @@ def f32_to_f64(bits: np.ndarray) -> np.ndarray:
     lib = _load()
     b = np.asarray(bits, dtype=np.uint32)
     return np.array([lib.dbf_oracle_f32_to_f64(int(v)) for v in b.ravel()]).reshape(b.shape)
+
+
+from .dbf_factorize import Factors, admm_u_step, admm_v_step, factorize, rho_of, svd_init, svid_project  # noqa: E402

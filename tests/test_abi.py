@@ -216,3 +216,32 @@ def test_segmented_planned_rejects_bad_tables(lib):
     z = np.array([0], dtype=np.int32)
     assert f(arr2, 1, np.array([0, 4], dtype=np.int32).ctypes.data, z.ctypes.data, 1, 60, 48, 0x1000, dbf.BF16,
              0x1000, dbf.F32, 4, 0, 0x1000, 1 << 30, None) == dbf.ERR_ALIGNMENT
+
+
+def test_factorize_rejects_bad_arguments(lib):
+    import double_binary_rank_b200 as dbf
+    f = lib.dbf_factorize
+    q = lib.dbf_factorize_workspace_bytes
+    p = 0x1000
+    n, m, k = 96, 80, 40
+    need = q(n, m, k, 3, 24)
+    assert need > 4 * (n * k + k * m + 4 * max(n * k, k * m) + k * k)
+    assert q(n, m, k, 3, 0) == 0 and q(0, m, k, 3, 24) == 0 and q(n, m, k, -1, 24) == 0
+    assert q(1 << 24, m, k, 1, 24) == 0
+    args = lambda **kw: dict(dict(W=p, n=n, m=m, k=k, U0=p, V0=p, outer=3, admm=4, svid=24, rho=1.0, A=p, B=p,
+                                  al=p, be=p, ga=p, obj=p, ws=p, wsb=need), **kw)
+    call = lambda a: f(a["W"], a["n"], a["m"], a["k"], a["U0"], a["V0"], a["outer"], a["admm"], a["svid"], a["rho"],
+                       a["A"], a["B"], a["al"], a["be"], a["ga"], a["obj"], a["ws"], a["wsb"], None)
+    assert call(args(W=None)) == dbf.ERR_INVALID_ARG
+    assert call(args(admm=0)) == dbf.ERR_INVALID_ARG
+    assert call(args(svid=0)) == dbf.ERR_INVALID_ARG
+    assert call(args(rho=0.0)) == dbf.ERR_INVALID_ARG
+    assert call(args(rho=float("nan"))) == dbf.ERR_INVALID_ARG
+    assert call(args(rho=float("inf"))) == dbf.ERR_INVALID_ARG
+    assert call(args(outer=-1)) == dbf.ERR_INVALID_ARG
+    assert call(args(n=1 << 24)) == dbf.ERR_UNSUPPORTED
+    assert call(args(W=p + 2)) == dbf.ERR_ALIGNMENT
+    assert call(args(obj=p + 2)) == dbf.ERR_ALIGNMENT
+    assert call(args(wsb=need - 1)) == dbf.ERR_WORKSPACE
+    assert call(args(ws=None)) == dbf.ERR_WORKSPACE
+    assert call(args(ws=p + 16)) == dbf.ERR_ALIGNMENT

@@ -15,8 +15,10 @@ def dbf():
     return m
 
 
+# rows of 1..2188 packed words: several 64-word runs per row, ragged runs and
+# a ragged last word
 SHAPES = [(1, 1), (1, 31), (3, 32), (5, 33), (17, 100), (16, 5888), (64, 4096), (4096, 64),
-          (256, 16), (37, 1000)]
+          (256, 16), (37, 1000), (3, 4136), (2, 2100), (7, 70000)]
 
 
 @pytest.mark.parametrize("shape", SHAPES)
@@ -30,10 +32,11 @@ def test_pack_int8_bitexact(dbf, shape):
     assert np.array_equal(back, s)
 
 
+@pytest.mark.parametrize("cols", [77, 4136])
 @pytest.mark.parametrize("dtype", [torch.float32, torch.float16, torch.bfloat16])
-def test_pack_latents_sign_convention(dbf, dtype):
+def test_pack_latents_sign_convention(dbf, dtype, cols):
     rng = np.random.default_rng(5)
-    h = rng.standard_normal((9, 77)).astype(np.float32)
+    h = rng.standard_normal((9, cols)).astype(np.float32)
     h[0, :6] = [0.0, -0.0, 1e-3, -1e-3, 5.0, -5.0]
     ht = torch.from_numpy(h).to(dtype)
     hq = ht.float().numpy()                    # the values the kernel sees

@@ -27,7 +27,10 @@ def unpack_np(words, rows, k):
     return oracle.unpack(np.ascontiguousarray(words.cpu().numpy()).view(np.uint32).reshape(-1), rows, k)
 
 
-@pytest.mark.parametrize("n,m", [(300, 200), (1024, 4096), (77, 1000)])
+# single-read kernel with 4, 8 and 12 float4 columns per thread (m % 4 == 0,
+# m <= 12288, ragged last band); two-pass kernels for m % 4 != 0 and m > 12288
+@pytest.mark.parametrize("n,m", [(300, 200), (1024, 4096), (77, 1000), (64, 5000), (40, 9000), (1, 12288),
+                                 (129, 1001), (33, 12300)])
 def test_svid_matches_oracle(dbf, n, m):
     rng = np.random.default_rng(n + m)
     X = rng.standard_normal((n, m)).astype(np.float32)
