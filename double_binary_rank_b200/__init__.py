@@ -332,7 +332,8 @@ def forward_segmented_planned(layers, seg_offsets, seg_adapter, x: torch.Tensor,
 
 
 def svid(X: torch.Tensor, iters: int = 24, subtract: bool = False, signs: Optional[torch.Tensor] = None,
-         s_out: Optional[torch.Tensor] = None, s_in: Optional[torch.Tensor] = None, stream=None):
+         s_out: Optional[torch.Tensor] = None, s_in: Optional[torch.Tensor] = None,
+         scratch: Optional[torch.Tensor] = None, stream=None):
     """X ~ sign(X) . (s_out s_in^T) (dbf_svid). X: fp32 [n, m] on the device,
     replaced by the residual when subtract. Returns (packed signs, s_out, s_in)."""
     assert X.dtype == torch.float32 and X.is_contiguous()
@@ -344,7 +345,8 @@ def svid(X: torch.Tensor, iters: int = 24, subtract: bool = False, signs: Option
         s_out = torch.empty(n, dtype=torch.float16, device=dev)
     if s_in is None:
         s_in = torch.empty(m, dtype=torch.float16, device=dev)
-    scratch = alloc_workspace(int(_lib.dbf_svid_scratch_bytes(n, m, iters)), dev)
+    if scratch is None:
+        scratch = alloc_workspace(int(_lib.dbf_svid_scratch_bytes(n, m, iters)), dev)
     _check(_lib.dbf_svid(_ptr(X), n, m, iters, int(subtract), _ptr(signs), signs.stride(0), _ptr(s_out), _ptr(s_in),
                          _ptr(scratch), scratch.numel(), _stream(stream)), "dbf_svid")
     return signs, s_out, s_in

@@ -111,7 +111,7 @@ dbf_status dbf_svid(float *X, int64_t n, int64_t m, int32_t iters, int subtract,
 }
 
 namespace {
-constexpr int64_t kFactorMaxDim = int64_t(65535) * 128;   // GEMM grid rows of 128 stay <= 65535
+constexpr int64_t kFactorMaxDim = int64_t(65535) * 32;   // transpose grids of 32-row tiles stay <= 65535
 
 bool factor_args_ok(int64_t n, int64_t m, int64_t k, int32_t outer, int32_t svid_iters)
 {

@@ -13,15 +13,18 @@
 //   rho = rho_rel * trace(Gram) / k.
 //
 // Work per outer iteration (k x k Gram and inverse, n x k and k x m
-// right-hand sides) is dense fp32 contraction: a register-tiled SIMT GEMM
-// (128 x 128 tiles, 8 x 8 outputs per thread, double-buffered shared
-// memory) does all of it, including the rank-64 updates of the blocked
-// inverse. The inverse of the SPD matrix V V^T + rho I is an in-place
-// blocked sweep (Gauss-Jordan without pivoting, stable for SPD): per 64-wide
-// pivot block, the block's inverse D (one CTA), E = P D with P the block
-// column, A -= E P^T, then the block row / column / diagonal are set to E^T,
-// E and -D; after all blocks A holds -(V V^T + rho I)^-1. The SVID
-// projection is the library's power iteration (fp32 scales).
+// right-hand sides) is dense fp32 contraction, every product written as
+// A B^T of K-major operands (the V-subproblem runs on V^T; W^T, U^T and V
+// come from transposes): on the tensor cores as three TF32 products per
+// operand pair when the operands allow (dbf_tf32.cu), else on a
+// register-tiled SIMT GEMM (128 x 128 tiles, 8 x 8 outputs per thread,
+// double-buffered shared memory). The inverse of the SPD matrix
+// V V^T + rho I is an in-place blocked sweep (Gauss-Jordan without
+// pivoting, stable for SPD): per 128-wide pivot block, the block's inverse
+// D (one CTA), E = P D with P the block column, A -= E P^T, then the block
+// row / column / diagonal are set to E^T, E and -D; after all blocks A holds
+// -(V V^T + rho I)^-1. The SVID projection is the library's power
+// iteration (fp32 scales).
 #include "dbf_internal.cuh"
 
 namespace dbf {
@@ -212,8 +215,52 @@ cudaError_t sgemm(bool ta, bool tb, int64_t M, int64_t N, int64_t K, float alpha
     return cudaGetLastError();
 }
 
+// out [cols x rows] = in [rows x cols]^T, 32 x 32 tiles through shared memory
+__global__ void __launch_bounds__(256) transpose_f32_kernel(const float *__restrict__ in, int64_t rows, int64_t cols,
+                                                            float *__restrict__ out)
+{
+    __shared__ float tile[32][33];
+    const int64_t c0 = static_cast<int64_t>(blockIdx.x) * 32, r0 = static_cast<int64_t>(blockIdx.y) * 32;
+    const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;   // 32 x 8 threads
+    for (int r = ty; r < 32; r += 8)
+        if (r0 + r < rows && c0 + tx < cols) tile[r][tx] = in[(r0 + r) * cols + c0 + tx];
+    __syncthreads();
+    for (int c = ty; c < 32; c += 8)
+        if (c0 + c < cols && r0 + tx < rows) out[(c0 + c) * rows + r0 + tx] = tile[tx][c];
+}
+
+cudaError_t transpose_f32(const float *in, int64_t rows, int64_t cols, float *out, cudaStream_t s)
+{
+    const dim3 grid(static_cast<unsigned>((cols + 31) / 32), static_cast<unsigned>((rows + 31) / 32));
+    transpose_f32_kernel<<<grid, 256, 0, s>>>(in, rows, cols, out);
+    return cudaGetLastError();
+}
+
+// Scratch for the lo planes of the tensor-core path.
+struct LoScratch {
+    float *p;
+    size_t floats;
+};
+
+// Cout[M x N] = alpha A B^T + beta Cin with A [M x K], B [N x K] (both
+// K-major): the tensor-core path (three TF32 products) when the operands
+// qualify, K fills at least one pipeline stage and the scratch holds the lo
+// planes, else the SIMT GEMM.
+cudaError_t gemm_nt(int64_t M, int64_t N, int64_t K, float alpha, const float *A, int64_t lda, const float *B,
+                    int64_t ldb, float beta, const float *Cin, int64_t ldci, float *Cout, int64_t ldco, cudaStream_t s,
+                    const LoScratch &lo, double *sumsq = nullptr, int32_t *status = nullptr)
+{
+    if (M <= 0 || N <= 0) return cudaSuccess;
+    if (K >= 32 && tf32x3_ok(M, N, K, A, lda, B, ldb) && lo.p && lo.floats >= tf32x3_scratch_floats(M, N, K))
+        return tf32x3_gemm(M, N, K, alpha, A, lda, B, ldb, beta, Cin, ldci, Cout, ldco, sumsq, status, lo.p, lo.floats,
+                           s);
+    return sgemm(false, true, M, N, K, alpha, A, lda, B, ldb, beta, Cin, ldci, Cout, ldco, s, sumsq);
+}
+
 // ---- blocked sweep inverse of an SPD matrix ---------------------------------
-constexpr int kSweepBlock = 64;
+constexpr int kSweepBlock = 128;
+constexpr int kSweepSeg = 16;                                         // columns per thread
+constexpr int kSweepThreads = kSweepBlock * kSweepBlock / kSweepSeg;   // 1024: 8 threads per row
 
 // P = A[:, p0 : p0 + bs] (k x bs, ld bs)
 __global__ void sweep_panel_kernel(const float *__restrict__ A, int64_t k, int64_t p0, int bs, float *__restrict__ P)
@@ -226,37 +273,64 @@ __global__ void sweep_panel_kernel(const float *__restrict__ A, int64_t k, int64
     }
 }
 
-// D = T^-1 for the bs x bs SPD block T = P[p0 : p0 + bs, :], by the scalar
-// sweep in shared memory (pivot p: T_ij -= T_ip T_pj / T_pp for i, j != p,
-// then T_ip *= 1 / T_pp, T_pj *= 1 / T_pp, T_pp = -1 / T_pp; after every
-// pivot T = -(original T)^-1). One CTA.
-__global__ void __launch_bounds__(256) sweep_block_inverse_kernel(const float *__restrict__ P, int64_t p0, int bs,
-                                                                  float *__restrict__ D)
+// D = T^-1 for the bs x bs SPD block T = P[p0 : p0 + bs, :] (bs <= 128), by
+// the scalar sweep (pivot p: T_ij -= T_ip T_pj / T_pp for i, j != p, then
+// T_ip *= 1 / T_pp, T_pj *= 1 / T_pp, T_pp = -1 / T_pp; after every pivot
+// T = -(original T)^-1). One CTA; thread t holds row t / 8, columns
+// 16 (t % 8) .. + 15 in registers. Per pivot the owners publish row p and
+// column p in shared memory; every element takes the general update
+// T_ij - (T_ip / T_pp) T_pj (which leaves row p and column p at zero), then
+// row p and column p are set.
+__global__ void __launch_bounds__(kSweepThreads) sweep_block_inverse_kernel(const float *__restrict__ P, int64_t p0,
+                                                                            int bs, float *__restrict__ D)
 {
-    __shared__ float T[kSweepBlock][kSweepBlock + 1];
-    __shared__ float colp[kSweepBlock], rowp[kSweepBlock];
+    __shared__ __align__(16) float rowp[kSweepBlock];
+    __shared__ float colp[kSweepBlock];
     const int tid = threadIdx.x;
-    for (int idx = tid; idx < bs * bs; idx += blockDim.x) T[idx / bs][idx % bs] = P[(p0 + idx / bs) * bs + idx % bs];
-    __syncthreads();
+    const int i = tid / (kSweepBlock / kSweepSeg), j0 = (tid % (kSweepBlock / kSweepSeg)) * kSweepSeg;
+    float t[kSweepSeg];
+#pragma unroll
+    for (int e = 0; e < kSweepSeg; ++e) t[e] = (i < bs && j0 + e < bs) ? P[(p0 + i) * bs + j0 + e] : 0.f;
     for (int p = 0; p < bs; ++p) {
-        if (tid < bs) {
-            colp[tid] = T[tid][p];
-            rowp[tid] = T[p][tid];
+        if (i == p) {
+#pragma unroll
+            for (int e = 0; e < kSweepSeg; ++e) rowp[j0 + e] = t[e];
+        }
+        if (p >= j0 && p < j0 + kSweepSeg) {
+            float v = 0.f;
+#pragma unroll
+            for (int e = 0; e < kSweepSeg; ++e)
+                if (j0 + e == p) v = t[e];
+            colp[i] = v;
         }
         __syncthreads();
         const float d = 1.0f / colp[p];
-        for (int idx = tid; idx < bs * bs; idx += blockDim.x) {
-            const int i = idx / bs, j = idx % bs;
-            float v;
-            if (i != p && j != p) v = T[i][j] - colp[i] * d * rowp[j];
-            else if (i == p && j == p) v = -d;
-            else if (j == p) v = colp[i] * d;
-            else v = d * rowp[j];
-            T[i][j] = v;
+        const float cid = colp[i] * d;
+        float r[kSweepSeg];
+#pragma unroll
+        for (int e = 0; e < kSweepSeg; e += 4) {
+            const float4 q = *reinterpret_cast<const float4 *>(&rowp[j0 + e]);
+            r[e] = q.x;
+            r[e + 1] = q.y;
+            r[e + 2] = q.z;
+            r[e + 3] = q.w;
         }
-        __syncthreads();
+#pragma unroll
+        for (int e = 0; e < kSweepSeg; ++e) t[e] = fmaf(-cid, r[e], t[e]);
+        if (i == p) {
+#pragma unroll
+            for (int e = 0; e < kSweepSeg; ++e) t[e] = d * r[e];
+        }
+        if (p >= j0 && p < j0 + kSweepSeg) {
+#pragma unroll
+            for (int e = 0; e < kSweepSeg; ++e)
+                if (j0 + e == p) t[e] = i == p ? -d : cid;
+        }
+        __syncthreads();   // row p and column p are read before the next pivot rewrites them
     }
-    for (int idx = tid; idx < bs * bs; idx += blockDim.x) D[idx] = -T[idx / bs][idx % bs];
+#pragma unroll
+    for (int e = 0; e < kSweepSeg; ++e)
+        if (i < bs && j0 + e < bs) D[i * bs + j0 + e] = -t[e];
 }
 
 // After A -= E P^T: the pivot block column and row become E and E^T, the
@@ -362,25 +436,35 @@ int ew_grid(int64_t count, int sms)
 }
 
 // A (k x k, SPD) <- -A^-1 in place. Scratch: P, E (k x kSweepBlock), D.
-cudaError_t sweep_inverse(float *A, int64_t k, float *P, float *E, float *D, int sms, cudaStream_t s)
+cudaError_t sweep_inverse(float *A, int64_t k, float *P, float *E, float *D, int sms, const LoScratch &lo,
+                          int32_t *status, cudaStream_t s)
 {
     cudaError_t e;
     for (int64_t p0 = 0; p0 < k; p0 += kSweepBlock) {
         const int bs = static_cast<int>(k - p0 < kSweepBlock ? k - p0 : kSweepBlock);
         sweep_panel_kernel<<<ew_grid(k * bs, sms), 256, 0, s>>>(A, k, p0, bs, P);
-        sweep_block_inverse_kernel<<<1, 256, 0, s>>>(P, p0, bs, D);
-        if ((e = sgemm(false, false, k, bs, bs, 1.f, P, bs, D, bs, 0.f, nullptr, 0, E, bs, s)) != cudaSuccess) return e;
-        if ((e = sgemm(false, true, k, k, bs, -1.f, E, bs, P, bs, 1.f, A, k, A, k, s)) != cudaSuccess) return e;
+        sweep_block_inverse_kernel<<<1, kSweepThreads, 0, s>>>(P, p0, bs, D);
+        // E = P D (D symmetric: P D^T), then A -= E P^T
+        if ((e = gemm_nt(k, bs, bs, 1.f, P, bs, D, bs, 0.f, nullptr, 0, E, bs, s, lo, nullptr, status)) != cudaSuccess)
+            return e;
+        if ((e = gemm_nt(k, k, bs, -1.f, E, bs, P, bs, 1.f, A, k, A, k, s, lo, nullptr, status)) != cudaSuccess)
+            return e;
         sweep_fixup_kernel<<<ew_grid(k * bs, sms), 256, 0, s>>>(A, k, p0, bs, E, D);
     }
     return cudaGetLastError();
 }
 
 // ---- workspace --------------------------------------------------------------
+// The V-subproblem runs on V^T (m x k) so that every product is A B^T with
+// K-major operands: W^T is formed once, Zu^T after each U-subproblem, Zv
+// from Zv^T after each V-subproblem.
 struct FactorWs {
-    float *Zu, *Zv, *C, *Lam, *X, *Rhs, *G, *P, *E, *D;
+    float *Zu, *Zv, *Zvt, *ZuT, *WT, *C, *Lam, *X, *Rhs, *G, *P, *E, *D;
     float *a, *m1, *m2, *b, *rho;
-    double *sumsq;   // [outer + 1]
+    uint32_t *bt_packed;   // sign(V^T) packed, m rows of ceil(k/32) words
+    LoScratch lo;          // lo planes of the tensor-core products
+    double *sumsq;         // [outer + 1]
+    int32_t *status;       // a tensor-core GEMM wait that expired
     void *svid;
     size_t bytes;
 };
@@ -399,6 +483,9 @@ FactorWs carve(void *base, int64_t n, int64_t m, int64_t k, int outer, int svid_
     const size_t mx = nk > km ? nk : km;
     w.Zu = reinterpret_cast<float *>(take(nk * 4));
     w.Zv = reinterpret_cast<float *>(take(km * 4));
+    w.Zvt = reinterpret_cast<float *>(take(km * 4));
+    w.ZuT = reinterpret_cast<float *>(take(nk * 4));
+    w.WT = reinterpret_cast<float *>(take(static_cast<size_t>(n) * m * 4));
     w.C = reinterpret_cast<float *>(take(mx * 4));
     w.Lam = reinterpret_cast<float *>(take(mx * 4));
     w.X = reinterpret_cast<float *>(take(mx * 4));
@@ -412,10 +499,35 @@ FactorWs carve(void *base, int64_t n, int64_t m, int64_t k, int outer, int svid_
     w.m2 = reinterpret_cast<float *>(take(static_cast<size_t>(k) * 4));
     w.b = reinterpret_cast<float *>(take(static_cast<size_t>(m) * 4));
     w.rho = reinterpret_cast<float *>(take(4));
+    w.bt_packed = reinterpret_cast<uint32_t *>(take(static_cast<size_t>(m) * pitch_words(k) * 4));
     w.sumsq = reinterpret_cast<double *>(take(static_cast<size_t>(outer + 1) * 8));
-    w.svid = take(svid_scratch_bytes(n > k ? n : k, k > m ? k : m, svid_iters));
+    w.status = reinterpret_cast<int32_t *>(take(4));
+    w.svid = take(svid_scratch_bytes(n > m ? n : m, k, svid_iters));   // projections of n x k and m x k
+    // the largest (M + N) ceil4(K) over the products of one outer iteration
+    const int64_t shapes[][3] = {{n, k, m}, {k, k, m}, {n, k, k}, {m, k, n}, {k, k, n}, {m, k, k}, {n, m, k},
+                                 {k, kSweepBlock, kSweepBlock}, {k, k, kSweepBlock}};
+    size_t lo_floats = 0;
+    for (const auto &sh : shapes) {
+        const size_t f = tf32x3_scratch_floats(sh[0], sh[1], sh[2]);
+        lo_floats = f > lo_floats ? f : lo_floats;
+    }
+    w.lo.p = reinterpret_cast<float *>(take(lo_floats * 4));
+    w.lo.floats = lo_floats;
     w.bytes = off;
     return w;
+}
+
+// a failed tensor-core GEMM wait makes the scale outputs NaN (visibly void)
+__global__ void poison_kernel(const int32_t *status, uint16_t *alpha, int64_t n, uint16_t *beta, int64_t k,
+                              uint16_t *gamma, int64_t m)
+{
+    if (*status == 0) return;
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n + k + m;
+         i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        if (i < n) alpha[i] = 0x7E00u;
+        else if (i < n + k) beta[i - n] = 0x7E00u;
+        else gamma[i - n - k] = 0x7E00u;
+    }
 }
 
 }  // namespace
@@ -434,68 +546,88 @@ cudaError_t factorize_run(const float *W, int64_t n, int64_t m, int64_t k, const
     const int sms = sm_count();
     const int64_t nk = n * k, km = k * m;
     cudaError_t e;
-    // project the start onto the constraint set: Zu = SVID(U0), Zv = SVID(V0)
+    // X (rows x cols) -> Z = SVID(X) with scales p (rows), q (cols); Lam = X - Z
     auto project = [&](int64_t rows, int64_t cols, float *p, float *q, float *Z) -> cudaError_t {
         cudaError_t r = svid_power(w.X, rows, cols, svid_iters, nullptr, nullptr, p, q, w.svid, s);
         if (r != cudaSuccess) return r;
         project_kernel<<<ew_grid(rows * cols, sms), 256, 0, s>>>(w.X, rows, cols, p, q, Z, w.Lam);
         return cudaGetLastError();
     };
+    // ||W - Zu Zv||_F into objective[slot], Zv taken as (Zv^T)^T
     auto objective_at = [&](int slot) -> cudaError_t {
         if (!objective) return cudaSuccess;
-        cudaError_t r = sgemm(false, false, n, m, k, -1.f, w.Zu, k, w.Zv, m, 1.f, W, m, nullptr, 0, s, w.sumsq + slot);
+        cudaError_t r =
+            gemm_nt(n, m, k, -1.f, w.Zu, k, w.Zvt, k, 1.f, W, m, nullptr, 0, s, w.lo, w.sumsq + slot, w.status);
         if (r != cudaSuccess) return r;
         objective_kernel<<<1, 1, 0, s>>>(w.sumsq + slot, objective + slot);
         return cudaGetLastError();
     };
+    // B = sign(V) packed from the V^T projection input: pack V^T, transpose bits
+    auto pack_b = [&]() -> cudaError_t {
+        cudaError_t r = launch_pack_ld(w.X, DBF_F32, m, k, w.bt_packed, pitch_words(k), nullptr, s);
+        if (r != cudaSuccess) return r;
+        return launch_transpose(w.bt_packed, m, k, B_packed, s);
+    };
     if ((e = cudaMemsetAsync(w.sumsq, 0, static_cast<size_t>(outer + 1) * 8, s)) != cudaSuccess) return e;
+    if ((e = cudaMemsetAsync(w.status, 0, 4, s)) != cudaSuccess) return e;
+    if ((e = transpose_f32(W, n, m, w.WT, s)) != cudaSuccess) return e;
+    // the start: Zu = SVID(U0); Zv^T = SVID(V0^T) (the projection commutes
+    // with transposition)
     if ((e = cudaMemcpyAsync(w.X, U0, nk * 4, cudaMemcpyDeviceToDevice, s)) != cudaSuccess) return e;
     if ((e = project(n, k, w.a, w.m1, w.Zu)) != cudaSuccess) return e;
     if (outer == 0 && (e = launch_pack_ld(w.X, DBF_F32, n, k, A_packed, pitch_words(k), nullptr, s)) != cudaSuccess)
         return e;
-    if ((e = cudaMemcpyAsync(w.X, V0, km * 4, cudaMemcpyDeviceToDevice, s)) != cudaSuccess) return e;
-    if ((e = project(k, m, w.m2, w.b, w.Zv)) != cudaSuccess) return e;
-    if (outer == 0 && (e = launch_pack_ld(w.X, DBF_F32, k, m, B_packed, pitch_words(m), nullptr, s)) != cudaSuccess)
-        return e;
+    if ((e = transpose_f32(V0, k, m, w.X, s)) != cudaSuccess) return e;
+    if ((e = project(m, k, w.b, w.m2, w.Zvt)) != cudaSuccess) return e;
+    if (outer == 0 && (e = pack_b()) != cudaSuccess) return e;
+    if ((e = transpose_f32(w.Zvt, m, k, w.Zv, s)) != cudaSuccess) return e;
     if ((e = objective_at(0)) != cudaSuccess) return e;
 
     for (int t = 0; t < outer; ++t) {
         const bool last = t + 1 == outer;
         // U-subproblem: C = W Zv^T, G = Zv Zv^T + rho I, G <- -G^-1
-        if ((e = sgemm(false, true, n, k, m, 1.f, W, m, w.Zv, m, 0.f, nullptr, 0, w.C, k, s)) != cudaSuccess) return e;
-        if ((e = sgemm(false, true, k, k, m, 1.f, w.Zv, m, w.Zv, m, 0.f, nullptr, 0, w.G, k, s)) != cudaSuccess)
+        if ((e = gemm_nt(n, k, m, 1.f, W, m, w.Zv, m, 0.f, nullptr, 0, w.C, k, s, w.lo, nullptr, w.status)) != cudaSuccess)
+            return e;
+        if ((e = gemm_nt(k, k, m, 1.f, w.Zv, m, w.Zv, m, 0.f, nullptr, 0, w.G, k, s, w.lo, nullptr, w.status)) != cudaSuccess)
             return e;
         rho_kernel<<<1, 256, 0, s>>>(w.G, k, rho_rel, w.rho);
-        if ((e = sweep_inverse(w.G, k, w.P, w.E, w.D, sms, s)) != cudaSuccess) return e;
+        if ((e = sweep_inverse(w.G, k, w.P, w.E, w.D, sms, w.lo, w.status, s)) != cudaSuccess) return e;
         if ((e = cudaMemsetAsync(w.Lam, 0, nk * 4, s)) != cudaSuccess) return e;
         for (int j = 0; j < admm_iters; ++j) {
             rhs_kernel<<<ew_grid(nk, sms), 256, 0, s>>>(w.C, w.Zu, w.Lam, w.rho, nk, w.Rhs);
-            // X = U + Lam = -(Rhs G) + Lam
-            if ((e = sgemm(false, false, n, k, k, -1.f, w.Rhs, k, w.G, k, 1.f, w.Lam, k, w.X, k, s)) != cudaSuccess)
+            // X = U + Lam = -(Rhs G) + Lam (G symmetric: Rhs G^T)
+            if ((e = gemm_nt(n, k, k, -1.f, w.Rhs, k, w.G, k, 1.f, w.Lam, k, w.X, k, s, w.lo, nullptr, w.status)) !=
+                cudaSuccess)
                 return e;
             if ((e = project(n, k, w.a, w.m1, w.Zu)) != cudaSuccess) return e;
         }
         if (last && (e = launch_pack_ld(w.X, DBF_F32, n, k, A_packed, pitch_words(k), nullptr, s)) != cudaSuccess)
             return e;
-        // V-subproblem: C = Zu^T W, G = Zu^T Zu + rho I, G <- -G^-1
-        if ((e = sgemm(true, false, k, m, n, 1.f, w.Zu, k, W, m, 0.f, nullptr, 0, w.C, m, s)) != cudaSuccess) return e;
-        if ((e = sgemm(true, false, k, k, n, 1.f, w.Zu, k, w.Zu, k, 0.f, nullptr, 0, w.G, k, s)) != cudaSuccess)
+        if ((e = transpose_f32(w.Zu, n, k, w.ZuT, s)) != cudaSuccess) return e;
+        // V-subproblem on V^T: C^T = W^T Zu, G = Zu^T Zu + rho I, G <- -G^-1
+        if ((e = gemm_nt(m, k, n, 1.f, w.WT, n, w.ZuT, n, 0.f, nullptr, 0, w.C, k, s, w.lo, nullptr, w.status)) !=
+            cudaSuccess)
+            return e;
+        if ((e = gemm_nt(k, k, n, 1.f, w.ZuT, n, w.ZuT, n, 0.f, nullptr, 0, w.G, k, s, w.lo, nullptr, w.status)) !=
+            cudaSuccess)
             return e;
         rho_kernel<<<1, 256, 0, s>>>(w.G, k, rho_rel, w.rho);
-        if ((e = sweep_inverse(w.G, k, w.P, w.E, w.D, sms, s)) != cudaSuccess) return e;
+        if ((e = sweep_inverse(w.G, k, w.P, w.E, w.D, sms, w.lo, w.status, s)) != cudaSuccess) return e;
         if ((e = cudaMemsetAsync(w.Lam, 0, km * 4, s)) != cudaSuccess) return e;
         for (int j = 0; j < admm_iters; ++j) {
-            rhs_kernel<<<ew_grid(km, sms), 256, 0, s>>>(w.C, w.Zv, w.Lam, w.rho, km, w.Rhs);
-            // X = V + Lam = -(G Rhs) + Lam
-            if ((e = sgemm(false, false, k, m, k, -1.f, w.G, k, w.Rhs, m, 1.f, w.Lam, m, w.X, m, s)) != cudaSuccess)
+            rhs_kernel<<<ew_grid(km, sms), 256, 0, s>>>(w.C, w.Zvt, w.Lam, w.rho, km, w.Rhs);
+            // X^T = V^T + Lam^T = -(Rhs^T G) + Lam^T
+            if ((e = gemm_nt(m, k, k, -1.f, w.Rhs, k, w.G, k, 1.f, w.Lam, k, w.X, k, s, w.lo, nullptr, w.status)) !=
+                cudaSuccess)
                 return e;
-            if ((e = project(k, m, w.m2, w.b, w.Zv)) != cudaSuccess) return e;
+            if ((e = project(m, k, w.b, w.m2, w.Zvt)) != cudaSuccess) return e;
         }
-        if (last && (e = launch_pack_ld(w.X, DBF_F32, k, m, B_packed, pitch_words(m), nullptr, s)) != cudaSuccess)
-            return e;
+        if (last && (e = pack_b()) != cudaSuccess) return e;
+        if ((e = transpose_f32(w.Zvt, m, k, w.Zv, s)) != cudaSuccess) return e;
         if ((e = objective_at(t + 1)) != cudaSuccess) return e;
     }
     factor_scales_kernel<<<ew_grid(n + k + m, sms), 256, 0, s>>>(w.a, n, w.m1, w.m2, k, w.b, m, alpha, beta, gamma);
+    poison_kernel<<<ew_grid(n + k + m, sms), 256, 0, s>>>(w.status, alpha, n, beta, k, gamma, m);
     return cudaGetLastError();
 }
 

@@ -65,6 +65,17 @@ cudaError_t svid_power(const float *X, int64_t n, int64_t m, int iters, uint16_t
 cudaError_t svid_run(float *X, int64_t n, int64_t m, int iters, int subtract, uint32_t *signs,
                      int64_t signs_ld, uint16_t *s_out, uint16_t *s_in, void *scratch, cudaStream_t s);
 
+// dense fp32 GEMM on the tensor cores (three TF32 products): Cout = alpha A B^T
+// + beta Cin, A [M x K] and B [N x K] K-major; tf32x3_ok says whether the
+// operands qualify (16-byte aligned, pitches a multiple of 4 floats); the lo
+// planes of A and B go to lo_scratch (tf32x3_scratch_floats(M, N, K) floats,
+// 16-byte aligned)
+bool tf32x3_ok(int64_t M, int64_t N, int64_t K, const float *A, int64_t lda, const float *B, int64_t ldb);
+size_t tf32x3_scratch_floats(int64_t M, int64_t N, int64_t K);
+cudaError_t tf32x3_gemm(int64_t M, int64_t N, int64_t K, float alpha, const float *A, int64_t lda, const float *B,
+                        int64_t ldb, float beta, const float *Cin, int64_t ldci, float *Cout, int64_t ldco,
+                        double *sumsq, int32_t *status, float *lo_scratch, size_t lo_scratch_floats, cudaStream_t s);
+
 // DBF factorisation (alternating ADMM with the SVID projection, fp32)
 size_t factorize_workspace_bytes(int64_t n, int64_t m, int64_t k, int outer, int svid_iters);
 cudaError_t factorize_run(const float *W, int64_t n, int64_t m, int64_t k, const float *U0, const float *V0,

@@ -12,7 +12,7 @@
 // One power iteration is u = |X| v_hat, then v = |X|^T u. When a row of X is
 // at most 12288 floats (a multiple of 4, 16-byte aligned) one persistent
 // kernel does both from a single read of X: each CTA streams bands of whole
-// rows into shared memory with bulk copies (a ring of four buffers, mbarrier
+// rows into shared memory with bulk copies (a ring of two buffers, mbarrier
 // completion), forms u for the band's rows by a block reduction, then adds
 // |X_band|^T u_band into per-thread registers (a thread owns fixed columns),
 // and flushes them with vector atomics at the end. Otherwise two kernels
@@ -93,7 +93,7 @@ constexpr int kFuseThreads = 256;
 constexpr int kFuseWarps = kFuseThreads / 32;
 constexpr int64_t kFuseMaxCols = 12288;         // 12 float4 columns per thread
 constexpr int kFuseMaxBand = 16;                // rows per band
-constexpr int kFuseStages = 4;                  // band buffers in the ring
+constexpr int kFuseStages = 2;                  // band buffers in the ring
 constexpr size_t kFuseBufBudget = 200 * 1024;   // bytes of all band buffers
 constexpr unsigned long long kWaitNs = 2000000000ull;   // bounded waits: 2 s
 

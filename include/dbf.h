@@ -184,11 +184,15 @@ dbf_status dbf_svid(float *X, int64_t n, int64_t m, int32_t iters, int subtract,
  *    start and after each outer iteration (fp32 scales; costs one n x m x k
  *    product per entry). NULL skips it.
  * ws: dbf_factorize_workspace_bytes(n, m, k, outer, svid_iters) bytes,
- *    256-byte aligned, scratch. Arithmetic is fp32 (products accumulated in
- *    fp32; the k x k inverse by an in-place blocked Gauss-Jordan sweep).
+ *    256-byte aligned, scratch. Arithmetic is fp32: products on the tensor
+ *    cores as three TF32 products per operand pair (fp32 accumulation; about
+ *    2^-20 relative per product) when the operands allow (m and k multiples
+ *    of 4), else fp32 FMA; the k x k inverse by an in-place blocked
+ *    Gauss-Jordan sweep. A tensor-core wait that expires (1 s) makes alpha,
+ *    beta and gamma NaN.
  * U0 and V0 must not be zero (a zero Gram matrix gives rho = 0 and NaN).
  * Errors: DBF_ERR_INVALID_ARG, DBF_ERR_ALIGNMENT, DBF_ERR_WORKSPACE,
- *    DBF_ERR_UNSUPPORTED (a dimension above 65535 * 128), DBF_ERR_CUDA. */
+ *    DBF_ERR_UNSUPPORTED (a dimension above 65535 * 32), DBF_ERR_CUDA. */
 size_t dbf_factorize_workspace_bytes(int64_t n, int64_t m, int64_t k, int32_t outer, int32_t svid_iters);
 dbf_status dbf_factorize(const float *W, int64_t n, int64_t m, int64_t k, const float *U0, const float *V0,
                          int32_t outer, int32_t admm_iters, int32_t svid_iters, float rho_rel,
