@@ -274,131 +274,140 @@ __global__ void sweep_panel_kernel(const float *__restrict__ A, int64_t k, int64
 }
 
 // D = T^-1 for the bs x bs SPD block T = P[p0 : p0 + bs, :] (bs <= 128), by
-// the sweep four pivots at a time (pivot block Q = rows and columns
-// q .. q + 3, D4 = T_QQ^-1: T_ij -= T_iQ D4 T_Qj for i, j outside Q, then
-// T_iQ <- T_iQ D4, T_Qj <- D4 T_Qj, T_QQ <- -D4; after every block
-// T = -(original T)^-1). The block is padded to a multiple of 4 with
+// the sweep eight pivots at a time (pivot block Q = rows and columns
+// q .. q + 7, D8 = T_QQ^-1: T_ij -= T_iQ D8 T_Qj for i, j outside Q, then
+// T_iQ <- T_iQ D8, T_Qj <- D8 T_Qj, T_QQ <- -D8; after every block
+// T = -(original T)^-1). The block is padded to a multiple of 8 with
 // identity pivots, which leave the inverse of the rest unchanged. One CTA;
-// thread t holds row t / 8, columns 16 (t % 8) .. + 15 in registers; per
-// pivot block the owners publish rows Q and columns Q in shared memory, every
-// thread inverts the 4 x 4 block itself, and the four rows of Q are held by
-// exactly one warp.
+// thread t holds row t / 8, columns 16 (t % 8) .. + 15 in registers. Per
+// pivot block: the owners publish rows Q and columns Q in shared memory;
+// warp 0 inverts the 8 x 8 block (scalar sweep, lane a holds row a) and
+// publishes D8; every thread then forms its row's coefficients T_iQ D8 and
+// updates its 16 elements (rows Q, held by two whole warps, take D8 T_Qj).
 __global__ void __launch_bounds__(kSweepThreads) sweep_block_inverse_kernel(const float *__restrict__ P, int64_t p0,
                                                                             int bs, float *__restrict__ D)
 {
-    __shared__ __align__(16) float rowq[4][kSweepBlock];
-    __shared__ __align__(16) float colq[kSweepBlock][4];
-    const int tid = threadIdx.x;
+    constexpr int Q = 8;
+    __shared__ __align__(16) float rowq[Q][kSweepBlock];
+    __shared__ __align__(16) float colq[kSweepBlock][Q];
+    __shared__ __align__(16) float dq[Q][Q];
+    const int tid = threadIdx.x, lane = tid & 31;
     const int i = tid / (kSweepBlock / kSweepSeg), j0 = (tid % (kSweepBlock / kSweepSeg)) * kSweepSeg;
-    const int bs4 = (bs + 3) & ~3;
+    const int bs8 = (bs + Q - 1) & ~(Q - 1);
     float t[kSweepSeg];
 #pragma unroll
     for (int e = 0; e < kSweepSeg; ++e) {
         const int j = j0 + e;
-        t[e] = (i < bs && j < bs) ? P[(p0 + i) * bs + j] : (i == j && i < bs4 ? 1.f : 0.f);
+        t[e] = (i < bs && j < bs) ? P[(p0 + i) * bs + j] : (i == j && i < bs8 ? 1.f : 0.f);
     }
-    for (int q = 0; q < bs4; q += 4) {
-        const bool in_row = i >= q && i < q + 4;          // one whole warp
+    for (int q = 0; q < bs8; q += Q) {
+        const bool in_row = i >= q && i < q + Q;          // two whole warps
         const bool has_col = q >= j0 && q < j0 + kSweepSeg;
-        const int cq = (q - j0) >> 2;                      // which float4 of the segment holds columns Q
+        const bool hi_half = q - j0 >= Q;                  // columns Q are t[8 .. 15] rather than t[0 .. 7]
         if (in_row) {
 #pragma unroll
             for (int e = 0; e < kSweepSeg; e += 4)
                 *reinterpret_cast<float4 *>(&rowq[i - q][j0 + e]) = make_float4(t[e], t[e + 1], t[e + 2], t[e + 3]);
         }
         if (has_col) {
-            float4 v = make_float4(t[0], t[1], t[2], t[3]);
-            if (cq == 1) v = make_float4(t[4], t[5], t[6], t[7]);
-            if (cq == 2) v = make_float4(t[8], t[9], t[10], t[11]);
-            if (cq == 3) v = make_float4(t[12], t[13], t[14], t[15]);
-            *reinterpret_cast<float4 *>(&colq[i][0]) = v;
+            float4 v0 = make_float4(t[0], t[1], t[2], t[3]), v1 = make_float4(t[4], t[5], t[6], t[7]);
+            if (hi_half) {
+                v0 = make_float4(t[8], t[9], t[10], t[11]);
+                v1 = make_float4(t[12], t[13], t[14], t[15]);
+            }
+            *reinterpret_cast<float4 *>(&colq[i][0]) = v0;
+            *reinterpret_cast<float4 *>(&colq[i][4]) = v1;
         }
         __syncthreads();
-        // D4 = T_QQ^-1 by the scalar sweep on the 4 x 4 block (every thread)
-        float d4[4][4];
+        if (tid < 32) {
+            // D8 by the scalar sweep, lane a < 8 holding row a; the result is
+            // -D8, negated on the way out
+            float r[Q];
 #pragma unroll
-        for (int a = 0; a < 4; ++a)
+            for (int b = 0; b < Q; ++b) r[b] = lane < Q ? rowq[lane][q + b] : 0.f;
 #pragma unroll
-            for (int b = 0; b < 4; ++b) d4[a][b] = rowq[a][q + b];
+            for (int pv = 0; pv < Q; ++pv) {
+                float pr[Q];
 #pragma unroll
-        for (int pv = 0; pv < 4; ++pv) {
-            const float dinv = 1.0f / d4[pv][pv];
-            float c[4], r[4];
+                for (int b = 0; b < Q; ++b) pr[b] = __shfl_sync(0xffffffffu, r[b], pv);   // row pv
+                const float dinv = 1.0f / pr[pv];
+                const float c = r[pv];                                                    // this row's column pv
 #pragma unroll
-            for (int a = 0; a < 4; ++a) {
-                c[a] = d4[a][pv];
-                r[a] = d4[pv][a];
-            }
-#pragma unroll
-            for (int a = 0; a < 4; ++a)
-#pragma unroll
-                for (int b = 0; b < 4; ++b) {
-                    if (a != pv && b != pv) d4[a][b] -= c[a] * dinv * r[b];
-                    else if (a == pv && b == pv) d4[a][b] = -dinv;
-                    else if (b == pv) d4[a][b] = c[a] * dinv;
-                    else d4[a][b] = dinv * r[b];
+                for (int b = 0; b < Q; ++b) {
+                    if (lane == pv) r[b] = b == pv ? -dinv : dinv * pr[b];
+                    else r[b] = b == pv ? c * dinv : r[b] - c * dinv * pr[b];
                 }
+            }
+            if (lane < Q) {
+#pragma unroll
+                for (int b = 0; b < Q; ++b) dq[lane][b] = -r[b];
+            }
         }
-#pragma unroll
-        for (int a = 0; a < 4; ++a)
-#pragma unroll
-            for (int b = 0; b < 4; ++b) d4[a][b] = -d4[a][b];   // now T_QQ^-1
-        // this row's coefficients: c = T_iQ D4 (rows outside Q), or row i - q of D4
-        float cf[4];
-        {
-            const float4 ci = *reinterpret_cast<const float4 *>(&colq[i][0]);
-#pragma unroll
-            for (int b = 0; b < 4; ++b) cf[b] = ci.x * d4[0][b] + ci.y * d4[1][b] + ci.z * d4[2][b] + ci.w * d4[3][b];
-        }
+        __syncthreads();
+        float cf[Q];
         if (in_row) {
-            // T_Qj <- D4 T_Qj (row i - q of D4 times the old rows Q)
-            const int a = i - q;
-            const float w0 = a == 0 ? d4[0][0] : a == 1 ? d4[1][0] : a == 2 ? d4[2][0] : d4[3][0];
-            const float w1 = a == 0 ? d4[0][1] : a == 1 ? d4[1][1] : a == 2 ? d4[2][1] : d4[3][1];
-            const float w2 = a == 0 ? d4[0][2] : a == 1 ? d4[1][2] : a == 2 ? d4[2][2] : d4[3][2];
-            const float w3 = a == 0 ? d4[0][3] : a == 1 ? d4[1][3] : a == 2 ? d4[2][3] : d4[3][3];
+            // T_Qj <- D8 T_Qj; columns Q of these rows become -D8
+            float w[Q];
+#pragma unroll
+            for (int b = 0; b < Q; ++b) w[b] = dq[i - q][b];
 #pragma unroll
             for (int e = 0; e < kSweepSeg; e += 4) {
-                const float4 r0 = *reinterpret_cast<const float4 *>(&rowq[0][j0 + e]);
-                const float4 r1 = *reinterpret_cast<const float4 *>(&rowq[1][j0 + e]);
-                const float4 r2 = *reinterpret_cast<const float4 *>(&rowq[2][j0 + e]);
-                const float4 r3 = *reinterpret_cast<const float4 *>(&rowq[3][j0 + e]);
-                t[e] = w0 * r0.x + w1 * r1.x + w2 * r2.x + w3 * r3.x;
-                t[e + 1] = w0 * r0.y + w1 * r1.y + w2 * r2.y + w3 * r3.y;
-                t[e + 2] = w0 * r0.z + w1 * r1.z + w2 * r2.z + w3 * r3.z;
-                t[e + 3] = w0 * r0.w + w1 * r1.w + w2 * r2.w + w3 * r3.w;
-            }
-            // T_QQ <- -D4: row a of it, columns Q
-            cf[0] = -w0;
-            cf[1] = -w1;
-            cf[2] = -w2;
-            cf[3] = -w3;
-        } else {
-            // T_ij -= c T_Qj
+                float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-            for (int e = 0; e < kSweepSeg; e += 4) {
-                const float4 r0 = *reinterpret_cast<const float4 *>(&rowq[0][j0 + e]);
-                const float4 r1 = *reinterpret_cast<const float4 *>(&rowq[1][j0 + e]);
-                const float4 r2 = *reinterpret_cast<const float4 *>(&rowq[2][j0 + e]);
-                const float4 r3 = *reinterpret_cast<const float4 *>(&rowq[3][j0 + e]);
-                t[e] -= cf[0] * r0.x + cf[1] * r1.x + cf[2] * r2.x + cf[3] * r3.x;
-                t[e + 1] -= cf[0] * r0.y + cf[1] * r1.y + cf[2] * r2.y + cf[3] * r3.y;
-                t[e + 2] -= cf[0] * r0.z + cf[1] * r1.z + cf[2] * r2.z + cf[3] * r3.z;
-                t[e + 3] -= cf[0] * r0.w + cf[1] * r1.w + cf[2] * r2.w + cf[3] * r3.w;
-            }
-        }
-        // columns Q of this row: T_iQ D4 outside Q, -D4 inside
-        if (has_col) {
-#pragma unroll
-            for (int c4 = 0; c4 < 4; ++c4)
-                if (cq == c4) {
-                    t[4 * c4] = cf[0];
-                    t[4 * c4 + 1] = cf[1];
-                    t[4 * c4 + 2] = cf[2];
-                    t[4 * c4 + 3] = cf[3];
+                for (int b = 0; b < Q; ++b) {
+                    const float4 rb = *reinterpret_cast<const float4 *>(&rowq[b][j0 + e]);
+                    acc.x += w[b] * rb.x;
+                    acc.y += w[b] * rb.y;
+                    acc.z += w[b] * rb.z;
+                    acc.w += w[b] * rb.w;
                 }
+                t[e] = acc.x;
+                t[e + 1] = acc.y;
+                t[e + 2] = acc.z;
+                t[e + 3] = acc.w;
+            }
+#pragma unroll
+            for (int b = 0; b < Q; ++b) cf[b] = -w[b];
+        } else {
+            // coefficients T_iQ D8, then T_ij -= coefficients . T_Qj
+            float ci[Q];
+#pragma unroll
+            for (int b = 0; b < Q; ++b) ci[b] = colq[i][b];
+#pragma unroll
+            for (int b = 0; b < Q; ++b) {
+                float v = 0.f;
+#pragma unroll
+                for (int a = 0; a < Q; ++a) v += ci[a] * dq[a][b];
+                cf[b] = v;
+            }
+#pragma unroll
+            for (int e = 0; e < kSweepSeg; e += 4) {
+                float4 acc = make_float4(t[e], t[e + 1], t[e + 2], t[e + 3]);
+#pragma unroll
+                for (int b = 0; b < Q; ++b) {
+                    const float4 rb = *reinterpret_cast<const float4 *>(&rowq[b][j0 + e]);
+                    acc.x -= cf[b] * rb.x;
+                    acc.y -= cf[b] * rb.y;
+                    acc.z -= cf[b] * rb.z;
+                    acc.w -= cf[b] * rb.w;
+                }
+                t[e] = acc.x;
+                t[e + 1] = acc.y;
+                t[e + 2] = acc.z;
+                t[e + 3] = acc.w;
+            }
         }
-        __syncthreads();   // rows Q and columns Q are read before the next block rewrites them
+        // columns Q of this row: T_iQ D8 outside Q, -D8 inside
+        if (has_col) {
+            if (hi_half) {
+#pragma unroll
+                for (int b = 0; b < Q; ++b) t[Q + b] = cf[b];
+            } else {
+#pragma unroll
+                for (int b = 0; b < Q; ++b) t[b] = cf[b];
+            }
+        }
+        __syncthreads();   // rows Q, columns Q and D8 are read before the next block rewrites them
     }
 #pragma unroll
     for (int e = 0; e < kSweepSeg; ++e)
