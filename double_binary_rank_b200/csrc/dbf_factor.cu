@@ -288,11 +288,14 @@ __global__ void __launch_bounds__(kSweepThreads) sweep_block_inverse_kernel(cons
                                                                             int bs, float *__restrict__ D)
 {
     constexpr int Q = 8;
-    __shared__ __align__(16) float rowq[Q][kSweepBlock];
+    constexpr int kSegs = kSweepBlock / kSweepSeg, kSegPad = kSweepSeg + 4;
+    // rows Q, one padded run per 16-column segment: the eight segments of a
+    // float4 load start 80 bytes apart and so hit disjoint banks
+    __shared__ __align__(16) float rowq[Q][kSegs][kSegPad];
     __shared__ __align__(16) float colq[kSweepBlock][Q];
     __shared__ __align__(16) float dq[Q][Q];
     const int tid = threadIdx.x, lane = tid & 31;
-    const int i = tid / (kSweepBlock / kSweepSeg), j0 = (tid % (kSweepBlock / kSweepSeg)) * kSweepSeg;
+    const int i = tid / kSegs, sg = tid % kSegs, j0 = sg * kSweepSeg;
     const int bs8 = (bs + Q - 1) & ~(Q - 1);
     float t[kSweepSeg];
 #pragma unroll
@@ -307,7 +310,7 @@ __global__ void __launch_bounds__(kSweepThreads) sweep_block_inverse_kernel(cons
         if (in_row) {
 #pragma unroll
             for (int e = 0; e < kSweepSeg; e += 4)
-                *reinterpret_cast<float4 *>(&rowq[i - q][j0 + e]) = make_float4(t[e], t[e + 1], t[e + 2], t[e + 3]);
+                *reinterpret_cast<float4 *>(&rowq[i - q][sg][e]) = make_float4(t[e], t[e + 1], t[e + 2], t[e + 3]);
         }
         if (has_col) {
             float4 v0 = make_float4(t[0], t[1], t[2], t[3]), v1 = make_float4(t[4], t[5], t[6], t[7]);
@@ -324,7 +327,7 @@ __global__ void __launch_bounds__(kSweepThreads) sweep_block_inverse_kernel(cons
             // -D8, negated on the way out
             float r[Q];
 #pragma unroll
-            for (int b = 0; b < Q; ++b) r[b] = lane < Q ? rowq[lane][q + b] : 0.f;
+            for (int b = 0; b < Q; ++b) r[b] = lane < Q ? rowq[lane][(q + b) / kSweepSeg][(q + b) % kSweepSeg] : 0.f;
 #pragma unroll
             for (int pv = 0; pv < Q; ++pv) {
                 float pr[Q];
@@ -355,7 +358,7 @@ __global__ void __launch_bounds__(kSweepThreads) sweep_block_inverse_kernel(cons
                 float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
                 for (int b = 0; b < Q; ++b) {
-                    const float4 rb = *reinterpret_cast<const float4 *>(&rowq[b][j0 + e]);
+                    const float4 rb = *reinterpret_cast<const float4 *>(&rowq[b][sg][e]);
                     acc.x += w[b] * rb.x;
                     acc.y += w[b] * rb.y;
                     acc.z += w[b] * rb.z;
@@ -385,7 +388,7 @@ __global__ void __launch_bounds__(kSweepThreads) sweep_block_inverse_kernel(cons
                 float4 acc = make_float4(t[e], t[e + 1], t[e + 2], t[e + 3]);
 #pragma unroll
                 for (int b = 0; b < Q; ++b) {
-                    const float4 rb = *reinterpret_cast<const float4 *>(&rowq[b][j0 + e]);
+                    const float4 rb = *reinterpret_cast<const float4 *>(&rowq[b][sg][e]);
                     acc.x -= cf[b] * rb.x;
                     acc.y -= cf[b] * rb.y;
                     acc.z -= cf[b] * rb.z;

@@ -184,12 +184,14 @@ dbf_status dbf_svid(float *X, int64_t n, int64_t m, int32_t iters, int subtract,
  *    start and after each outer iteration (fp32 scales; costs one n x m x k
  *    product per entry). NULL skips it.
  * ws: dbf_factorize_workspace_bytes(n, m, k, outer, svid_iters) bytes,
- *    256-byte aligned, scratch. Arithmetic is fp32: products on the tensor
- *    cores as three TF32 products per operand pair (fp32 accumulation; about
- *    2^-20 relative per product) when the operands allow (m and k multiples
- *    of 4), else fp32 FMA; the k x k inverse by an in-place blocked
- *    Gauss-Jordan sweep. A tensor-core wait that expires (1 s) makes alpha,
- *    beta and gamma NaN.
+ *    256-byte aligned, scratch. Arithmetic is fp32: each product runs on the
+ *    tensor cores as three TF32 products per operand pair (fp32
+ *    accumulation; about 2^-20 relative per product, plus an accumulation
+ *    bias of about K/8 units of 2^-24) when its operands' row pitches are
+ *    multiples of 4 floats and its K is at least 32 (n, m and k multiples
+ *    of 4 make every product qualify), else as fp32 FMA; the k x k inverse
+ *    by an in-place blocked Gauss-Jordan sweep. A tensor-core wait that
+ *    expires (1 s) makes alpha, beta and gamma NaN.
  * U0 and V0 must not be zero (a zero Gram matrix gives rho = 0 and NaN).
  * Errors: DBF_ERR_INVALID_ARG, DBF_ERR_ALIGNMENT, DBF_ERR_WORKSPACE,
  *    DBF_ERR_UNSUPPORTED (a dimension above 65535 * 32), DBF_ERR_CUDA. */
