@@ -16,7 +16,11 @@ matmuls, the all-plus / rank-one / Sylvester-Hadamard closed forms, the
 matched sign-flip, envelope-linearity, power-of-two and rank-permutation
 invariants, bit-identical agreement in exact dyadic arithmetic, decoder
 agreement with numpy's fp16 / fp32 conversions, and the packed layout on
-hand-worked words. Every function here is pinned; none is "parity unpinned".
+hand-worked words. The backward (tests/test_oracle_backward_pins.py), the
+MBOK layer and SVID (tests/test_oracle_mbok_pins.py,
+tests/test_oracle_svid_pins.py) and the DBF factorisation in
+``dbf_factorize.py`` (tests/test_oracle_factorize_pins.py) carry their own
+pins. Every function here is pinned; none is "parity unpinned".
 """
 from __future__ import annotations
 
