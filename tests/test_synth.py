@@ -67,3 +67,20 @@ def test_segments_sorted_and_cover():
 def test_sample_rows_holds_ends():
     r = S.sample_rows(3, 2048, 128)
     assert r.size == 128 and r[0] == 0 and r[-1] == 2047 and np.all(np.diff(r) > 0)
+
+
+def test_weight_and_factor_start_recipes():
+    # W[i, j] = g r_i c_j with lognormal row / column scales; seeded, distinct
+    # streams for the weight and for the two start factors
+    W1, W2 = S.make_weight(3, 64, 48), S.make_weight(3, 64, 48)
+    assert W1.dtype == np.float32 and W1.shape == (64, 48) and np.array_equal(W1, W2)
+    assert not np.array_equal(W1, S.make_weight(4, 64, 48))
+    # row / column structure: the log of the row rms spreads with sigma 0.25
+    big = S.make_weight(5, 2000, 2000).astype(np.float64)
+    lr = np.log(np.sqrt((big ** 2).mean(axis=1)))
+    assert 0.2 < lr.std() < 0.3
+    U0, V0 = S.make_factor_start(6, 64, 48, 20, scale=2.0)
+    assert U0.shape == (64, 20) and V0.shape == (20, 48) and U0.dtype == np.float32
+    # U0 V0 entries have about the requested scale
+    UV = U0.astype(np.float64) @ V0.astype(np.float64)
+    assert 1.5 < np.sqrt((UV ** 2).mean()) < 2.6
