@@ -1,18 +1,28 @@
 """Benchmark of the double-binary layer forward on B200.
 
-Workload: the DBF full-weight MLP layer (DBF page, section 2 form with
-ell = 1): M = 4096 inputs, N = 11008 outputs, R = 5888 (~1.97 bits/weight),
-bf16 activations ~ N(0, 1), iid +-1 factors, fp16 lognormal(0, 0.5) scales.
-One step runs the whole forward (gamma scaling, sign accumulation over B2,
-beta scaling, sign accumulation over B1, alpha scaling, write) twice: once
-in the decode regime (1 token) and once in the prefill regime (2048 tokens).
-Reported: tokens/s for the whole job, the decode kernel pair against the HBM
-roofline and the prefill pair against the tensor-core roofline.
+Headline workload: the DBF full-weight MLP layer (DBF page, section 2 form
+with ell = 1): M = 4096 inputs, N = 11008 outputs, R = 5888 (~1.97
+bits/weight), bf16 activations ~ N(0, 1), iid +-1 factors, fp16
+lognormal(0, 0.5) scales. One step runs the whole forward (gamma scaling,
+sign accumulation over B2, beta scaling, sign accumulation over B1, alpha
+scaling, write) twice: once in the decode regime (1 token) and once in the
+prefill regime (2048 tokens). Reported: tokens/s for the whole job, the
+decode call against the HBM roofline and the prefill call against the
+tensor-core roofline.
 
-L2: every step reads a different one of 24 device copies of the layer
-(24 x 11.2 MB, more than twice the 126 MB L2), so the sign matrices come
-from HBM. Multi-GPU (torchrun): each rank runs the same per-GPU work
-(weak scaling); the timing is the max over ranks.
+The other four layer configurations are timed too, each against its own
+roofline and beside the fp64 oracle on the same token rows ("configs"): the
+tiny layer (256 x 256, R = 16, 4 fp32 tokens), the LoRDBA adapter branch
+(4096 x 4096, R = 64) at 1, 4, 16 and 64 tokens, 32 adapters (R = 32,
+ell = 2) routed over 256 tokens in one segmented call, and the large
+prefill layer (M = N = R = 8192) at 8192 tokens.
+
+L2: every headline step reads a different one of 24 device copies of the
+layer (24 x 11.2 MB, more than twice the 126 MB L2), so the sign matrices
+come from HBM; the per-configuration calls are timed one by one with a
+256 MB buffer written between calls (L2 flushed). Multi-GPU (torchrun):
+each rank runs the same per-GPU work (weak scaling); the timing is the max
+over ranks.
 
 python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
 """
@@ -146,14 +156,22 @@ def weak_scaling_value(world: int, tokens_per_step: int, steps: int, elapsed_ms:
     return world * tokens_per_step * steps / (elapsed_ms * 1e-3)
 
 
-def algorithmic(w, T):
-    """Algorithmic bytes and flops of one forward call (decode-path numbers
-    count the packed signs, scales, x in and y out)."""
-    sign_bytes = w.R * (w.M + w.N) / 8
-    scale_bytes = 2 * w.ell * (w.M + w.N + w.R)
-    act_bytes = T * w.M * 2 + T * w.N * 2
-    flops = 2 * T * w.ell * w.R * (w.M + w.N)
-    return sign_bytes + scale_bytes + act_bytes, flops
+def algorithmic(w, T, act_bytes=2, R=None, layers=1):
+    """Algorithmic bytes and flops of one forward call: the packed signs and
+    the scales of 'layers' layers, x in and y out (act_bytes per value)."""
+    R = w.R if R is None else R
+    sign_bytes = layers * R * (w.M + w.N) / 8
+    scale_bytes = layers * 2 * w.ell * (w.M + w.N + R)
+    io_bytes = T * w.M * act_bytes + T * w.N * act_bytes
+    flops = 2 * T * w.ell * R * (w.M + w.N)
+    return sign_bytes + scale_bytes + io_bytes, flops
+
+
+ORACLE_ROWS = 128   # prefill rows of the oracle sample (first, last, every 256-token tile)
+
+
+def oracle_rows(w):
+    return S.sample_rows_per_tile(w.seed, T_PREFILL, ORACLE_ROWS, 256)
 
 
 def oracle_sample_rate(w, L, x_dec, x_pre, rows, nthreads):
@@ -166,8 +184,28 @@ def oracle_sample_rate(w, L, x_dec, x_pre, rows, nthreads):
     return (1 + len(rows)) / dt, dt
 
 
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+def bench_config(w):
+    """The workload description both arms print (identical dicts)."""
+    return {"workload": w.description, "decode_tokens": T_DECODE, "prefill_tokens": T_PREFILL,
+            "l2": f"inputs larger than L2: {COPIES} rotating copies of the layer weights",
+            "oracle_sample": f"1 decode token + {ORACLE_ROWS} fixed seeded rows of the {T_PREFILL}-token prefill "
+                             "(first, last, and rows of every 256-token tile)"}
+
+
 def run_reference(args, rank, world):
-    """Reference arm: the fp64 CPU oracle, timed on the host cores."""
+    """Reference arm: the fp64 CPU oracle, timed on the host cores, on the
+    same sample the other arm's cpu_baseline uses."""
     import oracle
     w = S.WORKLOADS[WORKLOAD]
     if world > 1 and rank != 0:
@@ -175,27 +213,180 @@ def run_reference(args, rank, world):
     L = S.workload_layers(w)[0]
     x_dec = S.make_x(w.seed, T_DECODE, w.M, "bf16")
     x_pre = S.make_x(w.seed + 100, T_PREFILL, w.M, "bf16")
-    rows = S.sample_rows(w.seed, T_PREFILL, 7)
+    rows = oracle_rows(w)
     nthreads = oracle.default_threads()
     for _ in range(args.warmup):
-        oracle_sample_rate(w, L, x_dec, x_pre, rows[:1], nthreads)
+        oracle_sample_rate(w, L, x_dec, x_pre, rows[:8], nthreads)
     tokens = 0
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        rate, dt = oracle_sample_rate(w, L, x_dec, x_pre, rows, nthreads)
+        oracle_sample_rate(w, L, x_dec, x_pre, rows, nthreads)
         tokens += 1 + len(rows)
     dt = time.perf_counter() - t0
     value = tokens / dt
-    sample = f"per step: 1 decode token + {len(rows)} of the {T_PREFILL} prefill tokens (fixed seeded rows)"
+    sample = (f"per step: 1 decode token + {len(rows)} of the {T_PREFILL} prefill tokens (fixed seeded rows); "
+              f"CPU {cpu_model()}")
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * dt / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": w.description, "decode_tokens": T_DECODE, "prefill_tokens": T_PREFILL},
+        "config": bench_config(w),
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": nthreads, "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
+
+
+def oracle_rate(fn, tokens, min_s=0.3):
+    """tokens / second of repeated oracle calls (at least min_s of work)."""
+    n, t0 = 0, time.perf_counter()
+    while True:
+        fn()
+        n += 1
+        dt = time.perf_counter() - t0
+        if dt >= min_s:
+            return n * tokens / dt
+
+
+def measure_configs(dbf, dev, stream, run_oracle):
+    """Every layer configuration timed one call at a time (L2 flushed before
+    each call by writing a 256 MB buffer, outside the timed events), against
+    its roofline, beside the fp64 oracle on the same token rows."""
+    import torch
+    pk, pk_kind = peaks()
+    flush_buf = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    f16 = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.float16)).to(dev)
+    bf16 = lambda a: torch.from_numpy(a.view(np.int16)).to(dev).view(torch.bfloat16)
+    dev_layer = lambda L: dbf.Layer.from_signs(torch.from_numpy(L.b1).to(dev), torch.from_numpy(L.b2).to(dev),
+                                               f16(L.alpha), f16(L.beta), f16(L.gamma))
+    nthreads = None
+    if run_oracle:
+        import oracle
+        nthreads = oracle.default_threads()
+
+    def timed(fn, n):
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+        with torch.cuda.stream(stream):
+            for _ in range(3):
+                fn()
+            for a, b in ev:
+                flush_buf.zero_()
+                a.record(stream)
+                fn()
+                b.record(stream)
+        torch.cuda.synchronize(dev)
+        return max_over_ranks(statistics.mean(1e3 * a.elapsed_time(b) for a, b in ev), dev)
+
+    def entry(kernel, T, us, nbytes, flops, bound):
+        e = {"kernel": kernel, "tokens": T, "us_per_call": us, "tokens_per_s": T / (us * 1e-6),
+             "GB_per_s": nbytes / (us * 1e-6) / 1e9, "TFLOP_per_s": flops / (us * 1e-6) / 1e12,
+             "algorithmic_bytes": nbytes, "flops": flops, "bound": bound, "l2": "flushed before each call"}
+        if bound == "hbm":
+            e.update(peak=pk["hbm_gbs"], unit="GB/s", frac=e["GB_per_s"] / pk["hbm_gbs"],
+                     peak_source=f"{pk_kind} copy bandwidth")
+        else:
+            e.update(peak=pk["bf16_tflops"], unit="TFLOP/s", frac=e["TFLOP_per_s"] / pk["bf16_tflops"],
+                     peak_source=f"{pk_kind} bf16 dense (fp16 runs at the same rate)")
+        return e
+
+    out = {}
+    # ---- tiny layer: 4 fp32 tokens
+    w = S.WORKLOADS["tiny"]
+    L = S.workload_layers(w)[0]
+    dl = dev_layer(L)
+    xh = S.make_x(w.seed, 4, w.M, "f32")
+    x = torch.from_numpy(xh).to(dev)
+    y = torch.empty((4, w.N), dtype=torch.float32, device=dev)
+    ws = dbf.alloc_workspace(dbf.workspace_bytes(dl, 4), dev)
+    us = timed(lambda: dbf.forward(dl, x, y=y, ws=ws, stream=stream), 50)
+    nb, fl = algorithmic(w, 4, act_bytes=4)
+    e = entry(f"{w.description}: decode path, {dbf.forward_launches(dl, 4)} launch", 4, us, nb, fl, "hbm")
+    if run_oracle:
+        e["oracle_tokens_per_s"] = oracle_rate(lambda: oracle.forward(L, xh, nthreads=nthreads), 4)
+        e["oracle_tokens_per_s_1thread"] = oracle_rate(lambda: oracle.forward(L, xh, nthreads=1), 4)
+    out["tiny_T4"] = e
+    # ---- LoRDBA adapter branch at 1, 4, 16, 64 tokens
+    w = S.WORKLOADS["adapter"]
+    L = S.workload_layers(w)[0]
+    dl = dev_layer(L)
+    for T in w.tokens:
+        xh = S.make_x(w.seed, T, w.M, "bf16")
+        x = bf16(xh)
+        y = torch.empty((T, w.N), dtype=torch.bfloat16, device=dev)
+        ws = dbf.alloc_workspace(dbf.workspace_bytes(dl, T), dev)
+        us = timed(lambda: dbf.forward(dl, x, y=y, ws=ws, stream=stream), 50)
+        nb, fl = algorithmic(w, T)
+        e = entry(f"{w.description}: decode path, {dbf.forward_launches(dl, T)} launch(es)", T, us, nb, fl, "hbm")
+        if run_oracle:
+            e["oracle_tokens_per_s"] = oracle_rate(lambda: oracle.forward(L, xh, nthreads=nthreads), T)
+            e["oracle_tokens_per_s_1thread"] = oracle_rate(lambda: oracle.forward(L, xh, nthreads=1), T)
+        out[f"adapter_T{T}"] = e
+    # ---- DBF MLP layer, decode (1 token) and prefill (2048 tokens)
+    w = S.WORKLOADS["dbf_mlp"]
+    L = S.workload_layers(w)[0]
+    dl = dev_layer(L)
+    for T, seed in ((1, w.seed), (T_PREFILL, w.seed + 100)):
+        xh = S.make_x(seed, T, w.M, "bf16")
+        x = bf16(xh)
+        y = torch.empty((T, w.N), dtype=torch.bfloat16, device=dev)
+        ws = dbf.alloc_workspace(dbf.workspace_bytes(dl, T), dev)
+        us = timed(lambda: dbf.forward(dl, x, y=y, ws=ws, stream=stream), 50 if T == 1 else 10)
+        nb, fl = algorithmic(w, T)
+        path = "decode" if T == 1 else "prefill"
+        e = entry(f"{w.description}: {path} path, {dbf.forward_launches(dl, T)} launch(es)", T, us, nb, fl,
+                  "hbm" if T == 1 else "tensor")
+        if run_oracle:
+            rows = None if T == 1 else oracle_rows(w)
+            e["oracle_tokens_per_s"] = oracle_rate(lambda: oracle.forward(L, xh, rows=rows, nthreads=nthreads),
+                                                   T if rows is None else len(rows))
+            e["oracle_sample"] = "all tokens" if rows is None else f"{len(rows)} fixed seeded rows"
+        out[f"dbf_mlp_T{T}"] = e
+    # ---- 32 adapters (R = 32, ell = 2) over 256 tokens routed by id
+    w = S.WORKLOADS["segmented"]
+    Ls = S.workload_layers(w)
+    table = dbf.AdapterTable([dev_layer(La) for La in Ls], dev)
+    seg = S.make_segments(w.seed, 256, w.num_adapters)
+    xh = S.make_x(w.seed, 256, w.M, "bf16")[seg.order]
+    x = bf16(np.ascontiguousarray(xh))
+    y = torch.empty((256, w.N), dtype=torch.bfloat16, device=dev)
+    offs = torch.from_numpy(seg.offsets.astype(np.int32)).to(dev)
+    ids = torch.from_numpy(seg.adapter.astype(np.int32)).to(dev)
+    ws = dbf.alloc_workspace(dbf.segmented_workspace_bytes(w.R, w.ell, 256), dev)
+    us = timed(lambda: dbf.forward_segmented(table, offs, ids, x, y=y, ws=ws, stream=stream), 50)
+    nb, fl = algorithmic(w, 256, layers=w.num_adapters)
+    e = entry(f"{w.description}: one segmented call ({len(seg.adapter)} segments), two launches", 256, us, nb, fl,
+              "hbm")
+    if run_oracle:
+        e["oracle_tokens_per_s"] = oracle_rate(
+            lambda: oracle.forward_segmented(Ls, seg.offsets, seg.adapter, xh, nthreads=nthreads), 256)
+        e["oracle_tokens_per_s_1thread"] = oracle_rate(
+            lambda: oracle.forward_segmented(Ls, seg.offsets, seg.adapter, xh, nthreads=1), 256)
+    out["segmented_T256"] = e
+    del table
+    # ---- large prefill layer, M = N = R = 8192 at 8192 tokens
+    w = S.WORKLOADS["large_prefill"]
+    L = S.workload_layers(w)[0]
+    dl = dev_layer(L)
+    T = 8192
+    xh = S.make_x(w.seed, T, w.M, "bf16")
+    x = bf16(xh)
+    y = torch.empty((T, w.N), dtype=torch.bfloat16, device=dev)
+    ws = dbf.alloc_workspace(dbf.workspace_bytes(dl, T), dev)
+    us = timed(lambda: dbf.forward(dl, x, y=y, ws=ws, stream=stream), 10)
+    nb, fl = algorithmic(w, T)
+    e = entry(f"{w.description}: prefill path (fp16 operand pre-pass + two tcgen05 GEMM launches)", T, us, nb, fl,
+              "tensor")
+    if run_oracle:
+        rows = S.sample_rows_per_tile(w.seed, T, ORACLE_ROWS, 256)
+        e["oracle_tokens_per_s"] = oracle_rate(lambda: oracle.forward(L, xh, rows=rows, nthreads=nthreads), len(rows))
+        e["oracle_sample"] = f"{len(rows)} fixed seeded rows"
+    out[f"large_prefill_T{T}"] = e
+    if run_oracle:
+        out["oracle_threads"] = nthreads
+        out["oracle_cpu"] = cpu_model()
+    del flush_buf, x, y, ws
+    torch.cuda.empty_cache()
+    return out
 
 
 def main():
@@ -335,6 +526,30 @@ def main():
     stream_us = max_over_ranks(1e3 * s0.elapsed_time(s1) / n_stream, dev)
     del graph
 
+    # ---- a dependent chain, as through the layers of a served model: the
+    # input of call k+1 is the first M outputs of call k (one token). The
+    # chain's copies have alpha scaled by 2^-12 (exact) so that values stay
+    # finite over the chain; the work per call is the same.
+    chain = [dbf.Layer(Lk.M, Lk.N, Lk.R, Lk.ell, Lk.b1, Lk.b2, Lk.alpha * (2.0 ** -12), Lk.beta, Lk.gamma)
+             for Lk in layers]
+    ybuf = [torch.empty((T_DECODE, w.N), dtype=torch.bfloat16, device=dev) for _ in range(2)]
+    ybuf[1][:, :w.M].copy_(x_dec)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        for i in range(n_stream):
+            src, dst = ybuf[(i + 1) % 2], ybuf[i % 2]
+            dbf.forward(chain[i % COPIES], src[:, :w.M], y=dst, ws=ws_dec, static_weights=True, stream=stream)
+    graph.replay()
+    torch.cuda.synchronize(dev)
+    with torch.cuda.stream(stream):
+        s0.record(stream)
+        graph.replay()
+        s1.record(stream)
+    torch.cuda.synchronize(dev)
+    chain_us = max_over_ranks(1e3 * s0.elapsed_time(s1) / n_stream, dev)
+    chain_finite = bool(torch.isfinite(ybuf[(n_stream - 1) % 2].float()).all())
+    del graph, chain
+
     # ---- backward of the prefill batch (gradients through the layer for
     # training), timed separately: not part of the forward step above
     dy_h = S.make_x(w.seed + 200, T_PREFILL, w.N, "bf16")
@@ -457,6 +672,8 @@ def main():
                   + 2 * fn * fm * fk + 2 * fk * fk * fn + 2 * fk ** 3 + f_admm * 2 * fk * fk * fm)
     del Wf, U0f, V0f, f_ws
 
+    configs = measure_configs(dbf, dev, stream, run_oracle=(world == 1 and not args.no_cpu_baseline))
+
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
@@ -474,18 +691,22 @@ def main():
                 "kernel": "prefill forward (fp16 operand pre-pass + two tcgen05 GEMM launches), one call",
                 "peak_source": f"{pk_kind} bf16 dense (fp16 runs at the same rate)"}
     roof_dec = {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
-                "frac": gbs / pk["hbm_gbs"], "traffic": kernel_traffic("gemv_decode", "double_binary_rank_b200/csrc/dbf_gemv.cu"),
+                "frac": gbs / pk["hbm_gbs"], "traffic": kernel_traffic("decode", "double_binary_rank_b200/csrc/dbf_decode.cu"),
                 "kernel": f"decode forward ({dec_launches} launch: stage 1, grid barrier, stage 2), one call inside the step",
                 "peak_source": f"{pk_kind} copy bandwidth", "us_per_call": dec_us,
-                "stream_us_per_call": stream_us, "stream_frac": b_dec / (stream_us * 1e-6) / 1e9 / pk["hbm_gbs"]}
+                "stream_us_per_call": stream_us, "stream_frac": b_dec / (stream_us * 1e-6) / 1e9 / pk["hbm_gbs"],
+                "stream": f"{n_stream} independent calls back to back in a CUDA graph over the {COPIES} copies",
+                "chain_us_per_call": chain_us, "chain_frac": b_dec / (chain_us * 1e-6) / 1e9 / pk["hbm_gbs"],
+                "chain": f"{n_stream} dependent calls in a CUDA graph (x of call k+1 = first M outputs of call k)",
+                "chain_outputs_finite": chain_finite}
 
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f16", "data": "synthetic",
-        "config": {"workload": w.description, "decode_tokens": T_DECODE, "prefill_tokens": T_PREFILL,
-                   "l2": f"inputs larger than L2: {COPIES} rotating copies of the layer weights",
-                   "arithmetic": "prefill: fp16 x fp16 tensor cores, fp32 accumulate; decode: u8 x s8 tensor cores, exact int32 accumulate"},
+        "config": bench_config(w),
+        "arithmetic": "prefill: fp16 x fp16 tensor cores, fp32 accumulate; decode: binary tensor-core products "
+                      "(and + popcount) over 24 bit planes of the fixed-point activations, exact integer sums",
         "roofline": roof_pre,
         "roofline_decode": roof_dec,
         "prefill_us_per_call": pre_us,
@@ -510,6 +731,7 @@ def main():
                       "frac": fact_flops / (fact_us * 1e-6) / 1e12 / fp32x3_peak,
                       "peak_source": f"{pk_kind} bf16 dense x nominal TF32/BF16 ratio 1.1/2.25, / 3 TF32 products "
                                      "per fp32 multiply-add"},
+        "configs": configs,
         "clocks": clk.summary(),
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": args.steps * (dec_launches + pre_launches),
@@ -517,10 +739,12 @@ def main():
     if world == 1 and not args.no_cpu_baseline:
         import oracle
         nthreads = oracle.default_threads()
-        rows = S.sample_rows(w.seed, T_PREFILL, 1023)
+        rows = oracle_rows(w)
         rate, dt = oracle_sample_rate(w, L, x_dec_h, x_pre_h, rows, nthreads)
         line["cpu_baseline"] = {"value": rate, "unit": "tokens/s", "cores": nthreads, "kind": "oracle",
-                                "sample": f"1 decode token + {len(rows)} fixed seeded rows of the {T_PREFILL}-token prefill ({dt:.1f} s)"}
+                                "cpu": cpu_model(),
+                                "sample": f"1 decode token + {len(rows)} fixed seeded rows of the {T_PREFILL}-token "
+                                          f"prefill ({dt:.1f} s)"}
     print(json.dumps(line), flush=True)
 
 

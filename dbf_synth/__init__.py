@@ -285,3 +285,30 @@ def sample_rows(seed: int, T: int, n: int) -> np.ndarray:
             break
         picks.add(int(v % np.uint64(T)))
     return np.array(sorted(picks), dtype=np.int64)
+
+
+def sample_rows_per_tile(seed: int, T: int, n: int, tile: int) -> np.ndarray:
+    """A fixed, sorted subset of n token rows of T, stratified over tiles of
+    'tile' consecutive rows: every tile holds at least floor(n / tiles) rows
+    (at least one when n >= tiles), and 0 and T-1 are always included."""
+    tiles = (T + tile - 1) // tile
+    if n >= T:
+        return np.arange(T, dtype=np.int64)
+    if n < max(2, tiles):
+        raise ValueError("fewer rows than tiles")
+    key = stream_key(seed, 0x5B, 0, 0)
+    words = iter(raw_u64(key, 64 * n + 64).tolist())
+    picks = {0, T - 1}
+    per = n // tiles
+    for t in range(tiles):
+        lo, hi = t * tile, min(T, (t + 1) * tile)
+        have = sum(1 for p in picks if lo <= p < hi)
+        while have < per:
+            r = lo + next(words) % (hi - lo)
+            if r not in picks:
+                picks.add(r)
+                have += 1
+    while len(picks) < n:
+        r = next(words) % T
+        picks.add(r)
+    return np.array(sorted(picks), dtype=np.int64)

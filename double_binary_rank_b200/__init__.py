@@ -80,6 +80,7 @@ _SIGS = {
                                              ctypes.c_int, _vp, _sz, _vp, _vp]),
     "dbf_forward_decode_noalloc": (ctypes.c_int, [_LP, _vp, ctypes.c_int, _vp, ctypes.c_int, _i64,
                                                   ctypes.c_int, _vp]),
+    "dbf_debug_set_decode_wait_ns": (None, [ctypes.c_uint64]),
     "dbf_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "dbf_version": (ctypes.c_char_p, []),
 }
@@ -205,9 +206,29 @@ def forward_launches(layer: Layer, T: int, path: str = "auto") -> int:
     return int(_lib.dbf_forward_launches(ctypes.byref(d), T, _PATHS[path]))
 
 
+WS_HEADER_BYTES, WS_STATUS_OFFSET = 256, 8
+
+
 def alloc_workspace(nbytes: int, device) -> torch.Tensor:
     # zeroed: the first 256 bytes are a header that must start at zero
-    return torch.zeros(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+    return torch.zeros(max(int(nbytes), WS_HEADER_BYTES), dtype=torch.uint8, device=device)
+
+
+def workspace_status(ws: torch.Tensor) -> int:
+    """The workspace header's device status word (DBF_ERR_TIMEOUT after a
+    bounded device wait expired in a call on this workspace, else OK); reads
+    it with a device-to-host copy on the current stream."""
+    return int(ws[WS_STATUS_OFFSET:WS_STATUS_OFFSET + 4].view(torch.int32).item())
+
+
+def clear_workspace_status(ws: torch.Tensor) -> None:
+    ws[WS_STATUS_OFFSET:WS_STATUS_OFFSET + 4].zero_()
+
+
+def debug_set_decode_wait_ns(ns: int) -> None:
+    """Time limit of the single-launch decode kernel's bounded waits for later
+    calls (0 restores the default of 2 s); for tests of the timeout path."""
+    _lib.dbf_debug_set_decode_wait_ns(int(ns))
 
 
 def _flags(accumulate: bool, static_weights: bool) -> int:

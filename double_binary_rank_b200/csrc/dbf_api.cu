@@ -147,6 +147,8 @@ dbf_status dbf_factorize(const float *W, int64_t n, int64_t m, int64_t k, const 
 
 int64_t dbf_gemm_min_tokens(void) { return kGemmMinTokens; }
 
+void dbf_debug_set_decode_wait_ns(uint64_t ns) { set_decode_wait_ns(ns); }
+
 size_t dbf_workspace_bytes(const dbf_layer *L, int64_t T, dbf_path path)
 {
     if (!L || L->M <= 0 || L->N <= 0 || L->R <= 0 || L->ell < 1 || L->ell > kMaxEll || T < 0)
@@ -154,7 +156,7 @@ size_t dbf_workspace_bytes(const dbf_layer *L, int64_t T, dbf_path path)
     if (path != DBF_PATH_AUTO && path != DBF_PATH_GEMV && path != DBF_PATH_GEMM) return 0;
     const dbf_path p = resolve(*L, T, path);
     if (p == DBF_PATH_GEMM) return gemm_shape_ok(*L) ? gemm_workspace_bytes(*L, T) : 0;
-    return gemv_workspace_bytes(L->R, L->ell, T);
+    return gemv_layer_workspace_bytes(*L, T);
 }
 
 int32_t dbf_forward_launches(const dbf_layer *L, int64_t T, dbf_path path)

@@ -12,24 +12,28 @@
 // Persistent kernel, one CTA per SM; each CTA walks 128 x 256 tiles of
 // D = A B^T (A: 128 sign rows, B: 256 token rows) with two 256-column
 // accumulators in tensor memory, so the epilogue of one tile overlaps the
-// K loop of the next:
-//   warp 0      TMA producer: fp16 activation tiles (64 K x 256 rows, 128-byte
-//               swizzle) into a 5-stage ring;
-//   warp 1      allocates 512 TMEM columns; one thread issues tcgen05.mma
-//               (M = 128, N = 256, K = 16) into the free accumulator and
-//               commits each stage back;
-//   warps 2..5  sign expansion, one tile row per thread: the row's packed
-//               words are read 16 bytes (two K steps) at a time into a
-//               register queue four loads deep, by a cursor that walks the
-//               CTA's tiles without divisions, and expanded to exact fp16 +-1
-//               (or +-alpha) pairs -- a shift and one LOP3 per two signs, the
-//               packed layout keeping columns 2p and 2p+1 in bits p and 16+p --
-//               written in the same 128-byte swizzled K-major layout;
-//   warps 6..9  epilogue, one per lane quarter: tcgen05.ld of a finished
-//               accumulator, scaling, stores, then the accumulator is handed
-//               back to the MMA warp.
-// Every wait is bounded; on expiry the CTA records DBF_ERR_TIMEOUT, stops
-// issuing work, and still frees its tensor memory.
+// K loop of the next. Warp roles of the forward instance (FwdCfg below; the
+// backward instance has one expansion group and eight epilogue warps):
+//   warp 0       TMA producer: fp16 activation tiles (64 K x 256 rows,
+//                128-byte swizzle) into a 4-stage ring;
+//   warp 1       allocates 512 TMEM columns; one thread issues tcgen05.mma
+//                (M = 128, N = 256, K = 16) into the free accumulator and
+//                commits each stage back;
+//   warps 2..9   sign expansion in two groups of four warps that take turns
+//                by pairs of K steps, one tile row per thread: the row's
+//                packed words are read 16 bytes (two K steps) at a time into
+//                a register queue four loads deep, by a cursor that walks the
+//                CTA's tiles without divisions, and expanded to exact fp16
+//                +-1 (or +-alpha) pairs -- a shift and one LOP3 per two
+//                signs, the packed layout keeping columns 2p and 2p+1 in bits
+//                p and 16+p -- written in the same 128-byte swizzled K-major
+//                layout into a 6-stage ring;
+//   warps 10..13 epilogue, one per TMEM lane quarter: tcgen05.ld of a
+//                finished accumulator, scaling, stores, then the accumulator
+//                is handed back to the MMA warp.
+// Every wait is bounded; on expiry the CTA records DBF_ERR_TIMEOUT and stops
+// issuing work; before it frees its tensor memory and ends, the TMA loads
+// and MMAs it already issued are waited for (bounded as well).
 #include "dbf_internal.cuh"
 
 #include <cuda.h>
@@ -205,6 +209,16 @@ __device__ __forceinline__ bool bar_wait(uint64_t *bar, uint32_t parity, volatil
     }
 }
 
+// Wait for phase 'parity' of a barrier whatever the abort flag says, bounded
+// by the same limit: used on the way out so that no asynchronous copy or MMA
+// of this CTA is still in flight when its shared and tensor memory are freed.
+__device__ __forceinline__ void drain_wait(uint64_t *bar, uint32_t parity)
+{
+    const unsigned long long t0 = global_ns();
+    while (!bar_try(bar, parity) && global_ns() - t0 < kWaitNs) {
+    }
+}
+
 __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, int c0, int c1, uint64_t *bar)
 {
     asm volatile(
@@ -274,6 +288,7 @@ __device__ __forceinline__ uint32_t sign_pair(uint32_t w, int p, uint32_t mag2)
 
 struct GemmSmem {
     uint64_t full_a[kMaxStages], empty_a[kMaxStages], full_b[kMaxStages], empty_b[kMaxStages], acc_full[2], acc_empty[2];
+    uint64_t drain;   // the MMA thread's last commit: every MMA it issued has completed
     uint32_t tmem_base;
     int abort;
 };
@@ -432,6 +447,7 @@ __global__ void __launch_bounds__(Cfg::kThreads, 1) gemm_kernel(const __grid_con
             bar_init(&sh->acc_full[i], 1);
             bar_init(&sh->acc_empty[i], kEpiWarps);
         }
+        bar_init(&sh->drain, 1);
         sh->abort = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         asm volatile("prefetch.tensormap [%0];" ::"l"(&tmB) : "memory");
@@ -451,6 +467,7 @@ __global__ void __launch_bounds__(Cfg::kThreads, 1) gemm_kernel(const __grid_con
         // ---------------- TMA producer ----------------
         if (lane == 0) {
             int s = 0;
+            int nb_issued = 0, na_issued = 0;   // TMA loads issued on each ring
             for (int j = 0; j < my_tiles && !*abort; ++j) {
                 const TileRef tr = tile_ref(g, blockIdx.x + j * gridDim.x, n_p);
                 const int c0 = tr.brow;
@@ -460,6 +477,7 @@ __global__ void __launch_bounds__(Cfg::kThreads, 1) gemm_kernel(const __grid_con
                     if (!bar_wait(&sh->empty_b[st], ((s / SB) & 1) ^ 1, abort)) break;
                     bar_expect_tx(&sh->full_b[st], B_BYTES);
                     tma_load_2d(smB + st * B_BYTES, &tmB, k * BK, c0, &sh->full_b[st]);
+                    nb_issued = s + 1;
                     if (g.dense_a) {
                         // a dense fp16 A operand: its tile comes by TMA too, in the
                         // same swizzled K-major layout the expansion writes
@@ -467,8 +485,16 @@ __global__ void __launch_bounds__(Cfg::kThreads, 1) gemm_kernel(const __grid_con
                         if (!bar_wait(&sh->empty_a[sa], ((s / SA) & 1) ^ 1, abort)) break;
                         bar_expect_tx(&sh->full_a[sa], A_BYTES);
                         tma_load_2d(smA + sa * A_BYTES, &tmA, k * BK, p0, &sh->full_a[sa]);
+                        na_issued = s + 1;
                     }
                 }
+            }
+            // After an abort, the loads already issued (at most the last SB,
+            // resp. SA, of each ring: earlier ones were consumed) land before
+            // the CTA ends and its shared memory is released. Bounded.
+            if (*abort) {
+                for (int b = nb_issued - 1; b >= 0 && b >= nb_issued - SB; --b) drain_wait(&sh->full_b[b % SB], (b / SB) & 1);
+                for (int b = na_issued - 1; b >= 0 && b >= na_issued - SA; --b) drain_wait(&sh->full_a[b % SA], (b / SA) & 1);
             }
         }
     } else if (warp == 1) {
@@ -495,8 +521,12 @@ __global__ void __launch_bounds__(Cfg::kThreads, 1) gemm_kernel(const __grid_con
                     mma_commit(&sh->empty_a[sa]);   // each commit arrives once these MMAs are done
                     mma_commit(&sh->empty_b[sb]);
                 }
-                mma_commit(&sh->acc_full[ab]);
+                if (ok) mma_commit(&sh->acc_full[ab]);
             }
+            // every MMA issued (also on an abort) has completed before tensor
+            // memory is freed and the CTA ends
+            mma_commit(&sh->drain);
+            drain_wait(&sh->drain, 0);
         }
     } else if (warp < 2 + kExpandWarps) {
         if (g.dense_a) goto teardown;   // A tiles come by TMA
@@ -861,25 +891,21 @@ template <class Cfg>
 constexpr size_t gemm_smem() { return 1024 + Cfg::SA * A_BYTES + Cfg::SB * B_BYTES + sizeof(GemmSmem) + 64; }
 
 template <class Cfg>
-cudaError_t launch_gemm(const CUtensorMap &map, const GemmArgs &a, cudaStream_t s, const CUtensorMap *map_a = nullptr)
+cudaError_t launch_gemm(const CUtensorMap &map, const GemmArgs &args, cudaStream_t s, const CUtensorMap *map_a,
+                        int32_t *status)
 {
-    static bool configured = false;
-    if (!configured) {
-        cudaError_t e = cudaFuncSetAttribute(gemm_kernel<Cfg>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             static_cast<int>(gemm_smem<Cfg>()));
-        if (e != cudaSuccess) return e;
-        configured = true;
-    }
-    static int sms = 0;
-    if (!sms) {
-        int dev = 0, v = 0;
-        cudaGetDevice(&dev);
-        sms = (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && v > 0) ? v : 148;
-    }
+    GemmArgs a = args;
+    a.status = status;   // a bounded wait that expires stores DBF_ERR_TIMEOUT here
+    cudaError_t e = allow_smem(reinterpret_cast<const void *>(gemm_kernel<Cfg>), static_cast<int>(gemm_smem<Cfg>()));
+    if (e != cudaSuccess) return e;
+    const int sms = device_sms();
     const int tiles = a.ngroups ? a.tiles_total : ((a.P + BM - 1) / BM) * ((a.C + BN - 1) / BN);
     gemm_kernel<Cfg><<<tiles < sms ? tiles : sms, Cfg::kThreads, gemm_smem<Cfg>(), s>>>(map, map_a ? *map_a : map, a);
     return cudaGetLastError();
 }
+
+// the sticky status word of a workspace header
+int32_t *ws_status(void *ws) { return reinterpret_cast<int32_t *>(static_cast<char *>(ws) + kWsStatusOffset); }
 
 size_t u_bytes(const dbf_layer &L, int64_t T) { return align_up(static_cast<size_t>(L.ell) * T * L.M * 2, 256); }
 size_t v_bytes(const dbf_layer &L, int64_t T) { return align_up(static_cast<size_t>(T) * L.ell * L.R * 2, 256); }
@@ -896,6 +922,7 @@ size_t gemm_workspace_bytes(const dbf_layer &L, int64_t T) { return kWsHeaderByt
 cudaError_t gemm_forward(const dbf_layer &L, const void *x, dbf_dtype xd, void *y, dbf_dtype yd, int64_t T,
                          int flags, void *ws, cudaStream_t s)
 {
+    int32_t *st = ws_status(ws);
     if (T > (1 << 30) / L.ell) return cudaErrorInvalidValue;
     char *body = static_cast<char *>(ws) + kWsHeaderBytes;   // the header belongs to the decode path
     __half *U = reinterpret_cast<__half *>(body);
@@ -928,7 +955,7 @@ cudaError_t gemm_forward(const dbf_layer &L, const void *x, dbf_dtype xd, void *
     a1.ell = L.ell;
     a1.R = L.R;
     a1.N = L.N;
-    cudaError_t e = launch_gemm<FwdCfg>(mu, a1, s);
+    cudaError_t e = launch_gemm<FwdCfg>(mu, a1, s, nullptr, st);
     if (e != cudaSuccess) return e;
     GemmArgs a2 = {};
     a2.signs = L.b1_packed;
@@ -946,7 +973,7 @@ cudaError_t gemm_forward(const dbf_layer &L, const void *x, dbf_dtype xd, void *
     a2.yd = yd;
     a2.N = L.N;
     a2.accumulate = (flags & DBF_ACCUMULATE) ? 1 : 0;
-    return launch_gemm<FwdCfg>(mv, a2, s);
+    return launch_gemm<FwdCfg>(mv, a2, s, nullptr, st);
 }
 
 }  // namespace dbf
@@ -1009,7 +1036,7 @@ cudaError_t transpose_f16(const __half *in, int64_t C, int64_t K, __half *out, i
 // operands [P][cp] and [Q][cp], zero past the real length), fp32 out with row
 // pitch P: the dense GEMM of the sign-matrix gradients.
 cudaError_t dense_outer(const __half *A, int64_t P, const __half *Bm, int64_t Q, int64_t cp, float *out, bool acc,
-                        cudaStream_t s)
+                        int32_t *st, cudaStream_t s)
 {
     CUtensorMap ma, mb;
     if (!make_map(&ma, A, cp, P, BM) || !make_map(&mb, Bm, cp, Q, BN)) return cudaErrorInvalidValue;
@@ -1026,7 +1053,7 @@ cudaError_t dense_outer(const __half *A, int64_t P, const __half *Bm, int64_t Q,
     g.yd = DBF_F32;
     g.N = static_cast<int>(P);
     g.accumulate = acc ? 1 : 0;
-    return launch_gemm<FwdCfg>(mb, g, s, &ma);
+    return launch_gemm<FwdCfg>(mb, g, s, &ma, st);
 }
 
 GemmArgs sign_gemm_args(const uint32_t *signs, int P, int K, int C, int T, int ell, int stage)
@@ -1067,6 +1094,7 @@ cudaError_t gemm_backward(const dbf_layer &L, const uint32_t *b1t, const uint32_
                           const void *dy, dbf_dtype dyd, int64_t T, float *dx, float *dalpha, float *dbeta,
                           float *dgamma, float *db1, float *db2, int flags, void *ws, cudaStream_t s)
 {
+    int32_t *st = ws_status(ws);
     if (T > (1 << 30) / L.ell) return cudaErrorInvalidValue;
     const bool acc = (flags & DBF_ACCUMULATE) != 0;
     const int ell = L.ell, Ti = static_cast<int>(T), C = ell * Ti;
@@ -1096,21 +1124,21 @@ cudaError_t gemm_backward(const dbf_layer &L, const uint32_t *b1t, const uint32_
     g3.H32 = H32;
     g3.Vout = Vh;
     g3.cscale = L.beta;
-    if ((e = launch_gemm<BwdCfg>(mu, g3, s)) != cudaSuccess) return e;
+    if ((e = launch_gemm<BwdCfg>(mu, g3, s, nullptr, st)) != cudaSuccess) return e;
     // G4
     GemmArgs g4 = sign_gemm_args(b1t, L.R, L.N, C, Ti, ell, 4);
     g4.H32 = H32;
     g4.Vout = Vg;
     g4.cscale = L.beta;
     g4.red = dbeta;
-    if ((e = launch_gemm<BwdCfg>(ma, g4, s)) != cudaSuccess) return e;
+    if ((e = launch_gemm<BwdCfg>(ma, g4, s, nullptr, st)) != cudaSuccess) return e;
     // G5
     if (dalpha) {
         GemmArgs g5 = sign_gemm_args(L.b1_packed, L.N, L.R, C, Ti, ell, 5);
         g5.red = dalpha;
         g5.W = dy;
         g5.wd = dyd;
-        if ((e = launch_gemm<BwdCfg>(mvh, g5, s)) != cudaSuccess) return e;
+        if ((e = launch_gemm<BwdCfg>(mvh, g5, s, nullptr, st)) != cudaSuccess) return e;
     }
     // G6
     if (dx || dgamma) {
@@ -1121,7 +1149,7 @@ cudaError_t gemm_backward(const dbf_layer &L, const uint32_t *b1t, const uint32_
         g6.cscale = L.gamma;
         g6.dx = dx;
         g6.dx_mode = ell > 1 ? 2 : (acc ? 1 : 0);
-        if ((e = launch_gemm<BwdCfg>(mvg, g6, s)) != cudaSuccess) return e;
+        if ((e = launch_gemm<BwdCfg>(mvg, g6, s, nullptr, st)) != cudaSuccess) return e;
     }
     // sign-matrix gradients: dB1 = sum_c a_c v_c^T (N x R), dB2 = sum_c w_c u_c^T
     // (R x M), dense products contracting over the envelope-major token index
@@ -1131,12 +1159,12 @@ cudaError_t gemm_backward(const dbf_layer &L, const uint32_t *b1t, const uint32_
         if (db1) {
             if ((e = transpose_f16(Vh, C, L.R, Vht, b.cp, s)) != cudaSuccess) return e;
             if ((e = transpose_f16(A, C, L.N, At, b.cp, s)) != cudaSuccess) return e;
-            if ((e = dense_outer(Vht, L.R, At, L.N, b.cp, db1, acc, s)) != cudaSuccess) return e;
+            if ((e = dense_outer(Vht, L.R, At, L.N, b.cp, db1, acc, st, s)) != cudaSuccess) return e;
         }
         if (db2) {
             if ((e = transpose_f16(U, C, L.M, Ut, b.cp, s)) != cudaSuccess) return e;
             if ((e = transpose_f16(Vg, C, L.R, Vgt, b.cp, s)) != cudaSuccess) return e;
-            if ((e = dense_outer(Ut, L.M, Vgt, L.R, b.cp, db2, acc, s)) != cudaSuccess) return e;
+            if ((e = dense_outer(Ut, L.M, Vgt, L.R, b.cp, db2, acc, st, s)) != cudaSuccess) return e;
         }
     }
     return cudaSuccess;
@@ -1163,6 +1191,7 @@ cudaError_t mbok_forward(int M, int N, int K, const uint32_t *w_packed, const ui
                          const void *x, dbf_dtype xd, void *y, dbf_dtype yd, int64_t T, int flags, void *ws,
                          cudaStream_t s)
 {
+    int32_t *st = ws_status(ws);
     if (T > (1 << 30) / K) return cudaErrorInvalidValue;
     __half *U = reinterpret_cast<__half *>(static_cast<char *>(ws) + kWsHeaderBytes);
     cudaError_t e = scale_cast(x, xd, s_in, M, T, K, U, s, 1);
@@ -1185,7 +1214,7 @@ cudaError_t mbok_forward(int M, int N, int K, const uint32_t *w_packed, const ui
     a.yd = yd;
     a.N = N;
     a.accumulate = (flags & DBF_ACCUMULATE) ? 1 : 0;
-    return launch_gemm<FwdCfg>(mu, a, s);
+    return launch_gemm<FwdCfg>(mu, a, s, nullptr, st);
 }
 
 }  // namespace dbf
@@ -1200,6 +1229,7 @@ cudaError_t gemm_forward_grouped(const dbf_layer *const *layers, const int *off,
                                  const void *x, dbf_dtype xd, void *y, dbf_dtype yd, int64_t T, int flags, void *ws,
                                  cudaStream_t s)
 {
+    int32_t *st = ws_status(ws);
     if (count < 1 || count > kMaxGroups) return cudaErrorInvalidValue;
     const dbf_layer &L = *layers[0];
     if (T > (1 << 30) / L.ell) return cudaErrorInvalidValue;
@@ -1263,9 +1293,9 @@ cudaError_t gemm_forward_grouped(const dbf_layer *const *layers, const int *off,
     a1.ngroups = a2.ngroups = count;
     a1.tiles_total = t1;
     a2.tiles_total = t2;
-    cudaError_t e = launch_gemm<FwdCfg>(mu, a1, s);
+    cudaError_t e = launch_gemm<FwdCfg>(mu, a1, s, nullptr, st);
     if (e != cudaSuccess) return e;
-    return launch_gemm<FwdCfg>(mv, a2, s);
+    return launch_gemm<FwdCfg>(mv, a2, s, nullptr, st);
 }
 
 }  // namespace dbf

@@ -1,4 +1,7 @@
-// Decode-regime forward: two sign-accumulation GEMVs with per-channel scaling.
+// Decode-regime forward in two launches: two sign-accumulation GEMVs with
+// per-channel scaling, for the calls the single-launch kernel (dbf_decode.cu)
+// does not take -- more than eight (token, envelope) columns, M or R above
+// 8192 -- and for segmented multi-adapter serving.
 //
 // LoRDBA page, section 2 ("Kernel de Inferencia"): the forward is two
 // sign-accumulation matrix products interleaved with per-channel scaling;
@@ -46,7 +49,6 @@ constexpr int kWarps = 8;
 constexpr int kThreads = kWarps * 32;
 constexpr int kMaxCtas = 160;      // per segment; sizes the per-CTA partial sums
 constexpr int kSmemCap = 220 * 1024;
-constexpr int kCoResidentSmem = 113 * 1024;   // two CTAs per SM (228 KB, 1 KB reserved per CTA)
 constexpr int kPrefetchCap = 128 * 1024;
 constexpr unsigned long long kWaitNs = 2000000000ull;   // bounded wait: 2 s
 
@@ -78,9 +80,6 @@ struct GemvParams {
     int32_t off_digits, off_colinfo, off_tiles, off_bar, off_ubuf, off_rscale;
     int32_t nb_max;               // row blocks per CTA batch (tiles)
     int32_t pdl_wait;             // launched as a programmatic dependent of the previous kernel
-    // single-launch decode: second slice, its row scales, and the barrier counter
-    int32_t off_s2, off_rscale2, slice_rows2;
-    unsigned *hdr;
 };
 
 // Bytes per digit column: 32 per packed word (one byte per column of K),
@@ -231,7 +230,7 @@ struct Smem {
     int *tiles;          // [nb_max][16][kMaxBcols] int32
     uint32_t *signs;     // [prefetch_rows][pitch]
     float4 *ubuf;        // staging of gamma.x quads when K needs several load rounds
-    uint64_t *bar;       // [0] sign slice, [1] digit image, [2] second sign slice (single launch)
+    uint64_t *bar;       // [0] sign slice, [1] digit image
     int *flag;
 };
 
@@ -753,566 +752,7 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_kernel(const GemvParams P)
     }
 }
 
-// ---- single-launch decode ------------------------------------------------------
-// When every column of the call fits one pass (T ell <= 8) the two stages run
-// in one kernel: each CTA owns a range of stage-1 rows and a range of
-// stage-2 rows, copies both sign slices to shared memory at once, and the
-// exchange of the v image goes through a grid-wide barrier on a counter in
-// the workspace header instead of a kernel boundary.
-//
-// Barrier counter: header word 0 counts arrivals, word 1 is the count at which
-// the current call's barrier started. Every CTA reads word 1 (after the
-// previous kernel in the stream has completed), adds one arrival, waits until
-// G arrivals past that start, and writes start + G back to word 1. Each CTA
-// arrives exactly once, even after a timed-out wait, so the two words are
-// equal again when the kernel ends. They must be equal (zero) when the
-// workspace is first used.
-
-// Digits of one stage-1 column u = gamma_i . x_t (layout and scales as in
-// stage1_column). Two threads per packed word: unit (w, hf) holds columns
-// 32w + 8hf + [0, 8) and 32w + 16 + 8hf + [0, 8), which make up the quads
-// k0 = 32w + 8hf + 2p, p = 0..3. VEC: 16-byte loads (K % 8 == 0 and gamma
-// 16-byte aligned).
-constexpr int kFusedUnits = 2;   // units per thread held in registers
-
-// max |beta| over every envelope and rank (the same value in every CTA). The
-// first 8192 values are loaded by beta_prefetch, 16 bytes per thread and
-// load, so that their latency overlaps other loads; beta_absmax folds them
-// and reads any rest. fp16 magnitudes order like their bit patterns, so the
-// maximum is taken on the bits, two at a time.
-constexpr int kBetaVecs = 4;   // 16-byte beta loads per thread in the first round
-
-__device__ __forceinline__ bool beta_vec_ok(const dbf_layer &L)
-{
-    return (reinterpret_cast<uintptr_t>(L.beta) & 15u) == 0;
-}
-
-__device__ __forceinline__ void beta_prefetch(const dbf_layer &L, uint4 (&bq)[kBetaVecs])
-{
-    const int nv = beta_vec_ok(L) ? L.R * L.ell / 8 : 0;
-    const uint4 *bp = reinterpret_cast<const uint4 *>(L.beta);
-#pragma unroll
-    for (int e = 0; e < kBetaVecs; ++e) {
-        const int idx = threadIdx.x + e * kThreads;
-        bq[e] = idx < nv ? __ldg(bp + idx) : make_uint4(0u, 0u, 0u, 0u);
-    }
-}
-
-// max |beta| of this thread's share, as a float bit pattern
-__device__ __forceinline__ unsigned beta_absmax(const dbf_layer &L, const uint4 (&bq)[kBetaVecs])
-{
-    const int nb = L.R * L.ell;
-    const int nv = beta_vec_ok(L) ? nb / 8 : 0;
-    unsigned m2 = 0u;   // two 16-bit magnitudes
-#pragma unroll
-    for (int e = 0; e < kBetaVecs; ++e) {
-        m2 = __vmaxu2(m2, bq[e].x & 0x7FFF7FFFu);
-        m2 = __vmaxu2(m2, bq[e].y & 0x7FFF7FFFu);
-        m2 = __vmaxu2(m2, bq[e].z & 0x7FFF7FFFu);
-        m2 = __vmaxu2(m2, bq[e].w & 0x7FFF7FFFu);
-    }
-    const uint4 *bp = reinterpret_cast<const uint4 *>(L.beta);
-    for (int v0 = threadIdx.x + kBetaVecs * kThreads; v0 < nv; v0 += kBetaVecs * kThreads) {
-        uint4 w[kBetaVecs];
-#pragma unroll
-        for (int e = 0; e < kBetaVecs; ++e) {
-            const int idx = v0 + e * kThreads;
-            w[e] = idx < nv ? __ldg(bp + idx) : make_uint4(0u, 0u, 0u, 0u);
-        }
-#pragma unroll
-        for (int e = 0; e < kBetaVecs; ++e) {
-            m2 = __vmaxu2(m2, w[e].x & 0x7FFF7FFFu);
-            m2 = __vmaxu2(m2, w[e].y & 0x7FFF7FFFu);
-            m2 = __vmaxu2(m2, w[e].z & 0x7FFF7FFFu);
-            m2 = __vmaxu2(m2, w[e].w & 0x7FFF7FFFu);
-        }
-    }
-    for (int base = nv * 8 + threadIdx.x; base < nb; base += 8 * kThreads) {
-        unsigned h[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-            const int idx = base + e * kThreads;
-            h[e] = idx < nb ? (__ldg(L.beta + idx) & 0x7FFFu) : 0u;
-        }
-#pragma unroll
-        for (int e = 0; e < 8; ++e) m2 = __vmaxu2(m2, h[e]);
-    }
-    const unsigned bits = max(m2 & 0xFFFFu, m2 >> 16);
-    return __float_as_uint(__half2float(__ushort_as_half(static_cast<unsigned short>(bits))));
-}
-
-// Row scales of a CTA in two steps, so that their load latency overlaps other
-// work: fetch into registers, later store to shared memory.
-__device__ __forceinline__ void fetch_row_scales(const uint16_t *scale, int ld, int ell, int row_lo, int nrows,
-                                                 float (&v)[kScalesPerThread])
-{
-    const int n = nrows * ell;   // 0 when the CTA has no rows
-    if (ell == 1) {
-#pragma unroll
-        for (int e = 0; e < kScalesPerThread; ++e) {
-            const int idx = threadIdx.x + e * kThreads;
-            v[e] = idx < n ? ldg_h(scale + row_lo + idx) : 0.f;
-        }
-        return;
-    }
-#pragma unroll
-    for (int e = 0; e < kScalesPerThread; ++e) {
-        const int idx = threadIdx.x + e * kThreads;
-        const bool ok = idx < n;
-        const int i = ok ? idx / nrows : 0, r = ok ? idx - (idx / nrows) * nrows : 0;
-        v[e] = ok ? ldg_h(scale + static_cast<int64_t>(i) * ld + row_lo + r) : 0.f;
-    }
-}
-
-__device__ __forceinline__ void store_row_scales(const float (&v)[kScalesPerThread], int ell, int nrows, float *dst)
-{
-    const int n = nrows * ell;
-#pragma unroll
-    for (int e = 0; e < kScalesPerThread; ++e) {
-        const int idx = threadIdx.x + e * kThreads;
-        if (idx < n) dst[idx] = v[e];
-    }
-}
-
-
-template <bool XBF16, bool VEC>
-__device__ void fused_column(const GemvParams &P, const dbf_layer &L, int64_t t, int i, int lc, char *digits, int cb,
-                             const Smem &S, bool with_beta, const uint4 (&bq)[kBetaVecs])
-{
-    const int K = L.M;
-    const int pitch = static_cast<int>(pitch_words(K));
-    const int units = 2 * ((pitch + kGroupWords - 1) / kGroupWords * kGroupWords);
-    const int lane = threadIdx.x & 31;
-    const uint16_t *gp = L.gamma + static_cast<int64_t>(i) * K;
-    const int64_t xb = t * K;
-    // ---- loads: every one issued before any use (column info was zeroed and
-    // published by the caller)
-    float g[kFusedUnits][16], xv[kFusedUnits][16];
-#pragma unroll
-    for (int e = 0; e < kFusedUnits; ++e) {
-        const int u = threadIdx.x + e * kThreads;
-        const int w = u >> 1, hf = u & 1;
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {
-            const int k0 = 32 * w + 16 * half + 8 * hf;
-            if (VEC) {
-                const bool in = u < units && k0 < K;   // K % 8 == 0: a chunk is wholly in or out
-                const int kc = in ? k0 : 0;
-                const uint4 gw = __ldg(reinterpret_cast<const uint4 *>(gp + kc));
-                const __half *gh = reinterpret_cast<const __half *>(&gw);
-#pragma unroll
-                for (int c = 0; c < 8; ++c) g[e][8 * half + c] = in ? __half2float(gh[c]) : 0.f;
-                if (XBF16) {
-                    const uint4 xw = __ldg(reinterpret_cast<const uint4 *>(static_cast<const __nv_bfloat16 *>(P.x) + xb + kc));
-                    const __nv_bfloat16 *xh = reinterpret_cast<const __nv_bfloat16 *>(&xw);
-#pragma unroll
-                    for (int c = 0; c < 8; ++c) xv[e][8 * half + c] = __bfloat162float(xh[c]);
-                } else {
-                    const float4 *xf = reinterpret_cast<const float4 *>(static_cast<const float *>(P.x) + xb + kc);
-                    const float4 a = __ldg(xf), b = __ldg(xf + 1);
-                    xv[e][8 * half + 0] = a.x; xv[e][8 * half + 1] = a.y; xv[e][8 * half + 2] = a.z; xv[e][8 * half + 3] = a.w;
-                    xv[e][8 * half + 4] = b.x; xv[e][8 * half + 5] = b.y; xv[e][8 * half + 6] = b.z; xv[e][8 * half + 7] = b.w;
-                }
-            } else {
-#pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    const bool in = u < units && k0 + c < K;
-                    const int kk = in ? k0 + c : 0;
-                    g[e][8 * half + c] = in ? ldg_h(gp + kk) : 0.f;
-                    xv[e][8 * half + c] = ldg_x<XBF16>(P.x, xb + kk);
-                }
-            }
-        }
-    }
-    float m = 0.f;
-#pragma unroll
-    for (int e = 0; e < kFusedUnits; ++e)
-#pragma unroll
-        for (int c = 0; c < 16; ++c) {
-            xv[e][c] *= g[e][c];   // gamma . x, exact in fp32
-            m = fmaxf(m, fabsf(xv[e][c]));
-        }
-    const unsigned mw = warp_max(__float_as_uint(m));
-    if (lane == 0) atomicMax(&S.col[lc].amax, mw);
-    if (with_beta) {
-        const unsigned bw = warp_max(beta_absmax(L, bq));
-        if (lane == 0) atomicMax(S.bmax, bw);
-    }
-    __syncthreads();
-    const int sh = scale_exponent(__uint_as_float(S.col[lc].amax));
-    const bool plain = sh >= -126 && sh <= 126;
-    const float scale = plain ? exp2i(sh) : 0.f;
-    char *plane0 = digits + static_cast<size_t>(kPlanes * lc) * cb;
-    int sq = 0, sa = 0;
-#pragma unroll
-    for (int e = 0; e < kFusedUnits; ++e) {
-        const int u = threadIdx.x + e * kThreads;
-        if (u < units) {
-            const int w = u >> 1, hf = u & 1;
-#pragma unroll
-            for (int p = 0; p < 4; ++p) {
-                // quad k0, k0 + 16, k0 + 1, k0 + 17 with k0 = 32 w + 8 hf + 2 p
-                const int q0 = quantize(xv[e][2 * p], scale, sh, plain);
-                const int q1 = quantize(xv[e][8 + 2 * p], scale, sh, plain);
-                const int q2 = quantize(xv[e][2 * p + 1], scale, sh, plain);
-                const int q3 = quantize(xv[e][8 + 2 * p + 1], scale, sh, plain);
-                sq += q0 + q1 + q2 + q3;
-                sa += abs(q0) + abs(q1) + abs(q2) + abs(q3);
-                store_quad(plane0, cb, digit_offset(32 * w + 8 * hf + 2 * p), q0, q1, q2, q3);
-            }
-        }
-    }
-    const long long sq64 = warp_sum64(sq), sa64 = warp_sum64(sa);
-    if (lane == 0) {
-        atomicAdd(reinterpret_cast<unsigned long long *>(&S.col[lc].qsum), static_cast<unsigned long long>(sq64));
-        atomicAdd(reinterpret_cast<unsigned long long *>(&S.col[lc].qabs), static_cast<unsigned long long>(sa64));
-    }
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        S.col[lc].sh = sh;
-        const float bound = __uint_as_float(*S.bmax) * scale_pow2(static_cast<float>(S.col[lc].qabs), -sh) *
-                            (1.0f + 1.0f / 1024.0f);
-        S.col[lc].sh_next = scale_exponent(bound);
-    }
-}
-
-__device__ __forceinline__ unsigned ld_acquire(const unsigned *p)
-{
-    unsigned v;
-    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-    return v;
-}
-
-// Grid-wide barrier on the header counter (see above); false on timeout.
-__device__ bool grid_barrier(unsigned *hdr, unsigned start, int32_t *status, int *flag)
-{
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        __threadfence();
-        atomicAdd(hdr, 1u);
-        bool ok = true;
-        const unsigned long long t0 = global_ns();
-        while (ld_acquire(hdr) - start < gridDim.x) {
-            if (global_ns() - t0 > kWaitNs) {
-                ok = false;
-                set_status(status, DBF_ERR_TIMEOUT);
-                break;
-            }
-        }
-        __threadfence();
-        hdr[1] = start + gridDim.x;
-        *flag = ok ? 1 : 0;
-    }
-    __syncthreads();
-    return *flag != 0;
-}
-
-// Row stride in shared memory of a sign slice. The MMA units read 8 bytes per
-// lane from rows g = 0..7 at once; a stride of 0 or 16 words modulo 32 puts
-// those rows on the same banks, so such pitches get 4 words of padding (the
-// copy then goes row by row).
-__host__ __device__ inline int slice_stride(int pitch) { return (pitch % 16 == 0) ? pitch + 4 : pitch; }
-
-// Copy rows x pitch packed words into a slice with row stride
-// slice_stride(pitch); called by one whole warp after the barrier's
-// expect_tx. One bulk copy when unpadded, else one per row.
-__device__ __forceinline__ void copy_slice(uint32_t *dst, const uint32_t *src, int rows, int pitch, uint64_t *bar)
-{
-    if (rows <= 0) return;
-    const int lane = threadIdx.x & 31;
-    const int ss = slice_stride(pitch);
-    if (ss == pitch) {
-        if (lane == 0) bulk_copy(dst, src, static_cast<uint32_t>(rows) * pitch * 4u, bar);
-        return;
-    }
-    for (int r = lane; r < rows; r += 32)
-        bulk_g2s(dst + static_cast<int64_t>(r) * ss, src + static_cast<int64_t>(r) * pitch, static_cast<uint32_t>(pitch) * 4u,
-                 bar);
-}
-
-// Rows [rb_begin, rb_end) of one stage: MMA units over the CTA's row blocks in
-// chunks of nb_max, then the stage's epilogue (stage 1: v into the digit
-// image and the CTA's sums of q; stage 2: y).
-template <int STAGE>
-__device__ __forceinline__ void fused_rows(const GemvParams &P, const dbf_layer &L, int rb_begin, int rb_end,
-                                           const uint32_t *Sg, const uint32_t *slice, int sstride, int K, int rows,
-                                           const char *digits, const char *zero_col, int cb, int ncl,
-                                           const float *rscale, int nb_max, const Smem &S,
-                                           long long (&qpart_local)[kMaxNcl])
-{
-    const int warp = threadIdx.x >> 5;
-    const int lane = threadIdx.x & 31;
-    const int ell = L.ell;
-    const int pitch = static_cast<int>(pitch_words(K));
-    const bool even = (pitch % 2 == 0) && ((reinterpret_cast<uintptr_t>(Sg) & 7u) == 0);
-    const int ngrp = (pitch + kGroupWords - 1) / kGroupWords;
-    const int bcols = kPlanes * ncl;
-    const int ngroups = (bcols + 7) / 8;
-    const int ntok = ncl / ell;
-    const int row_lo = rb_begin * kRows;
-    const int nrows = min(rb_end * kRows, rows) - row_lo;
-    int *tiles = S.tiles;
-    for (int rbb = rb_begin; rbb < rb_end; rbb += nb_max) {
-        const int nb = min(nb_max, rb_end - rbb);
-        for (int idx = threadIdx.x; idx < nb * kRows * kMaxBcols; idx += blockDim.x) tiles[idx] = 0;
-        __syncthreads();
-        const int units = nb * ngrp;
-        int u = units * warp / kWarps;
-        const int uend = units * (warp + 1) / kWarps;
-        while (u < uend) {
-            const int b = u / ngrp;
-            const int g0 = u - b * ngrp;
-            const int g1 = min(ngrp, g0 + (uend - u));
-            const int row0 = (rbb + b) * kRows;
-            const int g = lane >> 2;
-            const bool va = row0 + g < rows, vb = row0 + g + 8 < rows;
-            if (slice) {
-                const uint32_t *base = slice + static_cast<int64_t>(row0 + g - row_lo) * sstride;
-                warp_run<true>(base, base + 8 * sstride, va, vb, pitch, even, g0, g1, digits, zero_col, ngroups, bcols,
-                               cb, tiles + b * kRows * kMaxBcols);
-            } else {
-                const uint32_t *base = Sg + static_cast<int64_t>(row0 + g) * pitch;
-                warp_run<false>(base, base + 8 * pitch, va, vb, pitch, even, g0, g1, digits, zero_col, ngroups, bcols,
-                                cb, tiles + b * kRows * kMaxBcols);
-            }
-            u += g1 - g0;
-        }
-        __syncthreads();
-        if (STAGE == 1) {
-            // v = beta . h, digitised with the scale every CTA derived alike
-            for (int idx = threadIdx.x; idx < nb * kRows * ncl; idx += blockDim.x) {
-                const int row = idx % (nb * kRows);
-                const int lc = idx / (nb * kRows);
-                const int r = rbb * kRows + row;
-                if (r >= rows) continue;
-                const ColInfo &ci = S.col[lc];
-                const float h =
-                    scale_pow2(__ll2float_rn(ci.qsum - 2 * plane_sum(tiles + row * kMaxBcols, lc)), -ci.sh);
-                const int tok = lc / ell, i = lc - tok * ell;
-                const float v = rscale[i * nrows + (r - row_lo)] * h;
-                const int sh2 = ci.sh_next;
-                const bool plain = sh2 >= -126 && sh2 <= 126;
-                const int q = quantize(v, plain ? exp2i(sh2) : 0.f, sh2, plain);
-                const uint32_t db = digit_bytes(q);
-                char *img = P.img + static_cast<size_t>(tok * P.ell_cap + i) * kPlanes * P.cb2 + digit_offset(r);
-                img[0] = static_cast<char>(db & 255u);
-                img[P.cb2] = static_cast<char>((db >> 8) & 255u);
-                img[2 * P.cb2] = static_cast<char>(db >> 16);
-#pragma unroll
-                for (int c = 0; c < kMaxNcl; ++c)
-                    if (c == lc) qpart_local[c] += q;
-            }
-        } else {
-            for (int idx = threadIdx.x; idx < nb * kRows * ntok; idx += blockDim.x) {
-                const int row = idx % (nb * kRows);
-                const int tok = idx / (nb * kRows);
-                const int n = rbb * kRows + row;
-                if (n >= rows) continue;
-                const int64_t t = tok;
-                float yv = (P.flags & DBF_ACCUMULATE) ? load_act(P.y, P.yd, t * P.N + n) : 0.f;
-                for (int i = 0; i < ell; ++i) {
-                    const int lc = tok * ell + i;
-                    const ColInfo &ci = S.col[lc];
-                    const float z =
-                        scale_pow2(__ll2float_rn(ci.qsum - 2 * plane_sum(tiles + row * kMaxBcols, lc)), -ci.sh);
-                    yv += rscale[i * nrows + (n - row_lo)] * z;
-                }
-                store_act(P.y, P.yd, t * P.N + n, yv);
-            }
-        }
-        __syncthreads();
-    }
-}
-
-template <bool XBF16, bool VEC>
-__global__ void __launch_bounds__(kThreads, 2) gemv_fused_kernel(const GemvParams P)
-{
-    extern __shared__ __align__(128) char smem[];
-    const int warp = threadIdx.x >> 5;
-    const int lane = threadIdx.x & 31;
-    pdl_trigger();
-    const bool early = (P.flags & DBF_WEIGHTS_STATIC) != 0;
-    if (!early) pdl_wait();
-
-    const dbf_layer &L = P.layer;
-    const int ell = L.ell;
-    const int ncl = static_cast<int>(P.T) * ell;
-    const int G = gridDim.x, b = blockIdx.x;
-    const int nrb1 = (L.R + kRows - 1) / kRows, nrb2 = (L.N + kRows - 1) / kRows;
-    const int rb1b = static_cast<int>(static_cast<int64_t>(nrb1) * b / G);
-    const int rb1e = static_cast<int>(static_cast<int64_t>(nrb1) * (b + 1) / G);
-    const int rb2b = static_cast<int>(static_cast<int64_t>(nrb2) * b / G);
-    const int rb2e = static_cast<int>(static_cast<int64_t>(nrb2) * (b + 1) / G);
-    const int pitch1 = static_cast<int>(pitch_words(L.M)), pitch2 = static_cast<int>(pitch_words(L.R));
-    const int cb1 = col_bytes(pitch1), cb2 = P.cb2;
-    const int lo1 = rb1b * kRows, lo2 = rb2b * kRows;
-    const int nrows1 = rb1e > rb1b ? min(rb1e * kRows, L.R) - lo1 : 0;
-    const int nrows2 = rb2e > rb2b ? min(rb2e * kRows, L.N) - lo2 : 0;
-
-    Smem S;
-    S.signs = reinterpret_cast<uint32_t *>(smem);   // stage-1 slice at offset 0
-    uint32_t *slice2 = reinterpret_cast<uint32_t *>(smem + P.off_s2);
-    S.digits = smem + P.off_digits;
-    S.col = reinterpret_cast<ColInfo *>(smem + P.off_colinfo);
-    S.bmax = reinterpret_cast<unsigned *>(S.col + kMaxNcl);
-    S.tiles = reinterpret_cast<int *>(smem + P.off_tiles);
-    S.bar = reinterpret_cast<uint64_t *>(smem + P.off_bar);
-    S.flag = reinterpret_cast<int *>(smem + P.off_bar + 32);
-    float *rs1 = reinterpret_cast<float *>(smem + P.off_rscale);
-    float *rs2 = reinterpret_cast<float *>(smem + P.off_rscale2);
-    const bool use1 = P.prefetch_rows > 0 && nrows1 > 0;
-    const bool use2 = P.slice_rows2 > 0 && nrows2 > 0;
-
-    // ---- both sign slices -> shared memory, in flight from the start
-    if (threadIdx.x == 0) {
-        bar_init(&S.bar[0], 1);
-        bar_init(&S.bar[1], 1);
-        bar_init(&S.bar[2], 1);
-        *S.bmax = 0u;
-        for (int lc = 0; lc < ncl; ++lc) {
-            S.col[lc].amax = 0u;
-            S.col[lc].qsum = 0;
-            S.col[lc].qabs = 0;
-        }
-        if (use1) bar_expect_tx(&S.bar[0], static_cast<uint32_t>(nrows1) * pitch1 * 4u);
-        if (use2) bar_expect_tx(&S.bar[2], static_cast<uint32_t>(nrows2) * pitch2 * 4u);
-    }
-    if (warp == 0) {
-        __syncwarp();
-        copy_slice(S.signs, L.b2_packed + static_cast<int64_t>(lo1) * pitch1, use1 ? nrows1 : 0, pitch1, &S.bar[0]);
-        copy_slice(slice2, L.b1_packed + static_cast<int64_t>(lo2) * pitch2, use2 ? nrows2 : 0, pitch2, &S.bar[2]);
-    }
-    // weights (signs and scales) may be read before the previous kernel ends
-    // only with static weights
-    if (!early) pdl_wait();
-    float sv1[kScalesPerThread], sv2[kScalesPerThread];
-    fetch_row_scales(L.beta, L.R, ell, lo1, nrows1, sv1);
-    fetch_row_scales(L.alpha, L.N, ell, lo2, nrows2, sv2);
-    uint4 bq[kBetaVecs];
-    beta_prefetch(L, bq);
-    if (early) pdl_wait();
-    // the barrier's starting count: stable once the previous kernel has completed
-    const unsigned start = threadIdx.x == 0 ? *reinterpret_cast<volatile unsigned *>(P.hdr + 1) : 0u;
-    char *zero1 = S.digits + static_cast<size_t>(kPlanes) * ncl * cb1;
-    for (int i = threadIdx.x; i < cb1 / 16; i += blockDim.x) reinterpret_cast<uint4 *>(zero1)[i] = make_uint4(0u, 0u, 0u, 0u);
-    __syncthreads();   // column info and *S.bmax zeroed
-
-    // ---- stage 1: digits of gamma . x, then the CTA's rows of v
-    for (int lc = 0; lc < ncl; ++lc) {
-        const int tok = lc / ell, i = lc - tok * ell;
-        fused_column<XBF16, VEC>(P, L, tok, i, lc, S.digits, cb1, S, lc == 0, bq);
-    }
-    // the row scales arrived during the digit build
-    store_row_scales(sv1, ell, nrows1, rs1);
-    store_row_scales(sv2, ell, nrows2, rs2);
-    __syncthreads();
-    bool ok = true;
-    long long qpart_local[kMaxNcl];
-#pragma unroll
-    for (int c = 0; c < kMaxNcl; ++c) qpart_local[c] = 0;
-    if (nrows1 > 0) {
-        if (use1) ok = wait_flag(S, 0, 0, P.status);
-        if (ok)
-            fused_rows<1>(P, L, rb1b, rb1e, L.b2_packed, use1 ? S.signs : nullptr, slice_stride(pitch1), L.M, L.R,
-                          S.digits, zero1, cb1,
-                          ncl, rs1, P.nb_max, S, qpart_local);
-    }
-    if (rb1e == nrb1 && rb1e > rb1b) {
-        // the owner of the last row block zeroes the image past the rank
-        const int kp2 = cb2 - 32;
-        for (int idx = threadIdx.x; idx < ncl * (kp2 - L.R); idx += blockDim.x) {
-            const int lc = idx / (kp2 - L.R);
-            const int r = L.R + idx % (kp2 - L.R);
-            const int tok = lc / ell, i = lc - tok * ell;
-            char *img = P.img + static_cast<size_t>(tok * P.ell_cap + i) * kPlanes * cb2 + digit_offset(r);
-            img[0] = 0;
-            img[cb2] = 0;
-            img[2 * cb2] = 0;
-        }
-    }
-    {
-        long long *red = reinterpret_cast<long long *>(S.tiles);
-        for (int lc = threadIdx.x; lc < ncl; lc += blockDim.x) red[lc] = 0;
-        __syncthreads();
-        for (int lc = 0; lc < ncl; ++lc) {
-            long long v = 0;
-#pragma unroll
-            for (int c = 0; c < kMaxNcl; ++c)
-                if (c == lc) v = qpart_local[c];
-            v = warp_sum64(v);
-            if (lane == 0) atomicAdd(reinterpret_cast<unsigned long long *>(&red[lc]), static_cast<unsigned long long>(v));
-        }
-        __syncthreads();
-        for (int lc = threadIdx.x; lc < ncl; lc += blockDim.x) {
-            const int tok = lc / ell, i = lc - tok * ell;
-            P.qpart[static_cast<int64_t>(b) * P.T * P.ell_cap + tok * P.ell_cap + i] = red[lc];
-        }
-    }
-
-    // ---- every CTA's image rows and sums are written
-    const bool passed = grid_barrier(P.hdr, start, P.status, S.flag);
-    if (!passed || !ok || nrows2 <= 0) {
-        if (use2) wait_flag(S, 2, 0, P.status);   // no copy left in flight
-        return;
-    }
-
-    // ---- stage 2: the v image (coherent 16-byte loads: other CTAs wrote it in
-    // this kernel), the sums of q, then the CTA's rows of y
-    {
-        // columns lc = tok ell + i are stored back to back (ell_cap == ell here)
-        const int n16 = ncl * kPlanes * cb2 / 16;
-        const uint4 *src = reinterpret_cast<const uint4 *>(P.img);
-        uint4 *dst = reinterpret_cast<uint4 *>(S.digits);
-        constexpr int kImgLoads = 8;
-        for (int i0 = threadIdx.x; i0 < n16; i0 += kImgLoads * kThreads) {
-            uint4 v[kImgLoads];
-#pragma unroll
-            for (int e = 0; e < kImgLoads; ++e) {
-                const int i = i0 + e * kThreads;
-                v[e] = i < n16 ? __ldcg(src + i) : make_uint4(0u, 0u, 0u, 0u);
-            }
-#pragma unroll
-            for (int e = 0; e < kImgLoads; ++e)
-                if (i0 + e * kThreads < n16) dst[i0 + e * kThreads] = v[e];
-        }
-    }
-    char *zero2 = S.digits + static_cast<size_t>(kPlanes) * ncl * cb2;
-    for (int i = threadIdx.x; i < cb2 / 16; i += blockDim.x) reinterpret_cast<uint4 *>(zero2)[i] = make_uint4(0u, 0u, 0u, 0u);
-    for (int lc = warp; lc < ncl; lc += kWarps) {
-        const int tok = lc / ell, i = lc - tok * ell;
-        const int64_t c = tok * P.ell_cap + i;
-        long long part[kMaxCtas / 32];
-#pragma unroll
-        for (int e = 0; e < kMaxCtas / 32; ++e) {
-            const int k = lane + 32 * e;
-            part[e] = k < G ? __ldcg(P.qpart + static_cast<int64_t>(k) * P.T * P.ell_cap + c) : 0;
-        }
-        long long sq = 0;
-#pragma unroll
-        for (int e = 0; e < kMaxCtas / 32; ++e) sq += part[e];
-        sq = warp_sum64(sq);
-        if (lane == 0) {
-            S.col[lc].qsum = sq;
-            S.col[lc].sh = S.col[lc].sh_next;
-        }
-    }
-    if (use2 && !wait_flag(S, 2, 0, P.status)) return;   // also publishes the image and the sums
-    __syncthreads();
-    fused_rows<2>(P, L, rb2b, rb2e, L.b1_packed, use2 ? slice2 : nullptr, slice_stride(pitch2), L.R, L.N, S.digits,
-                  zero2, cb2, ncl, rs2,
-                  P.nb_max, S, qpart_local);
-}
-
-int num_sms()
-{
-    static int sms = 0;
-    if (!sms) {
-        int dev = 0, v = 0;
-        cudaGetDevice(&dev);
-        sms = (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && v > 0) ? v : 148;
-    }
-    return sms;
-}
+int num_sms() { return device_sms(); }
 
 int quads_of(int pitch) { return (pitch + kGroupWords - 1) / kGroupWords * kGroupWords * 8; }
 
@@ -1379,17 +819,11 @@ cudaError_t launch(GemvParams P, int K, int rows_max, int nseg, int ctas, int ma
 {
     size_t smem = 0;
     if (!plan(P, STAGE, K, rows_max, ctas, max_ell, P.T, smem)) return cudaErrorInvalidValue;
-    static int configured = 0;
-    if (static_cast<int>(smem) > configured) {
-        cudaError_t e = cudaFuncSetAttribute(gemv_kernel<STAGE, SEG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             static_cast<int>(smem));
-        if (e != cudaSuccess) return e;
+    {
         // one carve-out for both stages: no L1/shared reconfiguration between
         // them, and a stage-2 CTA fits beside a stage-1 CTA
-        e = cudaFuncSetAttribute(gemv_kernel<STAGE, SEG>, cudaFuncAttributePreferredSharedMemoryCarveout,
-                                 cudaSharedmemCarveoutMaxShared);
+        cudaError_t e = allow_smem(reinterpret_cast<const void *>(gemv_kernel<STAGE, SEG>), static_cast<int>(smem), true);
         if (e != cudaSuccess) return e;
-        configured = static_cast<int>(smem);
     }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(ctas, nseg);
@@ -1405,114 +839,6 @@ cudaError_t launch(GemvParams P, int K, int rows_max, int nseg, int ctas, int ma
     cudaError_t e = cudaLaunchKernelEx(&cfg, gemv_kernel<STAGE, SEG>, P);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
-}
-
-// Single-launch plan: shared-memory offsets for both slices; false when the
-// call does not fit one pass, one register load round or shared memory.
-bool plan_fused(GemvParams &P, const dbf_layer &L, int G, size_t &smem)
-{
-    const int ncl = static_cast<int>(P.T) * L.ell;
-    if (P.T < 1 || ncl > kMaxNcl) return false;
-    const int pitch1 = static_cast<int>(pitch_words(L.M)), pitch2 = static_cast<int>(pitch_words(L.R));
-    if (2 * ((pitch1 + kGroupWords - 1) / kGroupWords * kGroupWords) > kFusedUnits * kThreads) return false;
-    const int nrb1 = (L.R + kRows - 1) / kRows, nrb2 = (L.N + kRows - 1) / kRows;
-    const int per1 = (nrb1 + G - 1) / G, per2 = (nrb2 + G - 1) / G;
-    if (per1 * kRows * L.ell > kScalesPerThread * kThreads || per2 * kRows * L.ell > kScalesPerThread * kThreads)
-        return false;
-    const int cb1 = col_bytes(pitch1), cb2 = col_bytes(pitch2);
-    int nb = per1 > per2 ? per1 : per2;   // every row block of a stage in one MMA pass
-    if (nb > 8) nb = 8;
-    const int nb_full = nb;
-    auto carve = [&](int rows1, int rows2, bool commit) -> size_t {
-        size_t off = align_up(static_cast<size_t>(rows1) * slice_stride(pitch1) * 4, 128);
-        const size_t o_s2 = off;
-        off = align_up(off + static_cast<size_t>(rows2) * slice_stride(pitch2) * 4, 128);
-        const size_t o_dig = off;
-        off += static_cast<size_t>(kPlanes * ncl + 1) * (cb1 > cb2 ? cb1 : cb2);
-        off = align_up(off, 16);
-        const size_t o_col = off;
-        off += static_cast<size_t>(kMaxNcl) * sizeof(ColInfo) + 16;
-        off = align_up(off, 16);
-        const size_t o_tiles = off;
-        off += static_cast<size_t>(nb) * kRows * kMaxBcols * 4;
-        off = align_up(off, 16);
-        const size_t o_bar = off;
-        off += 64;   // three mbarriers + wait flag
-        const size_t o_rs1 = off;
-        off += static_cast<size_t>(per1) * kRows * L.ell * 4;
-        off = align_up(off, 16);
-        const size_t o_rs2 = off;
-        off += static_cast<size_t>(per2) * kRows * L.ell * 4;
-        off = align_up(off, 16);
-        if (commit) {
-            P.off_s2 = static_cast<int>(o_s2);
-            P.off_digits = static_cast<int>(o_dig);
-            P.off_colinfo = static_cast<int>(o_col);
-            P.off_tiles = static_cast<int>(o_tiles);
-            P.off_bar = static_cast<int>(o_bar);
-            P.off_rscale = static_cast<int>(o_rs1);
-            P.off_rscale2 = static_cast<int>(o_rs2);
-            P.prefetch_rows = rows1;
-            P.slice_rows2 = rows2;
-            P.nb_max = nb;
-            P.ncl_pass = ncl;
-            P.pitch_max = pitch1;
-        }
-        return off;
-    };
-    // slices need whole 16-byte rows for the bulk copy
-    int rows1 = pitch1 % 4 == 0 ? per1 * kRows : 0;
-    int rows2 = pitch2 % 4 == 0 ? per2 * kRows : 0;
-    while (carve(rows1, rows2, false) > kSmemCap) {
-        if (rows2 > 0) rows2 = 0;
-        else if (rows1 > 0) rows1 = 0;
-        else return false;
-    }
-    // fewer row blocks per MMA pass when that lets two CTAs share an SM, so
-    // that the next call's CTAs can start their weight copies while this
-    // call finishes
-    while (nb > 2 && carve(rows1, rows2, false) > kCoResidentSmem) --nb;
-    if (carve(rows1, rows2, false) > kCoResidentSmem) nb = nb_full;
-    smem = carve(rows1, rows2, true);
-    return true;
-}
-
-template <bool XBF16, bool VEC>
-cudaError_t launch_fused(const GemvParams &P, int G, size_t smem, cudaStream_t s)
-{
-    static size_t configured = 0;
-    if (smem > configured) {
-        cudaError_t e = cudaFuncSetAttribute(gemv_fused_kernel<XBF16, VEC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             static_cast<int>(smem));
-        if (e != cudaSuccess) return e;
-        e = cudaFuncSetAttribute(gemv_fused_kernel<XBF16, VEC>, cudaFuncAttributePreferredSharedMemoryCarveout,
-                                 cudaSharedmemCarveoutMaxShared);
-        if (e != cudaSuccess) return e;
-        configured = smem;
-    }
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(G);
-    cfg.blockDim = dim3(kThreads);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = s;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, gemv_fused_kernel<XBF16, VEC>, P);
-    if (e != cudaSuccess) return e;
-    return cudaGetLastError();
-}
-
-// The single-launch plan for this layer and P.T, with its grid size.
-bool fused_plan_for(const dbf_layer &L, GemvParams &F, int &G, size_t &smem)
-{
-    const int nrb = ((L.R > L.N ? L.R : L.N) + kRows - 1) / kRows;
-    G = num_sms();
-    if (G > kMaxCtas) G = kMaxCtas;
-    if (G > nrb) G = nrb;
-    return plan_fused(F, L, G, smem);
 }
 
 struct WsLayout {
@@ -1535,7 +861,6 @@ void bind_workspace(GemvParams &P, int max_R, int max_ell, void *ws)
 {
     const WsLayout w = ws_layout(max_R, max_ell, P.T);
     char *body = static_cast<char *>(ws) + kWsHeaderBytes;
-    P.hdr = static_cast<unsigned *>(ws);
     P.img = body + w.img;
     P.qpart = reinterpret_cast<long long *>(body + w.qpart);
     P.sh2 = reinterpret_cast<int *>(body + w.sh2);
@@ -1569,18 +894,19 @@ cudaError_t run_both(GemvParams P, int M, int max_R, int N, int nseg, int budget
 
 size_t gemv_workspace_bytes(int64_t R, int64_t ell, int64_t T) { return kWsHeaderBytes + ws_layout(R, ell, T).total; }
 
-int gemv_launches(const dbf_layer &L, int64_t T)
+size_t gemv_layer_workspace_bytes(const dbf_layer &L, int64_t T)
 {
-    GemvParams F{};
-    F.T = T;
-    int G = 0;
-    size_t smem = 0;
-    return fused_plan_for(L, F, G, smem) ? 1 : 2;
+    const size_t a = gemv_workspace_bytes(L.R, L.ell, T), b = decode_workspace_bytes(L, T);
+    return a > b ? a : b;
 }
+
+int gemv_launches(const dbf_layer &L, int64_t T) { return decode_fits(L, T) ? 1 : 2; }
 
 cudaError_t gemv_forward(const dbf_layer &L, const void *x, dbf_dtype xd, void *y, dbf_dtype yd, int64_t T,
                          int flags, void *ws, cudaStream_t s)
 {
+    // one launch (binary tensor-core products, grid barrier) when the call fits it
+    if (decode_fits(L, T)) return decode_forward(L, x, xd, y, yd, T, flags, ws, s);
     GemvParams P{};
     P.layer = L;
     P.M = L.M;
@@ -1595,20 +921,6 @@ cudaError_t gemv_forward(const dbf_layer &L, const void *x, dbf_dtype xd, void *
     P.ell_cap = L.ell;
     P.R_cap = L.R;
     P.T = T;
-    // one launch when the call fits one pass
-    {
-        GemvParams F = P;
-        int G = 0;
-        size_t smem = 0;
-        if (fused_plan_for(L, F, G, smem)) {
-            bind_workspace(F, L.R, L.ell, ws);
-            F.stage1_ctas = G;
-            const bool vec = L.M % 8 == 0 && (reinterpret_cast<uintptr_t>(L.gamma) & 15u) == 0;
-            if (xd == DBF_BF16)
-                return vec ? launch_fused<true, true>(F, G, smem, s) : launch_fused<true, false>(F, G, smem, s);
-            return vec ? launch_fused<false, true>(F, G, smem, s) : launch_fused<false, false>(F, G, smem, s);
-        }
-    }
     return run_both<false>(P, L.M, L.R, L.N, 1, num_sms(), L.ell, ws, s);
 }
 

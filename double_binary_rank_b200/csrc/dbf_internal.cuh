@@ -16,9 +16,22 @@ constexpr int kMaxEll = 8;
 // single-launch decode kernel uses (its grid barrier counter); they must be
 // zero before the workspace's first use and every call leaves them valid.
 constexpr size_t kWsHeaderBytes = 256;
+// Header layout: bytes 0..7 the decode kernel's grid-barrier word (arrival
+// count in the low 32 bits, epoch in the high 32 bits; zero at first use),
+// bytes 8..11 a sticky int32 status that kernels whose bounded wait expired
+// set to DBF_ERR_TIMEOUT (never cleared by the library).
+constexpr size_t kWsStatusOffset = 8;
 
 // ---- packed layout helpers (see "Packed sign layout" in dbf.h) -----------
 __host__ __device__ inline int64_t pitch_words(int64_t k) { return (k + 31) / 32; }
+
+// ---- per-device launch state (dbf_device.cu) -------------------------------
+// SM count of the current device (148 if it cannot be read).
+int device_sms();
+// Allow 'kernel' at least 'bytes' of dynamic shared memory on the current
+// device (cudaFuncSetAttribute once per device and size; optionally the
+// largest shared-memory carve-out too).
+cudaError_t allow_smem(const void *kernel, int bytes, bool max_shared_carveout = false);
 
 // ---- launchers (each returns the first CUDA error it meets) --------------
 cudaError_t launch_pack(const void *src, dbf_dtype dt, int64_t rows, int64_t k, uint32_t *dst,
@@ -33,8 +46,18 @@ cudaError_t launch_transpose(const uint32_t *src, int64_t rows, int64_t k, uint3
 cudaError_t launch_ste(const float *db, const void *h, dbf_dtype hd, int64_t n, float tau, float *dh,
                        int accumulate, cudaStream_t s);
 
+// single-launch decode (binary tensor-core products, dbf_decode.cu): calls with
+// T * ell <= 8 and M, R <= 8192
+bool decode_fits(const dbf_layer &L, int64_t T);
+size_t decode_workspace_bytes(const dbf_layer &L, int64_t T);
+cudaError_t decode_forward(const dbf_layer &L, const void *x, dbf_dtype xd, void *y, dbf_dtype yd, int64_t T,
+                           int flags, void *ws, cudaStream_t s);
+// limit of the decode kernel's bounded waits for later calls (0: the default, 2 s)
+void set_decode_wait_ns(unsigned long long ns);
+
 // decode path
-size_t gemv_workspace_bytes(int64_t R, int64_t ell, int64_t T);
+size_t gemv_workspace_bytes(int64_t R, int64_t ell, int64_t T);   // two-launch and segmented kernels
+size_t gemv_layer_workspace_bytes(const dbf_layer &L, int64_t T);  // dbf_forward on the GEMV path
 int gemv_launches(const dbf_layer &L, int64_t T);   // 1 (single launch) or 2
 cudaError_t gemv_forward(const dbf_layer &L, const void *x, dbf_dtype xd, void *y, dbf_dtype yd,
                          int64_t T, int flags, void *ws, cudaStream_t s);

@@ -78,7 +78,7 @@ dbf_status dbf_forward_decode_noalloc(const dbf_layer *L, const void *x, dbf_dty
     if (!x || !y) return DBF_ERR_INVALID_ARG;
     if (!is_aligned(x, 16) || !is_aligned(y, 16)) return DBF_ERR_ALIGNMENT;
     // the fixed scratch must hold this call's decode workspace
-    if (gemv_workspace_bytes(L->R, L->ell, T) > kNoallocScratchBytes) return DBF_ERR_WORKSPACE;
+    if (gemv_layer_workspace_bytes(*L, T) > kNoallocScratchBytes) return DBF_ERR_WORKSPACE;
     void *scratch = nullptr;
     if (scratch_address(&scratch) != cudaSuccess) return DBF_ERR_CUDA;
     return gemv_forward(*L, x, x_dtype, y, y_dtype, T, flags, scratch, static_cast<cudaStream_t>(stream)) ==

@@ -483,12 +483,9 @@ cudaError_t launch_tf32x3(int64_t M, int64_t N, int64_t K, float alpha, const fl
     g.sumsq = sumsq;
     g.vec_c = (sumsq || (aligned16(Cout) && ldco % 4 == 0)) && (beta == 0.f || (aligned16(Cin) && ldci % 4 == 0));
     g.status = status;
-    static bool configured = false;
-    if (!configured) {
-        cudaError_t e = cudaFuncSetAttribute(tf32x3_kernel<Cfg>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             static_cast<int>(x_smem<Cfg>()));
+    {
+        cudaError_t e = allow_smem(reinterpret_cast<const void *>(tf32x3_kernel<Cfg>), static_cast<int>(x_smem<Cfg>()));
         if (e != cudaSuccess) return e;
-        configured = true;
     }
     const int64_t tiles = ((M + XM - 1) / XM) * ((N + Cfg::BN - 1) / Cfg::BN);
     if (tiles >= (int64_t(1) << 31)) return cudaErrorInvalidValue;

@@ -20,9 +20,26 @@
  * Conventions shared by every entry point
  * ---------------------------------------
  * - Every data pointer is a DEVICE pointer owned by the caller. The library
- *   allocates nothing, keeps no state between calls, never synchronises the
- *   device and enqueues all work on 'stream' (a cudaStream_t; NULL = the
- *   legacy default stream).
+ *   allocates nothing, never synchronises the device and enqueues all work on
+ *   'stream' (a cudaStream_t; NULL = the legacy default stream). The only
+ *   device state that outlives a call is the workspace header described
+ *   below, in memory the caller owns; host-side, the library caches per
+ *   device the SM count and the kernel attributes it has set.
+ * - Workspace header: every workspace (dbf_forward, dbf_backward,
+ *   dbf_forward_segmented, dbf_forward_segmented_planned, dbf_mbok_forward)
+ *   starts with DBF_WS_HEADER_BYTES bytes that must be zero before its first
+ *   use (cudaMemsetAsync once after allocating it); the rest is scratch.
+ *     bytes 0..7   the grid-barrier word of the single-launch decode kernel
+ *                  (arrival count and epoch); every call leaves it valid for
+ *                  the next, also when a wait timed out.
+ *     bytes 8..11  int32 device status of the calls made on the workspace:
+ *                  a kernel whose bounded wait expired (a grid barrier or a
+ *                  pipeline stage not reached within its time limit) stores
+ *                  DBF_ERR_TIMEOUT there, and the output of that call is
+ *                  incomplete. The library never clears it: read it (and
+ *                  zero it if wanted) by a copy once the calls are done.
+ *   Calls that share a workspace must be ordered on the GPU (one stream, or
+ *   events).
  * - Arguments are checked on the host before any launch; a failed check
  *   returns an error status and launches nothing. Data-dependent faults
  *   found by a kernel (NaN latents, bad segment tables) are reported through
@@ -60,6 +77,9 @@ typedef enum {
 } dbf_status;
 
 typedef enum { DBF_F32 = 0, DBF_BF16 = 1, DBF_F16 = 2, DBF_I8 = 3 } dbf_dtype;
+
+#define DBF_WS_HEADER_BYTES 256
+#define DBF_WS_STATUS_OFFSET 8
 
 /* Flags of dbf_forward / dbf_forward_segmented (bitwise or).
  * DBF_ACCUMULATE: y += branch instead of y = branch.
@@ -222,18 +242,16 @@ int32_t dbf_forward_launches(const dbf_layer *L, int64_t T, dbf_path path);
  *    dtype.
  * flags: DBF_ACCUMULATE | DBF_WEIGHTS_STATIC (see above); other bits must be 0.
  * ws: device workspace of at least dbf_workspace_bytes(L, T, path) bytes,
- *    256-byte aligned. Its first 256 bytes are a header (the grid-barrier
- *    counter of the single-launch decode kernel, which runs when T * ell <= 8):
- *    they must be zero before the workspace is first used (cudaMemsetAsync
- *    once after allocating it) and every call leaves them valid for the next;
- *    the rest is scratch. Calls that share a workspace must be ordered on the
- *    GPU (one stream, or events).
- * T == 0 is a no-op. Numerics: the GEMV path turns each activation column
- * (gamma.x, then beta.h) into 22-bit fixed point with one power-of-two scale
- * per column and accumulates sign sums exactly in integers (relative error
- * about 2^-22 of the column's largest value per element); the GEMM path
- * rounds gamma.x and beta.h to fp16 operands (|values| below 65504) and
- * accumulates in fp32.
+ *    256-byte aligned, starting with the header described above (zero before
+ *    first use; its status word reports device-side timeouts).
+ * T == 0 is a no-op. Paths: the GEMV path runs one kernel when T * ell <= 8
+ * and M, R <= 8192 (binary tensor-core products with a grid barrier, one CTA
+ * per SM, launched cooperatively), else two. Numerics: the GEMV path turns
+ * each activation column (gamma.x, then beta.h) into 22-bit fixed point with
+ * one power-of-two scale per column and accumulates sign sums exactly in
+ * integers (relative error about 2^-22 of the column's largest value per
+ * element); the GEMM path rounds gamma.x and beta.h to fp16 operands
+ * (|values| below 65504) and accumulates in fp32.
  * Errors: DBF_ERR_INVALID_ARG, DBF_ERR_ALIGNMENT, DBF_ERR_WORKSPACE,
  *    DBF_ERR_UNSUPPORTED (path GEMM on a shape it does not serve), DBF_ERR_CUDA. */
 dbf_status dbf_forward(const dbf_layer *L, const void *x, dbf_dtype x_dtype, void *y,
@@ -386,6 +404,17 @@ dbf_status dbf_forward_segmented(const dbf_layer *adapters_dev, int32_t num_adap
  * DBF_ERR_CUDA if the address lookup fails. */
 dbf_status dbf_forward_decode_noalloc(const dbf_layer *L, const void *x, dbf_dtype x_dtype, void *y,
                                       dbf_dtype y_dtype, int64_t T, int flags, void *stream);
+
+/* Time limit of the grid-barrier wait of the single-launch decode kernel
+ * for the calls made after this one, in this process: ns > 0 sets it, 0
+ * restores the default of 2 s (its waits for its own weight copies always
+ * keep the default). For tests of the timeout path: with a limit shorter than
+ * the time the CTAs take to arrive, the waiting CTAs give up, store
+ * DBF_ERR_TIMEOUT in the workspace status word and skip their share of stage
+ * 2 (y is left incomplete); the workspace stays usable, and a later call with
+ * the default limit is correct. Not for production use; not synchronised with
+ * calls in flight on other host threads. */
+void dbf_debug_set_decode_wait_ns(uint64_t ns);
 
 /* Static description of a status code. */
 const char *dbf_status_string(dbf_status s);

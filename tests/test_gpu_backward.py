@@ -130,6 +130,22 @@ def test_dbf_mlp_full_size(dbf):
         assert abs(v - loss) <= TOL * scale, (v, loss)
 
 
+def test_dbf_mlp_shape_elementwise(dbf):
+    # The DBF MLP layer's full shape (4096 -> 11008, R = 5888) at 64 tokens:
+    # every element of dx, dalpha, dbeta and dgamma against the oracle.
+    w = S.WORKLOADS["dbf_mlp"]
+    L = S.workload_layers(w)[0]
+    T = 64
+    x = S.make_x(w.seed + 300, T, w.M, "bf16")
+    dy = S.make_x(w.seed + 400, T, w.N, "bf16")
+    _, g = gpu_grads(dbf, L, x, dy)
+    ref = oracle.backward(L, x, dy)
+    assert rel_err(g.dx.cpu().numpy(), ref.dx) < TOL
+    assert rel_err(g.dalpha.cpu().numpy(), ref.dalpha) < TOL
+    assert rel_err(g.dbeta.cpu().numpy(), ref.dbeta) < TOL
+    assert rel_err(g.dgamma.cpu().numpy(), ref.dgamma) < TOL
+
+
 @pytest.mark.parametrize("case", [(256, 384, 128, 1, 37), (128, 256, 256, 2, 300), (384, 128, 128, 3, 5)],
                          ids=lambda c: "M{}N{}R{}l{}T{}".format(*c))
 def test_sign_matrix_gradients(dbf, case):

@@ -1,11 +1,14 @@
-"""The single-launch decode path (T * ell <= 8) against the fp64 oracle.
+"""The single-launch decode path (T * ell <= 8, M and R <= 8192) against
+the fp64 oracle.
 
 That path exchanges the rank-R intermediate through a grid-wide barrier
-whose counter lives in the workspace header, so besides plain parity these
-tests check that many calls sharing one workspace (with different grid
-sizes) stay correct, that the header is left consistent (arrival count ==
-starting count) after every call, and the size limits where the library
-switches to the two-launch path.
+whose word lives in the workspace header (arrival count in the low 32 bits,
+epoch in the high 32 bits), so besides plain parity these tests check that
+many calls sharing one workspace (with different grid sizes) stay correct,
+that every call leaves the arrival count at zero and advances the epoch by
+one, that a barrier wait that runs out of time is reported in the header's
+status word and leaves the workspace usable, and the size limits where the
+library switches to the two-launch path.
 """
 import numpy as np
 import pytest
@@ -25,7 +28,9 @@ def dbf():
 
 
 def header_words(ws):
-    return ws[:8].view(torch.int32).cpu().tolist()
+    """(arrival count, epoch) of the header's barrier word."""
+    lo, hi = ws[:8].view(torch.int32).cpu().tolist()
+    return lo & 0xFFFFFFFF, hi & 0xFFFFFFFF
 
 
 @pytest.mark.parametrize("T,ell", [(8, 1), (4, 2), (1, 8), (2, 3), (9, 1), (3, 3)])
@@ -41,7 +46,7 @@ def test_column_limit(dbf, T, ell):
 
 @pytest.mark.parametrize("M", [8192, 8224])
 def test_input_width_limit(dbf, M):
-    # one register round holds up to 8192 inputs; wider inputs take two launches
+    # the single launch takes up to 8192 inputs; wider inputs take two launches
     rng = np.random.default_rng(710 + M)
     L = random_layer(rng, M, 256, 96, 1)
     x = S.to_bf16_bits(rng.standard_normal((1, M)))
@@ -83,24 +88,51 @@ def test_shared_workspace_many_layers(dbf):
     torch.cuda.synchronize()
     for i, y in outs:
         assert rel_err(host_y(y), refs[i]) < 1e-4
-    a, b = header_words(ws)
-    assert a == b and a != 0
+    assert header_words(ws) == (0, 40)
+    assert dbf.workspace_status(ws) == dbf.OK
 
 
-def test_consistent_nonzero_header(dbf):
-    # only equality of the two header words matters, not their value
+def test_epoch_wraps(dbf):
+    # only a change of the epoch matters, not its value: it wraps past 2^32
     rng = np.random.default_rng(740)
     L = random_layer(rng, 640, 320, 96, 1)
     dl = dev_layer(L)
     x = S.to_bf16_bits(rng.standard_normal((2, 640)))
     ref = oracle.forward(L, x)
     ws = dbf.alloc_workspace(dbf.workspace_bytes(dl, 2), "cuda")
-    ws[:8].view(torch.int32).fill_(0x7FFFFFF0)   # wraps past 2^32 during the calls
+    ws[4:8].view(torch.int32).fill_(-2)   # epoch 0xFFFFFFFE
     for _ in range(3):
         got = host_y(dbf.forward(dl, dev_x(x), ws=ws, y_dtype=torch.float32))
         assert rel_err(got, ref) < 1e-4
-    a, b = header_words(ws)
-    assert a == b
+    assert header_words(ws) == (0, 1)
+
+
+def test_barrier_timeout_reported_and_workspace_recovers(dbf):
+    # A grid-barrier time limit of 1 ns: every CTA but the last to arrive gives
+    # up at once, stores DBF_ERR_TIMEOUT in the workspace status word and skips
+    # its stage-2 rows (the waits end; nothing faults or hangs). The barrier
+    # word is left consistent, and the next call, with the default limit, is
+    # correct.
+    w = S.WORKLOADS["dbf_mlp"]
+    L = S.workload_layers(w)[0]
+    dl = dev_layer(L)
+    xh = S.make_x(w.seed, 1, w.M, "bf16")
+    x = dev_x(xh)
+    ws = dbf.alloc_workspace(dbf.workspace_bytes(dl, 1), "cuda")
+    try:
+        dbf.debug_set_decode_wait_ns(1)
+        dbf.forward(dl, x, ws=ws, y_dtype=torch.float32)
+        torch.cuda.synchronize()
+    finally:
+        dbf.debug_set_decode_wait_ns(0)
+    assert dbf.workspace_status(ws) == dbf.ERR_TIMEOUT
+    assert header_words(ws) == (0, 1)
+    dbf.clear_workspace_status(ws)
+    y = dbf.forward(dl, x, ws=ws, y_dtype=torch.float32)
+    torch.cuda.synchronize()
+    assert dbf.workspace_status(ws) == dbf.OK
+    assert header_words(ws) == (0, 2)
+    assert rel_err(host_y(y), oracle.forward(L, xh)) < 1e-4
 
 
 def test_dbf_mlp_decode_repeat_bit_identical(dbf):

@@ -76,13 +76,24 @@ def test_gemm_matches_gemv(dbf):
     assert rel_err(a, b) < TOL
 
 
+def check_rows_cover_tiles(rows, T, tile=256):
+    """The sampled rows include the first and the last token and at least one
+    row of every 256-token tile of the GEMM, so that every tile the
+    persistent schedule hands out (including those past the first wave of
+    148) is checked."""
+    assert rows[0] == 0 and rows[-1] == T - 1
+    assert set(range((T + tile - 1) // tile)) <= set(int(r) // tile for r in rows)
+
+
 def test_dbf_mlp_prefill_sampled_rows(dbf):
-    # the DBF MLP layer at 2048 tokens, checked on a fixed sample of token rows
+    # the DBF MLP layer at 2048 tokens, checked on a fixed sample of 128 token rows
     w = S.WORKLOADS["dbf_mlp"]
     L = S.workload_layers(w)[0]
     T = 2048
     x = S.make_x(w.seed, T, w.M, "bf16")
-    rows = S.sample_rows(w.seed, T, 64)
+    rows = S.sample_rows_per_tile(w.seed, T, 128, 256)
+    assert len(rows) == 128
+    check_rows_cover_tiles(rows, T)
     ref = oracle.forward(L, x, rows=rows)
     got = run(dbf, L, x, y_dtype=torch.float32)[rows]
     assert rel_err(got, ref) < TOL
@@ -97,7 +108,54 @@ def test_large_prefill_sampled_rows(dbf):
     L = S.workload_layers(w)[0]
     T = 8192
     x = S.make_x(w.seed, T, w.M, "bf16")
-    rows = S.sample_rows(w.seed, T, 32)
+    rows = S.sample_rows_per_tile(w.seed, T, 128, 256)
+    assert len(rows) == 128
+    check_rows_cover_tiles(rows, T)
     ref = oracle.forward(L, x, rows=rows)
     got = run(dbf, L, x, y_dtype=torch.float32)[rows]
+    assert rel_err(got, ref) < TOL
+
+
+# Shape whose two GEMM stages each have 256 tiles (32 row tiles x 8 token
+# tiles), so the persistent kernel's CTAs wrap past the first 148 tiles.
+WRAP = dict(M=1024, N=4096, R=4096, T=2048)
+
+
+def test_gemm_matched_sign_flip_bit_identical(dbf):
+    # Negating column r of B1 and row r of B2 negates h_r and v_r exactly
+    # (round to nearest even is symmetric) and leaves every product of stage
+    # 2 unchanged, so with a fixed accumulation order y is bit-identical.
+    rng = np.random.default_rng(60)
+    L = random_layer(rng, WRAP["M"], WRAP["N"], WRAP["R"], 1)
+    x = S.to_bf16_bits(rng.standard_normal((WRAP["T"], WRAP["M"])))
+    y0 = run(dbf, L, x)
+    flip = rng.random(WRAP["R"]) < 0.5
+    L.b1[:, flip] *= -1
+    L.b2[flip, :] *= -1
+    y1 = run(dbf, L, x)
+    assert np.array_equal(y0, y1)
+
+
+def test_gemm_power_of_two_alpha_bit_exact(dbf):
+    # alpha -> 2 alpha doubles the fp16 A operand exactly, and scaling by two
+    # commutes with every fp32 rounding: y -> exactly 2 y.
+    rng = np.random.default_rng(61)
+    L = random_layer(rng, WRAP["M"], WRAP["N"], WRAP["R"], 1)
+    x = S.to_bf16_bits(rng.standard_normal((WRAP["T"], WRAP["M"])))
+    y0 = run(dbf, L, x)
+    L.alpha[:] = S.to_f16_bits(2.0 * L.alpha.view(np.float16).astype(np.float64))
+    y1 = run(dbf, L, x)
+    assert np.array_equal(y1, 2.0 * y0)
+
+
+def test_gemm_wrapping_shape_sampled_rows(dbf):
+    # the same shape against the oracle on rows of every token tile
+    rng = np.random.default_rng(62)
+    L = random_layer(rng, WRAP["M"], WRAP["N"], WRAP["R"], 1)
+    T = WRAP["T"]
+    x = S.to_bf16_bits(rng.standard_normal((T, WRAP["M"])))
+    rows = S.sample_rows_per_tile(62, T, 64, 256)
+    check_rows_cover_tiles(rows, T)
+    ref = oracle.forward(L, x, rows=rows)
+    got = run(dbf, L, x)[rows]
     assert rel_err(got, ref) < TOL

@@ -1,5 +1,6 @@
 """The seeded input generator: determinism, distributions, rounding, routing."""
 import numpy as np
+import pytest
 
 import dbf_synth as S
 
@@ -67,6 +68,16 @@ def test_segments_sorted_and_cover():
 def test_sample_rows_holds_ends():
     r = S.sample_rows(3, 2048, 128)
     assert r.size == 128 and r[0] == 0 and r[-1] == 2047 and np.all(np.diff(r) > 0)
+
+
+@pytest.mark.parametrize("T,n", [(2048, 128), (8192, 128), (2048, 64), (300, 2)])
+def test_sample_rows_per_tile_covers_every_tile(T, n):
+    r = S.sample_rows_per_tile(5, T, n, 256)
+    assert r.size == n and r[0] == 0 and r[-1] == T - 1 and np.all(np.diff(r) > 0)
+    tiles = (T + 255) // 256
+    counts = np.bincount(r // 256, minlength=tiles)
+    assert counts.min() >= n // tiles
+    assert np.array_equal(r, S.sample_rows_per_tile(5, T, n, 256))
 
 
 def test_weight_and_factor_start_recipes():

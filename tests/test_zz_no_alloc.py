@@ -2,9 +2,10 @@
 allocate device memory (a runtime that owns every allocation, or a thread
 that must not call cudaMalloc). It takes its scratch from a fixed device
 array in the library instead of a caller workspace. Its output must match
-dbf_forward's on two calls in a row (the array is shared between calls and
-keeps the previous call's contents). Collected last on purpose: if it fails,
-a run that stops at the first failure has already run every other test."""
+dbf_forward's, and the oracle's, on calls in a row (the array is shared
+between calls and keeps the previous call's contents). Collected last on
+purpose: if it fails, a run that stops at the first failure has already run
+every other test."""
 import ctypes
 
 import numpy as np
@@ -26,28 +27,36 @@ def _call_noalloc(dbf, layer, x, y):
 
 def test_noalloc_matches_forward_twice():
     import double_binary_rank_b200 as dbf
+    import oracle
     rng = np.random.default_rng(81)
     w = S.WORKLOADS["dbf_mlp"]
     L = S.workload_layers(w)[0]
     dl = dev_layer(L)
-    for call in range(2):
-        T = 1 + call
-        x = dev_x(S.make_x(w.seed + call, T, w.M, "bf16"))
+    # T = 1, 2: single-launch kernel; T = 16: the two-launch path through the
+    # same array; then single launches again, which also shows that the
+    # array's barrier word was left consistent by the earlier calls
+    for call, T in enumerate((1, 2, 16, 1, 2)):
+        xh = S.make_x(w.seed + call, T, w.M, "bf16")
+        x = dev_x(xh)
         ref = dbf.forward(dl, x, path="gemv", y_dtype=torch.float32)
         y = torch.full((T, w.N), float("nan"), device="cuda")
         st = _call_noalloc(dbf, dl, x, y)
         torch.cuda.synchronize()
         assert st == dbf.OK, dbf.status_string(st)
-        assert rel_err(host_y(y), host_y(ref)) < TOL
+        got = host_y(y)
+        assert rel_err(got, host_y(ref)) < TOL
+        assert rel_err(got, oracle.forward(L, xh)) < TOL
     # a second layer shape right after, through the same array
     L2 = random_layer(rng, 300, 170, 96, 2)
     d2 = dev_layer(L2)
-    x2 = dev_x(S.to_bf16_bits(rng.standard_normal((3, 300))))
+    x2h = S.to_bf16_bits(rng.standard_normal((3, 300)))
+    x2 = dev_x(x2h)
     ref2 = dbf.forward(d2, x2, path="gemv", y_dtype=torch.float32)
     y2 = torch.zeros((3, 170), device="cuda")
     assert _call_noalloc(dbf, d2, x2, y2) == dbf.OK
     torch.cuda.synchronize()
     assert rel_err(host_y(y2), host_y(ref2)) < TOL
+    assert rel_err(host_y(y2), oracle.forward(L2, x2h)) < TOL
 
 
 def test_noalloc_rejects_calls_beyond_its_scratch():
