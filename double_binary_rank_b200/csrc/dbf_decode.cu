@@ -42,10 +42,10 @@
 // in the high word). A CTA reads the epoch, then adds its arrival with an
 // acquire-release atomic; the arrival that brings the count to the grid size
 // stores (epoch + 1, count 0) with release semantics, and every other CTA
-// waits (acquire loads, bounded by a time limit) for the epoch to change. The
-// epoch can change only after every CTA has arrived, so a CTA that starts
-// late still reads the current epoch; the count is zero again once the last
-// CTA has arrived, whatever happened to the waits. A wait that runs out of
+// waits (acquire loads, bounded by a time limit) until it sees the full count
+// or the new epoch. The epoch can change only after every CTA has arrived, so
+// a CTA that starts late still reads the current epoch; the count is zero
+// again once the last CTA has arrived, whatever happened to the waits. A wait that runs out of
 // time stores DBF_ERR_TIMEOUT in the header's status word and the CTA skips
 // its stage-2 rows.
 #include "dbf_internal.cuh"
@@ -62,6 +62,7 @@ constexpr int kMaxCols = 8;              // (token, envelope) columns of one cal
 constexpr int kGroupWords = 8;           // packed words per MMA unit (256 columns of K)
 constexpr int kMaxWordsPerWarp = 32;     // M <= 8192
 constexpr int kSmemCap = 227 * 1024;
+constexpr int kMaxGrid = 160;            // CTAs at most (sizes the per-CTA sums in the workspace)
 constexpr unsigned long long kDefaultWaitNs = 2000000000ull;   // 2 s
 
 unsigned long long g_wait_ns = 0;   // 0: the default limit
@@ -84,13 +85,16 @@ struct DecodeParams {
     int ng1, ng2;                 // 256-column groups of K in stage 1, stage 2
     int max_rb1, max_rb2;         // row blocks of the largest CTA
     int bulk1, bulk2;             // slices copied by bulk asynchronous copies
+    int bulk_g, bulk_x;           // gamma and x staged by bulk copies (else element by element)
+    int gs_bytes, xs_bytes;       // staged gamma, and one token's x buffer (16-byte rounded)
+    int gpitch;                   // values per staged gamma row (M rounded up to 8)
     int tile_ld;                  // int32 per row of the partial-sum tile (8 per column group)
     int off_s2, off_dig, off_tile, off_misc, off_rs1, off_rs2;   // shared-memory offsets
     unsigned long long wait_ns;   // limit of the grid-barrier wait
 };
 
 struct Misc {
-    uint64_t bar[2];              // slice 1, slice 2 arrived
+    uint64_t bar[5];              // slice 1, slice 2, gamma, x buffers 0 and 1 arrived
     int flag;
     unsigned e0;                  // epoch read at entry
     unsigned bmax;                // max |beta| (fp32 bits)
@@ -167,6 +171,46 @@ __device__ __forceinline__ bool slice_wait(uint64_t *bar, const DecodeParams &P,
     return ms->flag != 0;
 }
 
+// Wait until token t's x (buffer t & 1, its (t / 2)-th copy) and, for the
+// first token, gamma are in shared memory: bulk copies are waited for by
+// thread 0 (bounded by the default limit), element copies by the barrier.
+__device__ __forceinline__ void token_wait(const DecodeParams &P, Misc *ms, int t)
+{
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        const unsigned long long t0 = global_ns();
+        const uint32_t par = static_cast<uint32_t>(t >> 1) & 1u;
+        while ((t == 0 && P.bulk_g && !bar_try(&ms->bar[2], 0)) || (P.bulk_x && !bar_try(&ms->bar[3 + (t & 1)], par))) {
+            if (global_ns() - t0 > kDefaultWaitNs) {
+                atomicExch(P.status, static_cast<int32_t>(DBF_ERR_TIMEOUT));
+                break;
+            }
+        }
+    }
+    __syncthreads();
+}
+
+// gamma_env[col] x_t[col] and the same at col + 1 (col even) from the
+// staged copies, exact in fp32; zero at and past m
+__device__ __forceinline__ float2 stage_u2(const uint16_t *gc, const unsigned char *xs, dbf_dtype xd, int col, int m)
+{
+    float2 x, g;
+    if (col + 1 < m) {
+        const __half2 gh = *reinterpret_cast<const __half2 *>(gc + col);
+        g = __half22float2(gh);
+        x = xd == DBF_BF16 ? __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(xs + 2 * col))
+                           : *reinterpret_cast<const float2 *>(xs + 4 * col);
+    } else if (col < m) {
+        g = make_float2(__half2float(__ushort_as_half(gc[col])), 0.f);
+        x = make_float2(xd == DBF_BF16 ? __bfloat162float(reinterpret_cast<const __nv_bfloat16 *>(xs)[col])
+                                       : reinterpret_cast<const float *>(xs)[col],
+                        0.f);
+    } else {
+        return make_float2(0.f, 0.f);
+    }
+    return make_float2(g.x * x.x, g.y * x.y);
+}
+
 __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
@@ -223,12 +267,6 @@ __device__ __forceinline__ int quantize(float u, int sh)
 __device__ __forceinline__ uint32_t digit_bytes(int q) { return static_cast<uint32_t>(q + 0x808080) ^ 0x808080u; }
 
 __device__ __forceinline__ float ldg_h(const uint16_t *p) { return __half2float(__ushort_as_half(__ldg(p))); }
-
-__device__ __forceinline__ float load_x(const void *x, dbf_dtype xd, int64_t i)
-{
-    if (xd == DBF_BF16) return __bfloat162float(static_cast<const __nv_bfloat16 *>(x)[i]);
-    return static_cast<const float *>(x)[i];
-}
 
 __device__ __forceinline__ long long warp_sum64(long long v)
 {
@@ -296,11 +334,13 @@ __device__ bool grid_sync(const DecodeParams &P, Misc *ms)
             const unsigned long long next = static_cast<unsigned long long>(ms->e0 + 1u) << 32;
             asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(P.sync), "l"(next) : "memory");
         } else {
+            // every CTA has arrived once the count reaches the grid size (seen
+            // before the last arrival resets it) or the epoch has moved on
             const unsigned long long t0 = global_ns();
             while (true) {
                 unsigned long long v;
                 asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(P.sync) : "memory");
-                if (static_cast<unsigned>(v >> 32) != ms->e0) break;
+                if (static_cast<unsigned>(v >> 32) != ms->e0 || static_cast<unsigned>(v) >= gridDim.x) break;
                 if (global_ns() - t0 > P.wait_ns) {
                     ok = false;
                     atomicExch(P.status, static_cast<int32_t>(DBF_ERR_TIMEOUT));
@@ -308,7 +348,6 @@ __device__ bool grid_sync(const DecodeParams &P, Misc *ms)
                 }
             }
         }
-        __threadfence();
         ms->flag = ok ? 1 : 0;
     }
     __syncthreads();
@@ -377,6 +416,11 @@ __device__ __forceinline__ long long digit_sum(const int *tr, int c)
 }
 
 // ---- the kernel -----------------------------------------------------------------
+// Every phase that runs once per call is a rolled loop: the kernel runs once
+// per CTA per call, so its instructions are fetched cold each time, and the
+// length of the code it executes, not its arithmetic, sets the time of those
+// phases. Inputs of the digit build (x and gamma) are staged in shared memory
+// by bulk copies, so those loops do not wait on global loads.
 __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const __grid_constant__ DecodeParams P)
 {
     extern __shared__ __align__(128) unsigned char smem[];
@@ -401,119 +445,212 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const __grid_consta
 
     uint32_t *s1 = reinterpret_cast<uint32_t *>(smem);
     uint32_t *s2 = reinterpret_cast<uint32_t *>(smem + P.off_s2);
+    // x and gamma are staged where the B1 slice goes; that slice is copied
+    // once the digits of gamma . x are built
+    const uint16_t *gs = reinterpret_cast<const uint16_t *>(smem + P.off_s2);
     char *dig = reinterpret_cast<char *>(smem + P.off_dig);
     int *tile = reinterpret_cast<int *>(smem + P.off_tile);
     Misc *ms = reinterpret_cast<Misc *>(smem + P.off_misc);
     float *rs1 = reinterpret_cast<float *>(smem + P.off_rs1);   // beta_i of the CTA's stage-1 rows
     float *rs2 = reinterpret_cast<float *>(smem + P.off_rs2);   // alpha_i of its stage-2 rows
 
+    if (tid < kMaxCols) {
+        ms->amax[tid] = 0u;
+        ms->qsum_u[tid] = 0;
+        ms->qabs_u[tid] = 0;
+        ms->qsum_v[tid] = 0;
+        ms->qpart_v[tid] = 0;
+    }
     if (tid == 0) {
-        bar_init(&ms->bar[0], 1);
-        bar_init(&ms->bar[1], 1);
+        for (int i = 0; i < 5; ++i) bar_init(&ms->bar[i], 1);
         ms->bmax = 0u;
-#pragma unroll
-        for (int c = 0; c < kMaxCols; ++c) {
-            ms->amax[c] = 0u;
-            ms->qsum_u[c] = 0;
-            ms->qabs_u[c] = 0;
-            ms->qsum_v[c] = 0;
-            ms->qpart_v[c] = 0;
-        }
     }
     __syncthreads();
-    // ---- both sign slices -> shared memory, in flight from here on
-    if (warp == 0) {
-        if (lane == 0) {
-            if (P.bulk1 && n1 > 0) bar_expect_tx(&ms->bar[0], static_cast<uint32_t>(n1) * P.pitch1 * 4u);
-            if (P.bulk2 && n2 > 0) bar_expect_tx(&ms->bar[1], static_cast<uint32_t>(n2) * P.pitch2 * 4u);
+    // ---- the B2 slice and gamma -> shared memory, in flight from here on
+    if (tid == 0) {
+        if (P.bulk1 && n1 > 0) bar_expect_tx(&ms->bar[0], static_cast<uint32_t>(n1) * P.pitch1 * 4u);
+        if (P.bulk_g) {
+            bar_expect_tx(&ms->bar[2], static_cast<uint32_t>(P.gs_bytes));
+            bulk_g2s(smem + P.off_s2, L.gamma, static_cast<uint32_t>(P.gs_bytes), &ms->bar[2]);
         }
+    }
+    if (warp == 0) {
         __syncwarp();
         if (P.bulk1) slice_bulk(s1, L.b2_packed + static_cast<int64_t>(lo1) * P.pitch1, n1, P.pitch1, P.stride1, &ms->bar[0]);
-        if (P.bulk2) slice_bulk(s2, L.b1_packed + static_cast<int64_t>(lo2) * P.pitch2, n2, P.pitch2, P.stride2, &ms->bar[1]);
     }
     slice_pad(s1, n1, rows1, P.pitch1, P.stride1);
-    slice_pad(s2, n2, rows2, P.pitch2, P.stride2);
     if (!P.bulk1) slice_plain(s1, L.b2_packed + static_cast<int64_t>(lo1) * P.pitch1, n1, P.pitch1, P.stride1);
-    if (!P.bulk2) slice_plain(s2, L.b1_packed + static_cast<int64_t>(lo2) * P.pitch2, n2, P.pitch2, P.stride2);
-    // ---- weight-side scales: the CTA's beta and alpha rows, max |beta|
-    for (int i = tid; i < rows1 * ell; i += kThreads) {
-        const int e = i / rows1, r = i - e * rows1;
-        rs1[i] = r < n1 ? ldg_h(L.beta + static_cast<int64_t>(e) * L.R + lo1 + r) : 0.f;
+    if (!P.bulk_g) {
+        // element by element, rows padded to a multiple of 8 values
+        uint16_t *g = reinterpret_cast<uint16_t *>(smem + P.off_s2);
+#pragma unroll 1
+        for (int i = tid; i < ell * L.M; i += kThreads) {
+            const int e = i / L.M;
+            g[e * P.gpitch + (i - e * L.M)] = __ldg(L.gamma + i);
+        }
     }
-    for (int i = tid; i < rows2 * ell; i += kThreads) {
-        const int e = i / rows2, r = i - e * rows2;
-        rs2[i] = r < n2 ? ldg_h(L.alpha + static_cast<int64_t>(e) * L.N + lo2 + r) : 0.f;
-    }
+    // ---- weight-side scales: the CTA's beta and alpha rows, max |beta|. The
+    // first round of all three is loaded together (one memory round trip for
+    // the usual sizes); any rest follows in rolled loops.
     {
-        // fp16 magnitudes order like their bit patterns: the maximum is taken on the bits
-        unsigned m2 = 0u;
+        // fp16 magnitudes order like their bit patterns: the maximum is taken on
+        // the bits, two at a time (16-byte loads when beta is 16-byte aligned)
         const int nb = L.R * ell;
-        for (int i = tid; i < nb; i += kThreads) m2 = max(m2, static_cast<unsigned>(__ldg(L.beta + i)) & 0x7FFFu);
+        const int nv = (reinterpret_cast<uintptr_t>(L.beta) & 15u) == 0 ? nb / 8 : 0;
+        const uint4 *bp = reinterpret_cast<const uint4 *>(L.beta);
+        constexpr int kV = 4;   // 16-byte beta loads per thread in the first round
+        uint4 w[kV];
 #pragma unroll
+        for (int e = 0; e < kV; ++e) {
+            const int i = tid + e * kThreads;
+            w[e] = i < nv ? __ldg(bp + i) : make_uint4(0u, 0u, 0u, 0u);
+        }
+        auto scale1 = [&](int i) {
+            const int e = i / rows1, r = i - e * rows1;
+            return r < n1 ? ldg_h(L.beta + static_cast<int64_t>(e) * L.R + lo1 + r) : 0.f;
+        };
+        auto scale2 = [&](int i) {
+            const int e = i / rows2, r = i - e * rows2;
+            return r < n2 ? ldg_h(L.alpha + static_cast<int64_t>(e) * L.N + lo2 + r) : 0.f;
+        };
+        const float v1 = tid < rows1 * ell ? scale1(tid) : 0.f;
+        const float v2 = tid < rows2 * ell ? scale2(tid) : 0.f;
+        unsigned m2 = 0u;
+#pragma unroll
+        for (int e = 0; e < kV; ++e) {
+            m2 = __vmaxu2(m2, w[e].x & 0x7FFF7FFFu);
+            m2 = __vmaxu2(m2, w[e].y & 0x7FFF7FFFu);
+            m2 = __vmaxu2(m2, w[e].z & 0x7FFF7FFFu);
+            m2 = __vmaxu2(m2, w[e].w & 0x7FFF7FFFu);
+        }
+        if (tid < rows1 * ell) rs1[tid] = v1;
+        if (tid < rows2 * ell) rs2[tid] = v2;
+#pragma unroll 1
+        for (int i = tid + kThreads; i < rows1 * ell; i += kThreads) rs1[i] = scale1(i);
+#pragma unroll 1
+        for (int i = tid + kThreads; i < rows2 * ell; i += kThreads) rs2[i] = scale2(i);
+#pragma unroll 1
+        for (int i = tid + kV * kThreads; i < nv; i += kThreads) {
+            const uint4 u = __ldg(bp + i);
+            m2 = __vmaxu2(__vmaxu2(m2, u.x & 0x7FFF7FFFu), __vmaxu2(u.y & 0x7FFF7FFFu, u.z & 0x7FFF7FFFu));
+            m2 = __vmaxu2(m2, u.w & 0x7FFF7FFFu);
+        }
+#pragma unroll 1
+        for (int i = nv * 8 + tid; i < nb; i += kThreads) m2 = max(m2, static_cast<unsigned>(__ldg(L.beta + i)) & 0x7FFFu);
+        m2 = max(m2 & 0xFFFFu, m2 >> 16);
         for (int o = 16; o; o >>= 1) m2 = max(m2, __shfl_xor_sync(0xffffffffu, m2, o));
         if (lane == 0) atomicMax(&ms->bmax, __float_as_uint(__half2float(__ushort_as_half(static_cast<unsigned short>(m2)))));
     }
     // the zero digit column of stage 1 (digit columns past 3C of an MMA column group)
+#pragma unroll 1
     for (int i = tid; i < P.cb1 / 16; i += kThreads)
         reinterpret_cast<uint4 *>(dig + static_cast<size_t>(ndcol) * P.cb1)[i] = make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll 1
+    for (int i = tid; i < rows1 * P.tile_ld; i += kThreads) tile[i] = 0;
+
+    // ---- activations: x, one token at a time, into two shared-memory buffers
+    // (the next token's copy is in flight while a token is digitised)
     if (early) pdl_wait();
     if (tid == 0) {
         unsigned long long v;
         asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(P.sync) : "memory");
         ms->e0 = static_cast<unsigned>(v >> 32);
     }
+    const int xsize = P.xd == DBF_BF16 ? 2 : 4;
+    auto stage_token = [&](int t) {
+        unsigned char *dst = smem + P.off_s2 + P.gs_bytes + (t & 1) * P.xs_bytes;
+        const unsigned char *src = static_cast<const unsigned char *>(P.x) + static_cast<int64_t>(t) * L.M * xsize;
+        if (P.bulk_x) {
+            if (tid == 0) {
+                // the buffer's previous token was read by generic loads: order
+                // them before the asynchronous write
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                bar_expect_tx(&ms->bar[3 + (t & 1)], static_cast<uint32_t>(L.M * xsize));
+                bulk_g2s(dst, src, static_cast<uint32_t>(L.M * xsize), &ms->bar[3 + (t & 1)]);
+            }
+        } else if (xsize == 2) {
+#pragma unroll 1
+            for (int i = tid; i < L.M; i += kThreads)
+                reinterpret_cast<uint16_t *>(dst)[i] = reinterpret_cast<const uint16_t *>(src)[i];
+        } else {
+#pragma unroll 1
+            for (int i = tid; i < L.M; i += kThreads)
+                reinterpret_cast<uint32_t *>(dst)[i] = reinterpret_cast<const uint32_t *>(src)[i];
+        }
+    };
+    stage_token(0);
+    if (P.T > 1) stage_token(1);
 
     // ---- stage 1 operand: digits of q = round(gamma_i . x_t 2^sh) per column.
-    // Warp w builds words w, w + 8, ... (up to the last 256-column group, zeros
-    // past M); lane l holds the column bit l stands for.
+    // A half warp takes one packed word per step: lane p (of 16) the columns
+    // 2p and 2p + 1, which bits p and 16 + p stand for. Two passes over
+    // shared memory: the column's max |gamma . x|, then its digits.
     const bool do1 = n1 > 0;
-    for (int c = 0; c < C; ++c) {
-        const int tok = c / ell, env = c - tok * ell;
-        const uint16_t *gp = L.gamma + static_cast<int64_t>(env) * L.M;
-        const int64_t xb = static_cast<int64_t>(tok) * L.M;
-        const int nw = P.ng1 * kGroupWords;
-        float u[kMaxWordsPerWarp];
-        float m = 0.f;
-#pragma unroll
-        for (int j = 0; j < kMaxWordsPerWarp; ++j) {
-            const int w = warp + j * kWarps;
-            const int col = 32 * w + col_of_bit(lane);
-            const bool in = w < P.pitch1 && col < L.M;
-            u[j] = in ? ldg_h(gp + col) * load_x(P.x, P.xd, xb + col) : 0.f;   // exact in fp32
-            m = fmaxf(m, fabsf(u[j]));
-        }
-#pragma unroll
-        for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-        if (lane == 0) atomicMax(&ms->amax[c], __float_as_uint(m));
-        __syncthreads();
-        const int sh = scale_exponent(__uint_as_float(ms->amax[c]));
-        int sq = 0, sa = 0;
-        char *d0 = dig + static_cast<size_t>(kDigits * c) * P.cb1;
-#pragma unroll
-        for (int j = 0; j < kMaxWordsPerWarp; ++j) {
-            const int w = warp + j * kWarps;
-            if (w < nw) {   // warp-uniform
-                const int q = quantize(u[j], sh);
-                sq += q;
-                sa += abs(q);
-                if (do1) {
-                    const uint32_t db = digit_bytes(q);
-                    const int off = digit_byte(w, lane);
-                    d0[off] = static_cast<char>(db & 255u);
-                    d0[P.cb1 + off] = static_cast<char>((db >> 8) & 255u);
-                    d0[2 * P.cb1 + off] = static_cast<char>(db >> 16);
-                }
+    const int nwp = P.ng1 * kGroupWords / 2;   // word pairs, up to the last 256-column group
+    const int hp = lane & 15, hw = lane >> 4;
+#pragma unroll 1
+    for (int tok = 0; tok < P.T; ++tok) {
+        token_wait(P, ms, tok);
+        const unsigned char *xs = smem + P.off_s2 + P.gs_bytes + (tok & 1) * P.xs_bytes;
+#pragma unroll 1
+        for (int env = 0; env < ell; ++env) {
+            const int c = tok * ell + env;
+            const uint16_t *gc = gs + static_cast<int64_t>(env) * P.gpitch;
+            float m = 0.f;
+            // unrolled by four: the iterations' shared-memory loads overlap
+#pragma unroll 4
+            for (int wp = warp; wp < nwp; wp += kWarps) {
+                const int col = 64 * wp + 32 * hw + 2 * hp;
+                const float2 u = stage_u2(gc, xs, P.xd, col, L.M);
+                m = fmaxf(m, fmaxf(fabsf(u.x), fabsf(u.y)));
             }
+            for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+            if (lane == 0) atomicMax(&ms->amax[c], __float_as_uint(m));
+            __syncthreads();
+            const int sh = scale_exponent(__uint_as_float(ms->amax[c]));
+            int sq = 0, sa = 0;
+            char *d0 = dig + static_cast<size_t>(kDigits * c) * P.cb1;
+#pragma unroll 4
+            for (int wp = warp; wp < nwp; wp += kWarps) {
+                const int w = 2 * wp + hw;
+                const float2 u = stage_u2(gc, xs, P.xd, 32 * w + 2 * hp, L.M);
+                const int q0 = quantize(u.x, sh), q1 = quantize(u.y, sh);
+                sq += q0 + q1;
+                sa += abs(q0) + abs(q1);
+                const uint32_t d0b = digit_bytes(q0), d1b = digit_bytes(q1);
+                const int off = digit_byte(w, hp);   // bit hp; bit 16 + hp is two bytes on
+                d0[off] = static_cast<char>(d0b & 255u);
+                d0[off + 2] = static_cast<char>(d1b & 255u);
+                d0[P.cb1 + off] = static_cast<char>((d0b >> 8) & 255u);
+                d0[P.cb1 + off + 2] = static_cast<char>((d1b >> 8) & 255u);
+                d0[2 * P.cb1 + off] = static_cast<char>(d0b >> 16);
+                d0[2 * P.cb1 + off + 2] = static_cast<char>(d1b >> 16);
+            }
+            const long long sq64 = warp_sum64(sq), sa64 = warp_sum64(sa);
+            if (lane == 0) {
+                atomicAdd(reinterpret_cast<unsigned long long *>(&ms->qsum_u[c]), static_cast<unsigned long long>(sq64));
+                atomicAdd(reinterpret_cast<unsigned long long *>(&ms->qabs_u[c]), static_cast<unsigned long long>(sa64));
+            }
+            if (tid == 0) ms->sh_u[c] = sh;
         }
-        const long long sq64 = warp_sum64(sq), sa64 = warp_sum64(sa);
-        if (lane == 0) {
-            atomicAdd(reinterpret_cast<unsigned long long *>(&ms->qsum_u[c]), static_cast<unsigned long long>(sq64));
-            atomicAdd(reinterpret_cast<unsigned long long *>(&ms->qabs_u[c]), static_cast<unsigned long long>(sa64));
+        if (tok + 2 < P.T) {
+            __syncthreads();   // every read of this token's buffer is done
+            stage_token(tok + 2);
         }
-        if (tid == 0) ms->sh_u[c] = sh;
     }
-    for (int i = tid; i < rows1 * P.tile_ld; i += kThreads) tile[i] = 0;
     __syncthreads();
+    // ---- the B1 slice -> shared memory (over the staged x and gamma, which
+    // are no longer read: the generic reads are ordered before the copy)
+    if (warp == 0) {
+        if (lane == 0) {
+            if (P.bulk2 && n2 > 0) bar_expect_tx(&ms->bar[1], static_cast<uint32_t>(n2) * P.pitch2 * 4u);
+        }
+        __syncwarp();
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        if (P.bulk2) slice_bulk(s2, L.b1_packed + static_cast<int64_t>(lo2) * P.pitch2, n2, P.pitch2, P.stride2, &ms->bar[1]);
+    }
+    slice_pad(s2, n2, rows2, P.pitch2, P.stride2);
+    if (!P.bulk2) slice_plain(s2, L.b1_packed + static_cast<int64_t>(lo2) * P.pitch2, n2, P.pitch2, P.stride2);
     if (tid < C) {
         // |v_r| = |beta_r h_r| <= max|beta| sum|q| 2^-sh; the factor covers the
         // fp32 roundings of h and of beta h
@@ -528,9 +665,13 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const __grid_consta
         if (ok1) {
             sign_sums(s1, P.stride1, rows1 / 16, P.ng1, dig, P.cb1, ndcol, tile, P.tile_ld);
             __syncthreads();
-            long long qp[kMaxCols];
+            // one (row, column) per thread and step; each thread's sums of q of v
+            // per column (at most two elements: int32) are reduced per warp and
+            // added to shared memory
+            int qv[kMaxCols];
 #pragma unroll
-            for (int c = 0; c < kMaxCols; ++c) qp[c] = 0;
+            for (int c = 0; c < kMaxCols; ++c) qv[c] = 0;
+#pragma unroll 1
             for (int i = tid; i < n1 * C; i += kThreads) {
                 const int c = i / n1, lr = i - c * n1;
                 const int env = c - (c / ell) * ell;
@@ -544,21 +685,22 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const __grid_consta
                 im[2 * P.cb2] = static_cast<char>(db >> 16);
 #pragma unroll
                 for (int cc = 0; cc < kMaxCols; ++cc)
-                    if (cc == c) qp[cc] += q;
+                    if (cc == c) qv[cc] += q;
             }
-            for (int c = 0; c < C; ++c) {
-                long long v = 0;
 #pragma unroll
-                for (int cc = 0; cc < kMaxCols; ++cc)
-                    if (cc == c) v = qp[cc];
-                v = warp_sum64(v);
-                if (lane == 0) atomicAdd(reinterpret_cast<unsigned long long *>(&ms->qpart_v[c]), static_cast<unsigned long long>(v));
+            for (int c = 0; c < kMaxCols; ++c) {
+                if (c < C) {
+                    const int w = __reduce_add_sync(0xffffffffu, qv[c]);
+                    if (lane == 0 && w) atomicAdd(reinterpret_cast<unsigned long long *>(&ms->qpart_v[c]),
+                                                  static_cast<unsigned long long>(static_cast<long long>(w)));
+                }
             }
         }
     }
     // digits of v past the rank, up to the last 256-column group, are zero
     if (r1e == P.nrb1 && r1e > r1b) {
         const int tail = P.ng2 * 256 - L.R;
+#pragma unroll 1
         for (int i = tid; i < C * tail; i += kThreads) {
             const int c = i / tail, r = L.R + (i - c * tail);
             char *im = P.img + static_cast<size_t>(kDigits * c) * P.cb2 + digit_offset(r);
@@ -579,12 +721,23 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const __grid_consta
     }
 
     // ---- stage 2: the digits of v (coherent 16-byte loads: other CTAs wrote
-    // them in this kernel), the sums of q of v, then the CTA's rows of y
+    // them in this kernel) and the sums of q of v, their loads in flight
+    // together, then the CTA's rows of y
     {
+        constexpr int kP = (kMaxGrid + 31) / 32;
+        long long part[kP];
+        if (warp < C) {
+#pragma unroll
+            for (int e = 0; e < kP; ++e) {
+                const int k = lane + 32 * e;
+                part[e] = k < G ? __ldcg(P.qpart + static_cast<int64_t>(k) * C + warp) : 0;
+            }
+        }
         const int n16 = ndcol * P.cb2 / 16;
         const uint4 *src = reinterpret_cast<const uint4 *>(P.img);
         uint4 *dst = reinterpret_cast<uint4 *>(dig);
         constexpr int kLoads = 8;
+#pragma unroll 1
         for (int i0 = tid; i0 < n16; i0 += kLoads * kThreads) {
             uint4 v[kLoads];
 #pragma unroll
@@ -596,15 +749,18 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const __grid_consta
             for (int e = 0; e < kLoads; ++e)
                 if (i0 + e * kThreads < n16) dst[i0 + e * kThreads] = v[e];
         }
+        if (warp < C) {
+            long long sum = 0;
+#pragma unroll
+            for (int e = 0; e < kP; ++e) sum += part[e];
+            sum = warp_sum64(sum);
+            if (lane == 0) ms->qsum_v[warp] = sum;
+        }
     }
-    if (warp < C) {
-        long long s = 0;
-        for (int k = lane; k < G; k += 32) s += __ldcg(P.qpart + static_cast<int64_t>(k) * C + warp);
-        s = warp_sum64(s);
-        if (lane == 0) ms->qsum_v[warp] = s;
-    }
+#pragma unroll 1
     for (int i = tid; i < P.cb2 / 16; i += kThreads)
         reinterpret_cast<uint4 *>(dig + static_cast<size_t>(ndcol) * P.cb2)[i] = make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll 1
     for (int i = tid; i < rows2 * P.tile_ld; i += kThreads) tile[i] = 0;
     if (P.bulk2) {
         if (!slice_wait(&ms->bar[1], P, ms)) return;
@@ -614,10 +770,12 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const __grid_consta
     sign_sums(s2, P.stride2, rows2 / 16, P.ng2, dig, P.cb2, ndcol, tile, P.tile_ld);
     __syncthreads();
     // ---- y = [acc] y + sum_i alpha_i . z_i, one (token, row) per thread
+#pragma unroll 1
     for (int i = tid; i < P.T * n2; i += kThreads) {
         const int tok = i / n2, lr = i - tok * n2;
         const int64_t yi = static_cast<int64_t>(tok) * L.N + lo2 + lr;
         float yv = (P.flags & DBF_ACCUMULATE) ? load_act(P.y, P.yd, yi) : 0.f;
+#pragma unroll 1
         for (int env = 0; env < ell; ++env) {
             const int c = tok * ell + env;
             const long long s = digit_sum(tile + lr * P.tile_ld, c);
@@ -629,7 +787,6 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const __grid_consta
 }
 
 // ---- host side ----------------------------------------------------------------
-constexpr int kMaxGrid = 160;   // CTAs at most (sizes the per-CTA sums in the workspace)
 
 // Row stride of a slice: whole 8-word groups, and a stride of 8 or 24 words
 // modulo 32 so that the 8-byte A-fragment loads of rows g = 0..3 (a half
@@ -683,9 +840,15 @@ bool decode_plan(const dbf_layer &L, int64_t T, int sms, DecodeParams *out, size
     P.tile_ld = 8 * ((kDigits * P.C + 7) / 8);
     const int rows1 = P.max_rb1 * 16, rows2 = P.max_rb2 * 16;
     const int cbm = P.cb1 > P.cb2 ? P.cb1 : P.cb2;
+    // gamma and x are staged in the B1 slice's region (fp32 x: 4 bytes per value)
+    P.gpitch = (L.M + 7) / 8 * 8;
+    P.gs_bytes = static_cast<int>(static_cast<size_t>(L.ell) * P.gpitch * 2);
+    P.xs_bytes = static_cast<int>(align_up(static_cast<size_t>(L.M) * 4, 16));   // fp32 x at most
+    const size_t s2_bytes = static_cast<size_t>(rows2) * P.stride2 * 4;
+    const size_t stage_bytes = static_cast<size_t>(P.gs_bytes) + 2 * static_cast<size_t>(P.xs_bytes);
     size_t off = align_up(static_cast<size_t>(rows1) * P.stride1 * 4, 128);
     P.off_s2 = static_cast<int>(off);
-    off = align_up(off + static_cast<size_t>(rows2) * P.stride2 * 4, 128);
+    off = align_up(off + (s2_bytes > stage_bytes ? s2_bytes : stage_bytes), 128);
     P.off_dig = static_cast<int>(off);
     off = align_up(off + static_cast<size_t>(kDigits * P.C + 1) * cbm, 16);
     P.off_tile = static_cast<int>(off);
@@ -740,6 +903,10 @@ cudaError_t decode_forward(const dbf_layer &L, const void *x, dbf_dtype xd, void
     P.img = w + kWsHeaderBytes;
     P.qpart = reinterpret_cast<long long *>(w + kWsHeaderBytes + img_bytes(P.C, P.ng2));
     P.wait_ns = g_wait_ns ? g_wait_ns : kDefaultWaitNs;
+    // staged inputs by bulk copies when whole 16-byte units (x is 16-byte
+    // aligned by the call's contract; gamma only 2-byte)
+    P.bulk_x = (static_cast<size_t>(L.M) * (xd == DBF_BF16 ? 2 : 4)) % 16 == 0;
+    P.bulk_g = (reinterpret_cast<uintptr_t>(L.gamma) & 15u) == 0 && L.M % 8 == 0;   // rows unpadded
     cudaError_t e = allow_smem(reinterpret_cast<const void *>(decode_kernel), static_cast<int>(smem), true);
     if (e != cudaSuccess) return e;
 

@@ -37,6 +37,7 @@
 #include "dbf_internal.cuh"
 
 #include <cuda.h>
+#include <mutex>
 #include <cudaTypedefs.h>
 
 namespace dbf {
@@ -50,9 +51,15 @@ constexpr int BK = 64;              // K per stage: one 128-byte swizzle row of 
 // backward, whose epilogues read and write an operand per element, takes
 // eight epilogue warps (two per TMEM lane quarter, each with half of the
 // columns) and one expansion group.
-template <int kGroups, int kSA, int kSB, int kEpi, bool kBackward>
+template <int kGroups, int kSA, int kSB, int kEpi, bool kBackward, bool kPairMode = false>
 struct GemmCfg {
     static constexpr bool kBwd = kBackward;      // epilogues of stages 3..6 compiled in
+    // CTA pairs (a cluster of two): tcgen05 cta_group::2 with M = 256 over the
+    // two SMs; each CTA holds its 128 sign rows of A and half of the 256 token
+    // rows of B, and its TMEM the accumulator of its 128 rows
+    static constexpr bool kPair = kPairMode;
+    static constexpr int kBRows = kPairMode ? 128 : 256;   // B rows a CTA loads per stage
+    static constexpr int kBBytes = kBRows * 64 * 2;
     static constexpr int SA = kSA;               // stages of expanded sign tiles (produced on chip)
     static constexpr int SB = kSB;               // stages of TMA activation tiles
     static constexpr int kExpandGroups = kGroups;
@@ -61,10 +68,10 @@ struct GemmCfg {
     static constexpr int kThreads = 32 * (2 + kExpandWarps + kEpiWarps);
 };
 using FwdCfg = GemmCfg<2, 6, 4, 4, false>;
+using FwdPairCfg = GemmCfg<2, 6, 6, 4, false, true>;
 using BwdCfg = GemmCfg<1, 4, 5, 8, true>;
 constexpr int kMaxStages = 8;
 constexpr int A_BYTES = BM * BK * 2;   // 16 KB
-constexpr int B_BYTES = BN * BK * 2;   // 32 KB
 constexpr int TMEM_COLS = 512;          // two 256-column accumulators
 constexpr unsigned long long kWaitNs = 1000000000ull;   // bounded waits: 1 s
 
@@ -125,9 +132,19 @@ struct TileRef {
     const GroupRef *gr;
 };
 
-__device__ __forceinline__ TileRef tile_ref(const GemmArgs &g, int tile, int n_p)
+__device__ __forceinline__ TileRef tile_ref(const GemmArgs &g, int tile, int n_p, int pair_rank = -1)
 {
     TileRef r;
+    if (pair_rank >= 0) {
+        // a pair tile: 256 sign rows, this CTA's 128 of them
+        r.p0 = (tile % n_p) * 2 * BM + pair_rank * BM;
+        r.brow = (tile / n_p) * BN;
+        r.t0 = r.brow;
+        r.t1 = g.C;
+        r.env = 0;
+        r.gr = nullptr;
+        return r;
+    }
     if (g.ngroups == 0) {
         r.p0 = (tile % n_p) * BM;
         r.brow = (tile / n_p) * BN;
@@ -219,6 +236,39 @@ __device__ __forceinline__ void drain_wait(uint64_t *bar, uint32_t parity)
     }
 }
 
+// ---- CTA-pair helpers ------------------------------------------------------
+// Shared-memory address of the same object in CTA 0 of the pair: bit 24 of
+// a shared::cluster address selects the CTA of the pair.
+__device__ __forceinline__ uint32_t pair_leader_addr(const void *p) { return smem_u32(p) & 0xFEFFFFFFu; }
+
+// Arrive on a barrier of the pair's CTA 0 (its MMA reads the tiles this CTA
+// wrote: the writer fences its generic stores to the async proxy first).
+__device__ __forceinline__ void bar_arrive_leader(uint64_t *bar)
+{
+    asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(pair_leader_addr(bar)) : "memory");
+}
+
+// Arrive on the same barrier in CTA 'rank' of the cluster.
+__device__ __forceinline__ void bar_arrive_rank(uint64_t *bar, uint32_t rank)
+{
+    asm volatile(
+        "{\n\t.reg .b32 ra;\n\t"
+        "mapa.shared::cluster.u32 ra, %0, %1;\n\t"
+        "mbarrier.arrive.shared::cluster.b64 _, [ra];\n\t}" ::"r"(smem_u32(bar)),
+        "r"(rank)
+        : "memory");
+}
+
+// Tile load of one CTA of a pair: the bytes are counted on CTA 0's barrier.
+__device__ __forceinline__ void tma_load_2d_pair(void *dst, const CUtensorMap *map, int c0, int c1, uint64_t *bar)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, "
+        "%3}], [%4];" ::"r"(smem_u32(dst)),
+        "l"(map), "r"(c0), "r"(c1), "r"(pair_leader_addr(bar))
+        : "memory");
+}
+
 __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, int c0, int c1, uint64_t *bar)
 {
     asm volatile(
@@ -260,6 +310,38 @@ __device__ __forceinline__ void mma_f16(uint32_t tmem_d, uint64_t a, uint64_t b,
         : "memory");
 }
 
+// The pair's MMA (issued by CTA 0): M = 256 (128 rows from each CTA's A
+// tile), N = 256 (128 columns from each CTA's B tile); each CTA's TMEM gets
+// the accumulator of its rows.
+constexpr uint32_t kIdescPair = (1u << 4) | (static_cast<uint32_t>(BN >> 3) << 17) | (static_cast<uint32_t>((2 * BM) >> 4) << 24);
+
+__device__ __forceinline__ void mma_f16_pair(uint32_t tmem_d, uint64_t a, uint64_t b, uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+        "l"(a), "l"(b), "r"(kIdescPair), "r"(accumulate)
+        : "memory");
+}
+
+// Commit of the pair's MMAs to the same barrier in both CTAs.
+__device__ __forceinline__ void mma_commit_pair_both(uint64_t *bar)
+{
+    asm volatile(
+        "{\n\t.reg .b16 msk;\n\t"
+        "mov.b16 msk, 3;\n\t"
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], msk;\n\t}" ::"r"(
+            smem_u32(bar))
+        : "memory");
+}
+
+__device__ __forceinline__ void mma_commit_pair_own(uint64_t *bar)
+{
+    asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+                 : "memory");
+}
+
 __device__ __forceinline__ void mma_commit(uint64_t *bar)
 {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
@@ -289,16 +371,10 @@ __device__ __forceinline__ uint32_t sign_pair(uint32_t w, int p, uint32_t mag2)
 struct GemmSmem {
     uint64_t full_a[kMaxStages], empty_a[kMaxStages], full_b[kMaxStages], empty_b[kMaxStages], acc_full[2], acc_empty[2];
     uint64_t drain;   // the MMA thread's last commit: every MMA it issued has completed
+    uint64_t exit_bar;   // CTA pairs: the peer is done with this CTA's shared memory
     uint32_t tmem_base;
     int abort;
 };
-
-__device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volatile int *abort)
-{
-    bool ok = true;
-    if ((threadIdx.x & 31) == 0) ok = bar_wait(bar, parity, abort);
-    return __shfl_sync(0xffffffffu, ok, 0);
-}
 
 // Epilogue of a grouped tile, 32 columns = tokens t0 .. t0 + 31 (those below
 // the group's end): stage 1 writes v = fp16(beta h) of envelope tr.env,
@@ -422,21 +498,31 @@ __global__ void __launch_bounds__(Cfg::kThreads, 1) gemm_kernel(const __grid_con
     // 1024-byte alignment for the swizzled tiles
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *smA = smem;
+    constexpr bool kPair = Cfg::kPair;
+    constexpr int kBBytes = Cfg::kBBytes;
     uint8_t *smB = smA + SA * A_BYTES;
-    GemmSmem *sh = reinterpret_cast<GemmSmem *>(smB + SB * B_BYTES);
+    GemmSmem *sh = reinterpret_cast<GemmSmem *>(smB + SB * kBBytes);
     volatile int *abort = &sh->abort;
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int n_p = (g.P + BM - 1) / BM;
+    // tiles are walked per CTA, or per CTA pair (rank 0 issues the pair's MMAs)
+    uint32_t rank = 0;
+    if (kPair) asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(rank));
+    const int unit = kPair ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
+    const int nunits = kPair ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
+    const int tile_rank = kPair ? static_cast<int>(rank) : -1;
+    const int n_p = (g.P + (kPair ? 2 * BM : BM) - 1) / (kPair ? 2 * BM : BM);
     const int n_c = (g.C + BN - 1) / BN;
     const int ntiles = g.ngroups ? g.tiles_total : n_p * n_c;
-    const int my_tiles = blockIdx.x < ntiles ? (ntiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+    const int my_tiles = unit < ntiles ? (ntiles - 1 - unit) / nunits + 1 : 0;
     const int nk = g.Ktot / BK;
+    auto wait = [&](uint64_t *bar, uint32_t parity) { return bar_wait(bar, parity, abort); };
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < SA; ++i) {
-            bar_init(&sh->full_a[i], g.dense_a ? 1 : 4);   // the TMA producer, or the four warps of one expansion group
+            // the TMA producer, or the four warps of one expansion group (of both CTAs of a pair)
+            bar_init(&sh->full_a[i], g.dense_a ? 1 : (kPair ? 8 : 4));
             bar_init(&sh->empty_a[i], 1);
         }
         for (int i = 0; i < SB; ++i) {
@@ -445,21 +531,33 @@ __global__ void __launch_bounds__(Cfg::kThreads, 1) gemm_kernel(const __grid_con
         }
         for (int i = 0; i < 2; ++i) {
             bar_init(&sh->acc_full[i], 1);
-            bar_init(&sh->acc_empty[i], kEpiWarps);
+            bar_init(&sh->acc_empty[i], kPair ? 2 * kEpiWarps : kEpiWarps);
         }
         bar_init(&sh->drain, 1);
+        bar_init(&sh->exit_bar, 1);
         sh->abort = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         asm volatile("prefetch.tensormap [%0];" ::"l"(&tmB) : "memory");
         if (g.dense_a) asm volatile("prefetch.tensormap [%0];" ::"l"(&tmA) : "memory");
     }
     if (warp == 1) {
-        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&sh->tmem_base)),
-                     "r"(TMEM_COLS));
-        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+        if (kPair) {
+            asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&sh->tmem_base)),
+                         "r"(TMEM_COLS));
+            asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;");
+        } else {
+            asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&sh->tmem_base)),
+                         "r"(TMEM_COLS));
+            asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+        }
     }
     tc_fence_before();
     __syncthreads();
+    if (kPair) {
+        // both CTAs' barriers are initialised before either reaches the other's
+        asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+        asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+    }
     tc_fence_after();
     const uint32_t tmem = sh->tmem_base;
 
@@ -469,14 +567,21 @@ __global__ void __launch_bounds__(Cfg::kThreads, 1) gemm_kernel(const __grid_con
             int s = 0;
             int nb_issued = 0, na_issued = 0;   // TMA loads issued on each ring
             for (int j = 0; j < my_tiles && !*abort; ++j) {
-                const TileRef tr = tile_ref(g, blockIdx.x + j * gridDim.x, n_p);
+                const TileRef tr = tile_ref(g, unit + j * nunits, n_p, tile_rank);
                 const int c0 = tr.brow;
                 const int p0 = tr.p0;
                 for (int k = 0; k < nk; ++k, ++s) {
                     const int st = s % SB;
-                    if (!bar_wait(&sh->empty_b[st], ((s / SB) & 1) ^ 1, abort)) break;
-                    bar_expect_tx(&sh->full_b[st], B_BYTES);
-                    tma_load_2d(smB + st * B_BYTES, &tmB, k * BK, c0, &sh->full_b[st]);
+                    if (!wait(&sh->empty_b[st], ((s / SB) & 1) ^ 1)) break;
+                    if (kPair) {
+                        // CTA 0's barrier counts the bytes of both halves of B
+                        if (rank == 0) bar_expect_tx(&sh->full_b[st], 2 * kBBytes);
+                        tma_load_2d_pair(smB + st * kBBytes, &tmB, k * BK, c0 + static_cast<int>(rank) * Cfg::kBRows,
+                                         &sh->full_b[st]);
+                    } else {
+                        bar_expect_tx(&sh->full_b[st], kBBytes);
+                        tma_load_2d(smB + st * kBBytes, &tmB, k * BK, c0, &sh->full_b[st]);
+                    }
                     nb_issued = s + 1;
                     if (g.dense_a) {
                         // a dense fp16 A operand: its tile comes by TMA too, in the
@@ -491,41 +596,55 @@ __global__ void __launch_bounds__(Cfg::kThreads, 1) gemm_kernel(const __grid_con
             }
             // After an abort, the loads already issued (at most the last SB,
             // resp. SA, of each ring: earlier ones were consumed) land before
-            // the CTA ends and its shared memory is released. Bounded.
-            if (*abort) {
+            // the CTA ends and its shared memory is released. Bounded. (In a
+            // pair, CTA 0's barriers count both CTAs' loads; CTA 1 is held by
+            // the exit handshake until CTA 0 has waited for them.)
+            if (*abort && (!kPair || rank == 0)) {
                 for (int b = nb_issued - 1; b >= 0 && b >= nb_issued - SB; --b) drain_wait(&sh->full_b[b % SB], (b / SB) & 1);
                 for (int b = na_issued - 1; b >= 0 && b >= na_issued - SA; --b) drain_wait(&sh->full_a[b % SA], (b / SA) & 1);
             }
         }
     } else if (warp == 1) {
-        // ---------------- MMA issuer ----------------
-        if (lane == 0) {
+        // ---------------- MMA issuer (CTA 0 of a pair issues for both) ----------------
+        if (lane == 0 && (!kPair || rank == 0)) {
             int s = 0;
             bool ok = true;
             for (int j = 0; j < my_tiles && ok; ++j) {
                 const int ab = j & 1;
-                ok = bar_wait(&sh->acc_empty[ab], ((j >> 1) & 1) ^ 1, abort);
+                ok = wait(&sh->acc_empty[ab], ((j >> 1) & 1) ^ 1);
                 if (!ok) break;
                 tc_fence_after();
                 const uint32_t dt = tmem + static_cast<uint32_t>(ab * BN);
                 for (int k = 0; k < nk; ++k, ++s) {
                     const int sa = s % SA, sb = s % SB;
-                    ok = bar_wait(&sh->full_a[sa], (s / SA) & 1, abort) && bar_wait(&sh->full_b[sb], (s / SB) & 1, abort);
+                    ok = wait(&sh->full_a[sa], (s / SA) & 1) && wait(&sh->full_b[sb], (s / SB) & 1);
                     if (!ok) break;
                     tc_fence_after();
                     const uint64_t da = sw128_desc(smem_u32(smA + sa * A_BYTES));
-                    const uint64_t db = sw128_desc(smem_u32(smB + sb * B_BYTES));
+                    const uint64_t db = sw128_desc(smem_u32(smB + sb * kBBytes));
+                    if (kPair) {
 #pragma unroll
-                    for (int kk = 0; kk < BK / 16; ++kk)   // 32 bytes of K per MMA: +2 in 16-byte units
-                        mma_f16(dt, da + 2 * kk, db + 2 * kk, (k | kk) != 0);
-                    mma_commit(&sh->empty_a[sa]);   // each commit arrives once these MMAs are done
-                    mma_commit(&sh->empty_b[sb]);
+                        for (int kk = 0; kk < BK / 16; ++kk)
+                            mma_f16_pair(dt, da + 2 * kk, db + 2 * kk, (k | kk) != 0);
+                        mma_commit_pair_both(&sh->empty_a[sa]);   // both CTAs' stages are free again
+                        mma_commit_pair_both(&sh->empty_b[sb]);
+                    } else {
+#pragma unroll
+                        for (int kk = 0; kk < BK / 16; ++kk)   // 32 bytes of K per MMA: +2 in 16-byte units
+                            mma_f16(dt, da + 2 * kk, db + 2 * kk, (k | kk) != 0);
+                        mma_commit(&sh->empty_a[sa]);   // each commit arrives once these MMAs are done
+                        mma_commit(&sh->empty_b[sb]);
+                    }
                 }
-                if (ok) mma_commit(&sh->acc_full[ab]);
+                if (ok) {
+                    if (kPair) mma_commit_pair_both(&sh->acc_full[ab]);
+                    else mma_commit(&sh->acc_full[ab]);
+                }
             }
             // every MMA issued (also on an abort) has completed before tensor
             // memory is freed and the CTA ends
-            mma_commit(&sh->drain);
+            if (kPair) mma_commit_pair_own(&sh->drain);
+            else mma_commit(&sh->drain);
             drain_wait(&sh->drain, 0);
         }
     } else if (warp < 2 + kExpandWarps) {
@@ -554,7 +673,7 @@ __global__ void __launch_bounds__(Cfg::kThreads, 1) gemm_kernel(const __grid_con
             }
         };
         auto seat_tile = [&]() {
-            const TileRef tr = tile_ref(g, blockIdx.x + cj * gridDim.x, n_p);
+            const TileRef tr = tile_ref(g, unit + cj * nunits, n_p, tile_rank);
             cgrow = tr.p0 + prow;
             cvalid = cgrow < g.P;
             carow = tr.gr ? tr.gr->arow : g.arow_scale;
@@ -619,8 +738,7 @@ __global__ void __launch_bounds__(Cfg::kThreads, 1) gemm_kernel(const __grid_con
         auto expand_pair = [&](int p, const uint4 &w, uint32_t mag) {
             const int s0 = 2 * p, s1 = 2 * p + 1;
             const int st0 = s0 % SA, st1 = s1 % SA;
-            ok = bar_wait(&sh->empty_a[st0], ((s0 / SA) & 1) ^ 1, abort) &&
-                 bar_wait(&sh->empty_a[st1], ((s1 / SA) & 1) ^ 1, abort);
+            ok = wait(&sh->empty_a[st0], ((s0 / SA) & 1) ^ 1) && wait(&sh->empty_a[st1], ((s1 / SA) & 1) ^ 1);
             ok = __all_sync(0xffffffffu, ok);
             if (!ok) return;
             write_stage(st0, w.x, w.y, mag);
@@ -628,8 +746,13 @@ __global__ void __launch_bounds__(Cfg::kThreads, 1) gemm_kernel(const __grid_con
             fence_proxy_async();   // generic-proxy writes -> visible to the tensor core
             __syncwarp();
             if (lane == 0) {
-                bar_arrive(&sh->full_a[st0]);
-                bar_arrive(&sh->full_a[st1]);
+                if (kPair) {   // CTA 0 issues the MMAs that read both CTAs' tiles
+                    bar_arrive_leader(&sh->full_a[st0]);
+                    bar_arrive_leader(&sh->full_a[st1]);
+                } else {
+                    bar_arrive(&sh->full_a[st0]);
+                    bar_arrive(&sh->full_a[st1]);
+                }
             }
         };
         for (int base = grp; base < total_pairs && ok; base += D * kExpandGroups) {
@@ -651,9 +774,11 @@ __global__ void __launch_bounds__(Cfg::kThreads, 1) gemm_kernel(const __grid_con
         constexpr int kColShare = BN / (kEpiWarps / 4);
         for (int j = 0; j < my_tiles; ++j) {
             const int ab = j & 1;
-            if (!warp_wait(&sh->acc_full[ab], (j >> 1) & 1, abort)) break;
+            bool got = true;
+            if (lane == 0) got = wait(&sh->acc_full[ab], (j >> 1) & 1);
+            if (!__shfl_sync(0xffffffffu, got, 0)) break;
             tc_fence_after();
-            const TileRef tr = tile_ref(g, blockIdx.x + j * gridDim.x, n_p);
+            const TileRef tr = tile_ref(g, unit + j * nunits, n_p, tile_rank);
             const int p0 = tr.p0, c0 = tr.brow;
             const int grow = p0 + q * 32 + lane;
             const uint32_t taddr = tmem + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(ab * BN);
@@ -722,17 +847,33 @@ __global__ void __launch_bounds__(Cfg::kThreads, 1) gemm_kernel(const __grid_con
             }
             tc_fence_before();   // the accumulator reads are done before it is handed back
             __syncwarp();
-            if (lane == 0) bar_arrive(&sh->acc_empty[ab]);
+            if (lane == 0) {
+                if (kPair) bar_arrive_leader(&sh->acc_empty[ab]);
+                else bar_arrive(&sh->acc_empty[ab]);
+            }
         }
     }
 
 teardown:
     tc_fence_before();
     __syncthreads();
+    if (kPair) {
+        // neither CTA of a pair ends while the other may still reach its shared
+        // memory (remote arrivals, the pair's MMAs and their commits): each
+        // tells the other it is done and waits (bounded) for the other
+        if (threadIdx.x == 0) {
+            bar_arrive_rank(&sh->exit_bar, rank ^ 1u);
+            const unsigned long long t0 = global_ns();
+            while (!bar_try(&sh->exit_bar, 0) && global_ns() - t0 < kWaitNs) {
+            }
+        }
+        __syncthreads();
+    }
     if (sh->abort && threadIdx.x == 0 && g.status) atomicExch(g.status, static_cast<int32_t>(DBF_ERR_TIMEOUT));
     if (warp == 1) {
         tc_fence_after();
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS));
+        if (kPair) asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS));
+        else asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS));
     }
 }
 
@@ -888,7 +1029,7 @@ bool make_map(CUtensorMap *map, const void *base, int64_t K, int64_t rows, int b
 }
 
 template <class Cfg>
-constexpr size_t gemm_smem() { return 1024 + Cfg::SA * A_BYTES + Cfg::SB * B_BYTES + sizeof(GemmSmem) + 64; }
+constexpr size_t gemm_smem() { return 1024 + Cfg::SA * A_BYTES + Cfg::SB * Cfg::kBBytes + sizeof(GemmSmem) + 64; }
 
 template <class Cfg>
 cudaError_t launch_gemm(const CUtensorMap &map, const GemmArgs &args, cudaStream_t s, const CUtensorMap *map_a,
@@ -901,6 +1042,52 @@ cudaError_t launch_gemm(const CUtensorMap &map, const GemmArgs &args, cudaStream
     const int sms = device_sms();
     const int tiles = a.ngroups ? a.tiles_total : ((a.P + BM - 1) / BM) * ((a.C + BN - 1) / BN);
     gemm_kernel<Cfg><<<tiles < sms ? tiles : sms, Cfg::kThreads, gemm_smem<Cfg>(), s>>>(map, map_a ? *map_a : map, a);
+    return cudaGetLastError();
+}
+
+// The forward's GEMMs on CTA pairs: clusters of two CTAs, each pair walking
+// 256-row x 256-token tiles (as many pairs as can be resident at once).
+template <class Cfg>
+cudaError_t launch_gemm_pair(const CUtensorMap &map, const GemmArgs &args, cudaStream_t s, int32_t *status)
+{
+    GemmArgs a = args;
+    a.status = status;
+    const size_t smem = gemm_smem<Cfg>();
+    cudaError_t e = allow_smem(reinterpret_cast<const void *>(gemm_kernel<Cfg>), static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    const int tiles = ((a.P + 2 * BM - 1) / (2 * BM)) * ((a.C + BN - 1) / BN);
+    cudaLaunchConfig_t cfg = {};
+    cfg.blockDim = dim3(Cfg::kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    // resident pairs: queried once per device (the query is slow next to a launch)
+    static std::mutex lock;
+    static int resident[64] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    int pairs = device_sms() / 2;
+    if (dev >= 0 && dev < 64) {
+        std::lock_guard<std::mutex> guard(lock);
+        if (!resident[dev]) {
+            cfg.gridDim = dim3(2 * pairs);
+            int n = 0;
+            resident[dev] = (cudaOccupancyMaxActiveClusters(&n, gemm_kernel<Cfg>, &cfg) == cudaSuccess && n > 0) ? n : pairs;
+            (void)cudaGetLastError();
+        }
+        if (resident[dev] < pairs) pairs = resident[dev];
+    }
+    if (pairs > tiles) pairs = tiles;
+    if (pairs < 1) pairs = 1;
+    cfg.gridDim = dim3(2 * pairs);
+    e = cudaLaunchKernelEx(&cfg, gemm_kernel<Cfg>, map, map, a);
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 
@@ -937,9 +1124,10 @@ cudaError_t gemm_forward(const dbf_layer &L, const void *x, dbf_dtype xd, void *
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
+    // CTA pairs: each CTA loads 128 of a tile's 256 token rows
     CUtensorMap mu, mv;
-    if (!make_map(&mu, U, L.M, static_cast<int64_t>(L.ell) * T)) return cudaErrorInvalidValue;
-    if (!make_map(&mv, V, static_cast<int64_t>(L.ell) * L.R, T)) return cudaErrorInvalidValue;
+    if (!make_map(&mu, U, L.M, static_cast<int64_t>(L.ell) * T, FwdPairCfg::kBRows)) return cudaErrorInvalidValue;
+    if (!make_map(&mv, V, static_cast<int64_t>(L.ell) * L.R, T, FwdPairCfg::kBRows)) return cudaErrorInvalidValue;
     GemmArgs a1 = {};
     a1.signs = L.b2_packed;
     a1.pitch = static_cast<int>(pitch_words(L.M));
@@ -955,7 +1143,7 @@ cudaError_t gemm_forward(const dbf_layer &L, const void *x, dbf_dtype xd, void *
     a1.ell = L.ell;
     a1.R = L.R;
     a1.N = L.N;
-    cudaError_t e = launch_gemm<FwdCfg>(mu, a1, s, nullptr, st);
+    cudaError_t e = launch_gemm_pair<FwdPairCfg>(mu, a1, s, st);
     if (e != cudaSuccess) return e;
     GemmArgs a2 = {};
     a2.signs = L.b1_packed;
@@ -973,7 +1161,7 @@ cudaError_t gemm_forward(const dbf_layer &L, const void *x, dbf_dtype xd, void *
     a2.yd = yd;
     a2.N = L.N;
     a2.accumulate = (flags & DBF_ACCUMULATE) ? 1 : 0;
-    return launch_gemm<FwdCfg>(mv, a2, s, nullptr, st);
+    return launch_gemm_pair<FwdPairCfg>(mv, a2, s, st);
 }
 
 }  // namespace dbf

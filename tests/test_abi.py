@@ -117,8 +117,8 @@ def test_segmented_rejects_bad_arguments(lib):
 def test_forward_launch_count(lib):
     # host-side query, no launch: GEMM path = pre-pass + two stages; GEMV path
     # = one kernel while T * ell <= 8, M <= 8192 and its shared memory fits
-    # (on this layer the digits of v take 17.8 KB per column: up to 7 columns),
-    # else two
+    # (on this layer the digits of v take 17.8 KB per column: up to 7
+    # columns), else two
     import double_binary_rank_b200 as dbf
     by = ctypes.byref
     L = _layer(M=4096, N=11008, R=5888, ell=1)

@@ -4,9 +4,9 @@ model on the CPU under adversarial schedules.
 The kernel's barrier word (workspace header, 8 bytes) holds an arrival count
 (low 32 bits) and an epoch (high 32 bits). Each CTA of a call reads the epoch
 after the previous kernel has completed, adds its arrival (atomic), and then:
-the arrival that brings the count to the grid size G stores (epoch + 1,
-count 0); every other CTA waits, with a time limit, until the epoch differs
-from the one it read, or gives up (timeout). This model runs that protocol
+the arrival that brings the count to the grid size G then stores (epoch + 1,
+count 0); every other CTA waits, with a time limit, until it sees the count at
+G or an epoch that differs from the one it read, or gives up (timeout). This model runs that protocol
 step by step with random interleavings, CTAs that start only after others
 have already given up, and random time limits, and checks that
 
@@ -34,7 +34,8 @@ def run_call(h, G, rng, limit=None, late=()):
     """One call of G CTAs; those in 'late' start only after the others have
     run for a while (each of them passed, gave up or is still waiting).
     Returns the sets of CTAs that passed and that gave up."""
-    # per CTA: program counter 0 read epoch, 1 arrive, 2 wait, 3 done
+    # per CTA: program counter 0 read epoch, 1 arrive, 2 wait, 3 done, 4 (the
+    # last arrival only) store the new epoch and reset the count
     pc = [0] * G
     e0 = [None] * G
     waited = [0] * G
@@ -52,14 +53,16 @@ def run_call(h, G, rng, limit=None, late=()):
             h.arrive = (h.arrive + 1) & MASK
             arrived.add(c)
             if ticket == G - 1:
-                h.arrive, h.epoch = 0, (e0[c] + 1) & MASK
                 passed.add(c)
                 passed_after_all.add(len(arrived) == G)
-                pc[c] = 3
+                pc[c] = 4
             else:
                 pc[c] = 2
+        elif pc[c] == 4:
+            h.arrive, h.epoch = 0, (e0[c] + 1) & MASK
+            pc[c] = 3
         elif pc[c] == 2:
-            if h.epoch != e0[c]:
+            if h.epoch != e0[c] or h.arrive >= G:
                 passed.add(c)
                 passed_after_all.add(len(arrived) == G)
                 pc[c] = 3
