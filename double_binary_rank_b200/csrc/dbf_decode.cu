@@ -1,4 +1,6 @@
-// Decode-regime forward in one launch.
+// Decode-regime forward in one launch, for calls of one layer whose
+// (token, envelope) columns number at most eight (the decode step itself);
+// longer calls and segmented adapters take dbf_decode_multi.cu.
 //
 // LoRDBA page, section 2 ("Kernel de Inferencia"): the forward is two
 // sign-accumulation products with per-channel scaling between them; DBF page,
@@ -42,8 +44,8 @@
 // in the high word). A CTA reads the epoch, then adds its arrival with an
 // acquire-release atomic; the arrival that brings the count to the grid size
 // stores (epoch + 1, count 0) with release semantics, and every other CTA
-// waits (acquire loads, bounded by a time limit) until it sees the full count
-// or the new epoch. The epoch can change only after every CTA has arrived, so
+// polls (bounded by a time limit counted from the CTA's entry) until it sees
+// the full count or the new epoch. The epoch can change only after every CTA has arrived, so
 // a CTA that starts late still reads the current epoch; the count is zero
 // again once the last CTA has arrived, whatever happened to the waits. A wait that runs out of
 // time stores DBF_ERR_TIMEOUT in the header's status word and the CTA skips
@@ -64,8 +66,6 @@ constexpr int kMaxWordsPerWarp = 32;     // M <= 8192
 constexpr int kSmemCap = 227 * 1024;
 constexpr int kMaxGrid = 160;            // CTAs at most (sizes the per-CTA sums in the workspace)
 constexpr unsigned long long kDefaultWaitNs = 2000000000ull;   // 2 s
-
-unsigned long long g_wait_ns = 0;   // 0: the default limit
 
 struct DecodeParams {
     dbf_layer L;
@@ -95,12 +95,14 @@ struct DecodeParams {
 
 struct Misc {
     uint64_t bar[5];              // slice 1, slice 2, gamma, x buffers 0 and 1 arrived
+    unsigned long long t_entry;   // %globaltimer at the CTA's entry
     int flag;
     unsigned e0;                  // epoch read at entry
     unsigned bmax;                // max |beta| (fp32 bits)
     unsigned amax[kMaxCols];      // max |gamma . x| per column (fp32 bits)
     int sh_u[kMaxCols], sh_v[kMaxCols];
-    long long qsum_u[kMaxCols], qabs_u[kMaxCols], qsum_v[kMaxCols], qpart_v[kMaxCols];
+    long long qsum_u[kMaxCols], qabs_u[kMaxCols], qsum_v[kMaxCols];
+    long long wq[kWarps][kMaxCols], wa[kWarps][kMaxCols];   // per-warp partial sums
 };
 
 // ---- small device helpers ----------------------------------------------------
@@ -275,6 +277,15 @@ __device__ __forceinline__ long long warp_sum64(long long v)
     return v;
 }
 
+// Exact warp sum of per-thread int32 values: 16-bit halves summed separately
+// (one reduction instruction each).
+__device__ __forceinline__ long long warp_sum_exact(int v)
+{
+    const unsigned lo = __reduce_add_sync(0xffffffffu, static_cast<unsigned>(v) & 0xFFFFu);
+    const int hi = __reduce_add_sync(0xffffffffu, v >> 16);
+    return static_cast<long long>(hi) * 65536 + lo;
+}
+
 // Copy rows [0, n) of a packed matrix slice into shared memory with row
 // stride 'stride': bulk copies issued by one warp (one copy when unpadded).
 __device__ __forceinline__ void slice_bulk(uint32_t *dst, const uint32_t *src, int n, int pitch, int stride,
@@ -324,7 +335,8 @@ __device__ bool grid_sync(const DecodeParams &P, Misc *ms)
     __syncthreads();
     if (threadIdx.x == 0) {
         bool ok = true;
-        __threadfence();
+        // the release half of the arrival covers the CTA's writes, ordered
+        // before it by the barrier above
         unsigned ticket;
         asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;"
                      : "=r"(ticket)
@@ -335,18 +347,20 @@ __device__ bool grid_sync(const DecodeParams &P, Misc *ms)
             asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(P.sync), "l"(next) : "memory");
         } else {
             // every CTA has arrived once the count reaches the grid size (seen
-            // before the last arrival resets it) or the epoch has moved on
-            const unsigned long long t0 = global_ns();
+            // before the last arrival resets it) or the epoch has moved on;
+            // relaxed polls, then one acquire fence. The limit counts from
+            // the CTA's entry and is checked before each poll.
             while (true) {
-                unsigned long long v;
-                asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(P.sync) : "memory");
-                if (static_cast<unsigned>(v >> 32) != ms->e0 || static_cast<unsigned>(v) >= gridDim.x) break;
-                if (global_ns() - t0 > P.wait_ns) {
+                if (global_ns() - ms->t_entry > P.wait_ns) {
                     ok = false;
                     atomicExch(P.status, static_cast<int32_t>(DBF_ERR_TIMEOUT));
                     break;
                 }
+                unsigned long long v;
+                asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(P.sync) : "memory");
+                if (static_cast<unsigned>(v >> 32) != ms->e0 || static_cast<unsigned>(v) >= gridDim.x) break;
             }
+            asm volatile("fence.acq_rel.gpu;" ::: "memory");
         }
         ms->flag = ok ? 1 : 0;
     }
@@ -456,12 +470,10 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const __grid_consta
 
     if (tid < kMaxCols) {
         ms->amax[tid] = 0u;
-        ms->qsum_u[tid] = 0;
-        ms->qabs_u[tid] = 0;
         ms->qsum_v[tid] = 0;
-        ms->qpart_v[tid] = 0;
     }
     if (tid == 0) {
+        ms->t_entry = global_ns();
         for (int i = 0; i < 5; ++i) bar_init(&ms->bar[i], 1);
         ms->bmax = 0u;
     }
@@ -626,10 +638,11 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const __grid_consta
                 d0[2 * P.cb1 + off] = static_cast<char>(d0b >> 16);
                 d0[2 * P.cb1 + off + 2] = static_cast<char>(d1b >> 16);
             }
-            const long long sq64 = warp_sum64(sq), sa64 = warp_sum64(sa);
+            // per-warp partial sums through shared memory (no 64-bit shared atomics)
+            const long long sq64 = warp_sum_exact(sq), sa64 = warp_sum_exact(sa);
             if (lane == 0) {
-                atomicAdd(reinterpret_cast<unsigned long long *>(&ms->qsum_u[c]), static_cast<unsigned long long>(sq64));
-                atomicAdd(reinterpret_cast<unsigned long long *>(&ms->qabs_u[c]), static_cast<unsigned long long>(sa64));
+                ms->wq[warp][c] = sq64;
+                ms->wa[warp][c] = sa64;
             }
             if (tid == 0) ms->sh_u[c] = sh;
         }
@@ -652,25 +665,31 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const __grid_consta
     slice_pad(s2, n2, rows2, P.pitch2, P.stride2);
     if (!P.bulk2) slice_plain(s2, L.b1_packed + static_cast<int64_t>(lo2) * P.pitch2, n2, P.pitch2, P.stride2);
     if (tid < C) {
+        long long sq = 0, sa = 0;
+        for (int w = 0; w < kWarps; ++w) {
+            sq += ms->wq[w][tid];
+            sa += ms->wa[w][tid];
+        }
+        ms->qsum_u[tid] = sq;
+        ms->qabs_u[tid] = sa;
         // |v_r| = |beta_r h_r| <= max|beta| sum|q| 2^-sh; the factor covers the
         // fp32 roundings of h and of beta h
-        const float bound = __uint_as_float(ms->bmax) * scale_pow2(static_cast<float>(ms->qabs_u[tid]), -ms->sh_u[tid]) *
+        const float bound = __uint_as_float(ms->bmax) * scale_pow2(static_cast<float>(sa), -ms->sh_u[tid]) *
                             (1.0f + 1.0f / 1024.0f);
         ms->sh_v[tid] = scale_exponent(bound);
     }
 
     // ---- stage 1: h = B2 u for the CTA's row blocks, then v = beta . h as digits into the image
+    // (one (row, column) per thread and step; each thread's sums of q of v per
+    // column are reduced per warp and summed through shared memory)
+    int qv[kMaxCols];
+#pragma unroll
+    for (int c = 0; c < kMaxCols; ++c) qv[c] = 0;
     if (do1) {
         const bool ok1 = P.bulk1 ? slice_wait(&ms->bar[0], P, ms) : true;
         if (ok1) {
             sign_sums(s1, P.stride1, rows1 / 16, P.ng1, dig, P.cb1, ndcol, tile, P.tile_ld);
             __syncthreads();
-            // one (row, column) per thread and step; each thread's sums of q of v
-            // per column (at most two elements: int32) are reduced per warp and
-            // added to shared memory
-            int qv[kMaxCols];
-#pragma unroll
-            for (int c = 0; c < kMaxCols; ++c) qv[c] = 0;
 #pragma unroll 1
             for (int i = tid; i < n1 * C; i += kThreads) {
                 const int c = i / n1, lr = i - c * n1;
@@ -687,14 +706,6 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const __grid_consta
                 for (int cc = 0; cc < kMaxCols; ++cc)
                     if (cc == c) qv[cc] += q;
             }
-#pragma unroll
-            for (int c = 0; c < kMaxCols; ++c) {
-                if (c < C) {
-                    const int w = __reduce_add_sync(0xffffffffu, qv[c]);
-                    if (lane == 0 && w) atomicAdd(reinterpret_cast<unsigned long long *>(&ms->qpart_v[c]),
-                                                  static_cast<unsigned long long>(static_cast<long long>(w)));
-                }
-            }
         }
     }
     // digits of v past the rank, up to the last 256-column group, are zero
@@ -709,8 +720,20 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const __grid_consta
             im[2 * P.cb2] = 0;
         }
     }
+    __syncthreads();   // the digit build's partial sums have been read
+#pragma unroll
+    for (int c = 0; c < kMaxCols; ++c) {
+        if (c < C) {
+            const long long w = warp_sum_exact(qv[c]);
+            if (lane == 0) ms->wq[warp][c] = w;
+        }
+    }
     __syncthreads();
-    if (tid < C) P.qpart[static_cast<int64_t>(b) * C + tid] = ms->qpart_v[tid];
+    if (tid < C) {
+        long long sum = 0;
+        for (int w = 0; w < kWarps; ++w) sum += ms->wq[w][tid];
+        P.qpart[static_cast<int64_t>(b) * C + tid] = sum;
+    }
 
     // ---- every CTA's digits of v and its sums are written
     const bool passed = grid_sync(P, ms);
@@ -902,7 +925,7 @@ cudaError_t decode_forward(const dbf_layer &L, const void *x, dbf_dtype xd, void
     P.status = reinterpret_cast<int32_t *>(w + kWsStatusOffset);
     P.img = w + kWsHeaderBytes;
     P.qpart = reinterpret_cast<long long *>(w + kWsHeaderBytes + img_bytes(P.C, P.ng2));
-    P.wait_ns = g_wait_ns ? g_wait_ns : kDefaultWaitNs;
+    P.wait_ns = decode_wait_ns();
     // staged inputs by bulk copies when whole 16-byte units (x is 16-byte
     // aligned by the call's contract; gamma only 2-byte)
     P.bulk_x = (static_cast<size_t>(L.M) * (xd == DBF_BF16 ? 2 : 4)) % 16 == 0;
@@ -952,7 +975,5 @@ cudaError_t decode_forward(const dbf_layer &L, const void *x, dbf_dtype xd, void
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
-
-void set_decode_wait_ns(unsigned long long ns) { g_wait_ns = ns; }
 
 }  // namespace dbf

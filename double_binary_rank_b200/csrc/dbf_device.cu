@@ -1,10 +1,11 @@
-// Per-device launch state shared by the launchers: the current device's SM
-// count and the one-time kernel attributes (dynamic shared-memory limit,
-// carve-out). Both are properties of a device, so they are kept per device
+// Launch state shared by the launchers: the current device's SM count, the
+// one-time kernel attributes (dynamic shared-memory limit, carve-out), and
+// the grid-barrier time limit of the decode kernels. Both are properties of a device, so they are kept per device
 // (a process may drive several GPUs, one host thread each), looked up under
 // a lock and cached after the first call on each device.
 #include "dbf_internal.cuh"
 
+#include <atomic>
 #include <map>
 #include <mutex>
 #include <utility>
@@ -25,7 +26,18 @@ int current_device()
     return dev;
 }
 
+std::atomic<unsigned long long> g_decode_wait_ns{0};   // 0: the default limit
+constexpr unsigned long long kDecodeDefaultWaitNs = 2000000000ull;   // 2 s
+
 }  // namespace
+
+unsigned long long decode_wait_ns()
+{
+    const unsigned long long v = g_decode_wait_ns.load(std::memory_order_relaxed);
+    return v ? v : kDecodeDefaultWaitNs;
+}
+
+void set_decode_wait_ns(unsigned long long ns) { g_decode_wait_ns.store(ns, std::memory_order_relaxed); }
 
 int device_sms()
 {

@@ -1,7 +1,7 @@
 // Decode-regime forward in two launches: two sign-accumulation GEMVs with
-// per-channel scaling, for the calls the single-launch kernel (dbf_decode.cu)
-// does not take -- more than eight (token, envelope) columns, M or R above
-// 8192 -- and for segmented multi-adapter serving.
+// per-channel scaling, for the calls neither single-launch kernel
+// (dbf_decode.cu, dbf_decode_multi.cu) takes: M above 8192, more than 512
+// segments, or no plan that fits in shared memory.
 //
 // LoRDBA page, section 2 ("Kernel de Inferencia"): the forward is two
 // sign-accumulation matrix products interleaved with per-channel scaling;
@@ -35,6 +35,8 @@
 // and with static weights starts its sign copy before the previous kernel
 // has finished; every other read and every write waits for it.
 #include "dbf_internal.cuh"
+
+#include <algorithm>
 
 namespace dbf {
 namespace {
@@ -892,21 +894,29 @@ cudaError_t run_both(GemvParams P, int M, int max_R, int N, int nseg, int budget
 
 }  // namespace
 
-size_t gemv_workspace_bytes(int64_t R, int64_t ell, int64_t T) { return kWsHeaderBytes + ws_layout(R, ell, T).total; }
+size_t gemv_workspace_bytes(int64_t R, int64_t ell, int64_t T)
+{
+    // either kernel: the two launches here or the single launch
+    const size_t a = kWsHeaderBytes + ws_layout(R, ell, T).total;
+    const size_t b = multi_segmented_workspace_bytes(static_cast<int32_t>(R), static_cast<int32_t>(ell), T);
+    return a > b ? a : b;
+}
 
 size_t gemv_layer_workspace_bytes(const dbf_layer &L, int64_t T)
 {
     const size_t a = gemv_workspace_bytes(L.R, L.ell, T), b = decode_workspace_bytes(L, T);
-    return a > b ? a : b;
+    const size_t c = multi_workspace_bytes(L, T);
+    return std::max(a, std::max(b, c));
 }
 
-int gemv_launches(const dbf_layer &L, int64_t T) { return decode_fits(L, T) ? 1 : 2; }
+int gemv_launches(const dbf_layer &L, int64_t T) { return (decode_fits(L, T) || multi_fits(L, T)) ? 1 : 2; }
 
 cudaError_t gemv_forward(const dbf_layer &L, const void *x, dbf_dtype xd, void *y, dbf_dtype yd, int64_t T,
                          int flags, void *ws, cudaStream_t s)
 {
-    // one launch (binary tensor-core products, grid barrier) when the call fits it
+    // one launch (grid barrier) when the call fits one of the single-launch kernels
     if (decode_fits(L, T)) return decode_forward(L, x, xd, y, yd, T, flags, ws, s);
+    if (multi_fits(L, T)) return multi_forward(L, x, xd, y, yd, T, flags, ws, s);
     GemvParams P{};
     P.layer = L;
     P.M = L.M;
@@ -929,6 +939,10 @@ cudaError_t gemv_forward_segmented(const dbf_layer *adapters, int32_t num_adapte
                                    int32_t N, const void *x, dbf_dtype xd, void *y, dbf_dtype yd, int64_t T,
                                    int flags, void *ws, int32_t *status, cudaStream_t s)
 {
+    // one launch when the call fits it
+    if (multi_segmented_fits(S, max_R, max_ell, M, N, T))
+        return multi_forward_segmented(adapters, num_adapters, seg_off, seg_adp, S, max_R, max_ell, M, N, x, xd, y,
+                                       yd, T, flags, ws, status, s);
     GemvParams P{};
     P.adapters = adapters;
     P.num_adapters = num_adapters;

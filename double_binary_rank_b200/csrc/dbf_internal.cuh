@@ -46,13 +46,27 @@ cudaError_t launch_transpose(const uint32_t *src, int64_t rows, int64_t k, uint3
 cudaError_t launch_ste(const float *db, const void *h, dbf_dtype hd, int64_t n, float tau, float *dh,
                        int accumulate, cudaStream_t s);
 
-// single-launch decode (binary tensor-core products, dbf_decode.cu): calls with
-// T * ell <= 8 and M, R <= 8192
+// single-launch decode kernels (integer tensor-core products): dbf_decode.cu
+// for one layer with at most eight (token, envelope) columns, and
+// dbf_decode_multi.cu for more columns and for segmented adapters (M <= 8192,
+// at most 512 segments); *_fits says whether a call takes that kernel
 bool decode_fits(const dbf_layer &L, int64_t T);
 size_t decode_workspace_bytes(const dbf_layer &L, int64_t T);
 cudaError_t decode_forward(const dbf_layer &L, const void *x, dbf_dtype xd, void *y, dbf_dtype yd, int64_t T,
                            int flags, void *ws, cudaStream_t s);
-// limit of the decode kernel's bounded waits for later calls (0: the default, 2 s)
+bool multi_fits(const dbf_layer &L, int64_t T);
+size_t multi_workspace_bytes(const dbf_layer &L, int64_t T);
+cudaError_t multi_forward(const dbf_layer &L, const void *x, dbf_dtype xd, void *y, dbf_dtype yd, int64_t T,
+                          int flags, void *ws, cudaStream_t s);
+bool multi_segmented_fits(int32_t S, int32_t max_R, int32_t max_ell, int32_t M, int32_t N, int64_t T);
+size_t multi_segmented_workspace_bytes(int32_t max_R, int32_t max_ell, int64_t T);
+cudaError_t multi_forward_segmented(const dbf_layer *adapters, int32_t num_adapters, const int32_t *seg_off,
+                                    const int32_t *seg_adp, int32_t S, int32_t max_R, int32_t max_ell, int32_t M,
+                                    int32_t N, const void *x, dbf_dtype xd, void *y, dbf_dtype yd, int64_t T,
+                                    int flags, void *ws, int32_t *status, cudaStream_t s);
+// limit of the decode kernels' grid-barrier wait (dbf_device.cu): the value
+// for launches, and the setting for later calls (0: the default, 2 s)
+unsigned long long decode_wait_ns();
 void set_decode_wait_ns(unsigned long long ns);
 
 // decode path

@@ -406,10 +406,11 @@ dbf_status dbf_forward_decode_noalloc(const dbf_layer *L, const void *x, dbf_dty
                                       dbf_dtype y_dtype, int64_t T, int flags, void *stream);
 
 /* Time limit of the grid-barrier wait of the single-launch decode kernel
- * for the calls made after this one, in this process: ns > 0 sets it, 0
- * restores the default of 2 s (its waits for its own weight copies always
- * keep the default). For tests of the timeout path: with a limit shorter than
- * the time the CTAs take to arrive, the waiting CTAs give up, store
+ * for the calls made after this one, in this process, counted from each
+ * CTA's start and checked before every poll: ns > 0 sets it, 0 restores the
+ * default of 2 s (its waits for its own weight copies always keep the
+ * default). For tests of the timeout path: with a limit shorter than the time
+ * a CTA takes to reach the barrier, every CTA but the last to arrive gives up, stores
  * DBF_ERR_TIMEOUT in the workspace status word and skip their share of stage
  * 2 (y is left incomplete); the workspace stays usable, and a later call with
  * the default limit is correct. Not for production use; not synchronised with

@@ -116,22 +116,20 @@ def test_segmented_rejects_bad_arguments(lib):
 
 def test_forward_launch_count(lib):
     # host-side query, no launch: GEMM path = pre-pass + two stages; GEMV path
-    # = one kernel while T * ell <= 8, M <= 8192 and its shared memory fits
-    # (on this layer the digits of v take 17.8 KB per column: up to 7
-    # columns), else two
+    # = one kernel whenever M <= 8192 (any token count: the columns are cut
+    # into chunks), else two
     import double_binary_rank_b200 as dbf
     by = ctypes.byref
     L = _layer(M=4096, N=11008, R=5888, ell=1)
     assert lib.dbf_forward_launches(by(L), 2048, dbf.PATH_AUTO) == 3
     assert lib.dbf_forward_launches(by(L), 1, dbf.PATH_AUTO) == 1
-    assert lib.dbf_forward_launches(by(L), 7, dbf.PATH_GEMV) == 1
-    assert lib.dbf_forward_launches(by(L), 8, dbf.PATH_GEMV) == 2
+    for T in (7, 8, 64, 2048):
+        assert lib.dbf_forward_launches(by(L), T, dbf.PATH_GEMV) == 1
     L1 = _layer(M=4096, N=4096, R=64, ell=1)
-    assert lib.dbf_forward_launches(by(L1), 8, dbf.PATH_GEMV) == 1
-    assert lib.dbf_forward_launches(by(L1), 9, dbf.PATH_GEMV) == 2
+    for T in (8, 9, 64):
+        assert lib.dbf_forward_launches(by(L1), T, dbf.PATH_GEMV) == 1
     L2 = _layer(M=256, N=256, R=16, ell=3)
-    assert lib.dbf_forward_launches(by(L2), 2, dbf.PATH_GEMV) == 1
-    assert lib.dbf_forward_launches(by(L2), 3, dbf.PATH_GEMV) == 2
+    assert lib.dbf_forward_launches(by(L2), 3, dbf.PATH_GEMV) == 1
     L3 = _layer(M=8224, N=256, R=96, ell=1)   # M above 8192
     assert lib.dbf_forward_launches(by(L3), 1, dbf.PATH_GEMV) == 2
     assert lib.dbf_forward_launches(by(L), 0, dbf.PATH_AUTO) == 0

@@ -6,7 +6,8 @@ The kernel's barrier word (workspace header, 8 bytes) holds an arrival count
 after the previous kernel has completed, adds its arrival (atomic), and then:
 the arrival that brings the count to the grid size G then stores (epoch + 1,
 count 0); every other CTA waits, with a time limit, until it sees the count at
-G or an epoch that differs from the one it read, or gives up (timeout). This model runs that protocol
+G or an epoch that differs from the one it read, or gives up (the time
+limit is checked before each poll). This model runs that protocol
 step by step with random interleavings, CTAs that start only after others
 have already given up, and random time limits, and checks that
 
@@ -62,15 +63,16 @@ def run_call(h, G, rng, limit=None, late=()):
             h.arrive, h.epoch = 0, (e0[c] + 1) & MASK
             pc[c] = 3
         elif pc[c] == 2:
-            if h.epoch != e0[c] or h.arrive >= G:
+            # the time limit is checked before each poll
+            if limit is not None and waited[c] >= limit:
+                timed_out.add(c)
+                pc[c] = 3
+            elif h.epoch != e0[c] or h.arrive >= G:
                 passed.add(c)
                 passed_after_all.add(len(arrived) == G)
                 pc[c] = 3
             else:
                 waited[c] += 1
-                if limit is not None and waited[c] > limit:
-                    timed_out.add(c)
-                    pc[c] = 3
 
     # the early CTAs run interleaved for a while (each passes, gives up or is
     # still waiting), then the late ones start and everything runs interleaved

@@ -1,5 +1,5 @@
-"""The single-launch decode path (T * ell <= 8, M and R <= 8192) against
-the fp64 oracle.
+"""The single-launch decode path (one layer or segmented adapters, M <=
+8192) against the fp64 oracle.
 
 That path exchanges the rank-R intermediate through a grid-wide barrier
 whose word lives in the workspace header (arrival count in the low 32 bits,
@@ -7,8 +7,10 @@ epoch in the high 32 bits), so besides plain parity these tests check that
 many calls sharing one workspace (with different grid sizes) stay correct,
 that every call leaves the arrival count at zero and advances the epoch by
 one, that a barrier wait that runs out of time is reported in the header's
-status word and leaves the workspace usable, and the size limits where the
-library switches to the two-launch path.
+status word and leaves the workspace usable, the chunking of many tokens
+(ragged last chunks, several items per CTA), segments of adapters with
+different ranks and envelope counts, and the limits where the library
+switches to the two-launch path (M above 8192, more than 512 segments).
 """
 import numpy as np
 import pytest
@@ -34,8 +36,8 @@ def header_words(ws):
 
 
 @pytest.mark.parametrize("T,ell", [(8, 1), (4, 2), (1, 8), (2, 3), (9, 1), (3, 3)])
-def test_column_limit(dbf, T, ell):
-    # T * ell <= 8 runs in one launch, above it in two; both must match
+def test_token_envelope_mix(dbf, T, ell):
+    # chunks of whole tokens with up to eight (token, envelope) columns
     rng = np.random.default_rng(700 + 10 * T + ell)
     L = random_layer(rng, 512, 384, 160, ell)
     x = S.to_bf16_bits(rng.standard_normal((T, 512)))
@@ -150,3 +152,57 @@ def test_dbf_mlp_decode_repeat_bit_identical(dbf):
         assert np.array_equal(host_y(y), first)
     ref = oracle.forward(L, S.make_x(w.seed, 1, w.M, "bf16"))
     assert rel_err(first, ref) < 1e-4
+
+
+@pytest.mark.parametrize("M,N,R,ell,T", [(320, 200, 70, 3, 37), (256, 160, 128, 2, 300), (1000, 33, 7, 1, 129),
+                                          (4096, 4096, 64, 1, 64)])
+def test_many_tokens(dbf, M, N, R, ell, T):
+    # many chunks (ragged last chunk), several items per CTA with slice reloads
+    rng = np.random.default_rng(750 + T)
+    L = random_layer(rng, M, N, R, ell)
+    x = S.to_bf16_bits(rng.standard_normal((T, M)))
+    rows = None if M * N * R * T < 4e9 else list(range(0, T, 7)) + [T - 1]
+    ref = oracle.forward(L, x, rows=rows)
+    got = host_y(dbf.forward(dev_layer(L), dev_x(x), path="gemv", y_dtype=torch.float32))
+    assert rel_err(got if rows is None else got[rows], ref) < 1e-4
+
+
+def test_dbf_mlp_many_tokens_sampled(dbf):
+    # the DBF MLP layer through the decode kernel at 24 tokens (several chunks
+    # over the long rank), checked on sampled rows
+    w = S.WORKLOADS["dbf_mlp"]
+    L = S.workload_layers(w)[0]
+    x = S.make_x(w.seed + 7, 24, w.M, "bf16")
+    rows = [0, 5, 11, 17, 23]
+    ref = oracle.forward(L, x, rows=rows)
+    got = host_y(dbf.forward(dev_layer(L), dev_x(x), path="gemv", y_dtype=torch.float32))
+    assert rel_err(got[rows], ref) < 1e-4
+
+
+def i32(a):
+    return torch.tensor(np.asarray(a, dtype=np.int32), device="cuda")
+
+
+@pytest.mark.parametrize("S_", [40, 600])
+def test_segmented_mixed_adapters(dbf, S_):
+    # adapters of different ranks (below the largest) and envelope counts,
+    # segments of 0..9 tokens, some without an adapter; 600 segments take the
+    # two-launch path
+    rng = np.random.default_rng(760 + S_)
+    M, N = 288, 136
+    shapes = [(33, 1), (96, 2), (7, 3), (128, 1)]
+    layers = [random_layer(rng, M, N, R, ell) for R, ell in shapes]
+    counts = rng.integers(0, 10, size=S_)
+    if S_ > 100:
+        counts = np.minimum(counts, 1)
+    offsets = np.concatenate([[0], np.cumsum(counts)]).astype(np.int64)
+    T = int(offsets[-1])
+    adapter = rng.integers(-1, len(layers), size=S_)
+    x = S.to_bf16_bits(rng.standard_normal((T, M)))
+    ref = oracle.forward_segmented(layers, offsets, adapter, x)
+    table = dbf.AdapterTable([dev_layer(L) for L in layers], "cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    y = dbf.forward_segmented(table, i32(offsets), i32(adapter), dev_x(x), y_dtype=torch.float32, status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    assert rel_err(host_y(y), ref) < 1e-4

@@ -32,9 +32,8 @@ def test_noalloc_matches_forward_twice():
     w = S.WORKLOADS["dbf_mlp"]
     L = S.workload_layers(w)[0]
     dl = dev_layer(L)
-    # T = 1, 2: single-launch kernel; T = 16: the two-launch path through the
-    # same array; then single launches again, which also shows that the
-    # array's barrier word was left consistent by the earlier calls
+    # T = 1, 2, 16: the single-launch kernel (several calls sharing the
+    # array's barrier word)
     for call, T in enumerate((1, 2, 16, 1, 2)):
         xh = S.make_x(w.seed + call, T, w.M, "bf16")
         x = dev_x(xh)
@@ -46,6 +45,16 @@ def test_noalloc_matches_forward_twice():
         got = host_y(y)
         assert rel_err(got, host_y(ref)) < TOL
         assert rel_err(got, oracle.forward(L, xh)) < TOL
+    # a layer wider than the single launch takes (M > 8192): the two-launch
+    # path through the same array, then a single launch again
+    Lw = random_layer(rng, 8224, 256, 96, 1)
+    dw = dev_layer(Lw)
+    xwh = S.to_bf16_bits(rng.standard_normal((2, 8224)))
+    yw = torch.zeros((2, 256), device="cuda")
+    assert dbf._lib.dbf_forward_launches(ctypes.byref(dw.descriptor()), 2, dbf.PATH_GEMV) == 2
+    assert _call_noalloc(dbf, dw, dev_x(xwh), yw) == dbf.OK
+    torch.cuda.synchronize()
+    assert rel_err(host_y(yw), oracle.forward(Lw, xwh)) < TOL
     # a second layer shape right after, through the same array
     L2 = random_layer(rng, 300, 170, 96, 2)
     d2 = dev_layer(L2)
