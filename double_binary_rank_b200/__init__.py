@@ -59,7 +59,7 @@ _SIGS = {
     "dbf_factorize_workspace_bytes": (_sz, [_i64, _i64, _i64, _i32, _i32]),
     "dbf_factorize": (ctypes.c_int, [_vp, _i64, _i64, _i64, _vp, _vp, _i32, _i32, _i32, ctypes.c_float, _vp, _vp,
                                      _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
-    "dbf_gemm_min_tokens": (_i64, []),
+    "dbf_gemm_min_tokens": (_i64, [ctypes.c_void_p]),
     "dbf_workspace_bytes": (_sz, [_LP, _i64, ctypes.c_int]),
     "dbf_forward_launches": (_i32, [_LP, _i64, ctypes.c_int]),
     "dbf_forward": (ctypes.c_int, [_LP, _vp, ctypes.c_int, _vp, ctypes.c_int, _i64, ctypes.c_int,
@@ -124,8 +124,11 @@ def packed_bytes(rows: int, k: int) -> int:
     return int(_lib.dbf_packed_bytes(rows, k))
 
 
-def gemm_min_tokens() -> int:
-    return int(_lib.dbf_gemm_min_tokens())
+def gemm_min_tokens(layer) -> int:
+    """Smallest T at which the AUTO path takes the GEMM kernels on this layer
+    (-1: never)."""
+    d = layer.descriptor()
+    return int(_lib.dbf_gemm_min_tokens(ctypes.byref(d)))
 
 
 def pack_signs(src: torch.Tensor, out: Optional[torch.Tensor] = None,

@@ -9,7 +9,6 @@ namespace {
 
 using namespace dbf;
 
-constexpr int64_t kGemmMinTokens = 128;
 
 bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
@@ -30,10 +29,27 @@ dbf_status check_layer(const dbf_layer *L)
     return DBF_OK;
 }
 
+// Smallest T at which the tcgen05 GEMM path beats the decode kernels on
+// this shape (INT64_MAX if it never does or the shape cannot take it), from
+// two linear time models fit to B200 sweeps over T on four shapes:
+//   decode:  15 us + 8.4e-8 us per sign-MAC of the call, T ell R (M + N);
+//   GEMM:    65 us + 4.5e-7 us per packed sign bit R (M + N) (the expansion
+//            of the weights into tiles) + the flops 2 T ell R (M + N) at
+//            0.9 PFLOP/s.
+int64_t gemm_min_tokens(const dbf_layer &L)
+{
+    if (!gemm_shape_ok(L)) return INT64_MAX;
+    const double w = static_cast<double>(L.R) * (static_cast<double>(L.M) + L.N);
+    const double per_tok_gemv = 8.4e-8 * L.ell * w, per_tok_gemm = 2.0 * L.ell * w / 9e8;
+    if (per_tok_gemv <= per_tok_gemm) return INT64_MAX;
+    const double t = (65.0 - 15.0 + 4.5e-7 * w) / (per_tok_gemv - per_tok_gemm);
+    return t >= 9.0e18 ? INT64_MAX : static_cast<int64_t>(std::ceil(t));
+}
+
 // The path dbf_forward takes; DBF_PATH_GEMM only when the shape allows it.
 dbf_path resolve(const dbf_layer &L, int64_t T, dbf_path p)
 {
-    if (p == DBF_PATH_AUTO) return (gemm_shape_ok(L) && T >= kGemmMinTokens) ? DBF_PATH_GEMM : DBF_PATH_GEMV;
+    if (p == DBF_PATH_AUTO) return T >= gemm_min_tokens(L) ? DBF_PATH_GEMM : DBF_PATH_GEMV;
     return p;
 }
 
@@ -145,7 +161,12 @@ dbf_status dbf_factorize(const float *W, int64_t n, int64_t m, int64_t k, const 
                                    alpha, beta, gamma, objective, ws, static_cast<cudaStream_t>(stream)));
 }
 
-int64_t dbf_gemm_min_tokens(void) { return kGemmMinTokens; }
+int64_t dbf_gemm_min_tokens(const dbf_layer *L)
+{
+    if (!L || L->M <= 0 || L->N <= 0 || L->R <= 0 || L->ell < 1 || L->ell > kMaxEll) return -1;
+    const int64_t t = gemm_min_tokens(*L);
+    return t == INT64_MAX ? -1 : t;
+}
 
 void dbf_debug_set_decode_wait_ns(uint64_t ns) { set_decode_wait_ns(ns); }
 

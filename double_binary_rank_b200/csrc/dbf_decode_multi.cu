@@ -70,14 +70,12 @@
 namespace dbf {
 namespace {
 
-constexpr int kThreads = 512;
+constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
 constexpr int kDigits = 3;               // int8 digits per activation value
 constexpr int kChunkCols = 8;            // (token, envelope) columns per chunk at most
 constexpr int kGroupWords = 8;           // packed words per MMA unit (256 columns of K)
-constexpr int kMaxGroups = 3;            // MMA column groups (8 digit columns) per chunk
 constexpr int kMaxM = 8192;              // inputs at most (digit-build registers)
-constexpr int kUnitsPerThread = kMaxM / 4 / kThreads;   // (word, bit) units of the digit build
 constexpr int kSmemCap = 227 * 1024;
 constexpr int kMaxGrid = 160;
 constexpr int kMaxSegments = 512;        // segments of one call (shared-memory chunk table)
@@ -109,7 +107,8 @@ struct DecodeParams {
     int rows1, rows2;             // rows of an item at most (multiples of 16)
     int tile_ld;                  // int32 per tile row (8 per MMA column group)
     int gpitch, gs_bytes, xs_bytes;   // staged gamma (values per row, bytes) and one token's x buffer
-    int stage_g;                  // gamma staged in shared memory (else read from global memory)
+    int stage_g;                  // gamma staged in shared memory (else read from global memory: no room)
+    int word2;                    // stage 2 in the per-word layout (small ranks, see digit_offset_word)
     int off_s2, off_dig, off_tile, off_misc, off_rs1, off_rs2, off_seg;   // shared-memory offsets
     unsigned long long wait_ns;   // limit of the grid-barrier wait
 };
@@ -184,7 +183,7 @@ __device__ __forceinline__ bool bar_try(uint64_t *bar, uint32_t parity)
 // Thread 0 polls, bounded by the default limit whatever the grid barrier's
 // limit is (no copy is cut short); a timeout is recorded in the status word
 // and the CTA carries on.
-__device__ __forceinline__ void copy_wait(uint64_t *bar, uint32_t parity, int32_t *status)
+__device__ __noinline__ void copy_wait(uint64_t *bar, uint32_t parity, int32_t *status)
 {
     __syncthreads();
     if (threadIdx.x == 0) {
@@ -317,13 +316,40 @@ __host__ __device__ inline int slice_stride(int pitch)
 // warp, columns g = 0..3 and threads t = 0..3, then cover the 32 banks once).
 __host__ __device__ inline int col_bytes(int pitch) { return groups_of(pitch) * 256 + 32; }
 
+// Stage 2 of small ranks (at most four packed words per row of B1) uses a
+// per-word layout instead of whole groups, so that no MMA runs on padding:
+// one MMA per packed word, MMA thread t taking bits t + 8i of the word for
+// its first four K slots and bits t + 4 + 8i for its other four
+// ((word >> t) & 0x01010101 and (word >> (t + 4)) & 0x01010101, bytes in
+// {0, 1}); the digits of unit (word w, bit j) sit at
+// w * 32 + (j % 4) * 8 + (j / 4) * 4, thread t's eight bytes at w * 32 + 8t.
+constexpr int kWordPitchMax = 4;
+__host__ __device__ inline bool word_layout(int pitch) { return pitch <= kWordPitchMax; }
+__device__ __forceinline__ int digit_offset_word(int k)
+{
+    const int kk = k & 31;
+    const int bit = (kk & 1) ? 16 + (kk >> 1) : (kk >> 1);
+    return (k >> 5) * 32 + ((bit & 7) & 3) * 8 + ((bit & 7) >> 2) * 4 + (bit >> 3);
+}
+// row stride 4 modulo 8 words (the eight rows of a half MMA tile read one
+// word each from distinct banks); digit columns of whole 4-word units, 32
+// bytes apart modulo 128
+__host__ __device__ inline int slice_stride_word(int pitch) { return pitch + ((12 - pitch % 8) % 8); }
+__host__ __device__ inline int col_bytes_word(int pitch) { return (pitch + 3) / 4 * 4 * 32 + 32; }
+// Stage-2 layout: chosen once per call from the largest rank (every adapter
+// of a segmented call uses it). Row stride, bytes per digit column, and the
+// packed words of K that stage 2 reads per row (whole groups, or the words).
+__host__ __device__ inline int stride2_of(bool word, int pitch) { return word ? slice_stride_word(pitch) : slice_stride(pitch); }
+__host__ __device__ inline int cb2_of(bool word, int pitch) { return word ? col_bytes_word(pitch) : col_bytes(pitch); }
+__host__ __device__ inline int kwords2_of(bool word, int pitch) { return word ? pitch : groups_of(pitch) * kGroupWords; }
+
 // Rows [0, n) of a packed matrix (pitch words per row) into a shared slice of
 // 'stride' words per row: bulk copies issued by warp 0 with completion on
 // 'bar' (rows of whole 16-byte units), else plain loads by the CTA. Words
 // [pitch, stride) of every row and rows [n, rows) are zeroed (the MMA units
 // read whole groups). True if the caller has to wait on 'bar'.
-__device__ __forceinline__ bool slice_load(uint32_t *dst, const uint32_t *src, int n, int rows, int pitch, int stride,
-                                           uint64_t *bar)
+__device__ __noinline__ bool slice_load(uint32_t *dst, const uint32_t *src, int n, int rows, int pitch, int stride,
+                                       uint64_t *bar, bool pad)
 {
     const bool bulk = n > 0 && pitch % 4 == 0 && (reinterpret_cast<uintptr_t>(src) & 15u) == 0;
     if (bulk) {
@@ -353,7 +379,7 @@ __device__ __forceinline__ bool slice_load(uint32_t *dst, const uint32_t *src, i
             dst[r * stride + w] = __ldg(src + static_cast<int64_t>(r) * pitch + w);
         }
     }
-    const int padw = stride - pitch;
+    const int padw = pad ? stride - pitch : 0;
     for (int i = threadIdx.x; i < n * padw; i += kThreads) {
         const int r = i / padw;
         dst[r * stride + pitch + (i - r * padw)] = 0u;
@@ -363,7 +389,7 @@ __device__ __forceinline__ bool slice_load(uint32_t *dst, const uint32_t *src, i
 }
 
 // Grid barrier on the header word (see the file comment); false on timeout.
-__device__ bool grid_sync(const DecodeParams &P, Misc *ms)
+__device__ __noinline__ bool grid_sync(const DecodeParams &P, Misc *ms)
 {
     __syncthreads();
     if (threadIdx.x == 0) {
@@ -408,7 +434,7 @@ __device__ bool grid_sync(const DecodeParams &P, Misc *ms)
 // warps; for each column group a warp runs its units of one row block twice,
 // masks 0..3 and then 4..7 (four mask accumulators live at a time), and adds
 // the folded sums to the tile. Shared memory is addressed by 32-bit offsets.
-__device__ __forceinline__ void sign_sums(uint32_t slice, int stride, int nrb, int ng, uint32_t dig, int cb,
+__device__ __noinline__ void sign_sums(uint32_t slice, int stride, int nrb, int ng, uint32_t dig, int cb,
                                           int ndcol, int *tile, int tile_ld)
 {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -459,7 +485,48 @@ __device__ __forceinline__ void sign_sums(uint32_t slice, int stride, int nrb, i
     }
 }
 
+// The same in the per-word layout (stage 2 of small ranks): K = 'pitch'
+// packed words, one MMA per word and column group.
+__device__ __noinline__ void sign_sums_word(uint32_t slice, int stride, int nrb, int pitch, uint32_t dig, int cb,
+                                           int ndcol, int *tile, int tile_ld)
+{
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int g = lane >> 2, t = lane & 3;
+    const int units = nrb * pitch;
+    const int u_begin = static_cast<int>(static_cast<int64_t>(units) * warp / kWarps);
+    const int u_end = static_cast<int>(static_cast<int64_t>(units) * (warp + 1) / kWarps);
+    const int ncg = (ndcol + 7) >> 3;
+    for (int q = 0; q < ncg; ++q) {
+        const int col = q * 8 + g;
+        const uint32_t cp = dig + static_cast<uint32_t>((col < ndcol ? col : 0) * cb + t * 8);
+        for (int u = u_begin; u < u_end;) {
+            const int rb = u / pitch;
+            const int w0 = u - rb * pitch;
+            const int w1 = min(pitch, w0 + (u_end - u));
+            const uint32_t ra = slice + static_cast<uint32_t>((rb * 16 + g) * stride * 4);
+            const uint32_t rb8 = ra + static_cast<uint32_t>(8 * stride * 4);
+            int acc[4] = {0, 0, 0, 0};
+            for (int w = w0; w < w1; ++w) {
+                uint32_t wa, wb;
+                asm volatile("ld.shared.u32 %0, [%1];" : "=r"(wa) : "r"(ra + w * 4));
+                asm volatile("ld.shared.u32 %0, [%1];" : "=r"(wb) : "r"(rb8 + w * 4));
+                const uint2 bv = lds64(cp + w * 32);
+                mma_u8s8(acc, (wa >> t) & 0x01010101u, (wb >> t) & 0x01010101u, (wa >> (t + 4)) & 0x01010101u,
+                         (wb >> (t + 4)) & 0x01010101u, bv.x, bv.y);
+            }
+            int *tr = tile + (rb * 16 + g) * tile_ld + q * 8 + 2 * t;
+            atomicAdd(tr, acc[0]);
+            atomicAdd(tr + 1, acc[1]);
+            atomicAdd(tr + 8 * tile_ld, acc[2]);
+            atomicAdd(tr + 8 * tile_ld + 1, acc[3]);
+            u += w1 - w0;
+        }
+    }
+}
+
 // sum_k b_k q_k of one (row, chunk column) from the three digit columns of the tile
+
+
 __device__ __forceinline__ long long digit_sum(const int *tr, int l)
 {
     return static_cast<long long>(tr[kDigits * l]) + 256LL * tr[kDigits * l + 1] + 65536LL * tr[kDigits * l + 2];
@@ -467,18 +534,31 @@ __device__ __forceinline__ long long digit_sum(const int *tr, int l)
 
 // Scale rows [lo, lo + n) of each of 'ell' envelopes (fp16, row stride ld)
 // into dst[e * rows + r] as fp32, zero past n.
-__device__ __forceinline__ void load_scales(float *dst, const uint16_t *src, int ld, int ell, int lo, int n, int rows)
+__device__ __noinline__ void load_scales(float *dst, const uint16_t *src, int ld, int ell, int lo, int n, int rows)
 {
-    for (int i = threadIdx.x; i < rows * ell; i += kThreads) {
-        const int e = i / rows, r = i - e * rows;
-        dst[i] = r < n ? ldg_h(src + static_cast<int64_t>(e) * ld + lo + r) : 0.f;
+    // eight loads per thread in flight before their stores
+    constexpr int kBatch = 8;
+    const int total = rows * ell;
+    for (int base = threadIdx.x; base < total; base += kBatch * kThreads) {
+        float v[kBatch];
+#pragma unroll
+        for (int e = 0; e < kBatch; ++e) {
+            const int i = base + e * kThreads;
+            const int env = i / rows, r = i - env * rows;
+            v[e] = (i < total && r < n) ? ldg_h(src + static_cast<int64_t>(env) * ld + lo + r) : 0.f;
+        }
+#pragma unroll
+        for (int e = 0; e < kBatch; ++e) {
+            const int i = base + e * kThreads;
+            if (i < total) dst[i] = v[e];
+        }
     }
 }
 
 // max |beta| over all rows and envelopes of an adapter, into *out (fp32 bits;
 // zero beforehand, read after a barrier). fp16 magnitudes order like their
 // bit patterns, so the maximum is taken on the bits.
-__device__ __forceinline__ void beta_max(const dbf_layer &A, unsigned *out)
+__device__ __noinline__ void beta_max(const dbf_layer &A, unsigned *out)
 {
     const int nb = A.R * A.ell;
     unsigned m2 = 0u;
@@ -505,7 +585,7 @@ __device__ __forceinline__ void beta_max(const dbf_layer &A, unsigned *out)
 // segment s (cs[S] = chunk count), then t0[s], t1[s] and the adapter id
 // (-1: none; segments with a bad range, id or adapter shape contribute no
 // chunks and are reported). One layer: a single segment [0, T).
-__device__ void build_chunk_table(const DecodeParams &P, int *tab, Misc *ms)
+__device__ __noinline__ void build_chunk_table(const DecodeParams &P, int *tab, Misc *ms)
 {
     int *cs = tab, *st0 = tab + P.S + 1, *st1 = st0 + P.S, *sad = st1 + P.S;
     for (int s = threadIdx.x; s < P.S; s += kThreads) {
@@ -577,10 +657,65 @@ __device__ __forceinline__ dbf_layer adapter_of(const DecodeParams &P, int a)
     return P.segmented ? P.adapters[a] : P.L;
 }
 
+// One activation column of a chunk: q = round(gamma . x 2^sh) with sh from
+// the column's max |gamma . x|, as three digit columns at d0 (cb bytes
+// apart), in two rolled passes over the staged values (maximum, then
+// digits). A thread takes units (packed word w, mask j): the columns that
+// bits j, j + 8, j + 16 and j + 24 of word w stand for (2j, 2j + 16, 2j + 1
+// and 2j + 17 of the word) make one 32-bit word per digit. Returns sh; the
+// warp's sums of q and |q| go to wq and wa (per-warp partials).
+__device__ __noinline__ int digit_column(const uint16_t *gc, const unsigned char *xs, dbf_dtype xd, int m, int nunits,
+                                         char *d0, int cb, unsigned *amax, long long *wq, long long *wa)
+{
+    const int lane = threadIdx.x & 31;
+    float mx = 0.f;
+#pragma unroll 1
+    for (int unit = threadIdx.x; unit < nunits; unit += kThreads) {
+        const int col = 32 * (unit >> 3) + 2 * (unit & 7);
+        const float2 a = gamma_x2(gc, xs, xd, col, m), h = gamma_x2(gc, xs, xd, col + 16, m);
+        mx = fmaxf(fmaxf(mx, fmaxf(fabsf(a.x), fabsf(a.y))), fmaxf(fabsf(h.x), fabsf(h.y)));
+    }
+    // magnitudes order like their fp32 bit patterns
+    const unsigned mw = __reduce_max_sync(0xffffffffu, __float_as_uint(mx));
+    if (lane == 0) atomicMax(amax, mw);
+    __syncthreads();
+    const int sh = scale_exponent(__uint_as_float(*amax));
+    int sq = 0, sa = 0;   // |sum| < 2^31 per thread for M <= 8192
+#pragma unroll 1
+    for (int unit = threadIdx.x; unit < nunits; unit += kThreads) {
+        const int col = 32 * (unit >> 3) + 2 * (unit & 7);
+        const float2 a = gamma_x2(gc, xs, xd, col, m), h = gamma_x2(gc, xs, xd, col + 16, m);
+        const int q0 = quantize(a.x, sh), q1 = quantize(h.x, sh), q2 = quantize(a.y, sh), q3 = quantize(h.y, sh);
+        sq += (q0 + q1) + (q2 + q3);
+        sa += (abs(q0) + abs(q1)) + (abs(q2) + abs(q3));
+        const uint32_t D0 = digit_bytes(q0), D1 = digit_bytes(q1), D2 = digit_bytes(q2), D3 = digit_bytes(q3);
+        // byte k of digit word i = byte i of Dk
+        const uint32_t lo01 = __byte_perm(D0, D1, 0x5140), lo23 = __byte_perm(D2, D3, 0x5140);
+        const uint32_t hi01 = __byte_perm(D0, D1, 0x0062), hi23 = __byte_perm(D2, D3, 0x0062);
+        char *dp = d0 + unit_offset(unit >> 3, unit & 7);
+        *reinterpret_cast<uint32_t *>(dp) = __byte_perm(lo01, lo23, 0x5410);
+        *reinterpret_cast<uint32_t *>(dp + cb) = __byte_perm(lo01, lo23, 0x7632);
+        *reinterpret_cast<uint32_t *>(dp + 2 * cb) = __byte_perm(hi01, hi23, 0x5410);
+    }
+    const long long q64 = warp_sum_exact(sq), a64 = warp_sum_exact(sa);
+    if (lane == 0) {
+        *wq = q64;
+        *wa = a64;
+    }
+    return sh;
+}
+
 // ---- the kernel -----------------------------------------------------------------
-// Phases that run once per item are rolled loops (the kernel's instructions
-// are fetched cold each call). Per-warp partial sums go through shared
-// memory as plain stores (no 64-bit shared atomics).
+// Phases that run once per item are rolled loops and shared helpers called
+// out of line: the kernel's instructions are fetched cold each call, so the
+// length of the code a call executes sets the time of those phases. Per-warp
+// partial sums go through shared memory as plain stores.
+//
+// An item's slice and scale rows are reloaded only when its (adapter, row
+// range) differs from the previous item's, its digits only when its chunk
+// does. Stage-1 items run chunk by chunk (it = q * P1 + p: a CTA's items of
+// one chunk share the digits), stage-2 items range by range
+// (it = p * Q + q: a CTA's items of one adapter share the slice).
 __global__ void __launch_bounds__(kThreads, 2) decode_multi_kernel(const __grid_constant__ DecodeParams P)
 {
     extern __shared__ __align__(128) unsigned char smem[];
@@ -598,8 +733,8 @@ __global__ void __launch_bounds__(kThreads, 2) decode_multi_kernel(const __grid_
     char *dig = reinterpret_cast<char *>(smem + P.off_dig);
     int *tile = reinterpret_cast<int *>(smem + P.off_tile);
     Misc *ms = reinterpret_cast<Misc *>(smem + P.off_misc);
-    float *rs1 = reinterpret_cast<float *>(smem + P.off_rs1);                 // beta of the stage-1 item's rows
-    float *rs2 = reinterpret_cast<float *>(smem + P.off_rs2);                 // alpha of the stage-2 item's rows
+    float *rs1 = reinterpret_cast<float *>(smem + P.off_rs1);                 // beta of the stage-1 rows
+    float *rs2 = reinterpret_cast<float *>(smem + P.off_rs2);                 // alpha of the stage-2 rows
     int *tab = reinterpret_cast<int *>(smem + P.off_seg);
     const int xsize = P.xd == DBF_BF16 ? 2 : 4;
 
@@ -610,12 +745,8 @@ __global__ void __launch_bounds__(kThreads, 2) decode_multi_kernel(const __grid_
     }
     __syncthreads();
 
-    // copy-barrier phases used so far (the same in every thread)
-    uint32_t n_s1 = 0, n_s2 = 0, n_g = 0, n_x = 0;
-
-    const int nrb2 = (P.N + 15) / 16;
-    int Q = 0;
-    if (!P.segmented) Q = (P.T + P.tpc - 1) / P.tpc;
+    uint32_t n_s1 = 0, n_s2 = 0, n_g = 0, n_x = 0;   // copy-barrier phases used (the same in every thread)
+    int Q = P.segmented ? 0 : (P.T + P.tpc - 1) / P.tpc;
     int it1b = 0, it1e = 0, it2b = 0, it2e = 0;
     auto item_ranges = [&]() {
         const int I1 = Q * P.P1, I2 = Q * P.P2;
@@ -624,61 +755,103 @@ __global__ void __launch_bounds__(kThreads, 2) decode_multi_kernel(const __grid_
         it2b = static_cast<int>(static_cast<int64_t>(I2) * b / G);
         it2e = static_cast<int>(static_cast<int64_t>(I2) * (b + 1) / G);
     };
-    // the scale rows of the CTA's first item of each stage, and max |beta| of
-    // a single layer, are loaded once here
-    int rs1_item = -1, rs2_item = -1, bmax_of = -1;
-    auto first_scales = [&]() {
+    // loaded contexts: slice and scale rows per (adapter, range), gamma and
+    // max |beta| per adapter
+    int s1_a = -1, s1_p = -1, r1_a = -1, r1_p = -1, s2_a = -1, s2_p = -1, r2_a = -1, r2_p = -1;
+    int g_a = -1, bmax_a = -1;
+    bool s1_pending = false, s2_pending = false, g_pending = false;
+
+    // row range p of a rank split into P ranges of 16-row blocks
+    auto range_of = [](int rows_total, int parts, int p, int &lo, int &rows, int &n) {
+        const int nrb = (rows_total + 15) / 16;
+        const int blo = nrb * p / parts, bhi = nrb * (p + 1) / parts;
+        lo = blo * 16;
+        rows = (bhi - blo) * 16;
+        n = max(0, min(bhi * 16, rows_total) - lo);
+    };
+    auto load_s1 = [&](const dbf_layer &A, int a, int p) {
+        int lo, rows, n;
+        range_of(A.R, P.P1, p, lo, rows, n);
+        s1_pending = slice_load(s1, A.b2_packed + static_cast<int64_t>(lo) * P.pitch1, n, rows, P.pitch1, P.stride1,
+                                &ms->bar[0], true);
+        s1_a = a;
+        s1_p = p;
+    };
+    auto load_r1 = [&](const dbf_layer &A, int a, int p) {
+        int lo, rows, n;
+        range_of(A.R, P.P1, p, lo, rows, n);
+        load_scales(rs1, A.beta, A.R, A.ell, lo, n, rows);
+        r1_a = a;
+        r1_p = p;
+    };
+    auto load_s2 = [&](const dbf_layer &A, int a, int p) {
+        int lo, rows, n;
+        range_of(P.N, P.P2, p, lo, rows, n);
+        const int pitch2 = static_cast<int>(pitch_words(A.R));
+        s2_pending = slice_load(s2, A.b1_packed + static_cast<int64_t>(lo) * pitch2, n, rows, pitch2,
+                                stride2_of(P.word2, pitch2), &ms->bar[1], !P.word2);
+        s2_a = a;
+        s2_p = p;
+    };
+    auto load_r2 = [&](const dbf_layer &A, int a, int p) {
+        int lo, rows, n;
+        range_of(P.N, P.P2, p, lo, rows, n);
+        load_scales(rs2, A.alpha, P.N, A.ell, lo, n, rows);
+        r2_a = a;
+        r2_p = p;
+    };
+    // gamma of an adapter into rows of gpitch values: one bulk copy when its
+    // rows are whole 16-byte units at a 16-byte address, else plain copies
+    // (visible after the next barrier)
+    auto stage_gamma = [&](const dbf_layer &A, int a) {
+        if ((reinterpret_cast<uintptr_t>(A.gamma) & 15u) == 0 && P.M % 8 == 0) {
+            if (tid == 0) {
+                const uint32_t bytes = static_cast<uint32_t>(A.ell) * P.M * 2u;
+                fence_proxy_async();
+                bar_expect_tx(&ms->bar[2], bytes);
+                for (uint32_t off = 0; off < bytes; off += 65536u)
+                    bulk_g2s(reinterpret_cast<char *>(gs) + off, reinterpret_cast<const char *>(A.gamma) + off,
+                             min(65536u, bytes - off), &ms->bar[2]);
+            }
+            g_pending = true;
+        } else {
+            for (int i = tid; i < A.ell * P.M; i += kThreads) {
+                const int e = i / P.M;
+                gs[e * P.gpitch + (i - e * P.M)] = A.gamma[i];
+            }
+        }
+        g_a = a;
+    };
+    auto wait_gamma = [&]() {
+        if (g_pending) {
+            copy_wait(&ms->bar[2], n_g & 1u, P.status);
+            ++n_g;
+            g_pending = false;
+        }
+    };
+    // the CTA's first items: slice of stage 1, gamma, scale rows of both
+    // stages, max |beta| (one layer with static weights: before the previous
+    // kernel has finished)
+    auto first_items = [&]() {
         if (it1b < it1e) {
             const Chunk ch = chunk_of(P, tab, it1b / P.P1);
             if (ch.a >= 0) {
                 const dbf_layer A = adapter_of(P, ch.a);
-                const int p = it1b % P.P1, nrb = (A.R + 15) / 16;
-                const int blo = nrb * p / P.P1, bhi = nrb * (p + 1) / P.P1;
-                load_scales(rs1, A.beta, A.R, A.ell, blo * 16, max(0, min(bhi * 16, A.R) - blo * 16), (bhi - blo) * 16);
-                rs1_item = it1b;
-                if (!P.segmented) {
-                    beta_max(A, &ms->bmax);
-                    bmax_of = 0;
-                }
+                load_s1(A, ch.a, it1b % P.P1);
+                if (P.stage_g) stage_gamma(A, ch.a);
+                load_r1(A, ch.a, it1b % P.P1);
+                beta_max(A, &ms->bmax);
+                bmax_a = ch.a;
             }
         }
         if (it2b < it2e) {
-            const Chunk ch = chunk_of(P, tab, it2b / P.P2);
-            if (ch.a >= 0) {
-                const dbf_layer A = adapter_of(P, ch.a);
-                const int p = it2b % P.P2;
-                const int blo = nrb2 * p / P.P2, bhi = nrb2 * (p + 1) / P.P2;
-                load_scales(rs2, A.alpha, P.N, A.ell, blo * 16, max(0, min(bhi * 16, P.N) - blo * 16), (bhi - blo) * 16);
-                rs2_item = it2b;
-            }
+            const Chunk ch = chunk_of(P, tab, it2b % Q);
+            if (ch.a >= 0) load_r2(adapter_of(P, ch.a), ch.a, it2b / Q);
         }
     };
-    // one layer with static weights: the first stage-1 slice, gamma and the
-    // scales are in flight before the previous kernel has finished
-    int pre1 = -1;       // stage-1 item whose slice is in flight
-    int pre_g = -1;      // adapter whose gamma is staged or in flight
-    bool g_pending = false;
-    bool s1_wait = false;
     if (!P.segmented) item_ranges();
     if (early) {
-        if (it1b < it1e) {
-            const int p = it1b % P.P1;
-            const int nrb = (P.L.R + 15) / 16;
-            const int blo = nrb * p / P.P1, bhi = nrb * (p + 1) / P.P1;
-            const int lo = blo * 16, n = max(0, min(bhi * 16, P.L.R) - lo);
-            s1_wait = slice_load(s1, P.L.b2_packed + static_cast<int64_t>(lo) * P.pitch1, n, (bhi - blo) * 16,
-                                 P.pitch1, P.stride1, &ms->bar[0]);
-            pre1 = it1b;
-            if (P.stage_g) {
-                if (tid == 0) {
-                    bar_expect_tx(&ms->bar[2], static_cast<uint32_t>(P.gs_bytes));
-                    bulk_g2s(gs, P.L.gamma, static_cast<uint32_t>(P.gs_bytes), &ms->bar[2]);
-                }
-                pre_g = 0;
-                g_pending = true;
-            }
-        }
-        first_scales();
+        first_items();
         pdl_wait();
     }
     if (P.segmented) {
@@ -686,93 +859,59 @@ __global__ void __launch_bounds__(kThreads, 2) decode_multi_kernel(const __grid_
         Q = ms->Q;
         item_ranges();
     }
-    if (!early) first_scales();
+    if (!early) first_items();
     if (tid == 0) {
         unsigned long long v;
         asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(P.sync) : "memory");
         ms->e0 = static_cast<unsigned>(v >> 32);
     }
-
-    // the first stage-2 slice: copied over the staged activations once the
-    // CTA's last digits are built (or at once, with no stage-1 items)
-    bool s2_issued = false, s2_wait = false;
-    auto issue_s2 = [&](int it) {
-        const int q = it / P.P2, p = it % P.P2;
-        const Chunk ch = chunk_of(P, tab, q);
-        const int blo = nrb2 * p / P.P2, bhi = nrb2 * (p + 1) / P.P2;
-        const int lo = blo * 16, n = max(0, min(bhi * 16, P.N) - lo);
-        s2_wait = false;
-        if (ch.a >= 0) {
-            const dbf_layer A = adapter_of(P, ch.a);
-            const int pitch2 = static_cast<int>(pitch_words(A.R));
-            s2_wait = slice_load(s2, A.b1_packed + static_cast<int64_t>(lo) * pitch2, n, (bhi - blo) * 16, pitch2,
-                                 slice_stride(pitch2), &ms->bar[1]);
-        }
-    };
-    if (it1b >= it1e && it2b < it2e) {
-        if (g_pending) {
-            copy_wait(&ms->bar[2], 0u, P.status);   // gamma was staged over the stage-2 region
-            g_pending = false;
-            ++n_g;
-        }
+    // the first stage-2 slice goes over the staging buffers once the CTA's
+    // last digits are built (or at once, with no stage-1 items)
+    bool s2_issued = false;
+    auto issue_first_s2 = [&]() {
+        wait_gamma();
         __syncthreads();
-        issue_s2(it2b);
+        if (it2b < it2e) {
+            const Chunk ch = chunk_of(P, tab, it2b % Q);
+            if (ch.a >= 0) load_s2(adapter_of(P, ch.a), ch.a, it2b / Q);
+        }
         s2_issued = true;
-    }
+    };
+    if (it1b >= it1e) issue_first_s2();
+    const int q_last1 = it1e > it1b ? (it1e - 1) / P.P1 : -1;
 
     // ================= stage 1 =================
-    int cur_q = -1, cur_a = -1;
+    int dig_q = -1;
     for (int it = it1b; it < it1e; ++it) {
         const int q = it / P.P1, p = it % P.P1;
         const Chunk ch = chunk_of(P, tab, q);
         if (ch.a < 0) continue;   // no adapter: stage 2 writes the zero branch
         const dbf_layer A = adapter_of(P, ch.a);
         const int ell = A.ell, cc = ch.ntok * ell, ndcol = kDigits * cc;
-        const int nrb = (A.R + 15) / 16;
-        const int blo = nrb * p / P.P1, bhi = nrb * (p + 1) / P.P1;
-        const int lo = blo * 16, rows = (bhi - blo) * 16, n1 = max(0, min(bhi * 16, A.R) - lo);
-        // ---- the item's slice of B2
-        if (it != pre1) {
+        int lo, rows, n1;
+        range_of(A.R, P.P1, p, lo, rows, n1);
+        if (s1_a != ch.a || s1_p != p) {
             __syncthreads();   // the previous item's reads of the slice are done
-            s1_wait = slice_load(s1, A.b2_packed + static_cast<int64_t>(lo) * P.pitch1, n1, rows, P.pitch1, P.stride1,
-                                 &ms->bar[0]);
+            load_s1(A, ch.a, p);
         }
         // ---- digits of gamma . x for the chunk's columns (l = token * ell + i)
-        if (q != cur_q || ch.a != cur_a) {
+        if (dig_q != q) {
             __syncthreads();   // earlier reads of the staging buffers and digits are done
-            const bool new_adapter = ch.a != cur_a;
-            cur_q = q;
-            // gamma of the adapter (staged, or read from global memory)
+            dig_q = q;
             const uint16_t *gsrc = A.gamma;
             int gld = P.M;
             if (P.stage_g) {
-                if (pre_g != ch.a) {
-                    if (tid == 0) {
-                        fence_proxy_async();
-                        bar_expect_tx(&ms->bar[2], static_cast<uint32_t>(P.gs_bytes));
-                        bulk_g2s(gs, A.gamma, static_cast<uint32_t>(P.gs_bytes), &ms->bar[2]);
-                    }
-                    pre_g = ch.a;
-                    g_pending = true;
-                }
-                if (g_pending) {
-                    copy_wait(&ms->bar[2], n_g & 1u, P.status);
-                    ++n_g;
-                    g_pending = false;
-                }
+                if (g_a != ch.a) stage_gamma(A, ch.a);
+                wait_gamma();
                 gsrc = gs;
                 gld = P.gpitch;
             }
-            // max |beta| of the adapter
-            if (new_adapter) {
-                cur_a = ch.a;
-                if (bmax_of != ch.a) {
-                    __syncthreads();   // earlier reads of the maximum are done
-                    if (tid == 0) ms->bmax = 0u;
-                    __syncthreads();
-                    beta_max(A, &ms->bmax);
-                    bmax_of = ch.a;
-                }
+            if (bmax_a != ch.a) {
+                __syncthreads();   // earlier reads of the maximum are done
+                if (tid == 0) ms->bmax = 0u;
+                __syncthreads();
+                beta_max(A, &ms->bmax);
+                bmax_a = ch.a;
             }
             if (tid < kChunkCols) ms->amax[tid] = 0u;
             // tokens one at a time through the two x buffers
@@ -787,12 +926,9 @@ __global__ void __launch_bounds__(kThreads, 2) decode_multi_kernel(const __grid_
                         bar_expect_tx(&ms->bar[3 + (seq & 1u)], static_cast<uint32_t>(P.M * xsize));
                         bulk_g2s(dst, src, static_cast<uint32_t>(P.M * xsize), &ms->bar[3 + (seq & 1u)]);
                     }
-                } else if (xsize == 2) {
-                    for (int i = tid; i < P.M; i += kThreads)
-                        reinterpret_cast<uint16_t *>(dst)[i] = reinterpret_cast<const uint16_t *>(src)[i];
                 } else {
-                    for (int i = tid; i < P.M; i += kThreads)
-                        reinterpret_cast<uint32_t *>(dst)[i] = reinterpret_cast<const uint32_t *>(src)[i];
+                    for (int i = tid; i < P.M * xsize / 2; i += kThreads)
+                        reinterpret_cast<uint16_t *>(dst)[i] = reinterpret_cast<const uint16_t *>(src)[i];
                 }
             };
             const uint32_t x0 = n_x;
@@ -808,51 +944,9 @@ __global__ void __launch_bounds__(kThreads, 2) decode_multi_kernel(const __grid_
 #pragma unroll 1
                 for (int i = 0; i < ell; ++i) {
                     const int l = tok * ell + i;
-                    const uint16_t *gc = gsrc + static_cast<int64_t>(i) * gld;
-                    float4 u[kUnitsPerThread];
-                    float m = 0.f;
-#pragma unroll
-                    for (int e = 0; e < kUnitsPerThread; ++e) {
-                        const int unit = tid + e * kThreads;
-                        const int col = 32 * (unit >> 3) + 2 * (unit & 7);
-                        const bool in = unit < nunits;
-                        const float2 a = in ? gamma_x2(gc, xs, P.xd, col, P.M) : make_float2(0.f, 0.f);
-                        const float2 h = in ? gamma_x2(gc, xs, P.xd, col + 16, P.M) : make_float2(0.f, 0.f);
-                        u[e] = make_float4(a.x, h.x, a.y, h.y);   // bits j, j + 8, j + 16, j + 24
-                        m = fmaxf(fmaxf(m, fmaxf(fabsf(a.x), fabsf(a.y))), fmaxf(fabsf(h.x), fabsf(h.y)));
-                    }
-                    // magnitudes order like their fp32 bit patterns
-                    const unsigned mw = __reduce_max_sync(0xffffffffu, __float_as_uint(m));
-                    if (lane == 0) atomicMax(&ms->amax[l], mw);
-                    __syncthreads();
-                    const int sh = scale_exponent(__uint_as_float(ms->amax[l]));
-                    int sq = 0;   // |sum| <= 16 2^22 per thread
-                    int sa = 0;
-                    char *d0 = dig + static_cast<size_t>(kDigits * l) * P.cb1;
-#pragma unroll
-                    for (int e = 0; e < kUnitsPerThread; ++e) {
-                        const int unit = tid + e * kThreads;
-                        if (unit < nunits) {
-                            const int q0 = quantize(u[e].x, sh), q1 = quantize(u[e].y, sh);
-                            const int q2 = quantize(u[e].z, sh), q3 = quantize(u[e].w, sh);
-                            sq += (q0 + q1) + (q2 + q3);
-                            sa += (abs(q0) + abs(q1)) + (abs(q2) + abs(q3));
-                            const uint32_t D0 = digit_bytes(q0), D1 = digit_bytes(q1);
-                            const uint32_t D2 = digit_bytes(q2), D3 = digit_bytes(q3);
-                            // byte k of digit word i = byte i of Dk
-                            const uint32_t lo01 = __byte_perm(D0, D1, 0x5140), lo23 = __byte_perm(D2, D3, 0x5140);
-                            const uint32_t hi01 = __byte_perm(D0, D1, 0x0062), hi23 = __byte_perm(D2, D3, 0x0062);
-                            char *dp = d0 + unit_offset(unit >> 3, unit & 7);
-                            *reinterpret_cast<uint32_t *>(dp) = __byte_perm(lo01, lo23, 0x5410);
-                            *reinterpret_cast<uint32_t *>(dp + P.cb1) = __byte_perm(lo01, lo23, 0x7632);
-                            *reinterpret_cast<uint32_t *>(dp + 2 * P.cb1) = __byte_perm(hi01, hi23, 0x5410);
-                        }
-                    }
-                    const long long wq = warp_sum_exact(sq), wa = warp_sum_exact(sa);
-                    if (lane == 0) {
-                        ms->wq[warp][l] = wq;
-                        ms->wa[warp][l] = wa;
-                    }
+                    const int sh = digit_column(gsrc + static_cast<int64_t>(i) * gld, xs, P.xd, P.M, nunits,
+                                                dig + static_cast<size_t>(kDigits * l) * P.cb1, P.cb1, &ms->amax[l],
+                                                &ms->wq[warp][l], &ms->wa[warp][l]);
                     if (tid == 0) ms->sh_u[l] = sh;
                 }
                 if (tok + 2 < ch.ntok) {
@@ -875,23 +969,18 @@ __global__ void __launch_bounds__(kThreads, 2) decode_multi_kernel(const __grid_
                                     (1.0f + 1.0f / 1024.0f);
                 ms->sh_v[tid] = scale_exponent(bound);
             }
-            // the CTA's last digits: the first stage-2 slice may go over the staging buffers
-            if (!s2_issued && it2b < it2e && (it1e - 1) / P.P1 == q) {
-                __syncthreads();
-                issue_s2(it2b);
-                s2_issued = true;
-            }
+            if (!s2_issued && q == q_last1) issue_first_s2();
         }
         // ---- beta of the item's rows, the tile, then the sign sums
-        if (it != rs1_item) {
+        if (r1_a != ch.a || r1_p != p) {
             __syncthreads();   // the previous item's reads of the rows are done
-            load_scales(rs1, A.beta, A.R, ell, lo, n1, rows);
+            load_r1(A, ch.a, p);
         }
         for (int i = tid; i < rows * P.tile_ld; i += kThreads) tile[i] = 0;
-        if (s1_wait) {
+        if (s1_pending) {
             copy_wait(&ms->bar[0], n_s1 & 1u, P.status);
             ++n_s1;
-            s1_wait = false;
+            s1_pending = false;
         } else {
             __syncthreads();
         }
@@ -899,7 +988,8 @@ __global__ void __launch_bounds__(kThreads, 2) decode_multi_kernel(const __grid_
             sign_sums(smem_u32(s1), P.stride1, rows / 16, groups_of(P.pitch1), smem_u32(dig), P.cb1, ndcol, tile,
                       P.tile_ld);
         __syncthreads();
-        // ---- v = beta . h as digits into the image; sums of q of v per column
+        // ---- v = beta . h as digits into the image (stage-2 layout); sums of q of v per column
+        const int pitch2 = static_cast<int>(pitch_words(A.R));
         int qv[kChunkCols];
 #pragma unroll
         for (int c = 0; c < kChunkCols; ++c) qv[c] = 0;
@@ -907,12 +997,13 @@ __global__ void __launch_bounds__(kThreads, 2) decode_multi_kernel(const __grid_
         for (int i = tid; i < n1 * cc; i += kThreads) {
             const int l = i / n1, r = i - l * n1;
             const int tok = l / ell, env = l - tok * ell;
-            const long long s = digit_sum(tile + r * P.tile_ld, l);
-            const float h = scale_pow2(__ll2float_rn(ms->qsum_u[l] - 2 * s), -ms->sh_u[l]);
+            const long long sm = digit_sum(tile + r * P.tile_ld, l);
+            const float h = scale_pow2(__ll2float_rn(ms->qsum_u[l] - 2 * sm), -ms->sh_u[l]);
             const int qq = quantize(rs1[env * rows + r] * h, ms->sh_v[l]);
             const uint32_t db = digit_bytes(qq);
             const int64_t c = static_cast<int64_t>(ch.t0 + tok) * P.ell_cap + env;
-            char *im = P.img + static_cast<size_t>(c) * kDigits * P.cb2 + digit_offset(lo + r);
+            char *im = P.img + static_cast<size_t>(c) * kDigits * P.cb2 +
+                       (P.word2 ? digit_offset_word(lo + r) : digit_offset(lo + r));
             im[0] = static_cast<char>(db & 255u);
             im[P.cb2] = static_cast<char>((db >> 8) & 255u);
             im[2 * P.cb2] = static_cast<char>(db >> 16);
@@ -920,16 +1011,17 @@ __global__ void __launch_bounds__(kThreads, 2) decode_multi_kernel(const __grid_
             for (int c2 = 0; c2 < kChunkCols; ++c2)
                 if (c2 == l) qv[c2] += qq;
         }
-        // digits of v past the rank, to the end of its last group, are zero
-        // (whatever the padding bits of B1)
-        if (bhi == nrb) {
-            const int tail = groups_of(static_cast<int>(pitch_words(A.R))) * 256 - A.R;
+        // digits of v past the rank, to the end of the K words stage 2 reads,
+        // are zero (whatever the padding bits of B1)
+        if (lo + rows >= A.R) {
+            const int tail = kwords2_of(P.word2, pitch2) * 32 - A.R;
 #pragma unroll 1
             for (int i = tid; i < cc * tail; i += kThreads) {
                 const int l = i / tail, k = A.R + (i - l * tail);
                 const int tok = l / ell, env = l - tok * ell;
                 const int64_t c = static_cast<int64_t>(ch.t0 + tok) * P.ell_cap + env;
-                char *im = P.img + static_cast<size_t>(c) * kDigits * P.cb2 + digit_offset(k);
+                char *im = P.img + static_cast<size_t>(c) * kDigits * P.cb2 +
+                           (P.word2 ? digit_offset_word(k) : digit_offset(k));
                 im[0] = 0;
                 im[P.cb2] = 0;
                 im[2 * P.cb2] = 0;
@@ -952,32 +1044,23 @@ __global__ void __launch_bounds__(kThreads, 2) decode_multi_kernel(const __grid_
             if (n1 > 0) P.sh2[c] = ms->sh_v[tid];   // the same value from every item of the chunk
         }
     }
-    if (!s2_issued && it2b < it2e) {
-        if (g_pending) {
-            copy_wait(&ms->bar[2], n_g & 1u, P.status);   // gamma was staged over the stage-2 region
-            g_pending = false;
-            ++n_g;
-        }
-        __syncthreads();
-        issue_s2(it2b);
-        s2_issued = true;
-    }
-    if (g_pending) copy_wait(&ms->bar[2], n_g & 1u, P.status);   // no copy left in flight
+    if (!s2_issued) issue_first_s2();
+    wait_gamma();   // no copy left in flight
 
     // ---- every CTA's digits of v and its sums are written
     const bool passed = grid_sync(P, ms);
     if (!passed) {
-        if (s2_wait) copy_wait(&ms->bar[1], n_s2 & 1u, P.status);   // no copy left in flight
+        if (s2_pending) copy_wait(&ms->bar[1], n_s2 & 1u, P.status);   // no copy left in flight
         return;
     }
 
     // ================= stage 2 =================
-    cur_q = -1;
+    int img_q = -1;
     for (int it = it2b; it < it2e; ++it) {
-        const int q = it / P.P2, p = it % P.P2;
+        const int p = it / Q, q = it % Q;
         const Chunk ch = chunk_of(P, tab, q);
-        const int blo = nrb2 * p / P.P2, bhi = nrb2 * (p + 1) / P.P2;
-        const int lo = blo * 16, rows = (bhi - blo) * 16, n2 = max(0, min(bhi * 16, P.N) - lo);
+        int lo, rows, n2;
+        range_of(P.N, P.P2, p, lo, rows, n2);
         if (ch.a < 0) {
             // no adapter: the branch is zero
             if (!(P.flags & DBF_ACCUMULATE)) {
@@ -991,18 +1074,21 @@ __global__ void __launch_bounds__(kThreads, 2) decode_multi_kernel(const __grid_
         const dbf_layer A = adapter_of(P, ch.a);
         const int ell = A.ell, cc = ch.ntok * ell, ndcol = kDigits * cc;
         const int pitch2 = static_cast<int>(pitch_words(A.R));
-        if (it != it2b) {
+        if (s2_a != ch.a || s2_p != p) {
             __syncthreads();   // the previous item's reads of the slice are done
-            s2_wait = slice_load(s2, A.b1_packed + static_cast<int64_t>(lo) * pitch2, n2, rows, pitch2,
-                                 slice_stride(pitch2), &ms->bar[1]);
+            load_s2(A, ch.a, p);
+        }
+        if (r2_a != ch.a || r2_p != p) {
+            __syncthreads();   // the previous item's reads of the rows are done
+            load_r2(A, ch.a, p);
         }
         // ---- the chunk's digits of v (coherent 16-byte loads: other CTAs wrote
         // them in this kernel), its sums of q and scales: the first round of
         // both kinds of loads is in flight together
-        if (q != cur_q) {
+        if (img_q != q) {
             __syncthreads();   // earlier reads of the digits are done
-            cur_q = q;
-            const int n16 = groups_of(pitch2) * 16;   // 16-byte units of one digit row
+            img_q = q;
+            const int n16 = kwords2_of(P.word2, pitch2) * 2;   // 16-byte units of one digit row
             const int nimg = ndcol * n16;
             auto img_unit = [&](int i) {
                 const int dc = i / n16, k = i - dc * n16;
@@ -1020,6 +1106,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_multi_kernel(const __grid_
             }
             long long pv[kPart];
             int64_t cw = 0;
+            int shv = 0;
             if (warp < cc) {
                 const int tok = warp / ell, env = warp - tok * ell;
                 cw = static_cast<int64_t>(ch.t0 + tok) * P.ell_cap + env;
@@ -1028,6 +1115,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_multi_kernel(const __grid_
                     const int k = lane + 32 * e;
                     pv[e] = k < P.P1 ? __ldcg(P.qpart + cw * P.P1 + k) : 0;
                 }
+                shv = __ldcg(P.sh2 + cw);
             }
 #pragma unroll
             for (int e = 0; e < kImg; ++e) {
@@ -1045,25 +1133,26 @@ __global__ void __launch_bounds__(kThreads, 2) decode_multi_kernel(const __grid_
                 sum = warp_sum_exact64(sum);
                 if (lane == 0) {
                     ms->qsum_v[warp] = sum;
-                    ms->sh_v[warp] = __ldcg(P.sh2 + cw);
+                    ms->sh_v[warp] = shv;
                 }
             }
         }
-        if (it != rs2_item) {
-            __syncthreads();   // the previous item's reads of the rows are done
-            load_scales(rs2, A.alpha, P.N, ell, lo, n2, rows);
-        }
         for (int i = tid; i < rows * P.tile_ld; i += kThreads) tile[i] = 0;
-        if (s2_wait) {
+        if (s2_pending) {
             copy_wait(&ms->bar[1], n_s2 & 1u, P.status);
             ++n_s2;
-            s2_wait = false;
+            s2_pending = false;
         } else {
             __syncthreads();
         }
-        if (n2 > 0)
-            sign_sums(smem_u32(s2), slice_stride(pitch2), rows / 16, groups_of(pitch2), smem_u32(dig), P.cb2, ndcol,
-                      tile, P.tile_ld);
+        if (n2 > 0) {
+            if (P.word2)
+                sign_sums_word(smem_u32(s2), stride2_of(true, pitch2), rows / 16, pitch2, smem_u32(dig), P.cb2, ndcol,
+                               tile, P.tile_ld);
+            else
+                sign_sums(smem_u32(s2), stride2_of(false, pitch2), rows / 16, groups_of(pitch2), smem_u32(dig), P.cb2,
+                          ndcol, tile, P.tile_ld);
+        }
         __syncthreads();
         // ---- y = [acc] y + sum_i alpha_i . z_i, one (token, row) per thread
 #pragma unroll 1
@@ -1074,8 +1163,8 @@ __global__ void __launch_bounds__(kThreads, 2) decode_multi_kernel(const __grid_
 #pragma unroll 1
             for (int env = 0; env < ell; ++env) {
                 const int l = tok * ell + env;
-                const long long s = digit_sum(tile + r * P.tile_ld, l);
-                const float z = scale_pow2(__ll2float_rn(ms->qsum_v[l] - 2 * s), -ms->sh_v[l]);
+                const long long sm = digit_sum(tile + r * P.tile_ld, l);
+                const float z = scale_pow2(__ll2float_rn(ms->qsum_v[l] - 2 * sm), -ms->sh_v[l]);
                 yv += rs2[env * rows + r] * z;
             }
             store_act(P.y, P.yd, yi, yv);
@@ -1095,7 +1184,8 @@ struct WsLayout {
 WsLayout ws_layout(int64_t cols, int max_R)
 {
     WsLayout w;
-    const int cb2 = col_bytes(static_cast<int>(pitch_words(max_R)));
+    const int pitch2 = static_cast<int>(pitch_words(max_R));
+    const int cb2 = cb2_of(word_layout(pitch2), pitch2);
     const int64_t nrb1 = (max_R + 15) / 16;
     w.img = kWsHeaderBytes;
     w.qpart = w.img + align_up(static_cast<size_t>(cols) * kDigits * cb2, 256);
@@ -1172,9 +1262,10 @@ bool decode_plan(const CallShape &cs, int sms, DecodeParams *out, size_t *smem_o
         P.pitch1 = static_cast<int>(pitch_words(cs.M));
         const int pitch2 = static_cast<int>(pitch_words(cs.max_R));
         P.stride1 = slice_stride(P.pitch1);
-        P.stride2 = slice_stride(pitch2);
+        P.word2 = word_layout(pitch2);
+        P.stride2 = stride2_of(P.word2, pitch2);
         P.cb1 = col_bytes(P.pitch1);
-        P.cb2 = col_bytes(pitch2);
+        P.cb2 = cb2_of(P.word2, pitch2);
         P.gpitch = (cs.M + 7) / 8 * 8;
         P.gs_bytes = static_cast<int>(static_cast<size_t>(cs.ell_cap) * P.gpitch * 2);
         P.xs_bytes = static_cast<int>(align_up(static_cast<size_t>(cs.M) * cs.xsize, 16));
@@ -1216,7 +1307,8 @@ bool decode_plan(const CallShape &cs, int sms, DecodeParams *out, size_t *smem_o
         const double builds = std::min(k1, std::ceil(k1 / P.P1) + (P.P1 > 1 ? 1 : 0));
         const double c1 = builds * (0.3 + 0.55 * cc * cs.M / 4096.0) + (k1 - 1) * 1.0 +
                           k1 * (P.rows1 / 16) * ng1 * 8 * ncg * mma_us;
-        const double c2 = k2 * (0.3 + (P.rows2 / 16) * ng2 * 8 * ncg * mma_us) + (k2 - 1) * 1.0;
+        const double mma2 = P.word2 ? pitch2 * 1.4 : ng2 * 8.0;   // per-word MMAs issue about 1.4x slower
+        const double c2 = k2 * (0.3 + (P.rows2 / 16) * mma2 * ncg * mma_us) + (k2 - 1) * 1.0;
         const double cost = c1 + c2;
         if (cost < best_cost) {
             best_cost = cost;
@@ -1326,9 +1418,6 @@ cudaError_t multi_forward(const dbf_layer &L, const void *x, dbf_dtype xd, void 
     P.xd = xd;
     P.yd = yd;
     P.flags = flags;
-    // gamma staged only when its rows are whole 16-byte units at a 16-byte
-    // address (one bulk copy); otherwise read from global memory
-    if (P.stage_g && !((reinterpret_cast<uintptr_t>(L.gamma) & 15u) == 0 && L.M % 8 == 0)) P.stage_g = 0;
     set_workspace(P, ws, T * L.ell);
     return launch(P, smem, G, s);
 }
@@ -1368,9 +1457,6 @@ cudaError_t multi_forward_segmented(const dbf_layer *adapters, int32_t num_adapt
     P.xd = xd;
     P.yd = yd;
     P.flags = flags;
-    // the adapters' gamma pointers are known only on the device: gamma is
-    // read from global memory
-    P.stage_g = 0;
     set_workspace(P, ws, T * max_ell);
     return launch(P, smem, G, s);
 }

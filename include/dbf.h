@@ -95,8 +95,10 @@ enum { DBF_ACCUMULATE = 1, DBF_WEIGHTS_STATIC = 2 };
 /* GEMV: the decode kernel (few tokens, bandwidth bound, any shape).
  * GEMM: the prefill kernel (tcgen05 tensor cores; needs M % 128 == 0 and
  *       R % 128 == 0; any N).
- * AUTO: GEMM when the shape allows it and T is at least dbf_gemm_min_tokens(),
- *       else GEMV. */
+ * AUTO: GEMM when the shape allows it and T is at least
+ *       dbf_gemm_min_tokens(L) (from measured time models of both paths on
+ *       B200; about 13 tokens for a 4096 x 11008 layer at rank 5888, about 80
+ *       at 4096 x 4096 rank 1024, never for small adapter ranks), else GEMV. */
 typedef enum { DBF_PATH_AUTO = 0, DBF_PATH_GEMV = 1, DBF_PATH_GEMM = 2 } dbf_path;
 
 /* One layer or adapter. All pointers are device pointers, caller owned.
@@ -221,8 +223,10 @@ dbf_status dbf_factorize(const float *W, int64_t n, int64_t m, int64_t k, const 
                          uint32_t *a_signs, uint32_t *b_signs, uint16_t *alpha, uint16_t *beta,
                          uint16_t *gamma, float *objective, void *ws, size_t ws_bytes, void *stream);
 
-/* Smallest T for which DBF_PATH_AUTO takes the GEMM path on a shape it allows. */
-int64_t dbf_gemm_min_tokens(void);
+/* Smallest T for which DBF_PATH_AUTO takes the GEMM path on layer L; -1
+ * when it never does (shape outside the GEMM path, or the decode kernels
+ * stay faster at any T) or L is malformed. Host only, no device access. */
+int64_t dbf_gemm_min_tokens(const dbf_layer *L);
 
 /* Workspace bytes dbf_forward needs for this layer, T and path (AUTO is
  * resolved as dbf_forward resolves it). Returns 0 for invalid input. */

@@ -248,3 +248,18 @@ def test_factorize_rejects_bad_arguments(lib):
     assert call(args(wsb=need - 1)) == dbf.ERR_WORKSPACE
     assert call(args(ws=None)) == dbf.ERR_WORKSPACE
     assert call(args(ws=p + 16)) == dbf.ERR_ALIGNMENT
+
+
+def test_gemm_min_tokens(lib):
+    # AUTO's crossover per shape (host-side model fit to B200 sweeps): the
+    # measured crossovers were between 8 and 16 tokens on the DBF MLP layer and
+    # between 64 and 128 on a 4096 x 4096 rank-1024 layer; small adapter ranks
+    # stay on the decode kernels at any T; shapes outside the GEMM path never
+    # take it
+    by = ctypes.byref
+    assert 8 < lib.dbf_gemm_min_tokens(by(_layer(M=4096, N=11008, R=5888, ell=1))) <= 16
+    assert 64 < lib.dbf_gemm_min_tokens(by(_layer(M=4096, N=4096, R=1024, ell=1))) <= 128
+    assert lib.dbf_gemm_min_tokens(by(_layer(M=4096, N=4096, R=128, ell=1))) > 256
+    assert lib.dbf_gemm_min_tokens(by(_layer(M=4096, N=4096, R=64, ell=1))) == -1     # R % 128 != 0
+    assert lib.dbf_gemm_min_tokens(by(_layer(M=8192, N=8192, R=8192, ell=1))) < 64
+    assert lib.dbf_gemm_min_tokens(None) == -1

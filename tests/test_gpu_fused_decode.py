@@ -183,14 +183,16 @@ def i32(a):
     return torch.tensor(np.asarray(a, dtype=np.int32), device="cuda")
 
 
-@pytest.mark.parametrize("S_", [40, 600])
-def test_segmented_mixed_adapters(dbf, S_):
-    # adapters of different ranks (below the largest) and envelope counts,
-    # segments of 0..9 tokens, some without an adapter; 600 segments take the
-    # two-launch path
-    rng = np.random.default_rng(760 + S_)
+@pytest.mark.parametrize("S_,shapes", [(40, [(33, 1), (96, 2), (7, 3), (128, 1)]),
+                                       (40, [(33, 1), (300, 2), (7, 3)]),
+                                       (600, [(33, 1), (96, 2), (7, 3), (128, 1)])])
+def test_segmented_mixed_adapters(dbf, S_, shapes):
+    # adapters of different ranks (below the largest: small ranks in the
+    # per-word or the group layout of stage 2) and envelope counts, segments of
+    # 0..9 tokens, some without an adapter; 600 segments take the two-launch
+    # path
+    rng = np.random.default_rng(760 + S_ + len(shapes))
     M, N = 288, 136
-    shapes = [(33, 1), (96, 2), (7, 3), (128, 1)]
     layers = [random_layer(rng, M, N, R, ell) for R, ell in shapes]
     counts = rng.integers(0, 10, size=S_)
     if S_ > 100:
