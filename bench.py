@@ -25,6 +25,9 @@ each rank runs the same per-GPU work (weak scaling); the timing is the max
 over ranks.
 
 python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+python bench.py --profile NAME   (three calls of one configuration and exit,
+                                  for ncu captures: decode, prefill, tiny,
+                                  adapter64, segmented, large_prefill)
 """
 from __future__ import annotations
 
@@ -404,6 +407,45 @@ def measure_configs(dbf, dev, stream, run_oracle):
     return out
 
 
+def profile_calls(name: str, calls: int = 3):
+    """Three forward calls of one configuration on cuda:0 (seeded synthetic
+    inputs as in the timed runs), synchronised, for a profiler to capture."""
+    import torch
+    import double_binary_rank_b200 as dbf
+    dev = torch.device("cuda", 0)
+    f16 = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.float16)).to(dev)
+    bf16 = lambda a: torch.from_numpy(a.view(np.int16)).to(dev).view(torch.bfloat16)
+    dev_layer = lambda L: dbf.Layer.from_signs(torch.from_numpy(L.b1).to(dev), torch.from_numpy(L.b2).to(dev),
+                                               f16(L.alpha), f16(L.beta), f16(L.gamma))
+    if name == "segmented":
+        w = S.WORKLOADS["segmented"]
+        Ls = S.workload_layers(w)
+        table = dbf.AdapterTable([dev_layer(La) for La in Ls], dev)
+        seg = S.make_segments(w.seed, 256, w.num_adapters)
+        x = bf16(np.ascontiguousarray(S.make_x(w.seed, 256, w.M, "bf16")[seg.order]))
+        y = torch.empty((256, w.N), dtype=torch.bfloat16, device=dev)
+        offs = torch.from_numpy(seg.offsets.astype(np.int32)).to(dev)
+        ids = torch.from_numpy(seg.adapter.astype(np.int32)).to(dev)
+        ws = dbf.alloc_workspace(dbf.segmented_workspace_bytes(w.R, w.ell, 256), dev)
+        fn = lambda: dbf.forward_segmented(table, offs, ids, x, y=y, ws=ws)
+    else:
+        wname, T, kind = {"decode": ("dbf_mlp", 1, "bf16"), "prefill": ("dbf_mlp", T_PREFILL, "bf16"),
+                          "tiny": ("tiny", 4, "f32"), "adapter64": ("adapter", 64, "bf16"),
+                          "large_prefill": ("large_prefill", 8192, "bf16")}[name]
+        w = S.WORKLOADS[wname]
+        L = S.workload_layers(w)[0]
+        dl = dev_layer(L)
+        xh = S.make_x(w.seed, T, w.M, kind)
+        x = torch.from_numpy(xh).to(dev) if kind == "f32" else bf16(xh)
+        y = torch.empty((T, w.N), dtype=torch.float32 if kind == "f32" else torch.bfloat16, device=dev)
+        ws = dbf.alloc_workspace(dbf.workspace_bytes(dl, T), dev)
+        fn = lambda: dbf.forward(dl, x, y=y, ws=ws, static_weights=True)
+    for _ in range(calls):
+        fn()
+    torch.cuda.synchronize(dev)
+    print(f"profile {name}: {calls} calls done")
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -411,7 +453,12 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile", choices=["decode", "prefill", "tiny", "adapter64", "segmented", "large_prefill"],
+                    help="run three calls of one configuration and exit (no timing; for ncu captures)")
     args = ap.parse_args()
+    if args.profile:
+        profile_calls(args.profile)
+        return
     args.warmup = max(args.warmup, 3)
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
