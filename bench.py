@@ -767,8 +767,9 @@ def main():
         "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f16", "data": "synthetic",
         "config": bench_config(w),
-        "arithmetic": "prefill: fp16 x fp16 tensor cores, fp32 accumulate; decode: binary tensor-core products "
-                      "(and + popcount) over 24 bit planes of the fixed-point activations, exact integer sums",
+        "arithmetic": "prefill: fp16 x fp16 tensor cores (tcgen05), fp32 accumulate; decode: u8 x s8 integer "
+                      "tensor-core products of the sign bits with three int8 digits of 22-bit fixed-point "
+                      "activations, exact integer sums",
         "roofline": roof_pre,
         "roofline_decode": roof_dec,
         "prefill_us_per_call": pre_us,
