@@ -535,31 +535,60 @@ def main():
     tokens_per_step = T_DECODE + T_PREFILL
     value = weak_scaling_value(world, tokens_per_step, args.steps, elapsed_ms)
 
-    # ---- end to end through the public API: host buffers, copies timed
+    # ---- end to end through the public API: host buffers, copies timed.
+    # Every step copies its inputs in from pinned host memory and its outputs
+    # (both y) back out; the copies run on their own streams, double
+    # buffered, so that step i's output copy and step i+1's input copy
+    # overlap step i+1's compute (the link is full duplex).
     x_dec_pin = torch.from_numpy(x_dec_h.view(np.int16)).view(torch.bfloat16).pin_memory()
     x_pre_pin = torch.from_numpy(x_pre_h.view(np.int16)).view(torch.bfloat16).pin_memory()
     y_dec_pin = torch.empty((T_DECODE, w.N), dtype=torch.bfloat16).pin_memory()
     y_pre_pin = torch.empty((T_PREFILL, w.N), dtype=torch.bfloat16).pin_memory()
     e2e_steps = max(3, args.steps // 5)
+    h2d_s, d2h_s = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+    xd2 = [x_dec, torch.empty_like(x_dec)]
+    xp2 = [x_pre, torch.empty_like(x_pre)]
+    yd2 = [y_dec, torch.empty_like(y_dec)]
+    yp2 = [y_pre, torch.empty_like(y_pre)]
+    ev_in = [torch.cuda.Event() for _ in range(2)]
+    ev_comp = [torch.cuda.Event() for _ in range(2)]
+    ev_out = [torch.cuda.Event() for _ in range(2)]
 
     def e2e_step(i):
-        x_dec.copy_(x_dec_pin, non_blocking=True)
-        x_pre.copy_(x_pre_pin, non_blocking=True)
-        step(i)
-        y_dec_pin.copy_(y_dec, non_blocking=True)
-        y_pre_pin.copy_(y_pre, non_blocking=True)
+        b = i & 1
+        Lk = layers[i % COPIES]
+        with torch.cuda.stream(h2d_s):
+            if i >= 2:
+                h2d_s.wait_event(ev_comp[b])       # step i-2 has read this input buffer
+            xd2[b].copy_(x_dec_pin, non_blocking=True)
+            xp2[b].copy_(x_pre_pin, non_blocking=True)
+            ev_in[b].record(h2d_s)
+        stream.wait_event(ev_in[b])
+        if i >= 2:
+            stream.wait_event(ev_out[b])           # step i-2's outputs have left this buffer
+        dbf.forward(Lk, xd2[b], y=yd2[b], ws=ws_dec, static_weights=True, stream=stream)
+        dbf.forward(Lk, xp2[b], y=yp2[b], ws=ws_pre, static_weights=True, stream=stream)
+        ev_comp[b].record(stream)
+        with torch.cuda.stream(d2h_s):
+            d2h_s.wait_event(ev_comp[b])
+            y_dec_pin.copy_(yd2[b], non_blocking=True)
+            y_pre_pin.copy_(yp2[b], non_blocking=True)
+            ev_out[b].record(d2h_s)
 
-    with torch.cuda.stream(stream):
-        e2e_step(0)
+    for i in range(2):
+        e2e_step(i)
     torch.cuda.synchronize(dev)
     if world > 1:
         dist.barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with torch.cuda.stream(stream):
-        e0.record(stream)
-        for i in range(e2e_steps):
-            e2e_step(i)
-        e1.record(stream)
+    e0.record(stream)
+    h2d_s.wait_event(e0)
+    d2h_s.wait_event(e0)
+    for i in range(e2e_steps):
+        e2e_step(i)
+    stream.wait_event(ev_out[0])
+    stream.wait_event(ev_out[1])
+    e1.record(stream)
     torch.cuda.synchronize(dev)
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), dev)
     e2e_value = weak_scaling_value(world, tokens_per_step, e2e_steps, e2e_ms)
@@ -751,7 +780,12 @@ def main():
     roof_pre = {"bound": "tensor", "achieved": tfs, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
                 "frac": tfs / pk["bf16_tflops"], "traffic": kernel_traffic("gemm_prefill", "double_binary_rank_b200/csrc/dbf_gemm.cu"),
                 "kernel": "prefill forward (fp16 operand pre-pass + two tcgen05 GEMM launches), one call",
-                "peak_source": f"{pk_kind} bf16 dense (fp16 runs at the same rate)"}
+                "peak_source": f"{pk_kind} bf16 dense burst (fp16 runs at the same rate)"}
+    if pk.get("bf16_tflops_sustained"):
+        # the step loop keeps the tensor cores busy for the whole timed region:
+        # the fraction of the sustained (power-capped) figure, for context
+        roof_pre["peak_sustained"] = pk["bf16_tflops_sustained"]
+        roof_pre["frac_sustained"] = tfs / pk["bf16_tflops_sustained"]
     roof_dec = {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
                 "frac": gbs / pk["hbm_gbs"], "traffic": kernel_traffic("decode", "double_binary_rank_b200/csrc/dbf_decode.cu"),
                 "kernel": f"decode forward ({dec_launches} launch: stage 1, grid barrier, stage 2), one call inside the step",
@@ -796,7 +830,9 @@ def main():
                                      "per fp32 multiply-add"},
         "configs": configs,
         "clocks": clk.summary(),
-        "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "method": "x copied in from pinned host memory and both y copied out every step, on their own "
+                          "streams with double-buffered device tensors (overlapping the next step's compute)"},
         "gpu_launches": args.steps * (dec_launches + pre_launches),
     }
     if world == 1 and not args.no_cpu_baseline:

@@ -88,7 +88,7 @@ struct DecodeParams {
     int bulk_g, bulk_x;           // gamma and x staged by bulk copies (else element by element)
     int gs_bytes, xs_bytes;       // staged gamma, and one token's x buffer (16-byte rounded)
     int gpitch;                   // values per staged gamma row (M rounded up to 8)
-    int tile_ld;                  // int32 per row of the partial-sum tile (8 per column group)
+    int tile_ld;                  // int32 per row of the partial-sum tile (8 per column group, plus 1)
     int off_s2, off_dig, off_tile, off_misc, off_rs1, off_rs2;   // shared-memory offsets
     unsigned long long wait_ns;   // limit of the grid-barrier wait
 };
@@ -860,7 +860,7 @@ bool decode_plan(const dbf_layer &L, int64_t T, int sms, DecodeParams *out, size
     P.max_rb2 = (P.nrb2 + G - 1) / G;
     P.bulk1 = P.pitch1 % 4 == 0;
     P.bulk2 = P.pitch2 % 4 == 0;
-    P.tile_ld = 8 * ((kDigits * P.C + 7) / 8);
+    P.tile_ld = 8 * ((kDigits * P.C + 7) / 8) + 1;   // odd: the epilogue's row-per-lane reads hit distinct banks
     const int rows1 = P.max_rb1 * 16, rows2 = P.max_rb2 * 16;
     const int cbm = P.cb1 > P.cb2 ? P.cb1 : P.cb2;
     // gamma and x are staged in the B1 slice's region (fp32 x: 4 bytes per value)

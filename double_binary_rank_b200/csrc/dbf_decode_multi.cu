@@ -105,7 +105,7 @@ struct DecodeParams {
     int stride1, stride2;         // words per row of the shared slices (stride2 for the largest rank)
     int cb1, cb2;                 // bytes per digit column of u (stage 1) and v (stage 2)
     int rows1, rows2;             // rows of an item at most (multiples of 16)
-    int tile_ld;                  // int32 per tile row (8 per MMA column group)
+    int tile_ld;                  // int32 per tile row (8 per MMA column group, plus 1)
     int gpitch, gs_bytes, xs_bytes;   // staged gamma (values per row, bytes) and one token's x buffer
     int stage_g;                  // gamma staged in shared memory (else read from global memory: no room)
     int word2;                    // stage 2 in the per-word layout (small ranks, see digit_offset_word)
@@ -1220,7 +1220,7 @@ size_t smem_layout(DecodeParams &P)
     off = align_up(off + static_cast<size_t>(kDigits) * ccmax * cbm, 128);
     P.off_tile = static_cast<int>(off);
     const int rmax = P.rows1 > P.rows2 ? P.rows1 : P.rows2;
-    P.tile_ld = 8 * ((kDigits * ccmax + 7) / 8);
+    P.tile_ld = 8 * ((kDigits * ccmax + 7) / 8) + 1;   // odd: the epilogue's row-per-lane reads hit distinct banks
     off = align_up(off + static_cast<size_t>(rmax) * P.tile_ld * 4, 16);
     P.off_misc = static_cast<int>(off);
     off = align_up(off + sizeof(Misc), 16);
