@@ -12,10 +12,10 @@
 // Persistent kernel, one CTA per SM; each CTA walks 128 x 256 tiles of
 // D = A B^T (A: 128 sign rows, B: 256 token rows) with two 256-column
 // accumulators in tensor memory, so the epilogue of one tile overlaps the
-// K loop of the next. Warp roles of the forward instance (FwdCfg below; the
-// backward instance has one expansion group and eight epilogue warps):
+// K loop of the next. Warp roles (FwdCfg below, the single-CTA instance used
+// by the grouped, MBOK and dense products):
 //   warp 0       TMA producer: fp16 activation tiles (64 K x 256 rows,
-//                128-byte swizzle) into a 4-stage ring;
+//                128-byte swizzle) into a ring of SB stages;
 //   warp 1       allocates 512 TMEM columns; one thread issues tcgen05.mma
 //                (M = 128, N = 256, K = 16) into the free accumulator and
 //                commits each stage back;
@@ -27,10 +27,17 @@
 //                +-1 (or +-alpha) pairs -- a shift and one LOP3 per two
 //                signs, the packed layout keeping columns 2p and 2p+1 in bits
 //                p and 16+p -- written in the same 128-byte swizzled K-major
-//                layout into a 6-stage ring;
+//                layout into a ring of SA stages;
 //   warps 10..13 epilogue, one per TMEM lane quarter: tcgen05.ld of a
 //                finished accumulator, scaling, stores, then the accumulator
 //                is handed back to the MMA warp.
+// The forward stages (FwdPairCfg) and the backward sign GEMMs (BwdPairCfg:
+// one expansion group, eight epilogue warps) run on CTA pairs: clusters of
+// two CTAs, tcgen05 cta_group::2 with M = 256 over the pair, each CTA
+// expanding its 128 sign rows and loading half of the token tile (2-SM TMA
+// loads without multicast, counted by the leader CTA's barrier); the leader
+// issues the MMAs and commits to both CTAs' barriers, and each CTA's tensor
+// memory holds its 128 rows of the 256 x 256 accumulator.
 // Every wait is bounded; on expiry the CTA records DBF_ERR_TIMEOUT and stops
 // issuing work; before it frees its tensor memory and ends, the TMA loads
 // and MMAs it already issued are waited for (bounded as well).
@@ -69,7 +76,7 @@ struct GemmCfg {
 };
 using FwdCfg = GemmCfg<2, 6, 4, 4, false>;
 using FwdPairCfg = GemmCfg<2, 6, 6, 4, false, true>;
-using BwdCfg = GemmCfg<1, 4, 5, 8, true>;
+using BwdPairCfg = GemmCfg<1, 4, 8, 8, true, true>;
 constexpr int kMaxStages = 8;
 constexpr int A_BYTES = BM * BK * 2;   // 16 KB
 constexpr int TMEM_COLS = 512;          // two 256-column accumulators
@@ -1304,29 +1311,31 @@ cudaError_t gemm_backward(const dbf_layer &L, const uint32_t *b1t, const uint32_
     if ((e = scale_cast(x, xd, L.gamma, L.M, T, ell, U, s)) != cudaSuccess) return e;
     if ((e = scale_cast(dy, dyd, L.alpha, L.N, T, ell, A, s)) != cudaSuccess) return e;
     CUtensorMap mu, ma, mvh, mvg;
-    if (!make_map(&mu, U, L.M, C) || !make_map(&ma, A, L.N, C) || !make_map(&mvh, Vh, L.R, C) ||
-        !make_map(&mvg, Vg, L.R, C))
+    // the four sign GEMMs run on CTA pairs (each CTA loads half of a token tile)
+    constexpr int kb = BwdPairCfg::kBRows;
+    if (!make_map(&mu, U, L.M, C, kb) || !make_map(&ma, A, L.N, C, kb) || !make_map(&mvh, Vh, L.R, C, kb) ||
+        !make_map(&mvg, Vg, L.R, C, kb))
         return cudaErrorInvalidValue;
     // G3
     GemmArgs g3 = sign_gemm_args(L.b2_packed, L.R, L.M, C, Ti, ell, 3);
     g3.H32 = H32;
     g3.Vout = Vh;
     g3.cscale = L.beta;
-    if ((e = launch_gemm<BwdCfg>(mu, g3, s, nullptr, st)) != cudaSuccess) return e;
+    if ((e = launch_gemm_pair<BwdPairCfg>(mu, g3, s, st)) != cudaSuccess) return e;
     // G4
     GemmArgs g4 = sign_gemm_args(b1t, L.R, L.N, C, Ti, ell, 4);
     g4.H32 = H32;
     g4.Vout = Vg;
     g4.cscale = L.beta;
     g4.red = dbeta;
-    if ((e = launch_gemm<BwdCfg>(ma, g4, s, nullptr, st)) != cudaSuccess) return e;
+    if ((e = launch_gemm_pair<BwdPairCfg>(ma, g4, s, st)) != cudaSuccess) return e;
     // G5
     if (dalpha) {
         GemmArgs g5 = sign_gemm_args(L.b1_packed, L.N, L.R, C, Ti, ell, 5);
         g5.red = dalpha;
         g5.W = dy;
         g5.wd = dyd;
-        if ((e = launch_gemm<BwdCfg>(mvh, g5, s, nullptr, st)) != cudaSuccess) return e;
+        if ((e = launch_gemm_pair<BwdPairCfg>(mvh, g5, s, st)) != cudaSuccess) return e;
     }
     // G6
     if (dx || dgamma) {
@@ -1337,7 +1346,7 @@ cudaError_t gemm_backward(const dbf_layer &L, const uint32_t *b1t, const uint32_
         g6.cscale = L.gamma;
         g6.dx = dx;
         g6.dx_mode = ell > 1 ? 2 : (acc ? 1 : 0);
-        if ((e = launch_gemm<BwdCfg>(mvg, g6, s, nullptr, st)) != cudaSuccess) return e;
+        if ((e = launch_gemm_pair<BwdPairCfg>(mvg, g6, s, st)) != cudaSuccess) return e;
     }
     // sign-matrix gradients: dB1 = sum_c a_c v_c^T (N x R), dB2 = sum_c w_c u_c^T
     // (R x M), dense products contracting over the envelope-major token index
