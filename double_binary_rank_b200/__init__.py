@@ -11,7 +11,7 @@ from __future__ import annotations
 import ctypes
 import os
 from dataclasses import dataclass
-from typing import List, Optional, Sequence
+from typing import List, Optional, Sequence, Tuple
 
 import numpy as np
 import torch
@@ -81,6 +81,7 @@ _SIGS = {
     "dbf_forward_decode_noalloc": (ctypes.c_int, [_LP, _vp, ctypes.c_int, _vp, ctypes.c_int, _i64,
                                                   ctypes.c_int, _vp]),
     "dbf_debug_set_decode_wait_ns": (None, [ctypes.c_uint64]),
+    "dbf_debug_noalloc_header": (ctypes.c_int, [ctypes.POINTER(ctypes.c_uint64), ctypes.POINTER(ctypes.c_int32)]),
     "dbf_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "dbf_version": (ctypes.c_char_p, []),
 }
@@ -232,6 +233,15 @@ def debug_set_decode_wait_ns(ns: int) -> None:
     """Time limit of the single-launch decode kernel's bounded waits for later
     calls (0 restores the default of 2 s); for tests of the timeout path."""
     _lib.dbf_debug_set_decode_wait_ns(int(ns))
+
+
+def debug_noalloc_header() -> Tuple[int, int]:
+    """(barrier word, status) of the fixed array dbf_forward_decode_noalloc
+    uses on the current device; waits for all work on the device."""
+    word = ctypes.c_uint64(0)
+    status = ctypes.c_int32(0)
+    _check(_lib.dbf_debug_noalloc_header(ctypes.byref(word), ctypes.byref(status)), "dbf_debug_noalloc_header")
+    return int(word.value), int(status.value)
 
 
 def _flags(accumulate: bool, static_weights: bool) -> int:

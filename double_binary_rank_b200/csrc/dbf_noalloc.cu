@@ -24,6 +24,7 @@
 // runs concurrently) race on the array; callers must order them.
 #include "dbf_internal.cuh"
 
+#include <cstring>
 #include <mutex>
 
 namespace dbf {
@@ -85,6 +86,19 @@ dbf_status dbf_forward_decode_noalloc(const dbf_layer *L, const void *x, dbf_dty
                    cudaSuccess
                ? DBF_OK
                : DBF_ERR_CUDA;
+}
+
+dbf_status dbf_debug_noalloc_header(uint64_t *barrier_word, int32_t *status)
+{
+    using namespace dbf;
+    if (!barrier_word || !status) return DBF_ERR_INVALID_ARG;
+    void *scratch = nullptr;
+    if (scratch_address(&scratch) != cudaSuccess) return DBF_ERR_CUDA;
+    unsigned char h[kWsStatusOffset + sizeof(int32_t)];
+    if (cudaMemcpy(h, scratch, sizeof h, cudaMemcpyDeviceToHost) != cudaSuccess) return DBF_ERR_CUDA;
+    std::memcpy(barrier_word, h, sizeof(uint64_t));
+    std::memcpy(status, h + kWsStatusOffset, sizeof(int32_t));
+    return DBF_OK;
 }
 
 }  // extern "C"

@@ -409,6 +409,17 @@ dbf_status dbf_forward_segmented(const dbf_layer *adapters_dev, int32_t num_adap
 dbf_status dbf_forward_decode_noalloc(const dbf_layer *L, const void *x, dbf_dtype x_dtype, void *y,
                                       dbf_dtype y_dtype, int64_t T, int flags, void *stream);
 
+/* Reads the workspace header of the fixed array that
+ * dbf_forward_decode_noalloc uses on the current device: the grid-barrier
+ * word (arrival count in the low 32 bits, epoch in the high 32 bits) into
+ * *barrier_word and the int32 device status into *status. A synchronous
+ * device-to-host copy: it waits for all work on the device. For tests and
+ * diagnosis (the count is zero between calls; the status holds
+ * DBF_ERR_TIMEOUT after a call whose wait expired); not for the hot path.
+ * Errors: DBF_ERR_INVALID_ARG for a null pointer, DBF_ERR_CUDA if the
+ * address lookup or the copy fails. */
+dbf_status dbf_debug_noalloc_header(uint64_t *barrier_word, int32_t *status);
+
 /* Time limit of the grid-barrier wait of the single-launch decode kernel
  * for the calls made after this one, in this process, counted from each
  * CTA's start and checked before every poll: ns > 0 sets it, 0 restores the

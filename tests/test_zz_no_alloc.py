@@ -45,6 +45,11 @@ def test_noalloc_matches_forward_twice():
         got = host_y(y)
         assert rel_err(got, host_y(ref)) < TOL
         assert rel_err(got, oracle.forward(L, xh)) < TOL
+    # between calls the array's header holds a barrier word with no arrivals
+    # pending (the epoch moved on) and a clean status word
+    word, status = dbf.debug_noalloc_header()
+    assert word & 0xFFFFFFFF == 0 and word >> 32 > 0 and status == 0
+    epoch = word >> 32
     # a layer wider than the single launch takes (M > 8192): the two-launch
     # path through the same array, then a single launch again
     Lw = random_layer(rng, 8224, 256, 96, 1)
@@ -66,6 +71,8 @@ def test_noalloc_matches_forward_twice():
     torch.cuda.synchronize()
     assert rel_err(host_y(y2), host_y(ref2)) < TOL
     assert rel_err(host_y(y2), oracle.forward(L2, x2h)) < TOL
+    word, status = dbf.debug_noalloc_header()
+    assert word & 0xFFFFFFFF == 0 and word >> 32 > epoch and status == 0
 
 
 def test_noalloc_rejects_calls_beyond_its_scratch():
