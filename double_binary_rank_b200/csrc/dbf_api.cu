@@ -187,7 +187,7 @@ int32_t dbf_forward_launches(const dbf_layer *L, int64_t T, dbf_path path)
     if (path != DBF_PATH_AUTO && path != DBF_PATH_GEMV && path != DBF_PATH_GEMM) return 0;
     if (T == 0) return 0;
     const dbf_path p = resolve(*L, T, path);
-    if (p == DBF_PATH_GEMM) return gemm_shape_ok(*L) ? 3 : 0;
+    if (p == DBF_PATH_GEMM) return gemm_shape_ok(*L) ? gemm_forward_launches(*L) : 0;
     return gemv_launches(*L, T);
 }
 

@@ -44,7 +44,12 @@
 #include "dbf_internal.cuh"
 
 #include <cuda.h>
+#include <algorithm>
+#include <map>
 #include <mutex>
+#include <queue>
+#include <tuple>
+#include <vector>
 #include <cudaTypedefs.h>
 
 namespace dbf {
@@ -58,9 +63,10 @@ constexpr int BK = 64;              // K per stage: one 128-byte swizzle row of 
 // backward, whose epilogues read and write an operand per element, takes
 // eight epilogue warps (two per TMEM lane quarter, each with half of the
 // columns) and one expansion group.
-template <int kGroups, int kSA, int kSB, int kEpi, bool kBackward, bool kPairMode = false>
+template <int kGroups, int kSA, int kSB, int kEpi, bool kBackward, bool kPairMode = false, bool kFusedMode = false>
 struct GemmCfg {
     static constexpr bool kBwd = kBackward;      // epilogues of stages 3..6 compiled in
+    static constexpr bool kFused = kFusedMode;   // both forward stages in one launch (gemm_fused_kernel)
     // CTA pairs (a cluster of two): tcgen05 cta_group::2 with M = 256 over the
     // two SMs; each CTA holds its 128 sign rows of A and half of the 256 token
     // rows of B, and its TMEM the accumulator of its 128 rows
@@ -76,6 +82,7 @@ struct GemmCfg {
 };
 using FwdCfg = GemmCfg<2, 6, 4, 4, false>;
 using FwdPairCfg = GemmCfg<2, 6, 6, 4, false, true>;
+using FusedCfg = GemmCfg<2, 6, 6, 4, false, true, true>;
 using BwdPairCfg = GemmCfg<1, 4, 8, 8, true, true>;
 constexpr int kMaxStages = 8;
 constexpr int A_BYTES = BM * BK * 2;   // 16 KB
@@ -375,8 +382,12 @@ __device__ __forceinline__ uint32_t sign_pair(uint32_t w, int p, uint32_t mag2)
     return ((w << (15 - p)) & 0x80008000u) ^ mag2;
 }
 
+constexpr int kRing = 4;   // tile ring of the fused forward: entries in flight
+
 struct GemmSmem {
     uint64_t full_a[kMaxStages], empty_a[kMaxStages], full_b[kMaxStages], empty_b[kMaxStages], acc_full[2], acc_empty[2];
+    uint64_t tfull[kRing], tempty[kRing];   // fused forward: tile ring entries posted / given back
+    int ring[kRing];
     uint64_t drain;   // the MMA thread's last commit: every MMA it issued has completed
     uint64_t exit_bar;   // CTA pairs: the peer is done with this CTA's shared memory
     uint32_t tmem_base;
@@ -491,16 +502,153 @@ __device__ __forceinline__ void backward_chunk(const GemmArgs &g, const uint32_t
     if (g.red && i < g.ell && part != 0.f) atomicAdd(g.red + static_cast<int64_t>(i) * g.P + p, part);
 }
 
+// ---- the forward's two stages in one launch ---------------------------------
+// Stage-1 tiles (B2 rows x columns of u) come first, then the stage-2 tiles
+// (B1 rows x tokens), the last nh of them as two halves of 128 tokens so
+// that the last tiles to run are short. A pair takes its first tile by its
+// index and every later one from a claim counter, one tile ahead of the tile
+// it starts, so that the pairs that finish first take the remaining tiles;
+// CTA 0's producer posts each claimed tile in a ring of kRing entries in both
+// CTAs' shared memory, from which every role reads it. A stage-2 tile loads
+// rows of v that the stage-1 epilogues of other pairs write: each stage-1
+// epilogue warp counts its finished tile on the flag of the tile's column
+// block, and a producer loads v only once the flags of every block its tokens
+// need are complete (bounded wait). Tiles are claimed in order and a pair
+// only claims while it runs, so every stage-1 tile a stage-2 tile waits for
+// is held by a running pair that does not wait itself.
+struct FusedSched {
+    int n1, n2f, nh;         // stage-1 tiles; stage-2 tiles run whole; stage-2 tiles run as two halves
+    int n_p1, n_p2;          // pair row tiles per column block in stages 1 and 2
+    unsigned *ctr;           // claim counter (zeroed by the pre-pass)
+    unsigned *flags;         // per stage-1 column block: finished epilogue warps (zeroed by the pre-pass)
+    unsigned flag_target;    // arrivals that complete a column block
+};
+
+struct FusedTile {
+    int stage, t, half;      // half: -1 for a whole tile, else which 128 tokens of tile t
+};
+
+__device__ __forceinline__ FusedTile fused_decode(const FusedSched &fs, int u)
+{
+    FusedTile f;
+    if (u < fs.n1) {
+        f.stage = 1;
+        f.t = u;
+        f.half = -1;
+    } else if (u < fs.n1 + fs.n2f) {
+        f.stage = 2;
+        f.t = u - fs.n1;
+        f.half = -1;
+    } else {
+        const int h = u - fs.n1 - fs.n2f;
+        f.stage = 2;
+        f.t = fs.n2f + (h >> 1);
+        f.half = h & 1;
+    }
+    return f;
+}
+
+// Instruction descriptor of a half tile: M = 256 over the pair, N = 128.
+constexpr uint32_t kIdescPairHalf = (1u << 4) | (static_cast<uint32_t>(128 >> 3) << 17) | (static_cast<uint32_t>((2 * BM) >> 4) << 24);
+
+__device__ __forceinline__ void mma_f16_pair_n(uint32_t tmem_d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+        "l"(a), "l"(b), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// Wait with acquire at cluster scope (the ring's entries are written by CTA 0).
+__device__ __forceinline__ bool bar_try_cluster(uint64_t *bar, uint32_t parity)
+{
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return done != 0;
+}
+
+// Release-arrive on the barrier at shared::cluster address 'addr'.
+__device__ __forceinline__ void bar_arrive_cluster_addr(uint32_t addr)
+{
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(addr) : "memory");
+}
+
+__device__ __forceinline__ uint32_t peer_addr(const void *p, uint32_t rank)
+{
+    uint32_t a;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(a) : "r"(smem_u32(p)), "r"(rank));
+    return a;
+}
+
+__device__ __forceinline__ unsigned ld_acquire_u32(const unsigned *p)
+{
+    unsigned v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// Bounded wait with acquire at cluster scope; false (and the abort flag
+// raised) when the limit passes or another role already aborted.
+__device__ __forceinline__ bool bar_wait_cluster(uint64_t *bar, uint32_t parity, volatile int *abort)
+{
+    if (bar_try_cluster(bar, parity)) return true;
+    const unsigned long long t0 = global_ns();
+    while (true) {
+        if (bar_try_cluster(bar, parity)) return true;
+        if (*abort) return false;
+        if (global_ns() - t0 > kWaitNs) {
+            *abort = 1;
+            return false;
+        }
+    }
+}
+
+// Entry j of the pair's tile ring (one thread): the claimed tile, -1 after
+// the last one; false when the wait expired or another role aborted. The
+// slot is handed back to CTA 0's producer once read.
+__device__ __forceinline__ bool ring_get(GemmSmem *sh, int j, int &u)
+{
+    const int s = j % kRing;
+    if (!bar_wait_cluster(&sh->tfull[s], (j / kRing) & 1, &sh->abort)) return false;
+    u = *reinterpret_cast<volatile int *>(&sh->ring[s]);
+    bar_arrive_cluster_addr(pair_leader_addr(&sh->tempty[s]));
+    return true;
+}
+
+// The same for a whole warp: lane 0 reads, every lane gets the entry.
+__device__ __forceinline__ bool ring_get_warp(GemmSmem *sh, int j, int &u)
+{
+    int v = -1;
+    int ok = 1;
+    if ((threadIdx.x & 31) == 0) ok = ring_get(sh, j, v) ? 1 : 0;
+    u = __shfl_sync(0xffffffffu, v, 0);
+    return __shfl_sync(0xffffffffu, ok, 0) != 0;
+}
+
 // Persistent: CTA b takes tiles b, b + gridDim.x, ... (token-tile major, so
-// the CTAs running together share activation tiles in L2).
+// the CTAs running together share activation tiles in L2); in the fused
+// forward (g2 and fs given) the pairs claim tiles instead (see above), tmB
+// being the map of u and tmA the map of v.
 template <class Cfg>
-__global__ void __launch_bounds__(Cfg::kThreads, 1) gemm_kernel(const __grid_constant__ CUtensorMap tmB,
-                                                                const __grid_constant__ CUtensorMap tmA, const __grid_constant__ GemmArgs g)
+__device__ __forceinline__ void gemm_body(const CUtensorMap &tmB, const CUtensorMap &tmA, const GemmArgs &g,
+                                          const GemmArgs *g2, const FusedSched *fs)
 {
     constexpr int SA = Cfg::SA, SB = Cfg::SB, kExpandGroups = Cfg::kExpandGroups;
     constexpr int kExpandWarps = Cfg::kExpandWarps, kEpiWarps = Cfg::kEpiWarps;
+    constexpr bool kFused = Cfg::kFused;
     static_assert(SA <= kMaxStages && SB <= kMaxStages && kEpiWarps % 4 == 0 && BN % (32 * (kEpiWarps / 4)) == 0,
                   "pipeline shape");
+    static_assert(!kFused || (Cfg::kPair && !Cfg::kBwd && kEpiWarps == 4), "the fused forward runs on CTA pairs");
     extern __shared__ uint8_t smem_raw[];
     // 1024-byte alignment for the swizzled tiles
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -525,6 +673,9 @@ __global__ void __launch_bounds__(Cfg::kThreads, 1) gemm_kernel(const __grid_con
     const int my_tiles = unit < ntiles ? (ntiles - 1 - unit) / nunits + 1 : 0;
     const int nk = g.Ktot / BK;
     auto wait = [&](uint64_t *bar, uint32_t parity) { return bar_wait(bar, parity, abort); };
+    // the fused forward's view of a claimed tile: its stage's arguments, row
+    // tiles per column block, tile index and half
+    auto fused_args = [&](const FusedTile &f) -> const GemmArgs & { return f.stage == 1 ? g : *g2; };
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < SA; ++i) {
@@ -540,12 +691,21 @@ __global__ void __launch_bounds__(Cfg::kThreads, 1) gemm_kernel(const __grid_con
             bar_init(&sh->acc_full[i], 1);
             bar_init(&sh->acc_empty[i], kPair ? 2 * kEpiWarps : kEpiWarps);
         }
+        if (kFused) {
+            // every reader of the ring in both CTAs gives each entry back: the
+            // MMA thread of CTA 0, the producer of CTA 1, and the expansion and
+            // epilogue warps of both
+            for (int i = 0; i < kRing; ++i) {
+                bar_init(&sh->tfull[i], 1);
+                bar_init(&sh->tempty[i], 2 + 2 * (kExpandWarps + kEpiWarps));
+            }
+        }
         bar_init(&sh->drain, 1);
         bar_init(&sh->exit_bar, 1);
         sh->abort = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         asm volatile("prefetch.tensormap [%0];" ::"l"(&tmB) : "memory");
-        if (g.dense_a) asm volatile("prefetch.tensormap [%0];" ::"l"(&tmA) : "memory");
+        if (g.dense_a || kFused) asm volatile("prefetch.tensormap [%0];" ::"l"(&tmA) : "memory");
     }
     if (warp == 1) {
         if (kPair) {
@@ -573,31 +733,105 @@ __global__ void __launch_bounds__(Cfg::kThreads, 1) gemm_kernel(const __grid_con
         if (lane == 0) {
             int s = 0;
             int nb_issued = 0, na_issued = 0;   // TMA loads issued on each ring
-            for (int j = 0; j < my_tiles && !*abort; ++j) {
-                const TileRef tr = tile_ref(g, unit + j * nunits, n_p, tile_rank);
-                const int c0 = tr.brow;
-                const int p0 = tr.p0;
-                for (int k = 0; k < nk; ++k, ++s) {
-                    const int st = s % SB;
-                    if (!wait(&sh->empty_b[st], ((s / SB) & 1) ^ 1)) break;
-                    if (kPair) {
-                        // CTA 0's barrier counts the bytes of both halves of B
-                        if (rank == 0) bar_expect_tx(&sh->full_b[st], 2 * kBBytes);
-                        tma_load_2d_pair(smB + st * kBBytes, &tmB, k * BK, c0 + static_cast<int>(rank) * Cfg::kBRows,
-                                         &sh->full_b[st]);
-                    } else {
-                        bar_expect_tx(&sh->full_b[st], kBBytes);
-                        tma_load_2d(smB + st * kBBytes, &tmB, k * BK, c0, &sh->full_b[st]);
+            if (kFused) {
+                const int total = fs->n1 + fs->n2f + 2 * fs->nh;
+                // CTA 0 claims tile k of the pair and posts it in both rings
+                // (-1: no tile left); -2 when the ring wait gave up
+                auto claim = [&](int k) -> int {
+                    const int sl = k % kRing;
+                    if (!bar_wait_cluster(&sh->tempty[sl], ((k / kRing) & 1) ^ 1, abort)) return -2;
+                    int u = k == 0 ? unit : nunits + static_cast<int>(atomicAdd(fs->ctr, 1u));
+                    if (u >= total) u = -1;
+                    *reinterpret_cast<volatile int *>(&sh->ring[sl]) = u;
+                    const uint32_t peer_ring = peer_addr(&sh->ring[sl], 1u);
+                    asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(peer_ring), "r"(u) : "memory");
+                    bar_arrive_cluster_addr(smem_u32(&sh->tfull[sl]));
+                    bar_arrive_cluster_addr(peer_addr(&sh->tfull[sl], 1u));
+                    return u;
+                };
+                // the pair's first tile is its index: posted before the wait for
+                // the pre-pass, so that the sign expansion starts meanwhile
+                int u = -1;
+                if (rank == 0) u = claim(0);
+                griddep_wait();   // u and the claim state come from the pre-pass launched before
+                if (rank != 0 && !ring_get(sh, 0, u)) u = -1;
+                for (int j = 0; u >= 0 && !*abort; ++j) {
+                    int un = -1;   // the pair's next tile, claimed (CTA 0) or read (CTA 1) one tile ahead
+                    if (rank == 0) {
+                        un = claim(j + 1);
+                        if (un == -2) break;
                     }
-                    nb_issued = s + 1;
-                    if (g.dense_a) {
-                        // a dense fp16 A operand: its tile comes by TMA too, in the
-                        // same swizzled K-major layout the expansion writes
-                        const int sa = s % SA;
-                        if (!bar_wait(&sh->empty_a[sa], ((s / SA) & 1) ^ 1, abort)) break;
-                        bar_expect_tx(&sh->full_a[sa], A_BYTES);
-                        tma_load_2d(smA + sa * A_BYTES, &tmA, k * BK, p0, &sh->full_a[sa]);
-                        na_issued = s + 1;
+                    const FusedTile f = fused_decode(*fs, u);
+                    const GemmArgs &gs = fused_args(f);
+                    const TileRef tr = tile_ref(gs, f.t, f.stage == 1 ? fs->n_p1 : fs->n_p2, tile_rank);
+                    const int c0 = tr.brow + (f.half > 0 ? 128 : 0);
+                    const int brows = f.half >= 0 ? 64 : 128;   // B rows this CTA supplies
+                    const CUtensorMap *mp = f.stage == 1 ? &tmB : &tmA;
+                    bool ok = true;
+                    if (f.stage == 2 && c0 < g.T) {
+                        // the v rows of tokens [c0, t_hi) of every envelope: stage-1
+                        // column blocks (i T + t) / BN
+                        const int t_hi = min(c0 + 2 * brows, g.T);
+                        const unsigned long long t0 = global_ns();
+                        for (int i = 0; i < g.ell && ok; ++i) {
+                            const int b_lo = (i * g.T + c0) / BN, b_hi = (i * g.T + t_hi - 1) / BN;
+                            for (int b = b_lo; b <= b_hi && ok; ++b) {
+                                while (ld_acquire_u32(fs->flags + b) < fs->flag_target) {
+                                    if (*abort) { ok = false; break; }
+                                    if (global_ns() - t0 > kWaitNs) {
+                                        *abort = 1;
+                                        ok = false;
+                                        break;
+                                    }
+                                }
+                            }
+                        }
+                        // v was written through the generic proxy; the loads below use the async one
+                        asm volatile("fence.proxy.async.global;" ::: "memory");
+                    }
+                    if (!ok) break;
+                    const int nk_t = gs.Ktot / BK;
+                    for (int k = 0; k < nk_t; ++k, ++s) {
+                        const int st = s % SB;
+                        if (!wait(&sh->empty_b[st], ((s / SB) & 1) ^ 1)) break;
+                        if (rank == 0) bar_expect_tx(&sh->full_b[st], 2 * kBBytes);
+                        tma_load_2d_pair(smB + st * kBBytes, mp, k * BK, c0 + static_cast<int>(rank) * brows,
+                                         &sh->full_b[st]);
+                        nb_issued = s + 1;
+                    }
+                    if (rank == 0) {
+                        u = un;
+                    } else if (!ring_get(sh, j + 1, u)) {
+                        break;
+                    }
+                }
+            } else {
+                for (int j = 0; j < my_tiles && !*abort; ++j) {
+                    const TileRef tr = tile_ref(g, unit + j * nunits, n_p, tile_rank);
+                    const int c0 = tr.brow;
+                    const int p0 = tr.p0;
+                    for (int k = 0; k < nk; ++k, ++s) {
+                        const int st = s % SB;
+                        if (!wait(&sh->empty_b[st], ((s / SB) & 1) ^ 1)) break;
+                        if (kPair) {
+                            // CTA 0's barrier counts the bytes of both halves of B
+                            if (rank == 0) bar_expect_tx(&sh->full_b[st], 2 * kBBytes);
+                            tma_load_2d_pair(smB + st * kBBytes, &tmB, k * BK, c0 + static_cast<int>(rank) * Cfg::kBRows,
+                                             &sh->full_b[st]);
+                        } else {
+                            bar_expect_tx(&sh->full_b[st], kBBytes);
+                            tma_load_2d(smB + st * kBBytes, &tmB, k * BK, c0, &sh->full_b[st]);
+                        }
+                        nb_issued = s + 1;
+                        if (g.dense_a) {
+                            // a dense fp16 A operand: its tile comes by TMA too, in the
+                            // same swizzled K-major layout the expansion writes
+                            const int sa = s % SA;
+                            if (!bar_wait(&sh->empty_a[sa], ((s / SA) & 1) ^ 1, abort)) break;
+                            bar_expect_tx(&sh->full_a[sa], A_BYTES);
+                            tma_load_2d(smA + sa * A_BYTES, &tmA, k * BK, p0, &sh->full_a[sa]);
+                            na_issued = s + 1;
+                        }
                     }
                 }
             }
@@ -616,13 +850,24 @@ __global__ void __launch_bounds__(Cfg::kThreads, 1) gemm_kernel(const __grid_con
         if (lane == 0 && (!kPair || rank == 0)) {
             int s = 0;
             bool ok = true;
-            for (int j = 0; j < my_tiles && ok; ++j) {
+            for (int j = 0; ok; ++j) {
+                int nk_t = nk;
+                uint32_t idesc = kIdescPair;
+                if (kFused) {
+                    int u = -1;
+                    if (!ring_get(sh, j, u) || u < 0) break;
+                    const FusedTile f = fused_decode(*fs, u);
+                    nk_t = fused_args(f).Ktot / BK;
+                    if (f.half >= 0) idesc = kIdescPairHalf;
+                } else if (j >= my_tiles) {
+                    break;
+                }
                 const int ab = j & 1;
                 ok = wait(&sh->acc_empty[ab], ((j >> 1) & 1) ^ 1);
                 if (!ok) break;
                 tc_fence_after();
                 const uint32_t dt = tmem + static_cast<uint32_t>(ab * BN);
-                for (int k = 0; k < nk; ++k, ++s) {
+                for (int k = 0; k < nk_t; ++k, ++s) {
                     const int sa = s % SA, sb = s % SB;
                     ok = wait(&sh->full_a[sa], (s / SA) & 1) && wait(&sh->full_b[sb], (s / SB) & 1);
                     if (!ok) break;
@@ -632,7 +877,7 @@ __global__ void __launch_bounds__(Cfg::kThreads, 1) gemm_kernel(const __grid_con
                     if (kPair) {
 #pragma unroll
                         for (int kk = 0; kk < BK / 16; ++kk)
-                            mma_f16_pair(dt, da + 2 * kk, db + 2 * kk, (k | kk) != 0);
+                            mma_f16_pair_n(dt, da + 2 * kk, db + 2 * kk, idesc, (k | kk) != 0);
                         mma_commit_pair_both(&sh->empty_a[sa]);   // both CTAs' stages are free again
                         mma_commit_pair_both(&sh->empty_b[sb]);
                     } else {
@@ -661,70 +906,93 @@ __global__ void __launch_bounds__(Cfg::kThreads, 1) gemm_kernel(const __grid_con
         // each thread of a group owns one tile row.
         const int grp = (warp - 2) >> 2;
         const int prow = ((warp - 2) & 3) * 32 + lane;
-        const int npairs = nk / 2;                 // pairs of K steps (K is a multiple of 128)
-        const int total_pairs = my_tiles * npairs;
-        const int env_words = g.Kp / 32;           // packed words of one envelope block of K
         const uint32_t swz = static_cast<uint32_t>(prow & 7) << 4;
-        // cursor over this CTA's (tile, pair) sequence, advanced without divisions
+        // cursor over this CTA's (tile, pair) sequence, advanced without
+        // divisions; calive turns false past the last tile
         int cj = 0, cpair = 0, cword = 0, cenv = 0, cgrow = 0, cbase = 0;   // cbase: first word of the envelope block
+        int cnpairs = nk / 2;                     // pairs of K steps of the tile (K is a multiple of 128)
+        int cenv_words = g.Kp / 32;               // packed words of one envelope block of K
+        const GemmArgs *cg = &g;                  // the tile's arguments (fused: its stage's)
         const uint32_t *crow = nullptr;
-        bool cvalid = false;
+        bool cvalid = false, calive = true;
         uint32_t cmag = 0u;
         const uint16_t *carow = g.arow_scale;
         auto seat_mag = [&]() {
             if (carow) {
-                const uint32_t a = cvalid ? __ldg(carow + static_cast<int64_t>(cenv) * g.N + cgrow) : 0u;
+                const uint32_t a = cvalid ? __ldg(carow + static_cast<int64_t>(cenv) * cg->N + cgrow) : 0u;
                 cmag = a | (a << 16);
             } else {
                 cmag = cvalid ? 0x3C003C00u : 0u;   // +-1
             }
         };
         auto seat_tile = [&]() {
-            const TileRef tr = tile_ref(g, unit + cj * nunits, n_p, tile_rank);
+            int t = unit + cj * nunits, np = n_p;
+            if (kFused) {
+                int u = -1;
+                if (!ring_get_warp(sh, cj, u) || u < 0) {
+                    calive = false;
+                    return;
+                }
+                const FusedTile f = fused_decode(*fs, u);
+                cg = &fused_args(f);
+                np = f.stage == 1 ? fs->n_p1 : fs->n_p2;
+                t = f.t;
+                cnpairs = cg->Ktot / (2 * BK);
+                cenv_words = cg->Kp / 32;
+            } else if (cj >= my_tiles) {
+                calive = false;
+                return;
+            }
+            const TileRef tr = tile_ref(*cg, t, np, tile_rank);
             cgrow = tr.p0 + prow;
-            cvalid = cgrow < g.P;
-            carow = tr.gr ? tr.gr->arow : g.arow_scale;
-            crow = (tr.gr ? tr.gr->signs : g.signs) + static_cast<int64_t>(cvalid ? cgrow : 0) * g.pitch;
+            cvalid = cgrow < cg->P;
+            carow = tr.gr ? tr.gr->arow : cg->arow_scale;
+            crow = (tr.gr ? tr.gr->signs : cg->signs) + static_cast<int64_t>(cvalid ? cgrow : 0) * cg->pitch;
             seat_mag();
         };
         auto advance = [&]() {
-            if (++cpair == npairs) {
+            if (!calive) return;
+            if (++cpair == cnpairs) {
                 cpair = 0;
                 cword = 0;
                 cenv = 0;
                 cbase = 0;
-                if (++cj < my_tiles) seat_tile();
+                ++cj;
+                seat_tile();
             } else {
                 cword += 4;
-                if (cword == env_words) {
+                if (cword == cenv_words) {
                     cword = 0;
                     ++cenv;
-                    cbase += g.env_advance ? env_words : 0;   // a new block of the row, or the same row again
+                    cbase += cg->env_advance ? cenv_words : 0;   // a new block of the row, or the same row again
                     seat_mag();
                 }
             }
         };
         // this row's four words of the cursor's pair (two K steps) and the
         // magnitude pattern of its envelope block; then move on to the group's
-        // next pair
-        auto fetch = [&](uint4 &w, uint32_t &mag) {
+        // next pair. False when the cursor is past the last tile.
+        auto fetch = [&](uint4 &w, uint32_t &mag) -> bool {
+            if (!calive) return false;
             w = cvalid ? __ldg(reinterpret_cast<const uint4 *>(crow + cbase + cword)) : make_uint4(0u, 0u, 0u, 0u);
             mag = cmag;
 #pragma unroll
             for (int e = 0; e < kExpandGroups; ++e) advance();
+            return true;
         };
-        if (my_tiles > 0) seat_tile();
+        seat_tile();
 #pragma unroll
         for (int e = 0; e < kExpandGroups; ++e)
             if (e < grp) advance();
         constexpr int D = 4;   // pairs in flight per thread
         uint4 qw[D];
         uint32_t qm[D];
+        bool qa[D];
 #pragma unroll
         for (int d = 0; d < D; ++d) {
             qw[d] = make_uint4(0u, 0u, 0u, 0u);
             qm[d] = 0u;
-            if (grp + d * kExpandGroups < total_pairs) fetch(qw[d], qm[d]);
+            qa[d] = fetch(qw[d], qm[d]);
         }
         bool ok = true;
         auto write_stage = [&](int st, uint32_t w0, uint32_t w1, uint32_t mag) {
@@ -762,15 +1030,18 @@ __global__ void __launch_bounds__(Cfg::kThreads, 1) gemm_kernel(const __grid_con
                 }
             }
         };
-        for (int base = grp; base < total_pairs && ok; base += D * kExpandGroups) {
+        // slot d of the queue holds the group's pairs base + d * kExpandGroups
+        for (int base = grp; ok && qa[0]; base += D * kExpandGroups) {
 #pragma unroll
             for (int d = 0; d < D; ++d) {
-                const int p = base + d * kExpandGroups;
-                if (p < total_pairs && ok) {
+                if (qa[d] && ok) {
+                    const int p = base + d * kExpandGroups;
                     const uint4 w = qw[d];
                     const uint32_t mag = qm[d];
-                    if (p + D * kExpandGroups < total_pairs) fetch(qw[d], qm[d]);
+                    qa[d] = fetch(qw[d], qm[d]);
                     expand_pair(p, w, mag);
+                } else {
+                    qa[0] = false;   // the pairs after an empty slot are empty too
                 }
             }
         }
@@ -779,75 +1050,95 @@ __global__ void __launch_bounds__(Cfg::kThreads, 1) gemm_kernel(const __grid_con
         const int q = warp & 3;   // a warp reads the TMEM lane quarter warp % 4
         const int ch = kEpiWarps == 4 ? 0 : (warp - 2 - kExpandWarps) >> 2;   // which share of the columns
         constexpr int kColShare = BN / (kEpiWarps / 4);
-        for (int j = 0; j < my_tiles; ++j) {
+        if (kFused) griddep_wait();   // the flags it counts on are zeroed by the pre-pass
+        for (int j = 0;; ++j) {
+            TileRef tr;
+            const GemmArgs *ge = &g;
+            int ncols = BN, stage1 = g.stage == 1;
+            if (kFused) {
+                int u = -1;
+                if (!ring_get_warp(sh, j, u) || u < 0) break;
+                const FusedTile f = fused_decode(*fs, u);
+                ge = &fused_args(f);
+                tr = tile_ref(*ge, f.t, f.stage == 1 ? fs->n_p1 : fs->n_p2, tile_rank);
+                if (f.half >= 0) {
+                    ncols = 128;
+                    tr.brow += 128 * f.half;
+                }
+                stage1 = f.stage == 1;
+            } else {
+                if (j >= my_tiles) break;
+                tr = tile_ref(g, unit + j * nunits, n_p, tile_rank);
+            }
+            const GemmArgs &ga = *ge;
             const int ab = j & 1;
             bool got = true;
             if (lane == 0) got = wait(&sh->acc_full[ab], (j >> 1) & 1);
             if (!__shfl_sync(0xffffffffu, got, 0)) break;
             tc_fence_after();
-            const TileRef tr = tile_ref(g, unit + j * nunits, n_p, tile_rank);
             const int p0 = tr.p0, c0 = tr.brow;
             const int grow = p0 + q * 32 + lane;
             const uint32_t taddr = tmem + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(ab * BN);
-            const bool row_ok = grow < g.P;
-            for (int cc = ch * kColShare; cc < (ch + 1) * kColShare; cc += 32) {
+            const bool row_ok = grow < ga.P;
+            const int cc_end = min((ch + 1) * kColShare, ncols);
+            for (int cc = ch * kColShare; cc < cc_end; cc += 32) {
                 uint32_t v[32];
                 tmem_ld32(taddr + cc, v);   // every lane takes part (.sync.aligned)
                 if (!row_ok) continue;
                 if (tr.gr) {
-                    grouped_chunk(g, tr, v, tr.t0 + cc, grow);
+                    grouped_chunk(ga, tr, v, tr.t0 + cc, grow);
                     continue;
                 }
                 const int cb = c0 + cc;
-                if (g.stage == 1) {
+                if (stage1) {
                     // column c = i T + t; v[t, i R + r] = fp16(beta_i[r] h); (i, t)
                     // advance with c, beta reloaded only when i changes
-                    int i = cb / g.T, t = cb - i * g.T;
-                    const int64_t tstride = static_cast<int64_t>(g.ell) * g.R;
-                    float b = i < g.ell ? h2f(g.beta[static_cast<int64_t>(i) * g.R + grow]) : 0.f;
-                    __half *vp = g.V + static_cast<int64_t>(t) * tstride + static_cast<int64_t>(i) * g.R + grow;
+                    int i = cb / ga.T, t = cb - i * ga.T;
+                    const int64_t tstride = static_cast<int64_t>(ga.ell) * ga.R;
+                    float b = i < ga.ell ? h2f(ga.beta[static_cast<int64_t>(i) * ga.R + grow]) : 0.f;
+                    __half *vp = ga.V + static_cast<int64_t>(t) * tstride + static_cast<int64_t>(i) * ga.R + grow;
 #pragma unroll
                     for (int e = 0; e < 32; ++e) {
-                        if (cb + e < g.C) *vp = __float2half_rn(b * __uint_as_float(v[e]));
+                        if (cb + e < ga.C) *vp = __float2half_rn(b * __uint_as_float(v[e]));
                         vp += tstride;
-                        if (++t == g.T) {
+                        if (++t == ga.T) {
                             t = 0;
                             ++i;
-                            b = i < g.ell ? h2f(g.beta[static_cast<int64_t>(i) * g.R + grow]) : 0.f;
-                            vp = g.V + static_cast<int64_t>(i) * g.R + grow;
+                            b = i < ga.ell ? h2f(ga.beta[static_cast<int64_t>(i) * ga.R + grow]) : 0.f;
+                            vp = ga.V + static_cast<int64_t>(i) * ga.R + grow;
                         }
                     }
                 } else if (Cfg::kBwd) {
-                    backward_chunk(g, v, cb, grow);
+                    backward_chunk(ga, v, cb, grow);
                 } else {
-                    const int64_t base = static_cast<int64_t>(cb) * g.N + grow;
-                    const int n_ok = g.C - cb;   // tokens of this chunk inside the batch
+                    const int64_t base = static_cast<int64_t>(cb) * ga.N + grow;
+                    const int n_ok = ga.C - cb;   // tokens of this chunk inside the batch
                     // with accumulation the y_in values are loaded eight at a time,
                     // all eight in flight together
-                    if (g.yd == DBF_BF16) {
-                        __nv_bfloat16 *yp = static_cast<__nv_bfloat16 *>(g.y) + base;
+                    if (ga.yd == DBF_BF16) {
+                        __nv_bfloat16 *yp = static_cast<__nv_bfloat16 *>(ga.y) + base;
 #pragma unroll
                         for (int e0 = 0; e0 < 32; e0 += 8) {
                             float yin[8];
 #pragma unroll
                             for (int e = 0; e < 8; ++e)
-                                yin[e] = g.accumulate ? __bfloat162float(yp[static_cast<int64_t>(e0 + e < n_ok ? e0 + e : 0) * g.N]) : 0.f;
+                                yin[e] = ga.accumulate ? __bfloat162float(yp[static_cast<int64_t>(e0 + e < n_ok ? e0 + e : 0) * ga.N]) : 0.f;
 #pragma unroll
                             for (int e = 0; e < 8; ++e)
                                 if (e0 + e < n_ok)
-                                    yp[static_cast<int64_t>(e0 + e) * g.N] = __float2bfloat16_rn(__uint_as_float(v[e0 + e]) + yin[e]);
+                                    yp[static_cast<int64_t>(e0 + e) * ga.N] = __float2bfloat16_rn(__uint_as_float(v[e0 + e]) + yin[e]);
                         }
                     } else {
-                        float *yp = static_cast<float *>(g.y) + base;
+                        float *yp = static_cast<float *>(ga.y) + base;
 #pragma unroll
                         for (int e0 = 0; e0 < 32; e0 += 8) {
                             float yin[8];
 #pragma unroll
                             for (int e = 0; e < 8; ++e)
-                                yin[e] = g.accumulate ? yp[static_cast<int64_t>(e0 + e < n_ok ? e0 + e : 0) * g.N] : 0.f;
+                                yin[e] = ga.accumulate ? yp[static_cast<int64_t>(e0 + e < n_ok ? e0 + e : 0) * ga.N] : 0.f;
 #pragma unroll
                             for (int e = 0; e < 8; ++e)
-                                if (e0 + e < n_ok) yp[static_cast<int64_t>(e0 + e) * g.N] = __uint_as_float(v[e0 + e]) + yin[e];
+                                if (e0 + e < n_ok) yp[static_cast<int64_t>(e0 + e) * ga.N] = __uint_as_float(v[e0 + e]) + yin[e];
                         }
                     }
                 }
@@ -858,6 +1149,16 @@ __global__ void __launch_bounds__(Cfg::kThreads, 1) gemm_kernel(const __grid_con
                 if (kPair) bar_arrive_leader(&sh->acc_empty[ab]);
                 else bar_arrive(&sh->acc_empty[ab]);
             }
+            if (kFused && stage1) {
+                // this warp's v rows of the tile are written: count them on the
+                // column block's flag (every lane's stores ordered before it, for
+                // the generic and the async proxy)
+                asm volatile("fence.proxy.async.global;" ::: "memory");
+                __threadfence();
+                __syncwarp();
+                if (lane == 0)
+                    asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(fs->flags + c0 / BN) : "memory");
+            }
         }
     }
 
@@ -866,8 +1167,9 @@ teardown:
     __syncthreads();
     if (kPair) {
         // neither CTA of a pair ends while the other may still reach its shared
-        // memory (remote arrivals, the pair's MMAs and their commits): each
-        // tells the other it is done and waits (bounded) for the other
+        // memory (remote arrivals, the pair's MMAs and their commits, the
+        // tile ring): each tells the other it is done and waits (bounded) for
+        // the other
         if (threadIdx.x == 0) {
             bar_arrive_rank(&sh->exit_bar, rank ^ 1u);
             const unsigned long long t0 = global_ns();
@@ -882,6 +1184,25 @@ teardown:
         if (kPair) asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS));
         else asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS));
     }
+}
+
+template <class Cfg>
+__global__ void __launch_bounds__(Cfg::kThreads, 1) gemm_kernel(const __grid_constant__ CUtensorMap tmB,
+                                                                const __grid_constant__ CUtensorMap tmA, const __grid_constant__ GemmArgs g)
+{
+    gemm_body<Cfg>(tmB, tmA, g, nullptr, nullptr);
+}
+
+// The forward's two stages in one launch (see FusedSched): tmU and tmV are the
+// maps of u and v, g1 and g2 the two stages' arguments.
+template <class Cfg>
+__global__ void __launch_bounds__(Cfg::kThreads, 1) gemm_fused_kernel(const __grid_constant__ CUtensorMap tmU,
+                                                                      const __grid_constant__ CUtensorMap tmV,
+                                                                      const __grid_constant__ GemmArgs g1,
+                                                                      const __grid_constant__ GemmArgs g2,
+                                                                      const __grid_constant__ FusedSched fs)
+{
+    gemm_body<Cfg>(tmU, tmV, g1, &g2, &fs);
 }
 
 // out[k][c] = in[c][k] for an fp16 matrix in[C][K]; columns C .. Cp-1 of out
@@ -904,41 +1225,79 @@ __global__ void __launch_bounds__(256) transpose_f16_kernel(const uint16_t *__re
 }
 
 // u[(i T + t), m] = fp16(gamma_i[m] x[t, m]); eight columns per thread with
-// 16-byte loads and stores when M % 8 == 0 and gamma is 16-byte aligned.
+// 16-byte loads and stores when M % 8 == 0 and gamma is 16-byte aligned
+// (then a block takes whole rows).
 // tok_major: output row t ell + i (U is [T][ell M], blocks of one token side
 // by side) instead of i T + t.
+// zero[0 .. nzero-1] are cleared too (the fused forward's claim state), and
+// the launch that follows may start as soon as every block has begun.
 __global__ void __launch_bounds__(256) scale_cast_kernel(const void *x, dbf_dtype xd, const uint16_t *gamma, int M,
-                                                         int T, int ell, __half *U, int vec8, int tok_major)
+                                                         int T, int ell, __half *U, int vec8, int tok_major,
+                                                         unsigned *zero, int nzero)
 {
+    asm volatile("griddepcontrol.launch_dependents;");
+    if (blockIdx.x == 0)
+        for (int i = threadIdx.x; i < nzero; i += blockDim.x) zero[i] = 0u;
     const int64_t total = static_cast<int64_t>(ell) * T * M;
     if (vec8) {
-        const int64_t total8 = total / 8;
+        // rows r0, r0 + G, .. r0 + 3G of a block (G = gridDim.x) together, eight
+        // columns per thread: the row's (envelope, token) found once per row
+        // (ell T <= 2^30: 32-bit), all loads of the four rows in flight first
         const int M8 = M / 8;
-        for (int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; idx < total8;
-             idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-            const int64_t row = idx / M8;
-            const int m8 = static_cast<int>(idx - row * M8);
-            const int i = tok_major ? static_cast<int>(row % ell) : static_cast<int>(row / T);
-            const int64_t t = tok_major ? row / ell : row - static_cast<int64_t>(i) * T;
-            const uint4 gw = __ldg(reinterpret_cast<const uint4 *>(gamma + static_cast<int64_t>(i) * M) + m8);
-            float xv[8];
-            if (xd == DBF_BF16) {
-                const uint4 xw = __ldg(reinterpret_cast<const uint4 *>(static_cast<const __nv_bfloat16 *>(x) + t * M) + m8);
-                const __nv_bfloat16 *xb = reinterpret_cast<const __nv_bfloat16 *>(&xw);
+        const int nrows = ell * T;
+        constexpr int kU = 4;
+        for (int r0 = blockIdx.x; r0 < nrows; r0 += kU * gridDim.x) {
+            int64_t xrow[kU], grow_[kU];
+            bool rv[kU];
 #pragma unroll
-                for (int e = 0; e < 8; ++e) xv[e] = __bfloat162float(xb[e]);
-            } else {
-                const float4 *xf = reinterpret_cast<const float4 *>(static_cast<const float *>(x) + t * M) + 2 * m8;
-                const float4 a = __ldg(xf), b = __ldg(xf + 1);
-                xv[0] = a.x; xv[1] = a.y; xv[2] = a.z; xv[3] = a.w;
-                xv[4] = b.x; xv[5] = b.y; xv[6] = b.z; xv[7] = b.w;
+            for (int q = 0; q < kU; ++q) {
+                const int row = r0 + q * static_cast<int>(gridDim.x);
+                rv[q] = row < nrows;
+                const int i = tok_major ? row % ell : row / T;
+                const int t = tok_major ? row / ell : row - i * T;
+                xrow[q] = static_cast<int64_t>(t) * M;
+                grow_[q] = static_cast<int64_t>(i) * M;
             }
-            const __half *gh = reinterpret_cast<const __half *>(&gw);
-            uint4 out;
-            __half *oh = reinterpret_cast<__half *>(&out);
+            for (int m8 = threadIdx.x; m8 < M8; m8 += blockDim.x) {
+                uint4 gw[kU], xa[kU], xb[kU];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) oh[e] = __float2half_rn(__half2float(gh[e]) * xv[e]);
-            reinterpret_cast<uint4 *>(U)[idx] = out;
+                for (int q = 0; q < kU; ++q) {
+                    if (!rv[q]) continue;
+                    gw[q] = __ldg(reinterpret_cast<const uint4 *>(gamma + grow_[q]) + m8);
+                    if (xd == DBF_BF16) {
+                        xa[q] = __ldg(reinterpret_cast<const uint4 *>(static_cast<const __nv_bfloat16 *>(x) + xrow[q]) + m8);
+                    } else {
+                        const uint4 *xf = reinterpret_cast<const uint4 *>(static_cast<const float *>(x) + xrow[q]) + 2 * m8;
+                        xa[q] = __ldg(xf);
+                        xb[q] = __ldg(xf + 1);
+                    }
+                }
+#pragma unroll
+                for (int q = 0; q < kU; ++q) {
+                    if (!rv[q]) continue;
+                    float xv[8];
+                    if (xd == DBF_BF16) {
+                        const __nv_bfloat16 *xh = reinterpret_cast<const __nv_bfloat16 *>(&xa[q]);
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) xv[e] = __bfloat162float(xh[e]);
+                    } else {
+                        const float *f0 = reinterpret_cast<const float *>(&xa[q]);
+                        const float *f1 = reinterpret_cast<const float *>(&xb[q]);
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            xv[e] = f0[e];
+                            xv[4 + e] = f1[e];
+                        }
+                    }
+                    const __half *gh = reinterpret_cast<const __half *>(&gw[q]);
+                    uint4 out;
+                    __half *oh = reinterpret_cast<__half *>(&out);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) oh[e] = __float2half_rn(__half2float(gh[e]) * xv[e]);
+                    const int row = r0 + q * static_cast<int>(gridDim.x);
+                    reinterpret_cast<uint4 *>(U)[static_cast<int64_t>(row) * M8 + m8] = out;
+                }
+            }
         }
         return;
     }
@@ -1052,6 +1411,29 @@ cudaError_t launch_gemm(const CUtensorMap &map, const GemmArgs &args, cudaStream
     return cudaGetLastError();
 }
 
+// CTA pairs of 'kernel' (launched as in cfg) that can be resident at once:
+// queried once per kernel and device (the query is slow next to a launch).
+template <class K>
+int resident_pairs(K kernel, cudaLaunchConfig_t cfg)
+{
+    static std::mutex lock;
+    static int resident[64] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    int pairs = device_sms() / 2;
+    if (dev >= 0 && dev < 64) {
+        std::lock_guard<std::mutex> guard(lock);
+        if (!resident[dev]) {
+            cfg.gridDim = dim3(2 * pairs);
+            int n = 0;
+            resident[dev] = (cudaOccupancyMaxActiveClusters(&n, kernel, &cfg) == cudaSuccess && n > 0) ? n : pairs;
+            (void)cudaGetLastError();
+        }
+        if (resident[dev] < pairs) pairs = resident[dev];
+    }
+    return pairs;
+}
+
 // The forward's GEMMs on CTA pairs: clusters of two CTAs, each pair walking
 // 256-row x 256-token tiles (as many pairs as can be resident at once).
 template <class Cfg>
@@ -1074,26 +1456,112 @@ cudaError_t launch_gemm_pair(const CUtensorMap &map, const GemmArgs &args, cudaS
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    // resident pairs: queried once per device (the query is slow next to a launch)
-    static std::mutex lock;
-    static int resident[64] = {};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    int pairs = device_sms() / 2;
-    if (dev >= 0 && dev < 64) {
-        std::lock_guard<std::mutex> guard(lock);
-        if (!resident[dev]) {
-            cfg.gridDim = dim3(2 * pairs);
-            int n = 0;
-            resident[dev] = (cudaOccupancyMaxActiveClusters(&n, gemm_kernel<Cfg>, &cfg) == cudaSuccess && n > 0) ? n : pairs;
-            (void)cudaGetLastError();
-        }
-        if (resident[dev] < pairs) pairs = resident[dev];
-    }
+    int pairs = resident_pairs(gemm_kernel<Cfg>, cfg);
     if (pairs > tiles) pairs = tiles;
     if (pairs < 1) pairs = 1;
     cfg.gridDim = dim3(2 * pairs);
     e = cudaLaunchKernelEx(&cfg, gemm_kernel<Cfg>, map, map, a);
+    if (e != cudaSuccess) return e;
+    return cudaGetLastError();
+}
+
+// ---- the fused forward's schedule ----------------------------------------------
+// Makespan of the claim order (each pair claims its next tile when it starts
+// one) under a cost model: a tile costs its K steps plus two, a half tile
+// 0.55 of a whole one.
+double fused_makespan(int pairs, int n1, int n2, int nh, int nk1, int nk2)
+{
+    const int total = n1 + n2 - nh + 2 * nh;
+    auto cost = [&](int u) {
+        if (u < n1) return nk1 + 2.0;
+        if (u < n1 + n2 - nh) return nk2 + 2.0;
+        return 0.55 * (nk2 + 2.0);
+    };
+    std::vector<double> end(pairs, 0.0);
+    // min-heap of (time of the pair's next claim, pair)
+    std::priority_queue<std::pair<double, int>, std::vector<std::pair<double, int>>, std::greater<>> claims;
+    int u = 0;
+    for (int p = 0; p < pairs && u < total; ++p, ++u) {
+        end[p] = cost(u);
+        claims.push({0.0, p});
+    }
+    for (; u < total; ++u) {
+        const auto c = claims.top();
+        claims.pop();
+        const int p = c.second;
+        claims.push({end[p], p});   // it starts this tile when its current one ends, and claims again
+        end[p] += cost(u);
+    }
+    double m = 0.0;
+    for (double e : end) m = e > m ? e : m;
+    return m;
+}
+
+// Stage-2 tiles to run as halves: the count with the smallest modelled
+// makespan (the smallest such count), memoised per shape.
+int fused_halves(int pairs, int n1, int n2, int nk1, int nk2)
+{
+    static std::mutex lock;
+    static std::map<std::tuple<int, int, int, int, int>, int> memo;
+    const auto key = std::make_tuple(pairs, n1, n2, nk1, nk2);
+    {
+        std::lock_guard<std::mutex> guard(lock);
+        const auto it = memo.find(key);
+        if (it != memo.end()) return it->second;
+    }
+    const int hmax = std::min(n2, 2 * pairs);
+    const int step = std::max(1, pairs / 16);
+    int best = 0;
+    double best_t = fused_makespan(pairs, n1, n2, 0, nk1, nk2);
+    for (int nh = step; nh <= hmax; nh += step) {
+        const double t = fused_makespan(pairs, n1, n2, nh, nk1, nk2);
+        if (t < best_t - 1e-9) {
+            best_t = t;
+            best = nh;
+        }
+    }
+    std::lock_guard<std::mutex> guard(lock);
+    if (memo.size() > 256) memo.clear();
+    memo[key] = best;
+    return best;
+}
+
+constexpr int kFusedMinSteps = 32;   // K steps per stage below which the two-launch path runs
+
+// Both forward stages in one launch on CTA pairs; launched with programmatic
+// stream serialisation so that its prologue and first sign expansions
+// overlap the pre-pass (which clears the claim state it waits for).
+cudaError_t launch_fused(const CUtensorMap &mu, const CUtensorMap &mv, const GemmArgs &a1, const GemmArgs &a2,
+                         FusedSched fs, int n2, int nk1, int nk2, cudaStream_t s, int32_t *status)
+{
+    GemmArgs g1 = a1, g2 = a2;
+    g1.status = status;
+    g2.status = status;
+    const size_t smem = gemm_smem<FusedCfg>();
+    cudaError_t e = allow_smem(reinterpret_cast<const void *>(gemm_fused_kernel<FusedCfg>), static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.blockDim = dim3(FusedCfg::kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int pairs = resident_pairs(gemm_fused_kernel<FusedCfg>, cfg);
+    cfg.numAttrs = 2;
+    fs.nh = fused_halves(pairs, fs.n1, n2, nk1, nk2);
+    fs.n2f = n2 - fs.nh;
+    const int total = fs.n1 + fs.n2f + 2 * fs.nh;
+    if (pairs > total) pairs = total;
+    if (pairs < 1) pairs = 1;
+    cfg.gridDim = dim3(2 * pairs);
+    e = cudaLaunchKernelEx(&cfg, gemm_fused_kernel<FusedCfg>, mu, mv, g1, g2, fs);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
@@ -1106,12 +1574,26 @@ size_t v_bytes(const dbf_layer &L, int64_t T) { return align_up(static_cast<size
 
 }  // namespace
 
+int gemm_forward_launches(const dbf_layer &L)
+{
+    return (L.M / BK >= kFusedMinSteps && L.ell * L.R / BK >= kFusedMinSteps) ? 2 : 3;
+}
+
 bool gemm_shape_ok(const dbf_layer &L)
 {
     return L.M % 128 == 0 && L.R % 128 == 0 && L.M > 0 && L.R > 0 && L.N > 0;
 }
 
-size_t gemm_workspace_bytes(const dbf_layer &L, int64_t T) { return kWsHeaderBytes + u_bytes(L, T) + v_bytes(L, T); }
+// the fused forward's claim counter and stage-1 column-block flags
+size_t ctl_bytes(const dbf_layer &L, int64_t T)
+{
+    return align_up(4 * static_cast<size_t>(1 + (static_cast<int64_t>(L.ell) * T + BN - 1) / BN), 256);
+}
+
+size_t gemm_workspace_bytes(const dbf_layer &L, int64_t T)
+{
+    return kWsHeaderBytes + u_bytes(L, T) + v_bytes(L, T) + ctl_bytes(L, T);
+}
 
 cudaError_t gemm_forward(const dbf_layer &L, const void *x, dbf_dtype xd, void *y, dbf_dtype yd, int64_t T,
                          int flags, void *ws, cudaStream_t s)
@@ -1122,12 +1604,17 @@ cudaError_t gemm_forward(const dbf_layer &L, const void *x, dbf_dtype xd, void *
     __half *U = reinterpret_cast<__half *>(body);
     __half *V = reinterpret_cast<__half *>(body + u_bytes(L, T));
     const int Ti = static_cast<int>(T);
+    unsigned *ctl = reinterpret_cast<unsigned *>(body + u_bytes(L, T) + v_bytes(L, T));
+    const int nk1 = L.M / BK, nk2 = L.ell * L.R / BK;
+    const int n_c1 = static_cast<int>((static_cast<int64_t>(L.ell) * T + BN - 1) / BN);
+    const bool fused = gemm_forward_launches(L) == 2;
     {
         const int64_t total = static_cast<int64_t>(L.ell) * T * L.M;
-        int64_t blocks = (total + 255) / 256;
-        if (blocks > 148 * 32) blocks = 148 * 32;
         const int vec8 = (L.M % 8 == 0) && ((reinterpret_cast<uintptr_t>(L.gamma) & 15u) == 0);
-        scale_cast_kernel<<<static_cast<int>(blocks), 256, 0, s>>>(x, xd, L.gamma, L.M, Ti, L.ell, U, vec8, 0);
+        int64_t blocks = vec8 ? static_cast<int64_t>(L.ell) * T : (total + 255) / 256;
+        if (blocks > 8 * device_sms()) blocks = 8 * device_sms();
+        scale_cast_kernel<<<static_cast<int>(blocks), 256, 0, s>>>(x, xd, L.gamma, L.M, Ti, L.ell, U, vec8, 0,
+                                                                   fused ? ctl : nullptr, fused ? 1 + n_c1 : 0);
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
@@ -1150,8 +1637,6 @@ cudaError_t gemm_forward(const dbf_layer &L, const void *x, dbf_dtype xd, void *
     a1.ell = L.ell;
     a1.R = L.R;
     a1.N = L.N;
-    cudaError_t e = launch_gemm_pair<FwdPairCfg>(mu, a1, s, st);
-    if (e != cudaSuccess) return e;
     GemmArgs a2 = {};
     a2.signs = L.b1_packed;
     a2.pitch = static_cast<int>(pitch_words(L.R));
@@ -1168,6 +1653,19 @@ cudaError_t gemm_forward(const dbf_layer &L, const void *x, dbf_dtype xd, void *
     a2.yd = yd;
     a2.N = L.N;
     a2.accumulate = (flags & DBF_ACCUMULATE) ? 1 : 0;
+    if (fused) {
+        FusedSched fs = {};
+        fs.n_p1 = (L.R + 2 * BM - 1) / (2 * BM);
+        fs.n_p2 = (L.N + 2 * BM - 1) / (2 * BM);
+        fs.n1 = fs.n_p1 * n_c1;
+        fs.ctr = ctl;
+        fs.flags = ctl + 1;
+        fs.flag_target = static_cast<unsigned>(fs.n_p1 * 2 * FusedCfg::kEpiWarps);
+        const int n2 = fs.n_p2 * ((Ti + BN - 1) / BN);
+        return launch_fused(mu, mv, a1, a2, fs, n2, nk1, nk2, s, st);
+    }
+    cudaError_t e = launch_gemm_pair<FwdPairCfg>(mu, a1, s, st);
+    if (e != cudaSuccess) return e;
     return launch_gemm_pair<FwdPairCfg>(mv, a2, s, st);
 }
 
@@ -1181,11 +1679,11 @@ cudaError_t scale_cast(const void *x, dbf_dtype xd, const uint16_t *scale, int K
                        cudaStream_t s, int tok_major = 0)
 {
     const int64_t total = static_cast<int64_t>(ell) * T * K;
-    int64_t blocks = (total + 255) / 256;
-    if (blocks > 148 * 32) blocks = 148 * 32;
     const int vec8 = (K % 8 == 0) && ((reinterpret_cast<uintptr_t>(scale) & 15u) == 0);
+    int64_t blocks = vec8 ? static_cast<int64_t>(ell) * T : (total + 255) / 256;
+    if (blocks > 8 * device_sms()) blocks = 8 * device_sms();
     scale_cast_kernel<<<static_cast<int>(blocks), 256, 0, s>>>(x, xd, scale, K, static_cast<int>(T), ell, out, vec8,
-                                                               tok_major);
+                                                               tok_major, nullptr, 0);
     return cudaGetLastError();
 }
 

@@ -122,6 +122,9 @@ cudaError_t factorize_run(const float *W, int64_t n, int64_t m, int64_t k, const
 
 // prefill path (tcgen05)
 bool gemm_shape_ok(const dbf_layer &L);
+// launches of one prefill forward: the pre-pass and both stages in one
+// launch when both stages are at least 32 K steps deep, else three
+int gemm_forward_launches(const dbf_layer &L);
 size_t gemm_workspace_bytes(const dbf_layer &L, int64_t T);
 cudaError_t gemm_forward(const dbf_layer &L, const void *x, dbf_dtype xd, void *y, dbf_dtype yd,
                          int64_t T, int flags, void *ws, cudaStream_t s);

@@ -115,13 +115,17 @@ def test_segmented_rejects_bad_arguments(lib):
 
 
 def test_forward_launch_count(lib):
-    # host-side query, no launch: GEMM path = pre-pass + two stages; GEMV path
-    # = one kernel whenever M <= 8192 (any token count: the columns are cut
-    # into chunks), else two
+    # host-side query, no launch: GEMM path = pre-pass + one launch of both
+    # stages when both are at least 32 K steps deep (M >= 2048, ell R >= 2048),
+    # else pre-pass + two stages; GEMV path = one kernel whenever M <= 8192 (any
+    # token count: the columns are cut into chunks), else two
     import double_binary_rank_b200 as dbf
     by = ctypes.byref
     L = _layer(M=4096, N=11008, R=5888, ell=1)
-    assert lib.dbf_forward_launches(by(L), 2048, dbf.PATH_AUTO) == 3
+    assert lib.dbf_forward_launches(by(L), 2048, dbf.PATH_AUTO) == 2
+    assert lib.dbf_forward_launches(by(_layer(M=1024, N=4096, R=4096, ell=1)), 2048, dbf.PATH_GEMM) == 3
+    assert lib.dbf_forward_launches(by(_layer(M=2048, N=512, R=1024, ell=1)), 2048, dbf.PATH_GEMM) == 3
+    assert lib.dbf_forward_launches(by(_layer(M=2048, N=512, R=1024, ell=2)), 2048, dbf.PATH_GEMM) == 2
     assert lib.dbf_forward_launches(by(L), 1, dbf.PATH_AUTO) == 1
     for T in (7, 8, 64, 2048):
         assert lib.dbf_forward_launches(by(L), T, dbf.PATH_GEMV) == 1

@@ -159,3 +159,57 @@ def test_gemm_wrapping_shape_sampled_rows(dbf):
     ref = oracle.forward(L, x, rows=rows)
     got = run(dbf, L, x)[rows]
     assert rel_err(got, ref) < TOL
+
+
+# Shapes that take the single-launch forward (both stages at least 32 K steps
+# deep): tiles claimed at run time, stage-2 tiles that wait for the stage-1
+# column blocks they read, ragged rows and tokens; the second has two
+# envelopes whose column blocks straddle the envelope boundary (ell T = 2200),
+# and the last two run their final stage-2 tiles as 128-token halves.
+FUSED = [(2048, 1000, 2048, 1, 700), (2048, 2500, 1024, 2, 1100), (4096, 4096, 2048, 1, 1024)]
+
+
+@pytest.mark.parametrize("shape", FUSED, ids=lambda s: "M{}N{}R{}l{}T{}".format(*s))
+def test_fused_forward_against_oracle(dbf, shape):
+    M, N, R, ell, T = shape
+    rng = np.random.default_rng(sum(shape) + 11)
+    L = random_layer(rng, M, N, R, ell)
+    x = S.to_bf16_bits(rng.standard_normal((T, M)))
+    y_in = rng.standard_normal((T, N)).astype(np.float32)
+    ref = oracle.forward(L, x)
+    got = run(dbf, L, x)
+    assert rel_err(got, ref) < TOL
+    ref_acc = oracle.forward(L, x, y_in=y_in, accumulate=True)
+    assert rel_err(run(dbf, L, x, acc=True, y_in=y_in), ref_acc) < TOL
+    ok, worst = bf16_ok(run(dbf, L, x, y_dtype=torch.bfloat16), ref)
+    assert ok, worst
+
+
+def test_fused_forward_deterministic_and_exact(dbf):
+    # Which pair computes a tile depends on timing, its accumulation order
+    # does not: two calls agree bit for bit. Integer inputs with exact fp16
+    # operands and fp32 sums match the oracle exactly.
+    M, N, R, ell, T = 2048, 2500, 1024, 2, 1100
+    rng = np.random.default_rng(63)
+    L = exact_layer(rng, M, N, R, ell)
+    x = rng.integers(-1, 2, size=(T, M)).astype(np.float32)
+    a = run(dbf, L, x)
+    b = run(dbf, L, x)
+    assert np.array_equal(a, b)
+    assert np.array_equal(a, oracle.forward(L, x))
+
+
+@pytest.mark.parametrize("shape", [FUSED[2]], ids=lambda s: "M{}N{}R{}l{}T{}".format(*s))
+def test_fused_forward_sign_flip_and_alpha_scaling(dbf, shape):
+    # the two bit-exact invariants above, on the single-launch forward
+    M, N, R, ell, T = shape
+    rng = np.random.default_rng(64)
+    L = random_layer(rng, M, N, R, ell)
+    x = S.to_bf16_bits(rng.standard_normal((T, M)))
+    y0 = run(dbf, L, x)
+    flip = rng.random(R) < 0.5
+    L.b1[:, flip] *= -1
+    L.b2[flip, :] *= -1
+    assert np.array_equal(run(dbf, L, x), y0)
+    L.alpha[:] = S.to_f16_bits(2.0 * L.alpha.view(np.float16).astype(np.float64))
+    assert np.array_equal(run(dbf, L, x), 2.0 * y0)
