@@ -504,8 +504,11 @@ __device__ __forceinline__ void backward_chunk(const GemmArgs &g, const uint32_t
 
 // ---- the forward's two stages in one launch ---------------------------------
 // Stage-1 tiles (B2 rows x columns of u) come first, then the stage-2 tiles
-// (B1 rows x tokens), the last nh of them as two halves of 128 tokens so
-// that the last tiles to run are short. A pair takes its first tile by its
+// (B1 rows x tokens), the last nsk of them split in two halves of K, so that
+// the last tiles to run are short: each half sums its share of K, the half
+// that finishes first leaves its partial sums in the workspace and the other
+// adds them (fp32 addition commutes, so the sum does not depend on which
+// half finishes first) and writes y. A pair takes its first tile by its
 // index and every later one from a claim counter, one tile ahead of the tile
 // it starts, so that the pairs that finish first take the remaining tiles;
 // CTA 0's producer posts each claimed tile in a ring of kRing entries in both
@@ -517,15 +520,20 @@ __device__ __forceinline__ void backward_chunk(const GemmArgs &g, const uint32_t
 // only claims while it runs, so every stage-1 tile a stage-2 tile waits for
 // is held by a running pair that does not wait itself.
 struct FusedSched {
-    int n1, n2f, nh;         // stage-1 tiles; stage-2 tiles run whole; stage-2 tiles run as two halves
+    int n1, n2f, nsk;        // stage-1 tiles; stage-2 tiles run whole; stage-2 tiles split in K
+    int ksplit;              // K steps of the first half of a split tile (even)
     int n_p1, n_p2;          // pair row tiles per column block in stages 1 and 2
     unsigned *ctr;           // claim counter (zeroed by the pre-pass)
     unsigned *flags;         // per stage-1 column block: finished epilogue warps (zeroed by the pre-pass)
     unsigned flag_target;    // arrivals that complete a column block
+    // per split tile, CTA and TMEM lane quarter (zeroed by the pre-pass):
+    unsigned *sk_count;      // halves that reached the epilogue
+    unsigned *sk_ready;      // the first half's partial sums are written
+    float *sk_part;          // per split tile and CTA: 128 rows x 256 columns of partial sums, column-major
 };
 
 struct FusedTile {
-    int stage, t, half;      // half: -1 for a whole tile, else which 128 tokens of tile t
+    int stage, t, part;      // part: -1 for a whole tile, else which half of K of tile t
 };
 
 __device__ __forceinline__ FusedTile fused_decode(const FusedSched &fs, int u)
@@ -534,31 +542,25 @@ __device__ __forceinline__ FusedTile fused_decode(const FusedSched &fs, int u)
     if (u < fs.n1) {
         f.stage = 1;
         f.t = u;
-        f.half = -1;
+        f.part = -1;
     } else if (u < fs.n1 + fs.n2f) {
         f.stage = 2;
         f.t = u - fs.n1;
-        f.half = -1;
+        f.part = -1;
     } else {
         const int h = u - fs.n1 - fs.n2f;
         f.stage = 2;
         f.t = fs.n2f + (h >> 1);
-        f.half = h & 1;
+        f.part = h & 1;
     }
     return f;
 }
 
-// Instruction descriptor of a half tile: M = 256 over the pair, N = 128.
-constexpr uint32_t kIdescPairHalf = (1u << 4) | (static_cast<uint32_t>(128 >> 3) << 17) | (static_cast<uint32_t>((2 * BM) >> 4) << 24);
-
-__device__ __forceinline__ void mma_f16_pair_n(uint32_t tmem_d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t accumulate)
+// K steps [kb, ke) of a claimed tile with nk K steps in all.
+__device__ __forceinline__ void fused_krange(const FusedSched &fs, const FusedTile &f, int nk, int &kb, int &ke)
 {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
-        "l"(a), "l"(b), "r"(idesc), "r"(accumulate)
-        : "memory");
+    kb = f.part == 1 ? fs.ksplit : 0;
+    ke = f.part == 0 ? fs.ksplit : nk;
 }
 
 __device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
@@ -734,7 +736,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap &tmB, const CUtensor
             int s = 0;
             int nb_issued = 0, na_issued = 0;   // TMA loads issued on each ring
             if (kFused) {
-                const int total = fs->n1 + fs->n2f + 2 * fs->nh;
+                const int total = fs->n1 + fs->n2f + 2 * fs->nsk;
                 // CTA 0 claims tile k of the pair and posts it in both rings
                 // (-1: no tile left); -2 when the ring wait gave up
                 auto claim = [&](int k) -> int {
@@ -764,14 +766,13 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap &tmB, const CUtensor
                     const FusedTile f = fused_decode(*fs, u);
                     const GemmArgs &gs = fused_args(f);
                     const TileRef tr = tile_ref(gs, f.t, f.stage == 1 ? fs->n_p1 : fs->n_p2, tile_rank);
-                    const int c0 = tr.brow + (f.half > 0 ? 128 : 0);
-                    const int brows = f.half >= 0 ? 64 : 128;   // B rows this CTA supplies
+                    const int c0 = tr.brow;
                     const CUtensorMap *mp = f.stage == 1 ? &tmB : &tmA;
                     bool ok = true;
                     if (f.stage == 2 && c0 < g.T) {
                         // the v rows of tokens [c0, t_hi) of every envelope: stage-1
                         // column blocks (i T + t) / BN
-                        const int t_hi = min(c0 + 2 * brows, g.T);
+                        const int t_hi = min(c0 + BN, g.T);
                         const unsigned long long t0 = global_ns();
                         for (int i = 0; i < g.ell && ok; ++i) {
                             const int b_lo = (i * g.T + c0) / BN, b_hi = (i * g.T + t_hi - 1) / BN;
@@ -790,12 +791,13 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap &tmB, const CUtensor
                         asm volatile("fence.proxy.async.global;" ::: "memory");
                     }
                     if (!ok) break;
-                    const int nk_t = gs.Ktot / BK;
-                    for (int k = 0; k < nk_t; ++k, ++s) {
+                    int kb, ke;
+                    fused_krange(*fs, f, gs.Ktot / BK, kb, ke);
+                    for (int k = kb; k < ke; ++k, ++s) {
                         const int st = s % SB;
                         if (!wait(&sh->empty_b[st], ((s / SB) & 1) ^ 1)) break;
                         if (rank == 0) bar_expect_tx(&sh->full_b[st], 2 * kBBytes);
-                        tma_load_2d_pair(smB + st * kBBytes, mp, k * BK, c0 + static_cast<int>(rank) * brows,
+                        tma_load_2d_pair(smB + st * kBBytes, mp, k * BK, c0 + static_cast<int>(rank) * Cfg::kBRows,
                                          &sh->full_b[st]);
                         nb_issued = s + 1;
                     }
@@ -851,14 +853,12 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap &tmB, const CUtensor
             int s = 0;
             bool ok = true;
             for (int j = 0; ok; ++j) {
-                int nk_t = nk;
-                uint32_t idesc = kIdescPair;
+                int kb = 0, ke = nk;
                 if (kFused) {
                     int u = -1;
                     if (!ring_get(sh, j, u) || u < 0) break;
                     const FusedTile f = fused_decode(*fs, u);
-                    nk_t = fused_args(f).Ktot / BK;
-                    if (f.half >= 0) idesc = kIdescPairHalf;
+                    fused_krange(*fs, f, fused_args(f).Ktot / BK, kb, ke);
                 } else if (j >= my_tiles) {
                     break;
                 }
@@ -867,7 +867,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap &tmB, const CUtensor
                 if (!ok) break;
                 tc_fence_after();
                 const uint32_t dt = tmem + static_cast<uint32_t>(ab * BN);
-                for (int k = 0; k < nk_t; ++k, ++s) {
+                for (int k = kb; k < ke; ++k, ++s) {
                     const int sa = s % SA, sb = s % SB;
                     ok = wait(&sh->full_a[sa], (s / SA) & 1) && wait(&sh->full_b[sb], (s / SB) & 1);
                     if (!ok) break;
@@ -877,13 +877,13 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap &tmB, const CUtensor
                     if (kPair) {
 #pragma unroll
                         for (int kk = 0; kk < BK / 16; ++kk)
-                            mma_f16_pair_n(dt, da + 2 * kk, db + 2 * kk, idesc, (k | kk) != 0);
+                            mma_f16_pair(dt, da + 2 * kk, db + 2 * kk, (k != kb || kk) != 0);
                         mma_commit_pair_both(&sh->empty_a[sa]);   // both CTAs' stages are free again
                         mma_commit_pair_both(&sh->empty_b[sb]);
                     } else {
 #pragma unroll
                         for (int kk = 0; kk < BK / 16; ++kk)   // 32 bytes of K per MMA: +2 in 16-byte units
-                            mma_f16(dt, da + 2 * kk, db + 2 * kk, (k | kk) != 0);
+                            mma_f16(dt, da + 2 * kk, db + 2 * kk, (k != kb || kk) != 0);
                         mma_commit(&sh->empty_a[sa]);   // each commit arrives once these MMAs are done
                         mma_commit(&sh->empty_b[sb]);
                     }
@@ -937,8 +937,17 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap &tmB, const CUtensor
                 cg = &fused_args(f);
                 np = f.stage == 1 ? fs->n_p1 : fs->n_p2;
                 t = f.t;
-                cnpairs = cg->Ktot / (2 * BK);
+                int kb, ke;
+                fused_krange(*fs, f, cg->Ktot / BK, kb, ke);
+                cnpairs = (ke - kb) / 2;
                 cenv_words = cg->Kp / 32;
+                if (kb > 0) {
+                    // the second half of K starts inside the row: its envelope
+                    // block, and the word in it (a multiple of four: Kp % 128 == 0)
+                    cenv = kb * BK / cg->Kp;
+                    cword = (kb * BK - cenv * cg->Kp) / 32;
+                    cbase = cg->env_advance ? cenv * cenv_words : 0;
+                }
             } else if (cj >= my_tiles) {
                 calive = false;
                 return;
@@ -1054,18 +1063,16 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap &tmB, const CUtensor
         for (int j = 0;; ++j) {
             TileRef tr;
             const GemmArgs *ge = &g;
-            int ncols = BN, stage1 = g.stage == 1;
+            int stage1 = g.stage == 1;
+            int sk = -1;   // a tile split in K: its slot (tile, CTA, lane quarter)
             if (kFused) {
                 int u = -1;
                 if (!ring_get_warp(sh, j, u) || u < 0) break;
                 const FusedTile f = fused_decode(*fs, u);
                 ge = &fused_args(f);
                 tr = tile_ref(*ge, f.t, f.stage == 1 ? fs->n_p1 : fs->n_p2, tile_rank);
-                if (f.half >= 0) {
-                    ncols = 128;
-                    tr.brow += 128 * f.half;
-                }
                 stage1 = f.stage == 1;
+                if (f.part >= 0) sk = ((f.t - fs->n2f) * 2 + static_cast<int>(rank)) * 4 + q;
             } else {
                 if (j >= my_tiles) break;
                 tr = tile_ref(g, unit + j * nunits, n_p, tile_rank);
@@ -1080,10 +1087,41 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap &tmB, const CUtensor
             const int grow = p0 + q * 32 + lane;
             const uint32_t taddr = tmem + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(ab * BN);
             const bool row_ok = grow < ga.P;
-            const int cc_end = min((ch + 1) * kColShare, ncols);
-            for (int cc = ch * kColShare; cc < cc_end; cc += 32) {
+            // a split tile: the half that reaches its epilogue first stores its
+            // partial sums (this CTA's 128 rows, column-major) and the other
+            // waits for them, adds them to its own and writes y
+            bool sk_first = false;
+            float *sk_base = nullptr;
+            if (kFused && sk >= 0) {
+                unsigned old = 0;
+                if (lane == 0) old = atomicAdd(fs->sk_count + sk, 1u);
+                sk_first = __shfl_sync(0xffffffffu, old, 0) == 0;
+                sk_base = fs->sk_part + static_cast<int64_t>(sk >> 2) * (BM * BN) + q * 32 + lane;
+                if (!sk_first && lane == 0) {
+                    const unsigned long long t0 = global_ns();
+                    while (ld_acquire_u32(fs->sk_ready + sk) == 0) {
+                        if (*abort) break;
+                        if (global_ns() - t0 > kWaitNs) {
+                            *abort = 1;
+                            break;
+                        }
+                    }
+                }
+                __syncwarp();
+            }
+            for (int cc = ch * kColShare; cc < (ch + 1) * kColShare; cc += 32) {
                 uint32_t v[32];
                 tmem_ld32(taddr + cc, v);   // every lane takes part (.sync.aligned)
+                if (kFused && sk >= 0) {
+                    float *pc = sk_base + static_cast<int64_t>(cc) * BM;
+                    if (sk_first) {
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) pc[e * BM] = __uint_as_float(v[e]);
+                        continue;
+                    }
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) + pc[e * BM]);
+                }
                 if (!row_ok) continue;
                 if (tr.gr) {
                     grouped_chunk(ga, tr, v, tr.t0 + cc, grow);
@@ -1148,6 +1186,12 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap &tmB, const CUtensor
             if (lane == 0) {
                 if (kPair) bar_arrive_leader(&sh->acc_empty[ab]);
                 else bar_arrive(&sh->acc_empty[ab]);
+            }
+            if (kFused && sk >= 0 && sk_first) {
+                // the partial sums are written: the other half may read them
+                __threadfence();
+                __syncwarp();
+                if (lane == 0) asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(fs->sk_ready + sk) : "memory");
             }
             if (kFused && stage1) {
                 // this warp's v rows of the tile are written: count them on the
@@ -1466,16 +1510,19 @@ cudaError_t launch_gemm_pair(const CUtensorMap &map, const GemmArgs &args, cudaS
 }
 
 // ---- the fused forward's schedule ----------------------------------------------
+constexpr int kMaxSplit = 64;   // stage-2 tiles at most that run split in K
+
 // Makespan of the claim order (each pair claims its next tile when it starts
-// one) under a cost model: a tile costs its K steps plus two, a half tile
-// 0.55 of a whole one.
-double fused_makespan(int pairs, int n1, int n2, int nh, int nk1, int nk2)
+// one) when the last nsk stage-2 tiles run as two halves of K, under a cost
+// model: a tile costs its K steps plus two, a half its share plus three (the
+// exchange of partial sums).
+double fused_makespan(int pairs, int n1, int n2, int nsk, int nk1, int nk2)
 {
-    const int total = n1 + n2 - nh + 2 * nh;
+    const int total = n1 + n2 + nsk;
     auto cost = [&](int u) {
         if (u < n1) return nk1 + 2.0;
-        if (u < n1 + n2 - nh) return nk2 + 2.0;
-        return 0.55 * (nk2 + 2.0);
+        if (u < n1 + n2 - nsk) return nk2 + 2.0;
+        return 0.5 * nk2 + 3.0;
     };
     std::vector<double> end(pairs, 0.0);
     // min-heap of (time of the pair's next claim, pair)
@@ -1497,27 +1544,27 @@ double fused_makespan(int pairs, int n1, int n2, int nh, int nk1, int nk2)
     return m;
 }
 
-// Stage-2 tiles to run as halves: the count with the smallest modelled
-// makespan (the smallest such count), memoised per shape.
-int fused_halves(int pairs, int n1, int n2, int nk1, int nk2)
+// Stage-2 tiles to split in K (at most smax): the count with the smallest
+// modelled makespan (the smallest such count), memoised per shape.
+int fused_splits(int pairs, int n1, int n2, int nk1, int nk2, int smax)
 {
     static std::mutex lock;
-    static std::map<std::tuple<int, int, int, int, int>, int> memo;
-    const auto key = std::make_tuple(pairs, n1, n2, nk1, nk2);
+    static std::map<std::tuple<int, int, int, int, int, int>, int> memo;
+    const auto key = std::make_tuple(pairs, n1, n2, nk1, nk2, smax);
     {
         std::lock_guard<std::mutex> guard(lock);
         const auto it = memo.find(key);
         if (it != memo.end()) return it->second;
     }
-    const int hmax = std::min(n2, 2 * pairs);
+    const int hmax = std::min(n2, smax);
     const int step = std::max(1, pairs / 16);
     int best = 0;
     double best_t = fused_makespan(pairs, n1, n2, 0, nk1, nk2);
-    for (int nh = step; nh <= hmax; nh += step) {
-        const double t = fused_makespan(pairs, n1, n2, nh, nk1, nk2);
+    for (int nsk = step; nsk <= hmax; nsk += step) {
+        const double t = fused_makespan(pairs, n1, n2, nsk, nk1, nk2);
         if (t < best_t - 1e-9) {
             best_t = t;
-            best = nh;
+            best = nsk;
         }
     }
     std::lock_guard<std::mutex> guard(lock);
@@ -1555,9 +1602,10 @@ cudaError_t launch_fused(const CUtensorMap &mu, const CUtensorMap &mv, const Gem
     cfg.numAttrs = 1;
     int pairs = resident_pairs(gemm_fused_kernel<FusedCfg>, cfg);
     cfg.numAttrs = 2;
-    fs.nh = fused_halves(pairs, fs.n1, n2, nk1, nk2);
-    fs.n2f = n2 - fs.nh;
-    const int total = fs.n1 + fs.n2f + 2 * fs.nh;
+    fs.nsk = fused_splits(pairs, fs.n1, n2, nk1, nk2, std::min(n2, kMaxSplit));
+    fs.ksplit = (nk2 / 2) & ~1;
+    fs.n2f = n2 - fs.nsk;
+    const int total = fs.n1 + fs.n2f + 2 * fs.nsk;
     if (pairs > total) pairs = total;
     if (pairs < 1) pairs = 1;
     cfg.gridDim = dim3(2 * pairs);
@@ -1584,15 +1632,25 @@ bool gemm_shape_ok(const dbf_layer &L)
     return L.M % 128 == 0 && L.R % 128 == 0 && L.M > 0 && L.R > 0 && L.N > 0;
 }
 
-// the fused forward's claim counter and stage-1 column-block flags
-size_t ctl_bytes(const dbf_layer &L, int64_t T)
+// the fused forward's claim state: the claim counter, the stage-1
+// column-block flags and the split tiles' counters (zeroed by the pre-pass)
+int ctl_words(const dbf_layer &L, int64_t T)
 {
-    return align_up(4 * static_cast<size_t>(1 + (static_cast<int64_t>(L.ell) * T + BN - 1) / BN), 256);
+    return static_cast<int>(1 + (static_cast<int64_t>(L.ell) * T + BN - 1) / BN + 2 * 8 * kMaxSplit);
+}
+
+// the split tiles' partial sums: 256 x 256 fp32 per split tile
+size_t part_bytes(const dbf_layer &L, int64_t T)
+{
+    if (gemm_forward_launches(L) != 2) return 0;
+    const int64_t n2 = ((L.N + 2 * BM - 1) / (2 * BM)) * ((T + BN - 1) / BN);
+    return static_cast<size_t>(std::min<int64_t>(n2, kMaxSplit)) * 2 * BM * BN * 4;
 }
 
 size_t gemm_workspace_bytes(const dbf_layer &L, int64_t T)
 {
-    return kWsHeaderBytes + u_bytes(L, T) + v_bytes(L, T) + ctl_bytes(L, T);
+    return kWsHeaderBytes + u_bytes(L, T) + v_bytes(L, T) + align_up(4 * static_cast<size_t>(ctl_words(L, T)), 256) +
+           part_bytes(L, T);
 }
 
 cudaError_t gemm_forward(const dbf_layer &L, const void *x, dbf_dtype xd, void *y, dbf_dtype yd, int64_t T,
@@ -1614,7 +1672,7 @@ cudaError_t gemm_forward(const dbf_layer &L, const void *x, dbf_dtype xd, void *
         int64_t blocks = vec8 ? static_cast<int64_t>(L.ell) * T : (total + 255) / 256;
         if (blocks > 8 * device_sms()) blocks = 8 * device_sms();
         scale_cast_kernel<<<static_cast<int>(blocks), 256, 0, s>>>(x, xd, L.gamma, L.M, Ti, L.ell, U, vec8, 0,
-                                                                   fused ? ctl : nullptr, fused ? 1 + n_c1 : 0);
+                                                                   fused ? ctl : nullptr, fused ? ctl_words(L, T) : 0);
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
@@ -1661,6 +1719,9 @@ cudaError_t gemm_forward(const dbf_layer &L, const void *x, dbf_dtype xd, void *
         fs.ctr = ctl;
         fs.flags = ctl + 1;
         fs.flag_target = static_cast<unsigned>(fs.n_p1 * 2 * FusedCfg::kEpiWarps);
+        fs.sk_count = ctl + 1 + n_c1;
+        fs.sk_ready = fs.sk_count + 8 * kMaxSplit;
+        fs.sk_part = reinterpret_cast<float *>(reinterpret_cast<char *>(ctl) + align_up(4 * static_cast<size_t>(ctl_words(L, T)), 256));
         const int n2 = fs.n_p2 * ((Ti + BN - 1) / BN);
         return launch_fused(mu, mv, a1, a2, fs, n2, nk1, nk2, s, st);
     }
