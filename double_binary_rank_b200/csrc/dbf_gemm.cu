@@ -449,21 +449,35 @@ __device__ __forceinline__ float load_w(const void *w, dbf_dtype wd, int64_t i)
 __device__ __forceinline__ void backward_chunk(const GemmArgs &g, const uint32_t (&v)[32], int cb, int p)
 {
     const int i0 = cb / g.T, t0 = cb - i0 * g.T;
+    // the operand of each of the 32 columns, all loads issued before any is
+    // used (one straight block per operand type, read-only path)
     float w[32];
-    {
+    if (g.stage == 4) {
+#pragma unroll
+        for (int e = 0; e < 32; ++e) w[e] = __ldg(g.H32 + (cb + e < g.C ? static_cast<int64_t>(cb + e) * g.P + p : 0));
+    } else if (g.stage >= 5 && g.red) {
+        int64_t off[32];
         int t = t0;
 #pragma unroll
         for (int e = 0; e < 32; ++e) {
-            const bool ok = cb + e < g.C;
-            if (g.stage == 4) {
-                w[e] = g.H32[ok ? static_cast<int64_t>(cb + e) * g.P + p : 0];
-            } else if (g.stage >= 5 && g.red) {
-                w[e] = load_w(g.W, g.wd, ok ? static_cast<int64_t>(t) * g.P + p : 0);
-            } else {
-                w[e] = 0.f;
-            }
+            off[e] = cb + e < g.C ? static_cast<int64_t>(t) * g.P + p : 0;
             if (++t == g.T) t = 0;
         }
+        if (g.wd == DBF_BF16) {
+            const __nv_bfloat16 *wp = static_cast<const __nv_bfloat16 *>(g.W);
+            __nv_bfloat16 wb[32];
+#pragma unroll
+            for (int e = 0; e < 32; ++e) wb[e] = __ldg(wp + off[e]);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) w[e] = __bfloat162float(wb[e]);
+        } else {
+            const float *wp = static_cast<const float *>(g.W);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) w[e] = __ldg(wp + off[e]);
+        }
+    } else {
+#pragma unroll
+        for (int e = 0; e < 32; ++e) w[e] = 0.f;
     }
     int i = i0, t = t0;
     float cs = (g.cscale && i < g.ell) ? h2f(g.cscale[static_cast<int64_t>(i) * g.P + p]) : 0.f;
