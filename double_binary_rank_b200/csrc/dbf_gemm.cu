@@ -83,7 +83,8 @@ struct GemmCfg {
 using FwdCfg = GemmCfg<2, 6, 4, 4, false>;
 using FwdPairCfg = GemmCfg<2, 6, 6, 4, false, true>;
 using FusedCfg = GemmCfg<2, 6, 6, 4, false, true, true>;
-using BwdPairCfg = GemmCfg<1, 4, 8, 8, true, true>;
+using BwdPairCfg = GemmCfg<1, 6, 6, 8, true, true>;
+using BwdFusedCfg = GemmCfg<1, 6, 6, 8, true, true, true>;   // two sign GEMMs of the backward in one launch
 constexpr int kMaxStages = 8;
 constexpr int A_BYTES = BM * BK * 2;   // 16 KB
 constexpr int TMEM_COLS = 512;          // two 256-column accumulators
@@ -450,11 +451,12 @@ __device__ __forceinline__ void backward_chunk(const GemmArgs &g, const uint32_t
 {
     const int i0 = cb / g.T, t0 = cb - i0 * g.T;
     // the operand of each of the 32 columns, all loads issued before any is
-    // used (one straight block per operand type, read-only path)
+    // used (one straight block per operand type; dy and x through the
+    // read-only path, h not: the same launch may have written it)
     float w[32];
     if (g.stage == 4) {
 #pragma unroll
-        for (int e = 0; e < 32; ++e) w[e] = __ldg(g.H32 + (cb + e < g.C ? static_cast<int64_t>(cb + e) * g.P + p : 0));
+        for (int e = 0; e < 32; ++e) w[e] = g.H32[cb + e < g.C ? static_cast<int64_t>(cb + e) * g.P + p : 0];
     } else if (g.stage >= 5 && g.red) {
         int64_t off[32];
         int t = t0;
@@ -535,11 +537,16 @@ __device__ __forceinline__ void backward_chunk(const GemmArgs &g, const uint32_t
 // is held by a running pair that does not wait itself.
 struct FusedSched {
     int n1, n2f, nsk;        // stage-1 tiles; stage-2 tiles run whole; stage-2 tiles split in K
+    // what stage-2 tiles read of stage-1 output (flags, counted by stage-1
+    // epilogue warps): 1 their B operand, whole column blocks (the forward's
+    // v; flag per column block); 2 in their epilogue, the stage-1 tile of the
+    // same index (the backward's h; flag per tile); 0 nothing
+    int dep;
     int ksplit;              // K steps of the first half of a split tile (even)
     int n_p1, n_p2;          // pair row tiles per column block in stages 1 and 2
     unsigned *ctr;           // claim counter (zeroed by the pre-pass)
-    unsigned *flags;         // per stage-1 column block: finished epilogue warps (zeroed by the pre-pass)
-    unsigned flag_target;    // arrivals that complete a column block
+    unsigned *flags;         // finished stage-1 epilogue warps per column block (dep 1) or tile (dep 2); zeroed by the pre-pass
+    unsigned flag_target;    // arrivals that complete a block or tile
     // per split tile, CTA and TMEM lane quarter (zeroed by the pre-pass):
     unsigned *sk_count;      // halves that reached the epilogue
     unsigned *sk_ready;      // the first half's partial sums are written
@@ -664,7 +671,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap &tmB, const CUtensor
     constexpr bool kFused = Cfg::kFused;
     static_assert(SA <= kMaxStages && SB <= kMaxStages && kEpiWarps % 4 == 0 && BN % (32 * (kEpiWarps / 4)) == 0,
                   "pipeline shape");
-    static_assert(!kFused || (Cfg::kPair && !Cfg::kBwd && kEpiWarps == 4), "the fused forward runs on CTA pairs");
+    static_assert(!kFused || Cfg::kPair, "tiles are claimed by CTA pairs");
     extern __shared__ uint8_t smem_raw[];
     // 1024-byte alignment for the swizzled tiles
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -783,7 +790,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap &tmB, const CUtensor
                     const int c0 = tr.brow;
                     const CUtensorMap *mp = f.stage == 1 ? &tmB : &tmA;
                     bool ok = true;
-                    if (f.stage == 2 && c0 < g.T) {
+                    if (f.stage == 2 && fs->dep == 1 && c0 < g.T) {
                         // the v rows of tokens [c0, t_hi) of every envelope: stage-1
                         // column blocks (i T + t) / BN
                         const int t_hi = min(c0 + BN, g.T);
@@ -1078,15 +1085,21 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap &tmB, const CUtensor
             TileRef tr;
             const GemmArgs *ge = &g;
             int stage1 = g.stage == 1;
-            int sk = -1;   // a tile split in K: its slot (tile, CTA, lane quarter)
+            int sk = -1;         // a tile split in K: its slot (tile, CTA, epilogue warp)
+            int flag_out = -1;   // a stage-1 tile whose epilogue counts on a flag (dep 1: column block; 2: tile)
+            int flag_in = -1;    // a stage-2 tile whose epilogue waits for the stage-1 tile of this index (dep 2)
             if (kFused) {
                 int u = -1;
                 if (!ring_get_warp(sh, j, u) || u < 0) break;
                 const FusedTile f = fused_decode(*fs, u);
                 ge = &fused_args(f);
                 tr = tile_ref(*ge, f.t, f.stage == 1 ? fs->n_p1 : fs->n_p2, tile_rank);
-                stage1 = f.stage == 1;
-                if (f.part >= 0) sk = ((f.t - fs->n2f) * 2 + static_cast<int>(rank)) * 4 + q;
+                stage1 = ge->stage == 1;   // the forward's stage 1 (v); the backward's GEMMs have stages 3..6
+                if (!Cfg::kBwd && f.part >= 0)   // only the forward splits tiles in K
+                    sk = ((f.t - fs->n2f) * 2 + static_cast<int>(rank)) * kEpiWarps + (warp - 2 - kExpandWarps);
+                if (f.stage == 1 && fs->dep == 1) flag_out = tr.brow / BN;
+                if (f.stage == 1 && fs->dep == 2) flag_out = f.t;
+                if (f.stage == 2 && fs->dep == 2) flag_in = f.t;
             } else {
                 if (j >= my_tiles) break;
                 tr = tile_ref(g, unit + j * nunits, n_p, tile_rank);
@@ -1097,6 +1110,20 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap &tmB, const CUtensor
             if (lane == 0) got = wait(&sh->acc_full[ab], (j >> 1) & 1);
             if (!__shfl_sync(0xffffffffu, got, 0)) break;
             tc_fence_after();
+            if (kFused && flag_in >= 0) {
+                // the stage-1 tile this epilogue reads (its h) is complete
+                if (lane == 0) {
+                    const unsigned long long t0 = global_ns();
+                    while (ld_acquire_u32(fs->flags + flag_in) < fs->flag_target) {
+                        if (*abort) break;
+                        if (global_ns() - t0 > kWaitNs) {
+                            *abort = 1;
+                            break;
+                        }
+                    }
+                }
+                __syncwarp();
+            }
             const int p0 = tr.p0, c0 = tr.brow;
             const int grow = p0 + q * 32 + lane;
             const uint32_t taddr = tmem + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(ab * BN);
@@ -1110,7 +1137,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap &tmB, const CUtensor
                 unsigned old = 0;
                 if (lane == 0) old = atomicAdd(fs->sk_count + sk, 1u);
                 sk_first = __shfl_sync(0xffffffffu, old, 0) == 0;
-                sk_base = fs->sk_part + static_cast<int64_t>(sk >> 2) * (BM * BN) + q * 32 + lane;
+                sk_base = fs->sk_part + static_cast<int64_t>(sk / kEpiWarps) * (BM * BN) + q * 32 + lane;
                 if (!sk_first && lane == 0) {
                     const unsigned long long t0 = global_ns();
                     while (ld_acquire_u32(fs->sk_ready + sk) == 0) {
@@ -1207,15 +1234,15 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap &tmB, const CUtensor
                 __syncwarp();
                 if (lane == 0) asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(fs->sk_ready + sk) : "memory");
             }
-            if (kFused && stage1) {
-                // this warp's v rows of the tile are written: count them on the
-                // column block's flag (every lane's stores ordered before it, for
-                // the generic and the async proxy)
+            if (kFused && flag_out >= 0) {
+                // this warp's rows of the tile are written: count them on the
+                // flag (every lane's stores ordered before it, for the generic
+                // and the async proxy)
                 asm volatile("fence.proxy.async.global;" ::: "memory");
                 __threadfence();
                 __syncwarp();
                 if (lane == 0)
-                    asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(fs->flags + c0 / BN) : "memory");
+                    asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(fs->flags + flag_out) : "memory");
             }
         }
     }
@@ -1475,21 +1502,21 @@ template <class K>
 int resident_pairs(K kernel, cudaLaunchConfig_t cfg)
 {
     static std::mutex lock;
-    static int resident[64] = {};
+    static std::map<std::pair<int, const void *>, int> resident;
     int dev = 0;
     cudaGetDevice(&dev);
     int pairs = device_sms() / 2;
-    if (dev >= 0 && dev < 64) {
-        std::lock_guard<std::mutex> guard(lock);
-        if (!resident[dev]) {
-            cfg.gridDim = dim3(2 * pairs);
-            int n = 0;
-            resident[dev] = (cudaOccupancyMaxActiveClusters(&n, kernel, &cfg) == cudaSuccess && n > 0) ? n : pairs;
-            (void)cudaGetLastError();
-        }
-        if (resident[dev] < pairs) pairs = resident[dev];
+    std::lock_guard<std::mutex> guard(lock);
+    const auto key = std::make_pair(dev, reinterpret_cast<const void *>(kernel));
+    auto it = resident.find(key);
+    if (it == resident.end()) {
+        cfg.gridDim = dim3(2 * pairs);
+        int n = 0;
+        const int r = (cudaOccupancyMaxActiveClusters(&n, kernel, &cfg) == cudaSuccess && n > 0) ? n : pairs;
+        (void)cudaGetLastError();
+        it = resident.emplace(key, r).first;
     }
-    return pairs;
+    return it->second < pairs ? it->second : pairs;
 }
 
 // The forward's GEMMs on CTA pairs: clusters of two CTAs, each pair walking
@@ -1589,20 +1616,24 @@ int fused_splits(int pairs, int n1, int n2, int nk1, int nk2, int smax)
 
 constexpr int kFusedMinSteps = 32;   // K steps per stage below which the two-launch path runs
 
-// Both forward stages in one launch on CTA pairs; launched with programmatic
-// stream serialisation so that its prologue and first sign expansions
-// overlap the pre-pass (which clears the claim state it waits for).
+// Two GEMMs in one launch on CTA pairs (Cfg: FusedCfg for the forward's two
+// stages, BwdFusedCfg for pairs of the backward's independent sign GEMMs):
+// fs.n1 tiles of the first, n2 of the second. With pdl the launch allows
+// programmatic stream serialisation, so that its prologue and first sign
+// expansions overlap the pre-pass before it (which clears the claim state
+// it waits for). The forward (fs.dep) splits its last stage-2 tiles in K.
+template <class Cfg>
 cudaError_t launch_fused(const CUtensorMap &mu, const CUtensorMap &mv, const GemmArgs &a1, const GemmArgs &a2,
-                         FusedSched fs, int n2, int nk1, int nk2, cudaStream_t s, int32_t *status)
+                         FusedSched fs, int n2, int nk1, int nk2, bool pdl, cudaStream_t s, int32_t *status)
 {
     GemmArgs g1 = a1, g2 = a2;
     g1.status = status;
     g2.status = status;
-    const size_t smem = gemm_smem<FusedCfg>();
-    cudaError_t e = allow_smem(reinterpret_cast<const void *>(gemm_fused_kernel<FusedCfg>), static_cast<int>(smem));
+    const size_t smem = gemm_smem<Cfg>();
+    cudaError_t e = allow_smem(reinterpret_cast<const void *>(gemm_fused_kernel<Cfg>), static_cast<int>(smem));
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
-    cfg.blockDim = dim3(FusedCfg::kThreads);
+    cfg.blockDim = dim3(Cfg::kThreads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = s;
     cudaLaunchAttribute attr[2];
@@ -1614,16 +1645,19 @@ cudaError_t launch_fused(const CUtensorMap &mu, const CUtensorMap &mv, const Gem
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    int pairs = resident_pairs(gemm_fused_kernel<FusedCfg>, cfg);
-    cfg.numAttrs = 2;
-    fs.nsk = fused_splits(pairs, fs.n1, n2, nk1, nk2, std::min(n2, kMaxSplit));
+    int pairs = resident_pairs(gemm_fused_kernel<Cfg>, cfg);
+    cfg.numAttrs = pdl ? 2 : 1;
+    // only the forward (dep 1) splits tiles in K: the backward's epilogues
+    // have no exchange of partial sums
+    fs.nsk = fs.dep == 1 ? fused_splits(pairs, fs.n1, n2, nk1, nk2, std::min(n2, kMaxSplit)) : 0;
     fs.ksplit = (nk2 / 2) & ~1;
     fs.n2f = n2 - fs.nsk;
     const int total = fs.n1 + fs.n2f + 2 * fs.nsk;
+    if (total <= 0) return cudaSuccess;
     if (pairs > total) pairs = total;
     if (pairs < 1) pairs = 1;
     cfg.gridDim = dim3(2 * pairs);
-    e = cudaLaunchKernelEx(&cfg, gemm_fused_kernel<FusedCfg>, mu, mv, g1, g2, fs);
+    e = cudaLaunchKernelEx(&cfg, gemm_fused_kernel<Cfg>, mu, mv, g1, g2, fs);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
@@ -1737,7 +1771,8 @@ cudaError_t gemm_forward(const dbf_layer &L, const void *x, dbf_dtype xd, void *
         fs.sk_ready = fs.sk_count + 8 * kMaxSplit;
         fs.sk_part = reinterpret_cast<float *>(reinterpret_cast<char *>(ctl) + align_up(4 * static_cast<size_t>(ctl_words(L, T)), 256));
         const int n2 = fs.n_p2 * ((Ti + BN - 1) / BN);
-        return launch_fused(mu, mv, a1, a2, fs, n2, nk1, nk2, s, st);
+        fs.dep = 1;
+        return launch_fused<FusedCfg>(mu, mv, a1, a2, fs, n2, nk1, nk2, true, s, st);
     }
     cudaError_t e = launch_gemm_pair<FwdPairCfg>(mu, a1, s, st);
     if (e != cudaSuccess) return e;
@@ -1751,18 +1786,19 @@ namespace dbf {
 namespace {
 
 cudaError_t scale_cast(const void *x, dbf_dtype xd, const uint16_t *scale, int K, int64_t T, int ell, __half *out,
-                       cudaStream_t s, int tok_major = 0)
+                       cudaStream_t s, int tok_major = 0, unsigned *zero = nullptr, int nzero = 0)
 {
     const int64_t total = static_cast<int64_t>(ell) * T * K;
     const int vec8 = (K % 8 == 0) && ((reinterpret_cast<uintptr_t>(scale) & 15u) == 0);
     int64_t blocks = vec8 ? static_cast<int64_t>(ell) * T : (total + 255) / 256;
     if (blocks > 8 * device_sms()) blocks = 8 * device_sms();
     scale_cast_kernel<<<static_cast<int>(blocks), 256, 0, s>>>(x, xd, scale, K, static_cast<int>(T), ell, out, vec8,
-                                                               tok_major, nullptr, 0);
+                                                               tok_major, zero, nzero);
     return cudaGetLastError();
 }
 
 struct BwdLayout {
+    size_t ctl;                     // claim counters of the two fused launches (256 bytes)
     size_t u, a, h32, vh, vg;       // offsets after the header
     size_t ut, at, vht, vgt;        // transposed operands of the sign-matrix gradients
     size_t total;
@@ -1774,7 +1810,9 @@ BwdLayout bwd_layout(const dbf_layer &L, int64_t T, bool signs)
     const int64_t C = static_cast<int64_t>(L.ell) * T;
     BwdLayout b;
     b.cp = (C + 7) / 8 * 8;
-    b.u = 0;
+    b.ctl = 0;
+    // claim counters of the two fused launches and one flag per G3 tile
+    b.u = align_up(4 * static_cast<size_t>(2 + ((L.R + 255) / 256) * ((C + 255) / 256)), 256);
     b.a = b.u + align_up(static_cast<size_t>(C) * L.M * 2, 256);
     b.h32 = b.a + align_up(static_cast<size_t>(C) * L.N * 2, 256);
     b.vh = b.h32 + align_up(static_cast<size_t>(C) * L.R * 4, 256);
@@ -1881,7 +1919,14 @@ cudaError_t gemm_backward(const dbf_layer &L, const uint32_t *b1t, const uint32_
         if (dgamma && (e = cudaMemsetAsync(dgamma, 0, sizeof(float) * ell * L.M, s)) != cudaSuccess) return e;
         if (dx && ell > 1 && (e = cudaMemsetAsync(dx, 0, sizeof(float) * T * L.M, s)) != cudaSuccess) return e;
     }
-    if ((e = scale_cast(x, xd, L.gamma, L.M, T, ell, U, s)) != cudaSuccess) return e;
+    // G4 and G3, then G5 and G6, as two launches with tiles claimed at run time
+    // when every contraction is at least 32 K steps deep (else one launch each)
+    const bool fused = L.M / BK >= kFusedMinSteps && L.N / BK >= kFusedMinSteps && L.R / BK >= kFusedMinSteps;
+    unsigned *ctl = reinterpret_cast<unsigned *>(body + b.ctl);
+    const int n_g3 = ((L.R + 2 * BM - 1) / (2 * BM)) * ((C + BN - 1) / BN);   // G3 tiles (G4 the same)
+    if ((e = scale_cast(x, xd, L.gamma, L.M, T, ell, U, s, 0, fused ? ctl : nullptr, fused ? 2 + n_g3 : 0)) !=
+        cudaSuccess)
+        return e;
     if ((e = scale_cast(dy, dyd, L.alpha, L.N, T, ell, A, s)) != cudaSuccess) return e;
     CUtensorMap mu, ma, mvh, mvg;
     // the four sign GEMMs run on CTA pairs (each CTA loads half of a token tile)
@@ -1889,37 +1934,63 @@ cudaError_t gemm_backward(const dbf_layer &L, const uint32_t *b1t, const uint32_
     if (!make_map(&mu, U, L.M, C, kb) || !make_map(&ma, A, L.N, C, kb) || !make_map(&mvh, Vh, L.R, C, kb) ||
         !make_map(&mvg, Vg, L.R, C, kb))
         return cudaErrorInvalidValue;
-    // G3
     GemmArgs g3 = sign_gemm_args(L.b2_packed, L.R, L.M, C, Ti, ell, 3);
     g3.H32 = H32;
     g3.Vout = Vh;
     g3.cscale = L.beta;
-    if ((e = launch_gemm_pair<BwdPairCfg>(mu, g3, s, st)) != cudaSuccess) return e;
-    // G4
     GemmArgs g4 = sign_gemm_args(b1t, L.R, L.N, C, Ti, ell, 4);
     g4.H32 = H32;
     g4.Vout = Vg;
     g4.cscale = L.beta;
     g4.red = dbeta;
-    if ((e = launch_gemm_pair<BwdPairCfg>(ma, g4, s, st)) != cudaSuccess) return e;
-    // G5
+    GemmArgs g5 = {}, g6 = {};
     if (dalpha) {
-        GemmArgs g5 = sign_gemm_args(L.b1_packed, L.N, L.R, C, Ti, ell, 5);
+        g5 = sign_gemm_args(L.b1_packed, L.N, L.R, C, Ti, ell, 5);
         g5.red = dalpha;
         g5.W = dy;
         g5.wd = dyd;
-        if ((e = launch_gemm_pair<BwdPairCfg>(mvh, g5, s, st)) != cudaSuccess) return e;
     }
-    // G6
     if (dx || dgamma) {
-        GemmArgs g6 = sign_gemm_args(b2t, L.M, L.R, C, Ti, ell, 6);
+        g6 = sign_gemm_args(b2t, L.M, L.R, C, Ti, ell, 6);
         g6.red = dgamma;
         g6.W = x;
         g6.wd = xd;
         g6.cscale = L.gamma;
         g6.dx = dx;
         g6.dx_mode = ell > 1 ? 2 : (acc ? 1 : 0);
-        if ((e = launch_gemm_pair<BwdPairCfg>(mvg, g6, s, st)) != cudaSuccess) return e;
+    }
+    if (fused) {
+        // pair row tiles of P rows, token tiles of the C columns
+        auto rows = [](int P) { return (P + 2 * BM - 1) / (2 * BM); };
+        const int n_c = (C + BN - 1) / BN;
+        // G3 first, then G4, whose epilogue reads the h of the G3 tile of the
+        // same index: it waits for that tile's flag (G3 tiles are claimed
+        // first and never wait, so every flag is set)
+        FusedSched f1 = {};
+        f1.dep = 2;
+        f1.n_p1 = rows(L.R);
+        f1.n1 = f1.n_p1 * n_c;
+        f1.n_p2 = rows(L.R);
+        f1.ctr = ctl;
+        f1.flags = ctl + 2;
+        f1.flag_target = 2 * BwdFusedCfg::kEpiWarps;
+        if ((e = launch_fused<BwdFusedCfg>(mu, ma, g3, g4, f1, f1.n_p2 * n_c, L.M / BK, L.N / BK, true, s, st)) !=
+            cudaSuccess)
+            return e;
+        // G5 and G6 read what G3 and G4 wrote: a plain launch after them
+        FusedSched f2 = {};
+        f2.n_p1 = rows(L.N);
+        f2.n1 = dalpha ? f2.n_p1 * n_c : 0;
+        f2.n_p2 = rows(L.M);
+        f2.ctr = ctl + 1;
+        if ((e = launch_fused<BwdFusedCfg>(mvh, mvg, g5, g6, f2, (dx || dgamma) ? f2.n_p2 * n_c : 0, L.R / BK,
+                                           L.R / BK, false, s, st)) != cudaSuccess)
+            return e;
+    } else {
+        if ((e = launch_gemm_pair<BwdPairCfg>(mu, g3, s, st)) != cudaSuccess) return e;
+        if ((e = launch_gemm_pair<BwdPairCfg>(ma, g4, s, st)) != cudaSuccess) return e;
+        if (dalpha && (e = launch_gemm_pair<BwdPairCfg>(mvh, g5, s, st)) != cudaSuccess) return e;
+        if ((dx || dgamma) && (e = launch_gemm_pair<BwdPairCfg>(mvg, g6, s, st)) != cudaSuccess) return e;
     }
     // sign-matrix gradients: dB1 = sum_c a_c v_c^T (N x R), dB2 = sum_c w_c u_c^T
     // (R x M), dense products contracting over the envelope-major token index

@@ -72,6 +72,33 @@ def test_backward_matches_oracle(dbf, case, kind):
     assert rel_err(g.dgamma.cpu().numpy(), ref.dgamma) < TOL
 
 
+# Shapes whose contractions are all at least 32 K steps deep: the sign GEMMs
+# run as two launches (G4 with G3, G5 with G6) with tiles claimed at run
+# time; two envelopes with ell T across 256-column tiles, ragged rows.
+FUSED_CASES = [(2048, 2304, 2048, 2, 300), (2048, 2176, 2048, 1, 129)]
+
+
+@pytest.mark.parametrize("case", FUSED_CASES, ids=lambda c: "M{}N{}R{}l{}T{}".format(*c))
+def test_backward_claimed_tiles_match_oracle(dbf, case):
+    M, N, R, ell, T = case
+    rng = np.random.default_rng(M + 5 * N + ell + T)
+    L = random_layer(rng, M, N, R, ell)
+    x = S.to_bf16_bits(rng.standard_normal((T, M)))
+    dy = S.to_bf16_bits(rng.standard_normal((T, N)))
+    ref = oracle.backward(L, x, dy)
+    dl, g = gpu_grads(dbf, L, x, dy)
+    assert rel_err(g.dx.cpu().numpy(), ref.dx) < TOL
+    assert rel_err(g.dalpha.cpu().numpy(), ref.dalpha) < TOL
+    assert rel_err(g.dbeta.cpu().numpy(), ref.dbeta) < TOL
+    assert rel_err(g.dgamma.cpu().numpy(), ref.dgamma) < TOL
+    # without dalpha the second launch holds G6's tiles only
+    only = dbf.backward(dl, dev_x(x), dev_x(dy), want=("dx", "dbeta"))
+    torch.cuda.synchronize()
+    assert only.dalpha is None
+    assert rel_err(only.dx.cpu().numpy(), ref.dx) < TOL
+    assert rel_err(only.dbeta.cpu().numpy(), ref.dbeta) < TOL
+
+
 def test_backward_accumulate_and_optional_outputs(dbf):
     rng = np.random.default_rng(91)
     L = random_layer(rng, 256, 256, 128, 2)
