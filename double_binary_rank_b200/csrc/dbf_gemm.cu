@@ -2038,7 +2038,8 @@ cudaError_t mbok_forward(int M, int N, int K, const uint32_t *w_packed, const ui
     cudaError_t e = scale_cast(x, xd, s_in, M, T, K, U, s, 1);
     if (e != cudaSuccess) return e;
     CUtensorMap mu;
-    if (!make_map(&mu, U, static_cast<int64_t>(K) * M, T)) return cudaErrorInvalidValue;
+    // CTA pairs: each CTA loads 128 of a tile's 256 token rows
+    if (!make_map(&mu, U, static_cast<int64_t>(K) * M, T, FwdPairCfg::kBRows)) return cudaErrorInvalidValue;
     GemmArgs a = {};
     a.signs = w_packed;
     a.pitch = static_cast<int>(pitch_words(static_cast<int64_t>(K) * M));
@@ -2055,7 +2056,7 @@ cudaError_t mbok_forward(int M, int N, int K, const uint32_t *w_packed, const ui
     a.yd = yd;
     a.N = N;
     a.accumulate = (flags & DBF_ACCUMULATE) ? 1 : 0;
-    return launch_gemm<FwdCfg>(mu, a, s, nullptr, st);
+    return launch_gemm_pair<FwdPairCfg>(mu, a, s, st);
 }
 
 }  // namespace dbf
