@@ -428,6 +428,17 @@ def profile_calls(name: str, calls: int = 3):
         ws = dbf.alloc_workspace(dbf.backward_workspace_bytes(dl, T_PREFILL), dev)
         grads = dbf.backward(dl, x, dy, signs_t=signs_t, ws=ws)
         fn = lambda: dbf.backward(dl, x, dy, signs_t=signs_t, grads=grads, ws=ws)
+    elif name == "segmented_prefill":
+        # 32 adapters (4096 -> 4096, R = 128, two envelopes), 256 tokens each,
+        # through the host-planned segmented forward (grouped GEMMs)
+        n_ad, per, M = 32, 256, 4096
+        layers = [dev_layer(S.make_layer(0xDBF00007, M, M, 128, 2, 0.5, adapter=a)) for a in range(n_ad)]
+        offs = np.arange(0, (n_ad + 1) * per, per, dtype=np.int32)
+        ids = np.arange(n_ad, dtype=np.int32)
+        x = torch.randn((n_ad * per, M), device=dev).to(torch.bfloat16)
+        y = torch.empty((n_ad * per, M), dtype=torch.bfloat16, device=dev)
+        ws = dbf.alloc_workspace(dbf.segmented_planned_workspace_bytes(layers, offs, ids, M, M, n_ad * per), dev)
+        fn = lambda: dbf.forward_segmented_planned(layers, offs, ids, x, y=y, ws=ws)
     elif name == "segmented":
         w = S.WORKLOADS["segmented"]
         Ls = S.workload_layers(w)
@@ -465,7 +476,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--profile", choices=["decode", "prefill", "tiny", "adapter64", "segmented", "large_prefill",
-                                          "backward"],
+                                          "backward", "segmented_prefill"],
                     help="run three calls of one configuration and exit (no timing; for ncu captures)")
     args = ap.parse_args()
     if args.profile:

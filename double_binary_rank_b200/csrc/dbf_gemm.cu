@@ -1309,9 +1309,68 @@ __global__ void __launch_bounds__(256) transpose_f16_kernel(const uint16_t *__re
     }
 }
 
-// u[(i T + t), m] = fp16(gamma_i[m] x[t, m]); eight columns per thread with
-// 16-byte loads and stores when M % 8 == 0 and gamma is 16-byte aligned
-// (then a block takes whole rows).
+// Eight fp16 products of a row's 16-byte piece m8 (x in bf16 or fp32).
+__device__ __forceinline__ uint4 scale8(const uint4 &gw, const uint4 &xa, const uint4 &xb, dbf_dtype xd)
+{
+    float xv[8];
+    if (xd == DBF_BF16) {
+        const __nv_bfloat16 *xh = reinterpret_cast<const __nv_bfloat16 *>(&xa);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) xv[e] = __bfloat162float(xh[e]);
+    } else {
+        const float *f0 = reinterpret_cast<const float *>(&xa);
+        const float *f1 = reinterpret_cast<const float *>(&xb);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            xv[e] = f0[e];
+            xv[4 + e] = f1[e];
+        }
+    }
+    const __half *gh = reinterpret_cast<const __half *>(&gw);
+    uint4 out;
+    __half *oh = reinterpret_cast<__half *>(&out);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) oh[e] = __float2half_rn(__half2float(gh[e]) * xv[e]);
+    return out;
+}
+
+// One row u[row] = fp16(gamma . x[t]) by one warp: four 16-byte pieces per
+// lane in flight at a time (vectorised when M % 8 == 0 and gamma is 16-byte
+// aligned), else one column per lane.
+__device__ __forceinline__ void scale_row_warp(const void *x, dbf_dtype xd, const uint16_t *gp, int64_t xr, int M,
+                                               __half *up, bool vec8, int lane)
+{
+    if (vec8) {
+        const int M8 = M / 8;
+        for (int base = lane; base < M8; base += 4 * 32) {
+            uint4 gw[4], xa[4], xb[4];
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+                const int m8 = base + 32 * v;
+                if (m8 >= M8) continue;
+                gw[v] = __ldg(reinterpret_cast<const uint4 *>(gp) + m8);
+                if (xd == DBF_BF16) {
+                    xa[v] = __ldg(reinterpret_cast<const uint4 *>(static_cast<const __nv_bfloat16 *>(x) + xr) + m8);
+                } else {
+                    const uint4 *xf = reinterpret_cast<const uint4 *>(static_cast<const float *>(x) + xr) + 2 * m8;
+                    xa[v] = __ldg(xf);
+                    xb[v] = __ldg(xf + 1);
+                }
+            }
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+                const int m8 = base + 32 * v;
+                if (m8 < M8) reinterpret_cast<uint4 *>(up)[m8] = scale8(gw[v], xa[v], xb[v], xd);
+            }
+        }
+    } else {
+        for (int m = lane; m < M; m += 32) up[m] = __float2half_rn(h2f(gp[m]) * load_act(x, xd, xr + m));
+    }
+}
+
+// u[(i T + t), m] = fp16(gamma_i[m] x[t, m]); with M % 8 == 0 and gamma
+// 16-byte aligned a warp takes whole rows with 16-byte loads and stores,
+// else one column per thread.
 // tok_major: output row t ell + i (U is [T][ell M], blocks of one token side
 // by side) instead of i T + t.
 // zero[0 .. nzero-1] are cleared too (the fused forward's claim state), and
@@ -1325,64 +1384,15 @@ __global__ void __launch_bounds__(256) scale_cast_kernel(const void *x, dbf_dtyp
         for (int i = threadIdx.x; i < nzero; i += blockDim.x) zero[i] = 0u;
     const int64_t total = static_cast<int64_t>(ell) * T * M;
     if (vec8) {
-        // rows r0, r0 + G, .. r0 + 3G of a block (G = gridDim.x) together, eight
-        // columns per thread: the row's (envelope, token) found once per row
-        // (ell T <= 2^30: 32-bit), all loads of the four rows in flight first
-        const int M8 = M / 8;
-        const int nrows = ell * T;
-        constexpr int kU = 4;
-        for (int r0 = blockIdx.x; r0 < nrows; r0 += kU * gridDim.x) {
-            int64_t xrow[kU], grow_[kU];
-            bool rv[kU];
-#pragma unroll
-            for (int q = 0; q < kU; ++q) {
-                const int row = r0 + q * static_cast<int>(gridDim.x);
-                rv[q] = row < nrows;
-                const int i = tok_major ? row % ell : row / T;
-                const int t = tok_major ? row / ell : row - i * T;
-                xrow[q] = static_cast<int64_t>(t) * M;
-                grow_[q] = static_cast<int64_t>(i) * M;
-            }
-            for (int m8 = threadIdx.x; m8 < M8; m8 += blockDim.x) {
-                uint4 gw[kU], xa[kU], xb[kU];
-#pragma unroll
-                for (int q = 0; q < kU; ++q) {
-                    if (!rv[q]) continue;
-                    gw[q] = __ldg(reinterpret_cast<const uint4 *>(gamma + grow_[q]) + m8);
-                    if (xd == DBF_BF16) {
-                        xa[q] = __ldg(reinterpret_cast<const uint4 *>(static_cast<const __nv_bfloat16 *>(x) + xrow[q]) + m8);
-                    } else {
-                        const uint4 *xf = reinterpret_cast<const uint4 *>(static_cast<const float *>(x) + xrow[q]) + 2 * m8;
-                        xa[q] = __ldg(xf);
-                        xb[q] = __ldg(xf + 1);
-                    }
-                }
-#pragma unroll
-                for (int q = 0; q < kU; ++q) {
-                    if (!rv[q]) continue;
-                    float xv[8];
-                    if (xd == DBF_BF16) {
-                        const __nv_bfloat16 *xh = reinterpret_cast<const __nv_bfloat16 *>(&xa[q]);
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) xv[e] = __bfloat162float(xh[e]);
-                    } else {
-                        const float *f0 = reinterpret_cast<const float *>(&xa[q]);
-                        const float *f1 = reinterpret_cast<const float *>(&xb[q]);
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            xv[e] = f0[e];
-                            xv[4 + e] = f1[e];
-                        }
-                    }
-                    const __half *gh = reinterpret_cast<const __half *>(&gw[q]);
-                    uint4 out;
-                    __half *oh = reinterpret_cast<__half *>(&out);
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) oh[e] = __float2half_rn(__half2float(gh[e]) * xv[e]);
-                    const int row = r0 + q * static_cast<int>(gridDim.x);
-                    reinterpret_cast<uint4 *>(U)[static_cast<int64_t>(row) * M8 + m8] = out;
-                }
-            }
+        // one row per warp step (see scale_row_warp)
+        const int lane = threadIdx.x & 31;
+        const int nrows = ell * T;   // <= 2^30
+        const int nw = static_cast<int>((gridDim.x * blockDim.x) >> 5);
+        for (int row = static_cast<int>((blockIdx.x * blockDim.x + threadIdx.x) >> 5); row < nrows; row += nw) {
+            const int i = tok_major ? row % ell : row / T;
+            const int t = tok_major ? row / ell : row - i * T;
+            scale_row_warp(x, xd, gamma + static_cast<int64_t>(i) * M, static_cast<int64_t>(t) * M, M,
+                           U + static_cast<int64_t>(row) * M, true, lane);
         }
         return;
     }
@@ -1409,43 +1419,23 @@ __global__ void __launch_bounds__(256) scale_cast_grouped_kernel(const void *x, 
                                                                  const __grid_constant__ GammaGroups gg, int M, int T,
                                                                  int ell, __half *U, int vec8)
 {
-    // one row (i T + t) per block step: the group is found once per row
-    for (int64_t row = blockIdx.x; row < static_cast<int64_t>(ell) * T; row += gridDim.x) {
-        const int i = static_cast<int>(row / T);
-        const int t = static_cast<int>(row - static_cast<int64_t>(i) * T);
+    // one row (i T + t) per warp step; the row's group is found by the warp
+    // together (lane k tests groups k, k + 32, ...)
+    const int lane = threadIdx.x & 31;
+    const int nrows = ell * T;   // <= 2^30
+    const int nw = static_cast<int>((gridDim.x * blockDim.x) >> 5);
+    for (int row = static_cast<int>((blockIdx.x * blockDim.x + threadIdx.x) >> 5); row < nrows; row += nw) {
+        const int i = row / T;
+        const int t = row - i * T;
         int gi = -1;
-        for (int q = 0; q < gg.ngroups; ++q)
-            if (t >= gg.off[q] && t < gg.off[q] + gg.n[q]) gi = q;
-        if (gi < 0) continue;
+        for (int k = lane; k < gg.ngroups; k += 32)
+            if (t >= gg.off[k] && t < gg.off[k] + gg.n[k]) gi = k;
+        const unsigned found = __ballot_sync(0xffffffffu, gi >= 0);
+        if (!found) continue;
+        gi = __shfl_sync(0xffffffffu, gi, __ffs(found) - 1);
         const uint16_t *gp = gg.gamma[gi] + static_cast<int64_t>(i) * M;
-        __half *up = U + row * M;
-        if (vec8 && (reinterpret_cast<uintptr_t>(gp) & 15u) == 0) {
-            for (int m8 = threadIdx.x; m8 < M / 8; m8 += blockDim.x) {
-                const uint4 gw = __ldg(reinterpret_cast<const uint4 *>(gp) + m8);
-                float xv[8];
-                if (xd == DBF_BF16) {
-                    const uint4 xw = __ldg(reinterpret_cast<const uint4 *>(static_cast<const __nv_bfloat16 *>(x) +
-                                                                           static_cast<int64_t>(t) * M) + m8);
-                    const __nv_bfloat16 *xb = reinterpret_cast<const __nv_bfloat16 *>(&xw);
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) xv[e] = __bfloat162float(xb[e]);
-                } else {
-                    const float4 *xf = reinterpret_cast<const float4 *>(static_cast<const float *>(x) + static_cast<int64_t>(t) * M) + 2 * m8;
-                    const float4 c0 = __ldg(xf), c1 = __ldg(xf + 1);
-                    xv[0] = c0.x; xv[1] = c0.y; xv[2] = c0.z; xv[3] = c0.w;
-                    xv[4] = c1.x; xv[5] = c1.y; xv[6] = c1.z; xv[7] = c1.w;
-                }
-                const __half *gh = reinterpret_cast<const __half *>(&gw);
-                uint4 out;
-                __half *oh = reinterpret_cast<__half *>(&out);
-#pragma unroll
-                for (int e = 0; e < 8; ++e) oh[e] = __float2half_rn(__half2float(gh[e]) * xv[e]);
-                reinterpret_cast<uint4 *>(up)[m8] = out;
-            }
-        } else {
-            for (int m = threadIdx.x; m < M; m += blockDim.x)
-                up[m] = __float2half_rn(h2f(gp[m]) * load_act(x, xd, static_cast<int64_t>(t) * M + m));
-        }
+        scale_row_warp(x, xd, gp, static_cast<int64_t>(t) * M, M, U + static_cast<int64_t>(row) * M,
+                       vec8 && (reinterpret_cast<uintptr_t>(gp) & 15u) == 0, lane);
     }
 }
 
@@ -1717,7 +1707,7 @@ cudaError_t gemm_forward(const dbf_layer &L, const void *x, dbf_dtype xd, void *
     {
         const int64_t total = static_cast<int64_t>(L.ell) * T * L.M;
         const int vec8 = (L.M % 8 == 0) && ((reinterpret_cast<uintptr_t>(L.gamma) & 15u) == 0);
-        int64_t blocks = vec8 ? static_cast<int64_t>(L.ell) * T : (total + 255) / 256;
+        int64_t blocks = vec8 ? (static_cast<int64_t>(L.ell) * T + 7) / 8 : (total + 255) / 256;
         if (blocks > 8 * device_sms()) blocks = 8 * device_sms();
         scale_cast_kernel<<<static_cast<int>(blocks), 256, 0, s>>>(x, xd, L.gamma, L.M, Ti, L.ell, U, vec8, 0,
                                                                    fused ? ctl : nullptr, fused ? ctl_words(L, T) : 0);
@@ -1790,7 +1780,7 @@ cudaError_t scale_cast(const void *x, dbf_dtype xd, const uint16_t *scale, int K
 {
     const int64_t total = static_cast<int64_t>(ell) * T * K;
     const int vec8 = (K % 8 == 0) && ((reinterpret_cast<uintptr_t>(scale) & 15u) == 0);
-    int64_t blocks = vec8 ? static_cast<int64_t>(ell) * T : (total + 255) / 256;
+    int64_t blocks = vec8 ? (static_cast<int64_t>(ell) * T + 7) / 8 : (total + 255) / 256;
     if (blocks > 8 * device_sms()) blocks = 8 * device_sms();
     scale_cast_kernel<<<static_cast<int>(blocks), 256, 0, s>>>(x, xd, scale, K, static_cast<int>(T), ell, out, vec8,
                                                                tok_major, zero, nzero);
@@ -2087,8 +2077,8 @@ cudaError_t gemm_forward_grouped(const dbf_layer *const *layers, const int *off,
         gg.gamma[k] = layers[k]->gamma;
     }
     {
-        int64_t blocks = static_cast<int64_t>(L.ell) * T;
-        if (blocks > 148 * 16) blocks = 148 * 16;
+        int64_t blocks = (static_cast<int64_t>(L.ell) * T + 7) / 8;   // a warp per row
+        if (blocks > 8 * device_sms()) blocks = 8 * device_sms();
         scale_cast_grouped_kernel<<<static_cast<int>(blocks), 256, 0, s>>>(x, xd, gg, L.M, Ti, L.ell, U, L.M % 8 == 0);
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;
