@@ -741,6 +741,11 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap &tmB, const CUtensor
             asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
         }
     }
+    // A launch that follows with programmatic stream serialisation (the next
+    // decode call) may be set up now: it cannot become resident before this
+    // grid's CTAs leave their SMs, and it waits (griddepcontrol.wait) for
+    // this grid to complete before it touches anything this grid writes.
+    if (kFused) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     tc_fence_before();
     __syncthreads();
     if (kPair) {
