@@ -165,8 +165,10 @@ def test_gemm_wrapping_shape_sampled_rows(dbf):
 # deep): tiles claimed at run time, stage-2 tiles that wait for the stage-1
 # column blocks they read, ragged rows and tokens; the second has two
 # envelopes whose column blocks straddle the envelope boundary (ell T = 2200),
-# and the last two run their final stage-2 tiles as 128-token halves.
-FUSED = [(2048, 1000, 2048, 1, 700), (2048, 2500, 1024, 2, 1100), (4096, 4096, 2048, 1, 1024)]
+# the second and third split their last stage-2 tiles in K, and the last two
+# have one and three tokens (one column block).
+FUSED = [(2048, 1000, 2048, 1, 700), (2048, 2500, 1024, 2, 1100), (4096, 4096, 2048, 1, 1024),
+         (2048, 512, 2048, 1, 1), (2048, 768, 1024, 2, 3)]
 
 
 @pytest.mark.parametrize("shape", FUSED, ids=lambda s: "M{}N{}R{}l{}T{}".format(*s))
