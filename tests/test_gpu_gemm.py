@@ -102,6 +102,21 @@ def test_dbf_mlp_prefill_sampled_rows(dbf):
     assert ok, worst
 
 
+def test_dbf_mlp_prefill_deterministic(dbf):
+    # The DBF MLP layer at 2048 tokens takes the one-launch forward with its
+    # last stage-2 tiles split in K: which pair runs which tile, and which half
+    # of a split tile finishes first, vary between calls; y does not.
+    w = S.WORKLOADS["dbf_mlp"]
+    L = S.workload_layers(w)[0]
+    x = S.make_x(w.seed + 7, 2048, w.M, "bf16")
+    dl = dev_layer(L)
+    xd = dev_x(x)
+    a = dbf.forward(dl, xd, path="gemm", y_dtype=torch.float32)
+    b = dbf.forward(dl, xd, path="gemm", y_dtype=torch.float32)
+    torch.cuda.synchronize()
+    assert torch.equal(a, b)
+
+
 def test_large_prefill_sampled_rows(dbf):
     # M = N = R = 8192 at 8192 tokens, checked on a fixed sample of token rows
     w = S.WORKLOADS["large_prefill"]
