@@ -82,6 +82,8 @@ _SIGS = {
                                                   ctypes.c_int, _vp]),
     "dbf_debug_set_decode_wait_ns": (None, [ctypes.c_uint64]),
     "dbf_debug_noalloc_header": (ctypes.c_int, [ctypes.POINTER(ctypes.c_uint64), ctypes.POINTER(ctypes.c_int32)]),
+    "dbf_debug_fused_schedule": (ctypes.c_int, [_LP, _i64, ctypes.c_int32, ctypes.POINTER(ctypes.c_int32),
+                                                ctypes.POINTER(ctypes.c_double)]),
     "dbf_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "dbf_version": (ctypes.c_char_p, []),
 }

@@ -1776,6 +1776,28 @@ cudaError_t gemm_forward(const dbf_layer &L, const void *x, dbf_dtype xd, void *
 
 }  // namespace dbf
 
+// The one-launch forward's schedule as chosen for a layer and token count
+// with 'pairs' resident CTA pairs (host-side model; see dbf.h).
+extern "C" dbf_status dbf_debug_fused_schedule(const dbf_layer *L, int64_t T, int32_t pairs, int32_t *tiles,
+                                               double *makespan)
+{
+    using namespace dbf;
+    if (!L || !tiles || !makespan || T < 1 || pairs < 1 || L->M <= 0 || L->N <= 0 || L->R <= 0 || L->ell < 1)
+        return DBF_ERR_INVALID_ARG;
+    if (!gemm_shape_ok(*L) || gemm_forward_launches(*L) != 2) return DBF_ERR_UNSUPPORTED;
+    const int nk1 = L->M / BK, nk2 = L->ell * L->R / BK;
+    const int n_c1 = static_cast<int>((static_cast<int64_t>(L->ell) * T + BN - 1) / BN);
+    const int n1 = ((L->R + 2 * BM - 1) / (2 * BM)) * n_c1;
+    const int n2 = ((L->N + 2 * BM - 1) / (2 * BM)) * static_cast<int>((T + BN - 1) / BN);
+    const int nsk = fused_splits(pairs, n1, n2, nk1, nk2, std::min(n2, kMaxSplit));
+    tiles[0] = n1;
+    tiles[1] = n2;
+    tiles[2] = nsk;
+    makespan[0] = fused_makespan(pairs, n1, n2, 0, nk1, nk2);
+    makespan[1] = fused_makespan(pairs, n1, n2, nsk, nk1, nk2);
+    return DBF_OK;
+}
+
 // ---- backward (tcgen05, four sign GEMMs) ---------------------------------------
 namespace dbf {
 namespace {

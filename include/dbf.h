@@ -420,6 +420,17 @@ dbf_status dbf_forward_decode_noalloc(const dbf_layer *L, const void *x, dbf_dty
  * address lookup or the copy fails. */
 dbf_status dbf_debug_noalloc_header(uint64_t *barrier_word, int32_t *status);
 
+/* The schedule dbf_forward's prefill path would use for layer *L (shapes
+ * only: no pointer is read) and T tokens when 'pairs' CTA pairs can be
+ * resident: tiles[0] stage-1 tiles, tiles[1] stage-2 tiles, tiles[2] of them
+ * split in two halves of K; makespan[0] and makespan[1] the claim-order
+ * model's makespans (in K steps) without and with those splits. Host only,
+ * for tests of the model. DBF_ERR_UNSUPPORTED when the layer does not take
+ * the one-launch forward (a stage under 32 K steps, or M or R not a multiple
+ * of 128); DBF_ERR_INVALID_ARG for null pointers or non-positive sizes. */
+dbf_status dbf_debug_fused_schedule(const dbf_layer *L, int64_t T, int32_t pairs, int32_t *tiles,
+                                    double *makespan);
+
 /* Time limit of the grid-barrier wait of the single-launch decode kernel
  * for the calls made after this one, in this process, counted from each
  * CTA's start and checked before every poll: ns > 0 sets it, 0 restores the
