@@ -60,19 +60,28 @@ constexpr int BN = 256;             // token rows per tile (MMA N)
 constexpr int BK = 64;              // K per stage: one 128-byte swizzle row of fp16
 // Pipeline shapes, per kernel instance. The forward keeps two expansion
 // groups (alternating pairs of K steps) and four epilogue warps; the
-// backward, whose epilogues read and write an operand per element, takes
-// eight epilogue warps (two per TMEM lane quarter, each with half of the
-// columns) and one expansion group.
-template <int kGroups, int kSA, int kSB, int kEpi, bool kBackward, bool kPairMode = false, bool kFusedMode = false>
+// one-launch forward, whose 512-column tiles leave no accumulator free for
+// the next tile during an epilogue, and the backward, whose epilogues read
+// and write an operand per element, take eight epilogue warps (two per TMEM
+// lane quarter, each with half of the columns); the backward keeps one
+// expansion group.
+template <int kGroups, int kSA, int kSB, int kEpi, bool kBackward, bool kPairMode = false, bool kFusedMode = false,
+          bool kWideMode = false>
 struct GemmCfg {
     static constexpr bool kBwd = kBackward;      // epilogues of stages 3..6 compiled in
     static constexpr bool kFused = kFusedMode;   // both forward stages in one launch (gemm_fused_kernel)
+    // 512-token pair tiles: every expanded sign stage feeds two MMAs, one
+    // per 256-token half, into two accumulators that fill the 512 tensor
+    // memory columns (so one tile's epilogue is not overlapped with the next
+    // tile's MMAs); halves the sign expansion per flop
+    static constexpr bool kWide = kWideMode;
+    static constexpr int kTBN = kWideMode ? 2 * BN : BN;   // token rows per tile
     // CTA pairs (a cluster of two): tcgen05 cta_group::2 with M = 256 over the
     // two SMs; each CTA holds its 128 sign rows of A and half of the 256 token
     // rows of B, and its TMEM the accumulator of its 128 rows
     static constexpr bool kPair = kPairMode;
     static constexpr int kBRows = kPairMode ? 128 : 256;   // B rows a CTA loads per stage
-    static constexpr int kBBytes = kBRows * 64 * 2;
+    static constexpr int kBBytes = kBRows * 64 * 2 * (kWideMode ? 2 : 1);   // B bytes a CTA holds per stage
     static constexpr int SA = kSA;               // stages of expanded sign tiles (produced on chip)
     static constexpr int SB = kSB;               // stages of TMA activation tiles
     static constexpr int kExpandGroups = kGroups;
@@ -82,7 +91,7 @@ struct GemmCfg {
 };
 using FwdCfg = GemmCfg<2, 6, 4, 4, false>;
 using FwdPairCfg = GemmCfg<2, 6, 6, 4, false, true>;
-using FusedCfg = GemmCfg<2, 6, 6, 4, false, true, true>;
+using FusedCfg = GemmCfg<2, 6, 4, 8, false, true, true, true>;
 using BwdPairCfg = GemmCfg<1, 6, 6, 8, true, true>;
 using BwdFusedCfg = GemmCfg<1, 6, 6, 8, true, true, true>;   // two sign GEMMs of the backward in one launch
 constexpr int kMaxStages = 8;
@@ -147,13 +156,13 @@ struct TileRef {
     const GroupRef *gr;
 };
 
-__device__ __forceinline__ TileRef tile_ref(const GemmArgs &g, int tile, int n_p, int pair_rank = -1)
+__device__ __forceinline__ TileRef tile_ref(const GemmArgs &g, int tile, int n_p, int pair_rank = -1, int bn = BN)
 {
     TileRef r;
     if (pair_rank >= 0) {
         // a pair tile: 256 sign rows, this CTA's 128 of them
         r.p0 = (tile % n_p) * 2 * BM + pair_rank * BM;
-        r.brow = (tile / n_p) * BN;
+        r.brow = (tile / n_p) * bn;
         r.t0 = r.brow;
         r.t1 = g.C;
         r.env = 0;
@@ -402,6 +411,7 @@ __device__ __forceinline__ void grouped_chunk(const GemmArgs &g, const TileRef &
                                               int p)
 {
     const int n_ok = tr.t1 - t0;
+    if (n_ok <= 0) return;   // a chunk past the group's end: nothing to read or write
     if (g.stage == 1) {
         const float b = h2f(tr.gr->beta[static_cast<int64_t>(tr.env) * g.R + p]);
         const int64_t ts = static_cast<int64_t>(g.ell) * g.R;
@@ -668,9 +678,11 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap &tmB, const CUtensor
 {
     constexpr int SA = Cfg::SA, SB = Cfg::SB, kExpandGroups = Cfg::kExpandGroups;
     constexpr int kExpandWarps = Cfg::kExpandWarps, kEpiWarps = Cfg::kEpiWarps;
-    constexpr bool kFused = Cfg::kFused;
-    static_assert(SA <= kMaxStages && SB <= kMaxStages && kEpiWarps % 4 == 0 && BN % (32 * (kEpiWarps / 4)) == 0,
+    constexpr bool kFused = Cfg::kFused, kWide = Cfg::kWide;
+    constexpr int TBN = Cfg::kTBN;   // token rows per tile
+    static_assert(SA <= kMaxStages && SB <= kMaxStages && kEpiWarps % 4 == 0 && TBN % (32 * (kEpiWarps / 4)) == 0,
                   "pipeline shape");
+    static_assert(!kWide || (kFused && Cfg::kPair), "512-token tiles: the one-launch forward on CTA pairs");
     static_assert(!kFused || Cfg::kPair, "tiles are claimed by CTA pairs");
     extern __shared__ uint8_t smem_raw[];
     // 1024-byte alignment for the swizzled tiles
@@ -691,7 +703,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap &tmB, const CUtensor
     const int nunits = kPair ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
     const int tile_rank = kPair ? static_cast<int>(rank) : -1;
     const int n_p = (g.P + (kPair ? 2 * BM : BM) - 1) / (kPair ? 2 * BM : BM);
-    const int n_c = (g.C + BN - 1) / BN;
+    const int n_c = (g.C + TBN - 1) / TBN;
     const int ntiles = g.ngroups ? g.tiles_total : n_p * n_c;
     const int my_tiles = unit < ntiles ? (ntiles - 1 - unit) / nunits + 1 : 0;
     const int nk = g.Ktot / BK;
@@ -791,17 +803,17 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap &tmB, const CUtensor
                     }
                     const FusedTile f = fused_decode(*fs, u);
                     const GemmArgs &gs = fused_args(f);
-                    const TileRef tr = tile_ref(gs, f.t, f.stage == 1 ? fs->n_p1 : fs->n_p2, tile_rank);
+                    const TileRef tr = tile_ref(gs, f.t, f.stage == 1 ? fs->n_p1 : fs->n_p2, tile_rank, TBN);
                     const int c0 = tr.brow;
                     const CUtensorMap *mp = f.stage == 1 ? &tmB : &tmA;
                     bool ok = true;
                     if (f.stage == 2 && fs->dep == 1 && c0 < g.T) {
                         // the v rows of tokens [c0, t_hi) of every envelope: stage-1
-                        // column blocks (i T + t) / BN
-                        const int t_hi = min(c0 + BN, g.T);
+                        // column blocks (i T + t) / TBN
+                        const int t_hi = min(c0 + TBN, g.T);
                         const unsigned long long t0 = global_ns();
                         for (int i = 0; i < g.ell && ok; ++i) {
-                            const int b_lo = (i * g.T + c0) / BN, b_hi = (i * g.T + t_hi - 1) / BN;
+                            const int b_lo = (i * g.T + c0) / TBN, b_hi = (i * g.T + t_hi - 1) / TBN;
                             for (int b = b_lo; b <= b_hi && ok; ++b) {
                                 while (ld_acquire_u32(fs->flags + b) < fs->flag_target) {
                                     if (*abort) { ok = false; break; }
@@ -825,6 +837,9 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap &tmB, const CUtensor
                         if (rank == 0) bar_expect_tx(&sh->full_b[st], 2 * kBBytes);
                         tma_load_2d_pair(smB + st * kBBytes, mp, k * BK, c0 + static_cast<int>(rank) * Cfg::kBRows,
                                          &sh->full_b[st]);
+                        if (kWide)   // the second 256-token half, 16 KB further on
+                            tma_load_2d_pair(smB + st * kBBytes + kBBytes / 2, mp, k * BK,
+                                             c0 + BN + static_cast<int>(rank) * Cfg::kBRows, &sh->full_b[st]);
                         nb_issued = s + 1;
                     }
                     if (rank == 0) {
@@ -835,7 +850,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap &tmB, const CUtensor
                 }
             } else {
                 for (int j = 0; j < my_tiles && !*abort; ++j) {
-                    const TileRef tr = tile_ref(g, unit + j * nunits, n_p, tile_rank);
+                    const TileRef tr = tile_ref(g, unit + j * nunits, n_p, tile_rank, TBN);
                     const int c0 = tr.brow;
                     const int p0 = tr.p0;
                     for (int k = 0; k < nk; ++k, ++s) {
@@ -888,8 +903,10 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap &tmB, const CUtensor
                 } else if (j >= my_tiles) {
                     break;
                 }
-                const int ab = j & 1;
-                ok = wait(&sh->acc_empty[ab], ((j >> 1) & 1) ^ 1);
+                // two accumulators taking turns by tile, or (wide) one tile's
+                // two halves in them
+                const int ab = kWide ? 0 : (j & 1);
+                ok = wait(&sh->acc_empty[ab], (kWide ? (j & 1) : ((j >> 1) & 1)) ^ 1);
                 if (!ok) break;
                 tc_fence_after();
                 const uint32_t dt = tmem + static_cast<uint32_t>(ab * BN);
@@ -900,7 +917,17 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap &tmB, const CUtensor
                     tc_fence_after();
                     const uint64_t da = sw128_desc(smem_u32(smA + sa * A_BYTES));
                     const uint64_t db = sw128_desc(smem_u32(smB + sb * kBBytes));
-                    if (kPair) {
+                    if (kWide) {
+                        // the same sign stage for both token halves
+                        const uint64_t db1 = sw128_desc(smem_u32(smB + sb * kBBytes + kBBytes / 2));
+#pragma unroll
+                        for (int kk = 0; kk < BK / 16; ++kk) {
+                            mma_f16_pair(dt, da + 2 * kk, db + 2 * kk, (k != kb || kk) != 0);
+                            mma_f16_pair(dt + static_cast<uint32_t>(BN), da + 2 * kk, db1 + 2 * kk, (k != kb || kk) != 0);
+                        }
+                        mma_commit_pair_both(&sh->empty_a[sa]);
+                        mma_commit_pair_both(&sh->empty_b[sb]);
+                    } else if (kPair) {
 #pragma unroll
                         for (int kk = 0; kk < BK / 16; ++kk)
                             mma_f16_pair(dt, da + 2 * kk, db + 2 * kk, (k != kb || kk) != 0);
@@ -978,7 +1005,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap &tmB, const CUtensor
                 calive = false;
                 return;
             }
-            const TileRef tr = tile_ref(*cg, t, np, tile_rank);
+            const TileRef tr = tile_ref(*cg, t, np, tile_rank, TBN);
             cgrow = tr.p0 + prow;
             cvalid = cgrow < cg->P;
             carow = tr.gr ? tr.gr->arow : cg->arow_scale;
@@ -1084,7 +1111,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap &tmB, const CUtensor
         // ---------------- epilogue: one warp per TMEM lane quarter ----------------
         const int q = warp & 3;   // a warp reads the TMEM lane quarter warp % 4
         const int ch = kEpiWarps == 4 ? 0 : (warp - 2 - kExpandWarps) >> 2;   // which share of the columns
-        constexpr int kColShare = BN / (kEpiWarps / 4);
+        constexpr int kColShare = TBN / (kEpiWarps / 4);
         if (kFused) griddep_wait();   // the flags it counts on are zeroed by the pre-pass
         for (int j = 0;; ++j) {
             TileRef tr;
@@ -1098,21 +1125,21 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap &tmB, const CUtensor
                 if (!ring_get_warp(sh, j, u) || u < 0) break;
                 const FusedTile f = fused_decode(*fs, u);
                 ge = &fused_args(f);
-                tr = tile_ref(*ge, f.t, f.stage == 1 ? fs->n_p1 : fs->n_p2, tile_rank);
+                tr = tile_ref(*ge, f.t, f.stage == 1 ? fs->n_p1 : fs->n_p2, tile_rank, TBN);
                 stage1 = ge->stage == 1;   // the forward's stage 1 (v); the backward's GEMMs have stages 3..6
                 if (!Cfg::kBwd && f.part >= 0)   // only the forward splits tiles in K
                     sk = ((f.t - fs->n2f) * 2 + static_cast<int>(rank)) * kEpiWarps + (warp - 2 - kExpandWarps);
-                if (f.stage == 1 && fs->dep == 1) flag_out = tr.brow / BN;
+                if (f.stage == 1 && fs->dep == 1) flag_out = tr.brow / TBN;
                 if (f.stage == 1 && fs->dep == 2) flag_out = f.t;
                 if (f.stage == 2 && fs->dep == 2) flag_in = f.t;
             } else {
                 if (j >= my_tiles) break;
-                tr = tile_ref(g, unit + j * nunits, n_p, tile_rank);
+                tr = tile_ref(g, unit + j * nunits, n_p, tile_rank, TBN);
             }
             const GemmArgs &ga = *ge;
-            const int ab = j & 1;
+            const int ab = kWide ? 0 : (j & 1);
             bool got = true;
-            if (lane == 0) got = wait(&sh->acc_full[ab], (j >> 1) & 1);
+            if (lane == 0) got = wait(&sh->acc_full[ab], kWide ? (j & 1) : ((j >> 1) & 1));
             if (!__shfl_sync(0xffffffffu, got, 0)) break;
             tc_fence_after();
             if (kFused && flag_in >= 0) {
@@ -1142,7 +1169,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap &tmB, const CUtensor
                 unsigned old = 0;
                 if (lane == 0) old = atomicAdd(fs->sk_count + sk, 1u);
                 sk_first = __shfl_sync(0xffffffffu, old, 0) == 0;
-                sk_base = fs->sk_part + static_cast<int64_t>(sk / kEpiWarps) * (BM * BN) + q * 32 + lane;
+                sk_base = fs->sk_part + static_cast<int64_t>(sk / kEpiWarps) * (BM * TBN) + q * 32 + lane;
                 if (!sk_first && lane == 0) {
                     const unsigned long long t0 = global_ns();
                     while (ld_acquire_u32(fs->sk_ready + sk) == 0) {
@@ -1174,6 +1201,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap &tmB, const CUtensor
                     continue;
                 }
                 const int cb = c0 + cc;
+                if (cb >= ga.C) continue;   // a chunk past the last token (a ragged tile): nothing to read or write
                 if (stage1) {
                     // column c = i T + t; v[t, i R + r] = fp16(beta_i[r] h); (i, t)
                     // advance with c, beta reloaded only when i changes
@@ -1547,6 +1575,8 @@ cudaError_t launch_gemm_pair(const CUtensorMap &map, const GemmArgs &args, cudaS
 
 // ---- the fused forward's schedule ----------------------------------------------
 constexpr int kMaxSplit = 64;   // stage-2 tiles at most that run split in K
+// a split tile's counters: one per (split tile, CTA of the pair, epilogue warp)
+constexpr int kSkSlots = kMaxSplit * 2 * FusedCfg::kEpiWarps;
 
 // Makespan of the claim order (each pair claims its next tile when it starts
 // one) when the last nsk stage-2 tiles run as two halves of K, under a cost
@@ -1679,15 +1709,17 @@ bool gemm_shape_ok(const dbf_layer &L)
 // column-block flags and the split tiles' counters (zeroed by the pre-pass)
 int ctl_words(const dbf_layer &L, int64_t T)
 {
-    return static_cast<int>(1 + (static_cast<int64_t>(L.ell) * T + BN - 1) / BN + 2 * 8 * kMaxSplit);
+    constexpr int TBN = FusedCfg::kTBN;
+    return static_cast<int>(1 + (static_cast<int64_t>(L.ell) * T + TBN - 1) / TBN + 2 * kSkSlots);
 }
 
-// the split tiles' partial sums: 256 x 256 fp32 per split tile
+// the split tiles' partial sums: 256 x TBN fp32 per split tile
 size_t part_bytes(const dbf_layer &L, int64_t T)
 {
+    constexpr int TBN = FusedCfg::kTBN;
     if (gemm_forward_launches(L) != 2) return 0;
-    const int64_t n2 = ((L.N + 2 * BM - 1) / (2 * BM)) * ((T + BN - 1) / BN);
-    return static_cast<size_t>(std::min<int64_t>(n2, kMaxSplit)) * 2 * BM * BN * 4;
+    const int64_t n2 = ((L.N + 2 * BM - 1) / (2 * BM)) * ((T + TBN - 1) / TBN);
+    return static_cast<size_t>(std::min<int64_t>(n2, kMaxSplit)) * 2 * BM * TBN * 4;
 }
 
 size_t gemm_workspace_bytes(const dbf_layer &L, int64_t T)
@@ -1707,7 +1739,8 @@ cudaError_t gemm_forward(const dbf_layer &L, const void *x, dbf_dtype xd, void *
     const int Ti = static_cast<int>(T);
     unsigned *ctl = reinterpret_cast<unsigned *>(body + u_bytes(L, T) + v_bytes(L, T));
     const int nk1 = L.M / BK, nk2 = L.ell * L.R / BK;
-    const int n_c1 = static_cast<int>((static_cast<int64_t>(L.ell) * T + BN - 1) / BN);
+    constexpr int TBN = FusedCfg::kTBN;   // the one-launch forward's token rows per tile
+    const int n_c1 = static_cast<int>((static_cast<int64_t>(L.ell) * T + TBN - 1) / TBN);
     const bool fused = gemm_forward_launches(L) == 2;
     {
         const int64_t total = static_cast<int64_t>(L.ell) * T * L.M;
@@ -1763,9 +1796,9 @@ cudaError_t gemm_forward(const dbf_layer &L, const void *x, dbf_dtype xd, void *
         fs.flags = ctl + 1;
         fs.flag_target = static_cast<unsigned>(fs.n_p1 * 2 * FusedCfg::kEpiWarps);
         fs.sk_count = ctl + 1 + n_c1;
-        fs.sk_ready = fs.sk_count + 8 * kMaxSplit;
+        fs.sk_ready = fs.sk_count + kSkSlots;
         fs.sk_part = reinterpret_cast<float *>(reinterpret_cast<char *>(ctl) + align_up(4 * static_cast<size_t>(ctl_words(L, T)), 256));
-        const int n2 = fs.n_p2 * ((Ti + BN - 1) / BN);
+        const int n2 = fs.n_p2 * ((Ti + TBN - 1) / TBN);
         fs.dep = 1;
         return launch_fused<FusedCfg>(mu, mv, a1, a2, fs, n2, nk1, nk2, true, s, st);
     }
@@ -1786,9 +1819,10 @@ extern "C" dbf_status dbf_debug_fused_schedule(const dbf_layer *L, int64_t T, in
         return DBF_ERR_INVALID_ARG;
     if (!gemm_shape_ok(*L) || gemm_forward_launches(*L) != 2) return DBF_ERR_UNSUPPORTED;
     const int nk1 = L->M / BK, nk2 = L->ell * L->R / BK;
-    const int n_c1 = static_cast<int>((static_cast<int64_t>(L->ell) * T + BN - 1) / BN);
+    constexpr int TBN = FusedCfg::kTBN;
+    const int n_c1 = static_cast<int>((static_cast<int64_t>(L->ell) * T + TBN - 1) / TBN);
     const int n1 = ((L->R + 2 * BM - 1) / (2 * BM)) * n_c1;
-    const int n2 = ((L->N + 2 * BM - 1) / (2 * BM)) * static_cast<int>((T + BN - 1) / BN);
+    const int n2 = ((L->N + 2 * BM - 1) / (2 * BM)) * static_cast<int>((T + TBN - 1) / TBN);
     const int nsk = fused_splits(pairs, n1, n2, nk1, nk2, std::min(n2, kMaxSplit));
     tiles[0] = n1;
     tiles[1] = n2;

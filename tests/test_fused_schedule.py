@@ -27,14 +27,14 @@ def schedule(dbf, M, N, R, ell, T, pairs):
 
 
 def test_tile_counts(dbf):
-    # 256-row pair tiles of R (stage 1) and N (stage 2), 256-column blocks of
+    # 256-row pair tiles of R (stage 1) and N (stage 2), 512-column blocks of
     # ell T (stage 1) and T (stage 2)
     st, tiles, _ = schedule(dbf, 4096, 11008, 5888, 1, 2048, 74)
     assert st == dbf.OK
-    assert tiles[:2] == [23 * 8, 43 * 8]
+    assert tiles[:2] == [23 * 4, 43 * 4]
     st, tiles, _ = schedule(dbf, 2048, 2500, 1024, 2, 1100, 74)
     assert st == dbf.OK
-    assert tiles[:2] == [4 * math.ceil(2200 / 256), 10 * math.ceil(1100 / 256)]
+    assert tiles[:2] == [4 * math.ceil(2200 / 512), 10 * math.ceil(1100 / 512)]
 
 
 def test_single_wave_closed_form(dbf):
