@@ -1974,7 +1974,8 @@ cudaError_t gemm_backward(const dbf_layer &L, const uint32_t *b1t, const uint32_
     // when every contraction is at least 32 K steps deep (else one launch each)
     const bool fused = L.M / BK >= kFusedMinSteps && L.N / BK >= kFusedMinSteps && L.R / BK >= kFusedMinSteps;
     unsigned *ctl = reinterpret_cast<unsigned *>(body + b.ctl);
-    const int n_g3 = ((L.R + 2 * BM - 1) / (2 * BM)) * ((C + BN - 1) / BN);   // G3 tiles (G4 the same)
+    constexpr int TBN = BwdFusedCfg::kTBN;   // token columns per tile of the fused launches
+    const int n_g3 = ((L.R + 2 * BM - 1) / (2 * BM)) * ((C + TBN - 1) / TBN);   // G3 tiles (G4 the same)
     if ((e = scale_cast(x, xd, L.gamma, L.M, T, ell, U, s, 0, fused ? ctl : nullptr, fused ? 2 + n_g3 : 0)) !=
         cudaSuccess)
         return e;
@@ -2013,7 +2014,7 @@ cudaError_t gemm_backward(const dbf_layer &L, const uint32_t *b1t, const uint32_
     if (fused) {
         // pair row tiles of P rows, token tiles of the C columns
         auto rows = [](int P) { return (P + 2 * BM - 1) / (2 * BM); };
-        const int n_c = (C + BN - 1) / BN;
+        const int n_c = (C + TBN - 1) / TBN;
         // G3 first, then G4, whose epilogue reads the h of the G3 tile of the
         // same index: it waits for that tile's flag (G3 tiles are claimed
         // first and never wait, so every flag is set)
@@ -2074,9 +2075,10 @@ namespace dbf {
 
 bool mbok_shape_ok(int64_t M, int64_t N, int64_t K) { return M > 0 && N > 0 && K >= 1 && K <= 64 && M % 128 == 0; }
 
+// header, the fp16 operand (T x K M), the claim counter of the GEMM's tiles
 size_t mbok_workspace_bytes(int64_t M, int64_t K, int64_t T)
 {
-    return kWsHeaderBytes + align_up(static_cast<size_t>(T) * K * M * 2, 256);
+    return kWsHeaderBytes + align_up(static_cast<size_t>(T) * K * M * 2, 256) + 256;
 }
 
 cudaError_t mbok_forward(int M, int N, int K, const uint32_t *w_packed, const uint16_t *s_in, const uint16_t *s_out,
@@ -2086,7 +2088,9 @@ cudaError_t mbok_forward(int M, int N, int K, const uint32_t *w_packed, const ui
     int32_t *st = ws_status(ws);
     if (T > (1 << 30) / K) return cudaErrorInvalidValue;
     __half *U = reinterpret_cast<__half *>(static_cast<char *>(ws) + kWsHeaderBytes);
-    cudaError_t e = scale_cast(x, xd, s_in, M, T, K, U, s, 1);
+    unsigned *ctl = reinterpret_cast<unsigned *>(static_cast<char *>(ws) + kWsHeaderBytes +
+                                                 align_up(static_cast<size_t>(T) * K * M * 2, 256));
+    cudaError_t e = scale_cast(x, xd, s_in, M, T, K, U, s, 1, ctl, 1);   // also zeroes the claim counter
     if (e != cudaSuccess) return e;
     CUtensorMap mu;
     // CTA pairs: each CTA loads 128 of a tile's 256 token rows
@@ -2107,7 +2111,14 @@ cudaError_t mbok_forward(int M, int N, int K, const uint32_t *w_packed, const ui
     a.yd = yd;
     a.N = N;
     a.accumulate = (flags & DBF_ACCUMULATE) ? 1 : 0;
-    return launch_gemm_pair<FwdPairCfg>(mu, a, s, st);
+    // the one-launch kernel's 512-token pair tiles, all of them output tiles
+    // (no first stage), claimed at run time
+    constexpr int TBN = FusedCfg::kTBN;
+    FusedSched fs = {};
+    fs.n_p2 = (N + 2 * BM - 1) / (2 * BM);
+    fs.ctr = ctl;
+    const int n2 = fs.n_p2 * static_cast<int>((T + TBN - 1) / TBN);
+    return launch_fused<FusedCfg>(mu, mu, a, a, fs, n2, 0, K * M / BK, true, s, st);
 }
 
 }  // namespace dbf
