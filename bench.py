@@ -428,6 +428,27 @@ def profile_calls(name: str, calls: int = 3):
         ws = dbf.alloc_workspace(dbf.backward_workspace_bytes(dl, T_PREFILL), dev)
         grads = dbf.backward(dl, x, dy, signs_t=signs_t, ws=ws)
         fn = lambda: dbf.backward(dl, x, dy, signs_t=signs_t, grads=grads, ws=ws)
+    elif name == "mbok":
+        # the multi-boolean-kernel layer (4096 -> 4096, K = 3) at the prefill size
+        mb = S.make_mbok_layer(0xDBF00006, 4096, 4096, 3)
+        ml = dbf.MbokLayer.from_signs(torch.from_numpy(mb.w).to(dev), f16(mb.s_in), f16(mb.s_out))
+        x = bf16(S.make_x(0xDBF00006, T_PREFILL, 4096, "bf16"))
+        y = torch.empty((T_PREFILL, 4096), dtype=torch.bfloat16, device=dev)
+        ws = dbf.alloc_workspace(dbf.mbok_workspace_bytes(ml, T_PREFILL), dev)
+        fn = lambda: dbf.mbok_forward(ml, x, y=y, ws=ws)
+    elif name == "factorize":
+        # one outer iteration of the factorisation of an 11008 x 4096 fp32
+        # weight at k = 5888, 4 ADMM steps per factor (the bench's call);
+        # one call only (over a thousand launches)
+        n, m, k = 11008, 4096, 5888
+        gen = torch.Generator(device=dev)
+        gen.manual_seed(0xDBF00001)
+        W = torch.randn((n, m), device=dev, generator=gen)
+        U0 = 0.1 * torch.randn((n, k), device=dev, generator=gen)
+        V0 = 0.1 * torch.randn((k, m), device=dev, generator=gen)
+        ws = dbf.alloc_workspace(dbf.factorize_workspace_bytes(n, m, k, 1, 24), dev)
+        fn = lambda: dbf.factorize(W, U0, V0, outer=1, admm_iters=4, objective=False, ws=ws)
+        calls = 1
     elif name == "segmented_prefill":
         # 32 adapters (4096 -> 4096, R = 128, two envelopes), 256 tokens each,
         # through the host-planned segmented forward (grouped GEMMs)
@@ -476,7 +497,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--profile", choices=["decode", "prefill", "tiny", "adapter64", "segmented", "large_prefill",
-                                          "backward", "segmented_prefill"],
+                                          "backward", "segmented_prefill", "mbok", "factorize"],
                     help="run three calls of one configuration and exit (no timing; for ncu captures)")
     args = ap.parse_args()
     if args.profile:

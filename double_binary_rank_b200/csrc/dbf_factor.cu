@@ -245,15 +245,17 @@ struct LoScratch {
 // Cout[M x N] = alpha A B^T + beta Cin with A [M x K], B [N x K] (both
 // K-major): the tensor-core path (three TF32 products) when the operands
 // qualify, K fills at least one pipeline stage and the scratch holds the lo
-// planes, else the SIMT GEMM.
+// planes, else the SIMT GEMM. lower: a symmetric result of which only the
+// lower triangle is needed (the tensor-core path skips the tiles above the
+// diagonal; the SIMT GEMM computes all of it).
 cudaError_t gemm_nt(int64_t M, int64_t N, int64_t K, float alpha, const float *A, int64_t lda, const float *B,
                     int64_t ldb, float beta, const float *Cin, int64_t ldci, float *Cout, int64_t ldco, cudaStream_t s,
-                    const LoScratch &lo, double *sumsq = nullptr, int32_t *status = nullptr)
+                    const LoScratch &lo, double *sumsq = nullptr, int32_t *status = nullptr, bool lower = false)
 {
     if (M <= 0 || N <= 0) return cudaSuccess;
     if (K >= 32 && tf32x3_ok(M, N, K, A, lda, B, ldb) && lo.p && lo.floats >= tf32x3_scratch_floats(M, N, K))
         return tf32x3_gemm(M, N, K, alpha, A, lda, B, ldb, beta, Cin, ldci, Cout, ldco, sumsq, status, lo.p, lo.floats,
-                           s);
+                           s, lower);
     return sgemm(false, true, M, N, K, alpha, A, lda, B, ldb, beta, Cin, ldci, Cout, ldco, s, sumsq);
 }
 
@@ -262,14 +264,25 @@ constexpr int kSweepBlock = 128;
 constexpr int kSweepSeg = 16;                                         // columns per thread
 constexpr int kSweepThreads = kSweepBlock * kSweepBlock / kSweepSeg;   // 1024: 8 threads per row
 
-// P = A[:, p0 : p0 + bs] (k x bs, ld bs)
+// The sweep keeps the matrix symmetric and maintains its lower triangle
+// (and the diagonal blocks whole); the upper triangle is filled in at the end.
+// P = A[:, p0 : p0 + bs] (k x bs, ld bs): rows i >= p0 from the block column
+// (l fastest), rows i < p0 from the block row, A[p0 + l, i] (i fastest).
 __global__ void sweep_panel_kernel(const float *__restrict__ A, int64_t k, int64_t p0, int bs, float *__restrict__ P)
 {
+    const int64_t below = (k - p0) * bs;
     for (int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; idx < k * bs;
          idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-        const int64_t i = idx / bs;
-        const int l = static_cast<int>(idx - i * bs);
-        P[idx] = A[i * k + p0 + l];
+        if (idx < below) {
+            const int64_t d = idx / bs;
+            const int l = static_cast<int>(idx - d * bs);
+            P[(p0 + d) * bs + l] = A[(p0 + d) * k + p0 + l];
+        } else {
+            const int64_t j = idx - below;
+            const int l = static_cast<int>(j / p0);
+            const int64_t i = j - l * p0;
+            P[i * bs + l] = A[(p0 + l) * k + i];
+        }
     }
 }
 
@@ -417,25 +430,46 @@ __global__ void __launch_bounds__(kSweepThreads) sweep_block_inverse_kernel(cons
         if (i < bs && j0 + e < bs) D[i * bs + j0 + e] = -t[e];
 }
 
-// After A -= E P^T: the pivot block column and row become E and E^T, the
-// pivot block -D. Column writes run along l (contiguous in a row of A), row
-// writes along i (contiguous in a row of A).
+// After A -= E P^T: the pivot block becomes -D, the block column below it E
+// and the block row left of it E^T (the lower triangle's parts of the
+// pivot's row and column). Column writes run along l (contiguous in a row of
+// A), row writes along i (contiguous in a row of A).
 __global__ void sweep_fixup_kernel(float *__restrict__ A, int64_t k, int64_t p0, int bs, const float *__restrict__ E,
                                    const float *__restrict__ D)
 {
-    const int64_t total = k * bs;
-    for (int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; idx < total;
+    const int64_t below = (k - p0) * bs;
+    for (int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; idx < k * bs;
          idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-        {   // column block: (i, p0 + l), l fastest
-            const int64_t i = idx / bs;
-            const int l = static_cast<int>(idx - i * bs);
-            A[i * k + p0 + l] = (i >= p0 && i < p0 + bs) ? -D[(i - p0) * bs + l] : E[i * bs + l];
+        if (idx < below) {   // column block: (i, p0 + l), i >= p0
+            const int64_t i = p0 + idx / bs;
+            const int l = static_cast<int>(idx % bs);
+            A[i * k + p0 + l] = i < p0 + bs ? -D[(i - p0) * bs + l] : E[i * bs + l];
+        } else {   // row block: (p0 + l, i), i < p0
+            const int64_t j = idx - below;
+            const int l = static_cast<int>(j / p0);
+            const int64_t i = j - l * p0;
+            A[(p0 + l) * k + i] = E[i * bs + l];
         }
-        {   // row block: (p0 + l, i), i fastest
-            const int l = static_cast<int>(idx / k);
-            const int64_t i = idx - static_cast<int64_t>(l) * k;
-            if (i < p0 || i >= p0 + bs) A[(p0 + l) * k + i] = E[i * bs + l];
-        }
+    }
+}
+
+// The upper triangle of the symmetric k x k matrix A from its lower triangle,
+// through 32 x 32 tiles in shared memory (block (bx, by) writes the upper
+// tile at rows 32 by, columns 32 bx from the lower tile at rows 32 bx,
+// columns 32 by; blocks below the diagonal have nothing to do).
+__global__ void __launch_bounds__(256) sweep_mirror_kernel(float *__restrict__ A, int64_t k)
+{
+    __shared__ float t[32][33];
+    const int bx = blockIdx.x, by = blockIdx.y, tx = threadIdx.x;
+    if (bx < by) return;
+    for (int yy = threadIdx.y; yy < 32; yy += 8) {
+        const int64_t r = static_cast<int64_t>(bx) * 32 + yy, c = static_cast<int64_t>(by) * 32 + tx;
+        if (r < k && c < k) t[yy][tx] = A[r * k + c];
+    }
+    __syncthreads();
+    for (int yy = threadIdx.y; yy < 32; yy += 8) {
+        const int64_t r = static_cast<int64_t>(by) * 32 + yy, c = static_cast<int64_t>(bx) * 32 + tx;
+        if (r < k && c < k && c > r) A[r * k + c] = t[tx][yy];
     }
 }
 
@@ -519,7 +553,8 @@ int ew_grid(int64_t count, int sms)
     return static_cast<int>(g < sms * 8 ? (g > 0 ? g : 1) : sms * 8);
 }
 
-// A (k x k, SPD) <- -A^-1 in place. Scratch: P, E (k x kSweepBlock), D.
+// A (k x k, SPD; only its lower triangle is read) <- -A^-1 in place, all of
+// it. Scratch: P, E (k x kSweepBlock), D.
 cudaError_t sweep_inverse(float *A, int64_t k, float *P, float *E, float *D, int sms, const LoScratch &lo,
                           int32_t *status, cudaStream_t s)
 {
@@ -531,10 +566,12 @@ cudaError_t sweep_inverse(float *A, int64_t k, float *P, float *E, float *D, int
         // E = P D (D symmetric: P D^T), then A -= E P^T
         if ((e = gemm_nt(k, bs, bs, 1.f, P, bs, D, bs, 0.f, nullptr, 0, E, bs, s, lo, nullptr, status)) != cudaSuccess)
             return e;
-        if ((e = gemm_nt(k, k, bs, -1.f, E, bs, P, bs, 1.f, A, k, A, k, s, lo, nullptr, status)) != cudaSuccess)
+        if ((e = gemm_nt(k, k, bs, -1.f, E, bs, P, bs, 1.f, A, k, A, k, s, lo, nullptr, status, true)) != cudaSuccess)
             return e;
         sweep_fixup_kernel<<<ew_grid(k * bs, sms), 256, 0, s>>>(A, k, p0, bs, E, D);
     }
+    const unsigned nb = static_cast<unsigned>((k + 31) / 32);
+    sweep_mirror_kernel<<<dim3(nb, nb), dim3(32, 8), 0, s>>>(A, k);
     return cudaGetLastError();
 }
 
@@ -672,7 +709,8 @@ cudaError_t factorize_run(const float *W, int64_t n, int64_t m, int64_t k, const
         // U-subproblem: C = W Zv^T, G = Zv Zv^T + rho I, G <- -G^-1
         if ((e = gemm_nt(n, k, m, 1.f, W, m, w.Zv, m, 0.f, nullptr, 0, w.C, k, s, w.lo, nullptr, w.status)) != cudaSuccess)
             return e;
-        if ((e = gemm_nt(k, k, m, 1.f, w.Zv, m, w.Zv, m, 0.f, nullptr, 0, w.G, k, s, w.lo, nullptr, w.status)) != cudaSuccess)
+        if ((e = gemm_nt(k, k, m, 1.f, w.Zv, m, w.Zv, m, 0.f, nullptr, 0, w.G, k, s, w.lo, nullptr, w.status, true)) !=
+            cudaSuccess)
             return e;
         rho_kernel<<<1, 256, 0, s>>>(w.G, k, rho_rel, w.rho);
         if ((e = sweep_inverse(w.G, k, w.P, w.E, w.D, sms, w.lo, w.status, s)) != cudaSuccess) return e;
@@ -692,7 +730,7 @@ cudaError_t factorize_run(const float *W, int64_t n, int64_t m, int64_t k, const
         if ((e = gemm_nt(m, k, n, 1.f, w.WT, n, w.ZuT, n, 0.f, nullptr, 0, w.C, k, s, w.lo, nullptr, w.status)) !=
             cudaSuccess)
             return e;
-        if ((e = gemm_nt(k, k, n, 1.f, w.ZuT, n, w.ZuT, n, 0.f, nullptr, 0, w.G, k, s, w.lo, nullptr, w.status)) !=
+        if ((e = gemm_nt(k, k, n, 1.f, w.ZuT, n, w.ZuT, n, 0.f, nullptr, 0, w.G, k, s, w.lo, nullptr, w.status, true)) !=
             cudaSuccess)
             return e;
         rho_kernel<<<1, 256, 0, s>>>(w.G, k, rho_rel, w.rho);

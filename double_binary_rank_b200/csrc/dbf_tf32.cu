@@ -67,6 +67,7 @@ struct XArgs {
     double *sumsq;     // non-null: add the squares of the results, store nothing
     int vec_c;         // Cin / Cout rows allow float4 access
     int32_t *status;   // optional: DBF_ERR_TIMEOUT on a wait that expired
+    int lower;         // M == N: only the tiles that reach the lower triangle (row >= column somewhere)
 };
 
 template <int S>
@@ -194,10 +195,29 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32])
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
-// Row tile and column tile of tile t: groups of kRasterRows row tiles, row
-// tile fastest inside a group.
-__device__ __forceinline__ void tile_pos(int t, int n_m, int n_n, int &mt, int &nt)
+// Tiles of a lower-triangle product (M == N, BN = r XM): column tile nt
+// holds row tiles r nt .. n_m - 1, the ones whose rows reach its columns
+__host__ __device__ __forceinline__ int lower_tiles(int n_m, int n_n, int r)
 {
+    int t = 0;
+    for (int nt = 0; nt < n_n && r * nt < n_m; ++nt) t += n_m - r * nt;
+    return t;
+}
+
+// Row tile and column tile of tile t: groups of kRasterRows row tiles, row
+// tile fastest inside a group; lower-triangle products column by column
+// (their operands are a few MB: L2 holds them in any order).
+__device__ __forceinline__ void tile_pos(int t, int n_m, int n_n, int &mt, int &nt, int lower = 0, int r = 1)
+{
+    if (lower) {
+        nt = 0;
+        for (int c = n_m; t >= c && nt + 1 < n_n; c = n_m - r * nt) {
+            t -= c;
+            ++nt;
+        }
+        mt = r * nt + t;
+        return;
+    }
     const int per_group = kRasterRows * n_n;
     const int grp = t / per_group;
     const int local = t - grp * per_group;
@@ -288,7 +308,7 @@ __global__ void __launch_bounds__(X_THREADS, 1)
     const int lane = threadIdx.x & 31;
     const int n_m = static_cast<int>((g.M + XM - 1) / XM);
     const int n_n = static_cast<int>((g.N + BN - 1) / BN);
-    const int ntiles = n_m * n_n;
+    const int ntiles = g.lower ? lower_tiles(n_m, n_n, BN / XM) : n_m * n_n;
     const int my_tiles = static_cast<int>(blockIdx.x) < ntiles ? (ntiles - 1 - static_cast<int>(blockIdx.x)) / gridDim.x + 1 : 0;
     const int nk = static_cast<int>((g.K + XK - 1) / XK);
     const int nk3 = 3 * nk;   // stages per tile: K' = 3K
@@ -326,7 +346,8 @@ __global__ void __launch_bounds__(X_THREADS, 1)
             int s = 0;
             for (int j = 0; j < my_tiles && !*abort; ++j) {
                 int mt, nt;
-                tile_pos(static_cast<int>(blockIdx.x) + j * static_cast<int>(gridDim.x), n_m, n_n, mt, nt);
+                tile_pos(static_cast<int>(blockIdx.x) + j * static_cast<int>(gridDim.x), n_m, n_n, mt, nt, g.lower,
+                         BN / XM);
                 for (int kq = 0; kq < nk3; ++kq, ++s) {
                     const int seg = kq / nk, k = kq - seg * nk;   // segment 0: (A, B), 1: (A, lo B), 2: (lo A, B)
                     const int st = s % S;
@@ -386,7 +407,7 @@ __global__ void __launch_bounds__(X_THREADS, 1)
             if (!warp_wait(&sh->acc_full[ab], (j >> 1) & 1, abort)) break;
             tc_fence_after();
             int mt, nt;
-            tile_pos(static_cast<int>(blockIdx.x) + j * static_cast<int>(gridDim.x), n_m, n_n, mt, nt);
+            tile_pos(static_cast<int>(blockIdx.x) + j * static_cast<int>(gridDim.x), n_m, n_n, mt, nt, g.lower, BN / XM);
             const int64_t row = static_cast<int64_t>(mt) * XM + q * 32 + lane;
             const uint32_t taddr = tmem + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(ab * BN);
             float sq = 0.f;
@@ -451,7 +472,7 @@ int64_t ceil4(int64_t v) { return (v + 3) / 4 * 4; }
 template <class Cfg>
 cudaError_t launch_tf32x3(int64_t M, int64_t N, int64_t K, float alpha, const float *A, int64_t lda, const float *B,
                           int64_t ldb, float beta, const float *Cin, int64_t ldci, float *Cout, int64_t ldco,
-                          double *sumsq, int32_t *status, float *lo, cudaStream_t s)
+                          double *sumsq, int32_t *status, float *lo, bool lower, cudaStream_t s)
 {
     int dev = 0, sms = 0;
     cudaGetDevice(&dev);
@@ -483,12 +504,14 @@ cudaError_t launch_tf32x3(int64_t M, int64_t N, int64_t K, float alpha, const fl
     g.sumsq = sumsq;
     g.vec_c = (sumsq || (aligned16(Cout) && ldco % 4 == 0)) && (beta == 0.f || (aligned16(Cin) && ldci % 4 == 0));
     g.status = status;
+    g.lower = lower && M == N && !sumsq;
     {
         cudaError_t e = allow_smem(reinterpret_cast<const void *>(tf32x3_kernel<Cfg>), static_cast<int>(x_smem<Cfg>()));
         if (e != cudaSuccess) return e;
     }
-    const int64_t tiles = ((M + XM - 1) / XM) * ((N + Cfg::BN - 1) / Cfg::BN);
-    if (tiles >= (int64_t(1) << 31)) return cudaErrorInvalidValue;
+    const int64_t n_m = (M + XM - 1) / XM, n_n = (N + Cfg::BN - 1) / Cfg::BN;
+    if (n_m * n_n >= (int64_t(1) << 31)) return cudaErrorInvalidValue;
+    const int64_t tiles = g.lower ? lower_tiles(static_cast<int>(n_m), static_cast<int>(n_n), Cfg::BN / XM) : n_m * n_n;
     tf32x3_kernel<Cfg><<<static_cast<unsigned>(tiles < sms ? tiles : sms), X_THREADS, x_smem<Cfg>(), s>>>(ma, mal, mb,
                                                                                                          mbl, g);
     return cudaGetLastError();
@@ -509,13 +532,14 @@ size_t tf32x3_scratch_floats(int64_t M, int64_t N, int64_t K)
 
 cudaError_t tf32x3_gemm(int64_t M, int64_t N, int64_t K, float alpha, const float *A, int64_t lda, const float *B,
                         int64_t ldb, float beta, const float *Cin, int64_t ldci, float *Cout, int64_t ldco,
-                        double *sumsq, int32_t *status, float *lo_scratch, size_t lo_scratch_floats, cudaStream_t s)
+                        double *sumsq, int32_t *status, float *lo_scratch, size_t lo_scratch_floats, cudaStream_t s,
+                        bool lower)
 {
     if (!tf32x3_ok(M, N, K, A, lda, B, ldb) || !lo_scratch || !aligned16(lo_scratch) ||
         lo_scratch_floats < tf32x3_scratch_floats(M, N, K))
         return cudaErrorInvalidValue;
     return launch_tf32x3<XDefault>(M, N, K, alpha, A, lda, B, ldb, beta, Cin, ldci, Cout, ldco, sumsq, status,
-                                   lo_scratch, s);
+                                   lo_scratch, lower, s);
 }
 
 }  // namespace dbf
