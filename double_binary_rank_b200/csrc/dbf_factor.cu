@@ -250,12 +250,13 @@ struct LoScratch {
 // diagonal; the SIMT GEMM computes all of it).
 cudaError_t gemm_nt(int64_t M, int64_t N, int64_t K, float alpha, const float *A, int64_t lda, const float *B,
                     int64_t ldb, float beta, const float *Cin, int64_t ldci, float *Cout, int64_t ldco, cudaStream_t s,
-                    const LoScratch &lo, double *sumsq = nullptr, int32_t *status = nullptr, bool lower = false)
+                    const LoScratch &lo, double *sumsq = nullptr, int32_t *status = nullptr, bool lower = false,
+                    int max_ctas = 0)
 {
     if (M <= 0 || N <= 0) return cudaSuccess;
     if (K >= 32 && tf32x3_ok(M, N, K, A, lda, B, ldb) && lo.p && lo.floats >= tf32x3_scratch_floats(M, N, K))
         return tf32x3_gemm(M, N, K, alpha, A, lda, B, ldb, beta, Cin, ldci, Cout, ldco, sumsq, status, lo.p, lo.floats,
-                           s, lower);
+                           s, lower, max_ctas);
     return sgemm(false, true, M, N, K, alpha, A, lda, B, ldb, beta, Cin, ldci, Cout, ldco, s, sumsq);
 }
 
@@ -453,6 +454,24 @@ __global__ void sweep_fixup_kernel(float *__restrict__ A, int64_t k, int64_t p0,
     }
 }
 
+// T = A[p1 : p1 + bn, p1 : p1 + bn] - E[p1 : p1 + bn, :] P[p1 : p1 + bn, :]^T
+// (E, P: k x bs, ld bs; T: ld bn): the next pivot block as the current
+// block's trailing update will leave it, formed ahead of that update. A
+// thread per element, fp32 sums in the order of l.
+__global__ void __launch_bounds__(256) sweep_diag_kernel(const float *__restrict__ A, int64_t k, int64_t p1, int bn,
+                                                         const float *__restrict__ E, const float *__restrict__ P,
+                                                         int bs, float *__restrict__ T)
+{
+    const int idx = blockIdx.x * blockDim.x + threadIdx.x;
+    if (idx >= bn * bn) return;
+    const int a = idx / bn, b = idx - a * bn;
+    const float *ea = E + (p1 + a) * bs, *pb = P + (p1 + b) * bs;
+    float acc = 0.f;
+#pragma unroll 8
+    for (int l = 0; l < bs; ++l) acc = fmaf(ea[l], pb[l], acc);
+    T[idx] = A[(p1 + a) * k + p1 + b] - acc;
+}
+
 // The upper triangle of the symmetric k x k matrix A from its lower triangle,
 // through 32 x 32 tiles in shared memory (block (bx, by) writes the upper
 // tile at rows 32 by, columns 32 bx from the lower tile at rows 32 bx,
@@ -553,22 +572,85 @@ int ew_grid(int64_t count, int sms)
     return static_cast<int>(g < sms * 8 ? (g > 0 ? g : 1) : sms * 8);
 }
 
+// A second stream for the sweep's lookahead, with the events that order it
+// against the caller's stream (side == nullptr: no lookahead).
+struct SideStream {
+    cudaStream_t side;
+    cudaEvent_t ev_t, ev_d;   // next pivot block formed (caller's stream); its inverse done (side)
+};
+
+// Owns a SideStream for one call; no lookahead (side == nullptr) when the
+// caller's stream is being captured into a graph, the device has a single
+// SM, or creation fails.
+struct SideStreamOwner {
+    SideStream ss{};
+    SideStreamOwner(cudaStream_t s, int sms)
+    {
+        cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+        if (sms < 2 || cudaStreamIsCapturing(s, &cs) != cudaSuccess || cs != cudaStreamCaptureStatusNone) return;
+        if (cudaStreamCreateWithFlags(&ss.side, cudaStreamNonBlocking) != cudaSuccess) {
+            ss.side = nullptr;
+            return;
+        }
+        if (cudaEventCreateWithFlags(&ss.ev_t, cudaEventDisableTiming) != cudaSuccess ||
+            cudaEventCreateWithFlags(&ss.ev_d, cudaEventDisableTiming) != cudaSuccess)
+            release();
+    }
+    void release()
+    {
+        // resources of a stream or event with work pending are released
+        // once that work is done
+        if (ss.ev_t) cudaEventDestroy(ss.ev_t);
+        if (ss.ev_d) cudaEventDestroy(ss.ev_d);
+        if (ss.side) cudaStreamDestroy(ss.side);
+        ss = SideStream{};
+    }
+    ~SideStreamOwner() { release(); }
+    SideStreamOwner(const SideStreamOwner &) = delete;
+    SideStreamOwner &operator=(const SideStreamOwner &) = delete;
+};
+
 // A (k x k, SPD; only its lower triangle is read) <- -A^-1 in place, all of
-// it. Scratch: P, E (k x kSweepBlock), D.
-cudaError_t sweep_inverse(float *A, int64_t k, float *P, float *E, float *D, int sms, const LoScratch &lo,
-                          int32_t *status, cudaStream_t s)
+// it. Scratch: P, E (k x kSweepBlock), D (two kSweepBlock^2 buffers, used by
+// turns), T (kSweepBlock^2). Lookahead (ss.side set): once E of a pivot
+// block is known, the next pivot block is formed from it (sweep_diag_kernel)
+// and inverted on the side stream, on one SM, while the trailing update runs
+// on the others.
+cudaError_t sweep_inverse(float *A, int64_t k, float *P, float *E, float *D, float *T, int sms, const LoScratch &lo,
+                          int32_t *status, cudaStream_t s, const SideStream &ss)
 {
     cudaError_t e;
-    for (int64_t p0 = 0; p0 < k; p0 += kSweepBlock) {
-        const int bs = static_cast<int>(k - p0 < kSweepBlock ? k - p0 : kSweepBlock);
-        sweep_panel_kernel<<<ew_grid(k * bs, sms), 256, 0, s>>>(A, k, p0, bs, P);
-        sweep_block_inverse_kernel<<<1, kSweepThreads, 0, s>>>(P, p0, bs, D);
+    const bool la = ss.side != nullptr;
+    constexpr int64_t kBB = static_cast<int64_t>(kSweepBlock) * kSweepBlock;
+    auto bsize = [&](int64_t p) { return static_cast<int>(k - p < kSweepBlock ? k - p : kSweepBlock); };
+    sweep_panel_kernel<<<ew_grid(k * bsize(0), sms), 256, 0, s>>>(A, k, 0, bsize(0), P);
+    sweep_block_inverse_kernel<<<1, kSweepThreads, 0, s>>>(P, 0, bsize(0), D);
+    int j = 0;
+    for (int64_t p0 = 0; p0 < k; p0 += kSweepBlock, ++j) {
+        const int bs = bsize(p0);
+        const int64_t p1 = p0 + bs;   // the next pivot block
+        const bool next = p1 < k;
+        float *Dj = D + (j & 1) * kBB, *Dn = D + ((j + 1) & 1) * kBB;
+        if (la && j > 0 && (e = cudaStreamWaitEvent(s, ss.ev_d, 0)) != cudaSuccess) return e;
         // E = P D (D symmetric: P D^T), then A -= E P^T
-        if ((e = gemm_nt(k, bs, bs, 1.f, P, bs, D, bs, 0.f, nullptr, 0, E, bs, s, lo, nullptr, status)) != cudaSuccess)
+        if ((e = gemm_nt(k, bs, bs, 1.f, P, bs, Dj, bs, 0.f, nullptr, 0, E, bs, s, lo, nullptr, status)) != cudaSuccess)
             return e;
-        if ((e = gemm_nt(k, k, bs, -1.f, E, bs, P, bs, 1.f, A, k, A, k, s, lo, nullptr, status, true)) != cudaSuccess)
+        if (la && next) {
+            const int bn = bsize(p1);
+            sweep_diag_kernel<<<(bn * bn + 255) / 256, 256, 0, s>>>(A, k, p1, bn, E, P, bs, T);
+            if ((e = cudaEventRecord(ss.ev_t, s)) != cudaSuccess) return e;
+            if ((e = cudaStreamWaitEvent(ss.side, ss.ev_t, 0)) != cudaSuccess) return e;
+            sweep_block_inverse_kernel<<<1, kSweepThreads, 0, ss.side>>>(T, 0, bn, Dn);
+            if ((e = cudaEventRecord(ss.ev_d, ss.side)) != cudaSuccess) return e;
+        }
+        if ((e = gemm_nt(k, k, bs, -1.f, E, bs, P, bs, 1.f, A, k, A, k, s, lo, nullptr, status, true,
+                         la && next ? sms - 1 : 0)) != cudaSuccess)
             return e;
-        sweep_fixup_kernel<<<ew_grid(k * bs, sms), 256, 0, s>>>(A, k, p0, bs, E, D);
+        sweep_fixup_kernel<<<ew_grid(k * bs, sms), 256, 0, s>>>(A, k, p0, bs, E, Dj);
+        if (next) {
+            sweep_panel_kernel<<<ew_grid(k * bsize(p1), sms), 256, 0, s>>>(A, k, p1, bsize(p1), P);
+            if (!la) sweep_block_inverse_kernel<<<1, kSweepThreads, 0, s>>>(P, p1, bsize(p1), Dn);
+        }
     }
     const unsigned nb = static_cast<unsigned>((k + 31) / 32);
     sweep_mirror_kernel<<<dim3(nb, nb), dim3(32, 8), 0, s>>>(A, k);
@@ -580,7 +662,7 @@ cudaError_t sweep_inverse(float *A, int64_t k, float *P, float *E, float *D, int
 // K-major operands: W^T is formed once, Zu^T after each U-subproblem, Zv
 // from Zv^T after each V-subproblem.
 struct FactorWs {
-    float *Zu, *Zv, *Zvt, *ZuT, *WT, *C, *Lam, *X, *Rhs, *G, *P, *E, *D;
+    float *Zu, *Zv, *Zvt, *ZuT, *WT, *C, *Lam, *X, *Rhs, *G, *P, *E, *D, *T;
     float *a, *m1, *m2, *b, *rho;
     uint32_t *bt_packed;   // sign(V^T) packed, m rows of ceil(k/32) words
     LoScratch lo;          // lo planes of the tensor-core products
@@ -614,7 +696,8 @@ FactorWs carve(void *base, int64_t n, int64_t m, int64_t k, int outer, int svid_
     w.G = reinterpret_cast<float *>(take(static_cast<size_t>(k) * k * 4));
     w.P = reinterpret_cast<float *>(take(static_cast<size_t>(k) * kSweepBlock * 4));
     w.E = reinterpret_cast<float *>(take(static_cast<size_t>(k) * kSweepBlock * 4));
-    w.D = reinterpret_cast<float *>(take(kSweepBlock * kSweepBlock * 4));
+    w.D = reinterpret_cast<float *>(take(2 * kSweepBlock * kSweepBlock * 4));
+    w.T = reinterpret_cast<float *>(take(kSweepBlock * kSweepBlock * 4));
     w.a = reinterpret_cast<float *>(take(static_cast<size_t>(n) * 4));
     w.m1 = reinterpret_cast<float *>(take(static_cast<size_t>(k) * 4));
     w.m2 = reinterpret_cast<float *>(take(static_cast<size_t>(k) * 4));
@@ -667,6 +750,8 @@ cudaError_t factorize_run(const float *W, int64_t n, int64_t m, int64_t k, const
     const int sms = sm_count();
     const int64_t nk = n * k, km = k * m;
     cudaError_t e;
+    SideStreamOwner side(s, sms);   // the sweeps' lookahead stream
+    const SideStream &ss = side.ss;
     // X (rows x cols) -> Z = SVID(X) with scales p (rows), q (cols); Lam = X - Z
     auto project = [&](int64_t rows, int64_t cols, float *p, float *q, float *Z) -> cudaError_t {
         cudaError_t r = svid_power(w.X, rows, cols, svid_iters, nullptr, nullptr, p, q, w.svid, s);
@@ -713,7 +798,7 @@ cudaError_t factorize_run(const float *W, int64_t n, int64_t m, int64_t k, const
             cudaSuccess)
             return e;
         rho_kernel<<<1, 256, 0, s>>>(w.G, k, rho_rel, w.rho);
-        if ((e = sweep_inverse(w.G, k, w.P, w.E, w.D, sms, w.lo, w.status, s)) != cudaSuccess) return e;
+        if ((e = sweep_inverse(w.G, k, w.P, w.E, w.D, w.T, sms, w.lo, w.status, s, ss)) != cudaSuccess) return e;
         if ((e = cudaMemsetAsync(w.Lam, 0, nk * 4, s)) != cudaSuccess) return e;
         for (int j = 0; j < admm_iters; ++j) {
             rhs_kernel<<<ew_grid(nk, sms), 256, 0, s>>>(w.C, w.Zu, w.Lam, w.rho, nk, w.Rhs);
@@ -734,7 +819,7 @@ cudaError_t factorize_run(const float *W, int64_t n, int64_t m, int64_t k, const
             cudaSuccess)
             return e;
         rho_kernel<<<1, 256, 0, s>>>(w.G, k, rho_rel, w.rho);
-        if ((e = sweep_inverse(w.G, k, w.P, w.E, w.D, sms, w.lo, w.status, s)) != cudaSuccess) return e;
+        if ((e = sweep_inverse(w.G, k, w.P, w.E, w.D, w.T, sms, w.lo, w.status, s, ss)) != cudaSuccess) return e;
         if ((e = cudaMemsetAsync(w.Lam, 0, km * 4, s)) != cudaSuccess) return e;
         for (int j = 0; j < admm_iters; ++j) {
             rhs_kernel<<<ew_grid(km, sms), 256, 0, s>>>(w.C, w.Zvt, w.Lam, w.rho, km, w.Rhs);

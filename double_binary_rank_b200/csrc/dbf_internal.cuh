@@ -108,13 +108,14 @@ cudaError_t svid_run(float *X, int64_t n, int64_t m, int iters, int subtract, ui
 // planes of A and B go to lo_scratch (tf32x3_scratch_floats(M, N, K) floats,
 // 16-byte aligned). lower (M == N, no sumsq): only the tiles that reach the
 // lower triangle are computed; Cout entries above the diagonal outside them
-// are left as they were.
+// are left as they were. max_ctas > 0: at most that many CTAs (one per SM),
+// leaving the other SMs to work on another stream.
 bool tf32x3_ok(int64_t M, int64_t N, int64_t K, const float *A, int64_t lda, const float *B, int64_t ldb);
 size_t tf32x3_scratch_floats(int64_t M, int64_t N, int64_t K);
 cudaError_t tf32x3_gemm(int64_t M, int64_t N, int64_t K, float alpha, const float *A, int64_t lda, const float *B,
                         int64_t ldb, float beta, const float *Cin, int64_t ldci, float *Cout, int64_t ldco,
                         double *sumsq, int32_t *status, float *lo_scratch, size_t lo_scratch_floats, cudaStream_t s,
-                        bool lower = false);
+                        bool lower = false, int max_ctas = 0);
 
 // DBF factorisation (alternating ADMM with the SVID projection, fp32)
 size_t factorize_workspace_bytes(int64_t n, int64_t m, int64_t k, int outer, int svid_iters);

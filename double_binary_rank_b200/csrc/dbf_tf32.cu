@@ -472,7 +472,7 @@ int64_t ceil4(int64_t v) { return (v + 3) / 4 * 4; }
 template <class Cfg>
 cudaError_t launch_tf32x3(int64_t M, int64_t N, int64_t K, float alpha, const float *A, int64_t lda, const float *B,
                           int64_t ldb, float beta, const float *Cin, int64_t ldci, float *Cout, int64_t ldco,
-                          double *sumsq, int32_t *status, float *lo, bool lower, cudaStream_t s)
+                          double *sumsq, int32_t *status, float *lo, bool lower, int max_ctas, cudaStream_t s)
 {
     int dev = 0, sms = 0;
     cudaGetDevice(&dev);
@@ -512,6 +512,7 @@ cudaError_t launch_tf32x3(int64_t M, int64_t N, int64_t K, float alpha, const fl
     const int64_t n_m = (M + XM - 1) / XM, n_n = (N + Cfg::BN - 1) / Cfg::BN;
     if (n_m * n_n >= (int64_t(1) << 31)) return cudaErrorInvalidValue;
     const int64_t tiles = g.lower ? lower_tiles(static_cast<int>(n_m), static_cast<int>(n_n), Cfg::BN / XM) : n_m * n_n;
+    if (max_ctas > 0 && max_ctas < sms) sms = max_ctas;   // SMs left to other work on the device
     tf32x3_kernel<Cfg><<<static_cast<unsigned>(tiles < sms ? tiles : sms), X_THREADS, x_smem<Cfg>(), s>>>(ma, mal, mb,
                                                                                                          mbl, g);
     return cudaGetLastError();
@@ -533,13 +534,13 @@ size_t tf32x3_scratch_floats(int64_t M, int64_t N, int64_t K)
 cudaError_t tf32x3_gemm(int64_t M, int64_t N, int64_t K, float alpha, const float *A, int64_t lda, const float *B,
                         int64_t ldb, float beta, const float *Cin, int64_t ldci, float *Cout, int64_t ldco,
                         double *sumsq, int32_t *status, float *lo_scratch, size_t lo_scratch_floats, cudaStream_t s,
-                        bool lower)
+                        bool lower, int max_ctas)
 {
     if (!tf32x3_ok(M, N, K, A, lda, B, ldb) || !lo_scratch || !aligned16(lo_scratch) ||
         lo_scratch_floats < tf32x3_scratch_floats(M, N, K))
         return cudaErrorInvalidValue;
     return launch_tf32x3<XDefault>(M, N, K, alpha, A, lda, B, ldb, beta, Cin, ldci, Cout, ldco, sumsq, status,
-                                   lo_scratch, lower, s);
+                                   lo_scratch, lower, max_ctas, s);
 }
 
 }  // namespace dbf
