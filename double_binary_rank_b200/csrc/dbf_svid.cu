@@ -94,6 +94,10 @@ constexpr int kFuseWarps = kFuseThreads / 32;
 constexpr int64_t kFuseMaxCols = 12288;         // 12 float4 columns per thread
 constexpr int kFuseMaxBand = 16;                // rows per band
 constexpr int kFuseStages = 2;                  // band buffers in the ring
+// Converged power iteration (single-read path): the unit vectors v_in / |v_in|
+// and v_prev / |v_prev| of two successive iterations agree to within this in
+// every element; the remaining iterations then pass v on unchanged.
+constexpr float kSvidTol = 1e-6f;
 constexpr size_t kFuseBufBudget = 200 * 1024;   // bytes of all band buffers
 constexpr unsigned long long kWaitNs = 2000000000ull;   // bounded waits: 2 s
 
@@ -176,7 +180,8 @@ __device__ __forceinline__ void fma_abs(float4 &a, float4 x, float s)
 template <int NCH>
 __global__ void __launch_bounds__(kFuseThreads, 1)
     svid_iter_kernel(const float *__restrict__ X, int64_t n, int m, int band, const float *__restrict__ v_in,
-                     float *__restrict__ v_out, float *__restrict__ v_clear, float *__restrict__ u, float *norm2_u)
+                     float *__restrict__ v_out, float *__restrict__ v_clear, float *__restrict__ u, float *norm2_u,
+                     const float *__restrict__ v_prev)
 {
     extern __shared__ __align__(16) unsigned char smem[];
     const size_t buf_floats = static_cast<size_t>(band) * m;
@@ -232,6 +237,55 @@ __global__ void __launch_bounds__(kFuseThreads, 1)
         vh[c].w *= vs;
     }
     __syncthreads();   // red is reused below
+
+    if (v_prev) {
+        // converged? v_prev is the previous iteration's input: every CTA
+        // reads the same vectors and reduces them in the same order, so all
+        // of them take the same decision
+        float4 vp[NCH];
+        float psq = 0.f;
+#pragma unroll
+        for (int c = 0; c < NCH; ++c) {
+            const int col = 4 * tid + 1024 * c;
+            vp[c] = col < m ? *reinterpret_cast<const float4 *>(v_prev + col) : make_float4(0.f, 0.f, 0.f, 0.f);
+            psq += vp[c].x * vp[c].x + vp[c].y * vp[c].y + vp[c].z * vp[c].z + vp[c].w * vp[c].w;
+        }
+        for (int o = 16; o; o >>= 1) psq += __shfl_xor_sync(0xffffffffu, psq, o);
+        if (lane == 0) red[wid] = psq;
+        __syncthreads();
+        float p2 = 0.f;
+#pragma unroll
+        for (int w = 0; w < kFuseWarps; ++w) p2 += red[w];
+        const float ps = rsqrtf(p2);
+        float d = 0.f;
+#pragma unroll
+        for (int c = 0; c < NCH; ++c) {
+            d = fmaxf(d, fabsf(vh[c].x - vp[c].x * ps));
+            d = fmaxf(d, fabsf(vh[c].y - vp[c].y * ps));
+            d = fmaxf(d, fabsf(vh[c].z - vp[c].z * ps));
+            d = fmaxf(d, fabsf(vh[c].w - vp[c].w * ps));
+        }
+        for (int o = 16; o; o >>= 1) d = fmaxf(d, __shfl_xor_sync(0xffffffffu, d, o));
+        __syncthreads();   // every warp has read its p2 terms
+        if (lane == 0) red[wid] = d;
+        __syncthreads();
+        float dmax = 0.f;
+#pragma unroll
+        for (int w = 0; w < kFuseWarps; ++w) dmax = fmaxf(dmax, red[w]);
+        if (dmax <= kSvidTol) {
+            // pass the iterate on: v_out = v_in, |u|^2 as before (u itself is
+            // unchanged); the band copies issued above land before the exit
+            if (tid == 0)
+                for (int64_t j = 0; j < kFuseStages; ++j)
+                    if (blockIdx.x + j * grid < nb) bar_wait(&bar[j], 0u);
+            for (int64_t j = static_cast<int64_t>(blockIdx.x) * kFuseThreads + tid; j < m; j += grid * kFuseThreads)
+                v_out[j] = v_in[j];
+            if (blockIdx.x == 0 && tid == 0) *norm2_u = *(norm2_u - 2);
+            asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+            return;
+        }
+        __syncthreads();   // red is reused below
+    }
 
     float usq = 0.f;
     bool ok = true;
@@ -363,9 +417,11 @@ int fuse_band(const float *X, int64_t m)
     return static_cast<int>(b < kFuseMaxBand ? b : kFuseMaxBand);
 }
 
+// v_prev: the previous iteration's input (its norm slot is two floats
+// before norm2_u), or null for the first iteration
 template <int NCH>
 cudaError_t launch_iter(const float *X, int64_t n, int m, int band, const float *v_in, float *v_out, float *v_clear,
-                        float *u, float *norm2_u, int sms, cudaStream_t s)
+                        float *u, float *norm2_u, const float *v_prev, int sms, cudaStream_t s)
 {
     const size_t smem = kFuseStages * (static_cast<size_t>(band) * m * sizeof(float) + sizeof(uint64_t)) +
                         sizeof(float) * kFuseWarps * kFuseMaxBand;
@@ -383,15 +439,15 @@ cudaError_t launch_iter(const float *X, int64_t n, int m, int band, const float 
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, svid_iter_kernel<NCH>, X, n, m, band, v_in, v_out, v_clear, u, norm2_u);
+    return cudaLaunchKernelEx(&cfg, svid_iter_kernel<NCH>, X, n, m, band, v_in, v_out, v_clear, u, norm2_u, v_prev);
 }
 
 }  // namespace
 
-// Scratch: u [n], three v buffers [m] each, 2 iters + 2 norm slots.
+// Scratch: u [n], four v buffers [m] each, 2 iters + 2 norm slots.
 size_t svid_scratch_bytes(int64_t n, int64_t m, int iters)
 {
-    return align_up(static_cast<size_t>(n) * 4, 256) + 3 * align_up(static_cast<size_t>(m) * 4, 256) +
+    return align_up(static_cast<size_t>(n) * 4, 256) + 4 * align_up(static_cast<size_t>(m) * 4, 256) +
            align_up(static_cast<size_t>(2 * iters + 2) * 4, 256);
 }
 
@@ -401,8 +457,8 @@ cudaError_t svid_power(const float *X, int64_t n, int64_t m, int iters, uint16_t
     char *p = static_cast<char *>(scratch);
     float *u = reinterpret_cast<float *>(p);
     p += align_up(static_cast<size_t>(n) * 4, 256);
-    float *vb[3];
-    for (int i = 0; i < 3; ++i) {
+    float *vb[4];
+    for (int i = 0; i < 4; ++i) {
         vb[i] = reinterpret_cast<float *>(p);
         p += align_up(static_cast<size_t>(m) * 4, 256);
     }
@@ -414,20 +470,21 @@ cudaError_t svid_power(const float *X, int64_t n, int64_t m, int iters, uint16_t
     svid_fill_kernel<<<fill_grid, 256, 0, s>>>(vb[0], m, 1.0f / sqrtf(static_cast<float>(m)));
     const int band = fuse_band(X, m);
     if (band > 0) {
-        // iteration it reads vb[it % 3], accumulates into vb[(it + 1) % 3]
-        // and clears vb[(it + 2) % 3]
+        // iteration it reads vb[it % 4] (and, for the convergence test, its
+        // own predecessor's input vb[(it + 3) % 4]), accumulates into
+        // vb[(it + 1) % 4] and clears vb[(it + 2) % 4]
         if ((e = cudaMemsetAsync(vb[1], 0, static_cast<size_t>(m) * 4, s)) != cudaSuccess) return e;
         const int mi = static_cast<int>(m);
         for (int it = 0; it < iters; ++it) {
-            const float *vin = vb[it % 3];
-            float *vout = vb[(it + 1) % 3], *vclr = vb[(it + 2) % 3];
+            const float *vin = vb[it % 4], *vprev = it > 0 ? vb[(it + 3) % 4] : nullptr;
+            float *vout = vb[(it + 1) % 4], *vclr = vb[(it + 2) % 4];
             float *nu = norms + 2 * it;
-            if (m <= 4096) e = launch_iter<4>(X, n, mi, band, vin, vout, vclr, u, nu, sms, s);
-            else if (m <= 8192) e = launch_iter<8>(X, n, mi, band, vin, vout, vclr, u, nu, sms, s);
-            else e = launch_iter<12>(X, n, mi, band, vin, vout, vclr, u, nu, sms, s);
+            if (m <= 4096) e = launch_iter<4>(X, n, mi, band, vin, vout, vclr, u, nu, vprev, sms, s);
+            else if (m <= 8192) e = launch_iter<8>(X, n, mi, band, vin, vout, vclr, u, nu, vprev, sms, s);
+            else e = launch_iter<12>(X, n, mi, band, vin, vout, vclr, u, nu, vprev, sms, s);
             if (e != cudaSuccess) return e;
         }
-        float *vlast = vb[iters % 3], *nv = norms + 2 * (iters - 1) + 1;
+        float *vlast = vb[iters % 4], *nv = norms + 2 * (iters - 1) + 1;
         svid_norm_kernel<<<sms, kSvidThreads, 0, s>>>(vlast, m, nv);
         svid_scales_kernel<<<sms, kSvidThreads, 0, s>>>(u, n, norms + 2 * (iters - 1), vlast, m, nv, 1, s_out, s_in,
                                                        s_out32, s_in32);

@@ -164,7 +164,10 @@ dbf_status dbf_ste_backward(const float *db, const void *h, dbf_dtype h_dtype, i
  * section 2: the SVID projection inside the factorisation; Multi-Boolean
  * Architectures page, section 2: a boolean kernel with its scales, and
  * successive extraction of further kernels from the residual). The rank-1
- * factor comes from `iters` power iterations from the all-positive start.
+ * factor comes from at most `iters` power iterations from the all-positive
+ * start: when m is a multiple of 4 and at most 12288 (the single-read path)
+ * they stop early once two successive unit iterates agree to 1e-6 in every
+ * element (the remaining iterations would move the result by less than that).
  * signs: device, packed sign(X) (bit set = -1, sign(0) = +1), n rows with
  *    signs_ld_words words each (>= ceil(m/32); a larger pitch places the
  *    kernel inside a wider packed matrix, e.g. one block of an MBOK layer).
@@ -192,7 +195,7 @@ dbf_status dbf_svid(float *X, int64_t n, int64_t m, int32_t iters, int subtract,
  *     Z <- SVID(U + L),  L <- L + U - Z     (Z from the current U, L = 0),
  * the factor becoming Z, then the same on V with U fixed (operands
  * transposed); rho = rho_rel * trace(Gram) / k; SVID as in dbf_svid with
- * svid_iters power iterations.
+ * at most svid_iters power iterations.
  * W [n x m], U0 [n x k], V0 [k x m]: device fp32, row-major, read only; the
  *    start is the SVID projection of (U0, V0) (e.g. a truncated SVD split
  *    evenly, or any seeded matrices).
