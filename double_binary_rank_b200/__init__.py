@@ -56,6 +56,7 @@ _SIGS = {
     "dbf_transpose_signs": (ctypes.c_int, [_vp, _i64, _i64, _vp, _sz, _vp]),
     "dbf_svid_scratch_bytes": (_sz, [_i64, _i64, _i32]),
     "dbf_svid": (ctypes.c_int, [_vp, _i64, _i64, _i32, ctypes.c_int, _vp, _i64, _vp, _vp, _vp, _sz, _vp]),
+    "dbf_svid_iterations": (ctypes.c_int, [_vp, _i64, _i64, _i32, ctypes.POINTER(ctypes.c_int32)]),
     "dbf_factorize_workspace_bytes": (_sz, [_i64, _i64, _i64, _i32, _i32]),
     "dbf_factorize": (ctypes.c_int, [_vp, _i64, _i64, _i64, _vp, _vp, _i32, _i32, _i32, ctypes.c_float, _vp, _vp,
                                      _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
@@ -386,6 +387,13 @@ def svid(X: torch.Tensor, iters: int = 24, subtract: bool = False, signs: Option
     _check(_lib.dbf_svid(_ptr(X), n, m, iters, int(subtract), _ptr(signs), signs.stride(0), _ptr(s_out), _ptr(s_in),
                          _ptr(scratch), scratch.numel(), _stream(stream)), "dbf_svid")
     return signs, s_out, s_in
+
+
+def svid_iterations(scratch: torch.Tensor, n: int, m: int, iters: int) -> int:
+    """Power iterations the last svid call with this scratch ran (synchronous)."""
+    out = ctypes.c_int32(0)
+    _check(_lib.dbf_svid_iterations(_ptr(scratch), n, m, iters, ctypes.byref(out)), "dbf_svid_iterations")
+    return int(out.value)
 
 
 def factorize_workspace_bytes(n: int, m: int, k: int, outer: int, svid_iters: int = 24) -> int:

@@ -126,6 +126,13 @@ dbf_status dbf_svid(float *X, int64_t n, int64_t m, int32_t iters, int subtract,
                               static_cast<cudaStream_t>(stream)));
 }
 
+dbf_status dbf_svid_iterations(void *scratch, int64_t n, int64_t m, int32_t iters, int32_t *out)
+{
+    if (!scratch || !out || n <= 0 || m <= 0 || iters < 1 || iters > 1000) return DBF_ERR_INVALID_ARG;
+    if (!aligned(scratch, 256)) return DBF_ERR_ALIGNMENT;
+    return from_cuda(cudaMemcpy(out, svid_count_slot(scratch, n, m, iters), 4, cudaMemcpyDeviceToHost));
+}
+
 namespace {
 constexpr int64_t kFactorMaxDim = int64_t(65535) * 32;   // transpose grids of 32-row tiles stay <= 65535
 

@@ -96,6 +96,7 @@ cudaError_t mbok_forward(int M, int N, int K, const uint32_t *w_packed, const ui
 
 // SVID (sign times the best rank-1 fit of the magnitudes), by power iteration
 size_t svid_scratch_bytes(int64_t n, int64_t m, int iters);
+int *svid_count_slot(void *scratch, int64_t n, int64_t m, int iters);   // power iterations the last call ran
 // the power iteration alone: fp16 and/or fp32 scale outputs (null ones skipped)
 cudaError_t svid_power(const float *X, int64_t n, int64_t m, int iters, uint16_t *s_out, uint16_t *s_in,
                        float *s_out32, float *s_in32, void *scratch, cudaStream_t s);

@@ -181,7 +181,7 @@ template <int NCH>
 __global__ void __launch_bounds__(kFuseThreads, 1)
     svid_iter_kernel(const float *__restrict__ X, int64_t n, int m, int band, const float *__restrict__ v_in,
                      float *__restrict__ v_out, float *__restrict__ v_clear, float *__restrict__ u, float *norm2_u,
-                     const float *__restrict__ v_prev)
+                     const float *__restrict__ v_prev, int *count, int *conv, int prefetch_early)
 {
     extern __shared__ __align__(16) unsigned char smem[];
     const size_t buf_floats = static_cast<size_t>(band) * m;
@@ -203,15 +203,32 @@ __global__ void __launch_bounds__(kFuseThreads, 1)
                   &bar[j % kFuseStages]);
     };
 
+    // the first iterations fetch their first bands while the previous kernel
+    // still runs; later ones first look whether an earlier iteration found
+    // the iterate converged (then they read no band at all)
     if (tid == 0) {
         for (int st = 0; st < kFuseStages; ++st) bar_init(&bar[st], 1);
-        for (int st = 0; st < kFuseStages; ++st) issue(st);
+        if (prefetch_early)
+            for (int st = 0; st < kFuseStages; ++st) issue(st);
     }
     asm volatile("griddepcontrol.wait;" ::: "memory");   // v_in complete, v_clear no longer read
     __syncthreads();
 
     for (int64_t j = static_cast<int64_t>(blockIdx.x) * kFuseThreads + tid; j < m; j += grid * kFuseThreads)
         v_clear[j] = 0.f;
+    if (!prefetch_early) {
+        int f = 0;
+        if (tid == 0) f = *reinterpret_cast<volatile int *>(conv);
+        if (__syncthreads_or(f)) {
+            for (int64_t j = static_cast<int64_t>(blockIdx.x) * kFuseThreads + tid; j < m; j += grid * kFuseThreads)
+                v_out[j] = v_in[j];
+            if (blockIdx.x == 0 && tid == 0) *norm2_u = *(norm2_u - 2);
+            asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+            return;
+        }
+        if (tid == 0)
+            for (int st = 0; st < kFuseStages; ++st) issue(st);
+    }
 
     float4 vh[NCH], acc[NCH];
     float sq = 0.f;
@@ -274,7 +291,9 @@ __global__ void __launch_bounds__(kFuseThreads, 1)
         for (int w = 0; w < kFuseWarps; ++w) dmax = fmaxf(dmax, red[w]);
         if (dmax <= kSvidTol) {
             // pass the iterate on: v_out = v_in, |u|^2 as before (u itself is
-            // unchanged); the band copies issued above land before the exit
+            // unchanged), and tell the later iterations; the band copies
+            // issued above land before the exit
+            if (blockIdx.x == 0 && tid == 0) *conv = 1;
             if (tid == 0)
                 for (int64_t j = 0; j < kFuseStages; ++j)
                     if (blockIdx.x + j * grid < nb) bar_wait(&bar[j], 0u);
@@ -286,6 +305,7 @@ __global__ void __launch_bounds__(kFuseThreads, 1)
         }
         __syncthreads();   // red is reused below
     }
+    if (blockIdx.x == 0 && tid == 0) atomicAdd(count, 1);   // iterations that ran
 
     float usq = 0.f;
     bool ok = true;
@@ -418,10 +438,13 @@ int fuse_band(const float *X, int64_t m)
 }
 
 // v_prev: the previous iteration's input (its norm slot is two floats
-// before norm2_u), or null for the first iteration
+// before norm2_u), or null for the first iteration; count: iterations that
+// ran; conv: set once the iterate converged; prefetch_early: fetch the first
+// bands before the previous kernel's results are visible (no look at conv)
 template <int NCH>
 cudaError_t launch_iter(const float *X, int64_t n, int m, int band, const float *v_in, float *v_out, float *v_clear,
-                        float *u, float *norm2_u, const float *v_prev, int sms, cudaStream_t s)
+                        float *u, float *norm2_u, const float *v_prev, int *count, int *conv, int prefetch_early,
+                        int sms, cudaStream_t s)
 {
     const size_t smem = kFuseStages * (static_cast<size_t>(band) * m * sizeof(float) + sizeof(uint64_t)) +
                         sizeof(float) * kFuseWarps * kFuseMaxBand;
@@ -439,17 +462,31 @@ cudaError_t launch_iter(const float *X, int64_t n, int m, int band, const float 
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, svid_iter_kernel<NCH>, X, n, m, band, v_in, v_out, v_clear, u, norm2_u, v_prev);
+    return cudaLaunchKernelEx(&cfg, svid_iter_kernel<NCH>, X, n, m, band, v_in, v_out, v_clear, u, norm2_u, v_prev,
+                              count, conv, prefetch_early);
 }
 
 }  // namespace
 
-// Scratch: u [n], four v buffers [m] each, 2 iters + 2 norm slots.
+// Scratch: u [n], four v buffers [m] each, 2 iters + 2 norm slots, the count
+// of iterations that ran, the converged flag.
 size_t svid_scratch_bytes(int64_t n, int64_t m, int iters)
 {
     return align_up(static_cast<size_t>(n) * 4, 256) + 4 * align_up(static_cast<size_t>(m) * 4, 256) +
-           align_up(static_cast<size_t>(2 * iters + 2) * 4, 256);
+           align_up(static_cast<size_t>(2 * iters + 4) * 4, 256);
 }
+
+// the count slot of a scratch laid out for (n, m, iters)
+int *svid_count_slot(void *scratch, int64_t n, int64_t m, int iters)
+{
+    return reinterpret_cast<int *>(static_cast<char *>(scratch) + align_up(static_cast<size_t>(n) * 4, 256) +
+                                   4 * align_up(static_cast<size_t>(m) * 4, 256)) +
+           2 * iters + 2;
+}
+
+namespace {
+__global__ void svid_set_count_kernel(int *count, int v) { *count = v; }
+}  // namespace
 
 cudaError_t svid_power(const float *X, int64_t n, int64_t m, int iters, uint16_t *s_out, uint16_t *s_in,
                        float *s_out32, float *s_in32, void *scratch, cudaStream_t s)
@@ -465,7 +502,8 @@ cudaError_t svid_power(const float *X, int64_t n, int64_t m, int iters, uint16_t
     float *norms = reinterpret_cast<float *>(p);
     const int sms = sms_count();
     cudaError_t e;
-    if ((e = cudaMemsetAsync(norms, 0, static_cast<size_t>(2 * iters + 2) * 4, s)) != cudaSuccess) return e;
+    int *count = reinterpret_cast<int *>(norms) + 2 * iters + 2, *conv = count + 1;
+    if ((e = cudaMemsetAsync(norms, 0, static_cast<size_t>(2 * iters + 4) * 4, s)) != cudaSuccess) return e;
     const int fill_grid = (m + 255) / 256 < sms * 4 ? static_cast<int>((m + 255) / 256) : sms * 4;
     svid_fill_kernel<<<fill_grid, 256, 0, s>>>(vb[0], m, 1.0f / sqrtf(static_cast<float>(m)));
     const int band = fuse_band(X, m);
@@ -479,9 +517,9 @@ cudaError_t svid_power(const float *X, int64_t n, int64_t m, int iters, uint16_t
             const float *vin = vb[it % 4], *vprev = it > 0 ? vb[(it + 3) % 4] : nullptr;
             float *vout = vb[(it + 1) % 4], *vclr = vb[(it + 2) % 4];
             float *nu = norms + 2 * it;
-            if (m <= 4096) e = launch_iter<4>(X, n, mi, band, vin, vout, vclr, u, nu, vprev, sms, s);
-            else if (m <= 8192) e = launch_iter<8>(X, n, mi, band, vin, vout, vclr, u, nu, vprev, sms, s);
-            else e = launch_iter<12>(X, n, mi, band, vin, vout, vclr, u, nu, vprev, sms, s);
+            if (m <= 4096) e = launch_iter<4>(X, n, mi, band, vin, vout, vclr, u, nu, vprev, count, conv, it < 2, sms, s);
+            else if (m <= 8192) e = launch_iter<8>(X, n, mi, band, vin, vout, vclr, u, nu, vprev, count, conv, it < 2, sms, s);
+            else e = launch_iter<12>(X, n, mi, band, vin, vout, vclr, u, nu, vprev, count, conv, it < 2, sms, s);
             if (e != cudaSuccess) return e;
         }
         float *vlast = vb[iters % 4], *nv = norms + 2 * (iters - 1) + 1;
@@ -507,6 +545,7 @@ cudaError_t svid_power(const float *X, int64_t n, int64_t m, int iters, uint16_t
     }
     svid_scales_kernel<<<sms, kSvidThreads, 0, s>>>(u, n, norms + 2 * (iters - 1), v, m, norms + 2 * (iters - 1) + 1,
                                                    0, s_out, s_in, s_out32, s_in32);
+    svid_set_count_kernel<<<1, 1, 0, s>>>(count, iters);   // the two-pass path runs them all
     return cudaGetLastError();
 }
 

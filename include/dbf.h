@@ -183,6 +183,13 @@ dbf_status dbf_svid(float *X, int64_t n, int64_t m, int32_t iters, int subtract,
                     int64_t signs_ld_words, uint16_t *s_out, uint16_t *s_in, void *scratch,
                     size_t scratch_bytes, void *stream);
 
+/* The number of power iterations (1 .. iters) that the last dbf_svid call
+ * given this scratch, n, m and iters ran (it is kept in the scratch). A
+ * synchronous device-to-host copy that waits for all work on the device: for
+ * tests and measurement, not the hot path. Errors: DBF_ERR_INVALID_ARG,
+ * DBF_ERR_ALIGNMENT (scratch not 256-byte aligned), DBF_ERR_CUDA. */
+dbf_status dbf_svid_iterations(void *scratch, int64_t n, int64_t m, int32_t iters, int32_t *out);
+
 /* Double binary factorisation of a dense fp32 weight W (n x m, row-major):
  * W ~ (a . A . mid^T)(B . b^T) with sign matrices A (n x k), B (k x m) and
  * scale vectors a [n], mid [k], b [m] (DBF page, section 2: the

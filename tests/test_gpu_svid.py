@@ -45,6 +45,40 @@ def test_svid_matches_oracle(dbf, n, m):
     assert torch.equal(Xd.cpu(), torch.from_numpy(X))   # read only
 
 
+def test_svid_stops_once_converged(dbf):
+    # |X| exactly rank one: the second iterate is already the fixed point, so
+    # the single-read path runs two iterations and passes it on; the result
+    # is the oracle's
+    rng = np.random.default_rng(5)
+    n, m, iters = 512, 1024, 30
+    a0 = rng.uniform(0.5, 2.0, n)
+    b0 = rng.uniform(0.5, 2.0, m)
+    X = (np.where(rng.random((n, m)) < 0.5, -1.0, 1.0) * np.outer(a0, b0)).astype(np.float32)
+    S_ref, a_ref, b_ref = oracle.svid(X)
+    scratch = dbf.alloc_workspace(int(dbf._lib.dbf_svid_scratch_bytes(n, m, iters)), torch.device("cuda", 0))
+    signs, a, b = dbf.svid(torch.from_numpy(X).cuda(), iters=iters, scratch=scratch)
+    torch.cuda.synchronize()
+    assert dbf.svid_iterations(scratch, n, m, iters) <= 3
+    assert np.array_equal(unpack_np(signs, n, m), S_ref)
+    assert rel_err(a.float().cpu().numpy(), a_ref) < 2e-3
+    assert rel_err(b.float().cpu().numpy(), b_ref) < 2e-3
+    # a dense Gaussian matrix: stopping early gives the scales of a long run
+    X = rng.standard_normal((300, 200)).astype(np.float32)
+    Xd = torch.from_numpy(X).cuda()
+    s30 = dbf.alloc_workspace(int(dbf._lib.dbf_svid_scratch_bytes(300, 200, 30)), torch.device("cuda", 0))
+    _, a30, b30 = dbf.svid(Xd, iters=30, scratch=s30)
+    _, a200, b200 = dbf.svid(Xd, iters=200)
+    torch.cuda.synchronize()
+    assert 1 <= dbf.svid_iterations(s30, 300, 200, 30) <= 30
+    assert rel_err(a30.float().cpu().numpy(), a200.float().cpu().numpy()) < 1e-3
+    assert rel_err(b30.float().cpu().numpy(), b200.float().cpu().numpy()) < 1e-3
+    # the two-pass path (m % 4 != 0) runs every iteration
+    X = rng.standard_normal((64, 1001)).astype(np.float32)
+    s7 = dbf.alloc_workspace(int(dbf._lib.dbf_svid_scratch_bytes(64, 1001, 7)), torch.device("cuda", 0))
+    dbf.svid(torch.from_numpy(X).cuda(), iters=7, scratch=s7)
+    assert dbf.svid_iterations(s7, 64, 1001, 7) == 7
+
+
 def test_svid_subtract_forms_the_residual(dbf):
     rng = np.random.default_rng(11)
     X = rng.standard_normal((256, 384)).astype(np.float32)
