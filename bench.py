@@ -796,13 +796,18 @@ def main():
     f_ws = dbf.alloc_workspace(dbf.factorize_workspace_bytes(fn, fm, fk, 1, 24), dev)
     dbf.factorize(Wf, U0f, V0f, outer=1, admm_iters=f_admm, objective=False, ws=f_ws, stream=stream)
     torch.cuda.synchronize(dev)
-    q0, q1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with torch.cuda.stream(stream):
-        q0.record(stream)
-        dbf.factorize(Wf, U0f, V0f, outer=1, admm_iters=f_admm, objective=False, ws=f_ws, stream=stream)
-        q1.record(stream)
-    torch.cuda.synchronize(dev)
-    fact_us = max_over_ranks(1e3 * q0.elapsed_time(q1), dev)
+    # three timed calls, each bracketed by its own events; the median (the
+    # first call after the warm-up is at times several ms slower)
+    f_ms = []
+    for _ in range(3):
+        q0, q1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            q0.record(stream)
+            dbf.factorize(Wf, U0f, V0f, outer=1, admm_iters=f_admm, objective=False, ws=f_ws, stream=stream)
+            q1.record(stream)
+        torch.cuda.synchronize(dev)
+        f_ms.append(q0.elapsed_time(q1))
+    fact_us = max_over_ranks(1e3 * sorted(f_ms)[1], dev)
     # fp32 contraction flops of one outer iteration: W V^T, V V^T, the sweep
     # inverse, the U solves; U^T W, U^T U, the sweep inverse, the V solves
     fact_flops = (2 * fn * fm * fk + 2 * fk * fk * fm + 2 * fk ** 3 + f_admm * 2 * fn * fk * fk
@@ -870,7 +875,7 @@ def main():
         "factorize": {"kernel": "DBF factorisation of an 11008 x 4096 fp32 weight at k=5888: one outer iteration "
                                 "(4 ADMM steps per factor; products on tcgen05 as three TF32 MMAs each, fp32 "
                                 "accumulation; blocked sweep inverse; single-read SVID projections)",
-                      "ms_per_outer_iteration": fact_us / 1e3, "achieved": fact_flops / (fact_us * 1e-6) / 1e12,
+                      "ms_per_outer_iteration": fact_us / 1e3, "ms_three_calls": [round(v, 2) for v in f_ms], "achieved": fact_flops / (fact_us * 1e-6) / 1e12,
                       "unit": "TFLOP/s", "bound": "tensor", "peak": fp32x3_peak,
                       "frac": fact_flops / (fact_us * 1e-6) / 1e12 / fp32x3_peak,
                       "peak_source": f"{pk_kind} bf16 dense x nominal TF32/BF16 ratio 1.1/2.25, / 3 TF32 products "

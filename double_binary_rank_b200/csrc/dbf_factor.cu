@@ -457,45 +457,30 @@ __global__ void sweep_fixup_kernel(float *__restrict__ A, int64_t k, int64_t p0,
 // T = A[p1 : p1 + bn, p1 : p1 + bn] - E[p1 : p1 + bn, :] P[p1 : p1 + bn, :]^T
 // (E, P: k x bs, ld bs; T: ld bn): the next pivot block as the current
 // block's trailing update will leave it, formed ahead of that update. A CTA
-// takes 16 rows a: their E rows and the block's P rows (transposed) are
-// staged in shared memory (rows padded by one float: conflict-free), thread
-// (a, b0) sums columns b0, b0 + 16, ... in fp32 in the order of l.
-constexpr int kDiagRows = 16;
+// per 16 x 16 tile of T stages its 16 rows of E and of P in shared memory
+// (rows padded by one float: conflict-free) with all loads in flight; a
+// thread sums one element in fp32 in the order of l.
+constexpr int kDiagTile = 16;
 __global__ void __launch_bounds__(256) sweep_diag_kernel(const float *__restrict__ A, int64_t k, int64_t p1, int bn,
                                                          const float *__restrict__ E, const float *__restrict__ P,
                                                          int bs, float *__restrict__ T)
 {
-    extern __shared__ float sd[];
-    float *pt = sd;                          // [bs][bn + 1]: pt[l][b] = P[p1 + b, l]
-    float *es = sd + bs * (bn + 1);          // [kDiagRows][bs + 1]
-    const int tid = threadIdx.x, a0 = blockIdx.x * kDiagRows;
-    for (int i = tid; i < bn * bs; i += blockDim.x) {
-        const int b = i / bs, l = i - b * bs;
-        pt[l * (bn + 1) + b] = P[(p1 + b) * bs + l];
-    }
-    for (int i = tid; i < kDiagRows * bs; i += blockDim.x) {
-        const int r = i / bs, l = i - r * bs;
-        es[r * (bs + 1) + l] = a0 + r < bn ? E[(p1 + a0 + r) * bs + l] : 0.f;
+    __shared__ float es[kDiagTile][kSweepBlock + 1], ps[kDiagTile][kSweepBlock + 1];
+    const int tid = threadIdx.x;
+    const int a0 = blockIdx.y * kDiagTile, b0 = blockIdx.x * kDiagTile;
+#pragma unroll 8
+    for (int i = tid; i < kDiagTile * kSweepBlock; i += 256) {
+        const int r = i / kSweepBlock, l = i - r * kSweepBlock;
+        const bool lok = l < bs;
+        es[r][l] = lok && a0 + r < bn ? E[(p1 + a0 + r) * bs + l] : 0.f;
+        ps[r][l] = lok && b0 + r < bn ? P[(p1 + b0 + r) * bs + l] : 0.f;
     }
     __syncthreads();
-    const int r = tid >> 4, b0 = tid & 15;
-    constexpr int kCols = kSweepBlock / 16;
-    float acc[kCols];
-#pragma unroll
-    for (int j = 0; j < kCols; ++j) acc[j] = 0.f;
-    for (int l = 0; l < bs; ++l) {
-        const float e = es[r * (bs + 1) + l];
-#pragma unroll
-        for (int j = 0; j < kCols; ++j)
-            if (b0 + 16 * j < bn) acc[j] = fmaf(e, pt[l * (bn + 1) + b0 + 16 * j], acc[j]);
-    }
-    const int a = a0 + r;
-    if (a < bn)
-#pragma unroll
-        for (int j = 0; j < kCols; ++j) {
-            const int b = b0 + 16 * j;
-            if (b < bn) T[a * bn + b] = A[(p1 + a) * k + p1 + b] - acc[j];
-        }
+    const int ra = tid >> 4, rb = tid & 15;
+    float acc = 0.f;
+    for (int l = 0; l < bs; ++l) acc = fmaf(es[ra][l], ps[rb][l], acc);
+    const int a = a0 + ra, b = b0 + rb;
+    if (a < bn && b < bn) T[a * bn + b] = A[(p1 + a) * k + p1 + b] - acc;
 }
 
 // The upper triangle of the symmetric k x k matrix A from its lower triangle,
@@ -662,12 +647,8 @@ cudaError_t sweep_inverse(float *A, int64_t k, float *P, float *E, float *D, flo
         if ((e = gemm_nt(k, bs, bs, 1.f, P, bs, Dj, bs, 0.f, nullptr, 0, E, bs, s, lo, nullptr, status)) != cudaSuccess)
             return e;
         if (la && next) {
-            const int bn = bsize(p1);
-            const int dsm = static_cast<int>(sizeof(float)) * (bs * (bn + 1) + kDiagRows * (bs + 1));
-            if ((e = cudaFuncSetAttribute(sweep_diag_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, dsm)) !=
-                cudaSuccess)
-                return e;
-            sweep_diag_kernel<<<(bn + kDiagRows - 1) / kDiagRows, 256, dsm, s>>>(A, k, p1, bn, E, P, bs, T);
+            const int bn = bsize(p1), nt = (bn + kDiagTile - 1) / kDiagTile;
+            sweep_diag_kernel<<<dim3(nt, nt), 256, 0, s>>>(A, k, p1, bn, E, P, bs, T);
             if ((e = cudaEventRecord(ss.ev_t, s)) != cudaSuccess) return e;
             if ((e = cudaStreamWaitEvent(ss.side, ss.ev_t, 0)) != cudaSuccess) return e;
             sweep_block_inverse_kernel<<<1, kSweepThreads, 0, ss.side>>>(T, 0, bn, Dn);
