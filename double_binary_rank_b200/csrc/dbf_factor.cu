@@ -251,12 +251,14 @@ struct LoScratch {
 cudaError_t gemm_nt(int64_t M, int64_t N, int64_t K, float alpha, const float *A, int64_t lda, const float *B,
                     int64_t ldb, float beta, const float *Cin, int64_t ldci, float *Cout, int64_t ldco, cudaStream_t s,
                     const LoScratch &lo, double *sumsq = nullptr, int32_t *status = nullptr, bool lower = false,
-                    int max_ctas = 0)
+                    int max_ctas = 0, const float *A_lo = nullptr, const float *B_lo = nullptr,
+                    float *C_lo = nullptr)
 {
     if (M <= 0 || N <= 0) return cudaSuccess;
     if (K >= 32 && tf32x3_ok(M, N, K, A, lda, B, ldb) && lo.p && lo.floats >= tf32x3_scratch_floats(M, N, K))
         return tf32x3_gemm(M, N, K, alpha, A, lda, B, ldb, beta, Cin, ldci, Cout, ldco, sumsq, status, lo.p, lo.floats,
-                           s, lower, max_ctas);
+                           s, lower, max_ctas, A_lo, B_lo, C_lo);
+    if (A_lo || B_lo || C_lo) return cudaErrorInvalidValue;   // lo planes belong to the tensor-core path
     return sgemm(false, true, M, N, K, alpha, A, lda, B, ldb, beta, Cin, ldci, Cout, ldco, s, sumsq);
 }
 
@@ -265,25 +267,41 @@ constexpr int kSweepBlock = 128;
 constexpr int kSweepSeg = 16;                                         // columns per thread
 constexpr int kSweepThreads = kSweepBlock * kSweepBlock / kSweepSeg;   // 1024: 8 threads per row
 
+// whether gemm_nt takes the tensor-core path for these operands
+bool gemm_nt_tc(int64_t M, int64_t N, int64_t K, const float *A, int64_t lda, const float *B, int64_t ldb,
+                const LoScratch &lo)
+{
+    return M > 0 && N > 0 && K >= 32 && tf32x3_ok(M, N, K, A, lda, B, ldb) && lo.p &&
+           lo.floats >= tf32x3_scratch_floats(M, N, K);
+}
+
 // The sweep keeps the matrix symmetric and maintains its lower triangle
 // (and the diagonal blocks whole); the upper triangle is filled in at the end.
 // P = A[:, p0 : p0 + bs] (k x bs, ld bs): rows i >= p0 from the block column
 // (l fastest), rows i < p0 from the block row, A[p0 + l, i] (i fastest).
-__global__ void sweep_panel_kernel(const float *__restrict__ A, int64_t k, int64_t p0, int bs, float *__restrict__ P)
+// Plo (optional, ld bs): its lo plane for the tensor-core products.
+__global__ void sweep_panel_kernel(const float *__restrict__ A, int64_t k, int64_t p0, int bs, float *__restrict__ P,
+                                   float *__restrict__ Plo)
 {
     const int64_t below = (k - p0) * bs;
     for (int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; idx < k * bs;
          idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        int64_t o;
+        float v;
         if (idx < below) {
             const int64_t d = idx / bs;
             const int l = static_cast<int>(idx - d * bs);
-            P[(p0 + d) * bs + l] = A[(p0 + d) * k + p0 + l];
+            o = (p0 + d) * bs + l;
+            v = A[(p0 + d) * k + p0 + l];
         } else {
             const int64_t j = idx - below;
             const int l = static_cast<int>(j / p0);
             const int64_t i = j - l * p0;
-            P[i * bs + l] = A[(p0 + l) * k + i];
+            o = i * bs + l;
+            v = A[(p0 + l) * k + i];
         }
+        P[o] = v;
+        if (Plo) Plo[o] = tf32_lo(v);
     }
 }
 
@@ -299,7 +317,8 @@ __global__ void sweep_panel_kernel(const float *__restrict__ A, int64_t k, int64
 // publishes D8; every thread then forms its row's coefficients T_iQ D8 and
 // updates its 16 elements (rows Q, held by two whole warps, take D8 T_Qj).
 __global__ void __launch_bounds__(kSweepThreads) sweep_block_inverse_kernel(const float *__restrict__ P, int64_t p0,
-                                                                            int bs, float *__restrict__ D)
+                                                                            int bs, float *__restrict__ D,
+                                                                            float *__restrict__ Dlo)
 {
     constexpr int Q = 8;
     constexpr int kSegs = kSweepBlock / kSweepSeg, kSegPad = kSweepSeg + 4;
@@ -428,7 +447,10 @@ __global__ void __launch_bounds__(kSweepThreads) sweep_block_inverse_kernel(cons
     }
 #pragma unroll
     for (int e = 0; e < kSweepSeg; ++e)
-        if (i < bs && j0 + e < bs) D[i * bs + j0 + e] = -t[e];
+        if (i < bs && j0 + e < bs) {
+            D[i * bs + j0 + e] = -t[e];
+            if (Dlo) Dlo[i * bs + j0 + e] = tf32_lo(-t[e]);
+        }
 }
 
 // After A -= E P^T: the pivot block becomes -D, the block column below it E
@@ -623,44 +645,60 @@ struct SideStreamOwner {
 
 // A (k x k, SPD; only its lower triangle is read) <- -A^-1 in place, all of
 // it. Scratch: P, E (k x kSweepBlock), D (two kSweepBlock^2 buffers, used by
-// turns), T (kSweepBlock^2). Lookahead (ss.side set): once E of a pivot
-// block is known, the next pivot block is formed from it (sweep_diag_kernel)
-// and inverted on the side stream, on one SM, while the trailing update runs
-// on the others.
-cudaError_t sweep_inverse(float *A, int64_t k, float *P, float *E, float *D, float *T, int sms, const LoScratch &lo,
-                          int32_t *status, cudaStream_t s, const SideStream &ss)
+// turns), T (kSweepBlock^2), and the lo planes of P, E and D (the same
+// shapes: Plo, Elo, Dlo) that the panel, the E product's epilogue and the
+// block inverse write for the tensor-core products, which then split
+// nothing. Lookahead (ss.side set): once E of a pivot block is known, the
+// next pivot block is formed from it (sweep_diag_kernel) and inverted on the
+// side stream, on one SM, while the trailing update runs on the others.
+cudaError_t sweep_inverse(float *A, int64_t k, float *P, float *E, float *D, float *T, float *Plo, float *Elo,
+                          float *Dlo, int sms, const LoScratch &lo, int32_t *status, cudaStream_t s,
+                          const SideStream &ss)
 {
     cudaError_t e;
     const bool la = ss.side != nullptr;
     constexpr int64_t kBB = static_cast<int64_t>(kSweepBlock) * kSweepBlock;
     auto bsize = [&](int64_t p) { return static_cast<int>(k - p < kSweepBlock ? k - p : kSweepBlock); };
-    sweep_panel_kernel<<<ew_grid(k * bsize(0), sms), 256, 0, s>>>(A, k, 0, bsize(0), P);
-    sweep_block_inverse_kernel<<<1, kSweepThreads, 0, s>>>(P, 0, bsize(0), D);
+    // the lo planes are used when both products of a block take the
+    // tensor-core path (their K and pitches are bs)
+    auto lo_ok = [&](int bs) {
+        return gemm_nt_tc(k, bs, bs, P, bs, D, bs, lo) && gemm_nt_tc(k, k, bs, E, bs, P, bs, lo);
+    };
+    {
+        const int b0 = bsize(0);
+        const bool l0 = lo_ok(b0);
+        sweep_panel_kernel<<<ew_grid(k * b0, sms), 256, 0, s>>>(A, k, 0, b0, P, l0 ? Plo : nullptr);
+        sweep_block_inverse_kernel<<<1, kSweepThreads, 0, s>>>(P, 0, b0, D, l0 ? Dlo : nullptr);
+    }
     int j = 0;
     for (int64_t p0 = 0; p0 < k; p0 += kSweepBlock, ++j) {
         const int bs = bsize(p0);
         const int64_t p1 = p0 + bs;   // the next pivot block
         const bool next = p1 < k;
+        const bool lj = lo_ok(bs), ln = next && lo_ok(bsize(p1));
         float *Dj = D + (j & 1) * kBB, *Dn = D + ((j + 1) & 1) * kBB;
+        float *Dloj = Dlo + (j & 1) * kBB, *Dlon = Dlo + ((j + 1) & 1) * kBB;
         if (la && j > 0 && (e = cudaStreamWaitEvent(s, ss.ev_d, 0)) != cudaSuccess) return e;
         // E = P D (D symmetric: P D^T), then A -= E P^T
-        if ((e = gemm_nt(k, bs, bs, 1.f, P, bs, Dj, bs, 0.f, nullptr, 0, E, bs, s, lo, nullptr, status)) != cudaSuccess)
+        if ((e = gemm_nt(k, bs, bs, 1.f, P, bs, Dj, bs, 0.f, nullptr, 0, E, bs, s, lo, nullptr, status, false, 0,
+                         lj ? Plo : nullptr, lj ? Dloj : nullptr, lj ? Elo : nullptr)) != cudaSuccess)
             return e;
         if (la && next) {
             const int bn = bsize(p1), nt = (bn + kDiagTile - 1) / kDiagTile;
             sweep_diag_kernel<<<dim3(nt, nt), 256, 0, s>>>(A, k, p1, bn, E, P, bs, T);
             if ((e = cudaEventRecord(ss.ev_t, s)) != cudaSuccess) return e;
             if ((e = cudaStreamWaitEvent(ss.side, ss.ev_t, 0)) != cudaSuccess) return e;
-            sweep_block_inverse_kernel<<<1, kSweepThreads, 0, ss.side>>>(T, 0, bn, Dn);
+            sweep_block_inverse_kernel<<<1, kSweepThreads, 0, ss.side>>>(T, 0, bn, Dn, ln ? Dlon : nullptr);
             if ((e = cudaEventRecord(ss.ev_d, ss.side)) != cudaSuccess) return e;
         }
         if ((e = gemm_nt(k, k, bs, -1.f, E, bs, P, bs, 1.f, A, k, A, k, s, lo, nullptr, status, true,
-                         la && next ? sms - 1 : 0)) != cudaSuccess)
+                         la && next ? sms - 1 : 0, lj ? Elo : nullptr, lj ? Plo : nullptr)) != cudaSuccess)
             return e;
         sweep_fixup_kernel<<<ew_grid(k * bs, sms), 256, 0, s>>>(A, k, p0, bs, E, Dj);
         if (next) {
-            sweep_panel_kernel<<<ew_grid(k * bsize(p1), sms), 256, 0, s>>>(A, k, p1, bsize(p1), P);
-            if (!la) sweep_block_inverse_kernel<<<1, kSweepThreads, 0, s>>>(P, p1, bsize(p1), Dn);
+            const int bn = bsize(p1);
+            sweep_panel_kernel<<<ew_grid(k * bn, sms), 256, 0, s>>>(A, k, p1, bn, P, ln ? Plo : nullptr);
+            if (!la) sweep_block_inverse_kernel<<<1, kSweepThreads, 0, s>>>(P, p1, bn, Dn, ln ? Dlon : nullptr);
         }
     }
     const unsigned nb = static_cast<unsigned>((k + 31) / 32);
@@ -673,7 +711,7 @@ cudaError_t sweep_inverse(float *A, int64_t k, float *P, float *E, float *D, flo
 // K-major operands: W^T is formed once, Zu^T after each U-subproblem, Zv
 // from Zv^T after each V-subproblem.
 struct FactorWs {
-    float *Zu, *Zv, *Zvt, *ZuT, *WT, *C, *Lam, *X, *Rhs, *G, *P, *E, *D, *T;
+    float *Zu, *Zv, *Zvt, *ZuT, *WT, *C, *Lam, *X, *Rhs, *G, *P, *E, *D, *T, *Plo, *Elo, *Dlo;
     float *a, *m1, *m2, *b, *rho;
     uint32_t *bt_packed;   // sign(V^T) packed, m rows of ceil(k/32) words
     LoScratch lo;          // lo planes of the tensor-core products
@@ -709,6 +747,9 @@ FactorWs carve(void *base, int64_t n, int64_t m, int64_t k, int outer, int svid_
     w.E = reinterpret_cast<float *>(take(static_cast<size_t>(k) * kSweepBlock * 4));
     w.D = reinterpret_cast<float *>(take(2 * kSweepBlock * kSweepBlock * 4));
     w.T = reinterpret_cast<float *>(take(kSweepBlock * kSweepBlock * 4));
+    w.Plo = reinterpret_cast<float *>(take(static_cast<size_t>(k) * kSweepBlock * 4));
+    w.Elo = reinterpret_cast<float *>(take(static_cast<size_t>(k) * kSweepBlock * 4));
+    w.Dlo = reinterpret_cast<float *>(take(2 * kSweepBlock * kSweepBlock * 4));
     w.a = reinterpret_cast<float *>(take(static_cast<size_t>(n) * 4));
     w.m1 = reinterpret_cast<float *>(take(static_cast<size_t>(k) * 4));
     w.m2 = reinterpret_cast<float *>(take(static_cast<size_t>(k) * 4));
@@ -809,7 +850,9 @@ cudaError_t factorize_run(const float *W, int64_t n, int64_t m, int64_t k, const
             cudaSuccess)
             return e;
         rho_kernel<<<1, 256, 0, s>>>(w.G, k, rho_rel, w.rho);
-        if ((e = sweep_inverse(w.G, k, w.P, w.E, w.D, w.T, sms, w.lo, w.status, s, ss)) != cudaSuccess) return e;
+        if ((e = sweep_inverse(w.G, k, w.P, w.E, w.D, w.T, w.Plo, w.Elo, w.Dlo, sms, w.lo, w.status, s, ss)) !=
+            cudaSuccess)
+            return e;
         if ((e = cudaMemsetAsync(w.Lam, 0, nk * 4, s)) != cudaSuccess) return e;
         for (int j = 0; j < admm_iters; ++j) {
             rhs_kernel<<<ew_grid(nk, sms), 256, 0, s>>>(w.C, w.Zu, w.Lam, w.rho, nk, w.Rhs);
@@ -830,7 +873,9 @@ cudaError_t factorize_run(const float *W, int64_t n, int64_t m, int64_t k, const
             cudaSuccess)
             return e;
         rho_kernel<<<1, 256, 0, s>>>(w.G, k, rho_rel, w.rho);
-        if ((e = sweep_inverse(w.G, k, w.P, w.E, w.D, w.T, sms, w.lo, w.status, s, ss)) != cudaSuccess) return e;
+        if ((e = sweep_inverse(w.G, k, w.P, w.E, w.D, w.T, w.Plo, w.Elo, w.Dlo, sms, w.lo, w.status, s, ss)) !=
+            cudaSuccess)
+            return e;
         if ((e = cudaMemsetAsync(w.Lam, 0, km * 4, s)) != cudaSuccess) return e;
         for (int j = 0; j < admm_iters; ++j) {
             rhs_kernel<<<ew_grid(km, sms), 256, 0, s>>>(w.C, w.Zvt, w.Lam, w.rho, km, w.Rhs);

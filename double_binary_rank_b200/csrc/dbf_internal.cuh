@@ -110,13 +110,18 @@ cudaError_t svid_run(float *X, int64_t n, int64_t m, int iters, int subtract, ui
 // 16-byte aligned). lower (M == N, no sumsq): only the tiles that reach the
 // lower triangle are computed; Cout entries above the diagonal outside them
 // are left as they were. max_ctas > 0: at most that many CTAs (one per SM),
-// leaving the other SMs to work on another stream.
+// leaving the other SMs to work on another stream. A_lo / B_lo: the lo
+// planes of A / B already formed (pitch ceil4(K); then not split again);
+// Cout_lo: also write the lo plane of the result (pitch ceil4(N)).
+// lo(x) = x - (x with its low 13 mantissa bits cleared), exact.
+__device__ __forceinline__ float tf32_lo(float x) { return x - __uint_as_float(__float_as_uint(x) & 0xFFFFE000u); }
 bool tf32x3_ok(int64_t M, int64_t N, int64_t K, const float *A, int64_t lda, const float *B, int64_t ldb);
 size_t tf32x3_scratch_floats(int64_t M, int64_t N, int64_t K);
 cudaError_t tf32x3_gemm(int64_t M, int64_t N, int64_t K, float alpha, const float *A, int64_t lda, const float *B,
                         int64_t ldb, float beta, const float *Cin, int64_t ldci, float *Cout, int64_t ldco,
                         double *sumsq, int32_t *status, float *lo_scratch, size_t lo_scratch_floats, cudaStream_t s,
-                        bool lower = false, int max_ctas = 0);
+                        bool lower = false, int max_ctas = 0, const float *A_lo = nullptr,
+                        const float *B_lo = nullptr, float *Cout_lo = nullptr);
 
 // DBF factorisation (alternating ADMM with the SVID projection, fp32)
 size_t factorize_workspace_bytes(int64_t n, int64_t m, int64_t k, int outer, int svid_iters);

@@ -68,6 +68,8 @@ struct XArgs {
     int vec_c;         // Cin / Cout rows allow float4 access
     int32_t *status;   // optional: DBF_ERR_TIMEOUT on a wait that expired
     int lower;         // M == N: only the tiles that reach the lower triangle (row >= column somewhere)
+    float *Cout_lo;    // optional: the lo plane of the result, pitch ldlo
+    int64_t ldlo;
 };
 
 template <int S>
@@ -269,6 +271,19 @@ __device__ __forceinline__ void epi_chunk(const XArgs &g, int64_t row, int64_t c
         for (int e = 0; e < 32; ++e)
             if (e < n_ok) cout[e] = out[e];
     }
+    if (g.Cout_lo) {
+        float *clo = g.Cout_lo + row * g.ldlo + c0;
+        if (full) {
+#pragma unroll
+            for (int e = 0; e < 32; e += 4)
+                *reinterpret_cast<float4 *>(clo + e) =
+                    make_float4(tf32_lo(out[e]), tf32_lo(out[e + 1]), tf32_lo(out[e + 2]), tf32_lo(out[e + 3]));
+        } else {
+#pragma unroll
+            for (int e = 0; e < 32; ++e)
+                if (e < n_ok) clo[e] = tf32_lo(out[e]);
+        }
+    }
 }
 
 // lo = x - (x with its low 13 mantissa bits cleared), rows x cols of a
@@ -284,10 +299,10 @@ __global__ void split_lo_kernel(const float *__restrict__ x, int64_t rows, int64
         const int64_t r = i / cols4, c = (i - r * cols4) * 4;
         const float4 v = *reinterpret_cast<const float4 *>(x + r * ld + c);
         float4 l;
-        l.x = v.x - __uint_as_float(__float_as_uint(v.x) & 0xFFFFE000u);
-        l.y = v.y - __uint_as_float(__float_as_uint(v.y) & 0xFFFFE000u);
-        l.z = v.z - __uint_as_float(__float_as_uint(v.z) & 0xFFFFE000u);
-        l.w = v.w - __uint_as_float(__float_as_uint(v.w) & 0xFFFFE000u);
+        l.x = tf32_lo(v.x);
+        l.y = tf32_lo(v.y);
+        l.z = tf32_lo(v.z);
+        l.w = tf32_lo(v.w);
         *reinterpret_cast<float4 *>(lo + r * ldl + c) = l;
     }
 }
@@ -472,21 +487,25 @@ int64_t ceil4(int64_t v) { return (v + 3) / 4 * 4; }
 template <class Cfg>
 cudaError_t launch_tf32x3(int64_t M, int64_t N, int64_t K, float alpha, const float *A, int64_t lda, const float *B,
                           int64_t ldb, float beta, const float *Cin, int64_t ldci, float *Cout, int64_t ldco,
-                          double *sumsq, int32_t *status, float *lo, bool lower, int max_ctas, cudaStream_t s)
+                          double *sumsq, int32_t *status, float *lo, bool lower, int max_ctas, const float *A_lo,
+                          const float *B_lo, float *Cout_lo, cudaStream_t s)
 {
     int dev = 0, sms = 0;
     cudaGetDevice(&dev);
     if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0) sms = 148;
     // lo planes of A and B (B's is A's when B is A)
     const int64_t ldl = ceil4(K);
-    float *Alo = lo, *Blo = (B == A && ldb == lda && N == M) ? lo : lo + M * ldl;
+    float *Alo = lo, *Blo = lo + M * ldl;
     auto split = [&](const float *x, int64_t rows, int64_t ld, float *out) {
         const int64_t total = rows * (ldl / 4);
         const int64_t grid = (total + 255) / 256 < sms * 8 ? (total + 255) / 256 : sms * 8;
         split_lo_kernel<<<static_cast<unsigned>(grid > 0 ? grid : 1), 256, 0, s>>>(x, rows, ldl / 4, ld, out, ldl);
     };
-    split(A, M, lda, Alo);
-    if (Blo != Alo) split(B, N, ldb, Blo);
+    if (A_lo) Alo = const_cast<float *>(A_lo);
+    else split(A, M, lda, Alo);
+    if (B_lo) Blo = const_cast<float *>(B_lo);
+    else if (B == A && ldb == lda && N == M) Blo = Alo;   // the same operand: the same plane
+    else split(B, N, ldb, Blo);
     CUtensorMap ma, mal, mb, mbl;
     if (!make_map_f32(&ma, A, K, M, lda, XM) || !make_map_f32(&mal, Alo, K, M, ldl, XM) ||
         !make_map_f32(&mb, B, K, N, ldb, Cfg::BN) || !make_map_f32(&mbl, Blo, K, N, ldl, Cfg::BN))
@@ -505,6 +524,9 @@ cudaError_t launch_tf32x3(int64_t M, int64_t N, int64_t K, float alpha, const fl
     g.vec_c = (sumsq || (aligned16(Cout) && ldco % 4 == 0)) && (beta == 0.f || (aligned16(Cin) && ldci % 4 == 0));
     g.status = status;
     g.lower = lower && M == N && !sumsq;
+    g.Cout_lo = sumsq ? nullptr : Cout_lo;
+    g.ldlo = ceil4(N);
+    if (g.Cout_lo && !aligned16(g.Cout_lo)) g.vec_c = 0;
     {
         cudaError_t e = allow_smem(reinterpret_cast<const void *>(tf32x3_kernel<Cfg>), static_cast<int>(x_smem<Cfg>()));
         if (e != cudaSuccess) return e;
@@ -534,13 +556,13 @@ size_t tf32x3_scratch_floats(int64_t M, int64_t N, int64_t K)
 cudaError_t tf32x3_gemm(int64_t M, int64_t N, int64_t K, float alpha, const float *A, int64_t lda, const float *B,
                         int64_t ldb, float beta, const float *Cin, int64_t ldci, float *Cout, int64_t ldco,
                         double *sumsq, int32_t *status, float *lo_scratch, size_t lo_scratch_floats, cudaStream_t s,
-                        bool lower, int max_ctas)
+                        bool lower, int max_ctas, const float *A_lo, const float *B_lo, float *Cout_lo)
 {
     if (!tf32x3_ok(M, N, K, A, lda, B, ldb) || !lo_scratch || !aligned16(lo_scratch) ||
         lo_scratch_floats < tf32x3_scratch_floats(M, N, K))
         return cudaErrorInvalidValue;
     return launch_tf32x3<XDefault>(M, N, K, alpha, A, lda, B, ldb, beta, Cin, ldci, Cout, ldco, sumsq, status,
-                                   lo_scratch, lower, max_ctas, s);
+                                   lo_scratch, lower, max_ctas, A_lo, B_lo, Cout_lo, s);
 }
 
 }  // namespace dbf
