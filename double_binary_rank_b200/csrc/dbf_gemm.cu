@@ -90,6 +90,7 @@ struct GemmCfg {
     static constexpr int kThreads = 32 * (2 + kExpandWarps + kEpiWarps);
 };
 using FwdCfg = GemmCfg<2, 6, 4, 4, false>;
+using GrpCfg = GemmCfg<2, 6, 4, 8, false>;   // grouped (segmented) launches: short K loops, epilogue-heavy
 using FwdPairCfg = GemmCfg<2, 6, 6, 4, false, true>;
 using FusedCfg = GemmCfg<2, 6, 4, 8, false, true, true, true>;
 using BwdPairCfg = GemmCfg<1, 6, 6, 8, true, true>;
@@ -2197,9 +2198,9 @@ cudaError_t gemm_forward_grouped(const dbf_layer *const *layers, const int *off,
     a1.ngroups = a2.ngroups = count;
     a1.tiles_total = t1;
     a2.tiles_total = t2;
-    cudaError_t e = launch_gemm<FwdCfg>(mu, a1, s, nullptr, st);
+    cudaError_t e = launch_gemm<GrpCfg>(mu, a1, s, nullptr, st);
     if (e != cudaSuccess) return e;
-    return launch_gemm<FwdCfg>(mv, a2, s, nullptr, st);
+    return launch_gemm<GrpCfg>(mv, a2, s, nullptr, st);
 }
 
 }  // namespace dbf
