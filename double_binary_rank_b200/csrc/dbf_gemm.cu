@@ -63,8 +63,8 @@ constexpr int BK = 64;              // K per stage: one 128-byte swizzle row of 
 // one-launch forward, whose 512-column tiles leave no accumulator free for
 // the next tile during an epilogue, and the backward, whose epilogues read
 // and write an operand per element, take eight epilogue warps (two per TMEM
-// lane quarter, each with half of the columns); the backward keeps one
-// expansion group.
+// lane quarter, each with half of the columns) and one expansion group (a
+// 512-column tile needs half the expanded signs per flop).
 template <int kGroups, int kSA, int kSB, int kEpi, bool kBackward, bool kPairMode = false, bool kFusedMode = false,
           bool kWideMode = false>
 struct GemmCfg {
@@ -92,7 +92,7 @@ struct GemmCfg {
 using FwdCfg = GemmCfg<2, 6, 4, 4, false>;
 using GrpCfg = GemmCfg<2, 6, 4, 8, false>;   // grouped (segmented) launches: short K loops, epilogue-heavy
 using FwdPairCfg = GemmCfg<2, 6, 6, 4, false, true>;
-using FusedCfg = GemmCfg<2, 6, 4, 8, false, true, true, true>;
+using FusedCfg = GemmCfg<1, 6, 4, 8, false, true, true, true>;
 using BwdPairCfg = GemmCfg<1, 6, 6, 8, true, true>;
 using BwdFusedCfg = GemmCfg<1, 6, 6, 8, true, true, true>;   // two sign GEMMs of the backward in one launch
 constexpr int kMaxStages = 8;
