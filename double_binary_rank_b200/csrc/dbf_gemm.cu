@@ -37,7 +37,10 @@
 // expanding its 128 sign rows and loading half of the token tile (2-SM TMA
 // loads without multicast, counted by the leader CTA's barrier); the leader
 // issues the MMAs and commits to both CTAs' barriers, and each CTA's tensor
-// memory holds its 128 rows of the 256 x 256 accumulator.
+// memory holds its 128 rows of the 256 x 256 accumulator. The one-launch
+// forward (FusedCfg, also the MBOK layer) takes 256 x 512 pair tiles: each
+// expanded sign stage feeds two MMAs, one per 256-token half, and the two
+// accumulators hold the two halves of one tile.
 // Every wait is bounded; on expiry the CTA records DBF_ERR_TIMEOUT and stops
 // issuing work; before it frees its tensor memory and ends, the TMA loads
 // and MMAs it already issued are waited for (bounded as well).
