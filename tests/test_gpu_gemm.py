@@ -216,6 +216,39 @@ def test_fused_forward_deterministic_and_exact(dbf):
     assert np.array_equal(a, oracle.forward(L, x))
 
 
+# shapes whose schedule on 74 CTA pairs (a full B200) splits the last
+# stage-2 tiles in two halves of K: 24 and 16 of them, ragged in N and T
+SPLIT = [(2048, 6000, 2048, 1, 1500), (2048, 7000, 2048, 2, 900)]
+
+
+@pytest.mark.parametrize("shape", SPLIT, ids=lambda s: "M{}N{}R{}l{}T{}".format(*s))
+def test_fused_forward_split_tiles(dbf, shape):
+    import ctypes
+    M, N, R, ell, T = shape
+    pairs = torch.cuda.get_device_properties(0).multi_processor_count // 2
+    Lc = dbf.DbfLayerC(M, N, R, ell, 0x1000, 0x1000, 0x1000, 0x1000, 0x1000)
+    tiles = (ctypes.c_int32 * 3)()
+    span = (ctypes.c_double * 2)()
+    assert dbf._lib.dbf_debug_fused_schedule(ctypes.byref(Lc), T, pairs, tiles, span) == dbf.OK
+    if pairs == 74:
+        assert tiles[2] > 0
+    rng = np.random.default_rng(sum(shape) + 12)
+    # integer inputs with exact fp16 operands and fp32 sums: the two halves'
+    # partial sums and their exchange are exact, so every element matches
+    # the oracle bit for bit, and two calls agree
+    L = exact_layer(rng, M, N, R, ell)
+    x = rng.integers(-1, 2, size=(T, M)).astype(np.float32)
+    a = run(dbf, L, x)
+    assert np.array_equal(a, run(dbf, L, x))
+    assert np.array_equal(a, oracle.forward(L, x))
+    # random inputs, accumulating into y
+    L = random_layer(rng, M, N, R, ell)
+    x = S.to_bf16_bits(rng.standard_normal((T, M)))
+    y_in = rng.standard_normal((T, N)).astype(np.float32)
+    ref = oracle.forward(L, x, y_in=y_in, accumulate=True)
+    assert rel_err(run(dbf, L, x, acc=True, y_in=y_in), ref) < TOL
+
+
 @pytest.mark.parametrize("shape", [FUSED[2]], ids=lambda s: "M{}N{}R{}l{}T{}".format(*s))
 def test_fused_forward_sign_flip_and_alpha_scaling(dbf, shape):
     # the two bit-exact invariants above, on the single-launch forward
