@@ -1405,6 +1405,8 @@ __device__ __forceinline__ void scale_row_warp(const void *x, dbf_dtype xd, cons
     }
 }
 
+constexpr int kCastPiece = 1024;   // columns a warp of the pre-pass converts at a time (a multiple of 8)
+
 // u[(i T + t), m] = fp16(gamma_i[m] x[t, m]); with M % 8 == 0 and gamma
 // 16-byte aligned a warp takes whole rows with 16-byte loads and stores,
 // else one column per thread.
@@ -1421,15 +1423,19 @@ __global__ void __launch_bounds__(256) scale_cast_kernel(const void *x, dbf_dtyp
         for (int i = threadIdx.x; i < nzero; i += blockDim.x) zero[i] = 0u;
     const int64_t total = static_cast<int64_t>(ell) * T * M;
     if (vec8) {
-        // one row per warp step (see scale_row_warp)
+        // one piece of kCastPiece columns of a row per warp step (see
+        // scale_row_warp): enough warps to keep HBM busy at small T
         const int lane = threadIdx.x & 31;
-        const int nrows = ell * T;   // <= 2^30
-        const int nw = static_cast<int>((gridDim.x * blockDim.x) >> 5);
-        for (int row = static_cast<int>((blockIdx.x * blockDim.x + threadIdx.x) >> 5); row < nrows; row += nw) {
+        const int npieces = (M + kCastPiece - 1) / kCastPiece;
+        const int64_t nitems = static_cast<int64_t>(ell) * T * npieces;
+        const int64_t nw = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+        for (int64_t w = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; w < nitems; w += nw) {
+            const int row = static_cast<int>(w / npieces);
+            const int c0 = static_cast<int>(w - static_cast<int64_t>(row) * npieces) * kCastPiece;
             const int i = tok_major ? row % ell : row / T;
             const int t = tok_major ? row / ell : row - i * T;
-            scale_row_warp(x, xd, gamma + static_cast<int64_t>(i) * M, static_cast<int64_t>(t) * M, M,
-                           U + static_cast<int64_t>(row) * M, true, lane);
+            scale_row_warp(x, xd, gamma + static_cast<int64_t>(i) * M + c0, static_cast<int64_t>(t) * M + c0,
+                           min(kCastPiece, M - c0), U + static_cast<int64_t>(row) * M + c0, true, lane);
         }
         return;
     }
@@ -1749,7 +1755,8 @@ cudaError_t gemm_forward(const dbf_layer &L, const void *x, dbf_dtype xd, void *
     {
         const int64_t total = static_cast<int64_t>(L.ell) * T * L.M;
         const int vec8 = (L.M % 8 == 0) && ((reinterpret_cast<uintptr_t>(L.gamma) & 15u) == 0);
-        int64_t blocks = vec8 ? (static_cast<int64_t>(L.ell) * T + 7) / 8 : (total + 255) / 256;
+        const int64_t pieces = (L.M + kCastPiece - 1) / kCastPiece;
+        int64_t blocks = vec8 ? (static_cast<int64_t>(L.ell) * T * pieces + 7) / 8 : (total + 255) / 256;
         if (blocks > 8 * device_sms()) blocks = 8 * device_sms();
         scale_cast_kernel<<<static_cast<int>(blocks), 256, 0, s>>>(x, xd, L.gamma, L.M, Ti, L.ell, U, vec8, 0,
                                                                    fused ? ctl : nullptr, fused ? ctl_words(L, T) : 0);
@@ -1845,7 +1852,8 @@ cudaError_t scale_cast(const void *x, dbf_dtype xd, const uint16_t *scale, int K
 {
     const int64_t total = static_cast<int64_t>(ell) * T * K;
     const int vec8 = (K % 8 == 0) && ((reinterpret_cast<uintptr_t>(scale) & 15u) == 0);
-    int64_t blocks = vec8 ? (static_cast<int64_t>(ell) * T + 7) / 8 : (total + 255) / 256;
+    const int64_t pieces = (K + kCastPiece - 1) / kCastPiece;
+    int64_t blocks = vec8 ? (static_cast<int64_t>(ell) * T * pieces + 7) / 8 : (total + 255) / 256;
     if (blocks > 8 * device_sms()) blocks = 8 * device_sms();
     scale_cast_kernel<<<static_cast<int>(blocks), 256, 0, s>>>(x, xd, scale, K, static_cast<int>(T), ell, out, vec8,
                                                                tok_major, zero, nzero);
