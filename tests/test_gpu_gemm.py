@@ -53,7 +53,10 @@ def test_gemm_exact_bit_identical(dbf, shape):
     assert np.array_equal(got, ref), float(np.max(np.abs(got - ref)))
 
 
-@pytest.mark.parametrize("shape", [(128, 48, 128, 1, 5), (512, 300, 384, 2, 260), (256, 1024, 256, 1, 513)],
+# M = 1152: the pre-pass converts rows in 1024-column pieces, the last one
+# partial
+@pytest.mark.parametrize("shape", [(128, 48, 128, 1, 5), (512, 300, 384, 2, 260), (256, 1024, 256, 1, 513),
+                                   (1152, 200, 256, 2, 37)],
                          ids=lambda s: "M{}N{}R{}l{}T{}".format(*s))
 @pytest.mark.parametrize("acc", [False, True])
 def test_gemm_random(dbf, shape, acc):
@@ -183,7 +186,7 @@ def test_gemm_wrapping_shape_sampled_rows(dbf):
 # the second and third split their last stage-2 tiles in K, and the last two
 # have one and three tokens (one column block).
 FUSED = [(2048, 1000, 2048, 1, 700), (2048, 2500, 1024, 2, 1100), (4096, 4096, 2048, 1, 1024),
-         (2048, 512, 2048, 1, 1), (2048, 768, 1024, 2, 3)]
+         (2048, 512, 2048, 1, 1), (2048, 768, 1024, 2, 3), (2176, 640, 2048, 1, 300)]
 
 
 @pytest.mark.parametrize("shape", FUSED, ids=lambda s: "M{}N{}R{}l{}T{}".format(*s))
